@@ -1,0 +1,17 @@
+"""dictionary_compressed_linear_b200 — B200-native forward of a DictLLM projection.
+
+Y = (X D_g) C_l with an NVFP4 dictionary D_g shared by a group of layers and a
+sparse NVFP4 coefficient matrix C_l per layer (DictLLM technical review, Eq. (1)),
+computed by hand-written sm_100a CUDA kernels behind the C ABI of
+``libdictproj.so`` (include/dictproj.h). This package is the thin Python
+binding of that ABI; it loads the in-tree library and fails loudly if it is
+missing.
+"""
+from .binding import (  # noqa: F401
+    PATH_AUTO, PATH_DECODE, PATH_PREFILL, DictprojError, Group, Layer, LIB_PATH, SIGNATURES, lib,
+    dictproj_check, dictproj_coefficient_stage, dictproj_dictionary_stage, dictproj_forward, dictproj_forward_path, dictproj_forward_status,
+    dictproj_group_export, dictproj_group_info, dictproj_group_packed_sizes, dictproj_group_upload,
+    dictproj_last_error, dictproj_layer_export, dictproj_layer_info, dictproj_layer_packed_entries,
+    dictproj_layer_upload, dictproj_pack, dictproj_pack_group, dictproj_pack_group_host,
+    dictproj_pack_layer, dictproj_pack_layer_host, dictproj_status_string, dictproj_version,
+)

@@ -1,0 +1,319 @@
+"""ctypes binding of libdictproj.so: argument marshalling only.
+
+Every function here has the name of the C entry point it calls (include/dictproj.h)
+and does nothing but convert Python / NumPy arguments to C types and raise on a
+non-zero status. All arithmetic of the forward pass runs in the library's CUDA
+kernels. Device buffers are passed as integer addresses (e.g. a torch tensor's
+``data_ptr()``); streams as integer handles (e.g. ``torch.cuda.current_stream().cuda_stream``).
+"""
+from __future__ import annotations
+
+import ctypes as C
+import os
+
+import numpy as np
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libdictproj.so")
+
+STATUS = {
+    0: "DICTPROJ_OK", -1: "DICTPROJ_ERR_NULL", -2: "DICTPROJ_ERR_SHAPE", -3: "DICTPROJ_ERR_ALIGN",
+    -4: "DICTPROJ_ERR_MISMATCH", -5: "DICTPROJ_ERR_RANGE", -6: "DICTPROJ_ERR_CUDA",
+    -7: "DICTPROJ_ERR_OOM", -8: "DICTPROJ_ERR_TIMEOUT", -9: "DICTPROJ_ERR_UNSUPPORTED",
+    -10: "DICTPROJ_ERR_VALUE",
+}
+PATH_AUTO, PATH_DECODE, PATH_PREFILL = 0, 1, 2
+
+
+class DictprojError(RuntimeError):
+    def __init__(self, status: int, message: str):
+        super().__init__(f"{STATUS.get(status, status)}: {message}")
+        self.status = status
+
+
+_u8p = C.POINTER(C.c_uint8)
+_u16p = C.POINTER(C.c_uint16)
+_u32p = C.POINTER(C.c_uint32)
+_i32p = C.POINTER(C.c_int32)
+_f32p = C.POINTER(C.c_float)
+_szp = C.POINTER(C.c_size_t)
+_intp = C.POINTER(C.c_int)
+
+# (name, restype, argtypes) for every entry point declared in include/dictproj.h
+SIGNATURES = [
+    ("dictproj_group_packed_sizes", C.c_int, [C.c_int, C.c_int, _szp, _szp]),
+    ("dictproj_pack_group_host", C.c_int, [_f32p, C.c_int, C.c_int, _u8p, _u8p, _f32p]),
+    ("dictproj_layer_packed_entries", C.c_int, [_i32p, C.c_int, C.c_int, _szp]),
+    ("dictproj_pack_layer_host", C.c_int,
+     [_i32p, _i32p, _f32p, C.c_int, C.c_int, _u32p, _u32p, _u8p, _u8p, _u8p, _u16p, _f32p]),
+    ("dictproj_group_upload", C.c_int,
+     [_u8p, _u8p, C.c_float, C.c_int, C.c_int, C.c_int, C.POINTER(C.c_void_p)]),
+    ("dictproj_pack_group", C.c_int, [_f32p, C.c_int, C.c_int, C.c_int, C.POINTER(C.c_void_p)]),
+    ("dictproj_layer_upload", C.c_int,
+     [_u32p, _u8p, _u8p, _u8p, _u16p, C.c_float, C.c_int, C.c_int, C.POINTER(C.c_void_p)]),
+    ("dictproj_pack_layer", C.c_int, [_i32p, _i32p, _f32p, C.c_int, C.c_int, C.POINTER(C.c_void_p)]),
+    ("dictproj_pack", C.c_int,
+     [_f32p, C.c_int, C.c_int, C.c_int, C.c_int, C.POINTER(_i32p), C.POINTER(_i32p),
+      C.POINTER(_f32p), _intp, C.POINTER(C.c_void_p), C.POINTER(C.c_void_p)]),
+    ("dictproj_group_export", C.c_int, [C.c_void_p, _u8p, _u8p, _f32p]),
+    ("dictproj_layer_export", C.c_int, [C.c_void_p, _u32p, _u8p, _u8p, _u8p, _u16p, _f32p]),
+    ("dictproj_group_info", C.c_int, [C.c_void_p, _intp, _intp, _intp]),
+    ("dictproj_layer_info", C.c_int, [C.c_void_p, _intp, _intp, _szp, _szp]),
+    ("dictproj_free_group", None, [C.c_void_p]),
+    ("dictproj_free_layer", None, [C.c_void_p]),
+    ("dictproj_forward", C.c_int, [C.c_void_p, C.c_int, C.c_void_p, C.c_void_p, C.c_void_p, C.c_void_p]),
+    ("dictproj_forward_path", C.c_int,
+     [C.c_void_p, C.c_int, C.c_void_p, C.c_void_p, C.c_void_p, C.c_void_p, C.c_int]),
+    ("dictproj_dictionary_stage", C.c_int, [C.c_void_p, C.c_int, C.c_void_p, C.c_void_p, C.c_void_p]),
+    ("dictproj_coefficient_stage", C.c_int, [C.c_void_p, C.c_int, C.c_void_p, C.c_void_p, C.c_void_p]),
+    ("dictproj_check", C.c_int, [C.c_void_p]),
+    ("dictproj_last_error", C.c_char_p, []),
+    ("dictproj_status_string", C.c_char_p, [C.c_int]),
+    ("dictproj_version", C.c_int, []),
+]
+
+_lib = None
+
+
+def lib():
+    """Load libdictproj.so (built in-tree). Raises if it is missing: there is no fallback."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing; build it with "
+                               "`python -m dictionary_compressed_linear_b200.build`")
+        L = C.CDLL(LIB_PATH)
+        for name, res, args in SIGNATURES:
+            f = getattr(L, name)
+            f.restype = res
+            f.argtypes = args
+        _lib = L
+    return _lib
+
+
+def dictproj_last_error() -> str:
+    return lib().dictproj_last_error().decode()
+
+
+def dictproj_status_string(status: int) -> str:
+    return lib().dictproj_status_string(int(status)).decode()
+
+
+def dictproj_version() -> int:
+    return lib().dictproj_version()
+
+
+def _check(status: int):
+    if status != 0:
+        raise DictprojError(status, dictproj_last_error())
+
+
+def _ptr(a: np.ndarray, ctype):
+    return a.ctypes.data_as(C.POINTER(ctype))
+
+
+# ---------------------------------------------------------------- host packing
+def dictproj_group_packed_sizes(d_in: int, k: int):
+    a, b = C.c_size_t(), C.c_size_t()
+    _check(lib().dictproj_group_packed_sizes(d_in, k, C.byref(a), C.byref(b)))
+    return a.value, b.value
+
+
+def dictproj_pack_group_host(D: np.ndarray) -> dict:
+    """D: fp32 (d_in, k) C-contiguous. Returns {'codes','scales','s'}."""
+    D = np.ascontiguousarray(D, dtype=np.float32)
+    d_in, k = D.shape
+    nc, ns = dictproj_group_packed_sizes(d_in, k)
+    codes = np.zeros(nc, np.uint8)
+    scales = np.zeros(ns, np.uint8)
+    s = C.c_float()
+    _check(lib().dictproj_pack_group_host(_ptr(D, C.c_float), d_in, k, _ptr(codes, C.c_uint8),
+                                          _ptr(scales, C.c_uint8), C.byref(s)))
+    return {"d_in": d_in, "k": k, "codes": codes, "scales": scales, "s": np.float32(s.value)}
+
+
+def dictproj_layer_packed_entries(col_ptr: np.ndarray, k: int, d_out: int) -> int:
+    col_ptr = np.ascontiguousarray(col_ptr, dtype=np.int32)
+    t = C.c_size_t()
+    _check(lib().dictproj_layer_packed_entries(_ptr(col_ptr, C.c_int32), k, d_out, C.byref(t)))
+    return t.value
+
+
+def dictproj_pack_layer_host(col_ptr, atom_idx, vals, k: int, d_out: int) -> dict:
+    col_ptr = np.ascontiguousarray(col_ptr, dtype=np.int32)
+    atom_idx = np.ascontiguousarray(atom_idx, dtype=np.int32)
+    vals = np.ascontiguousarray(vals, dtype=np.float32)
+    total = dictproj_layer_packed_entries(col_ptr, k, d_out)
+    nseg = -(-k // 256)
+    out = {
+        "col_ptr": np.zeros(d_out + 1, np.uint32), "nnz": np.zeros(d_out, np.uint32),
+        "codes": np.zeros(total // 2, np.uint8), "scales": np.zeros(total // 16, np.uint8),
+        "idx": np.zeros(total, np.uint8), "seg_start": np.zeros(d_out * nseg, np.uint16),
+    }
+    s = C.c_float()
+    _check(lib().dictproj_pack_layer_host(
+        _ptr(col_ptr, C.c_int32), _ptr(atom_idx, C.c_int32), _ptr(vals, C.c_float), k, d_out,
+        _ptr(out["col_ptr"], C.c_uint32), _ptr(out["nnz"], C.c_uint32), _ptr(out["codes"], C.c_uint8),
+        _ptr(out["scales"], C.c_uint8), _ptr(out["idx"], C.c_uint8), _ptr(out["seg_start"], C.c_uint16),
+        C.byref(s)))
+    out.update(k=k, d_out=d_out, nseg=nseg, s=np.float32(s.value))
+    return out
+
+
+# ---------------------------------------------------------------- device objects
+class Group:
+    """Owns a dictproj_group handle (packed D_g + Z scratch on the device)."""
+
+    def __init__(self, handle: int, d_in: int, k: int, max_tokens: int):
+        self.handle, self.d_in, self.k, self.max_tokens = handle, d_in, k, max_tokens
+
+    def free(self):
+        if self.handle:
+            lib().dictproj_free_group(self.handle)
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.free()
+        except Exception:
+            pass
+
+
+class Layer:
+    """Owns a dictproj_layer handle (packed C_l on the device)."""
+
+    def __init__(self, handle: int, k: int, d_out: int):
+        self.handle, self.k, self.d_out = handle, k, d_out
+
+    def free(self):
+        if self.handle:
+            lib().dictproj_free_layer(self.handle)
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.free()
+        except Exception:
+            pass
+
+
+def dictproj_group_upload(packed: dict, max_tokens: int) -> Group:
+    h = C.c_void_p()
+    codes = np.ascontiguousarray(packed["codes"], np.uint8)
+    scales = np.ascontiguousarray(packed["scales"], np.uint8)
+    _check(lib().dictproj_group_upload(_ptr(codes, C.c_uint8), _ptr(scales, C.c_uint8),
+                                       float(packed["s"]), packed["d_in"], packed["k"], max_tokens,
+                                       C.byref(h)))
+    return Group(h.value, packed["d_in"], packed["k"], max_tokens)
+
+
+def dictproj_pack_group(D: np.ndarray, max_tokens: int) -> Group:
+    D = np.ascontiguousarray(D, dtype=np.float32)
+    h = C.c_void_p()
+    _check(lib().dictproj_pack_group(_ptr(D, C.c_float), D.shape[0], D.shape[1], max_tokens, C.byref(h)))
+    return Group(h.value, D.shape[0], D.shape[1], max_tokens)
+
+
+def dictproj_layer_upload(packed: dict) -> Layer:
+    h = C.c_void_p()
+    a = {n: np.ascontiguousarray(packed[n]) for n in ("col_ptr", "codes", "scales", "idx", "seg_start")}
+    _check(lib().dictproj_layer_upload(_ptr(a["col_ptr"], C.c_uint32), _ptr(a["codes"], C.c_uint8),
+                                       _ptr(a["scales"], C.c_uint8), _ptr(a["idx"], C.c_uint8),
+                                       _ptr(a["seg_start"], C.c_uint16), float(packed["s"]),
+                                       packed["k"], packed["d_out"], C.byref(h)))
+    return Layer(h.value, packed["k"], packed["d_out"])
+
+
+def dictproj_pack_layer(col_ptr, atom_idx, vals, k: int, d_out: int) -> Layer:
+    col_ptr = np.ascontiguousarray(col_ptr, dtype=np.int32)
+    atom_idx = np.ascontiguousarray(atom_idx, dtype=np.int32)
+    vals = np.ascontiguousarray(vals, dtype=np.float32)
+    h = C.c_void_p()
+    _check(lib().dictproj_pack_layer(_ptr(col_ptr, C.c_int32), _ptr(atom_idx, C.c_int32),
+                                     _ptr(vals, C.c_float), k, d_out, C.byref(h)))
+    return Layer(h.value, k, d_out)
+
+
+def dictproj_pack(D, max_tokens: int, layers) -> tuple:
+    """layers: list of (col_ptr, atom_idx, vals, d_out). Returns (Group, [Layer])."""
+    D = np.ascontiguousarray(D, dtype=np.float32)
+    d_in, k = D.shape
+    n = len(layers)
+    keep = [(np.ascontiguousarray(c, np.int32), np.ascontiguousarray(a, np.int32),
+             np.ascontiguousarray(v, np.float32)) for c, a, v, _ in layers]
+    cp = (_i32p * n)(*[_ptr(c, C.c_int32) for c, _, _ in keep])
+    ai = (_i32p * n)(*[_ptr(a, C.c_int32) for _, a, _ in keep])
+    vv = (_f32p * n)(*[_ptr(v, C.c_float) for _, _, v in keep])
+    do = (C.c_int * n)(*[int(d) for *_, d in layers])
+    gh = C.c_void_p()
+    lh = (C.c_void_p * n)()
+    _check(lib().dictproj_pack(_ptr(D, C.c_float), d_in, k, max_tokens, n, cp, ai, vv, do,
+                               C.byref(gh), lh))
+    return Group(gh.value, d_in, k, max_tokens), [Layer(lh[i], k, layers[i][3]) for i in range(n)]
+
+
+def dictproj_group_export(g: Group) -> dict:
+    nc, ns = dictproj_group_packed_sizes(g.d_in, g.k)
+    codes, scales, s = np.zeros(nc, np.uint8), np.zeros(ns, np.uint8), C.c_float()
+    _check(lib().dictproj_group_export(g.handle, _ptr(codes, C.c_uint8), _ptr(scales, C.c_uint8),
+                                       C.byref(s)))
+    return {"d_in": g.d_in, "k": g.k, "codes": codes, "scales": scales, "s": np.float32(s.value)}
+
+
+def dictproj_layer_info(l: Layer) -> dict:
+    k, d_out, t, nz = C.c_int(), C.c_int(), C.c_size_t(), C.c_size_t()
+    _check(lib().dictproj_layer_info(l.handle, C.byref(k), C.byref(d_out), C.byref(t), C.byref(nz)))
+    return {"k": k.value, "d_out": d_out.value, "total": t.value, "nnz_total": nz.value}
+
+
+def dictproj_group_info(g: Group) -> dict:
+    d_in, k, mt = C.c_int(), C.c_int(), C.c_int()
+    _check(lib().dictproj_group_info(g.handle, C.byref(d_in), C.byref(k), C.byref(mt)))
+    return {"d_in": d_in.value, "k": k.value, "max_tokens": mt.value}
+
+
+def dictproj_layer_export(l: Layer) -> dict:
+    info = dictproj_layer_info(l)
+    T, d_out, k = info["total"], l.d_out, l.k
+    nseg = -(-k // 256)
+    out = {"col_ptr": np.zeros(d_out + 1, np.uint32), "codes": np.zeros(T // 2, np.uint8),
+           "scales": np.zeros(T // 16, np.uint8), "idx": np.zeros(T, np.uint8),
+           "seg_start": np.zeros(d_out * nseg, np.uint16)}
+    s = C.c_float()
+    _check(lib().dictproj_layer_export(l.handle, _ptr(out["col_ptr"], C.c_uint32), _ptr(out["codes"], C.c_uint8),
+                                       _ptr(out["scales"], C.c_uint8), _ptr(out["idx"], C.c_uint8),
+                                       _ptr(out["seg_start"], C.c_uint16), C.byref(s)))
+    out.update(k=k, d_out=d_out, nseg=nseg, s=np.float32(s.value))
+    return out
+
+
+# ---------------------------------------------------------------- forward
+def dictproj_forward(X_ptr: int, M: int, layer: Layer, group: Group, Y_ptr: int, stream: int = 0):
+    _check(lib().dictproj_forward(C.c_void_p(X_ptr), M, layer.handle, group.handle, C.c_void_p(Y_ptr),
+                                  C.c_void_p(stream)))
+
+
+def dictproj_forward_path(X_ptr: int, M: int, layer: Layer, group: Group, Y_ptr: int, stream: int = 0,
+                          path: int = PATH_AUTO):
+    _check(lib().dictproj_forward_path(C.c_void_p(X_ptr), M, layer.handle, group.handle,
+                                       C.c_void_p(Y_ptr), C.c_void_p(stream), path))
+
+
+def dictproj_forward_status(X_ptr, M, layer_handle, group_handle, Y_ptr, stream=0, path=PATH_AUTO) -> int:
+    """Raw status of a forward call (no exception), for boundary tests."""
+    return lib().dictproj_forward_path(C.c_void_p(X_ptr), M, layer_handle, group_handle,
+                                       C.c_void_p(Y_ptr), C.c_void_p(stream), path)
+
+
+def dictproj_dictionary_stage(X_ptr: int, M: int, group: Group, Z_ptr: int, stream: int = 0):
+    _check(lib().dictproj_dictionary_stage(C.c_void_p(X_ptr), M, group.handle, C.c_void_p(Z_ptr),
+                                           C.c_void_p(stream)))
+
+
+def dictproj_coefficient_stage(Z_ptr: int, M: int, layer: Layer, Y_ptr: int, stream: int = 0):
+    _check(lib().dictproj_coefficient_stage(C.c_void_p(Z_ptr), M, layer.handle, C.c_void_p(Y_ptr),
+                                            C.c_void_p(stream)))
+
+
+def dictproj_check(stream: int = 0):
+    _check(lib().dictproj_check(C.c_void_p(stream)))

@@ -1,0 +1,448 @@
+// C ABI of libdictproj: validation, handles, uploads and forward dispatch.
+// Every entry point validates its arguments before touching the device and
+// reports failures through a status code plus a thread-local message.
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstdlib>
+#include <cstring>
+#include <mutex>
+#include <new>
+#include <vector>
+
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+
+#include "dictproj.h"
+#include "dictproj_internal.h"
+#include "kernels.h"
+
+namespace dictproj {
+
+static thread_local char g_err[512] = "";
+
+int fail(int status, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_err, sizeof(g_err), fmt, ap);
+  va_end(ap);
+  return status;
+}
+void clear_error() { g_err[0] = 0; }
+
+static int cuda_fail(cudaError_t e, const char* what) {
+  return fail(DICTPROJ_ERR_CUDA, "%s: %s (%s)", what, cudaGetErrorName(e), cudaGetErrorString(e));
+}
+
+// Host-side fault injection for error-path tests: DICTPROJ_FAULT=alloc|copy.
+static bool fault(const char* kind) {
+  const char* f = std::getenv("DICTPROJ_FAULT");
+  return f && std::strcmp(f, kind) == 0;
+}
+
+static cudaError_t dmalloc(void** p, size_t n) {
+  if (fault("alloc")) return cudaErrorMemoryAllocation;
+  return cudaMalloc(p, n ? n : 16);
+}
+static cudaError_t h2d(void* d, const void* h, size_t n) {
+  if (fault("copy")) return cudaErrorInvalidValue;
+  return n ? cudaMemcpy(d, h, n, cudaMemcpyHostToDevice) : cudaSuccess;
+}
+
+// One-time per-device set-up (kernel attributes) and capability check.
+static std::mutex g_dev_mu;
+static std::vector<int> g_dev_ready;
+
+static int ensure_device(int* dev_out) {
+  int dev = -1;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  std::lock_guard<std::mutex> lk(g_dev_mu);
+  if ((int)g_dev_ready.size() <= dev) g_dev_ready.resize(dev + 1, 0);
+  if (!g_dev_ready[dev]) {
+    cudaDeviceProp prop;
+    if ((e = cudaGetDeviceProperties(&prop, dev)) != cudaSuccess) return cuda_fail(e, "cudaGetDeviceProperties");
+    if (prop.major != 10)
+      return fail(DICTPROJ_ERR_UNSUPPORTED, "device %d is sm_%d%d; this library is built for sm_100a", dev,
+                  prop.major, prop.minor);
+    if ((e = prepare_decode_kernels(dev)) != cudaSuccess) return cuda_fail(e, "kernel set-up");
+    g_dev_ready[dev] = 1;
+  }
+  *dev_out = dev;
+  return DICTPROJ_OK;
+}
+
+static int check_group_shape(int d_in, int k) {
+  if (d_in <= 0 || k <= 0 || d_in % 32 || k % 16)
+    return fail(DICTPROJ_ERR_SHAPE, "group: need d_in > 0 with d_in %% 32 == 0 and k > 0 with k %% 16 == 0 (got d_in=%d k=%d)", d_in, k);
+  if (k > 65535) return fail(DICTPROJ_ERR_SHAPE, "group: k=%d exceeds 65535", k);
+  return DICTPROJ_OK;
+}
+
+}  // namespace dictproj
+
+using namespace dictproj;
+
+extern "C" {
+
+const char* dictproj_last_error(void) { return g_err; }
+
+const char* dictproj_status_string(int s) {
+  switch (s) {
+    case DICTPROJ_OK: return "DICTPROJ_OK";
+    case DICTPROJ_ERR_NULL: return "DICTPROJ_ERR_NULL";
+    case DICTPROJ_ERR_SHAPE: return "DICTPROJ_ERR_SHAPE";
+    case DICTPROJ_ERR_ALIGN: return "DICTPROJ_ERR_ALIGN";
+    case DICTPROJ_ERR_MISMATCH: return "DICTPROJ_ERR_MISMATCH";
+    case DICTPROJ_ERR_RANGE: return "DICTPROJ_ERR_RANGE";
+    case DICTPROJ_ERR_CUDA: return "DICTPROJ_ERR_CUDA";
+    case DICTPROJ_ERR_OOM: return "DICTPROJ_ERR_OOM";
+    case DICTPROJ_ERR_TIMEOUT: return "DICTPROJ_ERR_TIMEOUT";
+    case DICTPROJ_ERR_UNSUPPORTED: return "DICTPROJ_ERR_UNSUPPORTED";
+    case DICTPROJ_ERR_VALUE: return "DICTPROJ_ERR_VALUE";
+    default: return "DICTPROJ_ERR_UNKNOWN";
+  }
+}
+
+int dictproj_version(void) { return 10000; }
+
+int dictproj_group_packed_sizes(int d_in, int k, size_t* codes_bytes, size_t* scales_bytes) {
+  clear_error();
+  if (!codes_bytes || !scales_bytes) return fail(DICTPROJ_ERR_NULL, "group_packed_sizes: NULL output");
+  if (d_in <= 0 || k <= 0 || d_in % 16) return fail(DICTPROJ_ERR_SHAPE, "group_packed_sizes: need d_in %% 16 == 0 and k > 0");
+  *codes_bytes = (size_t)d_in * k / 2;
+  *scales_bytes = (size_t)d_in * k / 16;
+  return DICTPROJ_OK;
+}
+
+int dictproj_pack_group_host(const float* D, int d_in, int k, uint8_t* codes, uint8_t* scales, float* s_D) {
+  clear_error();
+  return pack_group_host(D, d_in, k, codes, scales, s_D);
+}
+
+int dictproj_layer_packed_entries(const int32_t* col_ptr, int k, int d_out, size_t* total) {
+  clear_error();
+  return layer_packed_entries(col_ptr, k, d_out, total);
+}
+
+int dictproj_pack_layer_host(const int32_t* col_ptr, const int32_t* atom_idx, const float* vals, int k,
+                             int d_out, uint32_t* pcol_ptr, uint32_t* nnz, uint8_t* codes,
+                             uint8_t* scales, uint8_t* idx, uint16_t* seg_start, float* s_C) {
+  clear_error();
+  return pack_layer_host(col_ptr, atom_idx, vals, k, d_out, pcol_ptr, nnz, codes, scales, idx, seg_start, s_C);
+}
+
+void dictproj_free_group(dictproj_group* g) {
+  if (!g) return;
+  cudaFree(g->codes);
+  cudaFree(g->scales);
+  cudaFree(g->z32);
+  cudaFree(g->z16);
+  cudaFree(g->dexp);
+  cudaFree(g->err);
+  delete g;
+}
+
+void dictproj_free_layer(dictproj_layer* l) {
+  if (!l) return;
+  cudaFree(l->col_ptr);
+  cudaFree(l->codes);
+  cudaFree(l->scales);
+  cudaFree(l->idx);
+  cudaFree(l->seg_start);
+  cudaFree(l->cexp);
+  delete l;
+}
+
+int dictproj_group_upload(const uint8_t* codes, const uint8_t* scales, float s_D, int d_in, int k,
+                          int max_tokens, dictproj_group** out) {
+  clear_error();
+  if (!codes || !scales || !out) return fail(DICTPROJ_ERR_NULL, "group_upload: NULL pointer");
+  *out = nullptr;
+  int st = check_group_shape(d_in, k);
+  if (st) return st;
+  if (max_tokens < 1) return fail(DICTPROJ_ERR_RANGE, "group_upload: max_tokens must be >= 1 (got %d)", max_tokens);
+  if (!(s_D > 0.0f) || !std::isfinite(s_D)) return fail(DICTPROJ_ERR_VALUE, "group_upload: s_D must be finite and > 0");
+  int dev;
+  if ((st = ensure_device(&dev))) return st;
+  dictproj_group* g = new (std::nothrow) dictproj_group();
+  if (!g) return fail(DICTPROJ_ERR_OOM, "group_upload: host allocation failed");
+  g->device = dev;
+  g->d_in = d_in;
+  g->k = k;
+  g->max_tokens = max_tokens;
+  g->s = s_D;
+  g->codes_bytes = (size_t)d_in * k / 2;
+  g->scales_bytes = (size_t)d_in * k / 16;
+  cudaError_t e;
+  if ((e = dmalloc((void**)&g->codes, g->codes_bytes)) || (e = dmalloc((void**)&g->scales, g->scales_bytes)) ||
+      (e = dmalloc((void**)&g->z32, (size_t)k * kDecodeMaxTokens * sizeof(float))) ||
+      (e = dmalloc((void**)&g->err, 16))) {
+    dictproj_free_group(g);
+    cudaGetLastError();
+    return fail(DICTPROJ_ERR_OOM, "group_upload: device allocation failed (%s)", cudaGetErrorName(e));
+  }
+  if ((e = h2d(g->codes, codes, g->codes_bytes)) || (e = h2d(g->scales, scales, g->scales_bytes)) ||
+      (e = cudaMemset(g->err, 0, 16)) || (e = cudaMemset(g->z32, 0, (size_t)k * kDecodeMaxTokens * sizeof(float)))) {
+    dictproj_free_group(g);
+    cudaGetLastError();
+    return cuda_fail(e, "group_upload: copy to device");
+  }
+  *out = g;
+  return DICTPROJ_OK;
+}
+
+int dictproj_pack_group(const float* D, int d_in, int k, int max_tokens, dictproj_group** out) {
+  clear_error();
+  if (!D || !out) return fail(DICTPROJ_ERR_NULL, "pack_group: NULL pointer");
+  *out = nullptr;
+  int st = check_group_shape(d_in, k);
+  if (st) return st;
+  if (max_tokens < 1) return fail(DICTPROJ_ERR_RANGE, "pack_group: max_tokens must be >= 1 (got %d)", max_tokens);
+  std::vector<uint8_t> codes, scales;
+  try {
+    codes.resize((size_t)d_in * k / 2);
+    scales.resize((size_t)d_in * k / 16);
+  } catch (...) {
+    return fail(DICTPROJ_ERR_OOM, "pack_group: host allocation failed");
+  }
+  float s = 0.f;
+  if ((st = pack_group_host(D, d_in, k, codes.data(), scales.data(), &s))) return st;
+  return dictproj_group_upload(codes.data(), scales.data(), s, d_in, k, max_tokens, out);
+}
+
+int dictproj_layer_upload(const uint32_t* pcol_ptr, const uint8_t* codes, const uint8_t* scales,
+                          const uint8_t* idx, const uint16_t* seg_start, float s_C, int k, int d_out,
+                          dictproj_layer** out) {
+  clear_error();
+  if (!pcol_ptr || !codes || !scales || !idx || !seg_start || !out)
+    return fail(DICTPROJ_ERR_NULL, "layer_upload: NULL pointer");
+  *out = nullptr;
+  if (k <= 0 || k % 16 || k > 65535 || d_out <= 0)
+    return fail(DICTPROJ_ERR_SHAPE, "layer_upload: need 0 < k <= 65535, k %% 16 == 0, d_out > 0 (got k=%d d_out=%d)", k, d_out);
+  if (!(s_C > 0.0f) || !std::isfinite(s_C)) return fail(DICTPROJ_ERR_VALUE, "layer_upload: s_C must be finite and > 0");
+  if (pcol_ptr[0] != 0) return fail(DICTPROJ_ERR_RANGE, "layer_upload: col_ptr[0] must be 0");
+  const int nseg = (k + 255) / 256;
+  for (int o = 0; o < d_out; ++o) {
+    const uint32_t n = pcol_ptr[o + 1] - pcol_ptr[o];
+    if (pcol_ptr[o + 1] < pcol_ptr[o] || n % 16 || n > (uint32_t)((k + 15) / 16 * 16))
+      return fail(DICTPROJ_ERR_RANGE, "layer_upload: column %d has a bad padded length %u", o, n);
+    const uint16_t* ss = seg_start + (size_t)o * nseg;
+    if (ss[0] != 0) return fail(DICTPROJ_ERR_RANGE, "layer_upload: seg_start[%d][0] != 0", o);
+    for (int s = 1; s < nseg; ++s)
+      if (ss[s] < ss[s - 1] || ss[s] > n) return fail(DICTPROJ_ERR_RANGE, "layer_upload: seg_start of column %d not monotone", o);
+  }
+  int dev, st;
+  if ((st = ensure_device(&dev))) return st;
+  dictproj_layer* l = new (std::nothrow) dictproj_layer();
+  if (!l) return fail(DICTPROJ_ERR_OOM, "layer_upload: host allocation failed");
+  l->device = dev;
+  l->k = k;
+  l->d_out = d_out;
+  l->nseg = nseg;
+  l->s = s_C;
+  l->total = pcol_ptr[d_out];
+  const size_t T = l->total;
+  cudaError_t e;
+  // +16 bytes on every array so rounded-up L2 prefetch ranges stay inside the allocation
+  if ((e = dmalloc((void**)&l->col_ptr, (d_out + 1) * sizeof(uint32_t) + 16)) ||
+      (e = dmalloc((void**)&l->codes, T / 2 + 16)) || (e = dmalloc((void**)&l->scales, T / 16 + 16)) ||
+      (e = dmalloc((void**)&l->idx, T + 16)) ||
+      (e = dmalloc((void**)&l->seg_start, (size_t)d_out * nseg * sizeof(uint16_t) + 16))) {
+    dictproj_free_layer(l);
+    cudaGetLastError();
+    return fail(DICTPROJ_ERR_OOM, "layer_upload: device allocation failed (%s)", cudaGetErrorName(e));
+  }
+  if ((e = h2d(l->col_ptr, pcol_ptr, (d_out + 1) * sizeof(uint32_t))) || (e = h2d(l->codes, codes, T / 2)) ||
+      (e = h2d(l->scales, scales, T / 16)) || (e = h2d(l->idx, idx, T)) ||
+      (e = h2d(l->seg_start, seg_start, (size_t)d_out * nseg * sizeof(uint16_t)))) {
+    dictproj_free_layer(l);
+    cudaGetLastError();
+    return cuda_fail(e, "layer_upload: copy to device");
+  }
+  // true entry count is not part of the packed arrays; derive it from the codes? No:
+  // callers that need it use dictproj_pack_layer, which records it below.
+  l->nnz_total = 0;
+  *out = l;
+  return DICTPROJ_OK;
+}
+
+int dictproj_pack_layer(const int32_t* col_ptr, const int32_t* atom_idx, const float* vals, int k, int d_out,
+                        dictproj_layer** out) {
+  clear_error();
+  if (!col_ptr || !out) return fail(DICTPROJ_ERR_NULL, "pack_layer: NULL pointer");
+  *out = nullptr;
+  if (k <= 0 || k % 16) return fail(DICTPROJ_ERR_SHAPE, "pack_layer: k must be a positive multiple of 16 (got %d)", k);
+  size_t total = 0;
+  int st = layer_packed_entries(col_ptr, k, d_out, &total);
+  if (st) return st;
+  const int nseg = (k + 255) / 256;
+  std::vector<uint32_t> pptr, nnz;
+  std::vector<uint8_t> codes, scales, idx;
+  std::vector<uint16_t> ss;
+  try {
+    pptr.resize(d_out + 1);
+    nnz.resize(d_out);
+    codes.resize(total / 2 + 1);
+    scales.resize(total / 16 + 1);
+    idx.resize(total + 1);
+    ss.resize((size_t)d_out * nseg);
+  } catch (...) {
+    return fail(DICTPROJ_ERR_OOM, "pack_layer: host allocation failed");
+  }
+  float s = 0.f;
+  if ((st = pack_layer_host(col_ptr, atom_idx, vals, k, d_out, pptr.data(), nnz.data(), codes.data(),
+                            scales.data(), idx.data(), ss.data(), &s)))
+    return st;
+  if ((st = dictproj_layer_upload(pptr.data(), codes.data(), scales.data(), idx.data(), ss.data(), s, k, d_out, out)))
+    return st;
+  (*out)->nnz_total = (size_t)col_ptr[d_out];
+  return DICTPROJ_OK;
+}
+
+int dictproj_pack(const float* D, int d_in, int k, int max_tokens, int n_layers, const int32_t* const* col_ptr,
+                  const int32_t* const* atom_idx, const float* const* vals, const int* d_out,
+                  dictproj_group** group_out, dictproj_layer** layers_out) {
+  clear_error();
+  if (!group_out || !layers_out || (n_layers > 0 && (!col_ptr || !atom_idx || !vals || !d_out)))
+    return fail(DICTPROJ_ERR_NULL, "pack: NULL pointer");
+  if (n_layers < 0) return fail(DICTPROJ_ERR_SHAPE, "pack: n_layers < 0");
+  *group_out = nullptr;
+  for (int i = 0; i < n_layers; ++i) layers_out[i] = nullptr;
+  int st = dictproj_pack_group(D, d_in, k, max_tokens, group_out);
+  if (st) return st;
+  for (int i = 0; i < n_layers; ++i) {
+    if ((st = dictproj_pack_layer(col_ptr[i], atom_idx[i], vals[i], k, d_out[i], &layers_out[i]))) {
+      for (int j = 0; j < i; ++j) {
+        dictproj_free_layer(layers_out[j]);
+        layers_out[j] = nullptr;
+      }
+      dictproj_free_group(*group_out);
+      *group_out = nullptr;
+      return st;
+    }
+  }
+  return DICTPROJ_OK;
+}
+
+int dictproj_group_export(const dictproj_group* g, uint8_t* codes, uint8_t* scales, float* s_D) {
+  clear_error();
+  if (!g || !codes || !scales || !s_D) return fail(DICTPROJ_ERR_NULL, "group_export: NULL pointer");
+  cudaError_t e;
+  if ((e = cudaMemcpy(codes, g->codes, g->codes_bytes, cudaMemcpyDeviceToHost)) ||
+      (e = cudaMemcpy(scales, g->scales, g->scales_bytes, cudaMemcpyDeviceToHost)))
+    return cuda_fail(e, "group_export");
+  *s_D = g->s;
+  return DICTPROJ_OK;
+}
+
+int dictproj_layer_export(const dictproj_layer* l, uint32_t* pcol_ptr, uint8_t* codes, uint8_t* scales,
+                          uint8_t* idx, uint16_t* seg_start, float* s_C) {
+  clear_error();
+  if (!l || !pcol_ptr || !codes || !scales || !idx || !seg_start || !s_C)
+    return fail(DICTPROJ_ERR_NULL, "layer_export: NULL pointer");
+  const size_t T = l->total;
+  cudaError_t e;
+  if ((e = cudaMemcpy(pcol_ptr, l->col_ptr, (l->d_out + 1) * sizeof(uint32_t), cudaMemcpyDeviceToHost)) ||
+      (e = cudaMemcpy(codes, l->codes, T / 2, cudaMemcpyDeviceToHost)) ||
+      (e = cudaMemcpy(scales, l->scales, T / 16, cudaMemcpyDeviceToHost)) ||
+      (e = cudaMemcpy(idx, l->idx, T, cudaMemcpyDeviceToHost)) ||
+      (e = cudaMemcpy(seg_start, l->seg_start, (size_t)l->d_out * l->nseg * sizeof(uint16_t), cudaMemcpyDeviceToHost)))
+    return cuda_fail(e, "layer_export");
+  *s_C = l->s;
+  return DICTPROJ_OK;
+}
+
+int dictproj_group_info(const dictproj_group* g, int* d_in, int* k, int* max_tokens) {
+  clear_error();
+  if (!g) return fail(DICTPROJ_ERR_NULL, "group_info: NULL handle");
+  if (d_in) *d_in = g->d_in;
+  if (k) *k = g->k;
+  if (max_tokens) *max_tokens = g->max_tokens;
+  return DICTPROJ_OK;
+}
+
+int dictproj_layer_info(const dictproj_layer* l, int* k, int* d_out, size_t* total, size_t* nnz_total) {
+  clear_error();
+  if (!l) return fail(DICTPROJ_ERR_NULL, "layer_info: NULL handle");
+  if (k) *k = l->k;
+  if (d_out) *d_out = l->d_out;
+  if (total) *total = l->total;
+  if (nnz_total) *nnz_total = l->nnz_total;
+  return DICTPROJ_OK;
+}
+
+int dictproj_forward_path(const void* X, int M, const dictproj_layer* layer, const dictproj_group* group,
+                          void* Y, void* stream, int path) {
+  clear_error();
+  if (!X || !Y || !layer || !group) return fail(DICTPROJ_ERR_NULL, "forward: NULL pointer");
+  if (M < 1 || M > group->max_tokens)
+    return fail(DICTPROJ_ERR_RANGE, "forward: M=%d outside [1, %d]", M, group->max_tokens);
+  if (layer->k != group->k) return fail(DICTPROJ_ERR_MISMATCH, "forward: layer k=%d != group k=%d", layer->k, group->k);
+  if (layer->device != group->device)
+    return fail(DICTPROJ_ERR_MISMATCH, "forward: layer on device %d, group on device %d", layer->device, group->device);
+  if (((uintptr_t)X & 15) || ((uintptr_t)Y & 15)) return fail(DICTPROJ_ERR_ALIGN, "forward: X and Y must be 16-byte aligned");
+  if (path < DICTPROJ_PATH_AUTO || path > DICTPROJ_PATH_PREFILL) return fail(DICTPROJ_ERR_RANGE, "forward: bad path %d", path);
+  if (path == DICTPROJ_PATH_DECODE && M > kDecodeMaxTokens)
+    return fail(DICTPROJ_ERR_UNSUPPORTED, "forward: decode path takes M <= %d (got %d)", kDecodeMaxTokens, M);
+  int dev = -1;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "forward: cudaGetDevice");
+  if (dev != group->device)
+    return fail(DICTPROJ_ERR_MISMATCH, "forward: current device %d, handles on device %d", dev, group->device);
+  cudaStream_t s = (cudaStream_t)stream;
+  const __half* x = static_cast<const __half*>(X);
+  __half* y = static_cast<__half*>(Y);
+  const bool decode = path == DICTPROJ_PATH_DECODE || (path == DICTPROJ_PATH_AUTO && M <= kDecodeMaxTokens);
+  if (decode) {
+    const int mp = decode_mp(M);
+    if ((e = launch_dict_decode(group, x, M, mp, group->z32, s)) != cudaSuccess) return cuda_fail(e, "forward: dictionary stage launch");
+    if ((e = launch_coeff_decode(layer, group->z32, M, mp, y, s)) != cudaSuccess) return cuda_fail(e, "forward: coefficient stage launch");
+    return DICTPROJ_OK;
+  }
+  // Token chunks of 8 through the decode kernels (prefill path until the
+  // tensor-core kernels take over).
+  for (int m0 = 0; m0 < M; m0 += kDecodeMaxTokens) {
+    const int mc = M - m0 < kDecodeMaxTokens ? M - m0 : kDecodeMaxTokens;
+    const int mp = decode_mp(mc);
+    if ((e = launch_dict_decode(group, x + (size_t)m0 * group->d_in, mc, mp, group->z32, s)) != cudaSuccess)
+      return cuda_fail(e, "forward: dictionary stage launch");
+    if ((e = launch_coeff_decode(layer, group->z32, mc, mp, y + (size_t)m0 * layer->d_out, s)) != cudaSuccess)
+      return cuda_fail(e, "forward: coefficient stage launch");
+  }
+  return DICTPROJ_OK;
+}
+
+int dictproj_forward(const void* X, int M, const dictproj_layer* layer, const dictproj_group* group, void* Y,
+                     void* stream) {
+  return dictproj_forward_path(X, M, layer, group, Y, stream, DICTPROJ_PATH_AUTO);
+}
+
+int dictproj_dictionary_stage(const void* X, int M, const dictproj_group* group, float* Z, void* stream) {
+  clear_error();
+  if (!X || !group || !Z) return fail(DICTPROJ_ERR_NULL, "dictionary_stage: NULL pointer");
+  if (M < 1 || M > group->max_tokens) return fail(DICTPROJ_ERR_RANGE, "dictionary_stage: M=%d outside [1, %d]", M, group->max_tokens);
+  if (M > kDecodeMaxTokens) return fail(DICTPROJ_ERR_UNSUPPORTED, "dictionary_stage: M must be <= %d", kDecodeMaxTokens);
+  if (((uintptr_t)X & 15) || ((uintptr_t)Z & 15)) return fail(DICTPROJ_ERR_ALIGN, "dictionary_stage: X and Z must be 16-byte aligned");
+  cudaError_t e = launch_dict_decode(group, static_cast<const __half*>(X), M, decode_mp(M), Z, (cudaStream_t)stream);
+  return e == cudaSuccess ? DICTPROJ_OK : cuda_fail(e, "dictionary_stage: launch");
+}
+
+int dictproj_coefficient_stage(const float* Z, int M, const dictproj_layer* layer, void* Y, void* stream) {
+  clear_error();
+  if (!Z || !layer || !Y) return fail(DICTPROJ_ERR_NULL, "coefficient_stage: NULL pointer");
+  if (M < 1) return fail(DICTPROJ_ERR_RANGE, "coefficient_stage: M=%d < 1", M);
+  if (M > kDecodeMaxTokens) return fail(DICTPROJ_ERR_UNSUPPORTED, "coefficient_stage: M must be <= %d", kDecodeMaxTokens);
+  if (((uintptr_t)Y & 15) || ((uintptr_t)Z & 15)) return fail(DICTPROJ_ERR_ALIGN, "coefficient_stage: Z and Y must be 16-byte aligned");
+  cudaError_t e = launch_coeff_decode(layer, Z, M, decode_mp(M), static_cast<__half*>(Y), (cudaStream_t)stream);
+  return e == cudaSuccess ? DICTPROJ_OK : cuda_fail(e, "coefficient_stage: launch");
+}
+
+int dictproj_check(void* stream) {
+  clear_error();
+  cudaError_t e = cudaStreamSynchronize((cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_fail(e, "check: stream synchronize");
+  return DICTPROJ_OK;
+}
+
+}  // extern "C"

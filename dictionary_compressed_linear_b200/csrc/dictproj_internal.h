@@ -1,0 +1,57 @@
+// Internal declarations shared by the host packer, the ABI layer and the kernels.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+
+#include "dictproj.h"
+
+namespace dictproj {
+
+// Record a formatted error message for dictproj_last_error() and return `status`.
+int fail(int status, const char* fmt, ...)
+#if defined(__GNUC__)
+    __attribute__((format(printf, 2, 3)))
+#endif
+    ;
+void clear_error();
+
+int pack_group_host(const float* D, int d_in, int k, uint8_t* codes, uint8_t* scales, float* s_D);
+int layer_packed_entries(const int32_t* col_ptr, int k, int d_out, size_t* total);
+int pack_layer_host(const int32_t* col_ptr, const int32_t* atom_idx, const float* vals, int k,
+                    int d_out, uint32_t* pcol_ptr, uint32_t* nnz, uint8_t* codes, uint8_t* scales,
+                    uint8_t* idx, uint16_t* seg_start, float* s_C);
+
+// Largest M served by the decode (GEMV) path.
+constexpr int kDecodeMaxTokens = 8;
+
+}  // namespace dictproj
+
+// Device-side state behind the opaque handles.
+struct dictproj_group {
+  int device;
+  int d_in, k, max_tokens;
+  float s;                 // s_D
+  uint8_t* codes;          // [k][d_in/2]
+  uint8_t* scales;         // [k][d_in/16]
+  size_t codes_bytes, scales_bytes;
+  // scratch
+  float* z32;              // decode Z, fp32 [k][8]
+  uint16_t* z16;           // prefill Z, fp16 [max_tokens][k] (allocated when max_tokens > 8)
+  uint16_t* dexp;          // prefill: D expanded to fp16, atom-major [k][d_in]
+  unsigned int* err;       // device error word for bounded waits
+};
+
+struct dictproj_layer {
+  int device;
+  int k, d_out, nseg;
+  float s;                 // s_C
+  size_t total;            // padded entries
+  size_t nnz_total;        // true entries
+  uint32_t* col_ptr;       // [d_out+1]
+  uint8_t* codes;          // [total/2]
+  uint8_t* scales;         // [total/16]
+  uint8_t* idx;            // [total]
+  uint16_t* seg_start;     // [d_out][nseg]
+  uint16_t* cexp;          // prefill: C expanded to fp16, [d_out][k] (lazy)
+};

@@ -1,0 +1,219 @@
+// Host-side NVFP4 packer for D_g and C_l (the export step of the DictLLM
+// technical review's Algorithm 2: dictionary, per-layer codes, scales, support).
+//
+// Encoders are written from the OCP E2M1 / E4M3 definitions with plain IEEE
+// fp32 arithmetic (compiled with -ffp-contract=off): E4M3 by scaling to the
+// format's quantum and rounding half-to-even with nearbyintf, E2M1 by rounding
+// on the three uniform sub-grids of its value set. Layouts are described in
+// include/dictproj.h.
+#include <cfenv>
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <thread>
+#include <vector>
+
+#include "dictproj_internal.h"
+
+namespace dictproj {
+
+static inline float e4m3_decode(uint8_t c) {
+  const int e = (c >> 3) & 15, m = c & 7;
+  const float mag = e == 0 ? std::ldexp((float)m, -9) : std::ldexp(1.0f + (float)m / 8.0f, e - 7);
+  return (c & 0x80) ? -mag : mag;
+}
+
+// Nearest E4M3 code to r >= 0 (finite), ties to even, saturating at 448 (0x7E).
+static inline uint8_t e4m3_encode_nonneg(float r) {
+  if (!(r > 0.0f)) return 0;
+  if (r >= 448.0f) return 0x7E;
+  int e2;
+  std::frexp(r, &e2);        // r = f * 2^e2, f in [0.5, 1)  ->  floor(log2 r) = e2 - 1
+  int E = e2 - 1;
+  if (E < -6) E = -6;        // subnormal range shares the 2^-6 binade's quantum
+  const float n = std::nearbyintf(std::ldexp(r, 3 - E));  // quanta of 2^(E-3), half-to-even
+  int ni = (int)n;
+  if (E == -6 && ni < 8) return (uint8_t)ni;  // subnormal (or zero)
+  if (ni == 16) { ni = 8; E += 1; }           // rounded up into the next binade
+  if (E > 8 || (E == 8 && ni > 14)) return 0x7E;
+  return (uint8_t)(((E + 7) << 3) | (ni - 8));
+}
+
+// Nearest E2M1 code to q, ties to even mantissa, saturating at 6; -0 -> 0.
+static inline uint8_t e2m1_encode(float q) {
+  const float a = std::fabs(q);
+  uint8_t mag;
+  if (a >= 6.0f) {
+    mag = 7;
+  } else if (a < 2.0f) {            // grid 0, .5, 1, 1.5, 2  -> codes 0..4
+    mag = (uint8_t)std::nearbyintf(a * 2.0f);
+  } else if (a < 4.0f) {            // grid 2, 3, 4           -> codes 4..6
+    mag = (uint8_t)((int)std::nearbyintf(a) + 2);
+  } else {                          // grid 4, 6              -> codes 6, 7
+    mag = (uint8_t)((int)std::nearbyintf(a * 0.5f) + 4);
+  }
+  return (q < 0.0f && mag != 0) ? (uint8_t)(mag | 8) : mag;
+}
+
+static inline float tensor_scale_from_amax(float amax) {
+  if (amax == 0.0f) return 1.0f;
+  return amax / 2688.0f;
+}
+
+// Quantise one block of 16 values given the tensor scale; writes 16 codes and
+// returns the scale code.
+static inline uint8_t quantize_block(const float* x, float s_t, uint8_t* codes16) {
+  float amax_b = 0.0f;
+  for (int i = 0; i < 16; ++i) amax_b = std::fmax(amax_b, std::fabs(x[i]));
+  const float den = 6.0f * s_t;
+  const float r = amax_b / den;
+  const uint8_t sc = e4m3_encode_nonneg(r);
+  const float scale = e4m3_decode(sc) * s_t;
+  for (int i = 0; i < 16; ++i) codes16[i] = scale == 0.0f ? 0 : e2m1_encode(x[i] / scale);
+  return sc;
+}
+
+template <class F>
+static void parallel_for(size_t n, F&& f) {
+  unsigned nt = std::thread::hardware_concurrency();
+  if (nt == 0) nt = 1;
+  if (nt > 32) nt = 32;
+  if (n < 4096 || nt == 1) { f(size_t(0), n); return; }
+  std::vector<std::thread> th;
+  const size_t chunk = (n + nt - 1) / nt;
+  for (unsigned t = 0; t < nt; ++t) {
+    const size_t a = t * chunk, b = std::min(n, a + chunk);
+    if (a >= b) break;
+    th.emplace_back([&, a, b] {
+      std::fesetround(FE_TONEAREST);
+      f(a, b);
+    });
+  }
+  for (auto& t : th) t.join();
+}
+
+int pack_group_host(const float* D, int d_in, int k, uint8_t* codes, uint8_t* scales, float* s_D) {
+  if (!D || !codes || !scales || !s_D) return fail(DICTPROJ_ERR_NULL, "pack_group_host: NULL pointer");
+  if (d_in <= 0 || k <= 0 || d_in % 16) return fail(DICTPROJ_ERR_SHAPE, "pack_group_host: need d_in > 0, d_in %% 16 == 0, k > 0 (got d_in=%d k=%d)", d_in, k);
+  std::fesetround(FE_TONEAREST);
+  const size_t n = (size_t)d_in * k;
+  // amax and finiteness
+  std::vector<float> part(64, 0.0f);
+  std::vector<int> bad(64, 0);
+  {
+    unsigned nt = std::min<unsigned>(64, std::max(1u, std::thread::hardware_concurrency()));
+    std::vector<std::thread> th;
+    const size_t chunk = (n + nt - 1) / nt;
+    for (unsigned t = 0; t < nt; ++t) {
+      th.emplace_back([&, t] {
+        const size_t a = t * chunk, b = std::min(n, a + chunk);
+        float m = 0.0f;
+        for (size_t i = a; i < b; ++i) {
+          if (!std::isfinite(D[i])) { bad[t] = 1; break; }
+          m = std::fmax(m, std::fabs(D[i]));
+        }
+        part[t] = m;
+      });
+    }
+    for (auto& t : th) t.join();
+  }
+  float amax = 0.0f;
+  for (int t = 0; t < 64; ++t) {
+    if (bad[t]) return fail(DICTPROJ_ERR_VALUE, "pack_group_host: non-finite value in D");
+    amax = std::fmax(amax, part[t]);
+  }
+  const float s = tensor_scale_from_amax(amax);
+  const int nb = d_in / 16;
+  // one task per atom: gather its d_in column of D (row-major d_in x k) into blocks
+  parallel_for((size_t)k, [&](size_t a0, size_t a1) {
+    float blk[16];
+    uint8_t c16[16];
+    for (size_t j = a0; j < a1; ++j) {
+      uint8_t* crow = codes + j * (size_t)(d_in / 2);
+      uint8_t* srow = scales + j * (size_t)nb;
+      for (int b = 0; b < nb; ++b) {
+        for (int i = 0; i < 16; ++i) blk[i] = D[(size_t)(16 * b + i) * k + j];
+        srow[b] = quantize_block(blk, s, c16);
+        for (int i = 0; i < 8; ++i) crow[8 * b + i] = (uint8_t)(c16[2 * i] | (c16[2 * i + 1] << 4));
+      }
+    }
+  });
+  *s_D = s;
+  return DICTPROJ_OK;
+}
+
+int layer_packed_entries(const int32_t* col_ptr, int k, int d_out, size_t* total) {
+  if (!col_ptr || !total) return fail(DICTPROJ_ERR_NULL, "layer_packed_entries: NULL pointer");
+  if (k <= 0 || k > 65535 || d_out <= 0) return fail(DICTPROJ_ERR_SHAPE, "layer: need 0 < k <= 65535 and d_out > 0 (got k=%d d_out=%d)", k, d_out);
+  if (col_ptr[0] != 0) return fail(DICTPROJ_ERR_RANGE, "layer: col_ptr[0] must be 0");
+  size_t t = 0;
+  for (int o = 0; o < d_out; ++o) {
+    const int64_t n = (int64_t)col_ptr[o + 1] - col_ptr[o];
+    if (n < 0 || n > k) return fail(DICTPROJ_ERR_RANGE, "layer: column %d has %lld entries (k=%d)", o, (long long)n, k);
+    t += (size_t)((n + 15) / 16) * 16;
+  }
+  *total = t;
+  return DICTPROJ_OK;
+}
+
+int pack_layer_host(const int32_t* col_ptr, const int32_t* atom_idx, const float* vals, int k,
+                    int d_out, uint32_t* pcol_ptr, uint32_t* nnz, uint8_t* codes, uint8_t* scales,
+                    uint8_t* idx, uint16_t* seg_start, float* s_C) {
+  if (!col_ptr || !pcol_ptr || !nnz || !codes || !scales || !idx || !seg_start || !s_C)
+    return fail(DICTPROJ_ERR_NULL, "pack_layer_host: NULL pointer");
+  size_t total = 0;
+  int st = layer_packed_entries(col_ptr, k, d_out, &total);
+  if (st) return st;
+  const size_t nz = (size_t)col_ptr[d_out];
+  if (nz && (!atom_idx || !vals)) return fail(DICTPROJ_ERR_NULL, "pack_layer_host: NULL atom_idx/vals");
+  std::fesetround(FE_TONEAREST);
+  float amax = 0.0f;
+  for (size_t i = 0; i < nz; ++i) {
+    if (!std::isfinite(vals[i])) return fail(DICTPROJ_ERR_VALUE, "pack_layer_host: non-finite value at %zu", i);
+    amax = std::fmax(amax, std::fabs(vals[i]));
+  }
+  for (int o = 0; o < d_out; ++o) {
+    for (int32_t q = col_ptr[o]; q < col_ptr[o + 1]; ++q) {
+      const int32_t a = atom_idx[q];
+      if (a < 0 || a >= k) return fail(DICTPROJ_ERR_RANGE, "pack_layer_host: atom %d out of [0,%d) in column %d", a, k, o);
+      if (q > col_ptr[o] && a <= atom_idx[q - 1]) return fail(DICTPROJ_ERR_RANGE, "pack_layer_host: atoms not ascending/unique in column %d", o);
+    }
+  }
+  const float s = tensor_scale_from_amax(amax);
+  const int nseg = (k + 255) / 256;
+  pcol_ptr[0] = 0;
+  for (int o = 0; o < d_out; ++o) {
+    const uint32_t n = (uint32_t)(col_ptr[o + 1] - col_ptr[o]);
+    nnz[o] = n;
+    pcol_ptr[o + 1] = pcol_ptr[o] + ((n + 15) / 16) * 16;
+  }
+  parallel_for((size_t)d_out, [&](size_t o0, size_t o1) {
+    float blk[16];
+    uint8_t c16[16];
+    for (size_t o = o0; o < o1; ++o) {
+      const int32_t b0 = col_ptr[o];
+      const int32_t n = col_ptr[o + 1] - b0;
+      const uint32_t p0 = pcol_ptr[o];
+      const uint32_t P = pcol_ptr[o + 1] - p0;
+      // segment starts: entries are ascending, so one pass
+      int q = 0;
+      for (int sgi = 0; sgi < nseg; ++sgi) {
+        while (q < n && atom_idx[b0 + q] < 256 * sgi) ++q;
+        seg_start[o * (size_t)nseg + sgi] = (uint16_t)q;
+      }
+      for (uint32_t e = 0; e < P; e += 16) {
+        for (int i = 0; i < 16; ++i) {
+          const uint32_t qq = e + i;
+          blk[i] = qq < (uint32_t)n ? vals[b0 + qq] : 0.0f;
+          idx[p0 + qq] = qq < (uint32_t)n ? (uint8_t)(atom_idx[b0 + qq] & 255) : 0;
+        }
+        scales[(p0 + e) / 16] = quantize_block(blk, s, c16);
+        for (int i = 0; i < 8; ++i) codes[(p0 + e) / 2 + i] = (uint8_t)(c16[2 * i] | (c16[2 * i + 1] << 4));
+      }
+    }
+  });
+  *s_C = s;
+  return DICTPROJ_OK;
+}
+
+}  // namespace dictproj

@@ -1,0 +1,200 @@
+/*
+ * dictproj.h — C ABI of the dictionary-compressed projection library (libdictproj.so).
+ *
+ * What it computes (DictLLM, arXiv 2611.08082; technical review "DictLLM: Shared
+ * Dictionaries for Post-Training Compression", Eq. (1)):
+ *
+ *     W_l ~= D_g C_l,    Z_l = X_l D_g,    Y_l ~= Z_l C_l
+ *
+ * Rows of X are tokens. D_g (d_in x k) is a dictionary shared by a group of
+ * layers; C_l (k x d_out) is a per-layer coefficient matrix with unstructured
+ * sparsity (review, "Prerequisites": each output column may use its own subset
+ * of atoms). Both are stored in NVFP4: 4-bit E2M1 values with one 8-bit E4M3
+ * scale per block of sixteen values (review, "From retained values to measured
+ * decoding": 4.5 bits per value) and one fp32 per-tensor scale.
+ *
+ * Packed layouts (bit-exact contract; the pages leave them open, so these are
+ * plain readings):
+ *   D_g:  codes  uint8[k][d_in/2]  element i of atom j at byte j*d_in/2 + i/2, even
+ *                                  i in the low nibble (atom-major = K-major);
+ *         scales uint8[k][d_in/16] one E4M3 per 16 consecutive d_in entries;
+ *         s_D    fp32.
+ *   C_l:  column o stores its nnz_o atoms in ascending order, zero-padded to
+ *         P_o = 16*ceil(nnz_o/16) entries (code 0, index 0);
+ *         col_ptr   uint32[d_out+1]  padded entry offsets;
+ *         codes     uint8[total/2]   entry e at byte e/2, even e in the low nibble;
+ *         scales    uint8[total/16]  one E4M3 per 16 consecutive stored entries;
+ *         idx       uint8[total]     atom mod 256 (the 8-bit index of the review's
+ *                                    Eq. (12), a = 8, relative to 256-atom segments);
+ *         seg_start uint16[d_out][ceil(k/256)] entry offset (from the column start)
+ *                                    of the first entry with atom >= 256*s;
+ *         s_C       fp32.
+ *   The atom of entry q of a column is 256*s(q) + idx[q], s(q) = max{s : seg_start[s] <= q}.
+ *
+ * Quantiser used by the packers (round to nearest; the paper's Hessian-aware
+ * quantiser needs calibration data and is not part of this library):
+ *   s_T = amax/2688 (1 if amax == 0); per block r = amax_b/(6 s_T) rounded to
+ *   the nearest E4M3 (ties to even, saturating at 448); each value
+ *   x/(E4M3(sc) s_T) rounded to the nearest E2M1 (ties to even mantissa,
+ *   saturating at 6, -0 written as 0); a block whose scale is 0 stores zeros.
+ *   All arithmetic is IEEE fp32.
+ *
+ * Conventions for every entry point:
+ *   - Returns a dictproj_status (0 = DICTPROJ_OK). Nothing throws across the ABI.
+ *     On error a thread-local message is available from dictproj_last_error().
+ *   - Arguments are validated before any allocation, copy or kernel launch; an
+ *     invalid call has no side effect.
+ *   - "host" pointers are ordinary CPU memory; "device" pointers are CUDA device
+ *     memory of the device that was current when the handle was created.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = the legacy default stream).
+ *   - The library owns the memory behind handles; the caller owns everything it
+ *     passes in (inputs are only read, outputs only written).
+ */
+#ifndef DICTPROJ_H
+#define DICTPROJ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum dictproj_status {
+  DICTPROJ_OK = 0,
+  DICTPROJ_ERR_NULL = -1,        /* a required pointer is NULL */
+  DICTPROJ_ERR_SHAPE = -2,       /* a size is zero, negative or not a multiple of 16 where required */
+  DICTPROJ_ERR_ALIGN = -3,       /* X or Y is not 16-byte aligned */
+  DICTPROJ_ERR_MISMATCH = -4,    /* layer and group disagree on k, or live on different devices */
+  DICTPROJ_ERR_RANGE = -5,       /* M outside [1, max_tokens], an atom index >= k, unsorted atoms */
+  DICTPROJ_ERR_CUDA = -6,        /* a CUDA runtime call or kernel launch failed (or no device) */
+  DICTPROJ_ERR_OOM = -7,         /* device or host allocation failed */
+  DICTPROJ_ERR_TIMEOUT = -8,     /* a bounded device-side wait gave up (read by dictproj_check) */
+  DICTPROJ_ERR_UNSUPPORTED = -9, /* valid but not supported here (e.g. not an sm_100 device) */
+  DICTPROJ_ERR_VALUE = -10       /* a non-finite input value */
+} dictproj_status;
+
+/* Opaque handles. A group owns the packed D_g on the device plus the scratch for
+ * Z; a layer owns the packed C_l. Calls that share a group use the group's Z
+ * scratch, so they must be ordered on one stream (or otherwise serialised). */
+typedef struct dictproj_group dictproj_group;
+typedef struct dictproj_layer dictproj_layer;
+
+/* ------------------------------------------------------------------------- */
+/* Host-only packing (no GPU needed). Review Algorithm 2, export step: the     */
+/* dictionary, per-layer codes, scales and support.                            */
+/* ------------------------------------------------------------------------- */
+
+/* Sizes of the packed D_g arrays. d_in % 16 == 0, k >= 1. */
+int dictproj_group_packed_sizes(int d_in, int k, size_t* codes_bytes, size_t* scales_bytes);
+
+/* Quantise D (host fp32, d_in x k, row-major) into caller buffers of the sizes
+ * above. Errors: NULL, SHAPE, VALUE (non-finite entry). */
+int dictproj_pack_group_host(const float* D, int d_in, int k, uint8_t* codes, uint8_t* scales,
+                             float* s_D);
+
+/* Total padded entries of C_l given its unpadded CSC column pointers
+ * (host int32[d_out+1], col_ptr[0] == 0, non-decreasing, each column <= k entries). */
+int dictproj_layer_packed_entries(const int32_t* col_ptr, int k, int d_out, size_t* total_entries);
+
+/* Quantise and lay out C_l (host CSC: col_ptr int32[d_out+1], atom_idx int32[nnz] ascending
+ * and unique within each column and < k, vals fp32[nnz]) into caller buffers:
+ * pcol_ptr uint32[d_out+1], nnz uint32[d_out], codes uint8[total/2], scales uint8[total/16],
+ * idx uint8[total], seg_start uint16[d_out*ceil(k/256)], s_C. k <= 65535.
+ * Errors: NULL, SHAPE, RANGE (bad index or order), VALUE (non-finite value). */
+int dictproj_pack_layer_host(const int32_t* col_ptr, const int32_t* atom_idx, const float* vals,
+                             int k, int d_out, uint32_t* pcol_ptr, uint32_t* nnz, uint8_t* codes,
+                             uint8_t* scales, uint8_t* idx, uint16_t* seg_start, float* s_C);
+
+/* ------------------------------------------------------------------------- */
+/* Device objects                                                             */
+/* ------------------------------------------------------------------------- */
+
+/* Upload an already packed D_g (host arrays as produced above) to the current
+ * device and allocate the Z scratch for up to max_tokens tokens per call.
+ * Errors: NULL, SHAPE, RANGE (max_tokens < 1), CUDA, OOM. */
+int dictproj_group_upload(const uint8_t* codes, const uint8_t* scales, float s_D, int d_in, int k,
+                          int max_tokens, dictproj_group** out);
+
+/* dictproj_pack_group_host + dictproj_group_upload. */
+int dictproj_pack_group(const float* D, int d_in, int k, int max_tokens, dictproj_group** out);
+
+/* Upload an already packed C_l. Errors: NULL, SHAPE, CUDA, OOM. */
+int dictproj_layer_upload(const uint32_t* pcol_ptr, const uint8_t* codes, const uint8_t* scales,
+                          const uint8_t* idx, const uint16_t* seg_start, float s_C, int k,
+                          int d_out, dictproj_layer** out);
+
+/* dictproj_pack_layer_host + dictproj_layer_upload. */
+int dictproj_pack_layer(const int32_t* col_ptr, const int32_t* atom_idx, const float* vals, int k,
+                        int d_out, dictproj_layer** out);
+
+/* Convenience: pack one group and its n_layers layers (all with the same k).
+ * On error nothing is left allocated. */
+int dictproj_pack(const float* D, int d_in, int k, int max_tokens, int n_layers,
+                  const int32_t* const* col_ptr, const int32_t* const* atom_idx,
+                  const float* const* vals, const int* d_out, dictproj_group** group_out,
+                  dictproj_layer** layers_out);
+
+/* Copy the packed bytes back to host buffers of the packed sizes (for
+ * bit-exact checks). Errors: NULL, CUDA. */
+int dictproj_group_export(const dictproj_group* g, uint8_t* codes, uint8_t* scales, float* s_D);
+int dictproj_layer_export(const dictproj_layer* l, uint32_t* pcol_ptr, uint8_t* codes,
+                          uint8_t* scales, uint8_t* idx, uint16_t* seg_start, float* s_C);
+
+/* Shape queries. Any output pointer may be NULL. */
+int dictproj_group_info(const dictproj_group* g, int* d_in, int* k, int* max_tokens);
+int dictproj_layer_info(const dictproj_layer* l, int* k, int* d_out, size_t* total_entries,
+                        size_t* nnz_total);
+
+void dictproj_free_group(dictproj_group* g); /* NULL is a no-op */
+void dictproj_free_layer(dictproj_layer* l); /* NULL is a no-op */
+
+/* ------------------------------------------------------------------------- */
+/* Forward                                                                    */
+/* ------------------------------------------------------------------------- */
+
+/* Y = X * (D_g) * (C_l) (Eq. (1)): X device fp16 [M][d_in] row-major, Y device
+ * fp16 [M][d_out] row-major, both 16-byte aligned; 1 <= M <= group max_tokens.
+ * Accumulation is fp32; Z is fp32 for M <= 8 (decode path) and fp16 with s_D
+ * applied before rounding for larger M (prefill path).
+ * Asynchronous on `stream`: no allocation, no host synchronisation. Kernels are
+ * launched with programmatic dependent launch; each kernel waits for the
+ * preceding work on the stream before it reads X or writes Z / Y (packed
+ * weights, which nothing writes after upload, may be prefetched earlier).
+ * Errors (checked before any launch): NULL, RANGE (M), MISMATCH (k or device),
+ * ALIGN; CUDA if a launch fails. */
+int dictproj_forward(const void* X, int M, const dictproj_layer* layer,
+                     const dictproj_group* group, void* Y, void* stream);
+
+/* Forward with an explicit path: DICTPROJ_PATH_AUTO, DICTPROJ_PATH_DECODE (M <= 8)
+ * or DICTPROJ_PATH_PREFILL (any M). Errors as dictproj_forward, plus
+ * UNSUPPORTED for DECODE with M > 8. */
+enum { DICTPROJ_PATH_AUTO = 0, DICTPROJ_PATH_DECODE = 1, DICTPROJ_PATH_PREFILL = 2 };
+int dictproj_forward_path(const void* X, int M, const dictproj_layer* layer,
+                          const dictproj_group* group, void* Y, void* stream, int path);
+
+/* The two stages of Eq. (1) as separate calls (decode path, 1 <= M <= 8).
+ * Z is caller-owned device fp32 [k][mp], 16-byte aligned, mp = 1, 2, 4 or 8 = the
+ * smallest power of two >= M; column m of Z holds token m (columns >= M are zero).
+ *   dictionary stage:   Z = X D_g        (X device fp16 [M][d_in])
+ *   coefficient stage:  Y = Z C_l        (Y device fp16 [M][d_out])
+ * Same validation, ordering and asynchrony as dictproj_forward; UNSUPPORTED for M > 8. */
+int dictproj_dictionary_stage(const void* X, int M, const dictproj_group* group, float* Z, void* stream);
+int dictproj_coefficient_stage(const float* Z, int M, const dictproj_layer* layer, void* Y, void* stream);
+
+/* Read (and clear) the device error word that bounded device waits set, after
+ * synchronising `stream`. Returns OK or TIMEOUT (or CUDA). */
+int dictproj_check(void* stream);
+
+/* Last error message of the calling thread ("" if none). */
+const char* dictproj_last_error(void);
+/* Static name of a status code. */
+const char* dictproj_status_string(int status);
+/* Library ABI version (major*10000 + minor*100 + patch). */
+int dictproj_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DICTPROJ_H */

@@ -80,6 +80,25 @@ def forward_factored(X: np.ndarray, pd: dict, pc: dict) -> np.ndarray:
     return sparse_columns_product(Z, pc)
 
 
+def decode_projection(pd: dict, pc: dict) -> dict:
+    """Both factors decoded once: D-hat (d_in, k) and C's entries (atoms, values)."""
+    atoms, vals = decode_coeff_entries(pc)
+    return {"Dhat": decode_dictionary(pd), "atoms": atoms, "vals": vals,
+            "ptr": pc["col_ptr"].astype(np.int64), "d_out": pc["d_out"]}
+
+
+def forward_factored_decoded(X: np.ndarray, dec: dict) -> np.ndarray:
+    """(X D) C in fp64 on factors already decoded by decode_projection."""
+    Z = np.asarray(X).astype(np.float64) @ dec["Dhat"]
+    ptr = dec["ptr"]
+    Y = np.zeros((Z.shape[0], dec["d_out"]), dtype=np.float64)
+    contrib = Z[:, dec["atoms"]] * dec["vals"][None, :]
+    nonempty = np.flatnonzero(np.diff(ptr) > 0)
+    if nonempty.size:
+        Y[:, nonempty] = np.add.reduceat(contrib, ptr[nonempty], axis=1)
+    return Y
+
+
 def forward_reference(X: np.ndarray, pd: dict, pc: dict) -> np.ndarray:
     """X (D C) in fp64: decode both factors, expand W densely, multiply."""
     W = expand_weight(decode_dictionary(pd), decode_coeff_dense(pc))
@@ -145,5 +164,6 @@ def within_tolerance(y_test: np.ndarray, y_ref: np.ndarray, rel_fro: float = 5e-
 __all__ = [
     "SEG", "decode_dictionary", "decode_coeff_entries", "decode_coeff_dense", "expand_weight",
     "forward_dense", "sparse_columns_product", "forward_factored", "forward_reference",
-    "forward_brute", "sampled_outputs", "within_tolerance",
+    "forward_brute", "sampled_outputs", "within_tolerance", "decode_projection",
+    "forward_factored_decoded",
 ]

@@ -1,0 +1,206 @@
+"""Parity of the CUDA path (through the C ABI) against the fp64 oracle.
+
+Bar (fp16 in/out, fp32 accumulation): relative Frobenius error <= 5e-3 and every
+element |err| <= 1e-2 * (1 + |y|). Packed bytes are compared bit for bit.
+"""
+import numpy as np
+import pytest
+
+import synth
+
+pytestmark = pytest.mark.gpu
+
+torch = pytest.importorskip("torch")
+if not torch.cuda.is_available():  # pragma: no cover - CPU container
+    pytest.skip("needs a CUDA device", allow_module_level=True)
+
+import dictionary_compressed_linear_b200 as dp  # noqa: E402
+from gpu_helpers import (assert_parity, device_projection, oracle_forward,  # noqa: E402
+                         oracle_projection, run_forward)
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _build():
+    from dictionary_compressed_linear_b200 import build
+    build.build()
+
+
+def _case(cfg, group, ptype, layer, d_in, k, d_out, rho):
+    D = synth.gen_dictionary(cfg, group, ptype, d_in, k)
+    C = synth.gen_coeff(cfg, group, ptype, layer, k, d_out, rho)
+    return D, C
+
+
+# ------------------------------------------------------------------ tiny workload
+@pytest.mark.parametrize("M", [1, 4])
+def test_tiny_workload_all_layers(M):
+    w = synth.tiny()
+    for p in w.projections:
+        D, C = synth.projection_inputs(p)
+        g, l = device_projection(D, C, max_tokens=8)
+        pd, pc = oracle_projection(D, C)
+        X = synth.gen_activations(0, p.layer, p.site, M, p.d_in)
+        y = run_forward(g, l, X)
+        assert_parity(y, oracle_forward(X, pd, pc, dense=True), f"tiny layer {p.layer} M={M}")
+
+
+# ------------------------------------------------------------------ LLaMA shapes, decode
+@pytest.mark.parametrize("name", ["q", "o"])
+def test_attention_projection_m1(name):
+    w = synth.attention_group()
+    p = [q for q in w.projections if q.name == name and q.layer == 1][0]
+    D, C = synth.projection_inputs(p)
+    g, l = device_projection(D, C, max_tokens=8)
+    pd, pc = oracle_projection(D, C)
+    X = synth.gen_activations(1, p.layer, p.site, 1, p.d_in)
+    assert_parity(run_forward(g, l, X), oracle_forward(X, pd, pc), f"attn {name}")
+
+
+@pytest.mark.parametrize("name,M", [("gate", 1), ("down", 1), ("up", 8), ("down", 8)])
+def test_mlp_projection(name, M):
+    w = synth.mlp_groups()
+    p = [q for q in w.projections if q.name == name and q.layer == 0][0]
+    D, C = synth.projection_inputs(p)
+    g, l = device_projection(D, C, max_tokens=8)
+    pd, pc = oracle_projection(D, C)
+    X = synth.gen_activations(2, p.layer, p.site, M, p.d_in)
+    assert_parity(run_forward(g, l, X), oracle_forward(X, pd, pc), f"mlp {name} M={M}")
+
+
+# ------------------------------------------------------------------ ragged token counts
+@pytest.fixture(scope="module")
+def mid():
+    D, C = _case(10, 0, 0, 0, 512, 256, 300, 0.3)
+    g, l = device_projection(D, C, max_tokens=160)
+    pd, pc = oracle_projection(D, C)
+    return g, l, pd, pc
+
+
+@pytest.mark.parametrize("M", [1, 2, 3, 5, 6, 7, 8])
+def test_decode_ragged_m(mid, M):
+    g, l, pd, pc = mid
+    X = synth.gen_activations(10, M, 0, M, 512)
+    assert_parity(run_forward(g, l, X), oracle_forward(X, pd, pc, dense=True), f"M={M}")
+
+
+@pytest.mark.parametrize("M", [1, 8, 9, 40, 128, 160])
+def test_prefill_path(mid, M):
+    g, l, pd, pc = mid
+    X = synth.gen_activations(10, M, 1, M, 512, outlier_frac=0.01)
+    y = run_forward(g, l, X, path=dp.PATH_PREFILL)
+    assert_parity(y, oracle_forward(X, pd, pc, dense=True), f"prefill M={M}")
+
+
+# ------------------------------------------------------------------ degenerate layers
+def _custom_layer(k, d_out, cols, seed=0):
+    rng = np.random.default_rng(seed)
+    ptr = np.zeros(d_out + 1, np.int32)
+    ptr[1:] = np.cumsum([c.size for c in cols])
+    atoms = np.concatenate(cols).astype(np.int32) if cols else np.zeros(0, np.int32)
+    vals = (rng.standard_normal(atoms.size) / np.sqrt(k)).astype(np.float32)
+    return synth.SparseCoeff(k=k, d_out=d_out, col_ptr=ptr, atom_idx=atoms, vals=vals)
+
+
+@pytest.mark.parametrize("M", [1, 3, 8, 20])
+def test_degenerate_columns(M):
+    rng = np.random.default_rng(3)
+    k, d_in = 1008, 64
+    kinds = [0, k, 1, 15, 16, 17, 255, 256, 257, 3]
+    cols = []
+    for o in range(45):  # d_out not a multiple of the 32-column CTA tile
+        n = kinds[o % len(kinds)]
+        cols.append(np.sort(rng.choice(k, size=n, replace=False)))
+    cols[7] = np.array([0, 600, 1007])  # empty segments in between
+    cols[8] = np.arange(240, 272)  # one block straddling a segment boundary
+    C = _custom_layer(k, 45, cols)
+    D = synth.gen_dictionary(11, 0, 0, d_in, k)
+    g, l = device_projection(D, C, max_tokens=32)
+    pd, pc = oracle_projection(D, C)
+    X = synth.gen_activations(11, 0, 0, M, d_in)
+    y = run_forward(g, l, X)
+    yr = oracle_forward(X, pd, pc, dense=True)
+    assert_parity(y, yr, f"degenerate M={M}")
+    assert np.all(y[:, 0] == 0.0)  # an empty column gives exact zeros
+
+
+def test_smallest_shapes():
+    D, C = _case(12, 0, 0, 0, 32, 16, 1, 1.0)
+    g, l = device_projection(D, C, max_tokens=1)
+    pd, pc = oracle_projection(D, C)
+    X = synth.gen_activations(12, 0, 0, 1, 32)
+    assert_parity(run_forward(g, l, X), oracle_forward(X, pd, pc, dense=True), "smallest")
+
+
+def test_all_zero_input_gives_zero():
+    D, C = _case(13, 0, 0, 0, 256, 128, 64, 0.5)
+    g, l = device_projection(D, C, max_tokens=4)
+    y = run_forward(g, l, np.zeros((4, 256), np.float16))
+    assert np.all(y == 0.0)
+
+
+# ------------------------------------------------------------------ bit-exact packed bytes
+def test_device_bytes_match_oracle_layout():
+    D, C = _case(14, 0, 0, 0, 4096, 2048, 700, 0.3)
+    g, l = device_projection(D, C, max_tokens=1)
+    pd, pc = oracle_projection(D, C)
+    eg = dp.dictproj_group_export(g)
+    assert np.array_equal(eg["codes"], pd["codes"]) and np.array_equal(eg["scales"], pd["scales"])
+    assert eg["s"] == pd["s"]
+    el = dp.dictproj_layer_export(l)
+    for n in ("col_ptr", "codes", "scales", "idx", "seg_start"):
+        assert np.array_equal(el[n], pc[n]), n
+    assert el["s"] == pc["s"]
+
+
+# ------------------------------------------------------------------ determinism and graphs
+def test_deterministic_bits(mid):
+    g, l, pd, pc = mid
+    X = synth.gen_activations(10, 99, 0, 8, 512)
+    a = run_forward(g, l, X)
+    b = run_forward(g, l, X)
+    assert np.array_equal(a, b)
+
+
+def test_cuda_graph_capture_and_side_stream(mid):
+    g, l, pd, pc = mid
+    X = torch.from_numpy(synth.gen_activations(10, 98, 0, 4, 512)).cuda()
+    Y = torch.zeros((4, 300), dtype=torch.float16, device="cuda")
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        dp.dictproj_forward(X.data_ptr(), 4, l, g, Y.data_ptr(), s.cuda_stream)  # warm-up
+    s.synchronize()
+    ref = Y.clone()
+    Y.zero_()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=s):
+        dp.dictproj_forward(X.data_ptr(), 4, l, g, Y.data_ptr(), s.cuda_stream)
+    graph.replay()
+    torch.cuda.synchronize()
+    assert torch.equal(Y, ref)
+    yr = oracle_forward(X.cpu().numpy(), pd, pc, dense=True)
+    assert_parity(Y.float().cpu().numpy().astype(np.float64), yr, "graph")
+
+
+def test_chain_of_calls_sharing_a_group():
+    # two layers of one group, the second reading the first's output: the
+    # dependency wait must order Z scratch reuse and X reads
+    D = synth.gen_dictionary(15, 0, 0, 256, 128)
+    C1 = synth.gen_coeff(15, 0, 0, 0, 128, 256, 0.5)
+    C2 = synth.gen_coeff(15, 0, 0, 1, 128, 256, 0.5)
+    g = dp.dictproj_pack_group(D, 8)
+    l1 = dp.dictproj_pack_layer(C1.col_ptr, C1.atom_idx, C1.vals, 128, 256)
+    l2 = dp.dictproj_pack_layer(C2.col_ptr, C2.atom_idx, C2.vals, 128, 256)
+    pd, pc1 = oracle_projection(D, C1)
+    _, pc2 = oracle_projection(D, C2)
+    X = torch.from_numpy(synth.gen_activations(15, 0, 0, 2, 256)).cuda()
+    Y1 = torch.empty((2, 256), dtype=torch.float16, device="cuda")
+    Y2 = torch.empty((2, 256), dtype=torch.float16, device="cuda")
+    st = torch.cuda.current_stream().cuda_stream
+    for _ in range(3):
+        dp.dictproj_forward(X.data_ptr(), 2, l1, g, Y1.data_ptr(), st)
+        dp.dictproj_forward(Y1.data_ptr(), 2, l2, g, Y2.data_ptr(), st)
+    torch.cuda.synchronize()
+    y1 = Y1.float().cpu().numpy().astype(np.float64)
+    assert_parity(y1, oracle_forward(X.cpu().numpy(), pd, pc1, dense=True), "chain 1")
+    y2 = Y2.float().cpu().numpy().astype(np.float64)
+    assert_parity(y2, oracle_forward(Y1.cpu().numpy(), pd, pc2, dense=True), "chain 2")

@@ -1,0 +1,137 @@
+"""CPU tests of the C-ABI library: it loads, exports every declared symbol, its
+host packer matches the oracle's packed layouts bit for bit, and its host-side
+validation returns the documented status codes. No compute call needs a GPU here."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+import synth
+from oracle.pack import pack_coeff, pack_dictionary
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def dp():
+    import dictionary_compressed_linear_b200 as m
+    from dictionary_compressed_linear_b200 import build
+    build.build()
+    return m
+
+
+def _declared_symbols():
+    names = set()
+    for fn in os.listdir(os.path.join(ROOT, "include")):
+        if fn.endswith(".h"):
+            txt = open(os.path.join(ROOT, "include", fn)).read()
+            txt = re.sub(r"/\*.*?\*/", "", txt, flags=re.S)
+            names |= set(re.findall(r"\b(dictproj_[a-z0-9_]+)\s*\(", txt))
+    return names
+
+
+def test_library_exports_every_declared_symbol(dp):
+    lib = ctypes.CDLL(dp.LIB_PATH)
+    declared = _declared_symbols()
+    assert len(declared) >= 20
+    for name in sorted(declared):
+        assert hasattr(lib, name), name
+    bound = {n for n, _, _ in dp.SIGNATURES}
+    assert declared == bound, declared ^ bound
+
+
+def test_version_and_status_strings(dp):
+    assert dp.dictproj_version() >= 10000
+    assert dp.dictproj_status_string(0) == "DICTPROJ_OK"
+    assert dp.dictproj_status_string(-8) == "DICTPROJ_ERR_TIMEOUT"
+
+
+def _same_layer(a, b):
+    for n in ("col_ptr", "nnz", "codes", "scales", "idx", "seg_start"):
+        assert np.array_equal(a[n], b[n]), n
+    assert a["s"] == b["s"]
+
+
+@pytest.mark.parametrize("d_in,k", [(256, 128), (4096, 2048), (11008, 3072), (32, 16), (96, 272)])
+def test_group_packer_bit_exact(dp, d_in, k):
+    D = synth.gen_dictionary(7, d_in, k, d_in, k)
+    a = dp.dictproj_pack_group_host(D)
+    b = pack_dictionary(D)
+    assert np.array_equal(a["codes"], b["codes"])
+    assert np.array_equal(a["scales"], b["scales"])
+    assert a["s"] == b["s"]
+
+
+@pytest.mark.parametrize("k,d_out,rho", [(128, 256, 0.5), (2048, 512, 0.3), (3072, 300, 0.25),
+                                         (272, 45, 0.05), (16, 7, 1.0), (512, 33, 0.0)])
+def test_layer_packer_bit_exact(dp, k, d_out, rho):
+    C = synth.gen_coeff(7, k, d_out, 1, k, d_out, rho)
+    a = dp.dictproj_pack_layer_host(C.col_ptr, C.atom_idx, C.vals, k, d_out)
+    b = pack_coeff(C.col_ptr, C.atom_idx, C.vals, k, d_out)
+    _same_layer(a, b)
+
+
+def test_layer_packer_bit_exact_ragged_columns(dp):
+    # columns of different lengths, including empty and full ones, atoms in sparse segments
+    rng = np.random.default_rng(11)
+    k, d_out = 1000, 20
+    cols = []
+    for o in range(d_out):
+        n = [0, k, 1, 17, 255, 256, 3][o % 7]
+        cols.append(np.sort(rng.choice(k, size=n, replace=False)))
+    cols[5] = np.array([3, 700, 999])  # segments 1 and 2 empty
+    ptr = np.zeros(d_out + 1, np.int32)
+    ptr[1:] = np.cumsum([c.size for c in cols])
+    atoms = np.concatenate(cols).astype(np.int32)
+    vals = (rng.standard_normal(atoms.size) * np.exp(rng.uniform(-8, 4, atoms.size))).astype(np.float32)
+    vals[::7] = 0.0
+    a = dp.dictproj_pack_layer_host(ptr, atoms, vals, k, d_out)
+    b = pack_coeff(ptr, atoms, vals, k, d_out)
+    _same_layer(a, b)
+
+
+def test_group_packer_extreme_values(dp):
+    rng = np.random.default_rng(5)
+    D = (rng.standard_normal((64, 32)) * np.exp(rng.uniform(-30, 30, (64, 32)))).astype(np.float32)
+    D[:16, 0] = 0.0
+    D[16:32, 1] = 1e-38
+    a = dp.dictproj_pack_group_host(D)
+    b = pack_dictionary(D)
+    assert np.array_equal(a["codes"], b["codes"]) and np.array_equal(a["scales"], b["scales"])
+
+
+def test_host_validation(dp):
+    from dictionary_compressed_linear_b200 import DictprojError
+    with pytest.raises(DictprojError) as e:
+        dp.dictproj_pack_group_host(np.ones((24, 4), np.float32))
+    assert e.value.status == -2
+    bad = np.ones((32, 4), np.float32)
+    bad[3, 1] = np.nan
+    with pytest.raises(DictprojError) as e:
+        dp.dictproj_pack_group_host(bad)
+    assert e.value.status == -10
+    with pytest.raises(DictprojError) as e:  # unsorted atoms
+        dp.dictproj_pack_layer_host(np.array([0, 2]), np.array([5, 1]), np.ones(2), 16, 1)
+    assert e.value.status == -5
+    with pytest.raises(DictprojError) as e:  # atom out of range
+        dp.dictproj_pack_layer_host(np.array([0, 1]), np.array([16]), np.ones(1), 16, 1)
+    assert e.value.status == -5
+    with pytest.raises(DictprojError) as e:  # column longer than k
+        dp.dictproj_layer_packed_entries(np.array([0, 20]), 16, 1)
+    assert e.value.status == -5
+    lib = dp.lib()
+    assert lib.dictproj_pack_group_host(None, 32, 16, None, None, None) == -1
+    assert dp.dictproj_forward_status(0, 1, None, None, 0) == -1
+    assert "NULL" in dp.dictproj_last_error()
+
+
+def test_device_calls_fail_loudly_without_gpu(dp):
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present")
+    from dictionary_compressed_linear_b200 import DictprojError
+    with pytest.raises(DictprojError) as e:
+        dp.dictproj_pack_group(np.ones((32, 16), np.float32), 1)
+    assert e.value.status == -6

@@ -44,6 +44,12 @@ def test_tiny_workload_dense_equals_factored():
             assert F.within_tolerance(y2, y1)[0]
 
 
+def test_pre_decoded_forward_is_the_same():
+    X, pd, pc = _tiny_case(M=3)
+    dec = F.decode_projection(pd, pc)
+    assert np.array_equal(F.forward_factored_decoded(X, dec), F.forward_factored(X, pd, pc))
+
+
 def test_linearity_in_x():
     X, pd, pc = _tiny_case(M=3)
     X2, _, _ = _tiny_case(M=3, seed=5)
