@@ -151,6 +151,10 @@ void dictproj_free_layer(dictproj_layer* l) {
   cudaFree(l->idx);
   cudaFree(l->seg_start);
   cudaFree(l->cexp);
+  for (int i = 0; i < 2; ++i) {
+    cudaFree(l->chunks[i]);
+    cudaFree(l->cta_ptr[i]);
+  }
   delete l;
 }
 
@@ -231,6 +235,13 @@ int dictproj_layer_upload(const uint32_t* pcol_ptr, const uint8_t* codes, const 
     if (ss[0] != 0) return fail(DICTPROJ_ERR_RANGE, "layer_upload: seg_start[%d][0] != 0", o);
     for (int s = 1; s < nseg; ++s)
       if (ss[s] < ss[s - 1] || ss[s] > n) return fail(DICTPROJ_ERR_RANGE, "layer_upload: seg_start of column %d not monotone", o);
+    // every entry's atom 256*s(q) + idx[q] must be < k (the kernels index Z with it)
+    int s = 0;
+    for (uint32_t q = 0; q < n; ++q) {
+      while (s + 1 < nseg && ss[s + 1] <= q) ++s;
+      if (256 * s + (int)idx[pcol_ptr[o] + q] >= k)
+        return fail(DICTPROJ_ERR_RANGE, "layer_upload: column %d entry %u addresses atom >= k", o, q);
+    }
   }
   int dev, st;
   if ((st = ensure_device(&dev))) return st;
@@ -260,8 +271,34 @@ int dictproj_layer_upload(const uint32_t* pcol_ptr, const uint8_t* codes, const 
     cudaGetLastError();
     return cuda_fail(e, "layer_upload: copy to device");
   }
-  // true entry count is not part of the packed arrays; derive it from the codes? No:
-  // callers that need it use dictproj_pack_layer, which records it below.
+  // decode-path work plans: one and two CTAs per SM, entry-balanced column runs
+  int n_sm = 0, smem_sm = 0;
+  if ((e = cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess ||
+      (e = cudaDeviceGetAttribute(&smem_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev)) != cudaSuccess) {
+    dictproj_free_layer(l);
+    return cuda_fail(e, "layer_upload: device attributes");
+  }
+  l->smem_per_sm = smem_sm;
+  for (int pi = 0; pi < 2; ++pi) {
+    std::vector<uint32_t> plan;
+    std::vector<int> cta_ptr;
+    const int G = n_sm * (pi + 1);
+    if (!plan_coeff_chunks(pcol_ptr, d_out, nseg, G, plan, cta_ptr)) break;
+    if ((e = dmalloc((void**)&l->chunks[pi], plan.size() * sizeof(uint32_t))) ||
+        (e = dmalloc((void**)&l->cta_ptr[pi], cta_ptr.size() * sizeof(int)))) {
+      dictproj_free_layer(l);
+      cudaGetLastError();
+      return fail(DICTPROJ_ERR_OOM, "layer_upload: device allocation failed (%s)", cudaGetErrorName(e));
+    }
+    if ((e = h2d(l->chunks[pi], plan.data(), plan.size() * sizeof(uint32_t))) ||
+        (e = h2d(l->cta_ptr[pi], cta_ptr.data(), cta_ptr.size() * sizeof(int)))) {
+      dictproj_free_layer(l);
+      cudaGetLastError();
+      return cuda_fail(e, "layer_upload: copy to device");
+    }
+    l->n_cta[pi] = G;
+  }
+  // the true entry count is not part of the packed arrays; dictproj_pack_layer records it
   l->nnz_total = 0;
   *out = l;
   return DICTPROJ_OK;
@@ -442,6 +479,9 @@ int dictproj_check(void* stream) {
   clear_error();
   cudaError_t e = cudaStreamSynchronize((cudaStream_t)stream);
   if (e != cudaSuccess) return cuda_fail(e, "check: stream synchronize");
+  unsigned int word = 0;
+  if ((e = take_decode_error(&word)) != cudaSuccess) return cuda_fail(e, "check: read error word");
+  if (word) return fail(DICTPROJ_ERR_TIMEOUT, "check: a bounded device wait gave up (error word 0x%x)", word);
   return DICTPROJ_OK;
 }
 

@@ -54,4 +54,10 @@ struct dictproj_layer {
   uint8_t* idx;            // [total]
   uint16_t* seg_start;     // [d_out][nseg]
   uint16_t* cexp;          // prefill: C expanded to fp16, [d_out][k] (lazy)
+  // decode-path work plan (see plan_coeff_chunks): chunk {o_b, o_e, e_b, e_e}
+  // plan[0]: one CTA per SM; plan[1]: two CTAs per SM (used when two fit)
+  uint32_t* chunks[2];     // [n_chunks][4], device; NULL -> direct kernel
+  int* cta_ptr[2];         // [n_cta+1], device
+  int n_cta[2];
+  int smem_per_sm;         // bytes of shared memory per SM on this device
 };

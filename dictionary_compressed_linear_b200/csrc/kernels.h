@@ -4,6 +4,8 @@
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
+#include <vector>
+
 #include "dictproj_internal.h"
 
 namespace dictproj {
@@ -16,5 +18,11 @@ cudaError_t launch_dict_decode(const dictproj_group* g, const __half* X, int M, 
                                cudaStream_t stream);
 cudaError_t launch_coeff_decode(const dictproj_layer* l, const float* Z, int M, int mp, __half* Y,
                                 cudaStream_t stream);
+
+// Work plan of the chunked coefficient kernel for a grid of G CTAs (host side).
+bool plan_coeff_chunks(const uint32_t* pcol_ptr, int d_out, int nseg, int G, std::vector<uint32_t>& chunks,
+                       std::vector<int>& cta_ptr);
+// Read and clear the device error word of the decode kernels.
+cudaError_t take_decode_error(unsigned int* out);
 
 }  // namespace dictproj
