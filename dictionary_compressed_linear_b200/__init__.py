@@ -8,7 +8,8 @@ binding of that ABI; it loads the in-tree library and fails loudly if it is
 missing.
 """
 from .binding import (  # noqa: F401
-    PATH_AUTO, PATH_DECODE, PATH_PREFILL, DictprojError, Group, Layer, LIB_PATH, SIGNATURES, lib,
+    PATH_AUTO, PATH_DECODE, PATH_PREFILL, DeviceGroup, DeviceLayer, DictprojError, Group, Layer, LIB_PATH,
+    SIGNATURES, dictproj_forward_noalloc, dictproj_forward_noalloc_status, lib,
     dictproj_check, dictproj_coefficient_stage, dictproj_dictionary_stage, dictproj_forward, dictproj_forward_path, dictproj_forward_status,
     dictproj_group_export, dictproj_group_info, dictproj_group_packed_sizes, dictproj_group_upload,
     dictproj_last_error, dictproj_layer_export, dictproj_layer_info, dictproj_layer_packed_entries,

@@ -39,6 +39,18 @@ _f32p = C.POINTER(C.c_float)
 _szp = C.POINTER(C.c_size_t)
 _intp = C.POINTER(C.c_int)
 
+class DeviceGroup(C.Structure):
+    """dictproj_device_group: caller-owned device copies of a packed D_g."""
+    _fields_ = [("codes", C.c_void_p), ("scales", C.c_void_p), ("s", C.c_float), ("d_in", C.c_int),
+                ("k", C.c_int)]
+
+
+class DeviceLayer(C.Structure):
+    """dictproj_device_layer: caller-owned device copies of a packed C_l."""
+    _fields_ = [("col_ptr", C.c_void_p), ("codes", C.c_void_p), ("scales", C.c_void_p), ("idx", C.c_void_p),
+                ("seg_start", C.c_void_p), ("s", C.c_float), ("k", C.c_int), ("d_out", C.c_int)]
+
+
 # (name, restype, argtypes) for every entry point declared in include/dictproj.h
 SIGNATURES = [
     ("dictproj_group_packed_sizes", C.c_int, [C.c_int, C.c_int, _szp, _szp]),
@@ -66,6 +78,8 @@ SIGNATURES = [
      [C.c_void_p, C.c_int, C.c_void_p, C.c_void_p, C.c_void_p, C.c_void_p, C.c_int]),
     ("dictproj_dictionary_stage", C.c_int, [C.c_void_p, C.c_int, C.c_void_p, C.c_void_p, C.c_void_p]),
     ("dictproj_coefficient_stage", C.c_int, [C.c_void_p, C.c_int, C.c_void_p, C.c_void_p, C.c_void_p]),
+    ("dictproj_forward_noalloc", C.c_int,
+     [C.POINTER(DeviceGroup), C.POINTER(DeviceLayer), C.c_void_p, C.c_int, C.c_void_p, C.c_void_p]),
     ("dictproj_check", C.c_int, [C.c_void_p]),
     ("dictproj_last_error", C.c_char_p, []),
     ("dictproj_status_string", C.c_char_p, [C.c_int]),
@@ -313,6 +327,19 @@ def dictproj_dictionary_stage(X_ptr: int, M: int, group: Group, Z_ptr: int, stre
 def dictproj_coefficient_stage(Z_ptr: int, M: int, layer: Layer, Y_ptr: int, stream: int = 0):
     _check(lib().dictproj_coefficient_stage(C.c_void_p(Z_ptr), M, layer.handle, C.c_void_p(Y_ptr),
                                             C.c_void_p(stream)))
+
+
+def dictproj_forward_noalloc(group: DeviceGroup, layer: DeviceLayer, X_ptr: int, M: int, Y_ptr: int,
+                             stream: int = 0):
+    _check(lib().dictproj_forward_noalloc(C.byref(group), C.byref(layer), C.c_void_p(X_ptr), M,
+                                          C.c_void_p(Y_ptr), C.c_void_p(stream)))
+
+
+def dictproj_forward_noalloc_status(group: DeviceGroup, layer: DeviceLayer, X_ptr: int, M: int, Y_ptr: int,
+                                    stream: int = 0) -> int:
+    """Raw status of a no-allocation forward (no exception)."""
+    return lib().dictproj_forward_noalloc(C.byref(group), C.byref(layer), C.c_void_p(X_ptr), M,
+                                          C.c_void_p(Y_ptr), C.c_void_p(stream))
 
 
 def dictproj_check(stream: int = 0):

@@ -30,7 +30,7 @@ int fail(int status, const char* fmt, ...) {
 }
 void clear_error() { g_err[0] = 0; }
 
-static int cuda_fail(cudaError_t e, const char* what) {
+int cuda_fail(cudaError_t e, const char* what) {
   return fail(DICTPROJ_ERR_CUDA, "%s: %s (%s)", what, cudaGetErrorName(e), cudaGetErrorString(e));
 }
 
@@ -53,7 +53,7 @@ static cudaError_t h2d(void* d, const void* h, size_t n) {
 static std::mutex g_dev_mu;
 static std::vector<int> g_dev_ready;
 
-static int ensure_device(int* dev_out) {
+int ensure_device(int* dev_out) {
   int dev = -1;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");

@@ -423,11 +423,13 @@ k_coeff_decode_direct(const uint32_t* __restrict__ col_ptr, const uint8_t* __res
                       const uint8_t* __restrict__ scales, const uint8_t* __restrict__ idx,
                       const uint16_t* __restrict__ seg_start, int nseg, float s_C, int k, int d_out,
                       const float* __restrict__ Z, int M, __half* __restrict__ Y) {
-  extern __shared__ __align__(16) float zsd[];  // [k][MP]
+  extern __shared__ __align__(16) float zsd[];  // [k + 256][MP]; the tail is zero
   trigger_dependents();
   grid_dependency_wait();
   for (int i = threadIdx.x * 4; i < k * MP; i += blockDim.x * 4)
     *reinterpret_cast<float4*>(zsd + i) = *reinterpret_cast<const float4*>(Z + i);
+  // zero tail: an index byte in the last 256-atom segment never reads past the table
+  for (int i = k * MP + threadIdx.x; i < (k + 256) * MP; i += blockDim.x) zsd[i] = 0.f;
   __syncthreads();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int o = blockIdx.x * 8 + warp;
@@ -559,7 +561,7 @@ cudaError_t launch_coeff_decode(const dictproj_layer* l, const float* Z, int M, 
   void* args[] = {(void*)&col_ptr, (void*)&codes, (void*)&scales, (void*)&idx, (void*)&ss,
                   (void*)&nseg, (void*)&s, (void*)&k, (void*)&d_out, (void*)&Z, (void*)&M, (void*)&Y};
   const dim3 grid((d_out + 7) / 8), block(256);
-  const size_t smem = (size_t)k * mp * sizeof(float);
+  const size_t smem = (size_t)(k + 256) * mp * sizeof(float);
   switch (mp) {
     case 1: return launch_pdl((const void*)k_coeff_decode_direct<1>, grid, block, smem, stream, args);
     case 2: return launch_pdl((const void*)k_coeff_decode_direct<2>, grid, block, smem, stream, args);

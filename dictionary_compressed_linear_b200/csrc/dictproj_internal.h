@@ -4,6 +4,8 @@
 #include <cstddef>
 #include <cstdint>
 
+#include <cuda_runtime.h>
+
 #include "dictproj.h"
 
 namespace dictproj {
@@ -15,6 +17,11 @@ int fail(int status, const char* fmt, ...)
 #endif
     ;
 void clear_error();
+// Record a CUDA failure (DICTPROJ_ERR_CUDA) with the call that failed.
+int cuda_fail(cudaError_t e, const char* what);
+// Check the current device (sm_100) and set kernel attributes once per device;
+// allocates nothing.
+int ensure_device(int* dev_out);
 
 int pack_group_host(const float* D, int d_in, int k, uint8_t* codes, uint8_t* scales, float* s_D);
 int layer_packed_entries(const int32_t* col_ptr, int k, int d_out, size_t* total);

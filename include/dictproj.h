@@ -182,6 +182,47 @@ int dictproj_forward_path(const void* X, int M, const dictproj_layer* layer,
 int dictproj_dictionary_stage(const void* X, int M, const dictproj_group* group, float* Z, void* stream);
 int dictproj_coefficient_stage(const float* Z, int M, const dictproj_layer* layer, void* Y, void* stream);
 
+/* ------------------------------------------------------------------------- */
+/* Forward without allocation                                                 */
+/* ------------------------------------------------------------------------- */
+
+/* Caller-owned device copies of packed factors (the arrays produced by
+ * dictproj_pack_group_host / dictproj_pack_layer_host, copied to the device by
+ * the caller). All pointers are device pointers; the library only reads them. */
+typedef struct dictproj_device_group {
+  const uint8_t* codes;   /* [k][d_in/2] */
+  const uint8_t* scales;  /* [k][d_in/16] */
+  float s;                /* s_D */
+  int d_in, k;
+} dictproj_device_group;
+
+typedef struct dictproj_device_layer {
+  const uint32_t* col_ptr;    /* [d_out+1] */
+  const uint8_t* codes;       /* [total/2] */
+  const uint8_t* scales;      /* [total/16] */
+  const uint8_t* idx;         /* [total] */
+  const uint16_t* seg_start;  /* [d_out][ceil(k/256)] */
+  float s;                    /* s_C */
+  int k, d_out;
+} dictproj_device_layer;
+
+/* The decode-path forward (1 <= M <= 8) for callers that cannot allocate device
+ * memory at call time: runtimes that reserve all device memory up front in their
+ * own arena, and code enqueuing work while a stream is captured into a CUDA graph.
+ * It computes the same Y = X D_g C_l as dictproj_forward; the paper has no
+ * counterpart for this entry point (it is an integration convenience).
+ * Nothing is allocated: the Z scratch between the two stages is a file-scope
+ * device array of 49152 floats (192 KiB) that every GPU loading the library holds
+ * until exit; (k + 256) * mp must not exceed 49152, where mp = 1, 2, 4 or 8 is the
+ * smallest power of two >= M, else DICTPROJ_ERR_RANGE and nothing is launched.
+ * The first call with a given device current resolves the array's device address
+ * (cudaGetSymbolAddress); make that first call before any stream capture. All
+ * calls share the array: calls that overlap on the GPU race and must be
+ * serialised by the caller. X fp16 [M][d_in], Y fp16 [M][d_out], both device,
+ * 16-byte aligned. Errors: NULL, SHAPE, MISMATCH, RANGE, ALIGN, VALUE, CUDA. */
+int dictproj_forward_noalloc(const dictproj_device_group* group, const dictproj_device_layer* layer,
+                             const void* X, int M, void* Y, void* stream);
+
 /* Read (and clear) the device error word that bounded device waits set, after
  * synchronising `stream`. Returns OK or TIMEOUT (or CUDA). */
 int dictproj_check(void* stream);
