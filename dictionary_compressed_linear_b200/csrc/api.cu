@@ -179,15 +179,21 @@ int dictproj_group_upload(const uint8_t* codes, const uint8_t* scales, float s_D
   g->codes_bytes = (size_t)d_in * k / 2;
   g->scales_bytes = (size_t)d_in * k / 16;
   cudaError_t e;
+  if ((e = cudaDeviceGetAttribute(&g->n_sm, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) {
+    delete g;
+    return cuda_fail(e, "group_upload: SM count");
+  }
+  g->zslices = dict_max_slices(d_in, k, g->n_sm);
+  const size_t zbytes = (size_t)g->zslices * k * kDecodeMaxTokens * sizeof(float);
   if ((e = dmalloc((void**)&g->codes, g->codes_bytes)) || (e = dmalloc((void**)&g->scales, g->scales_bytes)) ||
-      (e = dmalloc((void**)&g->z32, (size_t)k * kDecodeMaxTokens * sizeof(float))) ||
+      (e = dmalloc((void**)&g->z32, zbytes)) ||
       (e = dmalloc((void**)&g->err, 16))) {
     dictproj_free_group(g);
     cudaGetLastError();
     return fail(DICTPROJ_ERR_OOM, "group_upload: device allocation failed (%s)", cudaGetErrorName(e));
   }
   if ((e = h2d(g->codes, codes, g->codes_bytes)) || (e = h2d(g->scales, scales, g->scales_bytes)) ||
-      (e = cudaMemset(g->err, 0, 16)) || (e = cudaMemset(g->z32, 0, (size_t)k * kDecodeMaxTokens * sizeof(float)))) {
+      (e = cudaMemset(g->err, 0, 16)) || (e = cudaMemset(g->z32, 0, zbytes))) {
     dictproj_free_group(g);
     cudaGetLastError();
     return cuda_fail(e, "group_upload: copy to device");
@@ -279,6 +285,8 @@ int dictproj_layer_upload(const uint32_t* pcol_ptr, const uint8_t* codes, const 
     return cuda_fail(e, "layer_upload: device attributes");
   }
   l->smem_per_sm = smem_sm;
+  l->n_sm = n_sm;
+  l->gather_ok = gather_supported(pcol_ptr, d_out, nseg);
   for (int pi = 0; pi < 2; ++pi) {
     std::vector<uint32_t> plan;
     std::vector<int> cta_ptr;
@@ -431,10 +439,13 @@ int dictproj_forward_path(const void* X, int M, const dictproj_layer* layer, con
   const __half* x = static_cast<const __half*>(X);
   __half* y = static_cast<__half*>(Y);
   const bool decode = path == DICTPROJ_PATH_DECODE || (path == DICTPROJ_PATH_AUTO && M <= kDecodeMaxTokens);
+  const DictPlan plan = dict_plan(group->d_in, group->k, group->n_sm, M < kDecodeMaxTokens ? M : kDecodeMaxTokens, false);
   if (decode) {
     const int mp = decode_mp(M);
-    if ((e = launch_dict_decode(group, x, M, mp, group->z32, s)) != cudaSuccess) return cuda_fail(e, "forward: dictionary stage launch");
-    if ((e = launch_coeff_decode(layer, group->z32, M, mp, y, s)) != cudaSuccess) return cuda_fail(e, "forward: coefficient stage launch");
+    if ((e = launch_dict_decode(group, x, M, mp, group->z32, plan, s)) != cudaSuccess)
+      return cuda_fail(e, "forward: dictionary stage launch");
+    if ((e = launch_coeff_decode(layer, group->z32, plan.slices, M, mp, y, s)) != cudaSuccess)
+      return cuda_fail(e, "forward: coefficient stage launch");
     return DICTPROJ_OK;
   }
   // Token chunks of 8 through the decode kernels (prefill path until the
@@ -442,9 +453,10 @@ int dictproj_forward_path(const void* X, int M, const dictproj_layer* layer, con
   for (int m0 = 0; m0 < M; m0 += kDecodeMaxTokens) {
     const int mc = M - m0 < kDecodeMaxTokens ? M - m0 : kDecodeMaxTokens;
     const int mp = decode_mp(mc);
-    if ((e = launch_dict_decode(group, x + (size_t)m0 * group->d_in, mc, mp, group->z32, s)) != cudaSuccess)
+    if ((e = launch_dict_decode(group, x + (size_t)m0 * group->d_in, mc, mp, group->z32, plan, s)) != cudaSuccess)
       return cuda_fail(e, "forward: dictionary stage launch");
-    if ((e = launch_coeff_decode(layer, group->z32, mc, mp, y + (size_t)m0 * layer->d_out, s)) != cudaSuccess)
+    if ((e = launch_coeff_decode(layer, group->z32, plan.slices, mc, mp, y + (size_t)m0 * layer->d_out, s)) !=
+        cudaSuccess)
       return cuda_fail(e, "forward: coefficient stage launch");
   }
   return DICTPROJ_OK;
@@ -461,7 +473,8 @@ int dictproj_dictionary_stage(const void* X, int M, const dictproj_group* group,
   if (M < 1 || M > group->max_tokens) return fail(DICTPROJ_ERR_RANGE, "dictionary_stage: M=%d outside [1, %d]", M, group->max_tokens);
   if (M > kDecodeMaxTokens) return fail(DICTPROJ_ERR_UNSUPPORTED, "dictionary_stage: M must be <= %d", kDecodeMaxTokens);
   if (((uintptr_t)X & 15) || ((uintptr_t)Z & 15)) return fail(DICTPROJ_ERR_ALIGN, "dictionary_stage: X and Z must be 16-byte aligned");
-  cudaError_t e = launch_dict_decode(group, static_cast<const __half*>(X), M, decode_mp(M), Z, (cudaStream_t)stream);
+  const DictPlan plan = dict_plan(group->d_in, group->k, group->n_sm, M, true);  // Z written complete
+  cudaError_t e = launch_dict_decode(group, static_cast<const __half*>(X), M, decode_mp(M), Z, plan, (cudaStream_t)stream);
   return e == cudaSuccess ? DICTPROJ_OK : cuda_fail(e, "dictionary_stage: launch");
 }
 
@@ -471,7 +484,7 @@ int dictproj_coefficient_stage(const float* Z, int M, const dictproj_layer* laye
   if (M < 1) return fail(DICTPROJ_ERR_RANGE, "coefficient_stage: M=%d < 1", M);
   if (M > kDecodeMaxTokens) return fail(DICTPROJ_ERR_UNSUPPORTED, "coefficient_stage: M must be <= %d", kDecodeMaxTokens);
   if (((uintptr_t)Y & 15) || ((uintptr_t)Z & 15)) return fail(DICTPROJ_ERR_ALIGN, "coefficient_stage: Z and Y must be 16-byte aligned");
-  cudaError_t e = launch_coeff_decode(layer, Z, M, decode_mp(M), static_cast<__half*>(Y), (cudaStream_t)stream);
+  cudaError_t e = launch_coeff_decode(layer, Z, 1, M, decode_mp(M), static_cast<__half*>(Y), (cudaStream_t)stream);
   return e == cudaSuccess ? DICTPROJ_OK : cuda_fail(e, "coefficient_stage: launch");
 }
 

@@ -5,26 +5,29 @@
 // so weight traffic overlaps the tail of the preceding work on the stream.
 //
 // Stage 1, dictionary (HBM-bound GEMV over packed NVFP4 D_g), k_dict_decode.
-//   One CTA per tile of 8 atoms, 8 warps splitting d_in into 32-element units.
-//   Each thread streams 16-byte code words of one atom through a 4-deep register
-//   ring (plus a bulk L2 prefetch of the whole tile), converts E2M1 pairs to
-//   f16x2 with the hardware cvt, multiplies by the block's E4M3 scale in fp16
-//   (an E2M1 x E4M3 product is exact in fp16) and feeds mma.sync m16n8k16 with
-//   D as the B operand (N = 8 atoms) and the tokens as A rows, fp32 accumulate.
-//   X is staged once in shared memory. Warp partials are summed in a fixed order;
-//   Z = s_D * sum as fp32 [k][mp].
+//   The grid is (k/16 atom tiles) x (d_in slices); each warp owns whole units of
+//   16 atoms x 128 d_in elements. A thread streams the 16-byte code words of two
+//   atoms through a register ring (raw weights are loaded before the dependency
+//   wait; a bulk L2 prefetch covers the rest of the CTA's slice), converts E2M1
+//   pairs to f16x2 with the hardware cvt, multiplies by the E4M3 block scale in
+//   fp16 (an E2M1 x E4M3 product is exact in fp16), and issues mma.sync m16n8k16
+//   with the atoms as the 16 rows of A and the tokens as the 8 columns of B, fp32
+//   accumulate. Warp partials are reduced in shared memory in a fixed order and
+//   each slice writes s_D * partial to Zpart[slice][k][mp].
 //
 // Stage 2, coefficients (sparse gather over column-compressed NVFP4 C_l),
 // k_coeff_decode.
-//   One persistent CTA per SM owns a run of columns balanced by stored entries.
-//   The run is cut (on the host, at upload) into chunks of at most 16384 entries
-//   of equal per-column padded length. Chunks stream through a two-stage shared
-//   memory ring with bulk async copies completing on mbarriers (the first two
-//   are issued before the dependency wait). Z is staged in shared memory. Every
-//   thread takes a contiguous run of 16-entry blocks (one E4M3 scale each):
-//   atom = 256*segment + idx, segment from the column's seg_start row; the block
-//   sum is scaled and stored per block; one warp per column then sums the block
-//   partials in a fixed order, so results are bit-reproducible.
+//   Persistent CTAs own runs of columns balanced by stored entries; the runs are
+//   cut on the host (at upload) into chunks of at most 16 columns of equal padded
+//   length and 16384 entries, which stream through a two-stage shared-memory ring
+//   with bulk async copies completing on mbarriers (the first two issued before
+//   the dependency wait). Z = sum of the slices (fixed order) is staged in shared
+//   memory. One warp per column: lane l sums a contiguous run of 8-entry
+//   half-blocks (atom = 256*segment + idx; at most one segment boundary per
+//   half-block takes a select, more falls back to a walk), scales each by its
+//   E4M3 block scale, and the warp reduces with shuffles in a fixed order, so
+//   results are bit-reproducible. Y = s_C * sum in fp16.
+
 #include <algorithm>
 #include <climits>
 #include <vector>
@@ -41,140 +44,155 @@ namespace dictproj {
 // =================================================================================
 // Stage 1: dictionary
 // =================================================================================
-constexpr int kDictWarps = 8;
-constexpr int kDictDepth = 4;     // register prefetch depth (iterations)
-constexpr int kDictAtoms = 8;     // atoms per CTA = MMA N
-constexpr size_t kDictXSmemMax = 96 * 1024;
+constexpr int kDictWarps = 8;     // warps per CTA; each owns whole 128-element units
+constexpr int kDictTile = 16;     // atoms per CTA = MMA M
 
+// A unit is 16 atoms x 128 d_in elements: thread (g, t) of a warp holds atoms g
+// and g+8 of the tile and elements [128u + 32t, 128u + 32t + 32).
 struct DictUnit {
-  uint4 w;       // 16 code bytes: 32 elements of this thread's atom
-  uint32_t sc;   // the two E4M3 block scales of those 32 elements
+  uint4 wa, wb;      // 16 code bytes of atoms g and g+8 (32 elements each)
+  uint32_t sa, sb;   // their two E4M3 block scales (2 bytes each)
 };
 
-__device__ __forceinline__ void load_unit(DictUnit& u, const uint8_t* c, const uint8_t* s, int unit, bool ok) {
+__device__ __forceinline__ void load_unit(DictUnit& u, const uint8_t* c0, const uint8_t* c1, const uint8_t* s0,
+                                          const uint8_t* s1, size_t off_c, size_t off_s, bool ok) {
   if (ok) {
-    u.w = ld_stream_v4(c + (size_t)unit * 16);
-    u.sc = ld_stream_u16(s + (size_t)unit * 2);
+    u.wa = ld_stream_v4(c0 + off_c);
+    u.wb = ld_stream_v4(c1 + off_c);
+    u.sa = ld_stream_u16(s0 + off_s);
+    u.sb = ld_stream_u16(s1 + off_s);
   } else {
-    u.w = make_uint4(0, 0, 0, 0);
-    u.sc = 0;
+    u.wa = make_uint4(0, 0, 0, 0);
+    u.wb = u.wa;
+    u.sa = u.sb = 0;
   }
 }
 
-// One 32-element unit: 8 MMAs of k = 16 (4 elements per thread each).
-// B (K x N = d_in-slots x atoms): b0:b1 <- elements 8q+4h+{0,1}, b2:b3 <- 8q+4h+{2,3}.
-// A (M x K = tokens x slots): row g (token g) the matching X values, row g+8 zero.
-__device__ __forceinline__ void dict_unit_mma(float acc[2][4], const DictUnit& u, const uint32_t xw[16]) {
-  const uint32_t h2 = e4m3x2_to_f16x2(u.sc);
-  const uint32_t s_lo = dup_lo(h2), s_hi = dup_hi(h2);
-  const uint32_t w[4] = {u.w.x, u.w.y, u.w.z, u.w.w};
+// One unit: 8 MMAs m16n8k16 with the atoms as the 16 rows of A (swap-AB) and the
+// tokens as the 8 columns of B; 4 elements per thread per MMA.
+// A: a0:a1 <- atom g, elements 8q+4h+{0,1}; a2:a3 <- atom g+8, same; a4:a5 / a6:a7 <- +{2,3}.
+// B: b0:b1 <- X[token g][same elements +{0,1}], b2:b3 <- +{2,3}.
+template <bool XS>
+__device__ __forceinline__ void dict_unit_mma(float acc[2][4], const DictUnit& u, const __half* px, bool xon) {
+  const uint32_t ha = e4m3x2_to_f16x2(u.sa), hb = e4m3x2_to_f16x2(u.sb);
+  const uint32_t wa[4] = {u.wa.x, u.wa.y, u.wa.z, u.wa.w};
+  const uint32_t wb[4] = {u.wb.x, u.wb.y, u.wb.z, u.wb.w};
 #pragma unroll
   for (int q = 0; q < 4; ++q) {
-    uint32_t f[4];
-    e2m1x8_to_f16x2x4(w[q], f);
-    const uint32_t sc = q < 2 ? s_lo : s_hi;
+    uint32_t fa[4], fb[4];
+    e2m1x8_to_f16x2x4(wa[q], fa);
+    e2m1x8_to_f16x2x4(wb[q], fb);
+    const uint32_t sa = q < 2 ? dup_lo(ha) : dup_hi(ha);
+    const uint32_t sb = q < 2 ? dup_lo(hb) : dup_hi(hb);
 #pragma unroll
-    for (int i = 0; i < 4; ++i) f[i] = hmul2_u32(f[i], sc);
+    for (int i = 0; i < 4; ++i) {
+      fa[i] = hmul2_u32(fa[i], sa);  // E2M1 x E4M3 is exact in fp16
+      fb[i] = hmul2_u32(fb[i], sb);
+    }
+    uint4 xv = make_uint4(0, 0, 0, 0);  // X elements 8q .. 8q+7 of this thread's range
+    if (xon) xv = XS ? *reinterpret_cast<const uint4*>(px + 8 * q) : ld_nc_v4(px + 8 * q);
+    const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
-      const uint32_t a[4] = {xw[4 * q + 2 * h], 0u, xw[4 * q + 2 * h + 1], 0u};
-      const uint32_t b[2] = {f[2 * h], f[2 * h + 1]};
+      const uint32_t a[4] = {fa[2 * h], fb[2 * h], fa[2 * h + 1], fb[2 * h + 1]};
+      const uint32_t b[2] = {xw[2 * h], xw[2 * h + 1]};
       mma_16816(acc[h], a, b);  // two independent accumulation chains
     }
   }
 }
 
-template <bool XS>
-__global__ void __launch_bounds__(kDictWarps * 32)
-k_dict_decode(const uint8_t* __restrict__ codes, const uint8_t* __restrict__ scales, float s_D,
-              int d_in, const __half* __restrict__ X, int M, int mp, float* __restrict__ Z) {
-  extern __shared__ __align__(16) unsigned char dsmem[];  // X rows, stride d_in + 8 halves
-  __shared__ float red[kDictWarps][8][kDictAtoms];
-  constexpr int P = 4 * kDictWarps;
-  const int tile = blockIdx.x;
+// Zpart[slice][atom][mp] = s_D * sum over the slice's units of X[m][i] * D[i][atom].
+// Grid: (k / 16 tiles) x (slices); slice y covers units [y*8*J, (y+1)*8*J).
+// RING = register prefetch depth in units (1, 2 or 4; at most J is useful).
+// XS: X rows of the slice are staged in shared memory (stride xlen + 8 halves).
+template <int RING, bool XS>
+__global__ void __launch_bounds__(kDictWarps * 32, 4)  // at most 64 registers
+k_dict_decode(const uint8_t* __restrict__ codes, const uint8_t* __restrict__ scales, float s_D, int d_in, int k,
+              const __half* __restrict__ X, int M, int mp, float* __restrict__ Zpart, int J) {
+  extern __shared__ __align__(16) unsigned char dsmem[];
+  __shared__ float red[kDictWarps][kDictTile][8];
+  const int tile = blockIdx.x, slice = blockIdx.y;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int g = lane >> 2, tig = lane & 3;
-  const int p = warp * 4 + tig;
-  const int n_units = d_in >> 5;
+  const int g = lane >> 2, t = lane & 3;
   const size_t crow = (size_t)(d_in >> 1), srow = (size_t)(d_in >> 4);
-  const uint8_t* c = codes + (size_t)(tile * kDictAtoms + g) * crow;
-  const uint8_t* s = scales + (size_t)(tile * kDictAtoms + g) * srow;
+  const uint8_t* c0 = codes + (size_t)(tile * kDictTile + g) * crow;
+  const uint8_t* c1 = c0 + 8 * crow;
+  const uint8_t* s0 = scales + (size_t)(tile * kDictTile + g) * srow;
+  const uint8_t* s1 = s0 + 8 * srow;
+  const int u_begin = slice * kDictWarps * J;
+  const int e_begin = u_begin * 128;
+  const int e_end = min(d_in, (u_begin + kDictWarps * J) * 128);
+  // element range of this thread in unit u: [128u + 32t, +32); valid iff it ends <= d_in
+  auto unit_of = [&](int j) { return u_begin + warp + kDictWarps * j; };
+  auto valid = [&](int u) { return 128 * u + 32 * t + 32 <= d_in; };
 
-  if (threadIdx.x == 0) {
-    prefetch_l2_range(codes, (size_t)tile * kDictAtoms * crow, (size_t)(tile + 1) * kDictAtoms * crow);
-    prefetch_l2_range(scales, (size_t)tile * kDictAtoms * srow, (size_t)(tile + 1) * kDictAtoms * srow);
+  if (threadIdx.x < kDictTile) {  // L2 prefetch of this CTA's slice of the 16 atom rows
+    const size_t row = (size_t)(tile * kDictTile + threadIdx.x);
+    prefetch_l2_range(codes, row * crow + e_begin / 2, row * crow + e_end / 2);
+    prefetch_l2_range(scales, row * srow + e_begin / 16, row * srow + e_end / 16);
   }
-  const int iters = (n_units + P - 1) / P;
-  DictUnit ring[kDictDepth];
+  DictUnit ring[RING];
 #pragma unroll
-  for (int d = 0; d < kDictDepth; ++d) {
-    const int u = p + d * P;
-    load_unit(ring[d], c, s, u, d < iters && u < n_units);
+  for (int d = 0; d < RING; ++d) {
+    const int u = unit_of(d);
+    load_unit(ring[d], c0, c1, s0, s1, (size_t)u * 64 + 16 * t, (size_t)u * 8 + 2 * t, d < J && valid(u));
   }
   trigger_dependents();
-  grid_dependency_wait();  // X and Z belong to earlier work on the stream
+  grid_dependency_wait();  // X and the Z scratch belong to earlier work on the stream
 
-  const int xstride = XS ? d_in + 8 : d_in;
-  const __half* xs = X;
-  if constexpr (XS) {
+  const int xlen = e_end - e_begin;
+  const int xstride = XS ? xlen + 8 : d_in;
+  const __half* xr;
+  if constexpr (XS) {  // stage X[0:M][slice] once; one L2 round trip for the whole CTA
     __half* xsm = reinterpret_cast<__half*>(dsmem);
-    const int vec_per_row = d_in >> 3;  // 16-byte vectors per row
-    for (int i = threadIdx.x; i < M * vec_per_row; i += blockDim.x) {
-      const int r = i / vec_per_row, v = i - r * vec_per_row;
-      *reinterpret_cast<uint4*>(xsm + (size_t)r * xstride + v * 8) =
-          ld_nc_v4(X + (size_t)r * d_in + v * 8);
+    const int vpr = xlen >> 3;  // 16-byte vectors per row
+    for (int i = threadIdx.x; i < M * vpr; i += blockDim.x) {
+      const int r = i / vpr, v = i - r * vpr;
+      *reinterpret_cast<uint4*>(xsm + (size_t)r * xstride + 8 * v) =
+          ld_nc_v4(X + (size_t)r * d_in + e_begin + 8 * v);
     }
     __syncthreads();
-    xs = xsm;
+    xr = xsm + (size_t)g * xstride - e_begin;  // index with absolute element numbers
+  } else {
+    xr = X + (size_t)g * d_in;
   }
   const bool xrow = g < M;
-  const __half* xr = xs + (size_t)g * xstride;
   float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-  for (int it0 = 0; it0 < iters; it0 += kDictDepth) {
+  for (int j0 = 0; j0 < J; j0 += RING) {
 #pragma unroll
-    for (int d = 0; d < kDictDepth; ++d) {
-      const int it = it0 + d;
-      if (it < iters) {
-        const int u = p + it * P;
-        uint32_t xw[16];
-        if (xrow && u < n_units) {
-#pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            const uint4 v = XS ? *reinterpret_cast<const uint4*>(xr + (size_t)u * 32 + q * 8)
-                               : ld_nc_v4(xr + (size_t)u * 32 + q * 8);
-            xw[4 * q] = v.x;
-            xw[4 * q + 1] = v.y;
-            xw[4 * q + 2] = v.z;
-            xw[4 * q + 3] = v.w;
-          }
-        } else {
-#pragma unroll
-          for (int q = 0; q < 16; ++q) xw[q] = 0u;
-        }
-        dict_unit_mma(acc, ring[d], xw);
-        const int un = p + (it + kDictDepth) * P;
-        load_unit(ring[d], c, s, un, (it + kDictDepth) < iters && un < n_units);
+    for (int d = 0; d < RING; ++d) {
+      const int j = j0 + d;
+      if (j < J) {
+        const int u = unit_of(j);
+        dict_unit_mma<XS>(acc, ring[d], xr + (size_t)u * 128 + 32 * t, xrow && valid(u));
+        const int un = unit_of(j + RING);
+        load_unit(ring[d], c0, c1, s0, s1, (size_t)un * 64 + 16 * t, (size_t)un * 8 + 2 * t,
+                  j + RING < J && valid(un));
       }
     }
   }
-  // acc[0], acc[1] = token g, atoms 2*tig, 2*tig+1 (acc[2], acc[3] are the zero rows g+8)
-  red[warp][g][2 * tig] = acc[0][0] + acc[1][0];
-  red[warp][g][2 * tig + 1] = acc[0][1] + acc[1][1];
+  // c0:c1 = atom g, tokens 2t, 2t+1; c2:c3 = atom g+8, tokens 2t, 2t+1
+  red[warp][g][2 * t] = acc[0][0] + acc[1][0];
+  red[warp][g][2 * t + 1] = acc[0][1] + acc[1][1];
+  red[warp][g + 8][2 * t] = acc[0][2] + acc[1][2];
+  red[warp][g + 8][2 * t + 1] = acc[0][3] + acc[1][3];
   __syncthreads();
-  if (threadIdx.x < 8 * kDictAtoms) {
-    const int n = threadIdx.x / kDictAtoms, a = threadIdx.x % kDictAtoms;
+  if (threadIdx.x < kDictTile * 8) {
+    const int a = threadIdx.x >> 3, n = threadIdx.x & 7;
     float sum = 0.f;
 #pragma unroll
-    for (int w = 0; w < kDictWarps; ++w) sum += red[w][n][a];
-    if (n < mp) Z[(size_t)(tile * kDictAtoms + a) * mp + n] = sum * s_D;
+    for (int w = 0; w < kDictWarps; ++w) sum += red[w][a][n];
+    if (n < mp) Zpart[((size_t)slice * k + tile * kDictTile + a) * mp + n] = sum * s_D;
   }
 }
 
 // =================================================================================
 // Stage 2: coefficients
 // =================================================================================
-constexpr int kCoeffThreads = 512;
+constexpr int kCoeffWarps = 16;
+constexpr int kCoeffThreads = kCoeffWarps * 32;
 constexpr int kChunkEntries = 16384;
+constexpr int kChunkCols = kCoeffWarps;  // one column per warp per chunk
 constexpr int kSegBytes = 8192;
 // stage layout (bytes): idx | codes | scales | seg_start
 constexpr int kStIdx = 0;
@@ -183,18 +201,19 @@ constexpr int kStScales = kStCodes + kChunkEntries / 2 + 16;
 constexpr int kStSeg = kStScales + kChunkEntries / 16 + 32;
 constexpr int kStageBytes = kStSeg + kSegBytes + 32;
 
+// Z rows live in shared memory at byte address zaddr + atom * MP * 4.
 template <int MP>
-__device__ __forceinline__ void fma_z(float blk[MP], const float* z, float v) {
+__device__ __forceinline__ void fma_z(float blk[MP], uint32_t a, float v) {
   if constexpr (MP == 1) {
-    blk[0] = fmaf(z[0], v, blk[0]);
+    blk[0] = fmaf(lds_f32(a), v, blk[0]);
   } else if constexpr (MP == 2) {
-    const float2 t = *reinterpret_cast<const float2*>(z);
+    const float2 t = lds_f32x2(a);
     blk[0] = fmaf(t.x, v, blk[0]);
     blk[1] = fmaf(t.y, v, blk[1]);
   } else {
 #pragma unroll
     for (int m = 0; m < MP; m += 4) {
-      const float4 t = *reinterpret_cast<const float4*>(z + m);
+      const float4 t = lds_f32x4(a + 4 * m);
       blk[m] = fmaf(t.x, v, blk[m]);
       blk[m + 1] = fmaf(t.y, v, blk[m + 1]);
       blk[m + 2] = fmaf(t.z, v, blk[m + 2]);
@@ -203,48 +222,59 @@ __device__ __forceinline__ void fma_z(float blk[MP], const float* z, float v) {
   }
 }
 
+// seg_start row readers: shared-memory row (byte address) or global row.
+struct SegShared {
+  uint32_t a;
+  __device__ __forceinline__ int operator()(int j) const { return (int)lds_u16(a + 2u * (uint32_t)j); }
+};
+struct SegGlobal {
+  const uint16_t* p;
+  __device__ __forceinline__ int operator()(int j) const { return (int)p[j]; }
+};
+
 // Segment bookkeeping: s(q) = max{s : ss[s] <= q}; `nb` = ss[s+1] (INT_MAX past the last).
-__device__ __forceinline__ void advance_segment(int q, int& s, int& nb, const uint16_t* ss, int nseg) {
+template <class SS>
+__device__ __forceinline__ void advance_segment(int q, int& s, int& nb, const SS& ss, int nseg) {
   while (q >= nb) {
     ++s;
-    nb = (s + 1 < nseg) ? (int)ss[s + 1] : INT_MAX;
+    nb = (s + 1 < nseg) ? ss(s + 1) : INT_MAX;
   }
 }
 
-// Sum of one 16-entry block (entries q0 .. q0+15 of a column, segment state
-// valid for q0): returns blk[m] = sum_e Z[m][atom_e] * E2M1(code_e), unscaled.
-// With at most one segment boundary inside the block, entry i uses segment s
-// for i < t and s+1 from t on (a select); otherwise entries advance one by one.
-template <int MP>
-__device__ __forceinline__ void block_sum(float blk[MP], const float* zs, uint4 iv, uint2 cv, int q0, int s,
-                                          int nb, const uint16_t* ss, int nseg) {
-  const uint32_t iw[4] = {iv.x, iv.y, iv.z, iv.w};
-  const uint32_t cw[2] = {cv.x, cv.y};
-  float a0[MP], a1[MP];  // two independent accumulation chains (even / odd entries)
+// Sum of NE consecutive entries (q0 .. q0+NE-1 of a column; segment state valid
+// for q0) given their index bytes `iw` and codes `cw`; unscaled. Z is read from
+// shared memory at zaddr (32-bit addresses throughout).
+// With at most one segment boundary inside, entry i uses segment s for i < t and
+// s+1 from t on (a select); otherwise the entries advance one by one.
+template <int MP, int NE, class SS>
+__device__ __forceinline__ void entries_sum(float blk[MP], uint32_t zaddr, const uint32_t* iw, const uint32_t* cw,
+                                            int q0, int s, int nb, int nb2, const SS& ss, int nseg) {
+  // nb, nb2: the first two segment starts after q0 (INT_MAX if none)
+  constexpr uint32_t kRow = MP * 4;  // bytes per atom row of Z
+  float a0[MP], a1[MP];              // two independent accumulation chains (even / odd entries)
 #pragma unroll
   for (int m = 0; m < MP; ++m) a0[m] = a1[m] = 0.f;
-  const int nb2 = (s + 2 < nseg) ? (int)ss[s + 2] : INT_MAX;
-  if (q0 + 15 < nb2) {
-    const int t = min(nb - q0, 16);
-    const float* z0 = zs + (size_t)(s << 8) * MP;
-    const float* z1 = z0 + 256 * MP;
+  if (q0 + NE - 1 < nb2) {
+    const int t = min(nb - q0, NE);
+    const uint32_t z0 = zaddr + ((uint32_t)s << 8) * kRow;
+    const uint32_t z1 = z0 + 256u * kRow;
 #pragma unroll
-    for (int j = 0; j < 2; ++j) {
+    for (int j = 0; j < NE / 8; ++j) {
       uint32_t f[4];
       e2m1x8_to_f16x2x4(cw[j], f);
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
         const float2 v = __half22float2(*reinterpret_cast<const __half2*>(&f[i]));
         const int e0 = 8 * j + 2 * i, e1 = e0 + 1;
-        const uint32_t b0 = (iw[e0 >> 2] >> ((e0 & 3) * 8)) & 0xFFu;
-        const uint32_t b1 = (iw[e1 >> 2] >> ((e1 & 3) * 8)) & 0xFFu;
-        fma_z<MP>(a0, (e0 >= t ? z1 : z0) + b0 * MP, v.x);
-        fma_z<MP>(a1, (e1 >= t ? z1 : z0) + b1 * MP, v.y);
+        const uint32_t b0 = __byte_perm(iw[e0 >> 2], 0u, 0x4440u | (uint32_t)(e0 & 3));
+        const uint32_t b1 = __byte_perm(iw[e1 >> 2], 0u, 0x4440u | (uint32_t)(e1 & 3));
+        fma_z<MP>(a0, (e0 >= t ? z1 : z0) + b0 * kRow, v.x);
+        fma_z<MP>(a1, (e1 >= t ? z1 : z0) + b1 * kRow, v.y);
       }
     }
   } else {
 #pragma unroll
-    for (int j = 0; j < 2; ++j) {
+    for (int j = 0; j < NE / 8; ++j) {
       uint32_t f[4];
       e2m1x8_to_f16x2x4(cw[j], f);
 #pragma unroll
@@ -254,8 +284,8 @@ __device__ __forceinline__ void block_sum(float blk[MP], const float* zs, uint4 
         for (int h = 0; h < 2; ++h) {
           const int ent = 8 * j + 2 * i + h;
           advance_segment(q0 + ent, s, nb, ss, nseg);
-          const uint32_t a = ((uint32_t)s << 8) + ((iw[ent >> 2] >> ((ent & 3) * 8)) & 0xFFu);
-          fma_z<MP>(h ? a1 : a0, zs + (size_t)a * MP, h ? v.y : v.x);
+          const uint32_t b = __byte_perm(iw[ent >> 2], 0u, 0x4440u | (uint32_t)(ent & 3));
+          fma_z<MP>(h ? a1 : a0, zaddr + (((uint32_t)s << 8) + b) * kRow, h ? v.y : v.x);
         }
       }
     }
@@ -295,110 +325,105 @@ __device__ __forceinline__ void issue_chunk(unsigned char* st, uint64_t* bar, co
     bulk_g2s(st + kStSeg, reinterpret_cast<const uint8_t*>(seg_start) + r.seg_a0, r.seg_n, bar);
 }
 
+// Stage Z (sum of the dictionary stage's slices, fixed order) into shared memory.
 template <int MP>
-__global__ void __launch_bounds__(kCoeffThreads, 2)
+__device__ __forceinline__ void stage_z(float* zs, const float* __restrict__ Zpart, int nslices, int k, int nthr) {
+  const int n = k * MP;
+  for (int i = threadIdx.x * 4; i < n; i += nthr * 4) {
+    float4 a = *reinterpret_cast<const float4*>(Zpart + i);
+    for (int sl = 1; sl < nslices; ++sl) {
+      const float4 b = *reinterpret_cast<const float4*>(Zpart + (size_t)sl * n + i);
+      a.x += b.x;
+      a.y += b.y;
+      a.z += b.z;
+      a.w += b.w;
+    }
+    *reinterpret_cast<float4*>(zs + i) = a;
+  }
+}
+
+template <int MP>
+__global__ void __launch_bounds__(kCoeffThreads, 2)  // caps registers at 64; launched one CTA per SM
 k_coeff_decode(const uint4* __restrict__ chunks, const int* __restrict__ cta_ptr,
                const uint8_t* __restrict__ codes, const uint8_t* __restrict__ scales,
                const uint8_t* __restrict__ idx, const uint16_t* __restrict__ seg_start, int nseg,
-               float s_C, int k, int d_out, const float* __restrict__ Z, int M, __half* __restrict__ Y) {
+               float s_C, int k, int d_out, const float* __restrict__ Zpart, int nslices, int M,
+               __half* __restrict__ Y, int nst) {
   extern __shared__ __align__(128) unsigned char csmem[];
-  float* zs = reinterpret_cast<float*>(csmem);                      // [k][MP]
-  float* part = zs + (size_t)k * MP;                                 // [kChunkEntries/16][MP]
-  unsigned char* stage0 = reinterpret_cast<unsigned char*>(part + (kChunkEntries / 16) * MP);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(stage0 + 2 * kStageBytes);
+  float* zs = reinterpret_cast<float*>(csmem);  // [k][MP]
+  unsigned char* stage0 = reinterpret_cast<unsigned char*>(zs + (size_t)k * MP);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(stage0 + (size_t)nst * kStageBytes);
 
   const int c0 = cta_ptr[blockIdx.x], c1 = cta_ptr[blockIdx.x + 1];
   const int nch = c1 - c0;
   if (threadIdx.x == 0) {
-    mbar_init(&bars[0], 1);
-    mbar_init(&bars[1], 1);
+    for (int i = 0; i < nst; ++i) mbar_init(&bars[i], 1);
     fence_mbar_init();
   }
   __syncthreads();
-  if (threadIdx.x == 0) {
-    for (int i = 0; i < 2 && i < nch; ++i)
-      issue_chunk(stage0 + i * kStageBytes, &bars[i], chunks[c0 + i], nseg, idx, codes, scales, seg_start);
+  if (threadIdx.x == 0) {  // weights: issue the first nst chunks before the dependency wait
+    for (int i = 0; i < nst && i < nch; ++i)
+      issue_chunk(stage0 + (size_t)i * kStageBytes, &bars[i], chunks[c0 + i], nseg, idx, codes, scales,
+                  seg_start);
   }
   trigger_dependents();
   grid_dependency_wait();  // Z comes from the dictionary stage
 
-  for (int i = threadIdx.x * 4; i < k * MP; i += kCoeffThreads * 4)
-    *reinterpret_cast<float4*>(zs + i) = *reinterpret_cast<const float4*>(Z + i);
+  stage_z<MP>(zs, Zpart, nslices, k, kCoeffThreads);
   __syncthreads();
 
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t zs_a = smem_u32(zs);
   for (int ci = 0; ci < nch; ++ci) {
-    const int sti = ci & 1;
-    unsigned char* st = stage0 + sti * kStageBytes;
+    const int sti = ci % nst;
+    unsigned char* st = stage0 + (size_t)sti * kStageBytes;
     const uint4 ch = chunks[c0 + ci];
-    if (!mbar_wait_bounded(&bars[sti], (ci >> 1) & 1)) break;  // error recorded; leave
+    if (!mbar_wait_bounded(&bars[sti], (ci / nst) & 1)) break;  // error recorded; leave
     const StageRanges r = stage_ranges(ch, nseg);
     const int ncols = (int)(ch.y - ch.x);
     const int P = ncols ? (int)((ch.w - ch.z) / (uint32_t)ncols) : 0;
-    const int nbc = P >> 4;
-    const int nblk = ncols * nbc;
-    const uint8_t* idx_s = st + kStIdx;
-    const uint8_t* codes_s = st + kStCodes + ((ch.z >> 1) - r.codes_a0);
-    const uint8_t* scales_s = st + kStScales + ((ch.z >> 4) - r.scales_a0);
-    const uint16_t* seg_s = reinterpret_cast<const uint16_t*>(st + kStSeg + (2u * ch.x * nseg - r.seg_a0));
+    const uint32_t st_a = smem_u32(st);
+    const uint32_t idx_a = st_a + kStIdx;
+    const uint32_t codes_a = st_a + kStCodes + ((ch.z >> 1) - r.codes_a0);
+    const uint32_t scales_a = st_a + kStScales + ((ch.z >> 4) - r.scales_a0);
+    const uint32_t seg_a = st_a + kStSeg + (2u * ch.x * (uint32_t)nseg - r.seg_a0);
 
-    // phase A: every thread sums a contiguous run of blocks (one division per
-    // chunk; column and segment state advance incrementally)
-    if (nblk) {
-      const int R = (nblk + kCoeffThreads - 1) / kCoeffThreads;
-      const int b0 = threadIdx.x * R, b1 = min(nblk, b0 + R);
-      if (b0 < b1) {
-        int col = b0 / nbc;
-        int jb = b0 - col * nbc;
-        const uint16_t* ss = seg_s + (size_t)col * nseg;
-        int sgi = 0;
-        for (int j = 1; j < nseg; ++j) sgi += ((int)ss[j] <= (jb << 4));
-        int nb = (sgi + 1 < nseg) ? (int)ss[sgi + 1] : INT_MAX;
-        uint4 iv = *reinterpret_cast<const uint4*>(idx_s + 16 * b0);
-        uint2 cv = *reinterpret_cast<const uint2*>(codes_s + 8 * b0);
-        uint32_t scb = scales_s[b0];
-        for (int b = b0; b < b1; ++b) {
-          // prefetch the next block of the run
-          uint4 iv_n = iv;
-          uint2 cv_n = cv;
-          uint32_t sc_n = scb;
-          if (b + 1 < b1) {
-            iv_n = *reinterpret_cast<const uint4*>(idx_s + 16 * (b + 1));
-            cv_n = *reinterpret_cast<const uint2*>(codes_s + 8 * (b + 1));
-            sc_n = scales_s[b + 1];
-          }
-          const int q0 = jb << 4;
-          float blk[MP];
-          block_sum<MP>(blk, zs, iv, cv, q0, sgi, nb, ss, nseg);
-          const float sc = e4m3_to_f32(scb);
-#pragma unroll
-          for (int m = 0; m < MP; ++m) part[b * MP + m] = blk[m] * sc;
-          if (++jb == nbc) {  // next column
-            jb = 0;
-            ss += nseg;
-            sgi = 0;
-            nb = nseg > 1 ? (int)ss[1] : INT_MAX;
-            advance_segment(0, sgi, nb, ss, nseg);
-          } else {
-            advance_segment(jb << 4, sgi, nb, ss, nseg);
-          }
-          iv = iv_n;
-          cv = cv_n;
-          scb = sc_n;
-        }
-      }
-    }
-    __syncthreads();
-    if (threadIdx.x == 0 && ci + 2 < nch)
-      issue_chunk(st, &bars[sti], chunks[c0 + ci + 2], nseg, idx, codes, scales, seg_start);
-    // phase B: one warp per column sums its block partials in a fixed order
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    for (int col = warp; col < ncols; col += kCoeffThreads / 32) {
+    // One warp per column. At step i the warp covers entries [256i, 256i+256):
+    // lane l takes the half-block of 8 entries at 256i + 8l (consecutive lanes read
+    // consecutive index / code bytes). Segment boundaries of the window are
+    // scanned once per step by the whole warp (uniform loads).
+    const int nhb = P >> 3;
+    for (int col = warp; col < ncols; col += kCoeffWarps) {
+      const SegShared ss{seg_a + 2u * (uint32_t)(col * nseg)};
+      const uint32_t cb = (uint32_t)(col * P);
       float acc[MP];
 #pragma unroll
       for (int m = 0; m < MP; ++m) acc[m] = 0.f;
-      for (int j = lane; j < nbc; j += 32) {
+      int s_lo = 0;  // segment of the window start
+      for (int h0 = 0; h0 < nhb; h0 += 32) {
+        const int w = h0 << 3;
+        while (s_lo + 1 < nseg && ss(s_lo + 1) <= w) ++s_lo;
+        const int h = h0 + lane;
+        const int q0 = h << 3;
+        int sgi = s_lo, t1 = INT_MAX, t2 = INT_MAX;
+        for (int j = s_lo + 1; j < nseg; ++j) {  // uniform over the warp
+          const int b = ss(j);
+          if (b > w + 256 + 8) break;
+          if (b <= q0) sgi = j;
+          else if (t1 == INT_MAX) t1 = b;
+          else if (t2 == INT_MAX) t2 = b;
+        }
+        if (h < nhb) {
+          const uint32_t e = cb + (uint32_t)q0;  // chunk-relative entry offset
+          const uint2 iv = lds_u32x2(idx_a + e);
+          const uint32_t cv = lds_u32(codes_a + (e >> 1));
+          const float sc = e4m3_to_f32(lds_u8(scales_a + (e >> 4)));
+          const uint32_t iw[2] = {iv.x, iv.y};
+          float blk[MP];
+          entries_sum<MP, 8>(blk, zs_a, iw, &cv, q0, sgi, t1, t2, ss, nseg);
 #pragma unroll
-        for (int m = 0; m < MP; ++m) acc[m] += part[(col * nbc + j) * MP + m];
+          for (int m = 0; m < MP; ++m) acc[m] = fmaf(blk[m], sc, acc[m]);
+        }
       }
 #pragma unroll
       for (int m = 0; m < MP; ++m) {
@@ -411,7 +436,166 @@ k_coeff_decode(const uint4* __restrict__ chunks, const int* __restrict__ cta_ptr
           if (m < M) Y[(size_t)m * d_out + ch.x + col] = __float2half_rn(acc[m] * s_C);
       }
     }
-    __syncthreads();
+    __syncthreads();  // the stage is free again
+    if (threadIdx.x == 0 && ci + nst < nch)
+      issue_chunk(st, &bars[sti], chunks[c0 + ci + nst], nseg, idx, codes, scales, seg_start);
+  }
+}
+
+// Direct coefficient kernel for columns of at most kRmax*256 entries and k of
+// at most 32*256 atoms (nseg <= 32): one warp per column, lanes interleaved over
+// 8-entry half-blocks (coalesced, conflict-free loads straight from global/L2),
+// the column's loads double-buffered in registers across the warp's columns, and
+// the column's seg_start row held one value per lane (read with shuffles).
+constexpr int kRmax = 5;         // steps of 32 half-blocks held per column
+constexpr int kGatherWarps = 32;
+
+struct ColData {
+  uint2 iv[kRmax];      // 8 index bytes per step
+  uint32_t cv[kRmax];   // 8 codes (4 bytes) per step
+  uint32_t sc;          // E4M3 scale byte of each step, packed 8 bits apiece
+  int ssv;              // seg_start[lane] of the column (lane < nseg)
+};
+
+__device__ __forceinline__ void load_col(ColData& d, int o, int d_out, const uint32_t* __restrict__ col_ptr,
+                                         const uint8_t* __restrict__ idx, const uint8_t* __restrict__ codes,
+                                         const uint8_t* __restrict__ scales, const uint16_t* __restrict__ seg_start,
+                                         int nseg, int lane, uint32_t& cb, int& nhb) {
+  cb = 0;
+  nhb = 0;
+  d.sc = 0;
+  d.ssv = 0;
+#pragma unroll
+  for (int i = 0; i < kRmax; ++i) {
+    d.iv[i] = make_uint2(0, 0);
+    d.cv[i] = 0;
+  }
+  if (o >= d_out) return;
+  cb = col_ptr[o];
+  nhb = (int)((col_ptr[o + 1] - cb) >> 3);
+  if (lane < nseg) d.ssv = (int)seg_start[(size_t)o * nseg + lane];
+#pragma unroll
+  for (int i = 0; i < kRmax; ++i) {
+    const int h = 32 * i + lane;
+    if (h < nhb) {
+      const uint32_t e = cb + 8u * (uint32_t)h;
+      d.iv[i] = ld_stream_v2(idx + e);
+      d.cv[i] = *reinterpret_cast<const uint32_t*>(codes + (e >> 1));
+      d.sc |= ld_stream_u8(scales + (e >> 4)) << (8 * i);
+    }
+  }
+}
+
+template <int MP>
+__global__ void __launch_bounds__(kGatherWarps * 32, 1)  // 1024 threads, at most 64 registers
+k_coeff_gather(const uint32_t* __restrict__ col_ptr, const uint8_t* __restrict__ codes,
+               const uint8_t* __restrict__ scales, const uint8_t* __restrict__ idx,
+               const uint16_t* __restrict__ seg_start, int nseg, float s_C, int k, int d_out,
+               const float* __restrict__ Zpart, int nslices, int M, __half* __restrict__ Y, int cols_per_cta) {
+  extern __shared__ __align__(16) float zsg[];  // [k + 256][MP]; the tail is zero
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int o_begin = blockIdx.x * cols_per_cta;
+  const int o_end = min(d_out, o_begin + cols_per_cta);
+  if (threadIdx.x == 0 && o_begin < o_end) {  // bulk L2 prefetch of this CTA's columns
+    const size_t e0 = col_ptr[o_begin], e1 = col_ptr[o_end];
+    prefetch_l2_range(idx, e0, e1);
+    prefetch_l2_range(codes, e0 >> 1, e1 >> 1);
+    prefetch_l2_range(scales, e0 >> 4, e1 >> 4);
+    prefetch_l2_range(seg_start, (size_t)o_begin * nseg * 2, (size_t)o_end * nseg * 2);
+  }
+  ColData cur, nxt;
+  uint32_t cb, cb_n;
+  int nhb, nhb_n;
+  int o = o_begin + warp;
+  load_col(cur, o, o_end, col_ptr, idx, codes, scales, seg_start, nseg, lane, cb, nhb);
+  trigger_dependents();
+  grid_dependency_wait();  // Z comes from the dictionary stage
+
+  stage_z<MP>(zsg, Zpart, nslices, k, blockDim.x);
+  for (int i = k * MP + threadIdx.x; i < (k + 256) * MP; i += blockDim.x) zsg[i] = 0.f;
+  __syncthreads();
+  const uint32_t zs_a = smem_u32(zsg);
+  constexpr uint32_t kRow = MP * 4;
+
+  for (; o < o_end; o += kGatherWarps) {
+    load_col(nxt, o + kGatherWarps, o_end, col_ptr, idx, codes, scales, seg_start, nseg, lane, cb_n, nhb_n);
+    float acc[MP];
+#pragma unroll
+    for (int m = 0; m < MP; ++m) acc[m] = 0.f;
+    int s_lo = 0;  // segment of the current window start (uniform)
+#pragma unroll
+    for (int i = 0; i < kRmax; ++i) {
+      const int w = 256 * i;
+      if (w >= 8 * nhb) break;
+      while (s_lo + 1 < nseg && __shfl_sync(0xffffffffu, cur.ssv, s_lo + 1) <= w) ++s_lo;
+      const int q0 = w + 8 * lane;
+      // segment of q0 and the next two boundaries, from the window's boundaries
+      int sgi = s_lo, t1 = INT_MAX, t2 = INT_MAX;
+      for (int j = s_lo + 1; j < nseg; ++j) {
+        const int b = __shfl_sync(0xffffffffu, cur.ssv, j);
+        if (b > w + 256 + 8) break;
+        if (b <= q0) sgi = j;
+        else if (t1 == INT_MAX) t1 = b;
+        else if (t2 == INT_MAX) t2 = b;
+      }
+      if (32 * i + lane < nhb) {
+        const uint32_t iw[2] = {cur.iv[i].x, cur.iv[i].y};
+        float blk[MP];
+        float a0[MP], a1[MP];
+#pragma unroll
+        for (int m = 0; m < MP; ++m) a0[m] = a1[m] = 0.f;
+        uint32_t f[4];
+        e2m1x8_to_f16x2x4(cur.cv[i], f);
+        if (q0 + 7 < t2) {  // at most one boundary: entries e >= t use segment sgi+1
+          const int t = min(t1 - q0, 8);
+          const uint32_t z0 = zs_a + ((uint32_t)sgi << 8) * kRow;
+          const uint32_t z1 = z0 + 256u * kRow;
+#pragma unroll
+          for (int p = 0; p < 4; ++p) {
+            const float2 v = __half22float2(*reinterpret_cast<const __half2*>(&f[p]));
+            const int e0 = 2 * p, e1 = e0 + 1;
+            const uint32_t b0 = __byte_perm(iw[e0 >> 2], 0u, 0x4440u | (uint32_t)(e0 & 3));
+            const uint32_t b1 = __byte_perm(iw[e1 >> 2], 0u, 0x4440u | (uint32_t)(e1 & 3));
+            fma_z<MP>(a0, (e0 >= t ? z1 : z0) + b0 * kRow, v.x);
+            fma_z<MP>(a1, (e1 >= t ? z1 : z0) + b1 * kRow, v.y);
+          }
+        } else {  // several boundaries inside these 8 entries: walk them (row read from memory)
+          const uint16_t* ssrow = seg_start + (size_t)o * nseg;
+          int sg = sgi, nb = t1;
+#pragma unroll
+          for (int p = 0; p < 4; ++p) {
+            const float2 v = __half22float2(*reinterpret_cast<const __half2*>(&f[p]));
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh) {
+              const int ent = 2 * p + hh;
+              while (q0 + ent >= nb) {
+                ++sg;
+                nb = (sg + 1 < nseg) ? (int)ssrow[sg + 1] : INT_MAX;
+              }
+              const uint32_t b = __byte_perm(iw[ent >> 2], 0u, 0x4440u | (uint32_t)(ent & 3));
+              fma_z<MP>(hh ? a1 : a0, zs_a + (((uint32_t)sg << 8) + b) * kRow, hh ? v.y : v.x);
+            }
+          }
+        }
+        const float sc = e4m3_to_f32((cur.sc >> (8 * i)) & 0xFFu);
+#pragma unroll
+        for (int m = 0; m < MP; ++m) acc[m] = fmaf(a0[m] + a1[m], sc, acc[m]);
+        (void)blk;
+      }
+    }
+#pragma unroll
+    for (int m = 0; m < MP; ++m) {
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) acc[m] += __shfl_xor_sync(0xffffffffu, acc[m], off);
+    }
+    if (lane == 0) {
+#pragma unroll
+      for (int m = 0; m < MP; ++m)
+        if (m < M) Y[(size_t)m * d_out + o] = __float2half_rn(acc[m] * s_C);
+    }
+    cur = nxt;
+    cb = cb_n;
+    nhb = nhb_n;
   }
 }
 
@@ -422,12 +606,11 @@ __global__ void __launch_bounds__(256)
 k_coeff_decode_direct(const uint32_t* __restrict__ col_ptr, const uint8_t* __restrict__ codes,
                       const uint8_t* __restrict__ scales, const uint8_t* __restrict__ idx,
                       const uint16_t* __restrict__ seg_start, int nseg, float s_C, int k, int d_out,
-                      const float* __restrict__ Z, int M, __half* __restrict__ Y) {
+                      const float* __restrict__ Zpart, int nslices, int M, __half* __restrict__ Y) {
   extern __shared__ __align__(16) float zsd[];  // [k + 256][MP]; the tail is zero
   trigger_dependents();
   grid_dependency_wait();
-  for (int i = threadIdx.x * 4; i < k * MP; i += blockDim.x * 4)
-    *reinterpret_cast<float4*>(zsd + i) = *reinterpret_cast<const float4*>(Z + i);
+  stage_z<MP>(zsd, Zpart, nslices, k, blockDim.x);
   // zero tail: an index byte in the last 256-atom segment never reads past the table
   for (int i = k * MP + threadIdx.x; i < (k + 256) * MP; i += blockDim.x) zsd[i] = 0.f;
   __syncthreads();
@@ -439,14 +622,19 @@ k_coeff_decode_direct(const uint32_t* __restrict__ col_ptr, const uint8_t* __res
   if (o < d_out) {
     const uint32_t cb = col_ptr[o], ce = col_ptr[o + 1];
     const int nblk = (int)((ce - cb) >> 4);
-    const uint16_t* ss = seg_start + (size_t)o * nseg;
-    int s = 0, nb = nseg > 1 ? (int)ss[1] : INT_MAX;
+    const SegGlobal ss{seg_start + (size_t)o * nseg};
+    int s = 0, nb = nseg > 1 ? ss(1) : INT_MAX;
+    const uint32_t zs_a = smem_u32(zsd);
     for (int b = lane; b < nblk; b += 32) {
       const int q0 = b << 4;
       const size_t e = cb + (size_t)q0;
       advance_segment(q0, s, nb, ss, nseg);
+      const uint4 iv = ld_stream_v4(idx + e);
+      const uint2 cv = ld_stream_v2(codes + (e >> 1));
+      const uint32_t iw[4] = {iv.x, iv.y, iv.z, iv.w};
+      const uint32_t cw[2] = {cv.x, cv.y};
       float blk[MP];
-      block_sum<MP>(blk, zsd, ld_stream_v4(idx + e), ld_stream_v2(codes + (e >> 1)), q0, s, nb, ss, nseg);
+      entries_sum<MP, 16>(blk, zs_a, iw, cw, q0, s, nb, (s + 2 < nseg) ? ss(s + 2) : INT_MAX, ss, nseg);
       const float sc = e4m3_to_f32(ld_stream_u8(scales + (e >> 4)));
 #pragma unroll
       for (int m = 0; m < MP; ++m) acc[m] = fmaf(blk[m], sc, acc[m]);
@@ -484,11 +672,59 @@ static cudaError_t launch_pdl(const void* fn, dim3 grid, dim3 block, size_t smem
 
 int decode_mp(int M) { return M <= 1 ? 1 : M <= 2 ? 2 : M <= 4 ? 4 : 8; }
 
+// Ring depth: as many chunk stages as fit next to Z within half an SM's shared
+// memory (so the next kernel's CTAs can be resident alongside), at least 2.
+constexpr int kMaxStages = 4;
+constexpr size_t kCoeffSmemCap = 110 * 1024;
+
+static int coeff_stages(int k, int mp) {
+  const size_t z = (size_t)k * mp * 4;
+  if (z + 2 * (size_t)kStageBytes + 8 * kMaxStages > kCoeffSmemCap) return 2;
+  return (int)std::min<size_t>(kMaxStages, (kCoeffSmemCap - z - 8 * kMaxStages) / kStageBytes);
+}
+
 static size_t coeff_smem(int k, int mp) {
-  return (size_t)k * mp * 4 + (size_t)(kChunkEntries / 16) * mp * 4 + 2 * (size_t)kStageBytes + 16;
+  return (size_t)k * mp * 4 + (size_t)coeff_stages(k, mp) * kStageBytes + 8 * kMaxStages;
 }
 
 size_t coeff_decode_smem(int k, int mp) { return coeff_smem(k, mp); }
+
+// Dictionary-stage grid: (k/16 tiles) x slices, each warp J units of 128
+// elements. J is the smallest count that keeps at most two CTAs per SM and
+// lets the M rows of the slice's X fit kDictXsMax bytes of shared memory;
+// one_slice forces a single slice (Z written complete).
+constexpr size_t kDictXsMax = 96 * 1024;
+
+static size_t dict_xs_bytes(int xlen, int M) { return (size_t)M * (xlen + 8) * sizeof(__half); }
+
+DictPlan dict_plan(int d_in, int k, int n_sm, int M, bool one_slice) {
+  const int units = (d_in + 127) / 128;
+  const int tiles = k / kDictTile;
+  DictPlan p;
+  p.J = 1;
+  if (one_slice) {
+    p.J = (units + kDictWarps - 1) / kDictWarps;
+  } else {
+    // J grows until the grid fits four CTAs per SM (4 x 256 threads x 64
+    // registers fill the register file: the kernel is latency-bound, so resident
+    // warps matter most); it shrinks back while the slice's X rows would not fit
+    // the shared-memory cap
+    while (p.J < units) {
+      const size_t ctas = (size_t)tiles * ((units + kDictWarps * p.J - 1) / (kDictWarps * p.J));
+      if (ctas <= (size_t)4 * n_sm) break;
+      ++p.J;
+    }
+    while (p.J > 1 && dict_xs_bytes(std::min(d_in, kDictWarps * p.J * 128), M) > kDictXsMax) --p.J;
+  }
+  p.slices = (units + kDictWarps * p.J - 1) / (kDictWarps * p.J);
+  return p;
+}
+
+int dict_max_slices(int d_in, int k, int n_sm) {
+  int m = 1;
+  for (int M = 1; M <= kDecodeMaxTokens; ++M) m = std::max(m, dict_plan(d_in, k, n_sm, M, false).slices);
+  return m;
+}
 
 cudaError_t prepare_decode_kernels(int device) {
   int optin = 0;
@@ -503,12 +739,16 @@ cudaError_t prepare_decode_kernels(int device) {
                                   optin - (int)fa.sharedSizeBytes)))                                  \
       return e;                                                                                       \
   }
-  SET_SMEM(k_dict_decode<true>);
-  SET_SMEM(k_dict_decode<false>);
+  SET_SMEM((k_dict_decode<1, true>));
+  SET_SMEM((k_dict_decode<2, true>));
   SET_SMEM(k_coeff_decode<1>);
   SET_SMEM(k_coeff_decode<2>);
   SET_SMEM(k_coeff_decode<4>);
   SET_SMEM(k_coeff_decode<8>);
+  SET_SMEM(k_coeff_gather<1>);
+  SET_SMEM(k_coeff_gather<2>);
+  SET_SMEM(k_coeff_gather<4>);
+  SET_SMEM(k_coeff_gather<8>);
   SET_SMEM(k_coeff_decode_direct<1>);
   SET_SMEM(k_coeff_decode_direct<2>);
   SET_SMEM(k_coeff_decode_direct<4>);
@@ -517,22 +757,28 @@ cudaError_t prepare_decode_kernels(int device) {
   return e;
 }
 
-cudaError_t launch_dict_decode(const dictproj_group* g, const __half* X, int M, int mp, float* Z,
-                               cudaStream_t stream) {
+cudaError_t launch_dict_decode(const dictproj_group* g, const __half* X, int M, int mp, float* Zpart,
+                               const DictPlan& plan, cudaStream_t stream) {
   const uint8_t* codes = g->codes;
   const uint8_t* scales = g->scales;
   float s = g->s;
-  int d_in = g->d_in;
-  void* args[] = {(void*)&codes, (void*)&scales, (void*)&s, (void*)&d_in, (void*)&X,
-                  (void*)&M, (void*)&mp, (void*)&Z};
-  const size_t xs = (size_t)M * (d_in + 8) * sizeof(__half);
-  const dim3 grid(g->k / kDictAtoms), block(kDictWarps * 32);
-  if (xs <= kDictXSmemMax) return launch_pdl((const void*)k_dict_decode<true>, grid, block, xs, stream, args);
-  return launch_pdl((const void*)k_dict_decode<false>, grid, block, 0, stream, args);
+  int d_in = g->d_in, k = g->k, J = plan.J;
+  void* args[] = {(void*)&codes, (void*)&scales, (void*)&s, (void*)&d_in, (void*)&k, (void*)&X,
+                  (void*)&M, (void*)&mp, (void*)&Zpart, (void*)&J};
+  const dim3 grid(g->k / kDictTile, plan.slices), block(kDictWarps * 32);
+  const size_t xs = dict_xs_bytes(std::min(d_in, kDictWarps * plan.J * 128), M);
+  const bool use_xs = xs <= 200 * 1024;
+  const size_t smem = use_xs ? xs : 0;
+#define DICT_LAUNCH(R)                                                                                \
+  return use_xs ? launch_pdl((const void*)k_dict_decode<R, true>, grid, block, smem, stream, args)     \
+                : launch_pdl((const void*)k_dict_decode<R, false>, grid, block, 0, stream, args);
+  if (plan.J == 1) DICT_LAUNCH(1)
+  DICT_LAUNCH(2)
+#undef DICT_LAUNCH
 }
 
-cudaError_t launch_coeff_decode(const dictproj_layer* l, const float* Z, int M, int mp, __half* Y,
-                                cudaStream_t stream) {
+cudaError_t launch_coeff_decode(const dictproj_layer* l, const float* Zpart, int nslices, int M, int mp,
+                                __half* Y, cudaStream_t stream) {
   const uint8_t* codes = l->codes;
   const uint8_t* scales = l->scales;
   const uint8_t* idx = l->idx;
@@ -540,15 +786,32 @@ cudaError_t launch_coeff_decode(const dictproj_layer* l, const float* Z, int M, 
   int nseg = l->nseg;
   float s = l->s;
   int k = l->k, d_out = l->d_out;
+  if (l->gather_ok) {
+    const uint32_t* col_ptr = l->col_ptr;
+    int cpc = (d_out + l->n_sm - 1) / l->n_sm;
+    void* args[] = {(void*)&col_ptr, (void*)&codes, (void*)&scales, (void*)&idx, (void*)&ss, (void*)&nseg,
+                    (void*)&s, (void*)&k, (void*)&d_out, (void*)&Zpart, (void*)&nslices, (void*)&M, (void*)&Y,
+                    (void*)&cpc};
+    const dim3 grid((d_out + cpc - 1) / cpc), block(kGatherWarps * 32);
+    const size_t smem = (size_t)(k + 256) * mp * sizeof(float);
+    switch (mp) {
+      case 1: return launch_pdl((const void*)k_coeff_gather<1>, grid, block, smem, stream, args);
+      case 2: return launch_pdl((const void*)k_coeff_gather<2>, grid, block, smem, stream, args);
+      case 4: return launch_pdl((const void*)k_coeff_gather<4>, grid, block, smem, stream, args);
+      default: return launch_pdl((const void*)k_coeff_gather<8>, grid, block, smem, stream, args);
+    }
+  }
   if (l->chunks[0]) {
     const size_t smem = coeff_smem(k, mp);
-    // two CTAs per SM when their shared memory (plus the 1 KB the SM reserves per CTA) fits
-    const int pi = (l->chunks[1] && 2 * (smem + 1024) <= (size_t)l->smem_per_sm) ? 1 : 0;
+    // one CTA per SM (half the register file), leaving room for the next call's
+    // dictionary kernel to become resident and prefetch its weights
+    const int pi = 0;
     const uint4* chunks = reinterpret_cast<const uint4*>(l->chunks[pi]);
     const int* cta_ptr = l->cta_ptr[pi];
+    int nst = coeff_stages(k, mp);
     void* args[] = {(void*)&chunks, (void*)&cta_ptr, (void*)&codes, (void*)&scales, (void*)&idx,
-                    (void*)&ss, (void*)&nseg, (void*)&s, (void*)&k, (void*)&d_out, (void*)&Z,
-                    (void*)&M, (void*)&Y};
+                    (void*)&ss, (void*)&nseg, (void*)&s, (void*)&k, (void*)&d_out, (void*)&Zpart,
+                    (void*)&nslices, (void*)&M, (void*)&Y, (void*)&nst};
     const dim3 grid(l->n_cta[pi]), block(kCoeffThreads);
     switch (mp) {
       case 1: return launch_pdl((const void*)k_coeff_decode<1>, grid, block, smem, stream, args);
@@ -559,7 +822,8 @@ cudaError_t launch_coeff_decode(const dictproj_layer* l, const float* Z, int M, 
   }
   const uint32_t* col_ptr = l->col_ptr;
   void* args[] = {(void*)&col_ptr, (void*)&codes, (void*)&scales, (void*)&idx, (void*)&ss,
-                  (void*)&nseg, (void*)&s, (void*)&k, (void*)&d_out, (void*)&Z, (void*)&M, (void*)&Y};
+                  (void*)&nseg, (void*)&s, (void*)&k, (void*)&d_out, (void*)&Zpart, (void*)&nslices,
+                  (void*)&M, (void*)&Y};
   const dim3 grid((d_out + 7) / 8), block(256);
   const size_t smem = (size_t)(k + 256) * mp * sizeof(float);
   switch (mp) {
@@ -579,7 +843,7 @@ bool plan_coeff_chunks(const uint32_t* pcol_ptr, int d_out, int nseg, int G, std
   chunks.clear();
   cta_ptr.assign(G + 1, 0);
   const uint64_t T = pcol_ptr[d_out];
-  const int max_cols = std::max(1, std::min(kChunkEntries, kSegBytes / (2 * nseg)));
+  const int max_cols = std::max(1, std::min(kChunkCols, kSegBytes / (2 * nseg)));
   for (int o = 0; o < d_out; ++o)
     if (pcol_ptr[o + 1] - pcol_ptr[o] > (uint32_t)kChunkEntries) return false;
   int o = 0;
@@ -601,6 +865,13 @@ bool plan_coeff_chunks(const uint32_t* pcol_ptr, int d_out, int nseg, int G, std
     }
   }
   cta_ptr[G] = (int)(chunks.size() / 4);
+  return true;
+}
+
+bool gather_supported(const uint32_t* pcol_ptr, int d_out, int nseg) {
+  if (nseg > 32) return false;
+  for (int o = 0; o < d_out; ++o)
+    if (pcol_ptr[o + 1] - pcol_ptr[o] > (uint32_t)(kRmax * 256)) return false;
   return true;
 }
 

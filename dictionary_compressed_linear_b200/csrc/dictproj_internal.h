@@ -42,8 +42,10 @@ struct dictproj_group {
   uint8_t* codes;          // [k][d_in/2]
   uint8_t* scales;         // [k][d_in/16]
   size_t codes_bytes, scales_bytes;
+  int n_sm;                // SMs of the device (sizes the decode grid)
   // scratch
-  float* z32;              // decode Z, fp32 [k][8]
+  float* z32;              // decode Z partial sums, fp32 [zslices][k][8]
+  int zslices;             // d_in slices of the decode dictionary stage
   uint16_t* z16;           // prefill Z, fp16 [max_tokens][k] (allocated when max_tokens > 8)
   uint16_t* dexp;          // prefill: D expanded to fp16, atom-major [k][d_in]
   unsigned int* err;       // device error word for bounded waits
@@ -67,4 +69,6 @@ struct dictproj_layer {
   int* cta_ptr[2];         // [n_cta+1], device
   int n_cta[2];
   int smem_per_sm;         // bytes of shared memory per SM on this device
+  int n_sm;                // SMs of the device
+  bool gather_ok;          // the direct gather kernel serves this layer
 };

@@ -10,18 +10,29 @@
 
 namespace dictproj {
 
-// decode path (M <= 8): Z fp32 [k][mp], mp = next power of two >= M (at most 8)
+// decode path (M <= 8): Z fp32 [k][mp], mp = next power of two >= M (at most 8),
+// written by the dictionary stage as `slices` partial sums Zpart[slice][k][mp]
 int decode_mp(int M);
 size_t coeff_decode_smem(int k, int mp);
 cudaError_t prepare_decode_kernels(int device);
-cudaError_t launch_dict_decode(const dictproj_group* g, const __half* X, int M, int mp, float* Z,
-                               cudaStream_t stream);
-cudaError_t launch_coeff_decode(const dictproj_layer* l, const float* Z, int M, int mp, __half* Y,
-                                cudaStream_t stream);
+
+struct DictPlan {
+  int J;       // 128-element units per warp
+  int slices;  // d_in slices = grid.y
+};
+DictPlan dict_plan(int d_in, int k, int n_sm, int M, bool one_slice);
+int dict_max_slices(int d_in, int k, int n_sm);  // over all decode M
+cudaError_t launch_dict_decode(const dictproj_group* g, const __half* X, int M, int mp, float* Zpart,
+                               const DictPlan& plan, cudaStream_t stream);
+cudaError_t launch_coeff_decode(const dictproj_layer* l, const float* Zpart, int nslices, int M, int mp,
+                                __half* Y, cudaStream_t stream);
 
 // Work plan of the chunked coefficient kernel for a grid of G CTAs (host side).
 bool plan_coeff_chunks(const uint32_t* pcol_ptr, int d_out, int nseg, int G, std::vector<uint32_t>& chunks,
                        std::vector<int>& cta_ptr);
+// Whether the direct gather kernel serves a layer (every column <= 1280 padded
+// entries, at most 32 segments).
+bool gather_supported(const uint32_t* pcol_ptr, int d_out, int nseg);
 // Read and clear the device error word of the decode kernels.
 cudaError_t take_decode_error(unsigned int* out);
 

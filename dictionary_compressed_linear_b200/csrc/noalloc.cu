@@ -108,9 +108,10 @@ extern "C" int dictproj_forward_noalloc(const dictproj_device_group* group, cons
 
   cudaStream_t s = (cudaStream_t)stream;
   cudaError_t e;
-  if ((e = launch_dict_decode(&g, static_cast<const __half*>(X), M, mp, z, s)) != cudaSuccess)
+  const DictPlan plan = dict_plan(d_in, k, 1, M, true);  // one slice: Z fits the static array
+  if ((e = launch_dict_decode(&g, static_cast<const __half*>(X), M, mp, z, plan, s)) != cudaSuccess)
     return cuda_fail(e, "forward_noalloc: dictionary stage launch");
-  if ((e = launch_coeff_decode(&l, z, M, mp, static_cast<__half*>(Y), s)) != cudaSuccess)
+  if ((e = launch_coeff_decode(&l, z, 1, M, mp, static_cast<__half*>(Y), s)) != cudaSuccess)
     return cuda_fail(e, "forward_noalloc: coefficient stage launch");
   return DICTPROJ_OK;
 }
