@@ -201,12 +201,33 @@ class Stack:
         self.y = torch.zeros(self.y_elems, dtype=torch.float16, device="cuda")
         self.y_host = torch.zeros(self.y_elems, dtype=torch.float16).pin_memory()
 
-    def forward_all(self, dp, stream_handle):
-        xp, yp = self.x.data_ptr(), self.y.data_ptr()
+    def call_groups(self, batched):
+        """Projections issued together: the ones of one layer reading the same input
+        (q/k/v, gate/up) when batched, else one call per projection."""
+        calls, cur = [], []
         for i, p in enumerate(self.w.projections):
-            xo = self.x_off[(p.layer, p.site)][0]
-            dp.dictproj_forward(xp + 2 * xo, self.M, self.layers[i], self.groups[(p.group, p.ptype)],
-                                yp + 2 * self.y_off[i], stream_handle)
+            if cur and (not batched or (p.layer, p.site) != cur[-1][1]):
+                calls.append([j for j, _ in cur])
+                cur = []
+            cur.append((i, (p.layer, p.site)))
+        if cur:
+            calls.append([j for j, _ in cur])
+        return calls
+
+    def forward_all(self, dp, stream_handle, batched=True):
+        xp, yp = self.x.data_ptr(), self.y.data_ptr()
+        for call in self.call_groups(batched):
+            xs, ls, gs, ys = [], [], [], []
+            for i in call:
+                p = self.w.projections[i]
+                xs.append(xp + 2 * self.x_off[(p.layer, p.site)][0])
+                ls.append(self.layers[i])
+                gs.append(self.groups[(p.group, p.ptype)])
+                ys.append(yp + 2 * self.y_off[i])
+            if len(call) == 1:
+                dp.dictproj_forward(xs[0], self.M, ls[0], gs[0], ys[0], stream_handle)
+            else:
+                dp.dictproj_forward_batch(xs, self.M, ls, gs, ys, stream_handle)
 
 
 def capture(torch, stream, fn):
@@ -333,6 +354,8 @@ def main():
     ap.add_argument("--layers", type=int, default=32)
     ap.add_argument("--stage-reps", type=int, default=50)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-batch", action="store_true",
+                    help="one dictproj_forward per projection instead of batching q/k/v and gate/up")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -368,7 +391,8 @@ def main():
     stack = Stack(wl, M, torch, dp, log)
     stream = torch.cuda.Stream()
     sh = stream.cuda_stream
-    graph = capture(torch, stream, lambda: stack.forward_all(dp, sh))
+    graph = capture(torch, stream, lambda: stack.forward_all(dp, sh, batched=not args.no_batch))
+    calls_per_step = len(stack.call_groups(not args.no_batch))
     for _ in range(args.warmup):
         with torch.cuda.stream(stream):
             graph.replay()
@@ -393,7 +417,14 @@ def main():
     ms_per_step = ms / args.steps
     tokens = world * M * args.steps
     value = tokens / (ms / 1e3)
-    launches_per_step = 2 * len(wl.projections)
+    launches_per_step = 2 * calls_per_step
+    # the same step with one call per projection, for comparison
+    ms_unbatched = None
+    if not args.no_batch:
+        g_u = capture(torch, stream, lambda: stack.forward_all(dp, sh, batched=False))
+        time_replays(torch, stream, g_u, 5)
+        ms_unbatched = time_replays(torch, stream, g_u, max(10, args.steps // 4)) / max(10, args.steps // 4)
+        del g_u
 
     # ---------------- per-stage timing for the roofline (each stage alone, same launch config)
     kmax = max(p.k for p in wl.projections)
@@ -473,6 +504,9 @@ def main():
         "config": {"workload": f"{wl.name}: {args.layers} layers in {args.layers // 2} groups x 7 projection "
                                "types (LLaMA-7B shapes), NVFP4 D/C, C density U[0.2,0.4], M=1",
                    "tokens_per_step": M, "projections_per_step": len(wl.projections),
+                   "calls_per_step": calls_per_step,
+                   "batching": "q/k/v and gate/up share a call (dictproj_forward_batch)" if not args.no_batch
+                               else "one dictproj_forward per projection",
                    "weights": "nvfp4 (E2M1 + E4M3/16 + fp32)", "activations": "fp16", "accumulate": "fp32",
                    "l2": "inputs larger than L2 (packed weights ~2.6 GB, no flush needed)",
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
@@ -483,6 +517,7 @@ def main():
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clocks,
         "step": {"algorithmic_bytes": step_bytes, "GB/s": round(step_gbs, 1),
+                 "ms_per_step_one_call_per_projection": round(ms_unbatched, 5) if ms_unbatched else None,
                  "frac_of_peak": round(step_gbs / peak, 4),
                  "algorithmic_bytes_dictionary_once_per_group": step_bytes_once,
                  "GB/s_dictionary_once_per_group": round(step_bytes_once / (ms_per_step / 1e3) / 1e9, 1)},

@@ -76,6 +76,9 @@ SIGNATURES = [
     ("dictproj_forward", C.c_int, [C.c_void_p, C.c_int, C.c_void_p, C.c_void_p, C.c_void_p, C.c_void_p]),
     ("dictproj_forward_path", C.c_int,
      [C.c_void_p, C.c_int, C.c_void_p, C.c_void_p, C.c_void_p, C.c_void_p, C.c_int]),
+    ("dictproj_forward_batch", C.c_int,
+     [C.c_int, C.POINTER(C.c_void_p), C.c_int, C.POINTER(C.c_void_p), C.POINTER(C.c_void_p),
+      C.POINTER(C.c_void_p), C.c_void_p]),
     ("dictproj_dictionary_stage", C.c_int, [C.c_void_p, C.c_int, C.c_void_p, C.c_void_p, C.c_void_p]),
     ("dictproj_coefficient_stage", C.c_int, [C.c_void_p, C.c_int, C.c_void_p, C.c_void_p, C.c_void_p]),
     ("dictproj_forward_noalloc", C.c_int,
@@ -317,6 +320,14 @@ def dictproj_forward_status(X_ptr, M, layer_handle, group_handle, Y_ptr, stream=
     """Raw status of a forward call (no exception), for boundary tests."""
     return lib().dictproj_forward_path(C.c_void_p(X_ptr), M, layer_handle, group_handle,
                                        C.c_void_p(Y_ptr), C.c_void_p(stream), path)
+
+
+def dictproj_forward_batch(X_ptrs, M: int, layers, groups, Y_ptrs, stream: int = 0):
+    """Independent projections in one call (lists of equal length <= 4)."""
+    n = len(layers)
+    arr = lambda vals: (C.c_void_p * n)(*[C.c_void_p(v) for v in vals])
+    _check(lib().dictproj_forward_batch(n, arr(X_ptrs), M, arr([l.handle for l in layers]),
+                                        arr([g.handle for g in groups]), arr(Y_ptrs), C.c_void_p(stream)))
 
 
 def dictproj_dictionary_stage(X_ptr: int, M: int, group: Group, Z_ptr: int, stream: int = 0):

@@ -462,6 +462,59 @@ int dictproj_forward_path(const void* X, int M, const dictproj_layer* layer, con
   return DICTPROJ_OK;
 }
 
+int dictproj_forward_batch(int n, const void* const* X, int M, const dictproj_layer* const* layers,
+                           const dictproj_group* const* groups, void* const* Y, void* stream) {
+  clear_error();
+  if (!X || !layers || !groups || !Y) return fail(DICTPROJ_ERR_NULL, "forward_batch: NULL array");
+  if (n < 1 || n > DICTPROJ_MAX_BATCH)
+    return fail(DICTPROJ_ERR_RANGE, "forward_batch: n=%d outside [1, %d]", n, DICTPROJ_MAX_BATCH);
+  for (int i = 0; i < n; ++i) {
+    if (!X[i] || !Y[i] || !layers[i] || !groups[i]) return fail(DICTPROJ_ERR_NULL, "forward_batch: NULL entry %d", i);
+    if (M < 1 || M > groups[i]->max_tokens)
+      return fail(DICTPROJ_ERR_RANGE, "forward_batch: M=%d outside [1, %d] for entry %d", M, groups[i]->max_tokens, i);
+    if (layers[i]->k != groups[i]->k)
+      return fail(DICTPROJ_ERR_MISMATCH, "forward_batch: entry %d layer k=%d != group k=%d", i, layers[i]->k,
+                  groups[i]->k);
+    if (layers[i]->device != groups[i]->device || groups[i]->device != groups[0]->device)
+      return fail(DICTPROJ_ERR_MISMATCH, "forward_batch: entries on different devices");
+    if (((uintptr_t)X[i] & 15) || ((uintptr_t)Y[i] & 15))
+      return fail(DICTPROJ_ERR_ALIGN, "forward_batch: X and Y must be 16-byte aligned (entry %d)", i);
+    for (int j = 0; j < i; ++j)
+      if (groups[j] == groups[i]) return fail(DICTPROJ_ERR_MISMATCH, "forward_batch: group of entry %d repeated", i);
+  }
+  int dev = -1;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "forward_batch: cudaGetDevice");
+  if (dev != groups[0]->device)
+    return fail(DICTPROJ_ERR_MISMATCH, "forward_batch: current device %d, handles on device %d", dev, groups[0]->device);
+  if (M > kDecodeMaxTokens) {  // prefill: one projection after another
+    for (int i = 0; i < n; ++i) {
+      const int st = dictproj_forward_path(X[i], M, layers[i], groups[i], Y[i], stream, DICTPROJ_PATH_AUTO);
+      if (st) return st;
+    }
+    return DICTPROJ_OK;
+  }
+  const int mp = decode_mp(M);
+  DictPlan plans[kDecodeMaxBatch];
+  const __half* xs[kDecodeMaxBatch];
+  float* zs[kDecodeMaxBatch];
+  int ns[kDecodeMaxBatch];
+  __half* ys[kDecodeMaxBatch];
+  for (int i = 0; i < n; ++i) {
+    plans[i] = dict_plan(groups[i]->d_in, groups[i]->k, groups[i]->n_sm, M, false);
+    xs[i] = static_cast<const __half*>(X[i]);
+    zs[i] = groups[i]->z32;
+    ns[i] = plans[i].slices;
+    ys[i] = static_cast<__half*>(Y[i]);
+  }
+  cudaStream_t s = (cudaStream_t)stream;
+  if ((e = launch_dict_decode_batch(n, groups, xs, M, mp, zs, plans, s)) != cudaSuccess)
+    return cuda_fail(e, "forward_batch: dictionary stage launch");
+  if ((e = launch_coeff_decode_batch(n, layers, zs, ns, M, mp, ys, s)) != cudaSuccess)
+    return cuda_fail(e, "forward_batch: coefficient stage launch");
+  return DICTPROJ_OK;
+}
+
 int dictproj_forward(const void* X, int M, const dictproj_layer* layer, const dictproj_group* group, void* Y,
                      void* stream) {
   return dictproj_forward_path(X, M, layer, group, Y, stream, DICTPROJ_PATH_AUTO);

@@ -49,6 +49,36 @@ constexpr int kDictTile = 16;     // atoms per CTA = MMA M
 
 // A unit is 16 atoms x 128 d_in elements: thread (g, t) of a warp holds atoms g
 // and g+8 of the tile and elements [128u + 32t, 128u + 32t + 32).
+// By-value launch descriptors for batches of independent projections.
+constexpr int kMaxBatch = 4;
+struct DictProj {
+  const uint8_t* codes;
+  const uint8_t* scales;
+  const __half* X;
+  float* Zpart;
+  float s;
+  int d_in, k, J, tiles, block_begin;
+};
+struct DictBatch {
+  DictProj p[kMaxBatch];
+  int n, M, mp;
+};
+struct CoeffProj {
+  const uint32_t* col_ptr;
+  const uint8_t* codes;
+  const uint8_t* scales;
+  const uint8_t* idx;
+  const uint16_t* seg_start;
+  const float* Zpart;
+  __half* Y;
+  float s;
+  int nseg, k, d_out, nslices, cols_per_cta, block_begin;
+};
+struct CoeffBatch {
+  CoeffProj p[kMaxBatch];
+  int n, M;
+};
+
 struct DictUnit {
   uint4 wa, wb;      // 16 code bytes of atoms g and g+8 (32 elements each)
   uint32_t sa, sb;   // their two E4M3 block scales (2 bytes each)
@@ -102,16 +132,30 @@ __device__ __forceinline__ void dict_unit_mma(float acc[2][4], const DictUnit& u
 }
 
 // Zpart[slice][atom][mp] = s_D * sum over the slice's units of X[m][i] * D[i][atom].
-// Grid: (k / 16 tiles) x (slices); slice y covers units [y*8*J, (y+1)*8*J).
+// One launch serves up to kMaxBatch independent projections; projection i owns
+// blocks [block_begin, block_begin + tiles * slices) of the 1-D grid, block
+// (tile, slice) = (local % tiles, local / tiles); slice y covers units
+// [y*8*J, (y+1)*8*J).
 // RING = register prefetch depth in units (1, 2 or 4; at most J is useful).
 // XS: X rows of the slice are staged in shared memory (stride xlen + 8 halves).
 template <int RING, bool XS>
 __global__ void __launch_bounds__(kDictWarps * 32, 4)  // at most 64 registers
-k_dict_decode(const uint8_t* __restrict__ codes, const uint8_t* __restrict__ scales, float s_D, int d_in, int k,
-              const __half* __restrict__ X, int M, int mp, float* __restrict__ Zpart, int J) {
+k_dict_decode(const __grid_constant__ DictBatch batch) {
   extern __shared__ __align__(16) unsigned char dsmem[];
   __shared__ float red[kDictWarps][kDictTile][8];
-  const int tile = blockIdx.x, slice = blockIdx.y;
+  // projection of this CTA; its blocks are [block_begin, block_begin + tiles * slices)
+  int pi = 0;
+  while (pi + 1 < batch.n && (int)blockIdx.x >= batch.p[pi + 1].block_begin) ++pi;
+  const DictProj& pr = batch.p[pi];
+  const uint8_t* __restrict__ codes = pr.codes;
+  const uint8_t* __restrict__ scales = pr.scales;
+  const float s_D = pr.s;
+  const int d_in = pr.d_in, k = pr.k, J = pr.J;
+  const __half* __restrict__ X = pr.X;
+  float* __restrict__ Zpart = pr.Zpart;
+  const int M = batch.M, mp = batch.mp;
+  const int local = (int)blockIdx.x - pr.block_begin;
+  const int tile = local % pr.tiles, slice = local / pr.tiles;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = lane >> 2, t = lane & 3;
   const size_t crow = (size_t)(d_in >> 1), srow = (size_t)(d_in >> 4);
@@ -488,13 +532,23 @@ __device__ __forceinline__ void load_col(ColData& d, int o, int d_out, const uin
 
 template <int MP>
 __global__ void __launch_bounds__(kGatherWarps * 32, 1)  // 1024 threads, at most 64 registers
-k_coeff_gather(const uint32_t* __restrict__ col_ptr, const uint8_t* __restrict__ codes,
-               const uint8_t* __restrict__ scales, const uint8_t* __restrict__ idx,
-               const uint16_t* __restrict__ seg_start, int nseg, float s_C, int k, int d_out,
-               const float* __restrict__ Zpart, int nslices, int M, __half* __restrict__ Y, int cols_per_cta) {
+k_coeff_gather(const __grid_constant__ CoeffBatch batch) {
   extern __shared__ __align__(16) float zsg[];  // [k + 256][MP]; the tail is zero
+  int pi = 0;
+  while (pi + 1 < batch.n && (int)blockIdx.x >= batch.p[pi + 1].block_begin) ++pi;
+  const CoeffProj& pr = batch.p[pi];
+  const uint32_t* __restrict__ col_ptr = pr.col_ptr;
+  const uint8_t* __restrict__ codes = pr.codes;
+  const uint8_t* __restrict__ scales = pr.scales;
+  const uint8_t* __restrict__ idx = pr.idx;
+  const uint16_t* __restrict__ seg_start = pr.seg_start;
+  const int nseg = pr.nseg, k = pr.k, d_out = pr.d_out, nslices = pr.nslices, cols_per_cta = pr.cols_per_cta;
+  const float s_C = pr.s;
+  const float* __restrict__ Zpart = pr.Zpart;
+  __half* __restrict__ Y = pr.Y;
+  const int M = batch.M;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int o_begin = blockIdx.x * cols_per_cta;
+  const int o_begin = ((int)blockIdx.x - pr.block_begin) * cols_per_cta;
   const int o_end = min(d_out, o_begin + cols_per_cta);
   if (threadIdx.x == 0 && o_begin < o_end) {  // bulk L2 prefetch of this CTA's columns
     const size_t e0 = col_ptr[o_begin], e1 = col_ptr[o_end];
@@ -522,22 +576,33 @@ k_coeff_gather(const uint32_t* __restrict__ col_ptr, const uint8_t* __restrict__
     float acc[MP];
 #pragma unroll
     for (int m = 0; m < MP; ++m) acc[m] = 0.f;
-    int s_lo = 0;  // segment of the current window start (uniform)
+    // Lane j holds seg_start[j] (the first entry of segment j). For the window of
+    // 256 entries starting at w, a boundary b in (w, w+256) lies at the start of
+    // lane p = (b-w)/8's half-block when (b-w) % 8 == 0, else inside it; two
+    // OR-reduced lane masks give every lane its segment with two popcounts.
+    const bool is_bnd = lane >= 1 && lane < nseg;
 #pragma unroll
     for (int i = 0; i < kRmax; ++i) {
       const int w = 256 * i;
       if (w >= 8 * nhb) break;
-      while (s_lo + 1 < nseg && __shfl_sync(0xffffffffu, cur.ssv, s_lo + 1) <= w) ++s_lo;
+      const int b = cur.ssv;  // boundary held by this lane (meaningful iff is_bnd)
+      const int s_lo = __popc(__ballot_sync(0xffffffffu, is_bnd && b <= w));  // segment of entry w
+      const bool in_win = is_bnd && b > w && b < w + 256;
+      const int rel = b - w;
+      const uint32_t at_start = (in_win && (rel & 7) == 0) ? (1u << (rel >> 3)) : 0u;
+      const uint32_t inside = (in_win && (rel & 7) != 0) ? (1u << (rel >> 3)) : 0u;
+      const uint32_t A = __reduce_or_sync(0xffffffffu, at_start);
+      const uint32_t B = __reduce_or_sync(0xffffffffu, inside);
+      const int nwin = __popc(__ballot_sync(0xffffffffu, in_win));
+      const bool collide = nwin != __popc(A) + __popc(B) || (A & B) != 0u;  // two boundaries in one half-block
+      const uint32_t le = lane == 31 ? 0xffffffffu : ((2u << lane) - 1u);
+      const int before = __popc(A & le) + __popc(B & (le >> 1));  // boundaries <= q0 in the window
+      const int sgi = s_lo + before;                               // segment of q0
       const int q0 = w + 8 * lane;
-      // segment of q0 and the next two boundaries, from the window's boundaries
-      int sgi = s_lo, t1 = INT_MAX, t2 = INT_MAX;
-      for (int j = s_lo + 1; j < nseg; ++j) {
-        const int b = __shfl_sync(0xffffffffu, cur.ssv, j);
-        if (b > w + 256 + 8) break;
-        if (b <= q0) sgi = j;
-        else if (t1 == INT_MAX) t1 = b;
-        else if (t2 == INT_MAX) t2 = b;
-      }
+      // the boundary inside this half-block, if any, is segment sgi+1's start
+      const int bn = __shfl_sync(0xffffffffu, b, min(sgi + 1, 31));
+      const int t1 = ((B >> lane) & 1u) ? bn : INT_MAX;
+      const int t2 = collide ? q0 : INT_MAX;  // forces the walk for the whole window
       if (32 * i + lane < nhb) {
         const uint32_t iw[2] = {cur.iv[i].x, cur.iv[i].y};
         float blk[MP];
@@ -561,7 +626,9 @@ k_coeff_gather(const uint32_t* __restrict__ col_ptr, const uint8_t* __restrict__
           }
         } else {  // several boundaries inside these 8 entries: walk them (row read from memory)
           const uint16_t* ssrow = seg_start + (size_t)o * nseg;
-          int sg = sgi, nb = t1;
+          int sg = 0;
+          for (int j = 1; j < nseg; ++j) sg += ((int)ssrow[j] <= q0);
+          int nb = (sg + 1 < nseg) ? (int)ssrow[sg + 1] : INT_MAX;
 #pragma unroll
           for (int p = 0; p < 4; ++p) {
             const float2 v = __half22float2(*reinterpret_cast<const __half2*>(&f[p]));
@@ -757,24 +824,95 @@ cudaError_t prepare_decode_kernels(int device) {
   return e;
 }
 
-cudaError_t launch_dict_decode(const dictproj_group* g, const __half* X, int M, int mp, float* Zpart,
-                               const DictPlan& plan, cudaStream_t stream) {
-  const uint8_t* codes = g->codes;
-  const uint8_t* scales = g->scales;
-  float s = g->s;
-  int d_in = g->d_in, k = g->k, J = plan.J;
-  void* args[] = {(void*)&codes, (void*)&scales, (void*)&s, (void*)&d_in, (void*)&k, (void*)&X,
-                  (void*)&M, (void*)&mp, (void*)&Zpart, (void*)&J};
-  const dim3 grid(g->k / kDictTile, plan.slices), block(kDictWarps * 32);
-  const size_t xs = dict_xs_bytes(std::min(d_in, kDictWarps * plan.J * 128), M);
+cudaError_t launch_dict_decode_batch(int n, const dictproj_group* const* g, const __half* const* X, int M,
+                                     int mp, float* const* Zpart, const DictPlan* plans, cudaStream_t stream) {
+  DictBatch b{};
+  b.n = n;
+  b.M = M;
+  b.mp = mp;
+  int blocks = 0, maxJ = 1;
+  size_t xs = 0;
+  for (int i = 0; i < n; ++i) {
+    DictProj& p = b.p[i];
+    p.codes = g[i]->codes;
+    p.scales = g[i]->scales;
+    p.s = g[i]->s;
+    p.d_in = g[i]->d_in;
+    p.k = g[i]->k;
+    p.X = X[i];
+    p.Zpart = Zpart[i];
+    p.J = plans[i].J;
+    p.tiles = g[i]->k / kDictTile;
+    p.block_begin = blocks;
+    blocks += p.tiles * plans[i].slices;
+    maxJ = std::max(maxJ, p.J);
+    xs = std::max(xs, dict_xs_bytes(std::min(p.d_in, kDictWarps * p.J * 128), M));
+  }
+  void* args[] = {(void*)&b};
+  const dim3 grid(blocks), block(kDictWarps * 32);
   const bool use_xs = xs <= 200 * 1024;
   const size_t smem = use_xs ? xs : 0;
 #define DICT_LAUNCH(R)                                                                                \
   return use_xs ? launch_pdl((const void*)k_dict_decode<R, true>, grid, block, smem, stream, args)     \
                 : launch_pdl((const void*)k_dict_decode<R, false>, grid, block, 0, stream, args);
-  if (plan.J == 1) DICT_LAUNCH(1)
+  if (maxJ == 1) DICT_LAUNCH(1)
   DICT_LAUNCH(2)
 #undef DICT_LAUNCH
+}
+
+cudaError_t launch_dict_decode(const dictproj_group* g, const __half* X, int M, int mp, float* Zpart,
+                               const DictPlan& plan, cudaStream_t stream) {
+  return launch_dict_decode_batch(1, &g, &X, M, mp, &Zpart, &plan, stream);
+}
+
+static cudaError_t launch_gather_batch(int n, const dictproj_layer* const* l, const float* const* Zpart,
+                                       const int* nslices, int M, int mp, __half* const* Y, cudaStream_t stream) {
+  CoeffBatch b{};
+  b.n = n;
+  b.M = M;
+  int blocks = 0, kmax = 0;
+  for (int i = 0; i < n; ++i) {
+    CoeffProj& p = b.p[i];
+    p.col_ptr = l[i]->col_ptr;
+    p.codes = l[i]->codes;
+    p.scales = l[i]->scales;
+    p.idx = l[i]->idx;
+    p.seg_start = l[i]->seg_start;
+    p.nseg = l[i]->nseg;
+    p.k = l[i]->k;
+    p.d_out = l[i]->d_out;
+    p.s = l[i]->s;
+    p.Zpart = Zpart[i];
+    p.nslices = nslices[i];
+    p.Y = Y[i];
+    // columns per CTA: one CTA per SM for a single projection, shared out over the batch
+    const int ctas = std::max(1, l[i]->n_sm / n);
+    p.cols_per_cta = (p.d_out + ctas - 1) / ctas;
+    p.block_begin = blocks;
+    blocks += (p.d_out + p.cols_per_cta - 1) / p.cols_per_cta;
+    kmax = std::max(kmax, p.k);
+  }
+  void* args[] = {(void*)&b};
+  const dim3 grid(blocks), block(kGatherWarps * 32);
+  const size_t smem = (size_t)(kmax + 256) * mp * sizeof(float);
+  switch (mp) {
+    case 1: return launch_pdl((const void*)k_coeff_gather<1>, grid, block, smem, stream, args);
+    case 2: return launch_pdl((const void*)k_coeff_gather<2>, grid, block, smem, stream, args);
+    case 4: return launch_pdl((const void*)k_coeff_gather<4>, grid, block, smem, stream, args);
+    default: return launch_pdl((const void*)k_coeff_gather<8>, grid, block, smem, stream, args);
+  }
+}
+
+cudaError_t launch_coeff_decode_batch(int n, const dictproj_layer* const* l, const float* const* Zpart,
+                                      const int* nslices, int M, int mp, __half* const* Y, cudaStream_t stream) {
+  bool all_gather = true;
+  for (int i = 0; i < n; ++i) all_gather = all_gather && l[i]->gather_ok;
+  if (all_gather) return launch_gather_batch(n, l, Zpart, nslices, M, mp, Y, stream);
+  for (int i = 0; i < n; ++i) {
+    cudaError_t e = launch_coeff_decode(l[i], Zpart[i], nslices[i], M, mp, Y[i], stream);
+    if (e != cudaSuccess) return e;
+  }
+  return cudaSuccess;
 }
 
 cudaError_t launch_coeff_decode(const dictproj_layer* l, const float* Zpart, int nslices, int M, int mp,
@@ -786,21 +924,7 @@ cudaError_t launch_coeff_decode(const dictproj_layer* l, const float* Zpart, int
   int nseg = l->nseg;
   float s = l->s;
   int k = l->k, d_out = l->d_out;
-  if (l->gather_ok) {
-    const uint32_t* col_ptr = l->col_ptr;
-    int cpc = (d_out + l->n_sm - 1) / l->n_sm;
-    void* args[] = {(void*)&col_ptr, (void*)&codes, (void*)&scales, (void*)&idx, (void*)&ss, (void*)&nseg,
-                    (void*)&s, (void*)&k, (void*)&d_out, (void*)&Zpart, (void*)&nslices, (void*)&M, (void*)&Y,
-                    (void*)&cpc};
-    const dim3 grid((d_out + cpc - 1) / cpc), block(kGatherWarps * 32);
-    const size_t smem = (size_t)(k + 256) * mp * sizeof(float);
-    switch (mp) {
-      case 1: return launch_pdl((const void*)k_coeff_gather<1>, grid, block, smem, stream, args);
-      case 2: return launch_pdl((const void*)k_coeff_gather<2>, grid, block, smem, stream, args);
-      case 4: return launch_pdl((const void*)k_coeff_gather<4>, grid, block, smem, stream, args);
-      default: return launch_pdl((const void*)k_coeff_gather<8>, grid, block, smem, stream, args);
-    }
-  }
+  if (l->gather_ok) return launch_gather_batch(1, &l, &Zpart, &nslices, M, mp, &Y, stream);
   if (l->chunks[0]) {
     const size_t smem = coeff_smem(k, mp);
     // one CTA per SM (half the register file), leaving room for the next call's

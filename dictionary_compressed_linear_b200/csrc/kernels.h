@@ -26,6 +26,12 @@ cudaError_t launch_dict_decode(const dictproj_group* g, const __half* X, int M, 
                                const DictPlan& plan, cudaStream_t stream);
 cudaError_t launch_coeff_decode(const dictproj_layer* l, const float* Zpart, int nslices, int M, int mp,
                                 __half* Y, cudaStream_t stream);
+// Batches of up to 4 independent projections in one launch per stage.
+constexpr int kDecodeMaxBatch = 4;
+cudaError_t launch_dict_decode_batch(int n, const dictproj_group* const* g, const __half* const* X, int M,
+                                     int mp, float* const* Zpart, const DictPlan* plans, cudaStream_t stream);
+cudaError_t launch_coeff_decode_batch(int n, const dictproj_layer* const* l, const float* const* Zpart,
+                                      const int* nslices, int M, int mp, __half* const* Y, cudaStream_t stream);
 
 // Work plan of the chunked coefficient kernel for a grid of G CTAs (host side).
 bool plan_coeff_chunks(const uint32_t* pcol_ptr, int d_out, int nseg, int G, std::vector<uint32_t>& chunks,

@@ -166,6 +166,20 @@ void dictproj_free_layer(dictproj_layer* l); /* NULL is a no-op */
 int dictproj_forward(const void* X, int M, const dictproj_layer* layer,
                      const dictproj_group* group, void* Y, void* stream);
 
+/* Up to DICTPROJ_MAX_BATCH independent projections in one call: projection i
+ * computes Y[i] = X[i] D_g[i] C_l[i] exactly as dictproj_forward would (the same
+ * kernels and arithmetic, so bit-identical results). The projections must be
+ * independent: no Y[i] may be read as an X[j] of the same call; X entries may
+ * alias (e.g. the q, k and v projections of one layer read the same activation);
+ * the groups must be distinct (each call uses its group's Z scratch). For
+ * M <= 8 all projections share one launch per stage, which shortens the chain of
+ * dependent launches a decode step pays; larger M runs them one after another.
+ * Errors as dictproj_forward, plus RANGE (n outside [1, DICTPROJ_MAX_BATCH]) and
+ * MISMATCH (a group repeated or M above some group's max_tokens). */
+#define DICTPROJ_MAX_BATCH 4
+int dictproj_forward_batch(int n, const void* const* X, int M, const dictproj_layer* const* layers,
+                           const dictproj_group* const* groups, void* const* Y, void* stream);
+
 /* Forward with an explicit path: DICTPROJ_PATH_AUTO, DICTPROJ_PATH_DECODE (M <= 8)
  * or DICTPROJ_PATH_PREFILL (any M). Errors as dictproj_forward, plus
  * UNSUPPORTED for DECODE with M > 8. */

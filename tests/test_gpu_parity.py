@@ -204,3 +204,38 @@ def test_chain_of_calls_sharing_a_group():
     assert_parity(y1, oracle_forward(X.cpu().numpy(), pd, pc1, dense=True), "chain 1")
     y2 = Y2.float().cpu().numpy().astype(np.float64)
     assert_parity(y2, oracle_forward(Y1.cpu().numpy(), pd, pc2, dense=True), "chain 2")
+
+
+# ------------------------------------------------------------------ batched forward
+@pytest.mark.parametrize("M", [1, 3, 8, 12])
+def test_batch_matches_single_calls_bitwise(M):
+    shapes = [(512, 256, 300, 0.3), (512, 256, 200, 0.25), (1024, 512, 96, 0.4)]
+    projs = []
+    for i, (d_in, k, d_out, rho) in enumerate(shapes):
+        D = synth.gen_dictionary(16, i, 0, d_in, k)
+        C = synth.gen_coeff(16, i, 0, 0, k, d_out, rho)
+        g, l = device_projection(D, C, max_tokens=16)
+        projs.append((g, l, d_in, d_out))
+    Xs = [torch.from_numpy(synth.gen_activations(16, i, 0, M, d)).cuda() for i, (_, _, d, _) in enumerate(projs)]
+    Xs[1] = Xs[0]  # q/k/v style: two projections read the same activation
+    Ys = [torch.empty((M, do), dtype=torch.float16, device="cuda") for (_, _, _, do) in projs]
+    Yr = [torch.empty((M, do), dtype=torch.float16, device="cuda") for (_, _, _, do) in projs]
+    st = torch.cuda.current_stream().cuda_stream
+    dp.dictproj_forward_batch([x.data_ptr() for x in Xs], M, [p[1] for p in projs], [p[0] for p in projs],
+                              [y.data_ptr() for y in Ys], st)
+    for (g, l, _, _), x, y in zip(projs, Xs, Yr):
+        dp.dictproj_forward(x.data_ptr(), M, l, g, y.data_ptr(), st)
+    torch.cuda.synchronize()
+    for a, b in zip(Ys, Yr):
+        assert torch.equal(a, b)
+
+
+def test_batch_rejects_repeated_group():
+    D = synth.gen_dictionary(17, 0, 0, 64, 32)
+    C = synth.gen_coeff(17, 0, 0, 0, 32, 16, 0.5)
+    g, l = device_projection(D, C, max_tokens=2)
+    X = torch.zeros((1, 64), dtype=torch.float16, device="cuda")
+    Y = torch.zeros((1, 16), dtype=torch.float16, device="cuda")
+    with pytest.raises(dp.DictprojError) as e:
+        dp.dictproj_forward_batch([X.data_ptr()] * 2, 1, [l, l], [g, g], [Y.data_ptr()] * 2, 0)
+    assert e.value.status == -4
