@@ -10,7 +10,8 @@ missing.
 from .binding import (  # noqa: F401
     PATH_AUTO, PATH_DECODE, PATH_PREFILL, DeviceGroup, DeviceLayer, DictprojError, Group, Layer, LIB_PATH,
     SIGNATURES, dictproj_forward_noalloc, dictproj_forward_noalloc_status, lib,
-    dictproj_check, dictproj_coefficient_stage, dictproj_dictionary_stage, dictproj_forward, dictproj_forward_batch, dictproj_forward_path, dictproj_forward_status,
+    dictproj_check, dictproj_coefficient_stage, dictproj_dictionary_stage, dictproj_dictionary_stage_prefill,
+    dictproj_group_reserve_prefill, dictproj_forward, dictproj_forward_batch, dictproj_forward_path, dictproj_forward_status,
     dictproj_group_export, dictproj_group_info, dictproj_group_packed_sizes, dictproj_group_upload,
     dictproj_last_error, dictproj_layer_export, dictproj_layer_info, dictproj_layer_packed_entries,
     dictproj_layer_upload, dictproj_pack, dictproj_pack_group, dictproj_pack_group_host,

@@ -61,6 +61,7 @@ SIGNATURES = [
     ("dictproj_group_upload", C.c_int,
      [_u8p, _u8p, C.c_float, C.c_int, C.c_int, C.c_int, C.POINTER(C.c_void_p)]),
     ("dictproj_pack_group", C.c_int, [_f32p, C.c_int, C.c_int, C.c_int, C.POINTER(C.c_void_p)]),
+    ("dictproj_group_reserve_prefill", C.c_int, [C.c_void_p, C.c_int]),
     ("dictproj_layer_upload", C.c_int,
      [_u32p, _u8p, _u8p, _u8p, _u16p, C.c_float, C.c_int, C.c_int, C.POINTER(C.c_void_p)]),
     ("dictproj_pack_layer", C.c_int, [_i32p, _i32p, _f32p, C.c_int, C.c_int, C.POINTER(C.c_void_p)]),
@@ -81,6 +82,7 @@ SIGNATURES = [
       C.POINTER(C.c_void_p), C.c_void_p]),
     ("dictproj_dictionary_stage", C.c_int, [C.c_void_p, C.c_int, C.c_void_p, C.c_void_p, C.c_void_p]),
     ("dictproj_coefficient_stage", C.c_int, [C.c_void_p, C.c_int, C.c_void_p, C.c_void_p, C.c_void_p]),
+    ("dictproj_dictionary_stage_prefill", C.c_int, [C.c_void_p, C.c_int, C.c_void_p, C.c_void_p, C.c_void_p]),
     ("dictproj_forward_noalloc", C.c_int,
      [C.POINTER(DeviceGroup), C.POINTER(DeviceLayer), C.c_void_p, C.c_int, C.c_void_p, C.c_void_p]),
     ("dictproj_check", C.c_int, [C.c_void_p]),
@@ -333,6 +335,17 @@ def dictproj_forward_batch(X_ptrs, M: int, layers, groups, Y_ptrs, stream: int =
 def dictproj_dictionary_stage(X_ptr: int, M: int, group: Group, Z_ptr: int, stream: int = 0):
     _check(lib().dictproj_dictionary_stage(C.c_void_p(X_ptr), M, group.handle, C.c_void_p(Z_ptr),
                                            C.c_void_p(stream)))
+
+
+def dictproj_dictionary_stage_prefill(X_ptr: int, M: int, group: Group, Z_ptr: int, stream: int = 0):
+    """Z (device fp16 [M][k]) = s_D X D_g on the tensor cores."""
+    _check(lib().dictproj_dictionary_stage_prefill(C.c_void_p(X_ptr), M, group.handle, C.c_void_p(Z_ptr),
+                                                   C.c_void_p(stream)))
+
+
+def dictproj_group_reserve_prefill(group: Group, max_d_out: int):
+    """Reserve the group's prefill coefficient scratch for layers with up to max_d_out columns."""
+    _check(lib().dictproj_group_reserve_prefill(group.handle, max_d_out))
 
 
 def dictproj_coefficient_stage(Z_ptr: int, M: int, layer: Layer, Y_ptr: int, stream: int = 0):

@@ -66,6 +66,7 @@ int ensure_device(int* dev_out) {
       return fail(DICTPROJ_ERR_UNSUPPORTED, "device %d is sm_%d%d; this library is built for sm_100a", dev,
                   prop.major, prop.minor);
     if ((e = prepare_decode_kernels(dev)) != cudaSuccess) return cuda_fail(e, "kernel set-up");
+    if ((e = prepare_prefill_kernels(dev)) != cudaSuccess) return cuda_fail(e, "prefill kernel set-up");
     g_dev_ready[dev] = 1;
   }
   *dev_out = dev;
@@ -138,7 +139,7 @@ void dictproj_free_group(dictproj_group* g) {
   cudaFree(g->scales);
   cudaFree(g->z32);
   cudaFree(g->z16);
-  cudaFree(g->dexp);
+  cudaFree(g->cdense);
   cudaFree(g->err);
   delete g;
 }
@@ -150,7 +151,6 @@ void dictproj_free_layer(dictproj_layer* l) {
   cudaFree(l->scales);
   cudaFree(l->idx);
   cudaFree(l->seg_start);
-  cudaFree(l->cexp);
   for (int i = 0; i < 2; ++i) {
     cudaFree(l->chunks[i]);
     cudaFree(l->cta_ptr[i]);
@@ -185,8 +185,9 @@ int dictproj_group_upload(const uint8_t* codes, const uint8_t* scales, float s_D
   }
   g->zslices = dict_max_slices(d_in, k, g->n_sm);
   const size_t zbytes = (size_t)g->zslices * k * kDecodeMaxTokens * sizeof(float);
+  const size_t z16bytes = (size_t)max_tokens * k * sizeof(uint16_t);
   if ((e = dmalloc((void**)&g->codes, g->codes_bytes)) || (e = dmalloc((void**)&g->scales, g->scales_bytes)) ||
-      (e = dmalloc((void**)&g->z32, zbytes)) ||
+      (e = dmalloc((void**)&g->z32, zbytes)) || (e = dmalloc((void**)&g->z16, z16bytes)) ||
       (e = dmalloc((void**)&g->err, 16))) {
     dictproj_free_group(g);
     cudaGetLastError();
@@ -197,6 +198,10 @@ int dictproj_group_upload(const uint8_t* codes, const uint8_t* scales, float s_D
     dictproj_free_group(g);
     cudaGetLastError();
     return cuda_fail(e, "group_upload: copy to device");
+  }
+  if ((e = encode_dict_codes_map(g, &g->codes_map)) != cudaSuccess) {
+    dictproj_free_group(g);
+    return cuda_fail(e, "group_upload: tensor map of the dictionary codes");
   }
   *out = g;
   return DICTPROJ_OK;
@@ -219,6 +224,32 @@ int dictproj_pack_group(const float* D, int d_in, int k, int max_tokens, dictpro
   float s = 0.f;
   if ((st = pack_group_host(D, d_in, k, codes.data(), scales.data(), &s))) return st;
   return dictproj_group_upload(codes.data(), scales.data(), s, d_in, k, max_tokens, out);
+}
+
+int dictproj_group_reserve_prefill(dictproj_group* g, int max_d_out) {
+  clear_error();
+  if (!g) return fail(DICTPROJ_ERR_NULL, "group_reserve_prefill: NULL handle");
+  if (max_d_out < 1) return fail(DICTPROJ_ERR_RANGE, "group_reserve_prefill: max_d_out=%d < 1", max_d_out);
+  if (max_d_out <= g->cdense_cols) return DICTPROJ_OK;
+  int dev = -1;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "group_reserve_prefill: cudaGetDevice");
+  if (dev != g->device)
+    return fail(DICTPROJ_ERR_MISMATCH, "group_reserve_prefill: current device %d, group on device %d", dev, g->device);
+  uint16_t* p = nullptr;
+  if ((e = dmalloc((void**)&p, (size_t)max_d_out * g->k * sizeof(uint16_t))) != cudaSuccess) {
+    cudaGetLastError();
+    return fail(DICTPROJ_ERR_OOM, "group_reserve_prefill: device allocation failed (%s)", cudaGetErrorName(e));
+  }
+  // the old buffer may still be read by queued work of this group
+  if (g->cdense && (e = cudaDeviceSynchronize()) != cudaSuccess) {
+    cudaFree(p);
+    return cuda_fail(e, "group_reserve_prefill: synchronise before freeing the old scratch");
+  }
+  cudaFree(g->cdense);
+  g->cdense = p;
+  g->cdense_cols = max_d_out;
+  return DICTPROJ_OK;
 }
 
 int dictproj_layer_upload(const uint32_t* pcol_ptr, const uint8_t* codes, const uint8_t* scales,
@@ -367,6 +398,19 @@ int dictproj_pack(const float* D, int d_in, int k, int max_tokens, int n_layers,
       return st;
     }
   }
+  if (max_tokens > kDecodeMaxTokens && n_layers > 0) {  // prefill scratch for these layers
+    int dmax = 0;
+    for (int i = 0; i < n_layers; ++i) dmax = d_out[i] > dmax ? d_out[i] : dmax;
+    if ((st = dictproj_group_reserve_prefill(*group_out, dmax))) {
+      for (int i = 0; i < n_layers; ++i) {
+        dictproj_free_layer(layers_out[i]);
+        layers_out[i] = nullptr;
+      }
+      dictproj_free_group(*group_out);
+      *group_out = nullptr;
+      return st;
+    }
+  }
   return DICTPROJ_OK;
 }
 
@@ -448,17 +492,20 @@ int dictproj_forward_path(const void* X, int M, const dictproj_layer* layer, con
       return cuda_fail(e, "forward: coefficient stage launch");
     return DICTPROJ_OK;
   }
-  // Token chunks of 8 through the decode kernels (prefill path until the
-  // tensor-core kernels take over).
-  for (int m0 = 0; m0 < M; m0 += kDecodeMaxTokens) {
-    const int mc = M - m0 < kDecodeMaxTokens ? M - m0 : kDecodeMaxTokens;
-    const int mp = decode_mp(mc);
-    if ((e = launch_dict_decode(group, x + (size_t)m0 * group->d_in, mc, mp, group->z32, plan, s)) != cudaSuccess)
-      return cuda_fail(e, "forward: dictionary stage launch");
-    if ((e = launch_coeff_decode(layer, group->z32, plan.slices, mc, mp, y + (size_t)m0 * layer->d_out, s)) !=
-        cudaSuccess)
-      return cuda_fail(e, "forward: coefficient stage launch");
-  }
+  // Prefill: Z = s_D X D^ (fp16) and Y = s_C Z C^ as tensor-core GEMMs, C^ densified first.
+  if (layer->d_out > group->cdense_cols)
+    return fail(DICTPROJ_ERR_RANGE,
+                "forward: prefill needs the group's coefficient scratch for d_out=%d (reserved: %d); call "
+                "dictproj_group_reserve_prefill first",
+                layer->d_out, group->cdense_cols);
+  __half* z = reinterpret_cast<__half*>(group->z16);
+  __half* cd = reinterpret_cast<__half*>(group->cdense);
+  if ((e = launch_dict_prefill(group, x, M, z, s)) != cudaSuccess)
+    return cuda_fail(e, "forward: prefill dictionary stage launch");
+  if ((e = launch_densify_coeff(layer, cd, s)) != cudaSuccess)
+    return cuda_fail(e, "forward: prefill coefficient densify launch");
+  if ((e = launch_coeff_prefill(layer, z, cd, M, y, s)) != cudaSuccess)
+    return cuda_fail(e, "forward: prefill coefficient stage launch");
   return DICTPROJ_OK;
 }
 
@@ -531,6 +578,22 @@ int dictproj_dictionary_stage(const void* X, int M, const dictproj_group* group,
   return e == cudaSuccess ? DICTPROJ_OK : cuda_fail(e, "dictionary_stage: launch");
 }
 
+int dictproj_dictionary_stage_prefill(const void* X, int M, const dictproj_group* group, void* Z, void* stream) {
+  clear_error();
+  if (!X || !group || !Z) return fail(DICTPROJ_ERR_NULL, "dictionary_stage_prefill: NULL pointer");
+  if (M < 1) return fail(DICTPROJ_ERR_RANGE, "dictionary_stage_prefill: M=%d < 1", M);
+  if (((uintptr_t)X & 15) || ((uintptr_t)Z & 15))
+    return fail(DICTPROJ_ERR_ALIGN, "dictionary_stage_prefill: X and Z must be 16-byte aligned");
+  int dev = -1;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "dictionary_stage_prefill: cudaGetDevice");
+  if (dev != group->device)
+    return fail(DICTPROJ_ERR_MISMATCH, "dictionary_stage_prefill: current device %d, group on device %d", dev,
+                group->device);
+  e = launch_dict_prefill(group, static_cast<const __half*>(X), M, static_cast<__half*>(Z), (cudaStream_t)stream);
+  return e == cudaSuccess ? DICTPROJ_OK : cuda_fail(e, "dictionary_stage_prefill: launch");
+}
+
 int dictproj_coefficient_stage(const float* Z, int M, const dictproj_layer* layer, void* Y, void* stream) {
   clear_error();
   if (!Z || !layer || !Y) return fail(DICTPROJ_ERR_NULL, "coefficient_stage: NULL pointer");
@@ -547,6 +610,9 @@ int dictproj_check(void* stream) {
   if (e != cudaSuccess) return cuda_fail(e, "check: stream synchronize");
   unsigned int word = 0;
   if ((e = take_decode_error(&word)) != cudaSuccess) return cuda_fail(e, "check: read error word");
+  unsigned int word2 = 0;
+  if ((e = take_prefill_error(&word2)) != cudaSuccess) return cuda_fail(e, "check: read error word");
+  word |= word2;
   if (word) return fail(DICTPROJ_ERR_TIMEOUT, "check: a bounded device wait gave up (error word 0x%x)", word);
   return DICTPROJ_OK;
 }

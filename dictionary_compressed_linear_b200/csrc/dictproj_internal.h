@@ -4,6 +4,7 @@
 #include <cstddef>
 #include <cstdint>
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include "dictproj.h"
@@ -46,9 +47,11 @@ struct dictproj_group {
   // scratch
   float* z32;              // decode Z partial sums, fp32 [zslices][k][8]
   int zslices;             // d_in slices of the decode dictionary stage
-  uint16_t* z16;           // prefill Z, fp16 [max_tokens][k] (allocated when max_tokens > 8)
-  uint16_t* dexp;          // prefill: D expanded to fp16, atom-major [k][d_in]
+  uint16_t* z16;           // prefill Z, fp16 [max_tokens][k]
+  uint16_t* cdense;        // prefill coefficient operand, fp16 [d_out][k] for d_out <= cdense_cols
+  int cdense_cols;         // reserved output columns (dictproj_group_reserve_prefill)
   unsigned int* err;       // device error word for bounded waits
+  CUtensorMap codes_map;   // TMA map of codes: [k] rows x [d_in/2] bytes, box 32 x 256
 };
 
 struct dictproj_layer {
@@ -62,7 +65,6 @@ struct dictproj_layer {
   uint8_t* scales;         // [total/16]
   uint8_t* idx;            // [total]
   uint16_t* seg_start;     // [d_out][nseg]
-  uint16_t* cexp;          // prefill: C expanded to fp16, [d_out][k] (lazy)
   // decode-path work plan (see plan_coeff_chunks): chunk {o_b, o_e, e_b, e_e}
   // plan[0]: one CTA per SM; plan[1]: two CTAs per SM (used when two fit)
   uint32_t* chunks[2];     // [n_chunks][4], device; NULL -> direct kernel

@@ -42,4 +42,19 @@ bool gather_supported(const uint32_t* pcol_ptr, int d_out, int nseg);
 // Read and clear the device error word of the decode kernels.
 cudaError_t take_decode_error(unsigned int* out);
 
+// prefill path (any M; used for M > 8): tcgen05 GEMMs, Z fp16 [M][k]
+cudaError_t prepare_prefill_kernels(int device);
+cudaError_t encode_dict_codes_map(const dictproj_group* g, CUtensorMap* map);
+// Tile width (multiple of 16, <= 256) for `extent` elements split into tiles,
+// `other` tiles along the other side, n_sm SMs (prefill GEMM grids).
+int prefill_tile_width(long extent, long other, int n_sm);
+// Z = s_D X D^ (fp16 out, s_D applied in fp32 before rounding)
+cudaError_t launch_dict_prefill(const dictproj_group* g, const __half* X, int M, __half* Z, cudaStream_t stream);
+// Cd[o][a] = C^ densified to fp16 (zeros off the support), [d_out][k]
+cudaError_t launch_densify_coeff(const dictproj_layer* l, __half* Cd, cudaStream_t stream);
+// Y = s_C Z Cd^T
+cudaError_t launch_coeff_prefill(const dictproj_layer* l, const __half* Z, const __half* Cd, int M, __half* Y,
+                                 cudaStream_t stream);
+cudaError_t take_prefill_error(unsigned int* out);
+
 }  // namespace dictproj

@@ -1,0 +1,605 @@
+// Prefill path (M > 8 tokens): both stages of Y = (X·D_g)·C_l as tcgen05 GEMMs.
+//
+// At prefill the dictionary stage Z = X·D_g is a dense contraction with about
+// 2·M·d_in·k flops on d_in·k·9/16 bytes of packed dictionary, far above the
+// HBM ridge, so it runs on the 5th-generation tensor cores (DictLLM technical
+// review, Eq. (1) and "Efficiency" section; the compressed factors replace one
+// d_in x d_out product by a d_in x k product and a sparse k x d_out one).
+//
+//   k_prefill_gemm<true>   Z[M][k]   = s_D · X[M][d_in] · D^[d_in][k]
+//       A = X tile (128 tokens x 64 d_in, fp16) by TMA with 128-byte swizzle;
+//       B = 256 atoms x 64 d_in: the packed E2M1 codes arrive by TMA, eight
+//       producer warps decode them (E2M1 x E4M3 block scale, exact in fp16)
+//       straight into the swizzled K-major fp16 operand tile; one thread issues
+//       tcgen05.mma (M=128, N=256, K=16, fp32 accumulate in tensor memory).
+//       The epilogue applies s_D in fp32 before rounding Z to fp16 (the
+//       unscaled sum can exceed the fp16 range).
+//   k_densify_coeff         Cd[d_out][k] = C^ (fp16, zeros off the support)
+//   k_prefill_gemm<false>  Y[M][d_out] = s_C · Z[M][k] · Cd^T, both operands by
+//       TMA. At prefill the tensor cores run the zeros of C faster than CUDA
+//       cores run only its nonzeros (dense fp16 rate / fp32 FMA rate >> 1/rho).
+//
+// Every spin-wait is bounded; a wait that gives up sets bit 0 of the device
+// error word and the kernel unwinds (frees its tensor memory) without hanging.
+#include <cuda.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <mutex>
+
+#include "common.cuh"
+#include "dictproj_internal.h"
+#include "kernels.h"
+
+namespace dictproj {
+namespace {
+
+constexpr int BM = 128;                 // tokens per tile (MMA M, tensor-memory lanes)
+constexpr int BN = 256;                 // atoms / output columns per tile (MMA N)
+constexpr int BK = 64;                  // reduction elements per stage (one 128-byte swizzle row)
+constexpr int STAGES = 4;
+constexpr int A_BYTES = BM * BK * 2;    // 16 KB
+constexpr int B_BYTES = BN * BK * 2;    // 32 KB
+constexpr int kTA = 128;                // atoms per dictionary-stage tile (MMA M)
+constexpr int kGemmThreads = 320;       // warp 0 TMA, warp 1 MMA + TMEM, warps 2..9 producers/epilogue
+constexpr int kProducerWarps = 8;
+constexpr int kTmemCols = 256;          // fp32 accumulator: 128 lanes x 256 columns
+constexpr int kScaleAhead = 4;          // block-scale look-ahead, in stages of one producer group
+
+constexpr size_t kGemmSmem = (size_t)STAGES * (A_BYTES + B_BYTES) + 1024 + 256;
+
+// ---- tcgen05 / TMA primitives ------------------------------------------------------
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int x, int y, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];"
+      ::"r"(dst), "l"(map), "r"(x), "r"(y), "r"(smem_u32(bar))
+      : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+__device__ __forceinline__ void tc_fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_alloc(uint32_t* slot, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(slot)),
+               "r"(ncols)
+               : "memory");
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+// Shared-memory matrix descriptor: K-major operand, 128-byte swizzle, rows of
+// 128 bytes, 8-row groups 1024 bytes apart (stride byte offset), version 1.
+__device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t addr) {
+  return (uint64_t)((addr >> 4) & 0x3FFF) | (1ull << 16) | ((uint64_t)(1024 >> 4) << 32) | (1ull << 46) |
+         (2ull << 61);
+}
+// D (tensor memory) (+)= A (shared memory) x B (shared memory)
+__device__ __forceinline__ void mma_f16_ss(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                           uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+// D (tensor memory) (+)= A (tensor memory: lane = row, two fp16 per column) x B (shared memory)
+__device__ __forceinline__ void mma_f16_ts(uint32_t tmem_d, uint32_t tmem_a, uint64_t bdesc, uint32_t idesc,
+                                           uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(tmem_d),
+      "r"(tmem_a), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+// 16 consecutive 32-bit columns of this thread's lane; waits for completion.
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&v)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(taddr),
+      "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]), "r"(v[8]),
+      "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15])
+      : "memory");
+  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void mma_commit(uint64_t* bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
+               : "memory");
+}
+// 32 consecutive fp32 accumulator columns of this thread's lane.
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&v)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]),
+        "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15]),
+        "=r"(v[16]), "=r"(v[17]), "=r"(v[18]), "=r"(v[19]), "=r"(v[20]), "=r"(v[21]), "=r"(v[22]), "=r"(v[23]),
+        "=r"(v[24]), "=r"(v[25]), "=r"(v[26]), "=r"(v[27]), "=r"(v[28]), "=r"(v[29]), "=r"(v[30]), "=r"(v[31])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void sts_v4(uint32_t a, uint32_t x, uint32_t y, uint32_t z, uint32_t w) {
+  asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(a), "r"(x), "r"(y), "r"(z), "r"(w) : "memory");
+}
+__device__ __forceinline__ uint32_t pack_h2(float a, float b) {
+  __half2 h = __floats2half2_rn(a, b);
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+
+
+// One 128 x 256 output tile of out = scale · A · B^T with A (M x K) and B
+// (N x K) fp16 K-major, both brought by TMA with 128-byte swizzle; one thread
+// issues tcgen05.mma (M=128, N=256, K=16) into a fp32 accumulator in tensor
+// memory; eight warps run the epilogue.
+__global__ void __launch_bounds__(kGemmThreads, 1)
+    k_gemm_tma(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b, int M, int N,
+               int K, int bn, float scale, __half* __restrict__ out) {
+  extern __shared__ uint8_t smem_raw[];
+  // 128-byte swizzled operand tiles must start on 1024-byte shared-memory boundaries
+  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+  uint8_t* sa = smem;
+  uint8_t* sb = sa + STAGES * A_BYTES;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sb + STAGES * B_BYTES);
+  uint64_t* full = bars;               // TMA bytes of the stage landed
+  uint64_t* empty = bars + STAGES;     // MMAs of the stage completed
+  uint64_t* accf = bars + 2 * STAGES;  // accumulator complete
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accf + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int n0 = blockIdx.x * bn, m0 = blockIdx.y * BM;
+  const int nk = (K + BK - 1) / BK;
+  // kind::f16, A and B fp16, D fp32, K-major, M = 128, N = bn
+  const uint32_t idesc = (1u << 4) | ((uint32_t)(bn >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    mbar_init(accf, 1);
+    fence_mbar_init();
+  }
+  if (warp == 1) tmem_alloc(tmem_slot, kTmemCols);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  // A and B may be the previous kernels' output; nothing below reads or writes
+  // global memory before this point.
+  grid_dependency_wait();
+
+  if (warp == 0) {
+    if (lane == 0) {  // TMA producer
+      for (int s = 0; s < nk; ++s) {
+        const int slot = s % STAGES, round = s / STAGES;
+        if (s >= STAGES && !mbar_wait_bounded(&empty[slot], (round - 1) & 1)) break;
+        mbar_arrive_expect_tx(&full[slot], A_BYTES + bn * BK * 2);
+        tma_load_2d(smem_u32(sa + slot * A_BYTES), &tm_a, s * BK, m0, &full[slot]);
+        tma_load_2d(smem_u32(sb + slot * B_BYTES), &tm_b, s * BK, n0, &full[slot]);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {  // MMA issuer
+      for (int s = 0; s < nk; ++s) {
+        const int slot = s % STAGES, round = s / STAGES;
+        if (!mbar_wait_bounded(&full[slot], round & 1)) break;
+        tc_fence_after();
+        const uint32_t a = smem_u32(sa + slot * A_BYTES), b = smem_u32(sb + slot * B_BYTES);
+#pragma unroll
+        for (int j = 0; j < BK / 16; ++j)
+          mma_f16_ss(tmem, smem_desc_sw128(a + 32 * j), smem_desc_sw128(b + 32 * j), idesc, (s | j) != 0);
+        mma_commit(&empty[slot]);
+      }
+      mma_commit(accf);
+    }
+  } else {
+    // Epilogue: warp w reads tensor-memory lanes 32·(w % 4) .. +31 (its tokens)
+    // and every other 32-column chunk of the bn accumulator columns.
+    const int q = warp & 3, half = (warp - 2) >> 2;
+    const bool ok = mbar_wait_bounded(accf, 0);
+    tc_fence_after();
+    const int row = m0 + 32 * q + lane;
+    const bool vec = (N & 7) == 0;
+    const int nlim = min(N, n0 + bn);
+#pragma unroll 1
+    for (int c = half; 32 * c < bn; c += 2) {
+      const int col = 32 * c;
+      uint32_t v[32];
+      tmem_ld32(tmem + ((uint32_t)(32 * q) << 16) + col, v);
+      if (!ok || row >= M) continue;
+      __half* orow = out + (size_t)row * N;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int gc = n0 + col + 8 * j;
+        if (gc >= nlim) break;
+        float f[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) f[e] = __uint_as_float(v[8 * j + e]) * scale;
+        if (vec) {
+          uint4 o;
+          o.x = pack_h2(f[0], f[1]);
+          o.y = pack_h2(f[2], f[3]);
+          o.z = pack_h2(f[4], f[5]);
+          o.w = pack_h2(f[6], f[7]);
+          *reinterpret_cast<uint4*>(orow + gc) = o;
+        } else {
+          for (int e = 0; e < 8 && gc + e < nlim; ++e) orow[gc + e] = __float2half_rn(f[e]);
+        }
+      }
+    }
+  }
+  __syncwarp();
+  trigger_dependents();
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+// ---- dictionary stage: Z^T tile = D^T tile (tensor memory) x X tile (shared memory) -------------
+// The 128 atoms of a tile are the MMA's M rows: producer warps decode their
+// NVFP4 codes into fp16 and store them straight into tensor memory (operand A
+// of tcgen05.mma .kind::f16 with A in tensor memory), so the decoded
+// dictionary never passes through shared memory; only X (operand B, nt tokens
+// x 64) and the packed codes do. The accumulator holds Z^T (atoms x tokens).
+// The token-tile width nt (a multiple of 16, at most 256) is chosen per call so
+// that the tiles fill whole waves of the GPU.
+struct DictTile {
+  // Two producer groups of 8 warps take alternate stages, so that the latency of
+  // one stage's decode (shared-memory load, conversion, tensor-memory store and
+  // its wait) overlaps the next one's.
+  static constexpr int kGroups = 2;
+  static constexpr int kThreads = 64 + 32 * 8 * kGroups;
+  static constexpr int kMaxN = 256;
+  static constexpr int kStages = 6;
+  static constexpr int kXBytes = kMaxN * BK * 2;    // X tile slot: up to 256 tokens x 64 fp16
+  static constexpr int kRawBytes = kTA * BK / 2;    // codes: 128 atoms x 32 bytes
+  static constexpr int kAcol = kMaxN;               // first tensor-memory column of the A ring
+  static constexpr int kCols = 512;                 // accumulator + 32 per stage, rounded up
+  static_assert(kMaxN + 32 * kStages <= kCols, "tensor memory");
+  static constexpr size_t smem = (size_t)kStages * (kXBytes + kRawBytes) + 1024 + 256;
+};
+
+__global__ void __launch_bounds__(DictTile::kThreads, 1)
+    k_dict_prefill(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_codes,
+                   const uint8_t* __restrict__ scales, int M, int k, int d_in, int nt, float s_D,
+                   __half* __restrict__ Z) {
+  using T = DictTile;
+  constexpr int S = T::kStages;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+  uint8_t* sx = smem;
+  uint8_t* sr = sx + S * T::kXBytes;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sr + S * T::kRawBytes);
+  uint64_t* full = bars;           // X tile and codes of the stage landed
+  uint64_t* afull = bars + S;      // producers stored the decoded A slice in tensor memory
+  uint64_t* empty = bars + 2 * S;  // MMAs of the stage completed
+  uint64_t* accf = bars + 3 * S;   // accumulator complete
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accf + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int a0 = blockIdx.x * kTA, m0 = blockIdx.y * nt;
+  const int nk = (d_in + BK - 1) / BK;
+  // kind::f16, A and B fp16, D fp32, K-major, M = 128 atoms, N = nt tokens
+  const uint32_t idesc = (1u << 4) | ((uint32_t)(nt >> 3) << 17) | ((uint32_t)(kTA >> 4) << 24);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&afull[s], kProducerWarps);
+      mbar_init(&empty[s], 1);
+    }
+    mbar_init(accf, 1);
+    fence_mbar_init();
+  }
+  if (warp == 1) tmem_alloc(tmem_slot, T::kCols);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  grid_dependency_wait();  // X may be the previous kernel's output
+
+  if (warp == 0) {
+    if (lane == 0) {  // TMA producer: X tile and packed codes per stage
+      for (int s = 0; s < nk; ++s) {
+        const int slot = s % S, round = s / S;
+        if (s >= S && !mbar_wait_bounded(&empty[slot], (round - 1) & 1)) break;
+        mbar_arrive_expect_tx(&full[slot], nt * BK * 2 + T::kRawBytes);
+        tma_load_2d(smem_u32(sx + slot * T::kXBytes), &tm_x, s * BK, m0, &full[slot]);
+        tma_load_2d(smem_u32(sr + slot * T::kRawBytes), &tm_codes, s * (BK / 2), a0, &full[slot]);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {  // MMA issuer
+      for (int s = 0; s < nk; ++s) {
+        const int slot = s % S, round = s / S;
+        if (!mbar_wait_bounded(&full[slot], round & 1)) break;
+        if (!mbar_wait_bounded(&afull[slot], round & 1)) break;
+        tc_fence_after();
+        const uint32_t x = smem_u32(sx + slot * T::kXBytes);
+        const uint32_t a = tmem + T::kAcol + 32 * slot;
+#pragma unroll
+        for (int j = 0; j < BK / 16; ++j) mma_f16_ts(tmem, a + 8 * j, smem_desc_sw128(x + 32 * j), idesc, (s | j) != 0);
+        mma_commit(&empty[slot]);
+      }
+      mma_commit(accf);
+    }
+  } else {
+    // Warp w owns tensor-memory lanes 32·(w % 4) .. +31 (atoms a0 + that), half
+    // h of each stage's 64 reduction elements, and the stages s = g (mod groups).
+    const int e = warp - 2, g = e >> 3;
+    const int q = warp & 3, h = (e >> 2) & 1;
+    const int r = 32 * q + lane;
+    const bool row_ok = a0 + r < k;
+    const int nblk = d_in / 16;  // even
+    const uint8_t* srow = scales + (size_t)(row_ok ? a0 + r : 0) * nblk + 2 * h;
+    const uint32_t lane_base = (uint32_t)(32 * q) << 16;
+    // Two E4M3 block scales per stage (blocks 4s + 2h, +1) travel in a register
+    // ring loaded kScaleAhead of this group's stages ahead of use. The ring is
+    // indexed statically (the loop over it is unrolled): moving a register whose
+    // load is still in flight would wait for that load.
+    constexpr int G = T::kGroups, R = kScaleAhead;
+    auto scale_at = [&](int st) -> uint32_t {
+      return (row_ok && 4 * st + 2 * h < nblk) ? ld_stream_u16(srow + 4 * st) : 0u;
+    };
+    uint32_t scr[R];
+#pragma unroll
+    for (int i = 0; i < R; ++i) scr[i] = scale_at(g + G * i);
+    bool live = true;
+    for (int base = g; live && base < nk; base += G * R) {
+#pragma unroll
+      for (int i = 0; i < R; ++i) {
+        const int s = base + G * i;
+        if (!live || s >= nk) break;
+        const int slot = s % S, round = s / S;
+        const uint32_t sc = scr[i];
+        scr[i] = scale_at(s + G * R);
+        if (!mbar_wait_bounded(&full[slot], round & 1)) {
+          live = false;
+          break;
+        }
+        const uint4 c = lds_u32x4(smem_u32(sr + slot * T::kRawBytes) + r * 32 + 16 * h);
+        const uint32_t w[4] = {c.x, c.y, c.z, c.w};
+        const uint32_t hs = e4m3x2_to_f16x2(sc);
+        const uint32_t scl[2] = {dup_lo(hs), dup_hi(hs)};
+        uint32_t o[16];
+#pragma unroll
+        for (int cc = 0; cc < 4; ++cc) {
+          uint32_t f[4];
+          e2m1x8_to_f16x2x4(w[cc], f);
+#pragma unroll
+          for (int t = 0; t < 4; ++t) o[4 * cc + t] = hmul2_u32(f[t], scl[cc >> 1]);
+        }
+        tmem_st16(tmem + lane_base + T::kAcol + 32 * slot + 16 * h, o);
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&afull[slot]);
+      }
+    }
+    // Epilogue: Z[m][a0 + r]; the 32-token column chunks of the accumulator go
+    // round-robin to the 2·groups warps of each lane quadrant.
+    const bool ok = mbar_wait_bounded(accf, 0);
+    tc_fence_after();
+    const int lim = min(nt, M - m0);  // valid token columns of this tile
+#pragma unroll 1
+    for (int c = e >> 2; 32 * c < nt; c += 2 * G) {
+      const int col = 32 * c;
+      uint32_t v[32];
+      tmem_ld32(tmem + lane_base + col, v);
+      if (!ok || !row_ok) continue;
+      __half* zc = Z + (size_t)(m0 + col) * k + a0 + r;
+#pragma unroll
+      for (int j = 0; j < 32; ++j)
+        if (col + j < lim) zc[(size_t)j * k] = __float2half_rn(__uint_as_float(v[j]) * s_D);
+    }
+  }
+  __syncwarp();
+  trigger_dependents();
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, T::kCols);
+  }
+}
+
+// Dense fp16 copy of C^ (atom-major rows per output column: Cd[o][a]), zeros off
+// the support. One warp per column builds the row in shared memory, then writes
+// it out with 16-byte stores. Entries with code 0 (value 0, and the padding at
+// the end of each column) are skipped.
+__global__ void __launch_bounds__(256)
+    k_densify_coeff(const uint32_t* __restrict__ col_ptr, const uint8_t* __restrict__ codes,
+                    const uint8_t* __restrict__ scales, const uint8_t* __restrict__ idx,
+                    const uint16_t* __restrict__ seg_start, int k, int d_out, int nseg, __half* __restrict__ cd) {
+  extern __shared__ __align__(16) uint8_t dsm[];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int o = blockIdx.x * (blockDim.x >> 5) + warp;
+  grid_dependency_wait();  // Cd may still be read by the previous coefficient GEMM
+  if (o >= d_out) return;
+  __half* row = reinterpret_cast<__half*>(dsm) + (size_t)warp * k;
+  const uint32_t rbase = smem_u32(row);
+  for (int c = lane; c < k / 8; c += 32) sts_v4(rbase + 16 * c, 0, 0, 0, 0);
+  __syncwarp();
+  const uint32_t e0 = col_ptr[o], e1 = col_ptr[o + 1];
+  const uint16_t* ss = seg_start + (size_t)o * nseg;
+  int seg = 0;
+  for (uint32_t e = e0 + lane; e < e1; e += 32) {
+    const uint32_t q = e - e0;
+    while (seg + 1 < nseg && ss[seg + 1] <= q) ++seg;
+    const uint32_t byte = codes[e >> 1];
+    const uint32_t code = (e & 1) ? (byte >> 4) : (byte & 15);
+    if ((code & 7) == 0) continue;  // +-0
+    const uint32_t atom = 256u * seg + idx[e];
+    const uint32_t v = e2m1x2_to_f16x2(code);  // low half: the value
+    const uint32_t sc = e4m3x2_to_f16x2(scales[e >> 4]);
+    const uint32_t prod = hmul2_u32(v, sc);
+    asm volatile("st.shared.u16 [%0], %1;" ::"r"(rbase + 2 * atom), "h"((unsigned short)(prod & 0xFFFF))
+                 : "memory");
+  }
+  __syncwarp();
+  uint4* dst = reinterpret_cast<uint4*>(cd + (size_t)o * k);
+  for (int c = lane; c < k / 8; c += 32) dst[c] = lds_u32x4(rbase + 16 * c);
+}
+
+// ---- host side ---------------------------------------------------------------------------
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static std::mutex g_enc_mu;
+static EncodeTiledFn g_encode = nullptr;
+
+static cudaError_t get_encoder(EncodeTiledFn* fn) {
+  std::lock_guard<std::mutex> lk(g_enc_mu);
+  if (!g_encode) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    cudaError_t e = cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q);
+    if (e != cudaSuccess) return e;
+    if (q != cudaDriverEntryPointSuccess || !p) return cudaErrorNotSupported;
+    g_encode = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  *fn = g_encode;
+  return cudaSuccess;
+}
+
+// 2-D row-major map: rows x inner elements, row stride in bytes, box inner x rows.
+static cudaError_t encode_2d(CUtensorMap* map, CUtensorMapDataType type, const void* base, uint64_t inner,
+                             uint64_t rows, uint64_t row_bytes, uint32_t box_inner, uint32_t box_rows,
+                             CUtensorMapSwizzle swz) {
+  EncodeTiledFn enc;
+  cudaError_t e = get_encoder(&enc);
+  if (e != cudaSuccess) return e;
+  const cuuint64_t gdim[2] = {inner, rows};
+  const cuuint64_t gstride[1] = {row_bytes};
+  const cuuint32_t box[2] = {box_inner, box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  const CUresult r = enc(map, type, 2, const_cast<void*>(base), gdim, gstride, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                         swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+static cudaLaunchAttribute pdl_attr() {
+  cudaLaunchAttribute a;
+  a.id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  a.val.programmaticStreamSerializationAllowed = 1;
+  return a;
+}
+
+}  // namespace
+
+cudaError_t prepare_prefill_kernels(int device) {
+  (void)device;
+  cudaError_t e;
+  if ((e = cudaFuncSetAttribute(k_gemm_tma, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kGemmSmem)) ||
+      (e = cudaFuncSetAttribute(k_dict_prefill, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                (int)DictTile::smem)))
+    return e;
+  return cudaFuncSetAttribute(k_densify_coeff, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
+}
+
+cudaError_t take_prefill_error(unsigned int* out) {
+  unsigned int zero = 0;
+  cudaError_t e = cudaMemcpyFromSymbol(out, g_dictproj_error, sizeof(unsigned int));
+  if (e != cudaSuccess) return e;
+  return cudaMemcpyToSymbol(g_dictproj_error, &zero, sizeof(unsigned int));
+}
+
+cudaError_t encode_dict_codes_map(const dictproj_group* g, CUtensorMap* map) {
+  return encode_2d(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, g->codes, (uint64_t)g->d_in / 2, (uint64_t)g->k,
+                   (uint64_t)g->d_in / 2, BK / 2, kTA, CU_TENSOR_MAP_SWIZZLE_NONE);
+}
+
+// Width w (a multiple of 16, at most 256) of the tiles that split `extent`
+// elements, with `other` tiles along the other side: fewest padded columns per SM
+// over the waves the grid takes, counting each tile's fixed per-stage cost as 32
+// columns.
+int prefill_tile_width(long extent, long other, int n_sm) {
+  int best = 256;
+  double best_cost = 1e300;
+  for (long t = (extent + 255) / 256; t <= (extent + 15) / 16; ++t) {
+    const long w = ((extent + t - 1) / t + 15) / 16 * 16;
+    const long tiles = other * ((extent + w - 1) / w);
+    const long waves = (tiles + n_sm - 1) / n_sm;
+    const double cost = (double)waves * (double)(w + 32);
+    if (cost < best_cost) {
+      best_cost = cost;
+      best = (int)w;
+    }
+  }
+  return best;
+}
+
+cudaError_t launch_dict_prefill(const dictproj_group* g, const __half* X, int M, __half* Z, cudaStream_t stream) {
+  int nt = prefill_tile_width(M, (g->k + kTA - 1) / kTA, g->n_sm);
+  CUtensorMap tx;
+  cudaError_t e = encode_2d(&tx, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, X, (uint64_t)g->d_in, (uint64_t)M,
+                            (uint64_t)g->d_in * 2, BK, nt, CU_TENSOR_MAP_SWIZZLE_128B);
+  if (e != cudaSuccess) return e;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((g->k + kTA - 1) / kTA, (M + nt - 1) / nt);
+  cfg.blockDim = dim3(DictTile::kThreads);
+  cfg.dynamicSmemBytes = DictTile::smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1] = {pdl_attr()};
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const uint8_t* sc = g->scales;
+  int k = g->k, d_in = g->d_in;
+  float s = g->s;
+  void* args[] = {(void*)&tx, (void*)&g->codes_map, (void*)&sc, &M, &k, &d_in, &nt, &s, (void*)&Z};
+  return cudaLaunchKernelExC(&cfg, (const void*)k_dict_prefill, args);
+}
+
+cudaError_t launch_densify_coeff(const dictproj_layer* l, __half* Cd, cudaStream_t stream) {
+  const int warps = std::max(1, std::min(8, (int)((200 * 1024) / ((size_t)l->k * 2))));
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((l->d_out + warps - 1) / warps);
+  cfg.blockDim = dim3(32 * warps);
+  cfg.dynamicSmemBytes = (size_t)warps * l->k * 2;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1] = {pdl_attr()};
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int k = l->k, d_out = l->d_out, nseg = l->nseg;
+  void* args[] = {(void*)&l->col_ptr, (void*)&l->codes, (void*)&l->scales, (void*)&l->idx, (void*)&l->seg_start,
+                  &k, &d_out, &nseg, (void*)&Cd};
+  return cudaLaunchKernelExC(&cfg, (const void*)k_densify_coeff, args);
+}
+
+cudaError_t launch_coeff_prefill(const dictproj_layer* l, const __half* Z, const __half* Cd, int M, __half* Y,
+                                 cudaStream_t stream) {
+  CUtensorMap ta, tb;
+  cudaError_t e = encode_2d(&ta, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, Z, (uint64_t)l->k, (uint64_t)M,
+                            (uint64_t)l->k * 2, BK, BM, CU_TENSOR_MAP_SWIZZLE_128B);
+  if (e != cudaSuccess) return e;
+  int bn = prefill_tile_width(l->d_out, (M + BM - 1) / BM, l->n_sm);
+  e = encode_2d(&tb, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, Cd, (uint64_t)l->k, (uint64_t)l->d_out, (uint64_t)l->k * 2, BK,
+                bn, CU_TENSOR_MAP_SWIZZLE_128B);
+  if (e != cudaSuccess) return e;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((l->d_out + bn - 1) / bn, (M + BM - 1) / BM);
+  cfg.blockDim = dim3(kGemmThreads);
+  cfg.dynamicSmemBytes = kGemmSmem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1] = {pdl_attr()};
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int N = l->d_out, K = l->k;
+  float s = l->s;
+  void* args[] = {(void*)&ta, (void*)&tb, &M, &N, &K, &bn, &s, (void*)&Y};
+  return cudaLaunchKernelExC(&cfg, (const void*)k_gemm_tma, args);
+}
+
+}  // namespace dictproj

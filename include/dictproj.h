@@ -119,6 +119,15 @@ int dictproj_group_upload(const uint8_t* codes, const uint8_t* scales, float s_D
 /* dictproj_pack_group_host + dictproj_group_upload. */
 int dictproj_pack_group(const float* D, int d_in, int k, int max_tokens, dictproj_group** out);
 
+/* Reserve the group's prefill coefficient scratch for layers with up to max_d_out
+ * output columns: fp16 [max_d_out][k], the densified C_l that the prefill
+ * coefficient GEMM reads (2 * k * max_d_out bytes). Forwards with M > 8 (or
+ * DICTPROJ_PATH_PREFILL) need it and fail with RANGE before any launch without
+ * it, so that they never allocate. Growing an existing reservation synchronises
+ * the device first. dictproj_pack reserves for its layers when max_tokens > 8.
+ * Errors: NULL, RANGE (max_d_out < 1), MISMATCH (device), OOM, CUDA. */
+int dictproj_group_reserve_prefill(dictproj_group* g, int max_d_out);
+
 /* Upload an already packed C_l. Errors: NULL, SHAPE, CUDA, OOM. */
 int dictproj_layer_upload(const uint32_t* pcol_ptr, const uint8_t* codes, const uint8_t* scales,
                           const uint8_t* idx, const uint16_t* seg_start, float s_C, int k,
@@ -155,8 +164,10 @@ void dictproj_free_layer(dictproj_layer* l); /* NULL is a no-op */
 
 /* Y = X * (D_g) * (C_l) (Eq. (1)): X device fp16 [M][d_in] row-major, Y device
  * fp16 [M][d_out] row-major, both 16-byte aligned; 1 <= M <= group max_tokens.
- * Accumulation is fp32; Z is fp32 for M <= 8 (decode path) and fp16 with s_D
- * applied before rounding for larger M (prefill path).
+ * Accumulation is fp32; Z is fp32 for M <= 8 (decode path: CUDA-core GEMV and
+ * sparse gather) and fp16 with s_D applied before rounding for larger M (prefill
+ * path: tcgen05 GEMM on the dequantised dictionary, then the densified C_l as a
+ * second tcgen05 GEMM; needs dictproj_group_reserve_prefill for d_out).
  * Asynchronous on `stream`: no allocation, no host synchronisation. Kernels are
  * launched with programmatic dependent launch; each kernel waits for the
  * preceding work on the stream before it reads X or writes Z / Y (packed
@@ -195,6 +206,13 @@ int dictproj_forward_path(const void* X, int M, const dictproj_layer* layer,
  * Same validation, ordering and asynchrony as dictproj_forward; UNSUPPORTED for M > 8. */
 int dictproj_dictionary_stage(const void* X, int M, const dictproj_group* group, float* Z, void* stream);
 int dictproj_coefficient_stage(const float* Z, int M, const dictproj_layer* layer, void* Y, void* stream);
+
+/* The prefill dictionary stage alone (any M >= 1): Z = s_D * X * D_g on tcgen05
+ * tensor cores (fp16 operands, fp32 accumulation, s_D applied in fp32, then
+ * rounded to fp16). X device fp16 [M][d_in], Z caller-owned device fp16 [M][k],
+ * both 16-byte aligned. Same ordering and asynchrony as dictproj_forward.
+ * Errors: NULL, RANGE (M < 1), ALIGN, MISMATCH (device), CUDA. */
+int dictproj_dictionary_stage_prefill(const void* X, int M, const dictproj_group* group, void* Z, void* stream);
 
 /* ------------------------------------------------------------------------- */
 /* Forward without allocation                                                 */

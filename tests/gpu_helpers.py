@@ -12,6 +12,7 @@ def device_projection(D, C, max_tokens):
     """(group, layer) on the GPU via the library's packer."""
     g = dp.dictproj_pack_group(D, max_tokens)
     l = dp.dictproj_pack_layer(C.col_ptr, C.atom_idx, C.vals, C.k, C.d_out)
+    dp.dictproj_group_reserve_prefill(g, C.d_out)
     return g, l
 
 
