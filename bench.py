@@ -69,25 +69,99 @@ def measured_peaks():
     return FALLBACK_HBM_GBS, "fallback"
 
 
-def kernel_source_hash():
+def measured_tensor_peak():
+    """Dense fp16 tensor-core peak in TFLOP/s: the measured bf16 burst figure (fp16
+    and bf16 dense MMA have the same rate), else the fallback."""
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        if "bf16_tflops" in d:
+            return float(d["bf16_tflops"]), "measured (MEASURED_PEAKS.json bf16_tflops; fp16 dense rate is the same)"
+    return 1590.0, "fallback 1590 TFLOP/s"
+
+
+def kernel_source_hash(files=("decode.cu", "common.cuh")):
     h = hashlib.sha256()
-    for fn in ("decode.cu", "common.cuh"):
+    for fn in files:
         with open(os.path.join(ROOT, "dictionary_compressed_linear_b200", "csrc", fn), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
 
 
-def profiled_traffic(kernel_name):
-    """DRAM bytes per launch from the committed ncu summary, if the kernel is unchanged."""
+def profiled(kernel_name, key="bytes_per_launch"):
+    """A figure from the committed ncu summary (profiles/traffic.json), if the
+    kernel's source is unchanged since it was taken."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(path):
         return None
     with open(path) as f:
         d = json.load(f)
     e = d.get(kernel_name)
-    if not e or e.get("source_hash") != kernel_source_hash():
+    if not e:
         return None
-    return e.get("bytes_per_launch")
+    files = tuple(e.get("source_files", ["decode.cu", "common.cuh"]))
+    if e.get("source_hash") != kernel_source_hash(files):
+        return None
+    return e.get(key)
+
+
+def profiled_traffic(kernel_name, algorithmic_bytes):
+    """DRAM bytes of one launch: the measured DRAM / algorithmic byte ratio of the
+    ncu capture, scaled to this launch's algorithmic bytes (traffic grows in
+    proportion to the packed bytes a launch streams)."""
+    r = profiled(kernel_name, "traffic_ratio")
+    return None if r is None else int(round(r * algorithmic_bytes))
+
+
+# ----------------------------------------------------------------------------- prefill leg
+PREFILL_SHAPES = ("q", "gate", "down")
+
+
+def prefill_bench(torch, dp, stream, M=2048, reps=20):
+    """Prefill (M tokens) of one projection of each LLaMA-7B shape class: the
+    dictionary stage alone (tcgen05, the tensor-bound step) and the whole forward,
+    timed with CUDA events over graphs of `reps` calls alternating two weight sets
+    (C density 0.3, 1% of input channels x20, as in the prefill workload)."""
+    sh = stream.cuda_stream
+    peak, peak_src = measured_tensor_peak()
+    out = {"workload": f"prefill M={M}: q (4096->4096, k=2048), gate (4096->11008, k=3072), "
+                       "down (11008->4096, k=3072); C density 0.3; X fp16 N(0,1), 1% channels x20",
+           "peak_tflops": peak, "peak_source": peak_src, "shapes": {}}
+    for name in PREFILL_SHAPES:
+        d_in, d_out, k = synth.LLAMA7B_SHAPES[name]
+        pt = synth.PROJ_TYPES.index(name)
+        D = synth.gen_dictionary(4, 0, pt, d_in, k)
+        C = synth.gen_coeff(4, 0, pt, 0, k, d_out, 0.3)
+        pg = dp.dictproj_pack_group_host(D)
+        pc = dp.dictproj_pack_layer_host(C.col_ptr, C.atom_idx, C.vals, k, d_out)
+        gs = [dp.dictproj_group_upload(pg, M) for _ in range(2)]
+        for g in gs:
+            dp.dictproj_group_reserve_prefill(g, d_out)
+        ls = [dp.dictproj_layer_upload(pc) for _ in range(2)]
+        X = torch.from_numpy(synth.gen_activations(4, 0, synth.INPUT_SITE[name], M, d_in, 0.01)).cuda()
+        Z = torch.empty((M, k), dtype=torch.float16, device="cuda")
+        Y = torch.empty((M, d_out), dtype=torch.float16, device="cuda")
+        res = {}
+        for what in ("dictionary_stage", "forward"):
+            def chain():
+                for i in range(reps):
+                    if what == "dictionary_stage":
+                        dp.dictproj_dictionary_stage_prefill(X.data_ptr(), M, gs[i % 2], Z.data_ptr(), sh)
+                    else:
+                        dp.dictproj_forward(X.data_ptr(), M, ls[i % 2], gs[i % 2], Y.data_ptr(), sh)
+            g = capture(torch, stream, chain)
+            time_replays(torch, stream, g, 3)
+            ms = time_replays(torch, stream, g, 5) / (5 * reps)
+            del g
+            flops = 2.0 * M * d_in * k + (2.0 * M * k * d_out if what == "forward" else 0.0)
+            tf = flops / (ms / 1e3) / 1e12
+            res[what] = {"us": round(ms * 1e3, 2), "TFLOP/s": round(tf, 1), "frac": round(tf / peak, 4),
+                         "flops": flops}
+        res["dictionary_stage"]["tensor_pipe_util_ncu"] = profiled(f"k_dict_prefill:{name}", "tensor_util")
+        out["shapes"][name] = res
+        del gs, ls
+    return out
 
 
 # ----------------------------------------------------------------------------- clocks
@@ -354,6 +428,7 @@ def main():
     ap.add_argument("--layers", type=int, default=32)
     ap.add_argument("--stage-reps", type=int, default=50)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-prefill", action="store_true", help="skip the prefill (M=2048) leg")
     ap.add_argument("--no-batch", action="store_true",
                     help="one dictproj_forward per projection instead of batching q/k/v and gate/up")
     args = ap.parse_args()
@@ -456,17 +531,22 @@ def main():
     gbs_c = bytes_c / (ms_c / args.stage_reps / 1e3) / 1e9
     peak, peak_kind = measured_peaks()
     if ms_c >= ms_d:
-        dom, dom_name, gbs, per_launch, bytes_l = "coefficient stage", "k_coeff_decode", gbs_c, per_launch_c, bytes_c / n_launch
+        dom, dom_name, gbs, per_launch, bytes_l = "coefficient stage", "k_coeff_gather", gbs_c, per_launch_c, bytes_c / n_launch
     else:
         dom, dom_name, gbs, per_launch, bytes_l = "dictionary stage", "k_dict_decode", gbs_d, per_launch_d, bytes_d / n_launch
     roofline = {"bound": "hbm", "achieved": round(gbs, 1), "peak": peak, "unit": "GB/s",
-                "frac": round(gbs / peak, 4), "traffic": profiled_traffic(dom_name),
+                "frac": round(gbs / peak, 4), "traffic": profiled_traffic(dom_name, bytes_l),
                 "kernel": dom_name, "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)" if peak_kind == "measured" else "fallback 6650 GB/s",
                 "avg_launch_us": round(per_launch * 1e3, 3), "algorithmic_bytes_per_launch": int(bytes_l),
                 "stages": {"k_dict_decode": {"GB/s": round(gbs_d, 1), "avg_launch_us": round(per_launch_d * 1e3, 3),
-                                             "frac": round(gbs_d / peak, 4), "traffic": profiled_traffic("k_dict_decode")},
-                           "k_coeff_decode": {"GB/s": round(gbs_c, 1), "avg_launch_us": round(per_launch_c * 1e3, 3),
-                                              "frac": round(gbs_c / peak, 4), "traffic": profiled_traffic("k_coeff_decode")}}}
+                                             "frac": round(gbs_d / peak, 4),
+                                             "traffic": profiled_traffic("k_dict_decode", bytes_d / n_launch)},
+                           "k_coeff_gather": {"GB/s": round(gbs_c, 1), "avg_launch_us": round(per_launch_c * 1e3, 3),
+                                              "frac": round(gbs_c / peak, 4),
+                                              "traffic": profiled_traffic("k_coeff_gather", bytes_c / n_launch)}},
+                "timing": "each stage alone: a CUDA graph of the 224 stage calls of one step (dictionary stage "
+                          "with its Z written complete in one slice; coefficient stage reading it), CUDA events "
+                          "on the launching stream"}
 
     # ---------------- step-level accounting
     step_bytes = sum(d_bytes(p) + c_bytes(p) + 2 * M * (p.d_in + p.d_out) for p in wl.projections)
@@ -491,6 +571,12 @@ def main():
     if dist:
         dist.all_reduce(t_e, op=dist.ReduceOp.MAX)
     e2e_value = world * M * e2e_steps / (float(t_e.item()) / 1e3)
+
+    prefill = None
+    if not args.no_prefill:
+        del stack
+        torch.cuda.empty_cache()
+        prefill = prefill_bench(torch, dp, stream)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -521,6 +607,7 @@ def main():
                  "frac_of_peak": round(step_gbs / peak, 4),
                  "algorithmic_bytes_dictionary_once_per_group": step_bytes_once,
                  "GB/s_dictionary_once_per_group": round(step_bytes_once / (ms_per_step / 1e3) / 1e9, 1)},
+        "prefill": prefill,
     }
     if rank == 0:
         print(json.dumps(line), flush=True)
