@@ -114,6 +114,25 @@ def profiled_traffic(kernel_name, algorithmic_bytes):
     return None if r is None else int(round(r * algorithmic_bytes))
 
 
+# ----------------------------------------------------------------------------- ranks
+def max_over_ranks(value, dist, device):
+    """The largest `value` over all ranks (every rank gets it); `value` when there
+    is no process group. Rank timings are combined this way: the job takes as
+    long as its slowest replica."""
+    if dist is None:
+        return float(value)
+    import torch
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def replica_throughput(tokens_per_rank, world, ms):
+    """Whole-job tokens/s of `world` independent replicas that took `ms` (the
+    max over ranks) for `tokens_per_rank` tokens each."""
+    return world * tokens_per_rank / (ms / 1e3)
+
+
 # ----------------------------------------------------------------------------- prefill leg
 PREFILL_SHAPES = ("q", "gate", "down")
 
@@ -485,13 +504,9 @@ def main():
     if dist:
         dist.barrier()
     clocks = sampler.stop()
-    t_ms = torch.tensor([ms], device="cuda")
-    if dist:
-        dist.all_reduce(t_ms, op=dist.ReduceOp.MAX)
-    ms = float(t_ms.item())
+    ms = max_over_ranks(ms, dist, "cuda")
     ms_per_step = ms / args.steps
-    tokens = world * M * args.steps
-    value = tokens / (ms / 1e3)
+    value = replica_throughput(M * args.steps, world, ms)
     launches_per_step = 2 * calls_per_step
     # the same step with one call per projection, for comparison
     ms_unbatched = None
@@ -567,10 +582,7 @@ def main():
 
     time_replays(torch, stream, graph, 3, pre, post)
     ms_e2e = time_replays(torch, stream, graph, e2e_steps, pre, post)
-    t_e = torch.tensor([ms_e2e], device="cuda")
-    if dist:
-        dist.all_reduce(t_e, op=dist.ReduceOp.MAX)
-    e2e_value = world * M * e2e_steps / (float(t_e.item()) / 1e3)
+    e2e_value = replica_throughput(M * e2e_steps, world, max_over_ranks(ms_e2e, dist, "cuda"))
 
     prefill = None
     if not args.no_prefill:

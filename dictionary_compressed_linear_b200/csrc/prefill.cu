@@ -416,36 +416,63 @@ __global__ void __launch_bounds__(DictTile::kThreads, 1)
 
 // Dense fp16 copy of C^ (atom-major rows per output column: Cd[o][a]), zeros off
 // the support. One warp per column builds the row in shared memory, then writes
-// it out with 16-byte stores. Entries with code 0 (value 0, and the padding at
-// the end of each column) are skipped.
+// it out with 16-byte stores. A lane takes 4 consecutive stored entries per
+// 128-entry chunk (one 4-byte index load, one 2-byte code load, one scale byte:
+// columns are padded to multiples of 16 entries, so the loads are aligned), and
+// the next chunk's loads are issued before the current one is scattered.
+// Entries with code 0 (value 0, and the padding at the end of each column) are
+// skipped. The column's segment starts sit in shared memory.
 __global__ void __launch_bounds__(256)
     k_densify_coeff(const uint32_t* __restrict__ col_ptr, const uint8_t* __restrict__ codes,
                     const uint8_t* __restrict__ scales, const uint8_t* __restrict__ idx,
                     const uint16_t* __restrict__ seg_start, int k, int d_out, int nseg, __half* __restrict__ cd) {
   extern __shared__ __align__(16) uint8_t dsm[];
+  const int nw = blockDim.x >> 5;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int o = blockIdx.x * (blockDim.x >> 5) + warp;
+  const int o = blockIdx.x * nw + warp;
   grid_dependency_wait();  // Cd may still be read by the previous coefficient GEMM
   if (o >= d_out) return;
   __half* row = reinterpret_cast<__half*>(dsm) + (size_t)warp * k;
+  uint16_t* ss = reinterpret_cast<uint16_t*>(dsm + (size_t)nw * k * 2) + (size_t)warp * nseg;
   const uint32_t rbase = smem_u32(row);
   for (int c = lane; c < k / 8; c += 32) sts_v4(rbase + 16 * c, 0, 0, 0, 0);
+  for (int j = lane; j < nseg; j += 32) ss[j] = seg_start[(size_t)o * nseg + j];
   __syncwarp();
   const uint32_t e0 = col_ptr[o], e1 = col_ptr[o + 1];
-  const uint16_t* ss = seg_start + (size_t)o * nseg;
-  int seg = 0;
-  for (uint32_t e = e0 + lane; e < e1; e += 32) {
-    const uint32_t q = e - e0;
-    while (seg + 1 < nseg && ss[seg + 1] <= q) ++seg;
-    const uint32_t byte = codes[e >> 1];
-    const uint32_t code = (e & 1) ? (byte >> 4) : (byte & 15);
-    if ((code & 7) == 0) continue;  // +-0
-    const uint32_t atom = 256u * seg + idx[e];
-    const uint32_t v = e2m1x2_to_f16x2(code);  // low half: the value
-    const uint32_t sc = e4m3x2_to_f16x2(scales[e >> 4]);
-    const uint32_t prod = hmul2_u32(v, sc);
-    asm volatile("st.shared.u16 [%0], %1;" ::"r"(rbase + 2 * atom), "h"((unsigned short)(prod & 0xFFFF))
-                 : "memory");
+  int seg = 0;  // segment of this lane's entries; they only increase
+  uint32_t i4 = 0, c4 = 0, sc = 0;
+  {
+    const uint32_t e = e0 + 4 * lane;
+    if (e < e1) {
+      i4 = *reinterpret_cast<const uint32_t*>(idx + e);
+      c4 = *reinterpret_cast<const uint16_t*>(codes + (e >> 1));
+      sc = scales[e >> 4];
+    }
+  }
+  for (uint32_t base = e0; base < e1; base += 128) {
+    const uint32_t e = base + 4 * lane, en = e + 128;
+    uint32_t ni4 = 0, nc4 = 0, nsc = 0;  // next chunk, loaded before this one is scattered
+    if (en < e1) {
+      ni4 = *reinterpret_cast<const uint32_t*>(idx + en);
+      nc4 = *reinterpret_cast<const uint16_t*>(codes + (en >> 1));
+      nsc = scales[en >> 4];
+    }
+    if (e < e1) {
+      const uint32_t sv = e4m3x2_to_f16x2(sc) & 0xFFFF;
+#pragma unroll
+      for (int t = 0; t < 4; ++t) {
+        const uint32_t code = (c4 >> (4 * t)) & 15;
+        if ((code & 7) == 0) continue;  // +-0 and padding
+        const int q = (int)(e - e0) + t;
+        while (seg + 1 < nseg && (int)ss[seg + 1] <= q) ++seg;
+        const uint32_t atom = 256u * seg + ((i4 >> (8 * t)) & 255);
+        const uint32_t prod = hmul2_u32(e2m1x2_to_f16x2(code), sv);  // exact in fp16
+        row[atom] = __ushort_as_half((unsigned short)(prod & 0xFFFF));
+      }
+    }
+    i4 = ni4;
+    c4 = nc4;
+    sc = nsc;
   }
   __syncwarp();
   uint4* dst = reinterpret_cast<uint4*>(cd + (size_t)o * k);
@@ -563,11 +590,12 @@ cudaError_t launch_dict_prefill(const dictproj_group* g, const __half* X, int M,
 }
 
 cudaError_t launch_densify_coeff(const dictproj_layer* l, __half* Cd, cudaStream_t stream) {
-  const int warps = std::max(1, std::min(8, (int)((200 * 1024) / ((size_t)l->k * 2))));
+  const size_t per_warp = (size_t)l->k * 2 + (size_t)l->nseg * 2;
+  const int warps = std::max(1, std::min(8, (int)((200 * 1024) / per_warp)));
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((l->d_out + warps - 1) / warps);
   cfg.blockDim = dim3(32 * warps);
-  cfg.dynamicSmemBytes = (size_t)warps * l->k * 2;
+  cfg.dynamicSmemBytes = (size_t)warps * per_warp;
   cfg.stream = stream;
   cudaLaunchAttribute attr[1] = {pdl_attr()};
   cfg.attrs = attr;
