@@ -20,7 +20,7 @@ STATUS = {
     0: "DICTPROJ_OK", -1: "DICTPROJ_ERR_NULL", -2: "DICTPROJ_ERR_SHAPE", -3: "DICTPROJ_ERR_ALIGN",
     -4: "DICTPROJ_ERR_MISMATCH", -5: "DICTPROJ_ERR_RANGE", -6: "DICTPROJ_ERR_CUDA",
     -7: "DICTPROJ_ERR_OOM", -8: "DICTPROJ_ERR_TIMEOUT", -9: "DICTPROJ_ERR_UNSUPPORTED",
-    -10: "DICTPROJ_ERR_VALUE",
+    -10: "DICTPROJ_ERR_VALUE", -11: "DICTPROJ_ERR_IO",
 }
 PATH_AUTO, PATH_DECODE, PATH_PREFILL = 0, 1, 2
 
@@ -85,6 +85,20 @@ SIGNATURES = [
     ("dictproj_dictionary_stage_prefill", C.c_int, [C.c_void_p, C.c_int, C.c_void_p, C.c_void_p, C.c_void_p]),
     ("dictproj_forward_noalloc", C.c_int,
      [C.POINTER(DeviceGroup), C.POINTER(DeviceLayer), C.c_void_p, C.c_int, C.c_void_p, C.c_void_p]),
+    ("dictproj_rank_for_budget", C.c_int, [C.c_double, C.c_int, C.c_int, C.c_int, C.c_int, _intp]),
+    ("dictproj_budget", C.c_int, [C.c_int, C.c_int, C.c_int, C.c_int, C.c_double, C.POINTER(C.c_double),
+                                  C.POINTER(C.c_double), C.POINTER(C.c_double), C.POINTER(C.c_double)]),
+    ("dictproj_group_file_write", C.c_int, [C.c_char_p, _u8p, _u8p, C.c_float, C.c_int, C.c_int]),
+    ("dictproj_group_file_info", C.c_int, [C.c_char_p, _intp, _intp]),
+    ("dictproj_group_file_read", C.c_int, [C.c_char_p, _u8p, _u8p, _f32p, C.c_int, C.c_int]),
+    ("dictproj_layer_file_write", C.c_int, [C.c_char_p, _u32p, _u8p, _u8p, _u8p, _u16p, C.c_float, C.c_int, C.c_int]),
+    ("dictproj_layer_file_info", C.c_int, [C.c_char_p, _intp, _intp, _szp]),
+    ("dictproj_layer_file_read", C.c_int,
+     [C.c_char_p, _u32p, _u8p, _u8p, _u8p, _u16p, _f32p, C.c_int, C.c_int, C.c_size_t]),
+    ("dictproj_group_save", C.c_int, [C.c_void_p, C.c_char_p]),
+    ("dictproj_group_load", C.c_int, [C.c_char_p, C.c_int, C.POINTER(C.c_void_p)]),
+    ("dictproj_layer_save", C.c_int, [C.c_void_p, C.c_char_p]),
+    ("dictproj_layer_load", C.c_int, [C.c_char_p, C.POINTER(C.c_void_p)]),
     ("dictproj_check", C.c_int, [C.c_void_p]),
     ("dictproj_last_error", C.c_char_p, []),
     ("dictproj_status_string", C.c_char_p, [C.c_int]),
@@ -176,6 +190,65 @@ def dictproj_pack_layer_host(col_ptr, atom_idx, vals, k: int, d_out: int) -> dic
         _ptr(out["scales"], C.c_uint8), _ptr(out["idx"], C.c_uint8), _ptr(out["seg_start"], C.c_uint16),
         C.byref(s)))
     out.update(k=k, d_out=d_out, nseg=nseg, s=np.float32(s.value))
+    return out
+
+
+# ---------------------------------------------------------------- budget and packed files
+def dictproj_rank_for_budget(rho_fac: float, n: int, d_in: int, d_out: int, align: int = 1) -> int:
+    """Eq. (3): dictionary rank for a factorisation reduction rho_fac, rounded down to `align`."""
+    k = C.c_int()
+    _check(lib().dictproj_rank_for_budget(float(rho_fac), n, d_in, d_out, align, C.byref(k)))
+    return k.value
+
+
+def dictproj_budget(n: int, d_in: int, d_out: int, k: int, p: float) -> dict:
+    """Eq. (2): N0, Np, rho, G."""
+    v = [C.c_double() for _ in range(4)]
+    _check(lib().dictproj_budget(n, d_in, d_out, k, float(p), *[C.byref(x) for x in v]))
+    return dict(zip(("N0", "Np", "rho", "G"), [x.value for x in v]))
+
+
+def dictproj_group_file_write(path: str, packed: dict):
+    codes = np.ascontiguousarray(packed["codes"], np.uint8)
+    scales = np.ascontiguousarray(packed["scales"], np.uint8)
+    _check(lib().dictproj_group_file_write(os.fsencode(path), _ptr(codes, C.c_uint8), _ptr(scales, C.c_uint8),
+                                           float(packed["s"]), packed["d_in"], packed["k"]))
+
+
+def dictproj_group_file_read(path: str) -> dict:
+    d_in, k = C.c_int(), C.c_int()
+    _check(lib().dictproj_group_file_info(os.fsencode(path), C.byref(d_in), C.byref(k)))
+    out = {"codes": np.zeros(d_in.value * k.value // 2, np.uint8),
+           "scales": np.zeros(d_in.value * k.value // 16, np.uint8)}
+    s = C.c_float()
+    _check(lib().dictproj_group_file_read(os.fsencode(path), _ptr(out["codes"], C.c_uint8),
+                                          _ptr(out["scales"], C.c_uint8), C.byref(s), d_in.value, k.value))
+    out.update(d_in=d_in.value, k=k.value, s=np.float32(s.value))
+    return out
+
+
+def dictproj_layer_file_write(path: str, packed: dict):
+    a = {n: np.ascontiguousarray(packed[n]) for n in ("col_ptr", "codes", "scales", "idx", "seg_start")}
+    _check(lib().dictproj_layer_file_write(os.fsencode(path), _ptr(a["col_ptr"], C.c_uint32),
+                                           _ptr(a["codes"], C.c_uint8), _ptr(a["scales"], C.c_uint8),
+                                           _ptr(a["idx"], C.c_uint8), _ptr(a["seg_start"], C.c_uint16),
+                                           float(packed["s"]), packed["k"], packed["d_out"]))
+
+
+def dictproj_layer_file_read(path: str) -> dict:
+    k, d_out, total = C.c_int(), C.c_int(), C.c_size_t()
+    _check(lib().dictproj_layer_file_info(os.fsencode(path), C.byref(k), C.byref(d_out), C.byref(total)))
+    K, O, T = k.value, d_out.value, total.value
+    nseg = -(-K // 256)
+    out = {"col_ptr": np.zeros(O + 1, np.uint32), "codes": np.zeros(T // 2, np.uint8),
+           "scales": np.zeros(T // 16, np.uint8), "idx": np.zeros(T, np.uint8),
+           "seg_start": np.zeros(O * nseg, np.uint16)}
+    s = C.c_float()
+    _check(lib().dictproj_layer_file_read(os.fsencode(path), _ptr(out["col_ptr"], C.c_uint32),
+                                          _ptr(out["codes"], C.c_uint8), _ptr(out["scales"], C.c_uint8),
+                                          _ptr(out["idx"], C.c_uint8), _ptr(out["seg_start"], C.c_uint16),
+                                          C.byref(s), K, O, T))
+    out.update(k=K, d_out=O, nseg=nseg, s=np.float32(s.value))
     return out
 
 
@@ -330,6 +403,30 @@ def dictproj_forward_batch(X_ptrs, M: int, layers, groups, Y_ptrs, stream: int =
     arr = lambda vals: (C.c_void_p * n)(*[C.c_void_p(v) for v in vals])
     _check(lib().dictproj_forward_batch(n, arr(X_ptrs), M, arr([l.handle for l in layers]),
                                         arr([g.handle for g in groups]), arr(Y_ptrs), C.c_void_p(stream)))
+
+
+def dictproj_group_save(group: "Group", path: str):
+    _check(lib().dictproj_group_save(group.handle, os.fsencode(path)))
+
+
+def dictproj_group_load(path: str, max_tokens: int) -> "Group":
+    h = C.c_void_p()
+    _check(lib().dictproj_group_load(os.fsencode(path), max_tokens, C.byref(h)))
+    d_in, k, mt = C.c_int(), C.c_int(), C.c_int()
+    _check(lib().dictproj_group_info(h.value, C.byref(d_in), C.byref(k), C.byref(mt)))
+    return Group(h.value, d_in.value, k.value, mt.value)
+
+
+def dictproj_layer_save(layer: "Layer", path: str):
+    _check(lib().dictproj_layer_save(layer.handle, os.fsencode(path)))
+
+
+def dictproj_layer_load(path: str) -> "Layer":
+    h = C.c_void_p()
+    _check(lib().dictproj_layer_load(os.fsencode(path), C.byref(h)))
+    k, d_out = C.c_int(), C.c_int()
+    _check(lib().dictproj_layer_info(h.value, C.byref(k), C.byref(d_out), None, None))
+    return Layer(h.value, k.value, d_out.value)
 
 
 def dictproj_dictionary_stage(X_ptr: int, M: int, group: Group, Z_ptr: int, stream: int = 0):

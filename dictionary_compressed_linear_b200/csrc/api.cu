@@ -101,6 +101,7 @@ const char* dictproj_status_string(int s) {
     case DICTPROJ_ERR_TIMEOUT: return "DICTPROJ_ERR_TIMEOUT";
     case DICTPROJ_ERR_UNSUPPORTED: return "DICTPROJ_ERR_UNSUPPORTED";
     case DICTPROJ_ERR_VALUE: return "DICTPROJ_ERR_VALUE";
+    case DICTPROJ_ERR_IO: return "DICTPROJ_ERR_IO";
     default: return "DICTPROJ_ERR_UNKNOWN";
   }
 }

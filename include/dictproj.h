@@ -71,7 +71,8 @@ typedef enum dictproj_status {
   DICTPROJ_ERR_OOM = -7,         /* device or host allocation failed */
   DICTPROJ_ERR_TIMEOUT = -8,     /* a bounded device-side wait gave up (read by dictproj_check) */
   DICTPROJ_ERR_UNSUPPORTED = -9, /* valid but not supported here (e.g. not an sm_100 device) */
-  DICTPROJ_ERR_VALUE = -10       /* a non-finite input value */
+  DICTPROJ_ERR_VALUE = -10,      /* a non-finite input value; a corrupt packed file */
+  DICTPROJ_ERR_IO = -11          /* a file could not be opened, read or written */
 } dictproj_status;
 
 /* Opaque handles. A group owns the packed D_g on the device plus the scratch for
@@ -254,6 +255,52 @@ typedef struct dictproj_device_layer {
  * 16-byte aligned. Errors: NULL, SHAPE, MISMATCH, RANGE, ALIGN, VALUE, CUDA. */
 int dictproj_forward_noalloc(const dictproj_device_group* group, const dictproj_device_layer* layer,
                              const void* X, int M, void* Y, void* stream);
+
+/* ------------------------------------------------------------------------- */
+/* Budget helpers and packed-file export (host only, no device needed)        */
+/* ------------------------------------------------------------------------- */
+
+/* Rank of a group's dictionary for a factorisation budget, Eq. (3) of the
+ * DictLLM technical review ("The budget: trading shared rank against
+ * sparsity"): k = floor((1 - rho_fac) n d_in d_out / (d_in + n d_out)) for n
+ * layers of shape d_in x d_out, rounded down to a multiple of `align` (1 for
+ * the plain equation; 16 for the kernels here, which need k % 16 == 0).
+ * Errors: NULL, SHAPE (n, d_in, d_out, align < 1), RANGE (rho_fac outside
+ * [0, 1), or no rank left). */
+int dictproj_rank_for_budget(double rho_fac, int n, int d_in, int d_out, int align, int* k_out);
+
+/* Value counts of Eq. (2) of the review: N0 = n d_in d_out, Np = d_in k +
+ * n (1 - p) k d_out, rho = 1 - Np / N0, G = N0 / Np (p = fraction of the
+ * coefficients pruned). Any output may be NULL. Errors: SHAPE, RANGE (p). */
+int dictproj_budget(int n, int d_in, int d_out, int k, double p, double* N0, double* Np, double* rho, double* G);
+
+/* Packed-file export and import of one group (D_g) or one layer (C_l): the
+ * export step of the review's Algorithm 2 ("dictionary, per-layer codes, scales
+ * and support"). A file holds exactly the packed arrays of
+ * dictproj_pack_group_host / dictproj_pack_layer_host behind a 64-byte header
+ * (magic, shapes, the fp32 tensor scale, payload size, FNV-1a 64 checksum),
+ * little-endian. *_info reads the shapes so that the caller can size buffers;
+ * *_read checks magic, shapes against the caller's, sizes and the checksum.
+ * Errors: NULL, SHAPE, RANGE (bad layout on write), VALUE (non-finite scale;
+ * corrupt, truncated or foreign file), MISMATCH (buffer shapes), IO. */
+int dictproj_group_file_write(const char* path, const uint8_t* codes, const uint8_t* scales, float s_D, int d_in,
+                              int k);
+int dictproj_group_file_info(const char* path, int* d_in, int* k);
+int dictproj_group_file_read(const char* path, uint8_t* codes, uint8_t* scales, float* s_D, int d_in, int k);
+int dictproj_layer_file_write(const char* path, const uint32_t* pcol_ptr, const uint8_t* codes, const uint8_t* scales,
+                              const uint8_t* idx, const uint16_t* seg_start, float s_C, int k, int d_out);
+int dictproj_layer_file_info(const char* path, int* k, int* d_out, size_t* total_entries);
+int dictproj_layer_file_read(const char* path, uint32_t* pcol_ptr, uint8_t* codes, uint8_t* scales, uint8_t* idx,
+                             uint16_t* seg_start, float* s_C, int k, int d_out, size_t total_entries);
+
+/* Device handles to and from packed files: *_save exports the handle's packed
+ * bytes (dictproj_*_export) and writes them; *_load reads a file and uploads it
+ * (dictproj_group_upload / dictproj_layer_upload, which validate the layout).
+ * Errors: those of the calls they compose. */
+int dictproj_group_save(const dictproj_group* g, const char* path);
+int dictproj_group_load(const char* path, int max_tokens, dictproj_group** out);
+int dictproj_layer_save(const dictproj_layer* l, const char* path);
+int dictproj_layer_load(const char* path, dictproj_layer** out);
 
 /* Read (and clear) the device error word that bounded device waits set, after
  * synchronising `stream`. Returns OK or TIMEOUT (or CUDA). */

@@ -124,3 +124,21 @@ def test_pack_convenience_all_or_nothing():
     with pytest.raises(dp.DictprojError):
         dp.dictproj_pack(D, 2, [(good.col_ptr, good.atom_idx, good.vals, 8),
                                 (np.array([0, 1]), np.array([99]), np.ones(1, np.float32), 1)])
+
+
+def test_save_and_load_handles_through_files(tmp_path):
+    D, C = synth.gen_dictionary(0, 0, 0, 512, 256), synth.gen_coeff(0, 0, 0, 0, 256, 384, 0.3)
+    g = dp.dictproj_pack_group(D, 8)
+    l = dp.dictproj_pack_layer(C.col_ptr, C.atom_idx, C.vals, 256, 384)
+    dp.dictproj_group_save(g, str(tmp_path / "g.dpj"))
+    dp.dictproj_layer_save(l, str(tmp_path / "l.dpj"))
+    g2 = dp.dictproj_group_load(str(tmp_path / "g.dpj"), 8)
+    l2 = dp.dictproj_layer_load(str(tmp_path / "l.dpj"))
+    X = torch.from_numpy(synth.gen_activations(0, 0, 0, 3, 512)).cuda()
+    st = torch.cuda.current_stream().cuda_stream
+    Y1 = torch.empty((3, 384), dtype=torch.float16, device="cuda")
+    Y2 = torch.full((3, 384), float("nan"), dtype=torch.float16, device="cuda")
+    dp.dictproj_forward(X.data_ptr(), 3, l, g, Y1.data_ptr(), st)
+    dp.dictproj_forward(X.data_ptr(), 3, l2, g2, Y2.data_ptr(), st)
+    torch.cuda.synchronize()
+    assert torch.equal(Y1, Y2)

@@ -46,6 +46,9 @@ def test_version_and_status_strings(dp):
     assert dp.dictproj_version() >= 10000
     assert dp.dictproj_status_string(0) == "DICTPROJ_OK"
     assert dp.dictproj_status_string(-8) == "DICTPROJ_ERR_TIMEOUT"
+    from dictionary_compressed_linear_b200.binding import STATUS
+    for code, name in STATUS.items():
+        assert dp.dictproj_status_string(code) == name
 
 
 def _same_layer(a, b):
