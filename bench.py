@@ -81,11 +81,20 @@ def measured_tensor_peak():
     return 1590.0, "fallback 1590 TFLOP/s"
 
 
-def kernel_source_hash(files=("decode.cu", "common.cuh")):
+def kernel_source_hash(files=("decode.cu", "common.cuh"), region=None):
+    """sha256 prefix of the kernel sources; `region` = (start marker, end marker)
+    restricts the first file to the text between them (one kernel of a file)."""
     h = hashlib.sha256()
-    for fn in files:
+    for i, fn in enumerate(files):
         with open(os.path.join(ROOT, "dictionary_compressed_linear_b200", "csrc", fn), "rb") as f:
-            h.update(f.read())
+            data = f.read()
+        if region and i == 0:
+            a = data.find(region[0].encode())
+            b = data.find(region[1].encode(), a + 1)
+            if a < 0 or b < 0:
+                return None
+            data = data[a:b]
+        h.update(data)
     return h.hexdigest()[:16]
 
 
@@ -101,7 +110,8 @@ def profiled(kernel_name, key="bytes_per_launch"):
     if not e:
         return None
     files = tuple(e.get("source_files", ["decode.cu", "common.cuh"]))
-    if e.get("source_hash") != kernel_source_hash(files):
+    region = tuple(e["source_region"]) if e.get("source_region") else None
+    if e.get("source_hash") != kernel_source_hash(files, region):
         return None
     return e.get(key)
 

@@ -530,6 +530,102 @@ __device__ __forceinline__ void load_col(ColData& d, int o, int d_out, const uin
   }
 }
 
+// One column of the gather: Y[m][o] = s_C * sum over the column's stored
+// entries of Z[m][atom] * value (d holds the column's entries, loaded earlier).
+template <int MP>
+__device__ __forceinline__ void gather_column(const ColData& d, int o, int nhb, uint32_t zs_a, int nseg,
+                                              const uint16_t* __restrict__ seg_start, int lane, int M, int d_out,
+                                              float s_C, __half* __restrict__ Y) {
+  constexpr uint32_t kRow = MP * 4;
+    float acc[MP];
+#pragma unroll
+  for (int m = 0; m < MP; ++m) acc[m] = 0.f;
+  // Lane j holds seg_start[j] (the first entry of segment j). For the window of
+  // 256 entries starting at w, a boundary b in (w, w+256) lies at the start of
+  // lane p = (b-w)/8's half-block when (b-w) % 8 == 0, else inside it; two
+  // OR-reduced lane masks give every lane its segment with two popcounts.
+  const bool is_bnd = lane >= 1 && lane < nseg;
+#pragma unroll
+  for (int i = 0; i < kRmax; ++i) {
+    const int w = 256 * i;
+    if (w >= 8 * nhb) break;
+    const int b = d.ssv;  // boundary held by this lane (meaningful iff is_bnd)
+    const int s_lo = __popc(__ballot_sync(0xffffffffu, is_bnd && b <= w));  // segment of entry w
+    const bool in_win = is_bnd && b > w && b < w + 256;
+    const int rel = b - w;
+    const uint32_t at_start = (in_win && (rel & 7) == 0) ? (1u << (rel >> 3)) : 0u;
+    const uint32_t inside = (in_win && (rel & 7) != 0) ? (1u << (rel >> 3)) : 0u;
+    const uint32_t A = __reduce_or_sync(0xffffffffu, at_start);
+    const uint32_t B = __reduce_or_sync(0xffffffffu, inside);
+    const int nwin = __popc(__ballot_sync(0xffffffffu, in_win));
+    const bool collide = nwin != __popc(A) + __popc(B) || (A & B) != 0u;  // two boundaries in one half-block
+    const uint32_t le = lane == 31 ? 0xffffffffu : ((2u << lane) - 1u);
+    const int before = __popc(A & le) + __popc(B & (le >> 1));  // boundaries <= q0 in the window
+    const int sgi = s_lo + before;                               // segment of q0
+    const int q0 = w + 8 * lane;
+    // the boundary inside this half-block, if any, is segment sgi+1's start
+    const int bn = __shfl_sync(0xffffffffu, b, min(sgi + 1, 31));
+    const int t1 = ((B >> lane) & 1u) ? bn : INT_MAX;
+    const int t2 = collide ? q0 : INT_MAX;  // forces the walk for the whole window
+    if (32 * i + lane < nhb) {
+      const uint32_t iw[2] = {d.iv[i].x, d.iv[i].y};
+      float blk[MP];
+      float a0[MP], a1[MP];
+#pragma unroll
+      for (int m = 0; m < MP; ++m) a0[m] = a1[m] = 0.f;
+      uint32_t f[4];
+      e2m1x8_to_f16x2x4(d.cv[i], f);
+      if (q0 + 7 < t2) {  // at most one boundary: entries e >= t use segment sgi+1
+        const int t = min(t1 - q0, 8);
+        const uint32_t z0 = zs_a + ((uint32_t)sgi << 8) * kRow;
+        const uint32_t z1 = z0 + 256u * kRow;
+#pragma unroll
+        for (int p = 0; p < 4; ++p) {
+          const float2 v = __half22float2(*reinterpret_cast<const __half2*>(&f[p]));
+          const int e0 = 2 * p, e1 = e0 + 1;
+          const uint32_t b0 = __byte_perm(iw[e0 >> 2], 0u, 0x4440u | (uint32_t)(e0 & 3));
+          const uint32_t b1 = __byte_perm(iw[e1 >> 2], 0u, 0x4440u | (uint32_t)(e1 & 3));
+          fma_z<MP>(a0, (e0 >= t ? z1 : z0) + b0 * kRow, v.x);
+          fma_z<MP>(a1, (e1 >= t ? z1 : z0) + b1 * kRow, v.y);
+        }
+      } else {  // several boundaries inside these 8 entries: walk them (row read from memory)
+        const uint16_t* ssrow = seg_start + (size_t)o * nseg;
+        int sg = 0;
+        for (int j = 1; j < nseg; ++j) sg += ((int)ssrow[j] <= q0);
+        int nb = (sg + 1 < nseg) ? (int)ssrow[sg + 1] : INT_MAX;
+#pragma unroll
+        for (int p = 0; p < 4; ++p) {
+          const float2 v = __half22float2(*reinterpret_cast<const __half2*>(&f[p]));
+#pragma unroll
+          for (int hh = 0; hh < 2; ++hh) {
+            const int ent = 2 * p + hh;
+            while (q0 + ent >= nb) {
+              ++sg;
+              nb = (sg + 1 < nseg) ? (int)ssrow[sg + 1] : INT_MAX;
+            }
+            const uint32_t b = __byte_perm(iw[ent >> 2], 0u, 0x4440u | (uint32_t)(ent & 3));
+            fma_z<MP>(hh ? a1 : a0, zs_a + (((uint32_t)sg << 8) + b) * kRow, hh ? v.y : v.x);
+          }
+        }
+      }
+      const float sc = e4m3_to_f32((d.sc >> (8 * i)) & 0xFFu);
+#pragma unroll
+      for (int m = 0; m < MP; ++m) acc[m] = fmaf(a0[m] + a1[m], sc, acc[m]);
+      (void)blk;
+    }
+  }
+#pragma unroll
+  for (int m = 0; m < MP; ++m) {
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) acc[m] += __shfl_xor_sync(0xffffffffu, acc[m], off);
+  }
+  if (lane == 0) {
+#pragma unroll
+    for (int m = 0; m < MP; ++m)
+      if (m < M) Y[(size_t)m * d_out + o] = __float2half_rn(acc[m] * s_C);
+  }
+}
+
 template <int MP>
 __global__ void __launch_bounds__(kGatherWarps * 32, 1)  // 1024 threads, at most 64 registers
 k_coeff_gather(const __grid_constant__ CoeffBatch batch) {
@@ -557,11 +653,13 @@ k_coeff_gather(const __grid_constant__ CoeffBatch batch) {
     prefetch_l2_range(scales, e0 >> 4, e1 >> 4);
     prefetch_l2_range(seg_start, (size_t)o_begin * nseg * 2, (size_t)o_end * nseg * 2);
   }
-  ColData cur, nxt;
-  uint32_t cb, cb_n;
-  int nhb, nhb_n;
+  // Two column buffers in ping-pong: the next column's loads are in flight while
+  // this one is summed, and no buffer is ever copied (a copy would wait for them).
+  ColData ca, cbuf;
+  uint32_t pa, pb;
+  int na, nb;
   int o = o_begin + warp;
-  load_col(cur, o, o_end, col_ptr, idx, codes, scales, seg_start, nseg, lane, cb, nhb);
+  load_col(ca, o, o_end, col_ptr, idx, codes, scales, seg_start, nseg, lane, pa, na);
   trigger_dependents();
   grid_dependency_wait();  // Z comes from the dictionary stage
 
@@ -569,100 +667,13 @@ k_coeff_gather(const __grid_constant__ CoeffBatch batch) {
   for (int i = k * MP + threadIdx.x; i < (k + 256) * MP; i += blockDim.x) zsg[i] = 0.f;
   __syncthreads();
   const uint32_t zs_a = smem_u32(zsg);
-  constexpr uint32_t kRow = MP * 4;
 
-  for (; o < o_end; o += kGatherWarps) {
-    load_col(nxt, o + kGatherWarps, o_end, col_ptr, idx, codes, scales, seg_start, nseg, lane, cb_n, nhb_n);
-    float acc[MP];
-#pragma unroll
-    for (int m = 0; m < MP; ++m) acc[m] = 0.f;
-    // Lane j holds seg_start[j] (the first entry of segment j). For the window of
-    // 256 entries starting at w, a boundary b in (w, w+256) lies at the start of
-    // lane p = (b-w)/8's half-block when (b-w) % 8 == 0, else inside it; two
-    // OR-reduced lane masks give every lane its segment with two popcounts.
-    const bool is_bnd = lane >= 1 && lane < nseg;
-#pragma unroll
-    for (int i = 0; i < kRmax; ++i) {
-      const int w = 256 * i;
-      if (w >= 8 * nhb) break;
-      const int b = cur.ssv;  // boundary held by this lane (meaningful iff is_bnd)
-      const int s_lo = __popc(__ballot_sync(0xffffffffu, is_bnd && b <= w));  // segment of entry w
-      const bool in_win = is_bnd && b > w && b < w + 256;
-      const int rel = b - w;
-      const uint32_t at_start = (in_win && (rel & 7) == 0) ? (1u << (rel >> 3)) : 0u;
-      const uint32_t inside = (in_win && (rel & 7) != 0) ? (1u << (rel >> 3)) : 0u;
-      const uint32_t A = __reduce_or_sync(0xffffffffu, at_start);
-      const uint32_t B = __reduce_or_sync(0xffffffffu, inside);
-      const int nwin = __popc(__ballot_sync(0xffffffffu, in_win));
-      const bool collide = nwin != __popc(A) + __popc(B) || (A & B) != 0u;  // two boundaries in one half-block
-      const uint32_t le = lane == 31 ? 0xffffffffu : ((2u << lane) - 1u);
-      const int before = __popc(A & le) + __popc(B & (le >> 1));  // boundaries <= q0 in the window
-      const int sgi = s_lo + before;                               // segment of q0
-      const int q0 = w + 8 * lane;
-      // the boundary inside this half-block, if any, is segment sgi+1's start
-      const int bn = __shfl_sync(0xffffffffu, b, min(sgi + 1, 31));
-      const int t1 = ((B >> lane) & 1u) ? bn : INT_MAX;
-      const int t2 = collide ? q0 : INT_MAX;  // forces the walk for the whole window
-      if (32 * i + lane < nhb) {
-        const uint32_t iw[2] = {cur.iv[i].x, cur.iv[i].y};
-        float blk[MP];
-        float a0[MP], a1[MP];
-#pragma unroll
-        for (int m = 0; m < MP; ++m) a0[m] = a1[m] = 0.f;
-        uint32_t f[4];
-        e2m1x8_to_f16x2x4(cur.cv[i], f);
-        if (q0 + 7 < t2) {  // at most one boundary: entries e >= t use segment sgi+1
-          const int t = min(t1 - q0, 8);
-          const uint32_t z0 = zs_a + ((uint32_t)sgi << 8) * kRow;
-          const uint32_t z1 = z0 + 256u * kRow;
-#pragma unroll
-          for (int p = 0; p < 4; ++p) {
-            const float2 v = __half22float2(*reinterpret_cast<const __half2*>(&f[p]));
-            const int e0 = 2 * p, e1 = e0 + 1;
-            const uint32_t b0 = __byte_perm(iw[e0 >> 2], 0u, 0x4440u | (uint32_t)(e0 & 3));
-            const uint32_t b1 = __byte_perm(iw[e1 >> 2], 0u, 0x4440u | (uint32_t)(e1 & 3));
-            fma_z<MP>(a0, (e0 >= t ? z1 : z0) + b0 * kRow, v.x);
-            fma_z<MP>(a1, (e1 >= t ? z1 : z0) + b1 * kRow, v.y);
-          }
-        } else {  // several boundaries inside these 8 entries: walk them (row read from memory)
-          const uint16_t* ssrow = seg_start + (size_t)o * nseg;
-          int sg = 0;
-          for (int j = 1; j < nseg; ++j) sg += ((int)ssrow[j] <= q0);
-          int nb = (sg + 1 < nseg) ? (int)ssrow[sg + 1] : INT_MAX;
-#pragma unroll
-          for (int p = 0; p < 4; ++p) {
-            const float2 v = __half22float2(*reinterpret_cast<const __half2*>(&f[p]));
-#pragma unroll
-            for (int hh = 0; hh < 2; ++hh) {
-              const int ent = 2 * p + hh;
-              while (q0 + ent >= nb) {
-                ++sg;
-                nb = (sg + 1 < nseg) ? (int)ssrow[sg + 1] : INT_MAX;
-              }
-              const uint32_t b = __byte_perm(iw[ent >> 2], 0u, 0x4440u | (uint32_t)(ent & 3));
-              fma_z<MP>(hh ? a1 : a0, zs_a + (((uint32_t)sg << 8) + b) * kRow, hh ? v.y : v.x);
-            }
-          }
-        }
-        const float sc = e4m3_to_f32((cur.sc >> (8 * i)) & 0xFFu);
-#pragma unroll
-        for (int m = 0; m < MP; ++m) acc[m] = fmaf(a0[m] + a1[m], sc, acc[m]);
-        (void)blk;
-      }
-    }
-#pragma unroll
-    for (int m = 0; m < MP; ++m) {
-#pragma unroll
-      for (int off = 16; off > 0; off >>= 1) acc[m] += __shfl_xor_sync(0xffffffffu, acc[m], off);
-    }
-    if (lane == 0) {
-#pragma unroll
-      for (int m = 0; m < MP; ++m)
-        if (m < M) Y[(size_t)m * d_out + o] = __float2half_rn(acc[m] * s_C);
-    }
-    cur = nxt;
-    cb = cb_n;
-    nhb = nhb_n;
+  for (; o < o_end; o += 2 * kGatherWarps) {
+    load_col(cbuf, o + kGatherWarps, o_end, col_ptr, idx, codes, scales, seg_start, nseg, lane, pb, nb);
+    gather_column<MP>(ca, o, na, zs_a, nseg, seg_start, lane, M, d_out, s_C, Y);
+    if (o + kGatherWarps >= o_end) break;
+    load_col(ca, o + 2 * kGatherWarps, o_end, col_ptr, idx, codes, scales, seg_start, nseg, lane, pa, na);
+    gather_column<MP>(cbuf, o + kGatherWarps, nb, zs_a, nseg, seg_start, lane, M, d_out, s_C, Y);
   }
 }
 
