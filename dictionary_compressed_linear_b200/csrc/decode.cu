@@ -492,12 +492,13 @@ k_coeff_decode(const uint4* __restrict__ chunks, const int* __restrict__ cta_ptr
 // the column's loads double-buffered in registers across the warp's columns, and
 // the column's seg_start row held one value per lane (read with shuffles).
 constexpr int kRmax = 5;         // steps of 32 half-blocks held per column
+static_assert(kRmax <= 8, "one scale byte per step in a 64-bit word");
 constexpr int kGatherWarps = 32;
 
 struct ColData {
   uint2 iv[kRmax];      // 8 index bytes per step
   uint32_t cv[kRmax];   // 8 codes (4 bytes) per step
-  uint32_t sc;          // E4M3 scale byte of each step, packed 8 bits apiece
+  uint64_t sc;          // E4M3 scale byte of each step, packed 8 bits apiece (kRmax <= 8)
   int ssv;              // seg_start[lane] of the column (lane < nseg)
 };
 
@@ -525,7 +526,7 @@ __device__ __forceinline__ void load_col(ColData& d, int o, int d_out, const uin
       const uint32_t e = cb + 8u * (uint32_t)h;
       d.iv[i] = ld_stream_v2(idx + e);
       d.cv[i] = *reinterpret_cast<const uint32_t*>(codes + (e >> 1));
-      d.sc |= ld_stream_u8(scales + (e >> 4)) << (8 * i);
+      d.sc |= (uint64_t)ld_stream_u8(scales + (e >> 4)) << (8 * i);
     }
   }
 }
@@ -608,7 +609,7 @@ __device__ __forceinline__ void gather_column(const ColData& d, int o, int nhb, 
           }
         }
       }
-      const float sc = e4m3_to_f32((d.sc >> (8 * i)) & 0xFFu);
+      const float sc = e4m3_to_f32((uint32_t)(d.sc >> (8 * i)) & 0xFFu);
 #pragma unroll
       for (int m = 0; m < MP; ++m) acc[m] = fmaf(a0[m] + a1[m], sc, acc[m]);
       (void)blk;

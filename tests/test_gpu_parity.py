@@ -239,3 +239,17 @@ def test_batch_rejects_repeated_group():
     with pytest.raises(dp.DictprojError) as e:
         dp.dictproj_forward_batch([X.data_ptr()] * 2, 1, [l, l], [g, g], [Y.data_ptr()] * 2, 0)
     assert e.value.status == -4
+
+
+# ------------------------------------------------------------------ long columns
+@pytest.mark.parametrize("M", [1, 3])
+def test_columns_longer_than_1024_entries(M):
+    # k = 3072 at density 0.4 stores 1229 entries per column (1232 padded): the
+    # gather kernel holds such a column in five 256-entry windows, the last one
+    # past entry 1024
+    D, C = _case(18, 0, 0, 0, 512, 3072, 96, 0.4)
+    g, l = device_projection(D, C, max_tokens=8)
+    pd, pc = oracle_projection(D, C)
+    assert int(np.diff(pc["col_ptr"]).max()) > 1024
+    X = synth.gen_activations(18, 0, 0, M, 512)
+    assert_parity(run_forward(g, l, X), oracle_forward(X, pd, pc), f"long columns M={M}")
