@@ -152,10 +152,6 @@ void dictproj_free_layer(dictproj_layer* l) {
   cudaFree(l->scales);
   cudaFree(l->idx);
   cudaFree(l->seg_start);
-  for (int i = 0; i < 2; ++i) {
-    cudaFree(l->chunks[i]);
-    cudaFree(l->cta_ptr[i]);
-  }
   delete l;
 }
 
@@ -309,35 +305,13 @@ int dictproj_layer_upload(const uint32_t* pcol_ptr, const uint8_t* codes, const 
     cudaGetLastError();
     return cuda_fail(e, "layer_upload: copy to device");
   }
-  // decode-path work plans: one and two CTAs per SM, entry-balanced column runs
-  int n_sm = 0, smem_sm = 0;
-  if ((e = cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess ||
-      (e = cudaDeviceGetAttribute(&smem_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev)) != cudaSuccess) {
+  int n_sm = 0;
+  if ((e = cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) {
     dictproj_free_layer(l);
     return cuda_fail(e, "layer_upload: device attributes");
   }
-  l->smem_per_sm = smem_sm;
   l->n_sm = n_sm;
   l->gather_ok = gather_supported(pcol_ptr, d_out, nseg);
-  for (int pi = 0; pi < 2; ++pi) {
-    std::vector<uint32_t> plan;
-    std::vector<int> cta_ptr;
-    const int G = n_sm * (pi + 1);
-    if (!plan_coeff_chunks(pcol_ptr, d_out, nseg, G, plan, cta_ptr)) break;
-    if ((e = dmalloc((void**)&l->chunks[pi], plan.size() * sizeof(uint32_t))) ||
-        (e = dmalloc((void**)&l->cta_ptr[pi], cta_ptr.size() * sizeof(int)))) {
-      dictproj_free_layer(l);
-      cudaGetLastError();
-      return fail(DICTPROJ_ERR_OOM, "layer_upload: device allocation failed (%s)", cudaGetErrorName(e));
-    }
-    if ((e = h2d(l->chunks[pi], plan.data(), plan.size() * sizeof(uint32_t))) ||
-        (e = h2d(l->cta_ptr[pi], cta_ptr.data(), cta_ptr.size() * sizeof(int)))) {
-      dictproj_free_layer(l);
-      cudaGetLastError();
-      return cuda_fail(e, "layer_upload: copy to device");
-    }
-    l->n_cta[pi] = G;
-  }
   // the true entry count is not part of the packed arrays; dictproj_pack_layer records it
   l->nnz_total = 0;
   *out = l;

@@ -16,17 +16,20 @@
 //   each slice writes s_D * partial to Zpart[slice][k][mp].
 //
 // Stage 2, coefficients (sparse gather over column-compressed NVFP4 C_l),
-// k_coeff_decode.
-//   Persistent CTAs own runs of columns balanced by stored entries; the runs are
-//   cut on the host (at upload) into chunks of at most 16 columns of equal padded
-//   length and 16384 entries, which stream through a two-stage shared-memory ring
-//   with bulk async copies completing on mbarriers (the first two issued before
-//   the dependency wait). Z = sum of the slices (fixed order) is staged in shared
-//   memory. One warp per column: lane l sums a contiguous run of 8-entry
-//   half-blocks (atom = 256*segment + idx; at most one segment boundary per
-//   half-block takes a select, more falls back to a walk), scales each by its
-//   E4M3 block scale, and the warp reduces with shuffles in a fixed order, so
-//   results are bit-reproducible. Y = s_C * sum in fp16.
+// k_coeff_gather.
+//   One CTA per SM (1024 threads) owns a contiguous run of columns, one warp per
+//   column. Z = the sum of the dictionary stage's slices (fixed order) is staged
+//   in shared memory with a zero tail. A column's entries (index bytes, codes,
+//   scales, seg_start) are loaded straight from global memory into registers,
+//   the first column before the dependency wait and each next one while the
+//   current one is summed: lane l takes the 8-entry half-blocks 32i + l of the
+//   column (atom = 256*segment + idx; the segment of each 256-entry window comes
+//   from warp-wide ballots over seg_start, several boundaries inside one
+//   half-block fall back to a walk), scales each by its E4M3 block scale, and the
+//   warp reduces with shuffles in a fixed order, so results are bit-reproducible.
+//   Y = s_C * sum in fp16. Columns longer than 1280 stored entries, or k above
+//   8192 atoms, go to k_coeff_decode_direct (one warp per column, lanes over
+//   16-entry blocks, any length).
 
 #include <algorithm>
 #include <climits>
@@ -233,18 +236,6 @@ k_dict_decode(const __grid_constant__ DictBatch batch) {
 // =================================================================================
 // Stage 2: coefficients
 // =================================================================================
-constexpr int kCoeffWarps = 16;
-constexpr int kCoeffThreads = kCoeffWarps * 32;
-constexpr int kChunkEntries = 16384;
-constexpr int kChunkCols = kCoeffWarps;  // one column per warp per chunk
-constexpr int kSegBytes = 8192;
-// stage layout (bytes): idx | codes | scales | seg_start
-constexpr int kStIdx = 0;
-constexpr int kStCodes = kStIdx + kChunkEntries;
-constexpr int kStScales = kStCodes + kChunkEntries / 2 + 16;
-constexpr int kStSeg = kStScales + kChunkEntries / 16 + 32;
-constexpr int kStageBytes = kStSeg + kSegBytes + 32;
-
 // Z rows live in shared memory at byte address zaddr + atom * MP * 4.
 template <int MP>
 __device__ __forceinline__ void fma_z(float blk[MP], uint32_t a, float v) {
@@ -266,11 +257,7 @@ __device__ __forceinline__ void fma_z(float blk[MP], uint32_t a, float v) {
   }
 }
 
-// seg_start row readers: shared-memory row (byte address) or global row.
-struct SegShared {
-  uint32_t a;
-  __device__ __forceinline__ int operator()(int j) const { return (int)lds_u16(a + 2u * (uint32_t)j); }
-};
+// seg_start row reader (global row).
 struct SegGlobal {
   const uint16_t* p;
   __device__ __forceinline__ int operator()(int j) const { return (int)p[j]; }
@@ -338,37 +325,6 @@ __device__ __forceinline__ void entries_sum(float blk[MP], uint32_t zaddr, const
   for (int m = 0; m < MP; ++m) blk[m] = a0[m] + a1[m];
 }
 
-struct StageRanges {
-  uint32_t codes_a0, scales_a0, seg_a0;  // 16-byte aligned source offsets
-  uint32_t idx_n, codes_n, scales_n, seg_n;
-};
-
-__device__ __forceinline__ StageRanges stage_ranges(const uint4 ch, int nseg) {
-  // ch = {o_b, o_e, e_b, e_e}
-  StageRanges r;
-  r.idx_n = ch.w - ch.z;
-  r.codes_a0 = (ch.z >> 1) & ~15u;
-  r.codes_n = (((ch.w >> 1) + 15u) & ~15u) - r.codes_a0;
-  r.scales_a0 = (ch.z >> 4) & ~15u;
-  r.scales_n = (((ch.w >> 4) + 15u) & ~15u) - r.scales_a0;
-  const uint32_t sb = 2u * ch.x * (uint32_t)nseg, se = 2u * ch.y * (uint32_t)nseg;
-  r.seg_a0 = sb & ~15u;
-  r.seg_n = ((se + 15u) & ~15u) - r.seg_a0;
-  return r;
-}
-
-__device__ __forceinline__ void issue_chunk(unsigned char* st, uint64_t* bar, const uint4 ch, int nseg,
-                                           const uint8_t* idx, const uint8_t* codes, const uint8_t* scales,
-                                           const uint16_t* seg_start) {
-  const StageRanges r = stage_ranges(ch, nseg);
-  mbar_arrive_expect_tx(bar, r.idx_n + r.codes_n + r.scales_n + r.seg_n);
-  if (r.idx_n) bulk_g2s(st + kStIdx, idx + ch.z, r.idx_n, bar);
-  if (r.codes_n) bulk_g2s(st + kStCodes, codes + r.codes_a0, r.codes_n, bar);
-  if (r.scales_n) bulk_g2s(st + kStScales, scales + r.scales_a0, r.scales_n, bar);
-  if (r.seg_n)
-    bulk_g2s(st + kStSeg, reinterpret_cast<const uint8_t*>(seg_start) + r.seg_a0, r.seg_n, bar);
-}
-
 // Stage Z (sum of the dictionary stage's slices, fixed order) into shared memory.
 template <int MP>
 __device__ __forceinline__ void stage_z(float* zs, const float* __restrict__ Zpart, int nslices, int k, int nthr) {
@@ -383,106 +339,6 @@ __device__ __forceinline__ void stage_z(float* zs, const float* __restrict__ Zpa
       a.w += b.w;
     }
     *reinterpret_cast<float4*>(zs + i) = a;
-  }
-}
-
-template <int MP>
-__global__ void __launch_bounds__(kCoeffThreads, 2)  // caps registers at 64; launched one CTA per SM
-k_coeff_decode(const uint4* __restrict__ chunks, const int* __restrict__ cta_ptr,
-               const uint8_t* __restrict__ codes, const uint8_t* __restrict__ scales,
-               const uint8_t* __restrict__ idx, const uint16_t* __restrict__ seg_start, int nseg,
-               float s_C, int k, int d_out, const float* __restrict__ Zpart, int nslices, int M,
-               __half* __restrict__ Y, int nst) {
-  extern __shared__ __align__(128) unsigned char csmem[];
-  float* zs = reinterpret_cast<float*>(csmem);  // [k][MP]
-  unsigned char* stage0 = reinterpret_cast<unsigned char*>(zs + (size_t)k * MP);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(stage0 + (size_t)nst * kStageBytes);
-
-  const int c0 = cta_ptr[blockIdx.x], c1 = cta_ptr[blockIdx.x + 1];
-  const int nch = c1 - c0;
-  if (threadIdx.x == 0) {
-    for (int i = 0; i < nst; ++i) mbar_init(&bars[i], 1);
-    fence_mbar_init();
-  }
-  __syncthreads();
-  if (threadIdx.x == 0) {  // weights: issue the first nst chunks before the dependency wait
-    for (int i = 0; i < nst && i < nch; ++i)
-      issue_chunk(stage0 + (size_t)i * kStageBytes, &bars[i], chunks[c0 + i], nseg, idx, codes, scales,
-                  seg_start);
-  }
-  trigger_dependents();
-  grid_dependency_wait();  // Z comes from the dictionary stage
-
-  stage_z<MP>(zs, Zpart, nslices, k, kCoeffThreads);
-  __syncthreads();
-
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const uint32_t zs_a = smem_u32(zs);
-  for (int ci = 0; ci < nch; ++ci) {
-    const int sti = ci % nst;
-    unsigned char* st = stage0 + (size_t)sti * kStageBytes;
-    const uint4 ch = chunks[c0 + ci];
-    if (!mbar_wait_bounded(&bars[sti], (ci / nst) & 1)) break;  // error recorded; leave
-    const StageRanges r = stage_ranges(ch, nseg);
-    const int ncols = (int)(ch.y - ch.x);
-    const int P = ncols ? (int)((ch.w - ch.z) / (uint32_t)ncols) : 0;
-    const uint32_t st_a = smem_u32(st);
-    const uint32_t idx_a = st_a + kStIdx;
-    const uint32_t codes_a = st_a + kStCodes + ((ch.z >> 1) - r.codes_a0);
-    const uint32_t scales_a = st_a + kStScales + ((ch.z >> 4) - r.scales_a0);
-    const uint32_t seg_a = st_a + kStSeg + (2u * ch.x * (uint32_t)nseg - r.seg_a0);
-
-    // One warp per column. At step i the warp covers entries [256i, 256i+256):
-    // lane l takes the half-block of 8 entries at 256i + 8l (consecutive lanes read
-    // consecutive index / code bytes). Segment boundaries of the window are
-    // scanned once per step by the whole warp (uniform loads).
-    const int nhb = P >> 3;
-    for (int col = warp; col < ncols; col += kCoeffWarps) {
-      const SegShared ss{seg_a + 2u * (uint32_t)(col * nseg)};
-      const uint32_t cb = (uint32_t)(col * P);
-      float acc[MP];
-#pragma unroll
-      for (int m = 0; m < MP; ++m) acc[m] = 0.f;
-      int s_lo = 0;  // segment of the window start
-      for (int h0 = 0; h0 < nhb; h0 += 32) {
-        const int w = h0 << 3;
-        while (s_lo + 1 < nseg && ss(s_lo + 1) <= w) ++s_lo;
-        const int h = h0 + lane;
-        const int q0 = h << 3;
-        int sgi = s_lo, t1 = INT_MAX, t2 = INT_MAX;
-        for (int j = s_lo + 1; j < nseg; ++j) {  // uniform over the warp
-          const int b = ss(j);
-          if (b > w + 256 + 8) break;
-          if (b <= q0) sgi = j;
-          else if (t1 == INT_MAX) t1 = b;
-          else if (t2 == INT_MAX) t2 = b;
-        }
-        if (h < nhb) {
-          const uint32_t e = cb + (uint32_t)q0;  // chunk-relative entry offset
-          const uint2 iv = lds_u32x2(idx_a + e);
-          const uint32_t cv = lds_u32(codes_a + (e >> 1));
-          const float sc = e4m3_to_f32(lds_u8(scales_a + (e >> 4)));
-          const uint32_t iw[2] = {iv.x, iv.y};
-          float blk[MP];
-          entries_sum<MP, 8>(blk, zs_a, iw, &cv, q0, sgi, t1, t2, ss, nseg);
-#pragma unroll
-          for (int m = 0; m < MP; ++m) acc[m] = fmaf(blk[m], sc, acc[m]);
-        }
-      }
-#pragma unroll
-      for (int m = 0; m < MP; ++m) {
-#pragma unroll
-        for (int off = 16; off > 0; off >>= 1) acc[m] += __shfl_xor_sync(0xffffffffu, acc[m], off);
-      }
-      if (lane == 0) {
-#pragma unroll
-        for (int m = 0; m < MP; ++m)
-          if (m < M) Y[(size_t)m * d_out + ch.x + col] = __float2half_rn(acc[m] * s_C);
-      }
-    }
-    __syncthreads();  // the stage is free again
-    if (threadIdx.x == 0 && ci + nst < nch)
-      issue_chunk(st, &bars[sti], chunks[c0 + ci + nst], nseg, idx, codes, scales, seg_start);
   }
 }
 
@@ -751,23 +607,6 @@ static cudaError_t launch_pdl(const void* fn, dim3 grid, dim3 block, size_t smem
 
 int decode_mp(int M) { return M <= 1 ? 1 : M <= 2 ? 2 : M <= 4 ? 4 : 8; }
 
-// Ring depth: as many chunk stages as fit next to Z within half an SM's shared
-// memory (so the next kernel's CTAs can be resident alongside), at least 2.
-constexpr int kMaxStages = 4;
-constexpr size_t kCoeffSmemCap = 110 * 1024;
-
-static int coeff_stages(int k, int mp) {
-  const size_t z = (size_t)k * mp * 4;
-  if (z + 2 * (size_t)kStageBytes + 8 * kMaxStages > kCoeffSmemCap) return 2;
-  return (int)std::min<size_t>(kMaxStages, (kCoeffSmemCap - z - 8 * kMaxStages) / kStageBytes);
-}
-
-static size_t coeff_smem(int k, int mp) {
-  return (size_t)k * mp * 4 + (size_t)coeff_stages(k, mp) * kStageBytes + 8 * kMaxStages;
-}
-
-size_t coeff_decode_smem(int k, int mp) { return coeff_smem(k, mp); }
-
 // Dictionary-stage grid: (k/16 tiles) x slices, each warp J units of 128
 // elements. J is the smallest count that keeps at most two CTAs per SM and
 // lets the M rows of the slice's X fit kDictXsMax bytes of shared memory;
@@ -820,10 +659,6 @@ cudaError_t prepare_decode_kernels(int device) {
   }
   SET_SMEM((k_dict_decode<1, true>));
   SET_SMEM((k_dict_decode<2, true>));
-  SET_SMEM(k_coeff_decode<1>);
-  SET_SMEM(k_coeff_decode<2>);
-  SET_SMEM(k_coeff_decode<4>);
-  SET_SMEM(k_coeff_decode<8>);
   SET_SMEM(k_coeff_gather<1>);
   SET_SMEM(k_coeff_gather<2>);
   SET_SMEM(k_coeff_gather<4>);
@@ -937,25 +772,6 @@ cudaError_t launch_coeff_decode(const dictproj_layer* l, const float* Zpart, int
   float s = l->s;
   int k = l->k, d_out = l->d_out;
   if (l->gather_ok) return launch_gather_batch(1, &l, &Zpart, &nslices, M, mp, &Y, stream);
-  if (l->chunks[0]) {
-    const size_t smem = coeff_smem(k, mp);
-    // one CTA per SM (half the register file), leaving room for the next call's
-    // dictionary kernel to become resident and prefetch its weights
-    const int pi = 0;
-    const uint4* chunks = reinterpret_cast<const uint4*>(l->chunks[pi]);
-    const int* cta_ptr = l->cta_ptr[pi];
-    int nst = coeff_stages(k, mp);
-    void* args[] = {(void*)&chunks, (void*)&cta_ptr, (void*)&codes, (void*)&scales, (void*)&idx,
-                    (void*)&ss, (void*)&nseg, (void*)&s, (void*)&k, (void*)&d_out, (void*)&Zpart,
-                    (void*)&nslices, (void*)&M, (void*)&Y, (void*)&nst};
-    const dim3 grid(l->n_cta[pi]), block(kCoeffThreads);
-    switch (mp) {
-      case 1: return launch_pdl((const void*)k_coeff_decode<1>, grid, block, smem, stream, args);
-      case 2: return launch_pdl((const void*)k_coeff_decode<2>, grid, block, smem, stream, args);
-      case 4: return launch_pdl((const void*)k_coeff_decode<4>, grid, block, smem, stream, args);
-      default: return launch_pdl((const void*)k_coeff_decode<8>, grid, block, smem, stream, args);
-    }
-  }
   const uint32_t* col_ptr = l->col_ptr;
   void* args[] = {(void*)&col_ptr, (void*)&codes, (void*)&scales, (void*)&idx, (void*)&ss,
                   (void*)&nseg, (void*)&s, (void*)&k, (void*)&d_out, (void*)&Zpart, (void*)&nslices,
@@ -968,40 +784,6 @@ cudaError_t launch_coeff_decode(const dictproj_layer* l, const float* Zpart, int
     case 4: return launch_pdl((const void*)k_coeff_decode_direct<4>, grid, block, smem, stream, args);
     default: return launch_pdl((const void*)k_coeff_decode_direct<8>, grid, block, smem, stream, args);
   }
-}
-
-// Chunk plan for k_coeff_decode: CTA c owns the columns whose first entry falls in
-// [c*T/G, (c+1)*T/G); its run is cut into chunks of equal padded column length,
-// at most kChunkEntries entries and at most kSegBytes of seg_start rows.
-// Returns false if some column is longer than a chunk (use the direct kernel).
-bool plan_coeff_chunks(const uint32_t* pcol_ptr, int d_out, int nseg, int G, std::vector<uint32_t>& chunks,
-                       std::vector<int>& cta_ptr) {
-  chunks.clear();
-  cta_ptr.assign(G + 1, 0);
-  const uint64_t T = pcol_ptr[d_out];
-  const int max_cols = std::max(1, std::min(kChunkCols, kSegBytes / (2 * nseg)));
-  for (int o = 0; o < d_out; ++o)
-    if (pcol_ptr[o + 1] - pcol_ptr[o] > (uint32_t)kChunkEntries) return false;
-  int o = 0;
-  for (int c = 0; c < G; ++c) {
-    cta_ptr[c] = (int)(chunks.size() / 4);
-    const uint64_t hi = (c + 1 == G) ? UINT64_MAX : (T * (uint64_t)(c + 1)) / (uint64_t)G;
-    while (o < d_out && (c + 1 == G || (uint64_t)pcol_ptr[o] < hi)) {
-      const uint32_t P = pcol_ptr[o + 1] - pcol_ptr[o];
-      int o2 = o + 1;
-      while (o2 < d_out && (c + 1 == G || (uint64_t)pcol_ptr[o2] < hi) &&
-             pcol_ptr[o2 + 1] - pcol_ptr[o2] == P && (uint64_t)(o2 + 1 - o) * P <= (uint64_t)kChunkEntries &&
-             o2 + 1 - o <= max_cols)
-        ++o2;
-      chunks.push_back((uint32_t)o);
-      chunks.push_back((uint32_t)o2);
-      chunks.push_back(pcol_ptr[o]);
-      chunks.push_back(pcol_ptr[o2]);
-      o = o2;
-    }
-  }
-  cta_ptr[G] = (int)(chunks.size() / 4);
-  return true;
 }
 
 bool gather_supported(const uint32_t* pcol_ptr, int d_out, int nseg) {

@@ -65,12 +65,6 @@ struct dictproj_layer {
   uint8_t* scales;         // [total/16]
   uint8_t* idx;            // [total]
   uint16_t* seg_start;     // [d_out][nseg]
-  // decode-path work plan (see plan_coeff_chunks): chunk {o_b, o_e, e_b, e_e}
-  // plan[0]: one CTA per SM; plan[1]: two CTAs per SM (used when two fit)
-  uint32_t* chunks[2];     // [n_chunks][4], device; NULL -> direct kernel
-  int* cta_ptr[2];         // [n_cta+1], device
-  int n_cta[2];
-  int smem_per_sm;         // bytes of shared memory per SM on this device
   int n_sm;                // SMs of the device
-  bool gather_ok;          // the direct gather kernel serves this layer
+  bool gather_ok;          // the gather kernel serves this layer (else the direct kernel)
 };

@@ -13,7 +13,6 @@ namespace dictproj {
 // decode path (M <= 8): Z fp32 [k][mp], mp = next power of two >= M (at most 8),
 // written by the dictionary stage as `slices` partial sums Zpart[slice][k][mp]
 int decode_mp(int M);
-size_t coeff_decode_smem(int k, int mp);
 cudaError_t prepare_decode_kernels(int device);
 
 struct DictPlan {
@@ -33,11 +32,8 @@ cudaError_t launch_dict_decode_batch(int n, const dictproj_group* const* g, cons
 cudaError_t launch_coeff_decode_batch(int n, const dictproj_layer* const* l, const float* const* Zpart,
                                       const int* nslices, int M, int mp, __half* const* Y, cudaStream_t stream);
 
-// Work plan of the chunked coefficient kernel for a grid of G CTAs (host side).
-bool plan_coeff_chunks(const uint32_t* pcol_ptr, int d_out, int nseg, int G, std::vector<uint32_t>& chunks,
-                       std::vector<int>& cta_ptr);
-// Whether the direct gather kernel serves a layer (every column <= 1280 padded
-// entries, at most 32 segments).
+// Whether the gather kernel serves a layer (every column <= 1280 padded
+// entries, at most 32 segments); other layers use the direct kernel.
 bool gather_supported(const uint32_t* pcol_ptr, int d_out, int nseg);
 // Read and clear the device error word of the decode kernels.
 cudaError_t take_decode_error(unsigned int* out);
