@@ -342,11 +342,11 @@ __device__ __forceinline__ void stage_z(float* zs, const float* __restrict__ Zpa
   }
 }
 
-// Direct coefficient kernel for columns of at most kRmax*256 entries and k of
-// at most 32*256 atoms (nseg <= 32): one warp per column, lanes interleaved over
-// 8-entry half-blocks (coalesced, conflict-free loads straight from global/L2),
-// the column's loads double-buffered in registers across the warp's columns, and
-// the column's seg_start row held one value per lane (read with shuffles).
+// Gather kernel (k_coeff_gather) for columns of at most kRmax*256 entries and k
+// of at most 32*256 atoms (nseg <= 32): one warp per column, lanes interleaved
+// over 8-entry half-blocks (coalesced, conflict-free loads straight from
+// global/L2), the column's loads double-buffered in registers across the warp's
+// columns, and the column's seg_start row held one value per lane.
 constexpr int kRmax = 5;         // steps of 32 half-blocks held per column
 static_assert(kRmax <= 8, "one scale byte per step in a 64-bit word");
 constexpr int kGatherWarps = 32;
@@ -534,8 +534,10 @@ k_coeff_gather(const __grid_constant__ CoeffBatch batch) {
   }
 }
 
-// Fallback for layers whose columns do not fit a chunk (padded column length >
-// 16384 entries): lanes read blocks straight from global memory.
+// Direct kernel, for layers the gather does not hold (a column longer than
+// kRmax*256 stored entries, or more than 32 segments) and for the no-allocation
+// forward: one warp per column, lanes over 16-entry blocks read straight from
+// global memory, any column length.
 template <int MP>
 __global__ void __launch_bounds__(256)
 k_coeff_decode_direct(const uint32_t* __restrict__ col_ptr, const uint8_t* __restrict__ codes,

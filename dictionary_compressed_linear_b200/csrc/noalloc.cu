@@ -104,7 +104,8 @@ extern "C" int dictproj_forward_noalloc(const dictproj_device_group* group, cons
   l.scales = const_cast<uint8_t*>(layer->scales);
   l.idx = const_cast<uint8_t*>(layer->idx);
   l.seg_start = const_cast<uint16_t*>(layer->seg_start);
-  // no chunk plan: the coefficient stage reads the columns directly
+  // gather_ok stays false: the coefficient stage runs the direct kernel, whose
+  // shared memory is only Z
 
   cudaStream_t s = (cudaStream_t)stream;
   cudaError_t e;
