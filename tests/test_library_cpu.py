@@ -128,6 +128,26 @@ def test_host_validation(dp):
     assert lib.dictproj_pack_group_host(None, 32, 16, None, None, None) == -1
     assert dp.dictproj_forward_status(0, 1, None, None, 0) == -1
     assert "NULL" in dp.dictproj_last_error()
+    # the prefill entry points and the host helpers validate before touching a device
+    import ctypes as C
+    assert lib.dictproj_dictionary_stage_prefill(None, 16, None, None, None) == -1
+    assert lib.dictproj_group_reserve_prefill(None, 4096) == -1
+    assert lib.dictproj_forward_noalloc(None, None, None, 1, None, None) == -1
+    k = C.c_int()
+    assert lib.dictproj_rank_for_budget(0.2, 0, 4096, 4096, 1, C.byref(k)) == -2
+    assert lib.dictproj_rank_for_budget(-0.1, 1, 4096, 4096, 1, C.byref(k)) == -5
+    assert lib.dictproj_rank_for_budget(0.2, 1, 4096, 4096, 1, None) == -1
+    assert lib.dictproj_budget(1, 4096, 4096, 16, 1.5, None, None, None, None) == -5
+    assert lib.dictproj_group_file_write(None, None, None, 1.0, 64, 16) == -1
+    codes = np.zeros(64 * 16 // 2, np.uint8)
+    scales = np.zeros(64 * 16 // 16, np.uint8)
+    u8 = C.POINTER(C.c_uint8)
+    assert lib.dictproj_group_file_write(b"/nonexistent-dir/x.dpj", codes.ctypes.data_as(u8),
+                                         scales.ctypes.data_as(u8), 1.0, 64, 16) == -11
+    assert lib.dictproj_group_file_write(b"x.dpj", codes.ctypes.data_as(u8), scales.ctypes.data_as(u8),
+                                         float("nan"), 64, 16) == -10
+    assert lib.dictproj_group_file_write(b"x.dpj", codes.ctypes.data_as(u8), scales.ctypes.data_as(u8),
+                                         1.0, 48, 16) == -2
 
 
 def test_device_calls_fail_loudly_without_gpu(dp):
