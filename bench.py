@@ -145,6 +145,18 @@ def replica_throughput(tokens_per_rank, world, ms):
 
 # ----------------------------------------------------------------------------- prefill leg
 PREFILL_SHAPES = ("q", "gate", "down")
+PREFILL_TOKENS = (128, 512, 2048)
+
+
+def prefill_inputs(name, M):
+    """The prefill workload's inputs for one projection type at M tokens: D (fp32
+    d_in x k), C (density 0.3) and X (fp16 M x d_in, 1% of channels x20)."""
+    d_in, d_out, k = synth.LLAMA7B_SHAPES[name]
+    pt = synth.PROJ_TYPES.index(name)
+    D = synth.gen_dictionary(4, 0, pt, d_in, k)
+    C = synth.gen_coeff(4, 0, pt, 0, k, d_out, 0.3)
+    X = synth.gen_activations(4, 0, synth.INPUT_SITE[name], M, d_in, 0.01)
+    return D, C, X
 
 
 def prefill_bench(torch, dp, stream, M=2048, reps=20):
@@ -159,16 +171,14 @@ def prefill_bench(torch, dp, stream, M=2048, reps=20):
            "peak_tflops": peak, "peak_source": peak_src, "shapes": {}}
     for name in PREFILL_SHAPES:
         d_in, d_out, k = synth.LLAMA7B_SHAPES[name]
-        pt = synth.PROJ_TYPES.index(name)
-        D = synth.gen_dictionary(4, 0, pt, d_in, k)
-        C = synth.gen_coeff(4, 0, pt, 0, k, d_out, 0.3)
+        D, C, X_np = prefill_inputs(name, M)
         pg = dp.dictproj_pack_group_host(D)
         pc = dp.dictproj_pack_layer_host(C.col_ptr, C.atom_idx, C.vals, k, d_out)
         gs = [dp.dictproj_group_upload(pg, M) for _ in range(2)]
         for g in gs:
             dp.dictproj_group_reserve_prefill(g, d_out)
         ls = [dp.dictproj_layer_upload(pc) for _ in range(2)]
-        X = torch.from_numpy(synth.gen_activations(4, 0, synth.INPUT_SITE[name], M, d_in, 0.01)).cuda()
+        X = torch.from_numpy(X_np).cuda()
         Z = torch.empty((M, k), dtype=torch.float16, device="cuda")
         Y = torch.empty((M, d_out), dtype=torch.float16, device="cuda")
         res = {}
@@ -399,48 +409,73 @@ def cpu_baseline(workload, n_layers, budget_s=12.0):
                       f"scaled x{n_layers}; one-off decode+pack of the sample took {decode_s:.1f}s"}
 
 
-def run_reference(args):
-    """--impl reference: the oracle timed on the host cores (rank 0 only)."""
+def step_config(wl, n_layers, M, world, batched=True):
+    """The `config` object of the JSON line; both arms print the same one."""
+    return {"workload": f"{wl.name}: {n_layers} layers in {n_layers // 2} groups x 7 projection "
+                        "types (LLaMA-7B shapes), NVFP4 D/C, C density U[0.2,0.4], M=1",
+            "tokens_per_step": M, "projections_per_step": len(wl.projections),
+            "weights": "nvfp4 (E2M1 + E4M3/16 + fp32)", "activations": "fp16", "accumulate": "fp32",
+            "l2": "inputs larger than L2 (packed weights ~2.6 GB, no flush needed)",
+            "parallelism": f"replicas x{world}" if world > 1 else "single GPU"}
+
+
+def run_reference(args, budget_s=200.0):
+    """--impl reference: the oracle timed on the host cores (rank 0 only).
+
+    A step is the whole stack's forward: the fp64 factored forward of all
+    n_layers x 7 projections in model order, each layer reusing the 7 decoded
+    factors of layer 0 (same shapes; decoding all 224 would take minutes). If
+    warm-up + timed steps of the whole stack would not fit `budget_s`, a step is
+    instead the first S projections of that sequence and a step then counts as
+    S / (n_layers x 7) tokens, so that value and ms_per_step describe exactly
+    what was timed."""
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     if rank != 0:
         return 0
     from oracle import forward as F
     wl = synth.full_step(n_layers=args.layers)
+    t_setup = time.perf_counter()
     sample = oracle_layer_sample(wl)
-    per_type = {}
-    budget = 200.0
-    t_start = time.perf_counter()
-    for i in range(args.warmup):
-        p, dec, X = sample[i % len(sample)]
+    setup_s = time.perf_counter() - t_setup
+    n_proj = args.layers * len(sample)
+    # probe: one pass over the 7 projections gives the time per projection
+    t = time.perf_counter()
+    for p, dec, X in sample:
         F.forward_factored_decoded(X, dec)
-    steps = 0
-    for i in range(args.steps):
-        p, dec, X = sample[i % len(sample)]
-        t = time.perf_counter()
-        F.forward_factored_decoded(X, dec)
-        per_type.setdefault(p.name, []).append(time.perf_counter() - t)
-        steps += 1
-        if time.perf_counter() - t_start > budget and len(per_type) == len(sample):
-            break
-    # a step samples one projection; the stack has n_layers of each of the 7 types
-    layer_s = 0.0
-    for p, _, _ in sample:
-        ts = per_type.get(p.name)
-        layer_s += statistics.mean(ts) if ts else statistics.mean([statistics.mean(v) for v in per_type.values()])
-    value = 1.0 / (args.layers * layer_s)
-    wall = time.perf_counter() - t_start
+    per_proj = (time.perf_counter() - t) / len(sample)
+    steps_total = args.warmup + args.steps
+    S = n_proj
+    if steps_total * n_proj * per_proj > budget_s:
+        S = max(1, int(budget_s / (steps_total * per_proj)))
+    seq = [sample[i % len(sample)] for i in range(S)]
+
+    def one_step():
+        for p, dec, X in seq:
+            F.forward_factored_decoded(X, dec)
+
+    for _ in range(args.warmup):
+        one_step()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        one_step()
+    timed_s = time.perf_counter() - t0
+    ms_per_step = 1e3 * timed_s / args.steps
+    tokens_per_step = S / n_proj
+    value = tokens_per_step * args.steps / timed_s
+    what = (f"each step = the fp64 oracle's factored forward of all {n_proj} projections of the stack "
+            f"in model order" if S == n_proj else
+            f"each step = the first {S} of the stack's {n_proj} projections in model order "
+            f"({tokens_per_step:.4f} token per step), sized to fit {budget_s:.0f}s")
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
-        "steps": steps, "steps_requested": args.steps, "warmup": args.warmup,
-        "ms_per_step": 1e3 * args.layers * layer_s, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": wl.name, "layers": args.layers, "projections_per_step": 224, "tokens_per_step": 1},
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": step_config(wl, args.layers, 1, world),
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": len(os.sched_getaffinity(0)),
                          "kind": "oracle",
-                         "sample": "each step = the fp64 oracle's factored forward of one projection of "
-                                   "layer 0 (cycling q,k,v,o,gate,up,down; factors pre-decoded), "
-                                   f"scaled to {args.layers} layers x 7 types; {steps} steps in {wall:.0f}s"},
+                         "sample": f"{what}; every layer reuses layer 0's 7 decoded factors (pre-decoded in "
+                                   f"{setup_s:.0f}s); {args.steps} timed steps in {timed_s:.1f}s"},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -456,6 +491,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--layers", type=int, default=32)
     ap.add_argument("--stage-reps", type=int, default=50)
+    ap.add_argument("--ref-budget", type=float, default=200.0,
+                    help="--impl reference: seconds that warm-up plus timed steps may take")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-prefill", action="store_true", help="skip the prefill (M=2048) leg")
     ap.add_argument("--no-batch", action="store_true",
@@ -464,7 +501,7 @@ def main():
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     if args.impl == "reference":
-        return run_reference(args)
+        return run_reference(args, args.ref_budget)
 
     import torch
     import dictionary_compressed_linear_b200 as dp
@@ -609,15 +646,10 @@ def main():
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f16",
         "data": "synthetic",
-        "config": {"workload": f"{wl.name}: {args.layers} layers in {args.layers // 2} groups x 7 projection "
-                               "types (LLaMA-7B shapes), NVFP4 D/C, C density U[0.2,0.4], M=1",
-                   "tokens_per_step": M, "projections_per_step": len(wl.projections),
-                   "calls_per_step": calls_per_step,
-                   "batching": "q/k/v and gate/up share a call (dictproj_forward_batch)" if not args.no_batch
-                               else "one dictproj_forward per projection",
-                   "weights": "nvfp4 (E2M1 + E4M3/16 + fp32)", "activations": "fp16", "accumulate": "fp32",
-                   "l2": "inputs larger than L2 (packed weights ~2.6 GB, no flush needed)",
-                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
+        "config": step_config(wl, args.layers, M, world),
+        "calls_per_step": calls_per_step,
+        "batching": "q/k/v and gate/up share a call (dictproj_forward_batch)" if not args.no_batch
+                    else "one dictproj_forward per projection",
         "roofline": roofline,
         "cpu_baseline": cpu,
         "e2e": {"value": round(e2e_value, 2), "unit": "tokens/s", "h2d_bytes_per_step": h2d,

@@ -100,6 +100,7 @@ SIGNATURES = [
     ("dictproj_layer_save", C.c_int, [C.c_void_p, C.c_char_p]),
     ("dictproj_layer_load", C.c_int, [C.c_char_p, C.POINTER(C.c_void_p)]),
     ("dictproj_check", C.c_int, [C.c_void_p]),
+    ("dictproj_selftest_wait_timeout", C.c_int, [C.c_longlong, C.c_void_p]),
     ("dictproj_last_error", C.c_char_p, []),
     ("dictproj_status_string", C.c_char_p, [C.c_int]),
     ("dictproj_version", C.c_int, []),
@@ -465,3 +466,12 @@ def dictproj_forward_noalloc_status(group: DeviceGroup, layer: DeviceLayer, X_pt
 
 def dictproj_check(stream: int = 0):
     _check(lib().dictproj_check(C.c_void_p(stream)))
+
+
+def dictproj_check_status(stream: int = 0) -> int:
+    """dictproj_check without raising: the status code."""
+    return lib().dictproj_check(C.c_void_p(stream))
+
+
+def dictproj_selftest_wait_timeout(cycles: int, stream: int = 0):
+    _check(lib().dictproj_selftest_wait_timeout(int(cycles), C.c_void_p(stream)))

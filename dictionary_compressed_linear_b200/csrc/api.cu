@@ -461,6 +461,10 @@ int dictproj_forward_path(const void* X, int M, const dictproj_layer* layer, con
   const DictPlan plan = dict_plan(group->d_in, group->k, group->n_sm, M < kDecodeMaxTokens ? M : kDecodeMaxTokens, false);
   if (decode) {
     const int mp = decode_mp(M);
+    if (!coeff_smem_fits(group->k, mp, dev))
+      return fail(DICTPROJ_ERR_UNSUPPORTED,
+                  "forward: the decode path stages (k + 256) * %d floats of Z in shared memory; k=%d does not fit "
+                  "at M=%d", mp, group->k, M);
     if ((e = launch_dict_decode(group, x, M, mp, group->z32, plan, s)) != cudaSuccess)
       return cuda_fail(e, "forward: dictionary stage launch");
     if ((e = launch_coeff_decode(layer, group->z32, plan.slices, M, mp, y, s)) != cudaSuccess)
@@ -517,6 +521,11 @@ int dictproj_forward_batch(int n, const void* const* X, int M, const dictproj_la
     return DICTPROJ_OK;
   }
   const int mp = decode_mp(M);
+  for (int i = 0; i < n; ++i)
+    if (!coeff_smem_fits(groups[i]->k, mp, dev))
+      return fail(DICTPROJ_ERR_UNSUPPORTED,
+                  "forward_batch: the decode path stages (k + 256) * %d floats of Z in shared memory; k=%d "
+                  "(entry %d) does not fit at M=%d", mp, groups[i]->k, i, M);
   DictPlan plans[kDecodeMaxBatch];
   const __half* xs[kDecodeMaxBatch];
   float* zs[kDecodeMaxBatch];
@@ -575,8 +584,21 @@ int dictproj_coefficient_stage(const float* Z, int M, const dictproj_layer* laye
   if (M < 1) return fail(DICTPROJ_ERR_RANGE, "coefficient_stage: M=%d < 1", M);
   if (M > kDecodeMaxTokens) return fail(DICTPROJ_ERR_UNSUPPORTED, "coefficient_stage: M must be <= %d", kDecodeMaxTokens);
   if (((uintptr_t)Y & 15) || ((uintptr_t)Z & 15)) return fail(DICTPROJ_ERR_ALIGN, "coefficient_stage: Z and Y must be 16-byte aligned");
+  if (!coeff_smem_fits(layer->k, decode_mp(M), layer->device))
+    return fail(DICTPROJ_ERR_UNSUPPORTED, "coefficient_stage: (k + 256) * mp floats of Z do not fit in shared "
+                "memory (k=%d, M=%d)", layer->k, M);
   cudaError_t e = launch_coeff_decode(layer, Z, 1, M, decode_mp(M), static_cast<__half*>(Y), (cudaStream_t)stream);
   return e == cudaSuccess ? DICTPROJ_OK : cuda_fail(e, "coefficient_stage: launch");
+}
+
+int dictproj_selftest_wait_timeout(long long cycles, void* stream) {
+  clear_error();
+  if (cycles < 1 || cycles > (1ll << 31))
+    return fail(DICTPROJ_ERR_RANGE, "selftest_wait_timeout: cycles=%lld outside [1, 2^31]", cycles);
+  int dev, st;
+  if ((st = ensure_device(&dev))) return st;
+  cudaError_t e = launch_wait_probe(cycles, (cudaStream_t)stream);
+  return e == cudaSuccess ? DICTPROJ_OK : cuda_fail(e, "selftest_wait_timeout: launch");
 }
 
 int dictproj_check(void* stream) {

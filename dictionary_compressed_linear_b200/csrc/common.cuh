@@ -56,12 +56,13 @@ __device__ __forceinline__ uint4 ld_nc_v4(const void* p) {
 __device__ __forceinline__ void prefetch_l2_bulk(const void* p, uint32_t bytes) {
   asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
 }
-// Prefetch an arbitrary byte range in chunks (rounded outward to 16 bytes).
+// Prefetch the 16-byte chunks that lie wholly inside [begin, end) of a 16-byte
+// aligned array (rounded inward, so no address outside the range is named; the
+// partial chunks at the two ends are simply not prefetched).
 __device__ __forceinline__ void prefetch_l2_range(const void* base, size_t begin, size_t end) {
-  if (end <= begin) return;
   const char* b = static_cast<const char*>(base);
-  size_t a = begin & ~size_t(15);
-  size_t e = (end + 15) & ~size_t(15);
+  size_t a = (begin + 15) & ~size_t(15);
+  size_t e = end & ~size_t(15);
   while (a < e) {
     size_t n = e - a;
     if (n > 65536) n = 65536;
@@ -206,13 +207,17 @@ __device__ __forceinline__ uint32_t lds_u16(uint32_t a) {
 // a bounded wait gave up). Each kernel file exposes a host reader for it.
 static __device__ unsigned int g_dictproj_error;
 
-// Wait for `phase` of `bar` for at most ~2^31 SM clocks; on time-out record the
+// Default limit of a bounded device wait: 2^31 SM clocks (about one second).
+constexpr long long kWaitLimitCycles = 1ll << 31;
+
+// Wait for `phase` of `bar` for at most `limit` SM clocks; on time-out record the
 // error and return false (the caller then leaves its loop).
-__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t phase) {
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t phase,
+                                                  long long limit = kWaitLimitCycles) {
   if (mbar_try_wait(bar, phase)) return true;
   const long long t0 = clock64();
   while (!mbar_try_wait(bar, phase)) {
-    if (clock64() - t0 > (1ll << 31)) {
+    if (clock64() - t0 > limit) {
       atomicOr(&g_dictproj_error, 1u);
       return false;
     }

@@ -609,6 +609,15 @@ static cudaError_t launch_pdl(const void* fn, dim3 grid, dim3 block, size_t smem
 
 int decode_mp(int M) { return M <= 1 ? 1 : M <= 2 ? 2 : M <= 4 ? 4 : 8; }
 
+// Opt-in shared memory per block of each device, recorded by prepare_decode_kernels.
+constexpr int kMaxDevices = 64;
+static int g_smem_optin[kMaxDevices];
+
+bool coeff_smem_fits(int k, int mp, int device) {
+  if (device < 0 || device >= kMaxDevices) return false;
+  return (size_t)(k + 256) * mp * sizeof(float) <= (size_t)g_smem_optin[device];
+}
+
 // Dictionary-stage grid: (k/16 tiles) x slices, each warp J units of 128
 // elements. J is the smallest count that keeps at most two CTAs per SM and
 // lets the M rows of the slice's X fit kDictXsMax bytes of shared memory;
@@ -650,6 +659,7 @@ cudaError_t prepare_decode_kernels(int device) {
   int optin = 0;
   cudaError_t e = cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, device);
   if (e != cudaSuccess) return e;
+  if (device >= 0 && device < kMaxDevices) g_smem_optin[device] = optin;
   // dynamic limit = opt-in limit minus the kernel's static shared memory
 #define SET_SMEM(fn)                                                                                  \
   {                                                                                                   \
@@ -793,6 +803,30 @@ bool gather_supported(const uint32_t* pcol_ptr, int d_out, int nseg) {
   for (int o = 0; o < d_out; ++o)
     if (pcol_ptr[o + 1] - pcol_ptr[o] > (uint32_t)(kRmax * 256)) return false;
   return true;
+}
+
+// Self-test of the bounded-wait error path: one warp waits on an mbarrier that
+// expects two arrivals and receives one, so the wait can only end by its limit
+// of `cycles` SM clocks. Nothing else is in flight when it gives up.
+__global__ void k_wait_probe(long long cycles) {
+  __shared__ __align__(8) uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 2);
+    fence_mbar_init();
+  }
+  __syncwarp();
+  if (threadIdx.x == 0) {
+    uint64_t state;
+    asm volatile("mbarrier.arrive.shared::cta.b64 %0, [%1];" : "=l"(state) : "r"(smem_u32(&bar)) : "memory");
+    (void)state;
+    mbar_wait_bounded(&bar, 0, cycles);
+  }
+  __syncwarp();
+}
+
+cudaError_t launch_wait_probe(long long cycles, cudaStream_t stream) {
+  k_wait_probe<<<1, 32, 0, stream>>>(cycles);
+  return cudaGetLastError();
 }
 
 cudaError_t take_decode_error(unsigned int* out) {

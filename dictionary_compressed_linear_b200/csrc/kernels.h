@@ -35,6 +35,11 @@ cudaError_t launch_coeff_decode_batch(int n, const dictproj_layer* const* l, con
 // Whether the gather kernel serves a layer (every column <= 1280 padded
 // entries, at most 32 segments); other layers use the direct kernel.
 bool gather_supported(const uint32_t* pcol_ptr, int d_out, int nseg);
+// Whether the coefficient kernels' shared memory, (k + 256) * mp floats of Z,
+// fits the device's per-block limit.
+bool coeff_smem_fits(int k, int mp, int device);
+// One warp whose bounded wait can only end by its limit (error-path self-test).
+cudaError_t launch_wait_probe(long long cycles, cudaStream_t stream);
 // Read and clear the device error word of the decode kernels.
 cudaError_t take_decode_error(unsigned int* out);
 

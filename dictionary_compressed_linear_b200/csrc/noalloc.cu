@@ -78,6 +78,15 @@ extern "C" int dictproj_forward_noalloc(const dictproj_device_group* group, cons
                 k, mp, kStaticZFloats);
   if (((uintptr_t)X & 15) || ((uintptr_t)Y & 15))
     return fail(DICTPROJ_ERR_ALIGN, "forward_noalloc: X and Y must be 16-byte aligned");
+  // The kernels read the packed arrays with vector loads of up to 16 bytes and
+  // prefetch them in 16-byte chunks: every array must start on a 16-byte boundary.
+  const void* arrays[] = {group->codes, group->scales, layer->col_ptr, layer->codes,
+                          layer->scales, layer->idx, layer->seg_start};
+  const char* names[] = {"group codes", "group scales", "layer col_ptr", "layer codes",
+                         "layer scales", "layer idx", "layer seg_start"};
+  for (int i = 0; i < 7; ++i)
+    if ((uintptr_t)arrays[i] & 15)
+      return fail(DICTPROJ_ERR_ALIGN, "forward_noalloc: %s must be 16-byte aligned", names[i]);
   if (!(group->s > 0.0f) || !(layer->s > 0.0f)) return fail(DICTPROJ_ERR_VALUE, "forward_noalloc: scales must be > 0");
   int dev, st;
   if ((st = ensure_device(&dev))) return st;

@@ -64,7 +64,7 @@ typedef enum dictproj_status {
   DICTPROJ_OK = 0,
   DICTPROJ_ERR_NULL = -1,        /* a required pointer is NULL */
   DICTPROJ_ERR_SHAPE = -2,       /* a size is zero, negative or not a multiple of 16 where required */
-  DICTPROJ_ERR_ALIGN = -3,       /* X or Y is not 16-byte aligned */
+  DICTPROJ_ERR_ALIGN = -3,       /* X, Y or a caller-owned packed array is not 16-byte aligned */
   DICTPROJ_ERR_MISMATCH = -4,    /* layer and group disagree on k, or live on different devices */
   DICTPROJ_ERR_RANGE = -5,       /* M outside [1, max_tokens], an atom index >= k, unsorted atoms */
   DICTPROJ_ERR_CUDA = -6,        /* a CUDA runtime call or kernel launch failed (or no device) */
@@ -86,7 +86,9 @@ typedef struct dictproj_layer dictproj_layer;
 /* dictionary, per-layer codes, scales and support.                            */
 /* ------------------------------------------------------------------------- */
 
-/* Sizes of the packed D_g arrays. d_in % 16 == 0, k >= 1. */
+/* Sizes of the packed D_g arrays. d_in % 16 == 0, k >= 1 (the host packers accept
+ * any d_in that is a multiple of 16; device groups need d_in % 32 == 0 and
+ * k % 16 == 0, see dictproj_group_upload). */
 int dictproj_group_packed_sizes(int d_in, int k, size_t* codes_bytes, size_t* scales_bytes);
 
 /* Quantise D (host fp32, d_in x k, row-major) into caller buffers of the sizes
@@ -113,6 +115,7 @@ int dictproj_pack_layer_host(const int32_t* col_ptr, const int32_t* atom_idx, co
 
 /* Upload an already packed D_g (host arrays as produced above) to the current
  * device and allocate the Z scratch for up to max_tokens tokens per call.
+ * Shapes: d_in % 32 == 0, k % 16 == 0, 1 <= k <= 65535.
  * Errors: NULL, SHAPE, RANGE (max_tokens < 1), CUDA, OOM. */
 int dictproj_group_upload(const uint8_t* codes, const uint8_t* scales, float s_D, int d_in, int k,
                           int max_tokens, dictproj_group** out);
@@ -165,8 +168,12 @@ void dictproj_free_layer(dictproj_layer* l); /* NULL is a no-op */
 
 /* Y = X * (D_g) * (C_l) (Eq. (1)): X device fp16 [M][d_in] row-major, Y device
  * fp16 [M][d_out] row-major, both 16-byte aligned; 1 <= M <= group max_tokens.
- * Accumulation is fp32; Z is fp32 for M <= 8 (decode path: CUDA-core GEMV and
- * sparse gather) and fp16 with s_D applied before rounding for larger M (prefill
+ * Accumulation is fp32; Z is fp32 for M <= 8 (decode path: the dictionary GEMV on
+ * mma.sync tensor-core instructions, then the sparse gather on CUDA cores, which
+ * stages (k + 256) * mp floats of Z in shared memory, mp = 1, 2, 4 or 8 the
+ * smallest power of two >= M; k above 57856 / 28800 / 14272 / 7008 for
+ * mp = 1 / 2 / 4 / 8 does not fit the 227 KiB per-block limit and returns
+ * UNSUPPORTED before any launch) and fp16 with s_D applied before rounding for larger M (prefill
  * path: tcgen05 GEMM on the dequantised dictionary, then the densified C_l as a
  * second tcgen05 GEMM; needs dictproj_group_reserve_prefill for d_out).
  * Asynchronous on `stream`: no allocation, no host synchronisation. Kernels are
@@ -174,7 +181,8 @@ void dictproj_free_layer(dictproj_layer* l); /* NULL is a no-op */
  * preceding work on the stream before it reads X or writes Z / Y (packed
  * weights, which nothing writes after upload, may be prefetched earlier).
  * Errors (checked before any launch): NULL, RANGE (M), MISMATCH (k or device),
- * ALIGN; CUDA if a launch fails. */
+ * ALIGN, UNSUPPORTED (k too large for the decode path's shared memory); CUDA if
+ * a launch fails. */
 int dictproj_forward(const void* X, int M, const dictproj_layer* layer,
                      const dictproj_group* group, void* Y, void* stream);
 
@@ -221,7 +229,9 @@ int dictproj_dictionary_stage_prefill(const void* X, int M, const dictproj_group
 
 /* Caller-owned device copies of packed factors (the arrays produced by
  * dictproj_pack_group_host / dictproj_pack_layer_host, copied to the device by
- * the caller). All pointers are device pointers; the library only reads them. */
+ * the caller). All pointers are device pointers, each 16-byte aligned (the
+ * kernels use 16-byte vector loads and 16-byte L2 prefetches); the library only
+ * reads them. */
 typedef struct dictproj_device_group {
   const uint8_t* codes;   /* [k][d_in/2] */
   const uint8_t* scales;  /* [k][d_in/16] */
@@ -252,7 +262,8 @@ typedef struct dictproj_device_layer {
  * (cudaGetSymbolAddress); make that first call before any stream capture. All
  * calls share the array: calls that overlap on the GPU race and must be
  * serialised by the caller. X fp16 [M][d_in], Y fp16 [M][d_out], both device,
- * 16-byte aligned. Errors: NULL, SHAPE, MISMATCH, RANGE, ALIGN, VALUE, CUDA. */
+ * 16-byte aligned. Errors: NULL, SHAPE, MISMATCH, RANGE, ALIGN (X, Y or any packed
+ * array not 16-byte aligned), VALUE, CUDA. */
 int dictproj_forward_noalloc(const dictproj_device_group* group, const dictproj_device_layer* layer,
                              const void* X, int M, void* Y, void* stream);
 
@@ -305,6 +316,15 @@ int dictproj_layer_load(const char* path, dictproj_layer** out);
 /* Read (and clear) the device error word that bounded device waits set, after
  * synchronising `stream`. Returns OK or TIMEOUT (or CUDA). */
 int dictproj_check(void* stream);
+
+/* Self-test of the bounded-wait error path (diagnostic; no counterpart in the
+ * paper). Launches one warp on `stream` that waits on an mbarrier which can never
+ * complete, with a limit of `cycles` SM clocks (1 <= cycles <= 2^31). The wait
+ * gives up at the limit, sets the device error word and the kernel returns; no
+ * copy or tensor-core operation is in flight. A following dictproj_check(stream)
+ * then returns DICTPROJ_ERR_TIMEOUT and clears the word; the device stays usable.
+ * Errors: RANGE (cycles), UNSUPPORTED (not sm_100), CUDA. */
+int dictproj_selftest_wait_timeout(long long cycles, void* stream);
 
 /* Last error message of the calling thread ("" if none). */
 const char* dictproj_last_error(void);

@@ -143,6 +143,26 @@ def sampled_outputs(X: np.ndarray, pd: dict, pc: dict, rows, cols) -> np.ndarray
     return out
 
 
+def sampled_outputs_rows(X: np.ndarray, pd: dict, pc: dict, rows, cols) -> np.ndarray:
+    """Y[rows, cols] in the two-stage order of Eq. (1), restricted to what the
+    samples need: Z = X[r] D-hat for each distinct sampled token row r (fp64),
+    then for each sample the column's stored entries, sum of Z[r, atom] * value."""
+    rows = np.asarray(rows, np.int64)
+    cols = np.asarray(cols, np.int64)
+    Dhat = decode_dictionary(pd)
+    atoms, vals = decode_coeff_entries(pc)
+    ptr = pc["col_ptr"].astype(np.int64)
+    urows, inv = np.unique(rows, return_inverse=True)
+    Z = np.asarray(X)[urows].astype(np.float64) @ Dhat
+    out = np.zeros(rows.size)
+    for n in range(rows.size):
+        o = cols[n]
+        a = atoms[ptr[o]:ptr[o + 1]]
+        v = vals[ptr[o]:ptr[o + 1]]
+        out[n] = float(Z[inv[n], a] @ v)
+    return out
+
+
 def within_tolerance(y_test: np.ndarray, y_ref: np.ndarray, rel_fro: float = 5e-3,
                      elem: float = 1e-2):
     """The parity bar: relative Frobenius error <= 5e-3 and every element
@@ -164,6 +184,6 @@ def within_tolerance(y_test: np.ndarray, y_ref: np.ndarray, rel_fro: float = 5e-
 __all__ = [
     "SEG", "decode_dictionary", "decode_coeff_entries", "decode_coeff_dense", "expand_weight",
     "forward_dense", "sparse_columns_product", "forward_factored", "forward_reference",
-    "forward_brute", "sampled_outputs", "within_tolerance", "decode_projection",
+    "forward_brute", "sampled_outputs", "sampled_outputs_rows", "within_tolerance", "decode_projection",
     "forward_factored_decoded",
 ]

@@ -4,6 +4,7 @@ The path has no collective: ranks run independent replicas of the decode step
 and only the timing is combined (max over ranks). These tests run two gloo ranks
 as child processes on 127.0.0.1."""
 import os
+import time
 import socket
 import subprocess
 import sys
@@ -70,9 +71,11 @@ def test_reference_arm_on_a_nonzero_rank_does_nothing():
 
 def test_reference_arm_prints_one_json_line_with_the_contract_keys():
     import json
+    t0 = time.time()
     r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--steps", "7",
-                        "--warmup", "3"], env=dict(os.environ, RANK="0", WORLD_SIZE="1"), capture_output=True,
-                       text=True, timeout=600)
+                        "--warmup", "3", "--ref-budget", "6"], env=dict(os.environ, RANK="0", WORLD_SIZE="1"),
+                       capture_output=True, text=True, timeout=600)
+    wall = time.time() - t0
     assert r.returncode == 0, r.stderr
     lines = [l for l in r.stdout.splitlines() if l.strip()]
     assert len(lines) == 1
@@ -84,6 +87,10 @@ def test_reference_arm_prints_one_json_line_with_the_contract_keys():
     assert d["value"] > 0 and d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["value"] == d["value"]
     assert d["e2e"] == {"value": d["value"], "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
     assert d["metric"] == bench.METRIC
+    # the line describes what was timed: its steps fit the run, and it names the GPU arm's workload
+    assert d["ms_per_step"] * d["steps"] / 1e3 <= wall
+    wl = bench.synth.full_step(n_layers=32)
+    assert d["config"] == bench.step_config(wl, 32, 1, 1)
 
 
 def test_bench_refuses_fewer_than_three_warmup_steps():

@@ -253,3 +253,80 @@ def test_columns_longer_than_1024_entries(M):
     assert int(np.diff(pc["col_ptr"]).max()) > 1024
     X = synth.gen_activations(18, 0, 0, M, 512)
     assert_parity(run_forward(g, l, X), oracle_forward(X, pd, pc), f"long columns M={M}")
+
+
+# ------------------------------------------------------------------ layers the gather kernel does not hold
+@pytest.mark.parametrize("M", [1, 3, 8])
+def test_columns_longer_than_1280_entries(M):
+    # k = 3072 at density 0.9 stores 2765 entries per column (2768 padded),
+    # beyond the gather kernel's 1280; dictproj_forward routes the layer to the
+    # direct coefficient kernel
+    D, C = _case(19, 0, 0, 0, 256, 3072, 64, 0.9)
+    g, l = device_projection(D, C, max_tokens=8)
+    pd, pc = oracle_projection(D, C)
+    assert int(np.diff(pc["col_ptr"]).max()) > 1280
+    X = synth.gen_activations(19, 0, 0, M, 256)
+    assert_parity(run_forward(g, l, X), oracle_forward(X, pd, pc), f"columns > 1280 entries M={M}")
+
+
+@pytest.mark.parametrize("M", [1, 3, 4])
+def test_more_than_32_segments(M):
+    # k = 8448 has 33 segments of 256 atoms (the gather holds at most 32): the
+    # layer runs on the direct coefficient kernel
+    D, C = _case(20, 0, 0, 0, 256, 8448, 64, 0.05)
+    g, l = device_projection(D, C, max_tokens=8)
+    pd, pc = oracle_projection(D, C)
+    assert pc["nseg"] == 33
+    X = synth.gen_activations(20, 0, 0, M, 256)
+    assert_parity(run_forward(g, l, X), oracle_forward(X, pd, pc), f"33 segments M={M}")
+
+
+def test_k_beyond_shared_memory_is_rejected_before_launch():
+    # (k + 256) * 8 floats of Z exceed the per-block shared memory at M = 8 for
+    # k = 8192: UNSUPPORTED, nothing launched; k = 7008 is the largest that fits
+    D, C = _case(21, 0, 0, 0, 64, 8192, 32, 0.02)
+    g, l = device_projection(D, C, max_tokens=8)
+    X = torch.zeros((8, 64), dtype=torch.float16, device="cuda")
+    Y = torch.full((8, 32), 3.0, dtype=torch.float16, device="cuda")
+    st = torch.cuda.current_stream().cuda_stream
+    assert dp.dictproj_forward_status(X.data_ptr(), 8, l.handle, g.handle, Y.data_ptr(), st) == -9
+    assert "shared memory" in dp.dictproj_last_error()
+    torch.cuda.synchronize()
+    assert torch.all(Y == 3.0)
+    assert dp.dictproj_forward_status(X.data_ptr(), 4, l.handle, g.handle, Y.data_ptr(), st) == 0
+    torch.cuda.synchronize()
+    assert torch.all(Y[:4] == 0.0)
+
+
+@pytest.mark.parametrize("M", [1, 8])
+def test_largest_k_that_fits_at_m8(M):
+    D, C = _case(22, 0, 0, 0, 64, 7008, 48, 0.05)
+    g, l = device_projection(D, C, max_tokens=8)
+    pd, pc = oracle_projection(D, C)
+    X = synth.gen_activations(22, 0, 0, M, 64)
+    assert_parity(run_forward(g, l, X), oracle_forward(X, pd, pc), f"k=7008 M={M}")
+
+
+# ------------------------------------------------------------------ partial 128-element units of d_in
+@pytest.mark.parametrize("d_in", [160, 4128])
+@pytest.mark.parametrize("M", [1, 3, 8])
+def test_decode_d_in_not_a_multiple_of_128(d_in, M):
+    D, C = _case(23, 0, 0, 0, d_in, 512, 200, 0.3)
+    g, l = device_projection(D, C, max_tokens=8)
+    pd, pc = oracle_projection(D, C)
+    X = synth.gen_activations(23, 0, 0, M, d_in)
+    assert_parity(run_forward(g, l, X), oracle_forward(X, pd, pc, dense=True), f"d_in={d_in} M={M}")
+
+
+# ------------------------------------------------------------------ bounded waits
+def test_bounded_wait_times_out_and_the_device_stays_usable(mid):
+    g, l, pd, pc = mid
+    st = torch.cuda.current_stream().cuda_stream
+    assert dp.dictproj_check_status(st) == 0
+    dp.dictproj_selftest_wait_timeout(1 << 20, st)  # ~0.5 ms at 2 GHz; nothing can complete the wait
+    assert dp.dictproj_check_status(st) == -8
+    assert "gave up" in dp.dictproj_last_error()
+    assert dp.dictproj_check_status(st) == 0  # the word was cleared
+    X = synth.gen_activations(10, 77, 0, 2, 512)
+    assert_parity(run_forward(g, l, X), oracle_forward(X, pd, pc, dense=True), "after a timeout")
+    assert dp.dictproj_check_status(st) == 0

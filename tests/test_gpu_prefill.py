@@ -132,3 +132,28 @@ def test_prefill_in_cuda_graph():
     torch.cuda.synchronize()
     assert_parity(Y.float().cpu().numpy().astype(np.float64), oracle_forward(X_np, pd, pc), "graph replay")
     del graph
+
+
+@pytest.mark.parametrize("M", [128, 512, 2048])
+@pytest.mark.parametrize("name", ["q", "gate", "down"])
+def test_benchmarked_prefill_configurations(name, M):
+    """Exactly the inputs and launch configuration bench.py times for the prefill
+    leg (same seeds, same M, so the same token-tile width per shape), checked on
+    4000 sampled outputs: 16 token rows (first and last included) x 250 columns."""
+    import bench
+    D, C, X = bench.prefill_inputs(name, M)
+    pg = dp.dictproj_pack_group_host(D)
+    pc = dp.dictproj_pack_layer_host(C.col_ptr, C.atom_idx, C.vals, C.k, C.d_out)
+    g = dp.dictproj_group_upload(pg, M)
+    dp.dictproj_group_reserve_prefill(g, C.d_out)
+    l = dp.dictproj_layer_upload(pc)
+    y = run_forward(g, l, X)
+    assert np.all(np.isfinite(y))
+    pd_o, pc_o = oracle_projection(D, C)
+    rng = np.random.default_rng(1000 + M)
+    trows = np.unique(np.concatenate([[0, M - 1], rng.choice(M, 14, replace=False)]))
+    rows = np.repeat(trows, 250)
+    cols = np.concatenate([np.concatenate([[0, C.d_out - 1], rng.choice(C.d_out, 248, replace=False)])
+                           for _ in trows])
+    ref = F.sampled_outputs_rows(X, pd_o, pc_o, rows, cols)
+    assert_parity(y[rows, cols], ref, f"bench prefill {name} M={M}")

@@ -158,3 +158,24 @@ def test_device_calls_fail_loudly_without_gpu(dp):
     with pytest.raises(DictprojError) as e:
         dp.dictproj_pack_group(np.ones((32, 16), np.float32), 1)
     assert e.value.status == -6
+
+
+def test_noalloc_and_selftest_validate_before_any_device_call(dp):
+    # fake (never dereferenced) device addresses: validation rejects the call on
+    # the host, before any CUDA call, so this runs without a GPU
+    base = 1 << 40
+    g = dp.DeviceGroup(base, base + 4096, 1.0, 64, 32)
+    l = dp.DeviceLayer(base + 8192, base + 12288, base + 16384, base + 20480, base + 24576, 1.0, 32, 16)
+    for field in ("codes", "scales"):
+        gg = dp.DeviceGroup(base, base + 4096, 1.0, 64, 32)
+        setattr(gg, field, getattr(gg, field) + 8)
+        assert dp.dictproj_forward_noalloc_status(gg, l, base + 28672, 1, base + 32768, 0) == -3
+        assert "16-byte aligned" in dp.dictproj_last_error()
+    for field in ("col_ptr", "codes", "scales", "idx", "seg_start"):
+        ll = dp.DeviceLayer(base + 8192, base + 12288, base + 16384, base + 20480, base + 24576, 1.0, 32, 16)
+        setattr(ll, field, getattr(ll, field) + 2)
+        assert dp.dictproj_forward_noalloc_status(g, ll, base + 28672, 1, base + 32768, 0) == -3
+        assert field in dp.dictproj_last_error()
+    lib = dp.lib()
+    assert lib.dictproj_selftest_wait_timeout(0, None) == -5
+    assert lib.dictproj_selftest_wait_timeout((1 << 31) + 1, None) == -5

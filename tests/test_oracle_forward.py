@@ -128,6 +128,17 @@ def test_sampled_outputs_match_full():
     assert np.allclose(got, y[rows, cols], rtol=1e-12, atol=1e-12)
 
 
+def test_sampled_outputs_by_rows_match_dense_product():
+    # pinned to the dense X (D C) product, a different association of Eq. (1),
+    # with repeated rows, an out-of-order row list and more than one segment
+    X, pd, pc = _tiny_case(M=5, d_in=64, k=288, d_out=24, rho=0.4)
+    y = F.forward_reference(X, pd, pc)
+    rows = [4, 0, 1, 4, 2, 3, 0, 4]
+    cols = [23, 0, 5, 7, 19, 11, 13, 0]
+    got = F.sampled_outputs_rows(X, pd, pc, rows, cols)
+    assert np.allclose(got, y[rows, cols], rtol=1e-12, atol=1e-12)
+
+
 def test_tolerance_helper_flags_errors():
     y = np.linspace(-3, 3, 100)
     assert F.within_tolerance(y * (1 + 1e-4), y)[0]

@@ -2,7 +2,8 @@
 allocate device memory at call time (runtimes that reserve all device memory
 up front in their own arena; work enqueued while a stream is being captured
 into a CUDA graph). It keeps the Z scratch in a file-scope device array instead
-of allocating, and must give the same result as dictproj_forward.
+of allocating, and must match the fp64 oracle (and dictproj_forward) on two
+calls in a row.
 
 The test itself allocates its inputs and outputs with torch; only the entry
 point under test must not allocate. Collected last on purpose."""
@@ -18,7 +19,8 @@ if not torch.cuda.is_available():  # pragma: no cover
     pytest.skip("needs a CUDA device", allow_module_level=True)
 
 import dictionary_compressed_linear_b200 as dp  # noqa: E402
-from oracle.forward import within_tolerance  # noqa: E402
+from oracle.forward import forward_factored, within_tolerance  # noqa: E402
+from oracle.pack import pack_coeff, pack_dictionary  # noqa: E402
 
 
 def _device_views(pg, pc):
@@ -38,19 +40,22 @@ def _device_views(pg, pc):
     return g, l, keep
 
 
-@pytest.mark.parametrize("d_in,k,d_out,rho,M", [(4096, 2048, 4096, 0.3, 1), (4096, 2048, 4096, 0.3, 8),
-                                                (11008, 3072, 4096, 0.25, 3), (256, 128, 256, 0.5, 4)])
-def test_noalloc_matches_forward_twice(d_in, k, d_out, rho, M):
+@pytest.mark.parametrize("d_in,k,d_out,rho,M", [
+    (4096, 2048, 4096, 0.3, 1), (4096, 2048, 4096, 0.3, 8),  # attention projection
+    (11008, 3072, 4096, 0.25, 3),                             # down projection
+    (256, 128, 256, 0.5, 4),                                  # tiny shape
+    (256, 3072, 64, 0.9, 1),                                  # columns of 2768 padded entries
+    (256, 8448, 64, 0.05, 2),                                 # 33 segments of 256 atoms
+])
+def test_noalloc_matches_oracle_and_forward_twice(d_in, k, d_out, rho, M):
     D = synth.gen_dictionary(30, 0, 0, d_in, k)
     C = synth.gen_coeff(30, 0, 0, 0, k, d_out, rho)
     pg = dp.dictproj_pack_group_host(D)
     pc = dp.dictproj_pack_layer_host(C.col_ptr, C.atom_idx, C.vals, k, d_out)
-    g_ref = dp.dictproj_group_upload(pg, 8)
-    l_ref = dp.dictproj_layer_upload(pc)
-    X = torch.from_numpy(synth.gen_activations(30, 0, 0, M, d_in)).cuda()
+    X_np = synth.gen_activations(30, 0, 0, M, d_in)
+    X = torch.from_numpy(X_np).cuda()
     st = torch.cuda.current_stream().cuda_stream
-    Y_ref = torch.empty((M, d_out), dtype=torch.float16, device="cuda")
-    dp.dictproj_forward(X.data_ptr(), M, l_ref, g_ref, Y_ref.data_ptr(), st)
+    ref = forward_factored(X_np, pack_dictionary(D), pack_coeff(C.col_ptr, C.atom_idx, C.vals, k, d_out))
     g, l, keep = _device_views(pg, pc)
     outs = []
     for _ in range(2):  # two calls in a row share the static scratch
@@ -58,11 +63,18 @@ def test_noalloc_matches_forward_twice(d_in, k, d_out, rho, M):
         dp.dictproj_forward_noalloc(g, l, X.data_ptr(), M, Y.data_ptr(), st)
         torch.cuda.synchronize()
         outs.append(Y.float().cpu().numpy().astype(np.float64))
-    ref = Y_ref.float().cpu().numpy().astype(np.float64)
     for y in outs:
         ok, rf, worst = within_tolerance(y, ref)
         assert ok, (rf, worst)
     assert np.array_equal(outs[0], outs[1])
+    # and the allocating entry point agrees with it
+    g_ref = dp.dictproj_group_upload(pg, 8)
+    l_ref = dp.dictproj_layer_upload(pc)
+    Y_ref = torch.empty((M, d_out), dtype=torch.float16, device="cuda")
+    dp.dictproj_forward(X.data_ptr(), M, l_ref, g_ref, Y_ref.data_ptr(), st)
+    torch.cuda.synchronize()
+    ok, rf, worst = within_tolerance(outs[0], Y_ref.float().cpu().numpy().astype(np.float64))
+    assert ok, (rf, worst)
 
 
 def test_noalloc_rejects_sizes_beyond_the_static_scratch():
@@ -73,7 +85,8 @@ def test_noalloc_rejects_sizes_beyond_the_static_scratch():
     pg = dp.dictproj_pack_group_host(D)
     pc = dp.dictproj_pack_layer_host(C.col_ptr, C.atom_idx, C.vals, k, d_out)
     g, l, keep = _device_views(pg, pc)
-    X = torch.zeros((8, d_in), dtype=torch.float16, device="cuda")
+    X_np = synth.gen_activations(31, 0, 0, 8, d_in)
+    X = torch.from_numpy(X_np).cuda()
     Y = torch.full((8, d_out), 3.0, dtype=torch.float16, device="cuda")
     st = torch.cuda.current_stream().cuda_stream
     assert dp.dictproj_forward_noalloc_status(g, l, X.data_ptr(), 8, Y.data_ptr(), st) == -5
@@ -82,4 +95,7 @@ def test_noalloc_rejects_sizes_beyond_the_static_scratch():
     assert torch.all(Y == 3.0)
     assert dp.dictproj_forward_noalloc_status(g, l, X.data_ptr(), 1, Y.data_ptr(), st) == 0
     torch.cuda.synchronize()
-    assert torch.all(Y[0] == 0.0)
+    ref = forward_factored(X_np[:1], pack_dictionary(D), pack_coeff(C.col_ptr, C.atom_idx, C.vals, k, d_out))
+    ok, rf, worst = within_tolerance(Y[:1].float().cpu().numpy().astype(np.float64), ref)
+    assert ok, (rf, worst)
+    assert torch.all(Y[1:] == 3.0)
