@@ -35,6 +35,32 @@ def decode_coeff_entries(pc: dict):
     return coeff_entry_atoms(pc), vals
 
 
+def decode_coeff_bitmap_entries(pb: dict):
+    """(atoms int64, values fp64) of the stored entries of a bitmap-indexed C_l;
+    padding entries (no bit) get atom -1 and value 0."""
+    from .pack import bitmap_entry_atoms
+    codes = unpack_nibbles(pb["codes"])
+    sc = np.repeat(np.asarray(pb["scales"]), 16)
+    vals = E2M1_TABLE[codes] * E4M3_TABLE[sc] * float(pb["s"])
+    atoms = bitmap_entry_atoms(pb)
+    return atoms, np.where(atoms >= 0, vals, 0.0)
+
+
+def forward_factored_bitmap(X: np.ndarray, pd: dict, pb: dict) -> np.ndarray:
+    """(X D) C in fp64 with C in the bitmap index format: Y[:, o] = sum over the
+    column's set bits j, in order, of Z[:, j] times the j-th stored value."""
+    Z = np.asarray(X).astype(np.float64) @ decode_dictionary(pd)
+    atoms, vals = decode_coeff_bitmap_entries(pb)
+    ptr = pb["col_ptr"].astype(np.int64)
+    Y = np.zeros((Z.shape[0], pb["d_out"]), dtype=np.float64)
+    for o in range(pb["d_out"]):
+        a = atoms[ptr[o]:ptr[o + 1]]
+        v = vals[ptr[o]:ptr[o + 1]]
+        keep = a >= 0
+        Y[:, o] = Z[:, a[keep]] @ v[keep]
+    return Y
+
+
 def decode_coeff_dense(pc: dict) -> np.ndarray:
     """C-hat as a dense fp64 (k, d_out) matrix, zeros off the support."""
     k, d_out = pc["k"], pc["d_out"]
@@ -185,5 +211,5 @@ __all__ = [
     "SEG", "decode_dictionary", "decode_coeff_entries", "decode_coeff_dense", "expand_weight",
     "forward_dense", "sparse_columns_product", "forward_factored", "forward_reference",
     "forward_brute", "sampled_outputs", "sampled_outputs_rows", "within_tolerance", "decode_projection",
-    "forward_factored_decoded",
+    "forward_factored_decoded", "decode_coeff_bitmap_entries", "forward_factored_bitmap",
 ]

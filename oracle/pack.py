@@ -28,6 +28,11 @@ Coefficients C_l (k x d_out, column-compressed per output channel):
     to the column start, of the first entry whose atom is >= 256*s.  The atom of
     entry q is 256*s(q) + idx with s(q) = max{s : seg_start[s] <= q}; padding
     entries therefore sit in the last segment (atom 256*(nseg-1) < k).
+
+Bitmap-indexed C_l (pack_coeff_bitmap): the same values, codes, scales and
+padding; the index is one bit per logical position instead (Eq. (12), a = 0,
+h = 1): bitmap uint32[d_out][ceil(k/32)], bit j % 32 of word j // 32 of row o set
+iff atom j is retained in column o.
 """
 from __future__ import annotations
 
@@ -119,6 +124,54 @@ def pack_coeff(col_ptr: np.ndarray, atom_idx: np.ndarray, vals: np.ndarray, k: i
         "seg_start": seg_start.astype(np.uint16).reshape(-1),  # d_out * nseg
         "s": np.float32(s_c),
     }
+
+
+def pack_coeff_bitmap(col_ptr: np.ndarray, atom_idx: np.ndarray, vals: np.ndarray, k: int,
+                      d_out: int) -> dict:
+    """C_l with a bitmap support index: the review's Eq. (12) case a = 0, h = 1
+    ("From retained values to measured decoding": one bit per logical position,
+    no per-value index bits).
+
+    The stored values, their padding, blocks, codes, scales and s_C are exactly
+    those of pack_coeff (the index format does not change what is quantised).
+    In place of idx and seg_start each column o has a bitmap of k bits,
+    uint32[d_out][ceil(k/32)]: bit (j mod 32) of word j // 32 is set iff atom j
+    is retained in column o. Its set bits, in ascending order, are the column's
+    stored entries in storage order; padding entries have no bit."""
+    pc = pack_coeff(col_ptr, atom_idx, vals, k, d_out)
+    col_ptr = np.asarray(col_ptr, dtype=np.int64)
+    atom_idx = np.asarray(atom_idx, dtype=np.int64)
+    words = -(-k // 32)
+    mask = np.zeros((d_out, words * 32), dtype=bool)  # mask[o, j]: atom j retained in column o
+    mask[np.repeat(np.arange(d_out), np.diff(col_ptr)), atom_idx] = True
+    weights = np.uint64(1) << np.arange(32, dtype=np.uint64)  # bit b of a word has weight 2^b
+    bitmap = (mask.reshape(d_out, words, 32).astype(np.uint64) * weights).sum(axis=2).astype(np.uint32)
+    return {
+        "k": k,
+        "d_out": d_out,
+        "words": words,
+        "col_ptr": pc["col_ptr"],
+        "nnz": pc["nnz"],
+        "codes": pc["codes"],
+        "scales": pc["scales"],
+        "bitmap": bitmap.reshape(-1),  # d_out * ceil(k/32)
+        "s": pc["s"],
+    }
+
+
+def bitmap_entry_atoms(pb: dict) -> np.ndarray:
+    """Atom of every stored entry of a bitmap-indexed C_l (padding entries: -1):
+    the j-th stored entry of a column is the column's j-th set bit."""
+    d_out, words = pb["d_out"], pb["words"]
+    ptr = pb["col_ptr"].astype(np.int64)
+    bm = pb["bitmap"].reshape(d_out, words)
+    bits = (bm[:, :, None].astype(np.uint64) >> np.arange(32, dtype=np.uint64)) & np.uint64(1)
+    mask = bits.reshape(d_out, words * 32).astype(bool)  # mask[o, j]: bit j of row o
+    atoms = np.full(int(ptr[-1]), -1, dtype=np.int64)
+    for o in range(d_out):
+        set_bits = np.flatnonzero(mask[o])
+        atoms[ptr[o]:ptr[o] + set_bits.size] = set_bits
+    return atoms
 
 
 def coeff_entry_atoms(pc: dict) -> np.ndarray:
