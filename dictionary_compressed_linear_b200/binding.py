@@ -58,6 +58,8 @@ SIGNATURES = [
     ("dictproj_layer_packed_entries", C.c_int, [_i32p, C.c_int, C.c_int, _szp]),
     ("dictproj_pack_layer_host", C.c_int,
      [_i32p, _i32p, _f32p, C.c_int, C.c_int, _u32p, _u32p, _u8p, _u8p, _u8p, _u16p, _f32p]),
+    ("dictproj_pack_layer_bitmap_host", C.c_int,
+     [_i32p, _i32p, _f32p, C.c_int, C.c_int, _u32p, _u32p, _u8p, _u8p, _u32p, _f32p]),
     ("dictproj_group_upload", C.c_int,
      [_u8p, _u8p, C.c_float, C.c_int, C.c_int, C.c_int, C.POINTER(C.c_void_p)]),
     ("dictproj_pack_group", C.c_int, [_f32p, C.c_int, C.c_int, C.c_int, C.POINTER(C.c_void_p)]),
@@ -80,6 +82,8 @@ SIGNATURES = [
     ("dictproj_forward_batch", C.c_int,
      [C.c_int, C.POINTER(C.c_void_p), C.c_int, C.POINTER(C.c_void_p), C.POINTER(C.c_void_p),
       C.POINTER(C.c_void_p), C.c_void_p]),
+    ("dictproj_launch_count", C.c_int,
+     [C.c_int, C.POINTER(C.c_void_p), C.c_int, C.POINTER(C.c_void_p), C.POINTER(C.c_void_p), _intp]),
     ("dictproj_dictionary_stage", C.c_int, [C.c_void_p, C.c_int, C.c_void_p, C.c_void_p, C.c_void_p]),
     ("dictproj_coefficient_stage", C.c_int, [C.c_void_p, C.c_int, C.c_void_p, C.c_void_p, C.c_void_p]),
     ("dictproj_dictionary_stage_prefill", C.c_int, [C.c_void_p, C.c_int, C.c_void_p, C.c_void_p, C.c_void_p]),
@@ -191,6 +195,27 @@ def dictproj_pack_layer_host(col_ptr, atom_idx, vals, k: int, d_out: int) -> dic
         _ptr(out["scales"], C.c_uint8), _ptr(out["idx"], C.c_uint8), _ptr(out["seg_start"], C.c_uint16),
         C.byref(s)))
     out.update(k=k, d_out=d_out, nseg=nseg, s=np.float32(s.value))
+    return out
+
+
+def dictproj_pack_layer_bitmap_host(col_ptr, atom_idx, vals, k: int, d_out: int) -> dict:
+    """C_l with the bitmap support index (Eq. (12), a = 0, h = 1)."""
+    col_ptr = np.ascontiguousarray(col_ptr, dtype=np.int32)
+    atom_idx = np.ascontiguousarray(atom_idx, dtype=np.int32)
+    vals = np.ascontiguousarray(vals, dtype=np.float32)
+    total = dictproj_layer_packed_entries(col_ptr, k, d_out)
+    words = -(-k // 32)
+    out = {
+        "col_ptr": np.zeros(d_out + 1, np.uint32), "nnz": np.zeros(d_out, np.uint32),
+        "codes": np.zeros(total // 2, np.uint8), "scales": np.zeros(total // 16, np.uint8),
+        "bitmap": np.zeros(d_out * words, np.uint32),
+    }
+    s = C.c_float()
+    _check(lib().dictproj_pack_layer_bitmap_host(
+        _ptr(col_ptr, C.c_int32), _ptr(atom_idx, C.c_int32), _ptr(vals, C.c_float), k, d_out,
+        _ptr(out["col_ptr"], C.c_uint32), _ptr(out["nnz"], C.c_uint32), _ptr(out["codes"], C.c_uint8),
+        _ptr(out["scales"], C.c_uint8), _ptr(out["bitmap"], C.c_uint32), C.byref(s)))
+    out.update(k=k, d_out=d_out, words=words, s=np.float32(s.value))
     return out
 
 
@@ -475,3 +500,14 @@ def dictproj_check_status(stream: int = 0) -> int:
 
 def dictproj_selftest_wait_timeout(cycles: int, stream: int = 0):
     _check(lib().dictproj_selftest_wait_timeout(int(cycles), C.c_void_p(stream)))
+
+
+def dictproj_launch_count(X_ptrs, M: int, layers, groups) -> int:
+    """Kernels one forward call (a batch of len(layers) projections) launches."""
+    n = len(layers)
+    arr = C.c_void_p * n
+    cnt = C.c_int()
+    _check(lib().dictproj_launch_count(n, arr(*[C.c_void_p(int(x)) for x in X_ptrs]), M,
+                                       arr(*[l.handle for l in layers]), arr(*[g.handle for g in groups]),
+                                       C.byref(cnt)))
+    return cnt.value

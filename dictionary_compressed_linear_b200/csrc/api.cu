@@ -1,6 +1,7 @@
 // C ABI of libdictproj: validation, handles, uploads and forward dispatch.
 // Every entry point validates its arguments before touching the device and
 // reports failures through a status code plus a thread-local message.
+#include <algorithm>
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
@@ -67,6 +68,7 @@ int ensure_device(int* dev_out) {
                   prop.major, prop.minor);
     if ((e = prepare_decode_kernels(dev)) != cudaSuccess) return cuda_fail(e, "kernel set-up");
     if ((e = prepare_prefill_kernels(dev)) != cudaSuccess) return cuda_fail(e, "prefill kernel set-up");
+    if ((e = prepare_fused_kernels(dev)) != cudaSuccess) return cuda_fail(e, "fused kernel set-up");
     g_dev_ready[dev] = 1;
   }
   *dev_out = dev;
@@ -134,6 +136,13 @@ int dictproj_pack_layer_host(const int32_t* col_ptr, const int32_t* atom_idx, co
   return pack_layer_host(col_ptr, atom_idx, vals, k, d_out, pcol_ptr, nnz, codes, scales, idx, seg_start, s_C);
 }
 
+int dictproj_pack_layer_bitmap_host(const int32_t* col_ptr, const int32_t* atom_idx, const float* vals, int k,
+                                    int d_out, uint32_t* pcol_ptr, uint32_t* nnz, uint8_t* codes, uint8_t* scales,
+                                    uint32_t* bitmap, float* s_C) {
+  clear_error();
+  return pack_layer_bitmap_host(col_ptr, atom_idx, vals, k, d_out, pcol_ptr, nnz, codes, scales, bitmap, s_C);
+}
+
 void dictproj_free_group(dictproj_group* g) {
   if (!g) return;
   cudaFree(g->codes);
@@ -142,6 +151,9 @@ void dictproj_free_group(dictproj_group* g) {
   cudaFree(g->z16);
   cudaFree(g->cdense);
   cudaFree(g->err);
+  cudaFree(g->scales_pad);
+  cudaFree(g->zx);
+  cudaFree(g->fsync);
   delete g;
 }
 
@@ -152,6 +164,8 @@ void dictproj_free_layer(dictproj_layer* l) {
   cudaFree(l->scales);
   cudaFree(l->idx);
   cudaFree(l->seg_start);
+  cudaFree(l->cplan_off);
+  cudaFree(l->cplan);
   delete l;
 }
 
@@ -199,6 +213,12 @@ int dictproj_group_upload(const uint8_t* codes, const uint8_t* scales, float s_D
   if ((e = encode_dict_codes_map(g, &g->codes_map)) != cudaSuccess) {
     dictproj_free_group(g);
     return cuda_fail(e, "group_upload: tensor map of the dictionary codes");
+  }
+  bool fused = false;
+  if (fault("alloc") || (e = fused_group_setup(g, &fused)) != cudaSuccess) {
+    dictproj_free_group(g);
+    cudaGetLastError();
+    return fail(DICTPROJ_ERR_OOM, "group_upload: fused decode buffers (%s)", cudaGetErrorName(e));
   }
   *out = g;
   return DICTPROJ_OK;
@@ -312,6 +332,27 @@ int dictproj_layer_upload(const uint32_t* pcol_ptr, const uint8_t* codes, const 
   }
   l->n_sm = n_sm;
   l->gather_ok = gather_supported(pcol_ptr, d_out, nseg);
+  {  // column chunks of the fused decode kernel
+    std::vector<uint32_t> off;
+    std::vector<uint4> chunks;
+    int maxc = 0;
+    l->fused_ok = fused_layer_plan(pcol_ptr, d_out, nseg, n_sm, off, chunks, &maxc);
+    l->cplan_max = maxc;
+    if (l->fused_ok) {
+      if ((e = dmalloc((void**)&l->cplan_off, off.size() * sizeof(uint32_t))) ||
+          (e = dmalloc((void**)&l->cplan, std::max<size_t>(1, chunks.size()) * sizeof(uint4)))) {
+        dictproj_free_layer(l);
+        cudaGetLastError();
+        return fail(DICTPROJ_ERR_OOM, "layer_upload: device allocation failed (%s)", cudaGetErrorName(e));
+      }
+      if ((e = h2d(l->cplan_off, off.data(), off.size() * sizeof(uint32_t))) ||
+          (e = h2d(l->cplan, chunks.data(), chunks.size() * sizeof(uint4)))) {
+        dictproj_free_layer(l);
+        cudaGetLastError();
+        return cuda_fail(e, "layer_upload: copy to device");
+      }
+    }
+  }
   // the true entry count is not part of the packed arrays; dictproj_pack_layer records it
   l->nnz_total = 0;
   *out = l;
@@ -461,6 +502,12 @@ int dictproj_forward_path(const void* X, int M, const dictproj_layer* layer, con
   const DictPlan plan = dict_plan(group->d_in, group->k, group->n_sm, M < kDecodeMaxTokens ? M : kDecodeMaxTokens, false);
   if (decode) {
     const int mp = decode_mp(M);
+    FusedLaunchPlan fp;
+    if (fused_plan_launch(1, &group, &layer, &x, M, smem_optin_of(dev), &fp)) {
+      if ((e = launch_fused(1, &group, &layer, &x, &y, M, fp, kWaitLimitCycles, s)) != cudaSuccess)
+        return cuda_fail(e, "forward: fused decode launch");
+      return DICTPROJ_OK;
+    }
     if (!coeff_smem_fits(group->k, mp, dev))
       return fail(DICTPROJ_ERR_UNSUPPORTED,
                   "forward: the decode path stages (k + 256) * %d floats of Z in shared memory; k=%d does not fit "
@@ -521,6 +568,21 @@ int dictproj_forward_batch(int n, const void* const* X, int M, const dictproj_la
     return DICTPROJ_OK;
   }
   const int mp = decode_mp(M);
+  cudaStream_t s = (cudaStream_t)stream;
+  {
+    const __half* xs[kDecodeMaxBatch];
+    __half* ys[kDecodeMaxBatch];
+    for (int i = 0; i < n; ++i) {
+      xs[i] = static_cast<const __half*>(X[i]);
+      ys[i] = static_cast<__half*>(Y[i]);
+    }
+    FusedLaunchPlan fp;
+    if (fused_plan_launch(n, groups, layers, xs, M, smem_optin_of(dev), &fp)) {
+      if ((e = launch_fused(n, groups, layers, xs, ys, M, fp, kWaitLimitCycles, s)) != cudaSuccess)
+        return cuda_fail(e, "forward_batch: fused decode launch");
+      return DICTPROJ_OK;
+    }
+  }
   for (int i = 0; i < n; ++i)
     if (!coeff_smem_fits(groups[i]->k, mp, dev))
       return fail(DICTPROJ_ERR_UNSUPPORTED,
@@ -538,11 +600,35 @@ int dictproj_forward_batch(int n, const void* const* X, int M, const dictproj_la
     ns[i] = plans[i].slices;
     ys[i] = static_cast<__half*>(Y[i]);
   }
-  cudaStream_t s = (cudaStream_t)stream;
   if ((e = launch_dict_decode_batch(n, groups, xs, M, mp, zs, plans, s)) != cudaSuccess)
     return cuda_fail(e, "forward_batch: dictionary stage launch");
   if ((e = launch_coeff_decode_batch(n, layers, zs, ns, M, mp, ys, s)) != cudaSuccess)
     return cuda_fail(e, "forward_batch: coefficient stage launch");
+  return DICTPROJ_OK;
+}
+
+int dictproj_launch_count(int n, const void* const* X, int M, const dictproj_layer* const* layers,
+                          const dictproj_group* const* groups, int* count) {
+  clear_error();
+  if (!X || !layers || !groups || !count) return fail(DICTPROJ_ERR_NULL, "launch_count: NULL pointer");
+  if (n < 1 || n > DICTPROJ_MAX_BATCH) return fail(DICTPROJ_ERR_RANGE, "launch_count: n=%d outside [1, %d]", n, DICTPROJ_MAX_BATCH);
+  for (int i = 0; i < n; ++i)
+    if (!layers[i] || !groups[i]) return fail(DICTPROJ_ERR_NULL, "launch_count: NULL entry %d", i);
+  if (M < 1) return fail(DICTPROJ_ERR_RANGE, "launch_count: M=%d < 1", M);
+  if (M > kDecodeMaxTokens) {  // prefill: dictionary GEMM, densify, coefficient GEMM per projection
+    *count = 3 * n;
+    return DICTPROJ_OK;
+  }
+  const __half* xs[kDecodeMaxBatch];
+  for (int i = 0; i < n; ++i) xs[i] = static_cast<const __half*>(X[i]);
+  FusedLaunchPlan fp;
+  if (fused_plan_launch(n, groups, layers, xs, M, smem_optin_of(groups[0]->device), &fp)) {
+    *count = 1;
+    return DICTPROJ_OK;
+  }
+  bool all_gather = true;
+  for (int i = 0; i < n; ++i) all_gather = all_gather && layers[i]->gather_ok;
+  *count = 1 + (all_gather ? 1 : n);
   return DICTPROJ_OK;
 }
 

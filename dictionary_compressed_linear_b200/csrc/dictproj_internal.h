@@ -29,9 +29,15 @@ int layer_packed_entries(const int32_t* col_ptr, int k, int d_out, size_t* total
 int pack_layer_host(const int32_t* col_ptr, const int32_t* atom_idx, const float* vals, int k,
                     int d_out, uint32_t* pcol_ptr, uint32_t* nnz, uint8_t* codes, uint8_t* scales,
                     uint8_t* idx, uint16_t* seg_start, float* s_C);
+int pack_layer_bitmap_host(const int32_t* col_ptr, const int32_t* atom_idx, const float* vals, int k, int d_out,
+                           uint32_t* pcol_ptr, uint32_t* nnz, uint8_t* codes, uint8_t* scales, uint32_t* bitmap,
+                           float* s_C);
 
 // Largest M served by the decode (GEMV) path.
 constexpr int kDecodeMaxTokens = 8;
+
+// Default limit of a bounded device wait: 2^31 SM clocks (about one second).
+constexpr long long kWaitLimitCycles = 1ll << 31;
 
 }  // namespace dictproj
 
@@ -52,6 +58,16 @@ struct dictproj_group {
   int cdense_cols;         // reserved output columns (dictproj_group_reserve_prefill)
   unsigned int* err;       // device error word for bounded waits
   CUtensorMap codes_map;   // TMA map of codes: [k] rows x [d_in/2] bytes, box 32 x 256
+  // fused decode kernel
+  bool fused_ok;           // the fused kernel serves this group
+  CUtensorMap fmap_codes;  // codes: box 16 atoms x 128 bytes, 128-byte swizzle
+  CUtensorMap fmap_scales; // scales (row stride padded to 16 bytes): box 16 atoms x 32 bytes
+  uint8_t* scales_pad;     // padded copy of the scales when d_in/16 is not a multiple of 16
+  float* zx;               // partial-Z exchange buffer [zslots][k][mp]
+  int zslots;              // CTAs one 16-atom tile is split over, at most
+  int ppr;                 // 512-element pieces per atom row
+  int tp_bound;            // tiles one CTA's pieces span, at most
+  unsigned long long* fsync;  // [0] ticket, bytes 16.. flags[n_sm]
 };
 
 struct dictproj_layer {
@@ -67,4 +83,9 @@ struct dictproj_layer {
   uint16_t* seg_start;     // [d_out][nseg]
   int n_sm;                // SMs of the device
   bool gather_ok;          // the gather kernel serves this layer (else the direct kernel)
+  // fused decode kernel: column chunks of each of the n_sm positions
+  bool fused_ok;
+  uint32_t* cplan_off;     // [n_sm + 1]
+  uint4* cplan;            // {o_a, o_b, E_a, E_b}
+  int cplan_max;           // chunks of the busiest position
 };

@@ -156,11 +156,12 @@ int layer_packed_entries(const int32_t* col_ptr, int k, int d_out, size_t* total
   return DICTPROJ_OK;
 }
 
-int pack_layer_host(const int32_t* col_ptr, const int32_t* atom_idx, const float* vals, int k,
-                    int d_out, uint32_t* pcol_ptr, uint32_t* nnz, uint8_t* codes, uint8_t* scales,
-                    uint8_t* idx, uint16_t* seg_start, float* s_C) {
-  if (!col_ptr || !pcol_ptr || !nnz || !codes || !scales || !idx || !seg_start || !s_C)
-    return fail(DICTPROJ_ERR_NULL, "pack_layer_host: NULL pointer");
+// Quantise C_l and lay it out; the support goes to idx + seg_start (u8 index,
+// Eq. (12) a = 8) when they are given and to a bitmap (Eq. (12) a = 0, h = 1)
+// when `bitmap` is given. Codes, scales and padding are the same either way.
+static int pack_layer_core(const int32_t* col_ptr, const int32_t* atom_idx, const float* vals, int k,
+                           int d_out, uint32_t* pcol_ptr, uint32_t* nnz, uint8_t* codes, uint8_t* scales,
+                           uint8_t* idx, uint16_t* seg_start, uint32_t* bitmap, float* s_C) {
   size_t total = 0;
   int st = layer_packed_entries(col_ptr, k, d_out, &total);
   if (st) return st;
@@ -195,17 +196,24 @@ int pack_layer_host(const int32_t* col_ptr, const int32_t* atom_idx, const float
       const int32_t n = col_ptr[o + 1] - b0;
       const uint32_t p0 = pcol_ptr[o];
       const uint32_t P = pcol_ptr[o + 1] - p0;
-      // segment starts: entries are ascending, so one pass
-      int q = 0;
-      for (int sgi = 0; sgi < nseg; ++sgi) {
-        while (q < n && atom_idx[b0 + q] < 256 * sgi) ++q;
-        seg_start[o * (size_t)nseg + sgi] = (uint16_t)q;
+      if (seg_start) {  // segment starts: entries are ascending, so one pass
+        int q = 0;
+        for (int sgi = 0; sgi < nseg; ++sgi) {
+          while (q < n && atom_idx[b0 + q] < 256 * sgi) ++q;
+          seg_start[o * (size_t)nseg + sgi] = (uint16_t)q;
+        }
+      }
+      if (bitmap) {
+        const int words = (k + 31) / 32;
+        uint32_t* row = bitmap + o * (size_t)words;
+        for (int w = 0; w < words; ++w) row[w] = 0u;
+        for (int q = 0; q < n; ++q) row[atom_idx[b0 + q] >> 5] |= 1u << (atom_idx[b0 + q] & 31);
       }
       for (uint32_t e = 0; e < P; e += 16) {
         for (int i = 0; i < 16; ++i) {
           const uint32_t qq = e + i;
           blk[i] = qq < (uint32_t)n ? vals[b0 + qq] : 0.0f;
-          idx[p0 + qq] = qq < (uint32_t)n ? (uint8_t)(atom_idx[b0 + qq] & 255) : 0;
+          if (idx) idx[p0 + qq] = qq < (uint32_t)n ? (uint8_t)(atom_idx[b0 + qq] & 255) : 0;
         }
         scales[(p0 + e) / 16] = quantize_block(blk, s, c16);
         for (int i = 0; i < 8; ++i) codes[(p0 + e) / 2 + i] = (uint8_t)(c16[2 * i] | (c16[2 * i + 1] << 4));
@@ -214,6 +222,24 @@ int pack_layer_host(const int32_t* col_ptr, const int32_t* atom_idx, const float
   });
   *s_C = s;
   return DICTPROJ_OK;
+}
+
+int pack_layer_host(const int32_t* col_ptr, const int32_t* atom_idx, const float* vals, int k,
+                    int d_out, uint32_t* pcol_ptr, uint32_t* nnz, uint8_t* codes, uint8_t* scales,
+                    uint8_t* idx, uint16_t* seg_start, float* s_C) {
+  if (!col_ptr || !pcol_ptr || !nnz || !codes || !scales || !idx || !seg_start || !s_C)
+    return fail(DICTPROJ_ERR_NULL, "pack_layer_host: NULL pointer");
+  return pack_layer_core(col_ptr, atom_idx, vals, k, d_out, pcol_ptr, nnz, codes, scales, idx, seg_start, nullptr,
+                         s_C);
+}
+
+int pack_layer_bitmap_host(const int32_t* col_ptr, const int32_t* atom_idx, const float* vals, int k, int d_out,
+                           uint32_t* pcol_ptr, uint32_t* nnz, uint8_t* codes, uint8_t* scales, uint32_t* bitmap,
+                           float* s_C) {
+  if (!col_ptr || !pcol_ptr || !nnz || !codes || !scales || !bitmap || !s_C)
+    return fail(DICTPROJ_ERR_NULL, "pack_layer_bitmap_host: NULL pointer");
+  return pack_layer_core(col_ptr, atom_idx, vals, k, d_out, pcol_ptr, nnz, codes, scales, nullptr, nullptr, bitmap,
+                         s_C);
 }
 
 }  // namespace dictproj

@@ -109,6 +109,18 @@ int dictproj_pack_layer_host(const int32_t* col_ptr, const int32_t* atom_idx, co
                              int k, int d_out, uint32_t* pcol_ptr, uint32_t* nnz, uint8_t* codes,
                              uint8_t* scales, uint8_t* idx, uint16_t* seg_start, float* s_C);
 
+/* The same C_l with a bitmap support index instead of idx + seg_start: the
+ * review's Eq. (12) case a = 0, h = 1 (one bit per logical position; it saves
+ * bytes over the 8-bit index for every density above 1/8 and over dense NVFP4
+ * above 22.2% sparsity). Codes, scales, padding, pcol_ptr, nnz and s_C are
+ * exactly those of dictproj_pack_layer_host; bitmap is uint32[d_out][ceil(k/32)]
+ * with bit j % 32 of word j / 32 of row o set iff atom j is retained in column o
+ * (the set bits, ascending, are the column's stored entries in storage order;
+ * padding entries have no bit). Errors as dictproj_pack_layer_host. */
+int dictproj_pack_layer_bitmap_host(const int32_t* col_ptr, const int32_t* atom_idx, const float* vals,
+                                    int k, int d_out, uint32_t* pcol_ptr, uint32_t* nnz, uint8_t* codes,
+                                    uint8_t* scales, uint32_t* bitmap, float* s_C);
+
 /* ------------------------------------------------------------------------- */
 /* Device objects                                                             */
 /* ------------------------------------------------------------------------- */
@@ -199,6 +211,13 @@ int dictproj_forward(const void* X, int M, const dictproj_layer* layer,
 #define DICTPROJ_MAX_BATCH 4
 int dictproj_forward_batch(int n, const void* const* X, int M, const dictproj_layer* const* layers,
                            const dictproj_group* const* groups, void* const* Y, void* stream);
+
+/* Number of kernels that dictproj_forward_batch with these arguments (n = 1:
+ * dictproj_forward) launches: 1 for a decode call served by the fused kernel,
+ * 2 (or 1 + n) on the two-kernel decode path, 3 per projection at prefill.
+ * Host only; nothing is launched. Errors: NULL, RANGE. */
+int dictproj_launch_count(int n, const void* const* X, int M, const dictproj_layer* const* layers,
+                          const dictproj_group* const* groups, int* count);
 
 /* Forward with an explicit path: DICTPROJ_PATH_AUTO, DICTPROJ_PATH_DECODE (M <= 8)
  * or DICTPROJ_PATH_PREFILL (any M). Errors as dictproj_forward, plus

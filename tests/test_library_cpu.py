@@ -179,3 +179,15 @@ def test_noalloc_and_selftest_validate_before_any_device_call(dp):
     lib = dp.lib()
     assert lib.dictproj_selftest_wait_timeout(0, None) == -5
     assert lib.dictproj_selftest_wait_timeout((1 << 31) + 1, None) == -5
+
+
+@pytest.mark.parametrize("k,d_out,rho", [(128, 256, 0.5), (2048, 512, 0.3), (3072, 300, 0.25),
+                                         (272, 45, 0.05), (16, 7, 1.0), (40, 33, 0.0), (8448, 9, 0.1)])
+def test_bitmap_layer_packer_bit_exact(dp, k, d_out, rho):
+    from oracle.pack import pack_coeff_bitmap
+    C = synth.gen_coeff(7, k, d_out, 2, k, d_out, rho)
+    a = dp.dictproj_pack_layer_bitmap_host(C.col_ptr, C.atom_idx, C.vals, k, d_out)
+    b = pack_coeff_bitmap(C.col_ptr, C.atom_idx, C.vals, k, d_out)
+    for n in ("col_ptr", "nnz", "codes", "scales", "bitmap"):
+        assert np.array_equal(a[n], b[n]), n
+    assert a["s"] == b["s"] and a["words"] == b["words"]
