@@ -143,6 +143,63 @@ def replica_throughput(tokens_per_rank, world, ms):
     return world * tokens_per_rank / (ms / 1e3)
 
 
+# ----------------------------------------------------------------------------- per-shape decode rows
+SHAPE_ROWS = (("q", 1, 0.3), ("k", 1, 0.3), ("v", 1, 0.3), ("o", 1, 0.3),
+              ("gate", 2, 0.25), ("up", 2, 0.25), ("down", 2, 0.25))
+
+
+def call_bytes(d_in, d_out, k, rho, M):
+    """Algorithmic bytes of one projection call: packed D, packed C (u8 index,
+    unpadded), X and Y."""
+    n = synth.nnz_per_column(k, rho)
+    nseg = max(1, -(-k // 256))
+    return (d_in * k // 2 + d_in * k // 16 + 4 + 4 + d_out * (-(-n // 2) + -(-n // 16) + n + 2 * nseg + 4)
+            + 2 * M * (d_in + d_out))
+
+
+def per_shape_bench(torch, dp, stream, peak, tokens=(1, 8), reps=5):
+    """Each LLaMA-7B projection shape alone (densities of the attention and MLP
+    workloads: 0.3 and 0.25), one dictproj_forward per call, chained in a CUDA
+    graph over R device copies of the packed weights whose total exceeds 4x the L2
+    size, so that every call streams its weights from HBM."""
+    l2 = torch.cuda.get_device_properties(torch.cuda.current_device()).L2_cache_size
+    sh = stream.cuda_stream
+    rows = {}
+    for name, cfg, rho in SHAPE_ROWS:
+        d_in, d_out, k = synth.LLAMA7B_SHAPES[name]
+        pt = synth.PROJ_TYPES.index(name)
+        D = synth.gen_dictionary(cfg, 0, pt, d_in, k)
+        C = synth.gen_coeff(cfg, 0, pt, 0, k, d_out, rho)
+        pg = dp.dictproj_pack_group_host(D)
+        pc = dp.dictproj_pack_layer_host(C.col_ptr, C.atom_idx, C.vals, k, d_out)
+        R = -(-4 * l2 // call_bytes(d_in, d_out, k, rho, 1)) + 1
+        gs = [dp.dictproj_group_upload(pg, 8) for _ in range(R)]
+        ls = [dp.dictproj_layer_upload(pc) for _ in range(R)]
+        row = {"d_in": d_in, "d_out": d_out, "k": k, "density": rho, "weight_copies": R}
+        for M in tokens:
+            X = torch.from_numpy(synth.gen_activations(cfg, 0, synth.INPUT_SITE[name], M, d_in)).cuda()
+            Y = torch.empty((M, d_out), dtype=torch.float16, device="cuda")
+
+            def chain():
+                for i in range(R):
+                    dp.dictproj_forward(X.data_ptr(), M, ls[i], gs[i], Y.data_ptr(), sh)
+            g = capture(torch, stream, chain)
+            time_replays(torch, stream, g, 3)
+            ms = time_replays(torch, stream, g, reps) / (reps * R)
+            del g
+            b = call_bytes(d_in, d_out, k, rho, M)
+            gbs = b / (ms / 1e3) / 1e9
+            row[f"M={M}"] = {"us_per_call": round(ms * 1e3, 3), "bytes_per_call": b, "GB/s": round(gbs, 1),
+                             "frac": round(gbs / peak, 4),
+                             "launches_per_call": dp.dictproj_launch_count([X.data_ptr()], M, [ls[0]], [gs[0]])}
+        rows[name] = row
+        del gs, ls
+    return {"workload": "each projection shape alone: configs 1-2 (attention q/k/v/o 4096->4096 k=2048 density 0.3; "
+                        "gate/up 4096->11008 and down 11008->4096, k=3072, density 0.25), M=1 and M=8, "
+                        "one call per projection chained in a CUDA graph over R weight copies > 4x L2",
+            "peak_GB/s": peak, "rows": rows}
+
+
 # ----------------------------------------------------------------------------- prefill leg
 PREFILL_SHAPES = ("q", "gate", "down")
 PREFILL_TOKENS = (128, 512, 2048)
@@ -159,45 +216,57 @@ def prefill_inputs(name, M):
     return D, C, X
 
 
-def prefill_bench(torch, dp, stream, M=2048, reps=20):
+def prefill_bench(torch, dp, stream, tokens=PREFILL_TOKENS, reps=20):
     """Prefill (M tokens) of one projection of each LLaMA-7B shape class: the
     dictionary stage alone (tcgen05, the tensor-bound step) and the whole forward,
     timed with CUDA events over graphs of `reps` calls alternating two weight sets
-    (C density 0.3, 1% of input channels x20, as in the prefill workload)."""
+    (C density 0.3, 1% of input channels x20, as in the prefill workload).
+    TFLOP/s count the method's own work: 2 M d_in k for the dictionary stage and
+    2 M (d_in k + nnz) for the forward (the dense-equivalent 2 M (d_in k + k d_out)
+    that the densified coefficient GEMM executes is given beside it)."""
     sh = stream.cuda_stream
     peak, peak_src = measured_tensor_peak()
-    out = {"workload": f"prefill M={M}: q (4096->4096, k=2048), gate (4096->11008, k=3072), "
+    out = {"workload": "prefill, M in {128, 512, 2048}: q (4096->4096, k=2048), gate (4096->11008, k=3072), "
                        "down (11008->4096, k=3072); C density 0.3; X fp16 N(0,1), 1% channels x20",
            "peak_tflops": peak, "peak_source": peak_src, "shapes": {}}
     for name in PREFILL_SHAPES:
         d_in, d_out, k = synth.LLAMA7B_SHAPES[name]
-        D, C, X_np = prefill_inputs(name, M)
+        D, C, _ = prefill_inputs(name, 1)
+        nnz = int(C.col_ptr[-1])
         pg = dp.dictproj_pack_group_host(D)
         pc = dp.dictproj_pack_layer_host(C.col_ptr, C.atom_idx, C.vals, k, d_out)
-        gs = [dp.dictproj_group_upload(pg, M) for _ in range(2)]
+        Mmax = max(tokens)
+        gs = [dp.dictproj_group_upload(pg, Mmax) for _ in range(2)]
         for g in gs:
             dp.dictproj_group_reserve_prefill(g, d_out)
         ls = [dp.dictproj_layer_upload(pc) for _ in range(2)]
-        X = torch.from_numpy(X_np).cuda()
-        Z = torch.empty((M, k), dtype=torch.float16, device="cuda")
-        Y = torch.empty((M, d_out), dtype=torch.float16, device="cuda")
         res = {}
-        for what in ("dictionary_stage", "forward"):
-            def chain():
-                for i in range(reps):
-                    if what == "dictionary_stage":
-                        dp.dictproj_dictionary_stage_prefill(X.data_ptr(), M, gs[i % 2], Z.data_ptr(), sh)
-                    else:
-                        dp.dictproj_forward(X.data_ptr(), M, ls[i % 2], gs[i % 2], Y.data_ptr(), sh)
-            g = capture(torch, stream, chain)
-            time_replays(torch, stream, g, 3)
-            ms = time_replays(torch, stream, g, 5) / (5 * reps)
-            del g
-            flops = 2.0 * M * d_in * k + (2.0 * M * k * d_out if what == "forward" else 0.0)
-            tf = flops / (ms / 1e3) / 1e12
-            res[what] = {"us": round(ms * 1e3, 2), "TFLOP/s": round(tf, 1), "frac": round(tf / peak, 4),
-                         "flops": flops}
-        res["dictionary_stage"]["tensor_pipe_util_ncu"] = profiled(f"k_dict_prefill:{name}", "tensor_util")
+        for M in tokens:
+            X = torch.from_numpy(prefill_inputs(name, M)[2]).cuda()
+            Z = torch.empty((M, k), dtype=torch.float16, device="cuda")
+            Y = torch.empty((M, d_out), dtype=torch.float16, device="cuda")
+            r = {}
+            for what in ("dictionary_stage", "forward"):
+                def chain():
+                    for i in range(reps):
+                        if what == "dictionary_stage":
+                            dp.dictproj_dictionary_stage_prefill(X.data_ptr(), M, gs[i % 2], Z.data_ptr(), sh)
+                        else:
+                            dp.dictproj_forward(X.data_ptr(), M, ls[i % 2], gs[i % 2], Y.data_ptr(), sh)
+                g = capture(torch, stream, chain)
+                time_replays(torch, stream, g, 3)
+                ms = time_replays(torch, stream, g, 5) / (5 * reps)
+                del g
+                flops = 2.0 * M * d_in * k + (2.0 * M * nnz if what == "forward" else 0.0)
+                tf = flops / (ms / 1e3) / 1e12
+                r[what] = {"us": round(ms * 1e3, 2), "TFLOP/s": round(tf, 1), "frac": round(tf / peak, 4),
+                           "flops": flops}
+                if what == "forward":
+                    dense = 2.0 * M * (d_in * k + k * d_out)
+                    r[what]["dense_equivalent_TFLOP/s"] = round(dense / (ms / 1e3) / 1e12, 1)
+            if M == 2048:
+                r["dictionary_stage"]["tensor_pipe_util_ncu"] = profiled(f"k_dict_prefill:{name}", "tensor_util")
+            res[f"M={M}"] = r
         out["shapes"][name] = res
         del gs, ls
     return out
@@ -327,8 +396,10 @@ class Stack:
             calls.append([j for j, _ in cur])
         return calls
 
-    def forward_all(self, dp, stream_handle, batched=True):
+    def calls(self, batched):
+        """(X pointers, layers, groups, Y pointers) of every call of the step, in order."""
         xp, yp = self.x.data_ptr(), self.y.data_ptr()
+        out = []
         for call in self.call_groups(batched):
             xs, ls, gs, ys = [], [], [], []
             for i in call:
@@ -337,7 +408,16 @@ class Stack:
                 ls.append(self.layers[i])
                 gs.append(self.groups[(p.group, p.ptype)])
                 ys.append(yp + 2 * self.y_off[i])
-            if len(call) == 1:
+            out.append((xs, ls, gs, ys))
+        return out
+
+    def launches_per_step(self, dp, batched=True):
+        """Kernels one step launches, as the library reports for each of its calls."""
+        return sum(dp.dictproj_launch_count(xs, self.M, ls, gs) for xs, ls, gs, _ in self.calls(batched))
+
+    def forward_all(self, dp, stream_handle, batched=True):
+        for xs, ls, gs, ys in self.calls(batched):
+            if len(ls) == 1:
                 dp.dictproj_forward(xs[0], self.M, ls[0], gs[0], ys[0], stream_handle)
             else:
                 dp.dictproj_forward_batch(xs, self.M, ls, gs, ys, stream_handle)
@@ -494,7 +574,8 @@ def main():
     ap.add_argument("--ref-budget", type=float, default=200.0,
                     help="--impl reference: seconds that warm-up plus timed steps may take")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--no-prefill", action="store_true", help="skip the prefill (M=2048) leg")
+    ap.add_argument("--no-prefill", action="store_true", help="skip the prefill (M = 128, 512, 2048) leg")
+    ap.add_argument("--no-shapes", action="store_true", help="skip the per-projection-shape rows (M = 1, 8)")
     ap.add_argument("--no-batch", action="store_true",
                     help="one dictproj_forward per projection instead of batching q/k/v and gate/up")
     args = ap.parse_args()
@@ -554,7 +635,6 @@ def main():
     ms = max_over_ranks(ms, dist, "cuda")
     ms_per_step = ms / args.steps
     value = replica_throughput(M * args.steps, world, ms)
-    launches_per_step = 2 * calls_per_step
     # the same step with one call per projection, for comparison
     ms_unbatched = None
     if not args.no_batch:
@@ -563,55 +643,26 @@ def main():
         ms_unbatched = time_replays(torch, stream, g_u, max(10, args.steps // 4)) / max(10, args.steps // 4)
         del g_u
 
-    # ---------------- per-stage timing for the roofline (each stage alone, same launch config)
-    kmax = max(p.k for p in wl.projections)
-    zbuf = torch.zeros(kmax * 8, dtype=torch.float32, device="cuda")
-
-    def dict_only():
-        xp = stack.x.data_ptr()
-        for p in wl.projections:
-            dp.dictproj_dictionary_stage(xp + 2 * stack.x_off[(p.layer, p.site)][0], M,
-                                         stack.groups[(p.group, p.ptype)], zbuf.data_ptr(), sh)
-
-    def coeff_only():
-        yp = stack.y.data_ptr()
-        for i, p in enumerate(wl.projections):
-            dp.dictproj_coefficient_stage(zbuf.data_ptr(), M, stack.layers[i], yp + 2 * stack.y_off[i], sh)
-
-    g_d = capture(torch, stream, dict_only)
-    g_c = capture(torch, stream, coeff_only)
-    for g in (g_d, g_c):
-        time_replays(torch, stream, g, 3)
-    ms_d = time_replays(torch, stream, g_d, args.stage_reps)
-    ms_c = time_replays(torch, stream, g_c, args.stage_reps)
-    bytes_d = sum(stage_bytes(p, M)[0] for p in wl.projections)
-    bytes_c = sum(stage_bytes(p, M)[1] for p in wl.projections)
-    n_launch = len(wl.projections)
-    per_launch_d = ms_d / (args.stage_reps * n_launch)
-    per_launch_c = ms_c / (args.stage_reps * n_launch)
-    gbs_d = bytes_d / (ms_d / args.stage_reps / 1e3) / 1e9
-    gbs_c = bytes_c / (ms_c / args.stage_reps / 1e3) / 1e9
+    # ---------------- roofline of the step's kernel, from the timed step itself
+    launches_per_step = stack.launches_per_step(dp, batched=not args.no_batch)
+    step_bytes = sum(d_bytes(p) + c_bytes(p) + 2 * M * (p.d_in + p.d_out) for p in wl.projections)
     peak, peak_kind = measured_peaks()
-    if ms_c >= ms_d:
-        dom, dom_name, gbs, per_launch, bytes_l = "coefficient stage", "k_coeff_gather", gbs_c, per_launch_c, bytes_c / n_launch
-    else:
-        dom, dom_name, gbs, per_launch, bytes_l = "dictionary stage", "k_dict_decode", gbs_d, per_launch_d, bytes_d / n_launch
-    roofline = {"bound": "hbm", "achieved": round(gbs, 1), "peak": peak, "unit": "GB/s",
-                "frac": round(gbs / peak, 4), "traffic": profiled_traffic(dom_name, bytes_l),
-                "kernel": dom_name, "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)" if peak_kind == "measured" else "fallback 6650 GB/s",
-                "avg_launch_us": round(per_launch * 1e3, 3), "algorithmic_bytes_per_launch": int(bytes_l),
-                "stages": {"k_dict_decode": {"GB/s": round(gbs_d, 1), "avg_launch_us": round(per_launch_d * 1e3, 3),
-                                             "frac": round(gbs_d / peak, 4),
-                                             "traffic": profiled_traffic("k_dict_decode", bytes_d / n_launch)},
-                           "k_coeff_gather": {"GB/s": round(gbs_c, 1), "avg_launch_us": round(per_launch_c * 1e3, 3),
-                                              "frac": round(gbs_c / peak, 4),
-                                              "traffic": profiled_traffic("k_coeff_gather", bytes_c / n_launch)}},
-                "timing": "each stage alone: a CUDA graph of the 224 stage calls of one step (dictionary stage "
-                          "with its Z written complete in one slice; coefficient stage reading it), CUDA events "
-                          "on the launching stream"}
+    avg_launch_ms = ms_per_step / launches_per_step
+    bytes_per_launch = step_bytes / launches_per_step
+    achieved = bytes_per_launch / (avg_launch_ms / 1e3) / 1e9
+    roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+                "frac": round(achieved / peak, 4), "traffic": profiled_traffic("k_decode_fused", bytes_per_launch),
+                "kernel": "k_decode_fused",
+                "peak_source": "measured (MEASURED_PEAKS.json hbm_gbs)" if peak_kind == "measured" else "fallback 6650 GB/s",
+                "avg_launch_us": round(avg_launch_ms * 1e3, 3), "algorithmic_bytes_per_launch": int(bytes_per_launch),
+                "launches_per_step": launches_per_step,
+                "timing": "the timed step itself: CUDA events on the launching stream around the replays of the "
+                          "step's graph; the average launch duration is the step time over its launches"
+                          + (" (every launch is k_decode_fused, one per call)" if launches_per_step == calls_per_step
+                             else f" ({launches_per_step} launches for {calls_per_step} calls: some calls ran the "
+                                  "two-kernel path)")}
 
     # ---------------- step-level accounting
-    step_bytes = sum(d_bytes(p) + c_bytes(p) + 2 * M * (p.d_in + p.d_out) for p in wl.projections)
     d_once = sum(d_bytes(p) for p in {(q.group, q.ptype): q for q in wl.projections}.values())
     step_bytes_once = d_once + sum(c_bytes(p) + 2 * M * (p.d_in + p.d_out) for p in wl.projections)
     step_gbs = step_bytes / (ms_per_step / 1e3) / 1e9
@@ -631,10 +682,14 @@ def main():
     ms_e2e = time_replays(torch, stream, graph, e2e_steps, pre, post)
     e2e_value = replica_throughput(M * e2e_steps, world, max_over_ranks(ms_e2e, dist, "cuda"))
 
+    del graph
+    del stack
+    torch.cuda.empty_cache()
+    shapes = None
+    if not args.no_shapes:
+        shapes = per_shape_bench(torch, dp, stream, peak)
     prefill = None
     if not args.no_prefill:
-        del stack
-        torch.cuda.empty_cache()
         prefill = prefill_bench(torch, dp, stream)
 
     cpu = None
@@ -655,6 +710,7 @@ def main():
         "e2e": {"value": round(e2e_value, 2), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h},
         "gpu_launches": launches_per_step * args.steps,
+        "shapes": shapes,
         "clocks": clocks,
         "step": {"algorithmic_bytes": step_bytes, "GB/s": round(step_gbs, 1),
                  "ms_per_step_one_call_per_projection": round(ms_unbatched, 5) if ms_unbatched else None,
@@ -665,7 +721,6 @@ def main():
     }
     if rank == 0:
         print(json.dumps(line), flush=True)
-    del graph, g_d, g_c
     if dist:
         dist.barrier()
         dist.destroy_process_group()

@@ -4,6 +4,8 @@
 #include <cuda_fp16.h>
 #include <cstdint>
 
+#include "dictproj_internal.h"
+
 namespace dictproj {
 
 // ---- programmatic dependent launch -------------------------------------------
@@ -203,12 +205,30 @@ __device__ __forceinline__ uint32_t lds_u16(uint32_t a) {
   return v;
 }
 
+// Z rows live in shared memory at byte address zaddr + atom * MP * 4.
+template <int MP>
+__device__ __forceinline__ void fma_z(float blk[MP], uint32_t a, float v) {
+  if constexpr (MP == 1) {
+    blk[0] = fmaf(lds_f32(a), v, blk[0]);
+  } else if constexpr (MP == 2) {
+    const float2 t = lds_f32x2(a);
+    blk[0] = fmaf(t.x, v, blk[0]);
+    blk[1] = fmaf(t.y, v, blk[1]);
+  } else {
+#pragma unroll
+    for (int m = 0; m < MP; m += 4) {
+      const float4 t = lds_f32x4(a + 4 * m);
+      blk[m] = fmaf(t.x, v, blk[m]);
+      blk[m + 1] = fmaf(t.y, v, blk[m + 1]);
+      blk[m + 2] = fmaf(t.z, v, blk[m + 2]);
+      blk[m + 3] = fmaf(t.w, v, blk[m + 3]);
+    }
+  }
+}
+
 // Device error word of the translation unit that includes this header (bit 0:
 // a bounded wait gave up). Each kernel file exposes a host reader for it.
 static __device__ unsigned int g_dictproj_error;
-
-// Default limit of a bounded device wait: 2^31 SM clocks (about one second).
-constexpr long long kWaitLimitCycles = 1ll << 31;
 
 // Wait for `phase` of `bar` for at most `limit` SM clocks; on time-out record the
 // error and return false (the caller then leaves its loop).

@@ -236,27 +236,6 @@ k_dict_decode(const __grid_constant__ DictBatch batch) {
 // =================================================================================
 // Stage 2: coefficients
 // =================================================================================
-// Z rows live in shared memory at byte address zaddr + atom * MP * 4.
-template <int MP>
-__device__ __forceinline__ void fma_z(float blk[MP], uint32_t a, float v) {
-  if constexpr (MP == 1) {
-    blk[0] = fmaf(lds_f32(a), v, blk[0]);
-  } else if constexpr (MP == 2) {
-    const float2 t = lds_f32x2(a);
-    blk[0] = fmaf(t.x, v, blk[0]);
-    blk[1] = fmaf(t.y, v, blk[1]);
-  } else {
-#pragma unroll
-    for (int m = 0; m < MP; m += 4) {
-      const float4 t = lds_f32x4(a + 4 * m);
-      blk[m] = fmaf(t.x, v, blk[m]);
-      blk[m + 1] = fmaf(t.y, v, blk[m + 1]);
-      blk[m + 2] = fmaf(t.z, v, blk[m + 2]);
-      blk[m + 3] = fmaf(t.w, v, blk[m + 3]);
-    }
-  }
-}
-
 // seg_start row reader (global row).
 struct SegGlobal {
   const uint16_t* p;
@@ -612,6 +591,8 @@ int decode_mp(int M) { return M <= 1 ? 1 : M <= 2 ? 2 : M <= 4 ? 4 : 8; }
 // Opt-in shared memory per block of each device, recorded by prepare_decode_kernels.
 constexpr int kMaxDevices = 64;
 static int g_smem_optin[kMaxDevices];
+
+int smem_optin_of(int device) { return device >= 0 && device < kMaxDevices ? g_smem_optin[device] : 0; }
 
 bool coeff_smem_fits(int k, int mp, int device) {
   if (device < 0 || device >= kMaxDevices) return false;

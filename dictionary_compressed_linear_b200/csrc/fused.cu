@@ -1,0 +1,986 @@
+// Decode path (M <= 8 tokens), fused: both stages of Eq. (1) of the DictLLM
+// technical review, Z = X D_g and Y = Z C_l, in ONE kernel per call
+// (k_decode_fused), with every packed weight byte staged through shared memory
+// by the Tensor Memory Accelerator.
+//
+// Why one kernel. At decode a projection moves 9-25 MB of packed weights, which
+// HBM delivers in 1.3-3.7 us; two dependent kernels per call with a global Z
+// round trip cost more than that in fixed latency. Here:
+//   * one CTA per SM (grid = SM count); a producer warp streams the CTA's share
+//     of the packed D_g and C_l into a ring of 16 KB shared-memory slots with
+//     bulk / tensor TMA copies. Weights are never written after upload, so the
+//     producer starts streaming at once, before the kernel waits for the
+//     previous work on the stream (programmatic dependent launch): the ring of
+//     the next call fills while this call computes. A CTA uses at most half of
+//     an SM (M <= 4), so two consecutive calls are resident together.
+//   * stage 1: eight compute warps take 16-atom x 512-element pieces of D_g
+//     from the ring, decode E2M1 x E4M3 to fp16 (exact) and run swap-AB
+//     mma.sync m16n8k16 (atoms = the 16 rows, tokens = the 8 columns) with fp32
+//     accumulation. Pieces are dealt to CTAs evenly: each CTA gets a contiguous
+//     run of a projection's pieces, so a 16-atom tile is split over at most a
+//     few CTAs, whose partial sums (times s_D) go to a per-group exchange buffer
+//     Zx[slot][k][mp] in L2.
+//   * one grid-wide exchange: each CTA publishes a flag with this launch's epoch
+//     (from a 64-bit ticket every CTA takes at start, so aborted launches never
+//     confuse later ones); after all flags are seen, every CTA sums the slots of
+//     each tile in a fixed order into its shared-memory Z table (bit-exact,
+//     independent of timing).
+//   * stage 2: the compute warps take the CTA's column chunks of C_l (columns
+//     split over CTAs by bytes, so by nnz) from the ring; one warp per column,
+//     lanes over 8-entry half-blocks, the same per-window segment logic as the
+//     gather kernel, fp32 sums, fp16 Y.
+// Every wait is bounded (a second by default); a wait that gives up sets the
+// device error word and the CTA unwinds (the producer first waits, bounded,
+// for its copies in flight).
+#include <cuda.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <climits>
+#include <vector>
+
+#include "common.cuh"
+#include "dictproj_internal.h"
+#include "kernels.h"
+
+namespace dictproj {
+
+// ---------------------------------------------------------------------------------
+// geometry
+// ---------------------------------------------------------------------------------
+constexpr int kFWarps = 8;                       // compute warps
+constexpr int kFThreads = 32 * (kFWarps + 1);    // + one producer warp
+constexpr int kPieceElems = 512;                 // d_in elements of one D piece (per atom)
+constexpr int kPieceCodeBytes = 16 * 256;        // 16 atoms x 256 code bytes (two 128-B boxes)
+constexpr int kPieceScaleBytes = 16 * 32;        // 16 atoms x 32 scale bytes
+constexpr int kPiecesPerSlot = 3;
+constexpr int kSlotScaleOff = kPiecesPerSlot * kPieceCodeBytes;  // 12 KB
+constexpr int kTasksPerSlot = 4 * kPiecesPerSlot;                // 128-element quarters
+constexpr int kMaxCChunks = 64;                  // coefficient chunks one CTA may own in one launch
+constexpr int kFusedMaxBatch = 4;
+
+static_assert(kSlotScaleOff + kPiecesPerSlot * kPieceScaleBytes <= kFusedSlotBytes, "D pieces fit a slot");
+
+// Byte layout of one coefficient chunk (columns [o_a, o_b), entries [E_a, E_b))
+// in a ring slot: five 16-byte aligned runs copied from the packed arrays, each
+// rounded outward to 16 bytes (the arrays carry 16 bytes of slack at the end).
+struct CChunk {
+  uint32_t idx_src, idx_bytes;    // idx[E_a, E_b)
+  uint32_t code_src, code_bytes;  // codes[E_a/2, E_b/2)
+  uint32_t sc_src, sc_bytes;      // scales[E_a/16, E_b/16)
+  uint32_t ss_src, ss_bytes;      // seg_start rows o_a .. o_b-1 (bytes)
+  uint32_t cp_src, cp_bytes;      // col_ptr[o_a .. o_b] (bytes)
+  uint32_t code_dst, sc_dst, ss_dst, cp_dst, total;
+};
+
+__host__ __device__ inline uint32_t up16(uint32_t x) { return (x + 15u) & ~15u; }
+
+__host__ __device__ inline CChunk c_chunk_layout(uint32_t o_a, uint32_t o_b, uint32_t E_a, uint32_t E_b,
+                                                 uint32_t nseg) {
+  CChunk c;
+  c.idx_src = E_a;
+  c.idx_bytes = E_b - E_a;
+  c.code_src = (E_a >> 1) & ~15u;
+  c.code_bytes = up16(E_b >> 1) - c.code_src;
+  c.sc_src = (E_a >> 4) & ~15u;
+  c.sc_bytes = up16(E_b >> 4) - c.sc_src;
+  c.ss_src = (2u * o_a * nseg) & ~15u;
+  c.ss_bytes = up16(2u * o_b * nseg) - c.ss_src;
+  c.cp_src = (4u * o_a) & ~15u;
+  c.cp_bytes = up16(4u * (o_b + 1u)) - c.cp_src;
+  c.code_dst = c.idx_bytes;
+  c.sc_dst = c.code_dst + c.code_bytes;
+  c.ss_dst = c.sc_dst + c.sc_bytes;
+  c.cp_dst = c.ss_dst + c.ss_bytes;
+  c.total = c.cp_dst + c.cp_bytes;
+  return c;
+}
+
+// Even split of P pieces over G positions: position c gets
+// [c*q + min(c, r), (c+1)*q + min(c+1, r)) with P = q*G + r.
+__host__ __device__ inline int split_begin(int c, int q, int r) { return c * q + (c < r ? c : r); }
+__host__ __device__ inline int split_pos(int x, int q, int r) {
+  return x < r * (q + 1) ? x / (q + 1) : r + (x - r * (q + 1)) / q;
+}
+
+// ---------------------------------------------------------------------------------
+// launch parameters
+// ---------------------------------------------------------------------------------
+struct FusedProj {
+  CUtensorMap dcodes;    // D codes: [k] rows x [d_in/2] bytes, box 16 x 128, 128-B swizzle
+  CUtensorMap dscales;   // D scales: [k] rows x [d_in/16] bytes (row stride padded to 16), box 16 x 32
+  const __half* X;
+  __half* Y;
+  float* zx;             // [zslots][k][MP] partial Z of the tiles' pieces
+  const uint32_t* col_ptr;
+  const uint8_t* ccodes;
+  const uint8_t* cscales;
+  const uint8_t* cidx;
+  const uint16_t* seg_start;
+  const uint32_t* cplan_off;  // [G+1] first coefficient chunk of each position
+  const uint4* cplan;         // chunks {o_a, o_b, E_a, E_b}
+  float s_D, s_C;
+  int d_in, k, d_out, nseg;
+  int ppr, P, pq, pr, rot;    // pieces per atom row, pieces, P = pq*G + pr, position rotation
+  int xoff;                   // byte offset of its staged X rows in shared memory, -1: read X from global
+  int xfirst;                 // 1: this projection stages X at xoff (later ones with the same X reuse it)
+  int zt_off;                 // byte offset of its Z table in shared memory
+};
+
+struct FusedParams {
+  FusedProj p[kFusedMaxBatch];
+  unsigned long long* ticket;  // launches of this sync object x G CTAs so far
+  unsigned int* flags;         // [G] epoch + 1 of each CTA's published partial Z
+  long long wait_limit;        // SM clocks a bounded wait may take
+  int n, M, G, R;              // projections, tokens, CTAs, ring slots
+  int xrow;                    // bytes per staged X row
+  int red_off;                 // shared-memory offset of the per-warp partial sums
+  int n_tp;                    // tile pieces the red area holds per CTA
+  int zt_resident;             // 1: every projection's Z table is resident; 0: one table reloaded per projection
+  int bar_off;                 // offset of the barriers and chunk descriptors
+};
+
+// ---------------------------------------------------------------------------------
+// device helpers
+// ---------------------------------------------------------------------------------
+__device__ __forceinline__ void tma2d(uint32_t dst, const CUtensorMap* map, int x, int y, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];"
+      ::"r"(dst), "l"(map), "r"(x), "r"(y), "r"(smem_u32(bar))
+      : "memory");
+}
+__device__ __forceinline__ void bulk_g2s_u32(uint32_t dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+               ::"r"(dst), "l"(src), "r"(bytes), "r"(smem_u32(bar))
+               : "memory");
+}
+__device__ __forceinline__ void mbar_arrive_cta(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+__device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+__device__ __forceinline__ uint4 ld_cg_v4(const void* p) {
+  uint4 r;
+  asm volatile("ld.global.cg.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w) : "l"(p));
+  return r;
+}
+__device__ __forceinline__ float4 ld_cg_f4(const float* p) {
+  float4 r;
+  asm volatile("ld.global.cg.v4.f32 {%0,%1,%2,%3}, [%4];" : "=f"(r.x), "=f"(r.y), "=f"(r.z), "=f"(r.w) : "l"(p));
+  return r;
+}
+__device__ __forceinline__ unsigned int ld_relaxed_u32(const unsigned int* p) {
+  unsigned int v;
+  asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+__device__ __forceinline__ void st_release_u32(unsigned int* p, unsigned int v) {
+  asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+__device__ __forceinline__ void fence_acq_rel_gpu() { asm volatile("fence.acq_rel.gpu;" ::: "memory"); }
+__device__ __forceinline__ void sts_u32x4(uint32_t a, uint4 v) {
+  asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};" ::"r"(a), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w) : "memory");
+}
+__device__ __forceinline__ void sts_f32(uint32_t a, float v) {
+  asm volatile("st.shared.f32 [%0], %1;" ::"r"(a), "f"(v) : "memory");
+}
+__device__ __forceinline__ void sts_f32x4(uint32_t a, float4 v) {
+  asm volatile("st.shared.v4.f32 [%0], {%1,%2,%3,%4};" ::"r"(a), "f"(v.x), "f"(v.y), "f"(v.z), "f"(v.w) : "memory");
+}
+
+// Bounded wait on an mbarrier phase that also gives up when another warp of the
+// CTA has aborted (*abort != 0). Returns false when it gave up.
+__device__ __forceinline__ bool mbar_wait_or_abort(uint64_t* bar, uint32_t phase, volatile int* abort,
+                                                   long long limit) {
+  if (mbar_try_wait(bar, phase)) return true;
+  const long long t0 = clock64();
+  while (!mbar_try_wait(bar, phase)) {
+    if (*abort) return false;
+    if (clock64() - t0 > limit) {
+      atomicOr(&g_dictproj_error, 1u);
+      *abort = 1;
+      return false;
+    }
+  }
+  return true;
+}
+
+}  // namespace dictproj
+
+namespace dictproj {
+
+// ---------------------------------------------------------------------------------
+// stage 1: one 16-atom x 128-element quarter of a D piece
+// ---------------------------------------------------------------------------------
+// Thread (g, tq) of the warp takes the 16-byte chunk c16 = 2*tq + h of the atom
+// rows g and g+8 of the quarter's 128-byte box (rows are 128-byte swizzled: chunk
+// c of row r sits at position c ^ (r & 7)), i.e. 32 elements per atom, and the
+// same 32 elements of X for token g. mma.sync m16n8k16 with the atoms as the 16
+// rows of A and the tokens as the 8 columns of B: within each thread the same
+// element order is used for A and B, so the sum over k is unchanged.
+__device__ __forceinline__ void piece_quarter(float acc[2][4], uint32_t box, uint32_t scl, int g, int c16,
+                                              const uint32_t xw[4][4]) {
+  const uint32_t ra = box + g * 128 + ((uint32_t)(c16 ^ g) << 4);
+  const uint4 wa4 = lds_u32x4(ra), wb4 = lds_u32x4(ra + 1024);
+  const uint32_t ha = e4m3x2_to_f16x2(lds_u16(scl + g * 32 + 2 * c16));
+  const uint32_t hb = e4m3x2_to_f16x2(lds_u16(scl + (g + 8) * 32 + 2 * c16));
+  const uint32_t wa[4] = {wa4.x, wa4.y, wa4.z, wa4.w};
+  const uint32_t wb[4] = {wb4.x, wb4.y, wb4.z, wb4.w};
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    uint32_t fa[4], fb[4];
+    e2m1x8_to_f16x2x4(wa[q], fa);
+    e2m1x8_to_f16x2x4(wb[q], fb);
+    const uint32_t sa = q < 2 ? dup_lo(ha) : dup_hi(ha);
+    const uint32_t sb = q < 2 ? dup_lo(hb) : dup_hi(hb);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      fa[i] = hmul2_u32(fa[i], sa);  // E2M1 x E4M3 is exact in fp16
+      fb[i] = hmul2_u32(fb[i], sb);
+    }
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const uint32_t a[4] = {fa[2 * h], fb[2 * h], fa[2 * h + 1], fb[2 * h + 1]};
+      const uint32_t b[2] = {xw[q][2 * h], xw[q][2 * h + 1]};
+      mma_16816(acc[h], a, b);
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------------
+// stage 2: one column from a shared-memory chunk
+// ---------------------------------------------------------------------------------
+// idx_a / code_a / sc_a / ss_a: shared addresses of the column's first index
+// byte, first code byte, first scale byte and its seg_start row; nhb 8-entry
+// half-blocks. Lane l takes half-blocks 32 i + l; the segment of each entry
+// comes from per-window ballots over seg_start (one boundary per lane), several
+// boundaries inside one half-block fall back to a walk.
+template <int MP>
+__device__ __forceinline__ void column_sum(float acc[MP], uint32_t idx_a, uint32_t code_a, uint32_t sc_a,
+                                           uint32_t ss_a, int nhb, int nseg, uint32_t zs_a, int lane) {
+  constexpr uint32_t kRow = MP * 4;
+#pragma unroll
+  for (int m = 0; m < MP; ++m) acc[m] = 0.f;
+  const bool is_bnd = lane >= 1 && lane < nseg;
+  const int b = lane < nseg ? (int)lds_u16(ss_a + 2 * lane) : 0;
+  for (int i = 0; 256 * i < 8 * nhb; ++i) {
+    const int w = 256 * i;
+    const int s_lo = __popc(__ballot_sync(0xffffffffu, is_bnd && b <= w));
+    const bool in_win = is_bnd && b > w && b < w + 256;
+    const int rel = b - w;
+    const uint32_t at_start = (in_win && (rel & 7) == 0) ? (1u << (rel >> 3)) : 0u;
+    const uint32_t inside = (in_win && (rel & 7) != 0) ? (1u << (rel >> 3)) : 0u;
+    const uint32_t A = __reduce_or_sync(0xffffffffu, at_start);
+    const uint32_t B = __reduce_or_sync(0xffffffffu, inside);
+    const int nwin = __popc(__ballot_sync(0xffffffffu, in_win));
+    const bool collide = nwin != __popc(A) + __popc(B) || (A & B) != 0u;
+    const uint32_t le = lane == 31 ? 0xffffffffu : ((2u << lane) - 1u);
+    const int sgi = s_lo + __popc(A & le) + __popc(B & (le >> 1));  // segment of the lane's first entry
+    const int q0 = w + 8 * lane;
+    const int bn = __shfl_sync(0xffffffffu, b, min(sgi + 1, 31));
+    const int t1 = ((B >> lane) & 1u) ? bn : INT_MAX;
+    const int hb = 32 * i + lane;
+    if (hb < nhb) {
+      const uint2 iv = lds_u32x2(idx_a + 8 * hb);
+      const uint32_t iw[2] = {iv.x, iv.y};
+      uint32_t f[4];
+      e2m1x8_to_f16x2x4(lds_u32(code_a + 4 * hb), f);
+      float a0[MP], a1[MP];
+#pragma unroll
+      for (int m = 0; m < MP; ++m) a0[m] = a1[m] = 0.f;
+      if (!collide) {  // at most one boundary: entries e >= t use segment sgi+1
+        const int t = min(t1 - q0, 8);
+        const uint32_t z0 = zs_a + ((uint32_t)sgi << 8) * kRow;
+        const uint32_t z1 = z0 + 256u * kRow;
+#pragma unroll
+        for (int p = 0; p < 4; ++p) {
+          const float2 v = __half22float2(*reinterpret_cast<const __half2*>(&f[p]));
+          const int e0 = 2 * p, e1 = e0 + 1;
+          const uint32_t b0 = __byte_perm(iw[e0 >> 2], 0u, 0x4440u | (uint32_t)(e0 & 3));
+          const uint32_t b1 = __byte_perm(iw[e1 >> 2], 0u, 0x4440u | (uint32_t)(e1 & 3));
+          fma_z<MP>(a0, (e0 >= t ? z1 : z0) + b0 * kRow, v.x);
+          fma_z<MP>(a1, (e1 >= t ? z1 : z0) + b1 * kRow, v.y);
+        }
+      } else {  // walk the boundaries one entry at a time
+        int sg = 0;
+        for (int j = 1; j < nseg; ++j) sg += ((int)lds_u16(ss_a + 2 * j) <= q0);
+        int nb = (sg + 1 < nseg) ? (int)lds_u16(ss_a + 2 * (sg + 1)) : INT_MAX;
+#pragma unroll
+        for (int p = 0; p < 4; ++p) {
+          const float2 v = __half22float2(*reinterpret_cast<const __half2*>(&f[p]));
+#pragma unroll
+          for (int hh = 0; hh < 2; ++hh) {
+            const int ent = 2 * p + hh;
+            while (q0 + ent >= nb) {
+              ++sg;
+              nb = (sg + 1 < nseg) ? (int)lds_u16(ss_a + 2 * (sg + 1)) : INT_MAX;
+            }
+            const uint32_t bb = __byte_perm(iw[ent >> 2], 0u, 0x4440u | (uint32_t)(ent & 3));
+            fma_z<MP>(hh ? a1 : a0, zs_a + (((uint32_t)sg << 8) + bb) * kRow, hh ? v.y : v.x);
+          }
+        }
+      }
+      const float sc = e4m3_to_f32(lds_u8(sc_a + (hb >> 1)));
+#pragma unroll
+      for (int m = 0; m < MP; ++m) acc[m] = fmaf(a0[m] + a1[m], sc, acc[m]);
+    }
+  }
+#pragma unroll
+  for (int m = 0; m < MP; ++m) {
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) acc[m] += __shfl_xor_sync(0xffffffffu, acc[m], off);
+  }
+}
+
+}  // namespace dictproj
+
+namespace dictproj {
+
+// Shared-memory control block (at FusedParams::bar_off, 16-byte aligned):
+//   uint4   desc[kMaxCChunks]      coefficient chunks {o_a, o_b, E_a, E_b} of this CTA
+//   u64     full[R], empty[R], rdy mbarriers (ring slot filled / drained; control block ready)
+//   int     misc[8]                abort, flag value, coefficient chunks, D pieces, tile pieces
+//   int     loc[4][8]              per projection: x0, x1, first local piece, first tile piece,
+//                                  first tile, tiles, position
+//   uint8   desc_p[kMaxCChunks]    projection of each coefficient chunk
+constexpr int kCtlMisc = 8, kCtlLoc = 8;
+inline int fused_ctl_bytes(int R) { return 16 * kMaxCChunks + 16 * R + 8 + 4 * kCtlMisc + 4 * kCtlLoc * kFusedMaxBatch + kMaxCChunks; }
+
+template <int MP>
+__device__ __forceinline__ void load_ztable(const FusedProj& pp, uint32_t sbase, int tid) {
+  const uint32_t zt = sbase + pp.zt_off;
+  const int nv = pp.k * MP / 4;
+  for (int v = tid; v < nv; v += kFWarps * 32) {
+    const int e = 4 * v, a = (e / MP) >> 4;
+    const int pos0 = split_pos(a * pp.ppr, pp.pq, pp.pr);
+    const int pos1 = split_pos(a * pp.ppr + pp.ppr - 1, pp.pq, pp.pr);
+    float4 s = ld_cg_f4(pp.zx + e);
+    for (int sl = 1; sl <= pos1 - pos0; ++sl) {  // fixed order over the tile's pieces
+      const float4 b = ld_cg_f4(pp.zx + (size_t)sl * pp.k * MP + e);
+      s.x += b.x;
+      s.y += b.y;
+      s.z += b.z;
+      s.w += b.w;
+    }
+    sts_f32x4(zt + 4 * e, s);
+  }
+  const int tail = (pp.k + 256) * MP / 4;  // zero rows after the last atom (padding entries read them)
+  for (int v = nv + tid; v < tail; v += kFWarps * 32) sts_f32x4(zt + 16 * v, make_float4(0.f, 0.f, 0.f, 0.f));
+}
+
+template <int MP>
+__global__ void __launch_bounds__(kFThreads, 2) k_decode_fused(const __grid_constant__ FusedParams prm) {
+  extern __shared__ uint8_t fsm_raw[];
+  const uint32_t raw = smem_u32(fsm_raw);
+  const uint32_t sbase = (raw + 1023u) & ~1023u;  // 128-byte swizzled TMA boxes need 1024-byte alignment
+  uint8_t* sg = fsm_raw + (sbase - raw);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int G = prm.G, R = prm.R, n = prm.n, M = prm.M, cta = blockIdx.x;
+  const long long limit = prm.wait_limit;
+  uint4* desc = reinterpret_cast<uint4*>(sg + prm.bar_off);
+  uint64_t* full = reinterpret_cast<uint64_t*>(desc + kMaxCChunks);
+  uint64_t* empty = full + R;
+  uint64_t* rdy = empty + R;
+  int* misc = reinterpret_cast<int*>(rdy + 1);
+  volatile int* s_abort = misc;
+  int* loc = misc + kCtlMisc;
+  uint8_t* desc_p = reinterpret_cast<uint8_t*>(loc + kCtlLoc * kFusedMaxBatch);
+
+  if (threadIdx.x == kFWarps * 32) {
+    for (int i = 0; i < R; ++i) {
+      mbar_init(full + i, 1);
+      mbar_init(empty + i, kFWarps);
+    }
+    mbar_init(rdy, 1);
+    fence_mbar_init();
+    int N1 = 0, ntp = 0;
+    for (int p = 0; p < n; ++p) {
+      const FusedProj& pp = prm.p[p];
+      int pos = cta - pp.rot;
+      if (pos < 0) pos += G;
+      const int x0 = split_begin(pos, pp.pq, pp.pr), x1 = split_begin(pos + 1, pp.pq, pp.pr);
+      int* L = loc + kCtlLoc * p;
+      L[0] = x0;
+      L[1] = x1;
+      L[2] = N1;
+      L[3] = ntp;
+      L[4] = x1 > x0 ? x0 / pp.ppr : 0;
+      L[5] = x1 > x0 ? (x1 - 1) / pp.ppr - x0 / pp.ppr + 1 : 0;
+      L[6] = pos;
+      N1 += x1 - x0;
+      ntp += L[5];
+    }
+    misc[0] = 0;
+    misc[2] = 0;
+    misc[3] = N1;
+    misc[4] = ntp;
+    if (ntp > prm.n_tp) {  // the launcher sized the partial-sum area too small: refuse to run
+      atomicOr(&g_dictproj_error, 2u);
+      misc[0] = 1;
+    }
+  }
+  __syncthreads();
+  const int N1 = misc[3];
+  const int nD = (N1 + kPiecesPerSlot - 1) / kPiecesPerSlot;
+
+  if (warp == kFWarps) {
+    // ------------------------------------------------------------- producer warp
+    unsigned long long tk = 0;
+    if (lane == 0) tk = atomicAdd(prm.ticket, 1ull);  // before any dependent grid may start
+    auto issue = [&](int j) {
+      const int s = j % R;
+      const uint32_t dst = sbase + (uint32_t)s * kFusedSlotBytes;
+      if (j < nD) {
+        const int i0 = j * kPiecesPerSlot, np = min(kPiecesPerSlot, N1 - i0);
+        mbar_arrive_expect_tx(full + s, (uint32_t)np * (kPieceCodeBytes + kPieceScaleBytes));
+        for (int i = 0; i < np; ++i) {
+          const int L = i0 + i;
+          int p = 0;
+          for (int q = 1; q < n; ++q)
+            if (L >= loc[kCtlLoc * q + 2]) p = q;
+          const FusedProj& pp = prm.p[p];
+          const int x = loc[kCtlLoc * p] + L - loc[kCtlLoc * p + 2];
+          const int a = x / pp.ppr, pc = x - a * pp.ppr;
+          tma2d(dst + i * kPieceCodeBytes, &pp.dcodes, pc * 256, a * 16, full + s);
+          tma2d(dst + i * kPieceCodeBytes + 2048, &pp.dcodes, pc * 256 + 128, a * 16, full + s);
+          tma2d(dst + kSlotScaleOff + i * kPieceScaleBytes, &pp.dscales, pc * 32, a * 16, full + s);
+        }
+      } else {
+        const int t = j - nD;
+        const uint4 d = desc[t];
+        const FusedProj& pp = prm.p[desc_p[t]];
+        const CChunk c = c_chunk_layout(d.x, d.y, d.z, d.w, (uint32_t)pp.nseg);
+        mbar_arrive_expect_tx(full + s, c.total);
+        if (c.idx_bytes) bulk_g2s_u32(dst, pp.cidx + c.idx_src, c.idx_bytes, full + s);
+        if (c.code_bytes) bulk_g2s_u32(dst + c.code_dst, pp.ccodes + c.code_src, c.code_bytes, full + s);
+        if (c.sc_bytes) bulk_g2s_u32(dst + c.sc_dst, pp.cscales + c.sc_src, c.sc_bytes, full + s);
+        if (c.ss_bytes)
+          bulk_g2s_u32(dst + c.ss_dst, reinterpret_cast<const uint8_t*>(pp.seg_start) + c.ss_src, c.ss_bytes, full + s);
+        bulk_g2s_u32(dst + c.cp_dst, reinterpret_cast<const uint8_t*>(pp.col_ptr) + c.cp_src, c.cp_bytes, full + s);
+      }
+    };
+    int issued = 0;
+    if (lane == 0 && !*s_abort) {  // the first slots are free: start streaming D at once
+      issued = min(R, nD);
+      for (int j = 0; j < issued; ++j) issue(j);
+    }
+    // coefficient chunks of this CTA (position = CTA index) over all projections
+    int beg = 0, cnt = 0;
+    if (lane < n) {
+      const uint32_t* off = prm.p[lane].cplan_off;
+      beg = (int)off[cta];
+      cnt = (int)off[cta + 1] - beg;
+    }
+    int pre = cnt;  // inclusive prefix over the lanes (projections)
+#pragma unroll
+    for (int d = 1; d < 32; d <<= 1) {
+      const int v = __shfl_up_sync(0xffffffffu, pre, d);
+      if (lane >= d) pre += v;
+    }
+    int ex[kFusedMaxBatch], bg[kFusedMaxBatch];
+#pragma unroll
+    for (int q = 0; q < kFusedMaxBatch; ++q) {
+      ex[q] = __shfl_sync(0xffffffffu, pre - cnt, q);
+      bg[q] = __shfl_sync(0xffffffffu, beg, q);
+    }
+    const int total_raw = __shfl_sync(0xffffffffu, pre, n - 1);
+    const int total = total_raw > kMaxCChunks ? 0 : total_raw;
+    for (int t = lane; t < total; t += 32) {
+      int p = 0, b0 = bg[0], e0 = ex[0];
+#pragma unroll
+      for (int q = 1; q < kFusedMaxBatch; ++q)
+        if (q < n && t >= ex[q]) {
+          p = q;
+          b0 = bg[q];
+          e0 = ex[q];
+        }
+      desc[t] = prm.p[p].cplan[b0 + t - e0];
+      desc_p[t] = (uint8_t)p;
+    }
+    __syncwarp();
+    if (lane == 0) {
+      if (total_raw > kMaxCChunks) {  // the launcher checks this bound; refuse rather than drop chunks
+        atomicOr(&g_dictproj_error, 2u);
+        *s_abort = 1;
+      }
+      misc[2] = total;
+      misc[1] = (int)((unsigned int)(tk / (unsigned long long)G) + 1u);
+      mbar_arrive_cta(rdy);
+      trigger_dependents();
+      const int nall = nD + total;
+      for (int j = issued; j < nall; ++j) {
+        const int s = j % R;
+        if (j >= R && !mbar_wait_or_abort(empty + s, (uint32_t)(((j / R) + 1) & 1), s_abort, limit)) break;
+        if (*s_abort) break;
+        issue(j);
+        issued = j + 1;
+      }
+      if (*s_abort)  // let the copies in flight land before the CTA exits
+        for (int j = max(0, issued - R); j < issued; ++j) mbar_wait_bounded(full + j % R, (uint32_t)((j / R) & 1), limit);
+    }
+  } else {
+    // ------------------------------------------------------------- compute warps
+    const int tid = threadIdx.x;
+    const int g = lane >> 2, tq = lane & 3;
+    grid_dependency_wait();  // X, Zx, the flags and Y belong to earlier work on the stream
+    for (int i = tid; i < prm.n_tp * kFWarps * 16 * MP; i += kFWarps * 32) sts_f32(sbase + prm.red_off + 4 * i, 0.f);
+    for (int p = 0; p < n; ++p) {  // stage X rows (element order permuted within 512-byte blocks)
+      const FusedProj& pp = prm.p[p];
+      if (pp.xoff < 0 || !pp.xfirst) continue;
+      const int vpr = pp.ppr * 64;
+      for (int v = tid; v < M * vpr; v += kFWarps * 32) {
+        const int m = v / vpr, e = 8 * (v - m * vpr);
+        const uint32_t dst = sbase + pp.xoff + m * prm.xrow + (e >> 8) * 512 + ((e >> 3) & 3) * 128 + ((e >> 5) & 7) * 16;
+        const uint4 val = e < pp.d_in ? ld_cg_v4(pp.X + (size_t)m * pp.d_in + e) : make_uint4(0, 0, 0, 0);
+        sts_u32x4(dst, val);
+      }
+    }
+    named_bar_sync(1, kFWarps * 32);
+
+    // ---- stage 1: partial Z of this CTA's D pieces
+    float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+    int cur_tp = -1;
+    auto flush = [&](int tp) {
+      const uint32_t rb = sbase + prm.red_off + (uint32_t)((tp * kFWarps + warp) * 16 * MP) * 4;
+      const int m0 = 2 * tq, m1 = 2 * tq + 1;
+      if (m0 < MP) {
+        sts_f32(rb + (g * MP + m0) * 4, acc[0][0] + acc[1][0]);
+        sts_f32(rb + ((g + 8) * MP + m0) * 4, acc[0][2] + acc[1][2]);
+      }
+      if (m1 < MP) {
+        sts_f32(rb + (g * MP + m1) * 4, acc[0][1] + acc[1][1]);
+        sts_f32(rb + ((g + 8) * MP + m1) * 4, acc[0][3] + acc[1][3]);
+      }
+#pragma unroll
+      for (int h = 0; h < 2; ++h)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) acc[h][i] = 0.f;
+    };
+    for (int j = 0; j < nD; ++j) {
+      const int s = j % R;
+      bool ok = mbar_wait_or_abort(full + s, (uint32_t)((j / R) & 1), s_abort, limit);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) continue;
+      const int np = min(kPiecesPerSlot, N1 - j * kPiecesPerSlot);
+      const uint32_t slot = sbase + (uint32_t)s * kFusedSlotBytes;
+      for (int t = (warp + 4 * j) & 7; t < 4 * np; t += kFWarps) {  // quarters dealt round-robin, rotated per slot
+        const int L = j * kPiecesPerSlot + (t >> 2);
+        int p = 0;
+        for (int q = 1; q < n; ++q)
+          if (L >= loc[kCtlLoc * q + 2]) p = q;
+        const FusedProj& pp = prm.p[p];
+        const int x = loc[kCtlLoc * p] + L - loc[kCtlLoc * p + 2];
+        const int a = x / pp.ppr, pc = x - a * pp.ppr;
+        const int tp = loc[kCtlLoc * p + 3] + a - loc[kCtlLoc * p + 4];
+        if (tp != cur_tp) {
+          if (cur_tp >= 0) flush(cur_tp);
+          cur_tp = tp;
+        }
+        const int b = (t >> 1) & 1, h = t & 1, c16 = 2 * tq + h;
+        uint32_t xw[4][4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) xw[q][0] = xw[q][1] = xw[q][2] = xw[q][3] = 0u;
+        if (g < M) {
+          if (pp.xoff >= 0) {
+            const uint32_t xa = sbase + pp.xoff + g * prm.xrow + (2 * pc + b) * 512 + c16 * 16;
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              const uint4 v = lds_u32x4(xa + q * 128);
+              xw[q][0] = v.x;
+              xw[q][1] = v.y;
+              xw[q][2] = v.z;
+              xw[q][3] = v.w;
+            }
+          } else {
+            const int e0 = pc * kPieceElems + b * 256 + 32 * c16;
+            if (e0 < pp.d_in) {
+              const __half* xp = pp.X + (size_t)g * pp.d_in + e0;
+#pragma unroll
+              for (int q = 0; q < 4; ++q) {
+                const uint4 v = ld_cg_v4(xp + 8 * q);
+                xw[q][0] = v.x;
+                xw[q][1] = v.y;
+                xw[q][2] = v.z;
+                xw[q][3] = v.w;
+              }
+            }
+          }
+        }
+        const uint32_t piece = slot + (uint32_t)(t >> 2) * kPieceCodeBytes;
+        piece_quarter(acc, piece + b * 2048, slot + kSlotScaleOff + (uint32_t)(t >> 2) * kPieceScaleBytes + b * 16, g,
+                      c16, xw);
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cta(empty + s);
+    }
+    if (cur_tp >= 0) flush(cur_tp);
+    named_bar_sync(1, kFWarps * 32);
+
+    // ---- partial Z of each tile piece (sum over warps, times s_D) to the exchange buffer
+    const int ntp = misc[4];
+    if (!*s_abort) {
+      for (int v = tid; v < ntp * 16 * MP; v += kFWarps * 32) {
+        const int tp = v / (16 * MP), r = v - tp * 16 * MP;
+        float sum = 0.f;
+#pragma unroll
+        for (int w = 0; w < kFWarps; ++w) sum += lds_f32(sbase + prm.red_off + (uint32_t)((tp * kFWarps + w) * 16 * MP + r) * 4);
+        int p = 0;
+        for (int q = 0; q < n; ++q)
+          if (tp >= loc[kCtlLoc * q + 3] && tp < loc[kCtlLoc * q + 3] + loc[kCtlLoc * q + 5]) p = q;
+        const FusedProj& pp = prm.p[p];
+        const int a = loc[kCtlLoc * p + 4] + tp - loc[kCtlLoc * p + 3];
+        const int slot = loc[kCtlLoc * p + 6] - split_pos(a * pp.ppr, pp.pq, pp.pr);
+        pp.zx[((size_t)slot * pp.k + 16 * a) * MP + r] = sum * pp.s_D;
+      }
+    }
+    named_bar_sync(1, kFWarps * 32);
+
+    // ---- grid-wide exchange: publish this CTA's flag, wait for every CTA's
+    if (warp == 0) {
+      bool ok = mbar_wait_or_abort(rdy, 0, s_abort, limit);
+      ok = __all_sync(0xffffffffu, ok) && !*s_abort;
+      if (ok) {
+        const unsigned int fv = (unsigned int)misc[1];
+        if (lane == 0) {
+          __threadfence();
+          st_release_u32(prm.flags + cta, fv);
+        }
+        const long long t0 = clock64();
+        while (true) {
+          bool mine = true;
+          for (int f = lane; f < G; f += 32) mine = mine && ld_relaxed_u32(prm.flags + f) == fv;
+          if (__all_sync(0xffffffffu, mine)) break;
+          const bool give = __any_sync(0xffffffffu, *s_abort != 0 || clock64() - t0 > limit);
+          if (give) {
+            if (lane == 0 && !*s_abort) {
+              atomicOr(&g_dictproj_error, 1u);
+              *s_abort = 1;
+            }
+            break;
+          }
+        }
+        fence_acq_rel_gpu();
+      }
+    }
+    named_bar_sync(1, kFWarps * 32);
+
+    // ---- stage 2: Y = Z C over this CTA's column chunks
+    const int N2 = misc[2];
+    if (prm.zt_resident) {
+      if (!*s_abort)
+        for (int p = 0; p < n; ++p) load_ztable<MP>(prm.p[p], sbase, tid);
+      named_bar_sync(1, kFWarps * 32);
+    }
+    int cur_p = -1;
+    for (int i = 0; i < N2; ++i) {
+      const int j = nD + i, s = j % R;
+      const int p = desc_p[i];
+      if (!prm.zt_resident && p != cur_p) {  // one Z table at a time: reload between projections
+        named_bar_sync(1, kFWarps * 32);
+        if (!*s_abort) load_ztable<MP>(prm.p[p], sbase, tid);
+        named_bar_sync(1, kFWarps * 32);
+      }
+      cur_p = p;
+      bool ok = mbar_wait_or_abort(full + s, (uint32_t)((j / R) & 1), s_abort, limit);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) continue;
+      const FusedProj& pp = prm.p[p];
+      const uint4 d = desc[i];
+      const CChunk c = c_chunk_layout(d.x, d.y, d.z, d.w, (uint32_t)pp.nseg);
+      const uint32_t slot = sbase + (uint32_t)s * kFusedSlotBytes;
+      const int ncols = (int)(d.y - d.x);
+      const uint32_t zs = sbase + pp.zt_off;
+      for (int t = (warp + i) & 7; t < ncols; t += kFWarps) {
+        const uint32_t o = d.x + (uint32_t)t;
+        const uint32_t cpa = slot + c.cp_dst + 4u * o - c.cp_src;
+        const uint32_t e0 = lds_u32(cpa), e1 = lds_u32(cpa + 4);
+        float y[MP];
+        column_sum<MP>(y, slot + (e0 - d.z), slot + c.code_dst + (e0 >> 1) - c.code_src,
+                       slot + c.sc_dst + (e0 >> 4) - c.sc_src, slot + c.ss_dst + 2u * o * (uint32_t)pp.nseg - c.ss_src,
+                       (int)((e1 - e0) >> 3), pp.nseg, zs, lane);
+        if (lane == 0) {
+#pragma unroll
+          for (int m = 0; m < MP; ++m)
+            if (m < M) pp.Y[(size_t)m * pp.d_out + o] = __float2half_rn(y[m] * pp.s_C);
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cta(empty + s);
+    }
+  }
+  __syncthreads();
+}
+
+}  // namespace dictproj
+
+// =================================================================================
+// host side
+// =================================================================================
+namespace dictproj {
+
+static int fused_pieces_per_row(int d_in) { return (d_in + kPieceElems - 1) / kPieceElems; }
+
+// Largest number of tiles one position's piece range spans, and the largest
+// number of positions one tile is split over (the exchange buffer's slots).
+static void fused_split_bounds(int tiles, int ppr, int G, int* tp_bound, int* slots) {
+  const int P = tiles * ppr, q = P / G, r = P % G;
+  int tb = 0, sl = 1;
+  for (int c = 0; c < G; ++c) {
+    const int x0 = split_begin(c, q, r), x1 = split_begin(c + 1, q, r);
+    if (x1 > x0) tb = std::max(tb, (x1 - 1) / ppr - x0 / ppr + 1);
+  }
+  for (int a = 0; a < tiles; ++a)
+    sl = std::max(sl, split_pos(a * ppr + ppr - 1, q, r) - split_pos(a * ppr, q, r) + 1);
+  *tp_bound = tb;
+  *slots = sl;
+}
+
+cudaError_t fused_group_setup(dictproj_group* g, bool* ok) {
+  *ok = false;
+  g->fused_ok = false;
+  // the TMA boxes (128 code bytes, 32 scale bytes per atom row) fit inside a row
+  // from d_in = 512 on; k must keep the gather's segments in one warp
+  if (g->d_in < kPieceElems || g->k > 8192) return cudaSuccess;
+  const int tiles = g->k / 16;
+  g->ppr = fused_pieces_per_row(g->d_in);
+  fused_split_bounds(tiles, g->ppr, g->n_sm, &g->tp_bound, &g->zslots);
+  cudaError_t e;
+  const size_t srow = (size_t)g->d_in / 16;
+  const size_t spad = (srow + 15) & ~size_t(15);
+  const uint8_t* sbase = g->scales;
+  if (spad != srow) {  // tensor-map rows must be 16-byte multiples: a padded copy of the scales
+    if ((e = cudaMalloc((void**)&g->scales_pad, spad * g->k)) != cudaSuccess) return e;
+    if ((e = cudaMemset(g->scales_pad, 0, spad * g->k)) != cudaSuccess) return e;
+    if ((e = cudaMemcpy2D(g->scales_pad, spad, g->scales, srow, srow, g->k, cudaMemcpyDeviceToDevice)) != cudaSuccess)
+      return e;
+    sbase = g->scales_pad;
+  }
+  if ((e = encode_tiled_2d(&g->fmap_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, g->codes, (uint64_t)g->d_in / 2,
+                           (uint64_t)g->k, (uint64_t)g->d_in / 2, 128, 16, CU_TENSOR_MAP_SWIZZLE_128B)) != cudaSuccess)
+    return e;
+  if ((e = encode_tiled_2d(&g->fmap_scales, CU_TENSOR_MAP_DATA_TYPE_UINT8, sbase, (uint64_t)srow, (uint64_t)g->k,
+                           (uint64_t)spad, 32, 16, CU_TENSOR_MAP_SWIZZLE_NONE)) != cudaSuccess)
+    return e;
+  if ((e = cudaMalloc((void**)&g->zx, (size_t)g->zslots * g->k * kDecodeMaxTokens * sizeof(float))) != cudaSuccess)
+    return e;
+  const size_t sync_bytes = 16 + (size_t)g->n_sm * sizeof(unsigned int);
+  if ((e = cudaMalloc((void**)&g->fsync, sync_bytes)) != cudaSuccess) return e;
+  if ((e = cudaMemset(g->fsync, 0, sync_bytes)) != cudaSuccess) return e;
+  g->fused_ok = true;
+  *ok = true;
+  return cudaSuccess;
+}
+
+bool fused_layer_plan(const uint32_t* pcol_ptr, int d_out, int nseg, int G, std::vector<uint32_t>& off,
+                      std::vector<uint4>& chunks, int* max_per_pos) {
+  off.assign(G + 1, 0);
+  chunks.clear();
+  *max_per_pos = 0;
+  if (nseg > 32) return false;
+  auto fits = [&](int oa, int ob) {
+    return c_chunk_layout(oa, ob, pcol_ptr[oa], pcol_ptr[ob], nseg).total <= (uint32_t)kFusedSlotBytes;
+  };
+  // bytes streamed per column (balancing weight): entries + codes + scales + seg_start + col_ptr
+  std::vector<double> cum(d_out + 1, 0.0);
+  for (int o = 0; o < d_out; ++o) {
+    const double ne = (double)(pcol_ptr[o + 1] - pcol_ptr[o]);
+    cum[o + 1] = cum[o] + ne * (1.0 + 0.5 + 1.0 / 16) + 2.0 * nseg + 4.0;
+    if (!fits(o, o + 1)) return false;  // a column larger than a ring slot
+  }
+  auto lower = [&](int lo, int hi, double target) {  // first o in [lo, hi] with cum[o] >= target
+    return (int)(std::lower_bound(cum.begin() + lo, cum.begin() + hi + 1, target) - cum.begin());
+  };
+  int o_lo = 0;
+  for (int c = 0; c < G; ++c) {
+    const int o_hi = c == G - 1 ? d_out : std::max(o_lo, lower(o_lo, d_out, cum[d_out] * (c + 1) / G));
+    off[c] = (uint32_t)chunks.size();
+    if (o_hi > o_lo) {
+      int nch = 0;  // greedy count of slot-sized chunks
+      for (int a = o_lo; a < o_hi; ++nch) {
+        int b = a + 1;
+        while (b < o_hi && fits(a, b + 1)) ++b;
+        a = b;
+      }
+      // the same number of chunks, split evenly by bytes; greedy if one does not fit
+      std::vector<int> cut(nch + 1);
+      cut[0] = o_lo;
+      cut[nch] = o_hi;
+      bool even = true;
+      for (int i = 1; i < nch; ++i) {
+        const double t = cum[o_lo] + (cum[o_hi] - cum[o_lo]) * i / nch;
+        cut[i] = std::min(o_hi - 1, std::max(cut[i - 1] + 1, lower(o_lo, o_hi, t)));
+      }
+      for (int i = 0; i < nch; ++i) even = even && cut[i + 1] > cut[i] && fits(cut[i], cut[i + 1]);
+      if (!even) {
+        cut.assign(1, o_lo);
+        for (int a = o_lo; a < o_hi;) {
+          int b = a + 1;
+          while (b < o_hi && fits(a, b + 1)) ++b;
+          cut.push_back(b);
+          a = b;
+        }
+        nch = (int)cut.size() - 1;
+      }
+      for (int i = 0; i < nch; ++i)
+        chunks.push_back(make_uint4((uint32_t)cut[i], (uint32_t)cut[i + 1], pcol_ptr[cut[i]], pcol_ptr[cut[i + 1]]));
+      *max_per_pos = std::max(*max_per_pos, nch);
+    }
+    o_lo = o_hi;
+  }
+  off[G] = (uint32_t)chunks.size();
+  return true;
+}
+
+cudaError_t prepare_fused_kernels(int device) {
+  int optin = 0;
+  cudaError_t e = cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, device);
+  if (e != cudaSuccess) return e;
+  if ((e = cudaFuncSetAttribute(k_decode_fused<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, optin)) ||
+      (e = cudaFuncSetAttribute(k_decode_fused<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, optin)) ||
+      (e = cudaFuncSetAttribute(k_decode_fused<4>, cudaFuncAttributeMaxDynamicSharedMemorySize, optin)) ||
+      (e = cudaFuncSetAttribute(k_decode_fused<8>, cudaFuncAttributeMaxDynamicSharedMemorySize, optin)))
+    return e;
+  return cudaSuccess;
+}
+
+// Shared memory per CTA for two CTAs to share an SM (228 KB, 1 KB reserved each).
+constexpr int kCoResidentSmem = 113 * 1024;
+constexpr int kStageXMax = 48 * 1024;
+
+bool fused_plan_launch(int n, const dictproj_group* const* g, const dictproj_layer* const* l,
+                       const __half* const* X, int M, int smem_optin, FusedLaunchPlan* out) {
+  FusedLaunchPlan& pl = *out;
+  pl = FusedLaunchPlan{};
+  if (n < 1 || n > kFusedMaxBatch || M < 1 || M > kDecodeMaxTokens) return false;
+  const int mp = decode_mp(M);
+  int chunks = 0, tp = 0, max_ppr = 0;
+  for (int i = 0; i < n; ++i) {
+    if (!g[i]->fused_ok || !l[i]->fused_ok || g[i]->n_sm != g[0]->n_sm || l[i]->n_sm != g[0]->n_sm) return false;
+    chunks += l[i]->cplan_max;
+    tp += g[i]->tp_bound;
+    max_ppr = std::max(max_ppr, g[i]->ppr);
+  }
+  if (chunks > kMaxCChunks) return false;
+  pl.mp = mp;
+  pl.n_tp = std::max(tp, 1);
+  pl.xrow = max_ppr * 1024 + 16;
+  // distinct activations are staged once
+  int nx = 0, xtot = 0;
+  for (int i = 0; i < n; ++i) {
+    pl.xfirst[i] = 1;
+    pl.xslot[i] = nx;
+    for (int j = 0; j < i; ++j)
+      if (X[j] == X[i] && g[j]->d_in == g[i]->d_in) {
+        pl.xfirst[i] = 0;
+        pl.xslot[i] = pl.xslot[j];
+      }
+    if (pl.xfirst[i]) ++nx;
+  }
+  xtot = M * pl.xrow * nx;
+  pl.stage_x = xtot <= kStageXMax;
+  const int red = pl.n_tp * 8 * 16 * mp * 4;
+  const int stage1 = (pl.stage_x ? xtot : 0) + red;
+  int zall = 0, zone = 0;
+  for (int i = 0; i < n; ++i) {
+    const int zb = (g[i]->k + 256) * mp * 4;
+    zall += zb;
+    zone = std::max(zone, zb);
+  }
+  auto total = [&](int R, int U) { return 1024 + R * kFusedSlotBytes + U + fused_ctl_bytes(R); };
+  for (int pass = 0; pass < 2 && !pl.R; ++pass) {  // first: two CTAs per SM; then: one
+    const int cap = pass == 0 ? kCoResidentSmem : smem_optin;
+    const int rmin = pass == 0 ? 3 : 2;
+    for (int resident = 1; resident >= 0 && !pl.R; --resident) {
+      const int U = (std::max(stage1, resident ? zall : zone) + 15) & ~15;
+      for (int R = 8; R >= rmin; --R)
+        if (total(R, U) <= cap) {
+          pl.R = R;
+          pl.U = U;
+          pl.zt_resident = resident;
+          pl.smem = total(R, U);
+          break;
+        }
+    }
+  }
+  if (!pl.R) return false;
+  pl.red_off = pl.R * kFusedSlotBytes + (pl.stage_x ? xtot : 0);
+  pl.bar_off = pl.R * kFusedSlotBytes + pl.U;
+  int zo = pl.R * kFusedSlotBytes;
+  for (int i = 0; i < n; ++i) {
+    pl.xoff[i] = pl.stage_x ? pl.R * kFusedSlotBytes + pl.xslot[i] * M * pl.xrow : -1;
+    pl.zt_off[i] = zo;
+    if (pl.zt_resident) zo += (g[i]->k + 256) * mp * 4;
+  }
+  return true;
+}
+
+cudaError_t launch_fused(int n, const dictproj_group* const* g, const dictproj_layer* const* l,
+                         const __half* const* X, __half* const* Y, int M, const FusedLaunchPlan& pl,
+                         long long wait_limit, cudaStream_t stream) {
+  FusedParams prm;
+  memset(&prm, 0, sizeof(prm));
+  const int G = g[0]->n_sm;
+  int rot = 0;
+  for (int i = 0; i < n; ++i) {
+    FusedProj& p = prm.p[i];
+    p.dcodes = g[i]->fmap_codes;
+    p.dscales = g[i]->fmap_scales;
+    p.X = X[i];
+    p.Y = Y[i];
+    p.zx = g[i]->zx;
+    p.col_ptr = l[i]->col_ptr;
+    p.ccodes = l[i]->codes;
+    p.cscales = l[i]->scales;
+    p.cidx = l[i]->idx;
+    p.seg_start = l[i]->seg_start;
+    p.cplan_off = l[i]->cplan_off;
+    p.cplan = l[i]->cplan;
+    p.s_D = g[i]->s;
+    p.s_C = l[i]->s;
+    p.d_in = g[i]->d_in;
+    p.k = g[i]->k;
+    p.d_out = l[i]->d_out;
+    p.nseg = l[i]->nseg;
+    p.ppr = g[i]->ppr;
+    p.P = (g[i]->k / 16) * p.ppr;
+    p.pq = p.P / G;
+    p.pr = p.P % G;
+    p.rot = rot;
+    rot = (rot + p.pr) % G;  // the next projection's larger shares go to the following CTAs
+    p.xoff = pl.xoff[i];
+    p.xfirst = pl.xfirst[i];
+    p.zt_off = pl.zt_off[i];
+  }
+  prm.ticket = g[0]->fsync;
+  prm.flags = reinterpret_cast<unsigned int*>(g[0]->fsync + 2);
+  prm.wait_limit = wait_limit;
+  prm.n = n;
+  prm.M = M;
+  prm.G = G;
+  prm.R = pl.R;
+  prm.xrow = pl.xrow;
+  prm.red_off = pl.red_off;
+  prm.n_tp = pl.n_tp;
+  prm.zt_resident = pl.zt_resident;
+  prm.bar_off = pl.bar_off;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(G);
+  cfg.blockDim = dim3(kFThreads);
+  cfg.dynamicSmemBytes = pl.smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  switch (pl.mp) {
+    case 1: return cudaLaunchKernelEx(&cfg, k_decode_fused<1>, prm);
+    case 2: return cudaLaunchKernelEx(&cfg, k_decode_fused<2>, prm);
+    case 4: return cudaLaunchKernelEx(&cfg, k_decode_fused<4>, prm);
+    default: return cudaLaunchKernelEx(&cfg, k_decode_fused<8>, prm);
+  }
+}
+
+}  // namespace dictproj

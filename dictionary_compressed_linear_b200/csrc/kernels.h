@@ -43,6 +43,34 @@ cudaError_t launch_wait_probe(long long cycles, cudaStream_t stream);
 // Read and clear the device error word of the decode kernels.
 cudaError_t take_decode_error(unsigned int* out);
 
+// fused decode path (M <= 8): one kernel per call, both stages, weights staged
+// through shared memory by TMA (fused.cu)
+constexpr int kFusedSlotBytes = 16384;  // one ring slot
+struct FusedLaunchPlan {
+  int mp, R, U, smem, zt_resident, stage_x, xrow, red_off, bar_off, n_tp;
+  int xoff[4], xfirst[4], xslot[4], zt_off[4];
+};
+cudaError_t prepare_fused_kernels(int device);
+// Tensor maps, exchange buffer and sync words of a group (sets g->fused_ok when
+// the shape is served; allocation failures are returned).
+cudaError_t fused_group_setup(dictproj_group* g, bool* ok);
+// Column chunks of a layer for G positions: off[G+1] into chunks {o_a, o_b, E_a, E_b}.
+// False if a column does not fit a ring slot (the layer then runs the two-kernel path).
+bool fused_layer_plan(const uint32_t* pcol_ptr, int d_out, int nseg, int G, std::vector<uint32_t>& off,
+                      std::vector<uint4>& chunks, int* max_per_pos);
+// Shared-memory plan of one launch; false if the fused kernel does not serve it.
+bool fused_plan_launch(int n, const dictproj_group* const* g, const dictproj_layer* const* l,
+                       const __half* const* X, int M, int smem_optin, FusedLaunchPlan* out);
+cudaError_t launch_fused(int n, const dictproj_group* const* g, const dictproj_layer* const* l,
+                         const __half* const* X, __half* const* Y, int M, const FusedLaunchPlan& pl,
+                         long long wait_limit, cudaStream_t stream);
+int smem_optin_of(int device);
+
+// 2-D tensor map over a row-major array (rows x inner elements, row stride in bytes).
+cudaError_t encode_tiled_2d(CUtensorMap* map, CUtensorMapDataType type, const void* base, uint64_t inner,
+                            uint64_t rows, uint64_t row_bytes, uint32_t box_inner, uint32_t box_rows,
+                            CUtensorMapSwizzle swz);
+
 // prefill path (any M; used for M > 8): tcgen05 GEMMs, Z fp16 [M][k]
 cudaError_t prepare_prefill_kernels(int device);
 cudaError_t encode_dict_codes_map(const dictproj_group* g, CUtensorMap* map);

@@ -501,8 +501,10 @@ static cudaError_t get_encoder(EncodeTiledFn* fn) {
   return cudaSuccess;
 }
 
+}  // namespace
+
 // 2-D row-major map: rows x inner elements, row stride in bytes, box inner x rows.
-static cudaError_t encode_2d(CUtensorMap* map, CUtensorMapDataType type, const void* base, uint64_t inner,
+cudaError_t encode_tiled_2d(CUtensorMap* map, CUtensorMapDataType type, const void* base, uint64_t inner,
                              uint64_t rows, uint64_t row_bytes, uint32_t box_inner, uint32_t box_rows,
                              CUtensorMapSwizzle swz) {
   EncodeTiledFn enc;
@@ -515,6 +517,13 @@ static cudaError_t encode_2d(CUtensorMap* map, CUtensorMapDataType type, const v
   const CUresult r = enc(map, type, 2, const_cast<void*>(base), gdim, gstride, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                          swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+namespace {
+static cudaError_t encode_2d(CUtensorMap* map, CUtensorMapDataType type, const void* base, uint64_t inner,
+                             uint64_t rows, uint64_t row_bytes, uint32_t box_inner, uint32_t box_rows,
+                             CUtensorMapSwizzle swz) {
+  return encode_tiled_2d(map, type, base, inner, rows, row_bytes, box_inner, box_rows, swz);
 }
 
 static cudaLaunchAttribute pdl_attr() {
