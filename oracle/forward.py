@@ -61,6 +61,35 @@ def forward_factored_bitmap(X: np.ndarray, pd: dict, pb: dict) -> np.ndarray:
     return Y
 
 
+def decode_coeff_fmt_entries(pf: dict):
+    """(atoms, values fp64) of every stored entry of a C_l packed by
+    pack_coeff_fmt (any of Table 4's coefficient formats)."""
+    from . import valuefmt as VF
+    fmt = pf.get("fmt", "nvfp4")
+    if fmt == "nvfp4":
+        return decode_coeff_entries(pf)
+    if fmt == "fp16":
+        vals = VF.fp16_decode(pf["values"])
+    elif fmt == "fp8":
+        vals = VF.fp8_decode(pf["values"], pf["s"])
+    else:
+        vals = VF.int8_decode(pf["values"].view(np.int8), pf["s"])
+    return coeff_entry_atoms(pf), vals
+
+
+def forward_factored_fmt(X: np.ndarray, pd: dict, pf: dict) -> np.ndarray:
+    """(X D) C in fp64 with NVFP4 D and C in any of Table 4's formats."""
+    Z = np.asarray(X).astype(np.float64) @ decode_dictionary(pd)
+    atoms, vals = decode_coeff_fmt_entries(pf)
+    ptr = pf["col_ptr"].astype(np.int64)
+    Y = np.zeros((Z.shape[0], pf["d_out"]), dtype=np.float64)
+    contrib = Z[:, atoms] * vals[None, :]
+    nonempty = np.flatnonzero(np.diff(ptr) > 0)
+    if nonempty.size:
+        Y[:, nonempty] = np.add.reduceat(contrib, ptr[nonempty], axis=1)
+    return Y
+
+
 def decode_coeff_dense(pc: dict) -> np.ndarray:
     """C-hat as a dense fp64 (k, d_out) matrix, zeros off the support."""
     k, d_out = pc["k"], pc["d_out"]
@@ -212,4 +241,5 @@ __all__ = [
     "forward_dense", "sparse_columns_product", "forward_factored", "forward_reference",
     "forward_brute", "sampled_outputs", "sampled_outputs_rows", "within_tolerance", "decode_projection",
     "forward_factored_decoded", "decode_coeff_bitmap_entries", "forward_factored_bitmap",
+    "decode_coeff_fmt_entries", "forward_factored_fmt",
 ]

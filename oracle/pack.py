@@ -126,6 +126,40 @@ def pack_coeff(col_ptr: np.ndarray, atom_idx: np.ndarray, vals: np.ndarray, k: i
     }
 
 
+def pack_coeff_fmt(col_ptr: np.ndarray, atom_idx: np.ndarray, vals: np.ndarray, k: int, d_out: int,
+                   fmt: str) -> dict:
+    """C_l with its values in one of Table 4's coefficient formats (fp16, fp8,
+    int8; see valuefmt) and the same index, padding and column pointers as
+    pack_coeff. The values array holds one code per stored entry (padding
+    entries: code 0): uint8 for fp8 / int8 (int8 as two's complement), uint16
+    bit patterns for fp16; s is the per-tensor fp32 scale (1 for fp16)."""
+    from . import valuefmt as VF
+    if fmt == "nvfp4":
+        return pack_coeff(col_ptr, atom_idx, vals, k, d_out)
+    if fmt not in VF.FORMATS:
+        raise ValueError(f"unknown coefficient format {fmt}")
+    pc = pack_coeff(col_ptr, atom_idx, vals, k, d_out)
+    col_ptr = np.asarray(col_ptr, dtype=np.int64)
+    vals = np.asarray(vals, dtype=np.float32)
+    pptr = pc["col_ptr"].astype(np.int64)
+    total = int(pptr[-1])
+    pvals = np.zeros(total, dtype=np.float32)
+    for o in range(d_out):
+        n = int(col_ptr[o + 1] - col_ptr[o])
+        pvals[pptr[o]:pptr[o] + n] = vals[col_ptr[o]:col_ptr[o + 1]]
+    if fmt == "fp16":
+        s, codes = np.float32(1.0), VF.fp16_encode(pvals)
+    elif fmt == "fp8":
+        s = VF.fp8_scale(vals)
+        codes = VF.fp8_encode(pvals, s)
+    else:
+        s = VF.int8_scale(vals)
+        codes = VF.int8_encode(pvals, s).view(np.uint8)
+    out = {n: pc[n] for n in ("k", "d_out", "nseg", "col_ptr", "nnz", "idx", "seg_start")}
+    out.update(fmt=fmt, values=codes, s=np.float32(s))
+    return out
+
+
 def pack_coeff_bitmap(col_ptr: np.ndarray, atom_idx: np.ndarray, vals: np.ndarray, k: int,
                       d_out: int) -> dict:
     """C_l with a bitmap support index: the review's Eq. (12) case a = 0, h = 1
