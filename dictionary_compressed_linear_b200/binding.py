@@ -60,6 +60,9 @@ SIGNATURES = [
      [_i32p, _i32p, _f32p, C.c_int, C.c_int, _u32p, _u32p, _u8p, _u8p, _u8p, _u16p, _f32p]),
     ("dictproj_pack_layer_bitmap_host", C.c_int,
      [_i32p, _i32p, _f32p, C.c_int, C.c_int, _u32p, _u32p, _u8p, _u8p, _u32p, _f32p]),
+    ("dictproj_cfmt_value_bytes", C.c_int, [C.c_int]),
+    ("dictproj_pack_layer_fmt_host", C.c_int,
+     [_i32p, _i32p, _f32p, C.c_int, C.c_int, C.c_int, _u32p, _u32p, C.c_void_p, _u8p, _u16p, _f32p]),
     ("dictproj_group_upload", C.c_int,
      [_u8p, _u8p, C.c_float, C.c_int, C.c_int, C.c_int, C.POINTER(C.c_void_p)]),
     ("dictproj_pack_group", C.c_int, [_f32p, C.c_int, C.c_int, C.c_int, C.POINTER(C.c_void_p)]),
@@ -216,6 +219,32 @@ def dictproj_pack_layer_bitmap_host(col_ptr, atom_idx, vals, k: int, d_out: int)
         _ptr(out["col_ptr"], C.c_uint32), _ptr(out["nnz"], C.c_uint32), _ptr(out["codes"], C.c_uint8),
         _ptr(out["scales"], C.c_uint8), _ptr(out["bitmap"], C.c_uint32), C.byref(s)))
     out.update(k=k, d_out=d_out, words=words, s=np.float32(s.value))
+    return out
+
+
+CFMT = {"nvfp4": 0, "fp16": 1, "fp8": 2, "int8": 3}
+
+
+def dictproj_pack_layer_fmt_host(col_ptr, atom_idx, vals, k: int, d_out: int, fmt: str) -> dict:
+    """C_l with FP16 / FP8 / INT8 values (Table 4) and the u8 index."""
+    col_ptr = np.ascontiguousarray(col_ptr, dtype=np.int32)
+    atom_idx = np.ascontiguousarray(atom_idx, dtype=np.int32)
+    vals = np.ascontiguousarray(vals, dtype=np.float32)
+    total = dictproj_layer_packed_entries(col_ptr, k, d_out)
+    nseg = -(-k // 256)
+    f = CFMT[fmt]
+    vb = lib().dictproj_cfmt_value_bytes(f)
+    out = {
+        "col_ptr": np.zeros(d_out + 1, np.uint32), "nnz": np.zeros(d_out, np.uint32),
+        "values": np.zeros(total, np.uint16 if vb == 2 else np.uint8),
+        "idx": np.zeros(total, np.uint8), "seg_start": np.zeros(d_out * nseg, np.uint16),
+    }
+    s = C.c_float()
+    _check(lib().dictproj_pack_layer_fmt_host(
+        _ptr(col_ptr, C.c_int32), _ptr(atom_idx, C.c_int32), _ptr(vals, C.c_float), k, d_out, f,
+        _ptr(out["col_ptr"], C.c_uint32), _ptr(out["nnz"], C.c_uint32), out["values"].ctypes.data_as(C.c_void_p),
+        _ptr(out["idx"], C.c_uint8), _ptr(out["seg_start"], C.c_uint16), C.byref(s)))
+    out.update(k=k, d_out=d_out, nseg=nseg, fmt=fmt, s=np.float32(s.value))
     return out
 
 

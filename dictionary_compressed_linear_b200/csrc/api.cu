@@ -143,6 +143,22 @@ int dictproj_pack_layer_bitmap_host(const int32_t* col_ptr, const int32_t* atom_
   return pack_layer_bitmap_host(col_ptr, atom_idx, vals, k, d_out, pcol_ptr, nnz, codes, scales, bitmap, s_C);
 }
 
+int dictproj_cfmt_value_bytes(int fmt) {
+  switch (fmt) {
+    case DICTPROJ_CFMT_FP16: return 2;
+    case DICTPROJ_CFMT_FP8:
+    case DICTPROJ_CFMT_INT8: return 1;
+    default: return 0;
+  }
+}
+
+int dictproj_pack_layer_fmt_host(const int32_t* col_ptr, const int32_t* atom_idx, const float* vals, int k,
+                                 int d_out, int fmt, uint32_t* pcol_ptr, uint32_t* nnz, void* values,
+                                 uint8_t* idx, uint16_t* seg_start, float* s_C) {
+  clear_error();
+  return pack_layer_fmt_host(col_ptr, atom_idx, vals, k, d_out, fmt, pcol_ptr, nnz, values, idx, seg_start, s_C);
+}
+
 void dictproj_free_group(dictproj_group* g) {
   if (!g) return;
   cudaFree(g->codes);

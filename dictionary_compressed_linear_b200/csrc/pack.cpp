@@ -55,6 +55,32 @@ static inline uint8_t e2m1_encode(float q) {
   return (q < 0.0f && mag != 0) ? (uint8_t)(mag | 8) : mag;
 }
 
+// IEEE binary16 bits of x, round to nearest even, written from the format's
+// definition: quanta of 2^(E-10) in the binade [2^E, 2^(E+1)), 2^-24 below 2^-14
+// (subnormals; a value that rounds up to 2^-14 lands on the first normal code).
+// Returns false if |x| rounds beyond the largest finite value (65504).
+static inline bool fp16_encode(float x, uint16_t* out) {
+  const float a = std::fabs(x);
+  const uint16_t sign = std::signbit(x) ? 0x8000 : 0;
+  uint32_t bits;
+  if (a < 0x1p-14f) {
+    bits = (uint32_t)std::nearbyintf(std::ldexp(a, 24));  // 0 .. 1024
+  } else {
+    int e2;
+    std::frexp(a, &e2);
+    int E = e2 - 1;
+    uint32_t n = (uint32_t)std::nearbyintf(std::ldexp(a, 10 - E));  // 1024 .. 2048
+    if (n == 2048) {
+      n = 1024;
+      E += 1;
+    }
+    if (E > 15) return false;
+    bits = ((uint32_t)(E + 15) << 10) | (n - 1024);
+  }
+  *out = (uint16_t)(sign | bits);
+  return true;
+}
+
 static inline float tensor_scale_from_amax(float amax) {
   if (amax == 0.0f) return 1.0f;
   return amax / 2688.0f;
@@ -231,6 +257,59 @@ int pack_layer_host(const int32_t* col_ptr, const int32_t* atom_idx, const float
     return fail(DICTPROJ_ERR_NULL, "pack_layer_host: NULL pointer");
   return pack_layer_core(col_ptr, atom_idx, vals, k, d_out, pcol_ptr, nnz, codes, scales, idx, seg_start, nullptr,
                          s_C);
+}
+
+// C_l with its stored values in one of Table 4's coefficient formats (FP16,
+// FP8 E4M3, INT8) and the u8 index of the NVFP4 layout: one code per stored
+// entry (padding entries 0), one fp32 per-tensor scale (1 for FP16).
+int pack_layer_fmt_host(const int32_t* col_ptr, const int32_t* atom_idx, const float* vals, int k, int d_out,
+                        int fmt, uint32_t* pcol_ptr, uint32_t* nnz, void* values, uint8_t* idx,
+                        uint16_t* seg_start, float* s_C) {
+  if (fmt == DICTPROJ_CFMT_NVFP4)
+    return fail(DICTPROJ_ERR_RANGE, "pack_layer_fmt_host: NVFP4 coefficients are packed by dictproj_pack_layer_host");
+  if (fmt != DICTPROJ_CFMT_FP16 && fmt != DICTPROJ_CFMT_FP8 && fmt != DICTPROJ_CFMT_INT8)
+    return fail(DICTPROJ_ERR_RANGE, "pack_layer_fmt_host: unknown coefficient format %d", fmt);
+  if (!col_ptr || !pcol_ptr || !nnz || !values || !idx || !seg_start || !s_C)
+    return fail(DICTPROJ_ERR_NULL, "pack_layer_fmt_host: NULL pointer");
+  size_t total = 0;
+  int st = layer_packed_entries(col_ptr, k, d_out, &total);
+  if (st) return st;
+  // the index, padding and column pointers of the NVFP4 layout (its codes and scales are discarded)
+  std::vector<uint8_t> codes(total / 2 + 1), scales(total / 16 + 1);
+  float s_nv = 0.f;
+  if ((st = pack_layer_core(col_ptr, atom_idx, vals, k, d_out, pcol_ptr, nnz, codes.data(), scales.data(), idx,
+                            seg_start, nullptr, &s_nv)))
+    return st;
+  const size_t nz = (size_t)col_ptr[d_out];
+  float amax = 0.0f;
+  for (size_t i = 0; i < nz; ++i) amax = std::fmax(amax, std::fabs(vals[i]));
+  float s = 1.0f;
+  if (fmt == DICTPROJ_CFMT_FP8) s = amax == 0.0f ? 1.0f : amax / 448.0f;
+  if (fmt == DICTPROJ_CFMT_INT8) s = amax == 0.0f ? 1.0f : amax / 127.0f;
+  std::fesetround(FE_TONEAREST);
+  for (int o = 0; o < d_out; ++o) {
+    const int32_t b0 = col_ptr[o], n = col_ptr[o + 1] - b0;
+    const uint32_t p0 = pcol_ptr[o], P = pcol_ptr[o + 1] - p0;
+    for (uint32_t q = 0; q < P; ++q) {
+      const float x = q < (uint32_t)n ? vals[b0 + q] : 0.0f;
+      if (fmt == DICTPROJ_CFMT_FP16) {
+        uint16_t h;
+        if (!fp16_encode(x, &h))
+          return fail(DICTPROJ_ERR_VALUE, "pack_layer_fmt_host: value %g of column %d outside the fp16 range", x, o);
+        static_cast<uint16_t*>(values)[p0 + q] = h;
+      } else if (fmt == DICTPROJ_CFMT_FP8) {
+        const float r = x / s;
+        const uint8_t mag = e4m3_encode_nonneg(std::fabs(r));
+        static_cast<uint8_t*>(values)[p0 + q] = (r < 0.0f && mag) ? (uint8_t)(mag | 0x80) : mag;
+      } else {
+        float c = std::nearbyintf(x / s);
+        c = std::fmin(127.0f, std::fmax(-127.0f, c));
+        static_cast<int8_t*>(values)[p0 + q] = (int8_t)c;
+      }
+    }
+  }
+  *s_C = s;
+  return DICTPROJ_OK;
 }
 
 int pack_layer_bitmap_host(const int32_t* col_ptr, const int32_t* atom_idx, const float* vals, int k, int d_out,

@@ -121,6 +121,29 @@ int dictproj_pack_layer_bitmap_host(const int32_t* col_ptr, const int32_t* atom_
                                     int k, int d_out, uint32_t* pcol_ptr, uint32_t* nnz, uint8_t* codes,
                                     uint8_t* scales, uint32_t* bitmap, float* s_C);
 
+/* Coefficient value formats: NVFP4 (the default layout above) and the three
+ * other coefficient formats of the paper's Table 4 (with an NVFP4 dictionary). */
+enum { DICTPROJ_CFMT_NVFP4 = 0, DICTPROJ_CFMT_FP16 = 1, DICTPROJ_CFMT_FP8 = 2, DICTPROJ_CFMT_INT8 = 3 };
+
+/* Bytes of one stored coefficient value in format fmt (NVFP4: 0, it packs two
+ * per byte plus a scale per 16; see dictproj_pack_layer_host). */
+int dictproj_cfmt_value_bytes(int fmt);
+
+/* C_l with its values in FP16, FP8 or INT8 (Table 4) and the index of the NVFP4
+ * layout: pcol_ptr, nnz, idx and seg_start exactly as dictproj_pack_layer_host
+ * writes them; values holds one code per stored entry (padding entries 0):
+ *   DICTPROJ_CFMT_FP16  uint16 binary16 bits of x (round to nearest even), s_C = 1;
+ *   DICTPROJ_CFMT_FP8   uint8 E4M3FN: sign | the magnitude code nearest to |x| / s_C
+ *                       (ties to even, saturating at 448), s_C = amax / 448;
+ *   DICTPROJ_CFMT_INT8  int8 nearest integer to x / s_C (ties to even), clamped to
+ *                       [-127, 127], s_C = amax / 127 (s_C = 1 if amax = 0).
+ * Value = s_C * decoded code. values: total_entries codes of
+ * dictproj_cfmt_value_bytes(fmt) bytes. Errors: NULL, SHAPE, RANGE (format, index,
+ * order), VALUE (non-finite value; an FP16 value beyond 65504). */
+int dictproj_pack_layer_fmt_host(const int32_t* col_ptr, const int32_t* atom_idx, const float* vals, int k,
+                                 int d_out, int fmt, uint32_t* pcol_ptr, uint32_t* nnz, void* values,
+                                 uint8_t* idx, uint16_t* seg_start, float* s_C);
+
 /* ------------------------------------------------------------------------- */
 /* Device objects                                                             */
 /* ------------------------------------------------------------------------- */

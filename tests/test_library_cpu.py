@@ -191,3 +191,42 @@ def test_bitmap_layer_packer_bit_exact(dp, k, d_out, rho):
     for n in ("col_ptr", "nnz", "codes", "scales", "bitmap"):
         assert np.array_equal(a[n], b[n]), n
     assert a["s"] == b["s"] and a["words"] == b["words"]
+
+
+@pytest.mark.parametrize("fmt", ["fp16", "fp8", "int8"])
+@pytest.mark.parametrize("k,d_out,rho", [(128, 64, 0.5), (2048, 300, 0.3), (272, 45, 0.05), (16, 7, 1.0)])
+def test_value_format_packer_bit_exact(dp, fmt, k, d_out, rho):
+    from oracle.pack import pack_coeff_fmt
+    C = synth.gen_coeff(8, k, d_out, 3, k, d_out, rho)
+    vals = C.vals.copy()
+    if vals.size > 8:  # exercise ties, zeros, tiny and large magnitudes
+        vals[0] = 0.0
+        vals[1] = -0.0
+        vals[2] = 1e-30
+        vals[3] = float(np.max(np.abs(vals))) * 1.0
+        vals[4] = 3.0517578125e-05 * 1.5  # between fp16 subnormals
+    a = dp.dictproj_pack_layer_fmt_host(C.col_ptr, C.atom_idx, vals, k, d_out, fmt)
+    b = pack_coeff_fmt(C.col_ptr, C.atom_idx, vals, k, d_out, fmt)
+    for n in ("col_ptr", "nnz", "values", "idx", "seg_start"):
+        assert np.array_equal(a[n], b[n]), n
+    assert a["s"] == b["s"]
+
+
+def test_fp16_value_packer_matches_the_binary16_definition_everywhere(dp):
+    # magnitudes across the whole binary16 range, including subnormals and the
+    # rounding boundary at the top; compared with numpy's float16 cast
+    rng = np.random.default_rng(12)
+    e = rng.uniform(-27, 15.99, 20000)
+    x = (np.sign(rng.standard_normal(20000)) * 2.0 ** e).astype(np.float32)
+    x[:4] = [65504.0, -65504.0, 65519.0, 2.0 ** -25]
+    n = x.size
+    ptr = np.array([0, n], np.int32)
+    atoms = np.arange(n, dtype=np.int32)
+    a = dp.dictproj_pack_layer_fmt_host(ptr, atoms, x, n + (-n) % 16, 1, "fp16")
+    want = x.astype(np.float16).view(np.uint16)
+    assert np.array_equal(a["values"][:n], want)
+    from dictionary_compressed_linear_b200 import DictprojError
+    with pytest.raises(DictprojError) as e:
+        dp.dictproj_pack_layer_fmt_host(np.array([0, 1], np.int32), atoms[:1], np.array([65520.0], np.float32), 16, 1,
+                                        "fp16")
+    assert e.value.status == -10
