@@ -23,6 +23,7 @@ STATUS = {
     -10: "DICTPROJ_ERR_VALUE", -11: "DICTPROJ_ERR_IO",
 }
 PATH_AUTO, PATH_DECODE, PATH_PREFILL = 0, 1, 2
+CFMT = {"nvfp4": 0, "fp16": 1, "fp8": 2, "int8": 3}  # DICTPROJ_CFMT_*
 
 
 class DictprojError(RuntimeError):
@@ -61,6 +62,12 @@ SIGNATURES = [
     ("dictproj_pack_layer_bitmap_host", C.c_int,
      [_i32p, _i32p, _f32p, C.c_int, C.c_int, _u32p, _u32p, _u8p, _u8p, _u32p, _f32p]),
     ("dictproj_cfmt_value_bytes", C.c_int, [C.c_int]),
+    ("dictproj_layer_upload_fmt", C.c_int,
+     [_u32p, C.c_void_p, _u8p, _u16p, C.c_float, C.c_int, C.c_int, C.c_int, C.POINTER(C.c_void_p)]),
+    ("dictproj_pack_layer_fmt", C.c_int,
+     [_i32p, _i32p, _f32p, C.c_int, C.c_int, C.c_int, C.POINTER(C.c_void_p)]),
+    ("dictproj_layer_format", C.c_int, [C.c_void_p, _intp]),
+    ("dictproj_layer_export_fmt", C.c_int, [C.c_void_p, _u32p, C.c_void_p, _u8p, _u16p, _f32p]),
     ("dictproj_pack_layer_fmt_host", C.c_int,
      [_i32p, _i32p, _f32p, C.c_int, C.c_int, C.c_int, _u32p, _u32p, C.c_void_p, _u8p, _u16p, _f32p]),
     ("dictproj_group_upload", C.c_int,
@@ -222,9 +229,6 @@ def dictproj_pack_layer_bitmap_host(col_ptr, atom_idx, vals, k: int, d_out: int)
     return out
 
 
-CFMT = {"nvfp4": 0, "fp16": 1, "fp8": 2, "int8": 3}
-
-
 def dictproj_pack_layer_fmt_host(col_ptr, atom_idx, vals, k: int, d_out: int, fmt: str) -> dict:
     """C_l with FP16 / FP8 / INT8 values (Table 4) and the u8 index."""
     col_ptr = np.ascontiguousarray(col_ptr, dtype=np.int32)
@@ -379,6 +383,50 @@ def dictproj_pack_layer(col_ptr, atom_idx, vals, k: int, d_out: int) -> Layer:
     _check(lib().dictproj_pack_layer(_ptr(col_ptr, C.c_int32), _ptr(atom_idx, C.c_int32),
                                      _ptr(vals, C.c_float), k, d_out, C.byref(h)))
     return Layer(h.value, k, d_out)
+
+
+def dictproj_layer_upload_fmt(packed: dict) -> Layer:
+    """Upload a layer packed by dictproj_pack_layer_fmt_host (FP16 / FP8 / INT8 values)."""
+    h = C.c_void_p()
+    a = {n: np.ascontiguousarray(packed[n]) for n in ("col_ptr", "values", "idx", "seg_start")}
+    _check(lib().dictproj_layer_upload_fmt(_ptr(a["col_ptr"], C.c_uint32), a["values"].ctypes.data_as(C.c_void_p),
+                                           _ptr(a["idx"], C.c_uint8), _ptr(a["seg_start"], C.c_uint16),
+                                           float(packed["s"]), packed["k"], packed["d_out"], CFMT[packed["fmt"]],
+                                           C.byref(h)))
+    return Layer(h.value, packed["k"], packed["d_out"])
+
+
+def dictproj_pack_layer_fmt(col_ptr, atom_idx, vals, k: int, d_out: int, fmt: str) -> Layer:
+    col_ptr = np.ascontiguousarray(col_ptr, dtype=np.int32)
+    atom_idx = np.ascontiguousarray(atom_idx, dtype=np.int32)
+    vals = np.ascontiguousarray(vals, dtype=np.float32)
+    h = C.c_void_p()
+    _check(lib().dictproj_pack_layer_fmt(_ptr(col_ptr, C.c_int32), _ptr(atom_idx, C.c_int32),
+                                         _ptr(vals, C.c_float), k, d_out, CFMT[fmt], C.byref(h)))
+    return Layer(h.value, k, d_out)
+
+
+def dictproj_layer_format(layer: Layer) -> str:
+    f = C.c_int()
+    _check(lib().dictproj_layer_format(layer.handle, C.byref(f)))
+    return {v: k for k, v in CFMT.items()}[f.value]
+
+
+def dictproj_layer_export_fmt(layer: Layer) -> dict:
+    k, d_out = layer.k, layer.d_out
+    t, n = C.c_size_t(), C.c_size_t()
+    _check(lib().dictproj_layer_info(layer.handle, None, None, C.byref(t), C.byref(n)))
+    fmt = dictproj_layer_format(layer)
+    vb = lib().dictproj_cfmt_value_bytes(CFMT[fmt])
+    nseg = -(-k // 256)
+    out = {"col_ptr": np.zeros(d_out + 1, np.uint32), "values": np.zeros(t.value, np.uint16 if vb == 2 else np.uint8),
+           "idx": np.zeros(t.value, np.uint8), "seg_start": np.zeros(d_out * nseg, np.uint16)}
+    s = C.c_float()
+    _check(lib().dictproj_layer_export_fmt(layer.handle, _ptr(out["col_ptr"], C.c_uint32),
+                                           out["values"].ctypes.data_as(C.c_void_p), _ptr(out["idx"], C.c_uint8),
+                                           _ptr(out["seg_start"], C.c_uint16), C.byref(s)))
+    out.update(k=k, d_out=d_out, nseg=nseg, fmt=fmt, s=np.float32(s.value))
+    return out
 
 
 def dictproj_pack(D, max_tokens: int, layers) -> tuple:

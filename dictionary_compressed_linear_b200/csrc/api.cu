@@ -285,12 +285,15 @@ int dictproj_group_reserve_prefill(dictproj_group* g, int max_d_out) {
   return DICTPROJ_OK;
 }
 
-int dictproj_layer_upload(const uint32_t* pcol_ptr, const uint8_t* codes, const uint8_t* scales,
-                          const uint8_t* idx, const uint16_t* seg_start, float s_C, int k, int d_out,
-                          dictproj_layer** out) {
-  clear_error();
-  if (!pcol_ptr || !codes || !scales || !idx || !seg_start || !out)
+// Upload of a packed C_l in format fmt: NVFP4 (codes + scales) or FP16 / FP8 /
+// INT8 (values in `codes`, one per stored entry; `scales` unused).
+static int layer_upload_impl(const uint32_t* pcol_ptr, const uint8_t* codes, const uint8_t* scales,
+                             const uint8_t* idx, const uint16_t* seg_start, float s_C, int k, int d_out, int fmt,
+                             dictproj_layer** out) {
+  if (!pcol_ptr || !codes || (fmt == DICTPROJ_CFMT_NVFP4 && !scales) || !idx || !seg_start || !out)
     return fail(DICTPROJ_ERR_NULL, "layer_upload: NULL pointer");
+  if (fmt < DICTPROJ_CFMT_NVFP4 || fmt > DICTPROJ_CFMT_INT8)
+    return fail(DICTPROJ_ERR_RANGE, "layer_upload: unknown coefficient format %d", fmt);
   *out = nullptr;
   if (k <= 0 || k % 16 || k > 65535 || d_out <= 0)
     return fail(DICTPROJ_ERR_SHAPE, "layer_upload: need 0 < k <= 65535, k %% 16 == 0, d_out > 0 (got k=%d d_out=%d)", k, d_out);
@@ -323,19 +326,22 @@ int dictproj_layer_upload(const uint32_t* pcol_ptr, const uint8_t* codes, const 
   l->nseg = nseg;
   l->s = s_C;
   l->total = pcol_ptr[d_out];
+  l->cfmt = fmt;
   const size_t T = l->total;
+  const size_t code_bytes = fmt == DICTPROJ_CFMT_NVFP4 ? T / 2 : T * (size_t)dictproj_cfmt_value_bytes(fmt);
+  const size_t scale_bytes = fmt == DICTPROJ_CFMT_NVFP4 ? T / 16 : 0;
   cudaError_t e;
-  // +16 bytes on every array so rounded-up L2 prefetch ranges stay inside the allocation
+  // +16 bytes on every array so rounded-up copy ranges stay inside the allocation
   if ((e = dmalloc((void**)&l->col_ptr, (d_out + 1) * sizeof(uint32_t) + 16)) ||
-      (e = dmalloc((void**)&l->codes, T / 2 + 16)) || (e = dmalloc((void**)&l->scales, T / 16 + 16)) ||
+      (e = dmalloc((void**)&l->codes, code_bytes + 16)) || (e = dmalloc((void**)&l->scales, scale_bytes + 16)) ||
       (e = dmalloc((void**)&l->idx, T + 16)) ||
       (e = dmalloc((void**)&l->seg_start, (size_t)d_out * nseg * sizeof(uint16_t) + 16))) {
     dictproj_free_layer(l);
     cudaGetLastError();
     return fail(DICTPROJ_ERR_OOM, "layer_upload: device allocation failed (%s)", cudaGetErrorName(e));
   }
-  if ((e = h2d(l->col_ptr, pcol_ptr, (d_out + 1) * sizeof(uint32_t))) || (e = h2d(l->codes, codes, T / 2)) ||
-      (e = h2d(l->scales, scales, T / 16)) || (e = h2d(l->idx, idx, T)) ||
+  if ((e = h2d(l->col_ptr, pcol_ptr, (d_out + 1) * sizeof(uint32_t))) || (e = h2d(l->codes, codes, code_bytes)) ||
+      (e = h2d(l->scales, scales, scale_bytes)) || (e = h2d(l->idx, idx, T)) ||
       (e = h2d(l->seg_start, seg_start, (size_t)d_out * nseg * sizeof(uint16_t)))) {
     dictproj_free_layer(l);
     cudaGetLastError();
@@ -347,12 +353,12 @@ int dictproj_layer_upload(const uint32_t* pcol_ptr, const uint8_t* codes, const 
     return cuda_fail(e, "layer_upload: device attributes");
   }
   l->n_sm = n_sm;
-  l->gather_ok = gather_supported(pcol_ptr, d_out, nseg);
+  l->gather_ok = fmt == DICTPROJ_CFMT_NVFP4 && gather_supported(pcol_ptr, d_out, nseg);
   {  // column chunks of the fused decode kernel
     std::vector<uint32_t> off;
     std::vector<uint4> chunks;
     int maxc = 0;
-    l->fused_ok = fused_layer_plan(pcol_ptr, d_out, nseg, n_sm, off, chunks, &maxc);
+    l->fused_ok = fused_layer_plan(pcol_ptr, d_out, nseg, fmt, n_sm, off, chunks, &maxc);
     l->cplan_max = maxc;
     if (l->fused_ok) {
       if ((e = dmalloc((void**)&l->cplan_off, off.size() * sizeof(uint32_t))) ||
@@ -372,6 +378,83 @@ int dictproj_layer_upload(const uint32_t* pcol_ptr, const uint8_t* codes, const 
   // the true entry count is not part of the packed arrays; dictproj_pack_layer records it
   l->nnz_total = 0;
   *out = l;
+  return DICTPROJ_OK;
+}
+
+int dictproj_layer_upload(const uint32_t* pcol_ptr, const uint8_t* codes, const uint8_t* scales,
+                          const uint8_t* idx, const uint16_t* seg_start, float s_C, int k, int d_out,
+                          dictproj_layer** out) {
+  clear_error();
+  return layer_upload_impl(pcol_ptr, codes, scales, idx, seg_start, s_C, k, d_out, DICTPROJ_CFMT_NVFP4, out);
+}
+
+int dictproj_layer_upload_fmt(const uint32_t* pcol_ptr, const void* values, const uint8_t* idx,
+                              const uint16_t* seg_start, float s_C, int k, int d_out, int fmt,
+                              dictproj_layer** out) {
+  clear_error();
+  if (fmt == DICTPROJ_CFMT_NVFP4)
+    return fail(DICTPROJ_ERR_RANGE, "layer_upload_fmt: NVFP4 layers are uploaded by dictproj_layer_upload");
+  return layer_upload_impl(pcol_ptr, static_cast<const uint8_t*>(values), nullptr, idx, seg_start, s_C, k, d_out, fmt,
+                           out);
+}
+
+int dictproj_pack_layer_fmt(const int32_t* col_ptr, const int32_t* atom_idx, const float* vals, int k, int d_out,
+                            int fmt, dictproj_layer** out) {
+  clear_error();
+  if (!col_ptr || !out) return fail(DICTPROJ_ERR_NULL, "pack_layer_fmt: NULL pointer");
+  *out = nullptr;
+  if (fmt == DICTPROJ_CFMT_NVFP4) return dictproj_pack_layer(col_ptr, atom_idx, vals, k, d_out, out);
+  if (k <= 0 || k % 16) return fail(DICTPROJ_ERR_SHAPE, "pack_layer_fmt: k must be a positive multiple of 16 (got %d)", k);
+  if (fmt < DICTPROJ_CFMT_FP16 || fmt > DICTPROJ_CFMT_INT8)
+    return fail(DICTPROJ_ERR_RANGE, "pack_layer_fmt: unknown coefficient format %d", fmt);
+  size_t total = 0;
+  int st = layer_packed_entries(col_ptr, k, d_out, &total);
+  if (st) return st;
+  const int nseg = (k + 255) / 256;
+  std::vector<uint32_t> pptr, nnz;
+  std::vector<uint8_t> values, idx;
+  std::vector<uint16_t> ss;
+  try {
+    pptr.resize(d_out + 1);
+    nnz.resize(d_out);
+    values.resize(total * (size_t)dictproj_cfmt_value_bytes(fmt) + 2);
+    idx.resize(total + 1);
+    ss.resize((size_t)d_out * nseg);
+  } catch (...) {
+    return fail(DICTPROJ_ERR_OOM, "pack_layer_fmt: host allocation failed");
+  }
+  float s = 0.f;
+  if ((st = pack_layer_fmt_host(col_ptr, atom_idx, vals, k, d_out, fmt, pptr.data(), nnz.data(), values.data(),
+                                idx.data(), ss.data(), &s)))
+    return st;
+  if ((st = layer_upload_impl(pptr.data(), values.data(), nullptr, idx.data(), ss.data(), s, k, d_out, fmt, out)))
+    return st;
+  (*out)->nnz_total = (size_t)col_ptr[d_out];
+  return DICTPROJ_OK;
+}
+
+int dictproj_layer_format(const dictproj_layer* l, int* fmt) {
+  clear_error();
+  if (!l || !fmt) return fail(DICTPROJ_ERR_NULL, "layer_format: NULL pointer");
+  *fmt = l->cfmt;
+  return DICTPROJ_OK;
+}
+
+int dictproj_layer_export_fmt(const dictproj_layer* l, uint32_t* pcol_ptr, void* values, uint8_t* idx,
+                              uint16_t* seg_start, float* s_C) {
+  clear_error();
+  if (!l || !pcol_ptr || !values || !idx || !seg_start || !s_C)
+    return fail(DICTPROJ_ERR_NULL, "layer_export_fmt: NULL pointer");
+  if (l->cfmt == DICTPROJ_CFMT_NVFP4)
+    return fail(DICTPROJ_ERR_UNSUPPORTED, "layer_export_fmt: an NVFP4 layer is exported by dictproj_layer_export");
+  const size_t T = l->total;
+  cudaError_t e;
+  if ((e = cudaMemcpy(pcol_ptr, l->col_ptr, (l->d_out + 1) * sizeof(uint32_t), cudaMemcpyDeviceToHost)) ||
+      (e = cudaMemcpy(values, l->codes, T * (size_t)dictproj_cfmt_value_bytes(l->cfmt), cudaMemcpyDeviceToHost)) ||
+      (e = cudaMemcpy(idx, l->idx, T, cudaMemcpyDeviceToHost)) ||
+      (e = cudaMemcpy(seg_start, l->seg_start, (size_t)l->d_out * l->nseg * sizeof(uint16_t), cudaMemcpyDeviceToHost)))
+    return cuda_fail(e, "layer_export_fmt");
+  *s_C = l->s;
   return DICTPROJ_OK;
 }
 
@@ -462,6 +545,8 @@ int dictproj_layer_export(const dictproj_layer* l, uint32_t* pcol_ptr, uint8_t* 
   clear_error();
   if (!l || !pcol_ptr || !codes || !scales || !idx || !seg_start || !s_C)
     return fail(DICTPROJ_ERR_NULL, "layer_export: NULL pointer");
+  if (l->cfmt != DICTPROJ_CFMT_NVFP4)
+    return fail(DICTPROJ_ERR_UNSUPPORTED, "layer_export: the layer's values are not NVFP4; use dictproj_layer_export_fmt");
   const size_t T = l->total;
   cudaError_t e;
   if ((e = cudaMemcpy(pcol_ptr, l->col_ptr, (l->d_out + 1) * sizeof(uint32_t), cudaMemcpyDeviceToHost)) ||
@@ -524,6 +609,10 @@ int dictproj_forward_path(const void* X, int M, const dictproj_layer* layer, con
         return cuda_fail(e, "forward: fused decode launch");
       return DICTPROJ_OK;
     }
+    if (layer->cfmt != DICTPROJ_CFMT_NVFP4)
+      return fail(DICTPROJ_ERR_UNSUPPORTED,
+                  "forward: FP16 / FP8 / INT8 coefficients are decoded by the fused kernel only (d_in >= 512, k <= "
+                  "8192, Z within shared memory); this call falls outside it");
     if (!coeff_smem_fits(group->k, mp, dev))
       return fail(DICTPROJ_ERR_UNSUPPORTED,
                   "forward: the decode path stages (k + 256) * %d floats of Z in shared memory; k=%d does not fit "
@@ -599,6 +688,10 @@ int dictproj_forward_batch(int n, const void* const* X, int M, const dictproj_la
       return DICTPROJ_OK;
     }
   }
+  for (int i = 0; i < n; ++i)
+    if (layers[i]->cfmt != DICTPROJ_CFMT_NVFP4)
+      return fail(DICTPROJ_ERR_UNSUPPORTED, "forward_batch: entry %d has FP16 / FP8 / INT8 coefficients, which only "
+                  "the fused kernel decodes, and the batch falls outside it", i);
   for (int i = 0; i < n; ++i)
     if (!coeff_smem_fits(groups[i]->k, mp, dev))
       return fail(DICTPROJ_ERR_UNSUPPORTED,
@@ -686,6 +779,8 @@ int dictproj_coefficient_stage(const float* Z, int M, const dictproj_layer* laye
   if (M < 1) return fail(DICTPROJ_ERR_RANGE, "coefficient_stage: M=%d < 1", M);
   if (M > kDecodeMaxTokens) return fail(DICTPROJ_ERR_UNSUPPORTED, "coefficient_stage: M must be <= %d", kDecodeMaxTokens);
   if (((uintptr_t)Y & 15) || ((uintptr_t)Z & 15)) return fail(DICTPROJ_ERR_ALIGN, "coefficient_stage: Z and Y must be 16-byte aligned");
+  if (layer->cfmt != DICTPROJ_CFMT_NVFP4)
+    return fail(DICTPROJ_ERR_UNSUPPORTED, "coefficient_stage: NVFP4 coefficients only");
   if (!coeff_smem_fits(layer->k, decode_mp(M), layer->device))
     return fail(DICTPROJ_ERR_UNSUPPORTED, "coefficient_stage: (k + 256) * mp floats of Z do not fit in shared "
                 "memory (k=%d, M=%d)", layer->k, M);

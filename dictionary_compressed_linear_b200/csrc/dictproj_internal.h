@@ -86,6 +86,7 @@ struct dictproj_layer {
   uint16_t* seg_start;     // [d_out][nseg]
   int n_sm;                // SMs of the device
   bool gather_ok;          // the gather kernel serves this layer (else the direct kernel)
+  int cfmt;                // coefficient value format: NVFP4 (codes + scales) or FP16 / FP8 / INT8 (codes = values)
   // fused decode kernel: column chunks of each of the n_sm positions
   bool fused_ok;
   uint32_t* cplan_off;     // [n_sm + 1]

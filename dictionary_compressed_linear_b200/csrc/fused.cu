@@ -76,15 +76,20 @@ struct CChunk {
 
 __host__ __device__ inline uint32_t up16(uint32_t x) { return (x + 15u) & ~15u; }
 
+// Nibbles of one stored coefficient value: NVFP4 1 (plus a scale byte per 16),
+// FP8 / INT8 2, FP16 4.
+__host__ __device__ inline uint32_t cfmt_nibbles(int fmt) { return fmt == 0 ? 1u : fmt == 1 ? 4u : 2u; }
+
 __host__ __device__ inline CChunk c_chunk_layout(uint32_t o_a, uint32_t o_b, uint32_t E_a, uint32_t E_b,
-                                                 uint32_t nseg) {
+                                                 uint32_t nseg, int fmt) {
+  const uint32_t vn = cfmt_nibbles(fmt);
   CChunk c;
   c.idx_src = E_a;
   c.idx_bytes = E_b - E_a;
-  c.code_src = (E_a >> 1) & ~15u;
-  c.code_bytes = up16(E_b >> 1) - c.code_src;
-  c.sc_src = (E_a >> 4) & ~15u;
-  c.sc_bytes = up16(E_b >> 4) - c.sc_src;
+  c.code_src = ((E_a * vn) >> 1) & ~15u;
+  c.code_bytes = up16((E_b * vn) >> 1) - c.code_src;
+  c.sc_src = fmt == 0 ? (E_a >> 4) & ~15u : 0u;
+  c.sc_bytes = fmt == 0 ? up16(E_b >> 4) - c.sc_src : 0u;
   c.ss_src = (2u * o_a * nseg) & ~15u;
   c.ss_bytes = up16(2u * o_b * nseg) - c.ss_src;
   c.cp_src = (4u * o_a) & ~15u;
@@ -124,6 +129,7 @@ struct FusedProj {
   int d_in, k, d_out, nseg;
   int ppr, P, pq, pr, rot;    // pieces per atom row, pieces, P = pq*G + pr, position rotation
   int xoff;                   // byte offset of its staged X rows in shared memory, -1: read X from global
+  int cfmt;                   // coefficient value format (DICTPROJ_CFMT_*)
   int xfirst;                 // 1: this projection stages X at xoff (later ones with the same X reuse it)
   int zt_off;                 // byte offset of its Z table in shared memory
 };
@@ -257,7 +263,39 @@ __device__ __forceinline__ void piece_quarter(float acc[2][4], uint32_t box, uin
 // half-blocks. Lane l takes half-blocks 32 i + l; the segment of each entry
 // comes from per-window ballots over seg_start (one boundary per lane), several
 // boundaries inside one half-block fall back to a walk.
-template <int MP>
+// Eight stored values of half-block hb as four f16x2 (their fp16 forms are
+// exact: E2M1, E4M3 and small integers are fp16 numbers), for each format.
+template <int FMT>
+__device__ __forceinline__ void half_block_values(uint32_t code_a, int hb, uint32_t f[4]) {
+  if constexpr (FMT == 0) {  // NVFP4: 8 nibbles
+    e2m1x8_to_f16x2x4(lds_u32(code_a + 4 * hb), f);
+  } else if constexpr (FMT == 1) {  // FP16
+    const uint4 v = lds_u32x4(code_a + 16 * hb);
+    f[0] = v.x;
+    f[1] = v.y;
+    f[2] = v.z;
+    f[3] = v.w;
+  } else if constexpr (FMT == 2) {  // FP8 E4M3
+    const uint2 v = lds_u32x2(code_a + 8 * hb);
+    f[0] = e4m3x2_to_f16x2(v.x & 0xFFFF);
+    f[1] = e4m3x2_to_f16x2(v.x >> 16);
+    f[2] = e4m3x2_to_f16x2(v.y & 0xFFFF);
+    f[3] = e4m3x2_to_f16x2(v.y >> 16);
+  } else {  // INT8: |code| <= 127 is exact in fp16
+    const uint2 v = lds_u32x2(code_a + 8 * hb);
+    const uint32_t w[2] = {v.x, v.y};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const uint32_t word = w[i >> 1];
+      const int sh = 16 * (i & 1);
+      const __half2 h = __floats2half2_rn((float)(int8_t)((word >> sh) & 0xFF),
+                                          (float)(int8_t)((word >> (sh + 8)) & 0xFF));
+      f[i] = *reinterpret_cast<const uint32_t*>(&h);
+    }
+  }
+}
+
+template <int MP, int FMT>
 __device__ __forceinline__ void column_sum(float acc[MP], uint32_t idx_a, uint32_t code_a, uint32_t sc_a,
                                            uint32_t ss_a, int nhb, int nseg, uint32_t zs_a, int lane) {
   constexpr uint32_t kRow = MP * 4;
@@ -286,7 +324,7 @@ __device__ __forceinline__ void column_sum(float acc[MP], uint32_t idx_a, uint32
       const uint2 iv = lds_u32x2(idx_a + 8 * hb);
       const uint32_t iw[2] = {iv.x, iv.y};
       uint32_t f[4];
-      e2m1x8_to_f16x2x4(lds_u32(code_a + 4 * hb), f);
+      half_block_values<FMT>(code_a, hb, f);
       float a0[MP], a1[MP];
 #pragma unroll
       for (int m = 0; m < MP; ++m) a0[m] = a1[m] = 0.f;
@@ -322,9 +360,14 @@ __device__ __forceinline__ void column_sum(float acc[MP], uint32_t idx_a, uint32
           }
         }
       }
-      const float sc = e4m3_to_f32(lds_u8(sc_a + (hb >> 1)));
+      if constexpr (FMT == 0) {
+        const float sc = e4m3_to_f32(lds_u8(sc_a + (hb >> 1)));
 #pragma unroll
-      for (int m = 0; m < MP; ++m) acc[m] = fmaf(a0[m] + a1[m], sc, acc[m]);
+        for (int m = 0; m < MP; ++m) acc[m] = fmaf(a0[m] + a1[m], sc, acc[m]);
+      } else {
+#pragma unroll
+        for (int m = 0; m < MP; ++m) acc[m] += a0[m] + a1[m];
+      }
     }
   }
 #pragma unroll
@@ -451,7 +494,7 @@ __global__ void __launch_bounds__(kFThreads, 2) k_decode_fused(const __grid_cons
         const int t = j - nD;
         const uint4 d = desc[t];
         const FusedProj& pp = prm.p[desc_p[t]];
-        const CChunk c = c_chunk_layout(d.x, d.y, d.z, d.w, (uint32_t)pp.nseg);
+        const CChunk c = c_chunk_layout(d.x, d.y, d.z, d.w, (uint32_t)pp.nseg, pp.cfmt);
         mbar_arrive_expect_tx(full + s, c.total);
         if (c.idx_bytes) bulk_g2s_u32(dst, pp.cidx + c.idx_src, c.idx_bytes, full + s);
         if (c.code_bytes) bulk_g2s_u32(dst + c.code_dst, pp.ccodes + c.code_src, c.code_bytes, full + s);
@@ -509,6 +552,10 @@ __global__ void __launch_bounds__(kFThreads, 2) k_decode_fused(const __grid_cons
       misc[1] = (int)((unsigned int)(tk / (unsigned long long)G) + 1u);
       mbar_arrive_cta(rdy);
       trigger_dependents();
+      // Slots are freed only by the compute warps, which first wait for the
+      // previous grid on the stream; wait for it here too, so that the bounded
+      // waits below measure this kernel's own progress, however long that grid runs.
+      grid_dependency_wait();
       const int nall = nD + total;
       for (int j = issued; j < nall; ++j) {
         const int s = j % R;
@@ -688,7 +735,9 @@ __global__ void __launch_bounds__(kFThreads, 2) k_decode_fused(const __grid_cons
       if (!ok) continue;
       const FusedProj& pp = prm.p[p];
       const uint4 d = desc[i];
-      const CChunk c = c_chunk_layout(d.x, d.y, d.z, d.w, (uint32_t)pp.nseg);
+      const int fmt = pp.cfmt;
+      const CChunk c = c_chunk_layout(d.x, d.y, d.z, d.w, (uint32_t)pp.nseg, fmt);
+      const uint32_t vn = cfmt_nibbles(fmt);
       const uint32_t slot = sbase + (uint32_t)s * kFusedSlotBytes;
       const int ncols = (int)(d.y - d.x);
       const uint32_t zs = sbase + pp.zt_off;
@@ -696,10 +745,17 @@ __global__ void __launch_bounds__(kFThreads, 2) k_decode_fused(const __grid_cons
         const uint32_t o = d.x + (uint32_t)t;
         const uint32_t cpa = slot + c.cp_dst + 4u * o - c.cp_src;
         const uint32_t e0 = lds_u32(cpa), e1 = lds_u32(cpa + 4);
+        const uint32_t ia = slot + (e0 - d.z), ca = slot + c.code_dst + ((e0 * vn) >> 1) - c.code_src;
+        const uint32_t sa = slot + c.sc_dst + (e0 >> 4) - c.sc_src;
+        const uint32_t ssa = slot + c.ss_dst + 2u * o * (uint32_t)pp.nseg - c.ss_src;
+        const int nhb = (int)((e1 - e0) >> 3);
         float y[MP];
-        column_sum<MP>(y, slot + (e0 - d.z), slot + c.code_dst + (e0 >> 1) - c.code_src,
-                       slot + c.sc_dst + (e0 >> 4) - c.sc_src, slot + c.ss_dst + 2u * o * (uint32_t)pp.nseg - c.ss_src,
-                       (int)((e1 - e0) >> 3), pp.nseg, zs, lane);
+        switch (fmt) {  // uniform over the chunk
+          case 0: column_sum<MP, 0>(y, ia, ca, sa, ssa, nhb, pp.nseg, zs, lane); break;
+          case 1: column_sum<MP, 1>(y, ia, ca, sa, ssa, nhb, pp.nseg, zs, lane); break;
+          case 2: column_sum<MP, 2>(y, ia, ca, sa, ssa, nhb, pp.nseg, zs, lane); break;
+          default: column_sum<MP, 3>(y, ia, ca, sa, ssa, nhb, pp.nseg, zs, lane); break;
+        }
         if (lane == 0) {
 #pragma unroll
           for (int m = 0; m < MP; ++m)
@@ -773,20 +829,21 @@ cudaError_t fused_group_setup(dictproj_group* g, bool* ok) {
   return cudaSuccess;
 }
 
-bool fused_layer_plan(const uint32_t* pcol_ptr, int d_out, int nseg, int G, std::vector<uint32_t>& off,
+bool fused_layer_plan(const uint32_t* pcol_ptr, int d_out, int nseg, int fmt, int G, std::vector<uint32_t>& off,
                       std::vector<uint4>& chunks, int* max_per_pos) {
   off.assign(G + 1, 0);
   chunks.clear();
   *max_per_pos = 0;
   if (nseg > 32) return false;
   auto fits = [&](int oa, int ob) {
-    return c_chunk_layout(oa, ob, pcol_ptr[oa], pcol_ptr[ob], nseg).total <= (uint32_t)kFusedSlotBytes;
+    return c_chunk_layout(oa, ob, pcol_ptr[oa], pcol_ptr[ob], nseg, fmt).total <= (uint32_t)kFusedSlotBytes;
   };
-  // bytes streamed per column (balancing weight): entries + codes + scales + seg_start + col_ptr
+  // bytes streamed per column (balancing weight): index + values (+ scales) + seg_start + col_ptr
+  const double per_entry = 1.0 + cfmt_nibbles(fmt) * 0.5 + (fmt == 0 ? 1.0 / 16 : 0.0);
   std::vector<double> cum(d_out + 1, 0.0);
   for (int o = 0; o < d_out; ++o) {
     const double ne = (double)(pcol_ptr[o + 1] - pcol_ptr[o]);
-    cum[o + 1] = cum[o] + ne * (1.0 + 0.5 + 1.0 / 16) + 2.0 * nseg + 4.0;
+    cum[o + 1] = cum[o] + ne * per_entry + 2.0 * nseg + 4.0;
     if (!fits(o, o + 1)) return false;  // a column larger than a ring slot
   }
   auto lower = [&](int lo, int hi, double target) {  // first o in [lo, hi] with cum[o] >= target
@@ -937,6 +994,7 @@ cudaError_t launch_fused(int n, const dictproj_group* const* g, const dictproj_l
     p.seg_start = l[i]->seg_start;
     p.cplan_off = l[i]->cplan_off;
     p.cplan = l[i]->cplan;
+    p.cfmt = l[i]->cfmt;
     p.s_D = g[i]->s;
     p.s_C = l[i]->s;
     p.d_in = g[i]->d_in;

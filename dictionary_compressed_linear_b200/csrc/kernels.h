@@ -56,7 +56,7 @@ cudaError_t prepare_fused_kernels(int device);
 cudaError_t fused_group_setup(dictproj_group* g, bool* ok);
 // Column chunks of a layer for G positions: off[G+1] into chunks {o_a, o_b, E_a, E_b}.
 // False if a column does not fit a ring slot (the layer then runs the two-kernel path).
-bool fused_layer_plan(const uint32_t* pcol_ptr, int d_out, int nseg, int G, std::vector<uint32_t>& off,
+bool fused_layer_plan(const uint32_t* pcol_ptr, int d_out, int nseg, int fmt, int G, std::vector<uint32_t>& off,
                       std::vector<uint4>& chunks, int* max_per_pos);
 // Shared-memory plan of one launch; false if the fused kernel does not serve it.
 bool fused_plan_launch(int n, const dictproj_group* const* g, const dictproj_layer* const* l,

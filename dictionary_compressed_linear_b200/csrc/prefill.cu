@@ -422,6 +422,34 @@ __global__ void __launch_bounds__(DictTile::kThreads, 1)
 // the next chunk's loads are issued before the current one is scattered.
 // Entries with code 0 (value 0, and the padding at the end of each column) are
 // skipped. The column's segment starts sit in shared memory.
+// Four consecutive stored values (entry e, e % 4 == 0) in format FMT: raw code
+// bits (NVFP4: 4 nibbles, FP8 / INT8: 4 bytes, FP16: 4 halves) and, for NVFP4,
+// the block's E4M3 scale byte.
+template <int FMT>
+__device__ __forceinline__ uint2 load4_values(const uint8_t* codes, uint32_t e) {
+  if constexpr (FMT == 0) return make_uint2(*reinterpret_cast<const uint16_t*>(codes + (e >> 1)), 0u);
+  else if constexpr (FMT == 1) return *reinterpret_cast<const uint2*>(codes + 2 * e);
+  else return make_uint2(*reinterpret_cast<const uint32_t*>(codes + e), 0u);
+}
+// fp16 value of entry t (0..3) of a group loaded by load4_values (unscaled by s_C;
+// NVFP4: E2M1 x E4M3 block scale, exact in fp16), and whether it is zero.
+template <int FMT>
+__device__ __forceinline__ uint32_t value4(uint2 v, uint32_t sv, int t) {
+  if constexpr (FMT == 0) {
+    const uint32_t code = (v.x >> (4 * t)) & 15;
+    return (code & 7) == 0 ? 0u : hmul2_u32(e2m1x2_to_f16x2(code), sv) & 0xFFFF;
+  } else if constexpr (FMT == 1) {
+    return ((t < 2 ? v.x : v.y) >> (16 * (t & 1))) & 0xFFFF;
+  } else if constexpr (FMT == 2) {
+    const uint32_t b = (v.x >> (8 * t)) & 0xFF;
+    return (b & 0x7F) == 0 ? 0u : e4m3x2_to_f16x2(b) & 0xFFFF;
+  } else {
+    const int c = (int)(int8_t)((v.x >> (8 * t)) & 0xFF);
+    return (uint32_t)__half_as_ushort(__int2half_rn(c));
+  }
+}
+
+template <int FMT>
 __global__ void __launch_bounds__(256)
     k_densify_coeff(const uint32_t* __restrict__ col_ptr, const uint8_t* __restrict__ codes,
                     const uint8_t* __restrict__ scales, const uint8_t* __restrict__ idx,
@@ -440,34 +468,35 @@ __global__ void __launch_bounds__(256)
   __syncwarp();
   const uint32_t e0 = col_ptr[o], e1 = col_ptr[o + 1];
   int seg = 0;  // segment of this lane's entries; they only increase
-  uint32_t i4 = 0, c4 = 0, sc = 0;
+  uint32_t i4 = 0, sc = 0;
+  uint2 c4 = make_uint2(0, 0);
   {
     const uint32_t e = e0 + 4 * lane;
     if (e < e1) {
       i4 = *reinterpret_cast<const uint32_t*>(idx + e);
-      c4 = *reinterpret_cast<const uint16_t*>(codes + (e >> 1));
-      sc = scales[e >> 4];
+      c4 = load4_values<FMT>(codes, e);
+      if (FMT == 0) sc = scales[e >> 4];
     }
   }
   for (uint32_t base = e0; base < e1; base += 128) {
     const uint32_t e = base + 4 * lane, en = e + 128;
-    uint32_t ni4 = 0, nc4 = 0, nsc = 0;  // next chunk, loaded before this one is scattered
+    uint32_t ni4 = 0, nsc = 0;  // next chunk, loaded before this one is scattered
+    uint2 nc4 = make_uint2(0, 0);
     if (en < e1) {
       ni4 = *reinterpret_cast<const uint32_t*>(idx + en);
-      nc4 = *reinterpret_cast<const uint16_t*>(codes + (en >> 1));
-      nsc = scales[en >> 4];
+      nc4 = load4_values<FMT>(codes, en);
+      if (FMT == 0) nsc = scales[en >> 4];
     }
     if (e < e1) {
-      const uint32_t sv = e4m3x2_to_f16x2(sc) & 0xFFFF;
+      const uint32_t sv = FMT == 0 ? dup_lo(e4m3x2_to_f16x2(sc)) : 0u;
 #pragma unroll
       for (int t = 0; t < 4; ++t) {
-        const uint32_t code = (c4 >> (4 * t)) & 15;
-        if ((code & 7) == 0) continue;  // +-0 and padding
+        const uint32_t h = value4<FMT>(c4, sv, t);
+        if ((h & 0x7FFF) == 0) continue;  // +-0 and padding
         const int q = (int)(e - e0) + t;
         while (seg + 1 < nseg && (int)ss[seg + 1] <= q) ++seg;
         const uint32_t atom = 256u * seg + ((i4 >> (8 * t)) & 255);
-        const uint32_t prod = hmul2_u32(e2m1x2_to_f16x2(code), sv);  // exact in fp16
-        row[atom] = __ushort_as_half((unsigned short)(prod & 0xFFFF));
+        row[atom] = __ushort_as_half((unsigned short)h);
       }
     }
     i4 = ni4;
@@ -542,7 +571,11 @@ cudaError_t prepare_prefill_kernels(int device) {
       (e = cudaFuncSetAttribute(k_dict_prefill, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 (int)DictTile::smem)))
     return e;
-  return cudaFuncSetAttribute(k_densify_coeff, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
+  if ((e = cudaFuncSetAttribute(k_densify_coeff<0>, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024)) ||
+      (e = cudaFuncSetAttribute(k_densify_coeff<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024)) ||
+      (e = cudaFuncSetAttribute(k_densify_coeff<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024)))
+    return e;
+  return cudaFuncSetAttribute(k_densify_coeff<3>, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
 }
 
 cudaError_t take_prefill_error(unsigned int* out) {
@@ -612,7 +645,12 @@ cudaError_t launch_densify_coeff(const dictproj_layer* l, __half* Cd, cudaStream
   int k = l->k, d_out = l->d_out, nseg = l->nseg;
   void* args[] = {(void*)&l->col_ptr, (void*)&l->codes, (void*)&l->scales, (void*)&l->idx, (void*)&l->seg_start,
                   &k, &d_out, &nseg, (void*)&Cd};
-  return cudaLaunchKernelExC(&cfg, (const void*)k_densify_coeff, args);
+  switch (l->cfmt) {
+    case 0: return cudaLaunchKernelExC(&cfg, (const void*)k_densify_coeff<0>, args);
+    case 1: return cudaLaunchKernelExC(&cfg, (const void*)k_densify_coeff<1>, args);
+    case 2: return cudaLaunchKernelExC(&cfg, (const void*)k_densify_coeff<2>, args);
+    default: return cudaLaunchKernelExC(&cfg, (const void*)k_densify_coeff<3>, args);
+  }
 }
 
 cudaError_t launch_coeff_prefill(const dictproj_layer* l, const __half* Z, const __half* Cd, int M, __half* Y,

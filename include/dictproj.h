@@ -176,6 +176,29 @@ int dictproj_layer_upload(const uint32_t* pcol_ptr, const uint8_t* codes, const 
 int dictproj_pack_layer(const int32_t* col_ptr, const int32_t* atom_idx, const float* vals, int k,
                         int d_out, dictproj_layer** out);
 
+/* A C_l with FP16 / FP8 / INT8 values (dictproj_pack_layer_fmt_host's arrays,
+ * `values` of dictproj_cfmt_value_bytes(fmt) bytes per stored entry) on the
+ * current device. Such a layer is decoded by the fused decode kernel
+ * (M <= 8, d_in >= 512, k <= 8192) and by the prefill path; other calls with it
+ * return UNSUPPORTED before any launch. dictproj_layer_save refuses it (the
+ * packed file holds NVFP4 layers). Errors as dictproj_layer_upload, plus RANGE
+ * (fmt not FP16 / FP8 / INT8). */
+int dictproj_layer_upload_fmt(const uint32_t* pcol_ptr, const void* values, const uint8_t* idx,
+                              const uint16_t* seg_start, float s_C, int k, int d_out, int fmt,
+                              dictproj_layer** out);
+
+/* dictproj_pack_layer_fmt_host + dictproj_layer_upload_fmt (fmt NVFP4: dictproj_pack_layer). */
+int dictproj_pack_layer_fmt(const int32_t* col_ptr, const int32_t* atom_idx, const float* vals, int k,
+                            int d_out, int fmt, dictproj_layer** out);
+
+/* The coefficient value format of a layer (DICTPROJ_CFMT_*). Errors: NULL. */
+int dictproj_layer_format(const dictproj_layer* l, int* fmt);
+
+/* Copy an FP16 / FP8 / INT8 layer's packed arrays back to host buffers of the
+ * packed sizes. Errors: NULL, UNSUPPORTED (an NVFP4 layer), CUDA. */
+int dictproj_layer_export_fmt(const dictproj_layer* l, uint32_t* pcol_ptr, void* values, uint8_t* idx,
+                              uint16_t* seg_start, float* s_C);
+
 /* Convenience: pack one group and its n_layers layers (all with the same k).
  * On error nothing is left allocated. */
 int dictproj_pack(const float* D, int d_in, int k, int max_tokens, int n_layers,
@@ -184,7 +207,8 @@ int dictproj_pack(const float* D, int d_in, int k, int max_tokens, int n_layers,
                   dictproj_layer** layers_out);
 
 /* Copy the packed bytes back to host buffers of the packed sizes (for
- * bit-exact checks). Errors: NULL, CUDA. */
+ * bit-exact checks). Errors: NULL, UNSUPPORTED (a layer whose values are not
+ * NVFP4: dictproj_layer_export_fmt), CUDA. */
 int dictproj_group_export(const dictproj_group* g, uint8_t* codes, uint8_t* scales, float* s_D);
 int dictproj_layer_export(const dictproj_layer* l, uint32_t* pcol_ptr, uint8_t* codes,
                           uint8_t* scales, uint8_t* idx, uint16_t* seg_start, float* s_C);

@@ -46,6 +46,15 @@ def test_fused_shapes(d_in, k, d_out, rho, M):
     g, l = device_projection(D, C, max_tokens=8)
     pd, pc = oracle_projection(D, C)
     X = synth.gen_activations(40, M, 0, M, d_in)
+    if (k + 256) * 8 * 4 > 227 * 1024 and M > 4:
+        # Z of k atoms for 8 token slots exceeds shared memory: refused before any launch
+        Xd = torch.from_numpy(X).cuda()
+        Y = torch.full((M, d_out), 3.0, dtype=torch.float16, device="cuda")
+        st = torch.cuda.current_stream().cuda_stream
+        assert dp.dictproj_forward_status(Xd.data_ptr(), M, l.handle, g.handle, Y.data_ptr(), st) == -9
+        torch.cuda.synchronize()
+        assert torch.all(Y == 3.0)
+        return
     assert_parity(run_forward(g, l, X), oracle_forward(X, pd, pc), f"fused d_in={d_in} k={k} d_out={d_out} M={M}")
 
 
