@@ -90,6 +90,29 @@ def forward_factored_fmt(X: np.ndarray, pd: dict, pf: dict) -> np.ndarray:
     return Y
 
 
+def decode_coeff_block_entries(pk: dict):
+    """(atoms, values fp64) of every stored entry of a block-structured C_l:
+    entry 16 b + i is atom 16 * blk_idx[b] + i."""
+    codes = unpack_nibbles(pk["codes"])
+    sc = np.repeat(np.asarray(pk["scales"]), 16)
+    vals = E2M1_TABLE[codes] * E4M3_TABLE[sc] * float(pk["s"])
+    atoms = (pk["blk_idx"].astype(np.int64)[:, None] * 16 + np.arange(16)).reshape(-1)
+    return atoms, vals
+
+
+def forward_factored_blocks(X: np.ndarray, pd: dict, pk: dict) -> np.ndarray:
+    """(X D) C in fp64 with a block-structured C_l."""
+    Z = np.asarray(X).astype(np.float64) @ decode_dictionary(pd)
+    atoms, vals = decode_coeff_block_entries(pk)
+    ptr = pk["blk_ptr"].astype(np.int64) * 16
+    Y = np.zeros((Z.shape[0], pk["d_out"]), dtype=np.float64)
+    contrib = Z[:, atoms] * vals[None, :]
+    nonempty = np.flatnonzero(np.diff(ptr) > 0)
+    if nonempty.size:
+        Y[:, nonempty] = np.add.reduceat(contrib, ptr[nonempty], axis=1)
+    return Y
+
+
 def decode_coeff_dense(pc: dict) -> np.ndarray:
     """C-hat as a dense fp64 (k, d_out) matrix, zeros off the support."""
     k, d_out = pc["k"], pc["d_out"]
@@ -241,5 +264,5 @@ __all__ = [
     "forward_dense", "sparse_columns_product", "forward_factored", "forward_reference",
     "forward_brute", "sampled_outputs", "sampled_outputs_rows", "within_tolerance", "decode_projection",
     "forward_factored_decoded", "decode_coeff_bitmap_entries", "forward_factored_bitmap",
-    "decode_coeff_fmt_entries", "forward_factored_fmt",
+    "decode_coeff_fmt_entries", "forward_factored_fmt", "decode_coeff_block_entries", "forward_factored_blocks",
 ]

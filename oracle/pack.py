@@ -160,6 +160,42 @@ def pack_coeff_fmt(col_ptr: np.ndarray, atom_idx: np.ndarray, vals: np.ndarray, 
     return out
 
 
+BLOCK = 16
+
+
+def pack_coeff_blocks(col_ptr: np.ndarray, atom_idx: np.ndarray, vals: np.ndarray, k: int, d_out: int) -> dict:
+    """C_l with block-structured support (the review's "Let the accelerator
+    constrain the support"; the paper names block-structured sparsity as future
+    work): every column's support is a union of whole aligned blocks of 16
+    consecutive atoms. A kept block is exactly one NVFP4 block (its 16 values,
+    one E4M3 scale), so the values, codes and scales equal those of pack_coeff on
+    the same support, and the index is one uint16 block number per 16 values:
+      blk_ptr uint32[d_out+1]  kept blocks before each column;
+      blk_idx uint16[nblk]     block number (atom // 16), ascending per column;
+      codes   uint8[nblk*8], scales uint8[nblk], s fp32 (per tensor)."""
+    col_ptr = np.asarray(col_ptr, dtype=np.int64)
+    atom_idx = np.asarray(atom_idx, dtype=np.int64)
+    if k % BLOCK:
+        raise ValueError("k must be a multiple of 16")
+    for o in range(d_out):
+        a = atom_idx[col_ptr[o]:col_ptr[o + 1]]
+        if a.size % BLOCK or np.any(a.reshape(-1, BLOCK) != (a[::BLOCK, None] // BLOCK) * BLOCK + np.arange(BLOCK)):
+            raise ValueError(f"column {o}: support is not a union of aligned 16-atom blocks")
+    pc = pack_coeff(col_ptr, atom_idx, vals, k, d_out)
+    nblk = np.diff(col_ptr) // BLOCK
+    blk_ptr = np.zeros(d_out + 1, dtype=np.int64)
+    blk_ptr[1:] = np.cumsum(nblk)
+    return {
+        "k": k,
+        "d_out": d_out,
+        "blk_ptr": blk_ptr.astype(np.uint32),
+        "blk_idx": (atom_idx[::BLOCK] // BLOCK).astype(np.uint16),
+        "codes": pc["codes"],
+        "scales": pc["scales"],
+        "s": pc["s"],
+    }
+
+
 def pack_coeff_bitmap(col_ptr: np.ndarray, atom_idx: np.ndarray, vals: np.ndarray, k: int,
                       d_out: int) -> dict:
     """C_l with a bitmap support index: the review's Eq. (12) case a = 0, h = 1

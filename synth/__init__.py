@@ -115,6 +115,26 @@ def gen_coeff(cfg: int, group: int, ptype: int, layer: int, k: int, d_out: int,
                        atom_idx=sup.reshape(-1).copy(), vals=vals)
 
 
+def gen_coeff_blocks(cfg: int, group: int, ptype: int, layer: int, k: int, d_out: int, rho: float,
+                     block: int = 16) -> SparseCoeff:
+    """C_l (k x d_out) whose support is block-structured: every column keeps
+    nb = k/block - floor((1-rho) k/block) whole aligned blocks of `block`
+    consecutive atoms, drawn uniformly without replacement; the retained values
+    are N(0, 1/k)."""
+    if k % block:
+        raise ValueError("k must be a multiple of the block size")
+    kb = k // block
+    nb = kb - int(math.floor((1.0 - rho) * kb))
+    blocks = gen_support(cfg, group, ptype, layer, kb, d_out, nb)  # sorted block numbers per column
+    atoms = (blocks[:, :, None] * block + np.arange(block, dtype=np.int32)[None, None, :]).reshape(d_out, -1)
+    g = _rng(cfg, group, ptype, layer, T_CVALS)
+    vals = g.standard_normal(d_out * nb * block, dtype=np.float32)
+    vals *= np.float32(1.0 / math.sqrt(k))
+    col_ptr = (np.arange(d_out + 1, dtype=np.int64) * nb * block).astype(np.int32)
+    return SparseCoeff(k=k, d_out=d_out, col_ptr=col_ptr, atom_idx=atoms.reshape(-1).astype(np.int32).copy(),
+                       vals=vals)
+
+
 def gen_activations(cfg: int, layer: int, site: int, M: int, d_in: int,
                     outlier_frac: float = 0.0, outlier_gain: float = 20.0) -> np.ndarray:
     """X as fp16, shape (M, d_in), row-major."""
