@@ -17,6 +17,6 @@ from .binding import (  # noqa: F401
     dictproj_group_export, dictproj_group_info, dictproj_group_packed_sizes, dictproj_group_upload,
     dictproj_last_error, dictproj_layer_export, dictproj_layer_info, dictproj_layer_packed_entries,
     dictproj_layer_upload, dictproj_pack, dictproj_pack_group, dictproj_pack_group_host,
-    dictproj_pack_layer, dictproj_pack_layer_host, dictproj_pack_layer_bitmap_host, dictproj_pack_layer_fmt_host, CFMT, dictproj_layer_upload_fmt,
+    dictproj_pack_layer, dictproj_pack_layer_host, dictproj_pack_layer_bitmap_host, dictproj_pack_layer_blocks_host, dictproj_pack_layer_fmt_host, CFMT, dictproj_layer_upload_fmt,
     dictproj_pack_layer_fmt, dictproj_layer_format, dictproj_layer_export_fmt, dictproj_status_string, dictproj_version,
 )

@@ -61,6 +61,8 @@ SIGNATURES = [
      [_i32p, _i32p, _f32p, C.c_int, C.c_int, _u32p, _u32p, _u8p, _u8p, _u8p, _u16p, _f32p]),
     ("dictproj_pack_layer_bitmap_host", C.c_int,
      [_i32p, _i32p, _f32p, C.c_int, C.c_int, _u32p, _u32p, _u8p, _u8p, _u32p, _f32p]),
+    ("dictproj_pack_layer_blocks_host", C.c_int,
+     [_i32p, _i32p, _f32p, C.c_int, C.c_int, _u32p, _u16p, _u8p, _u8p, _f32p]),
     ("dictproj_cfmt_value_bytes", C.c_int, [C.c_int]),
     ("dictproj_layer_upload_fmt", C.c_int,
      [_u32p, C.c_void_p, _u8p, _u16p, C.c_float, C.c_int, C.c_int, C.c_int, C.POINTER(C.c_void_p)]),
@@ -226,6 +228,26 @@ def dictproj_pack_layer_bitmap_host(col_ptr, atom_idx, vals, k: int, d_out: int)
         _ptr(out["col_ptr"], C.c_uint32), _ptr(out["nnz"], C.c_uint32), _ptr(out["codes"], C.c_uint8),
         _ptr(out["scales"], C.c_uint8), _ptr(out["bitmap"], C.c_uint32), C.byref(s)))
     out.update(k=k, d_out=d_out, words=words, s=np.float32(s.value))
+    return out
+
+
+def dictproj_pack_layer_blocks_host(col_ptr, atom_idx, vals, k: int, d_out: int) -> dict:
+    """C_l with block-structured support: whole aligned 16-atom blocks per column."""
+    col_ptr = np.ascontiguousarray(col_ptr, dtype=np.int32)
+    atom_idx = np.ascontiguousarray(atom_idx, dtype=np.int32)
+    vals = np.ascontiguousarray(vals, dtype=np.float32)
+    nblk = int(col_ptr[-1]) // 16
+    out = {"blk_ptr": np.zeros(d_out + 1, np.uint32), "blk_idx": np.zeros(max(nblk, 1), np.uint16),
+           "codes": np.zeros(max(nblk, 1) * 8, np.uint8), "scales": np.zeros(max(nblk, 1), np.uint8)}
+    s = C.c_float()
+    _check(lib().dictproj_pack_layer_blocks_host(
+        _ptr(col_ptr, C.c_int32), _ptr(atom_idx, C.c_int32), _ptr(vals, C.c_float), k, d_out,
+        _ptr(out["blk_ptr"], C.c_uint32), _ptr(out["blk_idx"], C.c_uint16), _ptr(out["codes"], C.c_uint8),
+        _ptr(out["scales"], C.c_uint8), C.byref(s)))
+    out["blk_idx"] = out["blk_idx"][:nblk]
+    out["codes"] = out["codes"][:nblk * 8]
+    out["scales"] = out["scales"][:nblk]
+    out.update(k=k, d_out=d_out, s=np.float32(s.value))
     return out
 
 

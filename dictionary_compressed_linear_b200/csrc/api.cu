@@ -136,6 +136,13 @@ int dictproj_pack_layer_host(const int32_t* col_ptr, const int32_t* atom_idx, co
   return pack_layer_host(col_ptr, atom_idx, vals, k, d_out, pcol_ptr, nnz, codes, scales, idx, seg_start, s_C);
 }
 
+int dictproj_pack_layer_blocks_host(const int32_t* col_ptr, const int32_t* atom_idx, const float* vals, int k,
+                                    int d_out, uint32_t* blk_ptr, uint16_t* blk_idx, uint8_t* codes, uint8_t* scales,
+                                    float* s_C) {
+  clear_error();
+  return pack_layer_blocks_host(col_ptr, atom_idx, vals, k, d_out, blk_ptr, blk_idx, codes, scales, s_C);
+}
+
 int dictproj_pack_layer_bitmap_host(const int32_t* col_ptr, const int32_t* atom_idx, const float* vals, int k,
                                     int d_out, uint32_t* pcol_ptr, uint32_t* nnz, uint8_t* codes, uint8_t* scales,
                                     uint32_t* bitmap, float* s_C) {

@@ -32,6 +32,8 @@ int pack_layer_host(const int32_t* col_ptr, const int32_t* atom_idx, const float
 int pack_layer_fmt_host(const int32_t* col_ptr, const int32_t* atom_idx, const float* vals, int k, int d_out,
                         int fmt, uint32_t* pcol_ptr, uint32_t* nnz, void* values, uint8_t* idx,
                         uint16_t* seg_start, float* s_C);
+int pack_layer_blocks_host(const int32_t* col_ptr, const int32_t* atom_idx, const float* vals, int k, int d_out,
+                           uint32_t* blk_ptr, uint16_t* blk_idx, uint8_t* codes, uint8_t* scales, float* s_C);
 int pack_layer_bitmap_host(const int32_t* col_ptr, const int32_t* atom_idx, const float* vals, int k, int d_out,
                            uint32_t* pcol_ptr, uint32_t* nnz, uint8_t* codes, uint8_t* scales, uint32_t* bitmap,
                            float* s_C);

@@ -312,6 +312,44 @@ int pack_layer_fmt_host(const int32_t* col_ptr, const int32_t* atom_idx, const f
   return DICTPROJ_OK;
 }
 
+// C_l with block-structured support: every column's atoms are whole aligned
+// blocks of 16; a kept block is one NVFP4 block (codes, scale) with a uint16
+// block number. blk_ptr counts kept blocks before each column.
+int pack_layer_blocks_host(const int32_t* col_ptr, const int32_t* atom_idx, const float* vals, int k, int d_out,
+                           uint32_t* blk_ptr, uint16_t* blk_idx, uint8_t* codes, uint8_t* scales, float* s_C) {
+  if (!col_ptr || !blk_ptr || !blk_idx || !codes || !scales || !s_C)
+    return fail(DICTPROJ_ERR_NULL, "pack_layer_blocks_host: NULL pointer");
+  if (k <= 0 || k % 16 || k > 65535 || d_out <= 0)
+    return fail(DICTPROJ_ERR_SHAPE, "pack_layer_blocks_host: need 0 < k <= 65535, k %% 16 == 0, d_out > 0");
+  if (col_ptr[0] != 0) return fail(DICTPROJ_ERR_RANGE, "pack_layer_blocks_host: col_ptr[0] must be 0");
+  for (int o = 0; o < d_out; ++o) {
+    const int32_t b0 = col_ptr[o], n = col_ptr[o + 1] - b0;
+    if (n < 0 || n > k || n % 16)
+      return fail(DICTPROJ_ERR_RANGE, "pack_layer_blocks_host: column %d holds %d entries, not whole 16-atom blocks", o,
+                  n);
+    for (int32_t q = 0; q < n; ++q)
+      if (atom_idx[b0 + q] != (atom_idx[b0 + (q & ~15)] & ~15) + (q & 15) || (atom_idx[b0 + (q & ~15)] & 15))
+        return fail(DICTPROJ_ERR_RANGE, "pack_layer_blocks_host: column %d is not a union of aligned 16-atom blocks", o);
+  }
+  // values, padding-free blocks and scales exactly as the u8 layout packs them
+  size_t total = 0;
+  int st = layer_packed_entries(col_ptr, k, d_out, &total);
+  if (st) return st;
+  std::vector<uint32_t> pptr(d_out + 1), nnz(d_out);
+  std::vector<uint8_t> idx(total + 1);
+  std::vector<uint16_t> ss((size_t)d_out * ((k + 255) / 256));
+  if ((st = pack_layer_core(col_ptr, atom_idx, vals, k, d_out, pptr.data(), nnz.data(), codes, scales, idx.data(),
+                            ss.data(), nullptr, s_C)))
+    return st;
+  blk_ptr[0] = 0;
+  for (int o = 0; o < d_out; ++o) {
+    const int32_t b0 = col_ptr[o], nb = (col_ptr[o + 1] - b0) / 16;
+    for (int32_t b = 0; b < nb; ++b) blk_idx[blk_ptr[o] + b] = (uint16_t)(atom_idx[b0 + 16 * b] >> 4);
+    blk_ptr[o + 1] = blk_ptr[o] + (uint32_t)nb;
+  }
+  return DICTPROJ_OK;
+}
+
 int pack_layer_bitmap_host(const int32_t* col_ptr, const int32_t* atom_idx, const float* vals, int k, int d_out,
                            uint32_t* pcol_ptr, uint32_t* nnz, uint8_t* codes, uint8_t* scales, uint32_t* bitmap,
                            float* s_C) {

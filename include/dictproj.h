@@ -121,6 +121,22 @@ int dictproj_pack_layer_bitmap_host(const int32_t* col_ptr, const int32_t* atom_
                                     int k, int d_out, uint32_t* pcol_ptr, uint32_t* nnz, uint8_t* codes,
                                     uint8_t* scales, uint32_t* bitmap, float* s_C);
 
+/* C_l with block-structured support (review, "Let the accelerator constrain
+ * the support"; block-structured sparsity is the paper's named future work):
+ * every column's retained atoms are whole aligned blocks of 16 consecutive
+ * atoms (col_ptr / atom_idx as for dictproj_pack_layer_host, each column a union
+ * of such blocks). A kept block is one NVFP4 block, so codes and scales are
+ * exactly those of dictproj_pack_layer_host on the same support (no padding is
+ * needed); the index is one uint16 block number (atom / 16) per kept block:
+ *   blk_ptr uint32[d_out+1]  kept blocks before each column;
+ *   blk_idx uint16[nblk]     ascending within a column;
+ *   codes uint8[nblk*8], scales uint8[nblk], s_C fp32.
+ * Errors as dictproj_pack_layer_host, plus RANGE (a column that is not a union of
+ * aligned 16-atom blocks). */
+int dictproj_pack_layer_blocks_host(const int32_t* col_ptr, const int32_t* atom_idx, const float* vals,
+                                    int k, int d_out, uint32_t* blk_ptr, uint16_t* blk_idx, uint8_t* codes,
+                                    uint8_t* scales, float* s_C);
+
 /* Coefficient value formats: NVFP4 (the default layout above) and the three
  * other coefficient formats of the paper's Table 4 (with an NVFP4 dictionary). */
 enum { DICTPROJ_CFMT_NVFP4 = 0, DICTPROJ_CFMT_FP16 = 1, DICTPROJ_CFMT_FP8 = 2, DICTPROJ_CFMT_INT8 = 3 };

@@ -230,3 +230,24 @@ def test_fp16_value_packer_matches_the_binary16_definition_everywhere(dp):
         dp.dictproj_pack_layer_fmt_host(np.array([0, 1], np.int32), atoms[:1], np.array([65520.0], np.float32), 16, 1,
                                         "fp16")
     assert e.value.status == -10
+
+
+@pytest.mark.parametrize("k,d_out,rho", [(2048, 64, 0.3), (3072, 40, 0.25), (64, 9, 1.0), (512, 33, 0.0)])
+def test_block_layer_packer_bit_exact(dp, k, d_out, rho):
+    from oracle.pack import pack_coeff_blocks
+    C = synth.gen_coeff_blocks(9, k, d_out, 1, k, d_out, rho)
+    a = dp.dictproj_pack_layer_blocks_host(C.col_ptr, C.atom_idx, C.vals, k, d_out)
+    b = pack_coeff_blocks(C.col_ptr, C.atom_idx, C.vals, k, d_out)
+    for n in ("blk_ptr", "blk_idx", "codes", "scales"):
+        assert np.array_equal(a[n], b[n]), n
+    assert a["s"] == b["s"]
+
+
+def test_block_layer_packer_rejects_unaligned_supports(dp):
+    from dictionary_compressed_linear_b200 import DictprojError
+    with pytest.raises(DictprojError) as e:
+        dp.dictproj_pack_layer_blocks_host(np.array([0, 16]), np.arange(1, 17), np.ones(16), 32, 1)
+    assert e.value.status == -5
+    with pytest.raises(DictprojError) as e:
+        dp.dictproj_pack_layer_blocks_host(np.array([0, 8]), np.arange(8), np.ones(8), 32, 1)
+    assert e.value.status == -5
