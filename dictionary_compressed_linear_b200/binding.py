@@ -117,6 +117,7 @@ SIGNATURES = [
     ("dictproj_layer_load", C.c_int, [C.c_char_p, C.POINTER(C.c_void_p)]),
     ("dictproj_check", C.c_int, [C.c_void_p]),
     ("dictproj_selftest_wait_timeout", C.c_int, [C.c_longlong, C.c_void_p]),
+    ("dictproj_diag_phase_times", C.c_int, [C.POINTER(C.c_ulonglong), C.c_int, _intp]),
     ("dictproj_last_error", C.c_char_p, []),
     ("dictproj_status_string", C.c_char_p, [C.c_int]),
     ("dictproj_version", C.c_int, []),
@@ -610,3 +611,11 @@ def dictproj_launch_count(X_ptrs, M: int, layers, groups) -> int:
                                        arr(*[l.handle for l in layers]), arr(*[g.handle for g in groups]),
                                        C.byref(cnt)))
     return cnt.value
+
+
+def dictproj_diag_phase_times(max_ctas: int = 1024) -> np.ndarray:
+    """Phase marks (ns) of the last fused decode launch, shape (ctas, 16)."""
+    out = np.zeros(max_ctas * 16, np.uint64)
+    n = C.c_int()
+    _check(lib().dictproj_diag_phase_times(out.ctypes.data_as(C.POINTER(C.c_ulonglong)), max_ctas, C.byref(n)))
+    return out[:n.value * 16].reshape(n.value, 16)

@@ -805,6 +805,16 @@ int dictproj_selftest_wait_timeout(long long cycles, void* stream) {
   return e == cudaSuccess ? DICTPROJ_OK : cuda_fail(e, "selftest_wait_timeout: launch");
 }
 
+int dictproj_diag_phase_times(unsigned long long* out, int max_ctas, int* n_ctas) {
+  clear_error();
+  if (!out || !n_ctas) return fail(DICTPROJ_ERR_NULL, "diag_phase_times: NULL pointer");
+  if (max_ctas < 1) return fail(DICTPROJ_ERR_RANGE, "diag_phase_times: max_ctas=%d < 1", max_ctas);
+  int dev, st;
+  if ((st = ensure_device(&dev))) return st;
+  cudaError_t e = fused_phase_times(out, max_ctas, n_ctas);
+  return e == cudaSuccess ? DICTPROJ_OK : cuda_fail(e, "diag_phase_times");
+}
+
 int dictproj_check(void* stream) {
   clear_error();
   cudaError_t e = cudaStreamSynchronize((cudaStream_t)stream);

@@ -13,18 +13,19 @@
 //     previous work on the stream (programmatic dependent launch): the ring of
 //     the next call fills while this call computes. A CTA uses at most half of
 //     an SM (M <= 4), so two consecutive calls are resident together.
-//   * stage 1: eight compute warps take 16-atom x 512-element pieces of D_g
+//   * stage 1: twelve compute warps take 16-atom x 512-element pieces of D_g
 //     from the ring, decode E2M1 x E4M3 to fp16 (exact) and run swap-AB
 //     mma.sync m16n8k16 (atoms = the 16 rows, tokens = the 8 columns) with fp32
 //     accumulation. Pieces are dealt to CTAs evenly: each CTA gets a contiguous
 //     run of a projection's pieces, so a 16-atom tile is split over at most a
 //     few CTAs, whose partial sums (times s_D) go to a per-group exchange buffer
 //     Zx[slot][k][mp] in L2.
-//   * one grid-wide exchange: each CTA publishes a flag with this launch's epoch
-//     (from a 64-bit ticket every CTA takes at start, so aborted launches never
-//     confuse later ones); after all flags are seen, every CTA sums the slots of
-//     each tile in a fixed order into its shared-memory Z table (bit-exact,
-//     independent of timing).
+//   * one grid-wide exchange: each CTA adds one to a 64-bit arrival count when
+//     its partial Z is written and waits until the count reaches this launch's
+//     target (from a 64-bit ticket every CTA takes at start; every CTA adds
+//     exactly one per launch, aborted or not, so later launches stay aligned);
+//     then every CTA sums the slots of each tile in a fixed order into its
+//     shared-memory Z table (bit-exact, independent of timing).
 //   * stage 2: the compute warps take the CTA's column chunks of C_l (columns
 //     split over CTAs by bytes, so by nnz) from the ring; one warp per column,
 //     lanes over 8-entry half-blocks, the same per-window segment logic as the
@@ -49,7 +50,7 @@ namespace dictproj {
 // ---------------------------------------------------------------------------------
 // geometry
 // ---------------------------------------------------------------------------------
-constexpr int kFWarps = 8;                       // compute warps
+constexpr int kFWarps = 12;                      // compute warps (one D quarter each per full slot)
 constexpr int kFThreads = 32 * (kFWarps + 1);    // + one producer warp
 constexpr int kPieceElems = 512;                 // d_in elements of one D piece (per atom)
 constexpr int kPieceCodeBytes = 16 * 256;        // 16 atoms x 256 code bytes (two 128-B boxes)
@@ -136,8 +137,8 @@ struct FusedProj {
 
 struct FusedParams {
   FusedProj p[kFusedMaxBatch];
-  unsigned long long* ticket;  // launches of this sync object x G CTAs so far
-  unsigned int* flags;         // [G] epoch + 1 of each CTA's published partial Z
+  unsigned long long* ticket;  // launches of this sync object x G CTAs so far (one ticket per CTA)
+  unsigned long long* arrive;  // CTAs that published their partial Z, over all launches (one per CTA)
   long long wait_limit;        // SM clocks a bounded wait may take
   int n, M, G, R;              // projections, tokens, CTAs, ring slots
   int xrow;                    // bytes per staged X row
@@ -177,15 +178,26 @@ __device__ __forceinline__ float4 ld_cg_f4(const float* p) {
   asm volatile("ld.global.cg.v4.f32 {%0,%1,%2,%3}, [%4];" : "=f"(r.x), "=f"(r.y), "=f"(r.z), "=f"(r.w) : "l"(p));
   return r;
 }
-__device__ __forceinline__ unsigned int ld_relaxed_u32(const unsigned int* p) {
-  unsigned int v;
-  asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+__device__ __forceinline__ void fence_acq_rel_gpu() { asm volatile("fence.acq_rel.gpu;" ::: "memory"); }
+__device__ __forceinline__ void atom_add_release_u64(unsigned long long* p, unsigned long long v) {
+  asm volatile("red.release.gpu.global.add.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
+}
+__device__ __forceinline__ unsigned long long ld_acquire_u64(const unsigned long long* p) {
+  unsigned long long v;
+  asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
   return v;
 }
-__device__ __forceinline__ void st_release_u32(unsigned int* p, unsigned int v) {
-  asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+
+// Diagnostic: wall-clock (ns) at the phase boundaries of the last fused launch,
+// per CTA (slots 0-7 compute side, 8-11 producer side); read by
+// dictproj_diag_phase_times. A few stores per CTA and launch.
+constexpr int kPhaseCtas = 1024, kPhaseSlots = 16;
+static __device__ unsigned long long g_phase[kPhaseCtas * kPhaseSlots];
+__device__ __forceinline__ void phase_mark(int cta, int slot) {
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  if (cta < kPhaseCtas) g_phase[cta * kPhaseSlots + slot] = t;
 }
-__device__ __forceinline__ void fence_acq_rel_gpu() { asm volatile("fence.acq_rel.gpu;" ::: "memory"); }
 __device__ __forceinline__ void sts_u32x4(uint32_t a, uint4 v) {
   asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};" ::"r"(a), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w) : "memory");
 }
@@ -465,6 +477,7 @@ __global__ void __launch_bounds__(kFThreads, 2) k_decode_fused(const __grid_cons
     }
   }
   __syncthreads();
+  if (threadIdx.x == 0) phase_mark(cta, 0);
   const int N1 = misc[3];
   const int nD = (N1 + kPiecesPerSlot - 1) / kPiecesPerSlot;
 
@@ -508,6 +521,7 @@ __global__ void __launch_bounds__(kFThreads, 2) k_decode_fused(const __grid_cons
     if (lane == 0 && !*s_abort) {  // the first slots are free: start streaming D at once
       issued = min(R, nD);
       for (int j = 0; j < issued; ++j) issue(j);
+      phase_mark(cta, 8);
     }
     // coefficient chunks of this CTA (position = CTA index) over all projections
     int beg = 0, cnt = 0;
@@ -549,13 +563,17 @@ __global__ void __launch_bounds__(kFThreads, 2) k_decode_fused(const __grid_cons
         *s_abort = 1;
       }
       misc[2] = total;
-      misc[1] = (int)((unsigned int)(tk / (unsigned long long)G) + 1u);
+      const unsigned long long base = (tk / (unsigned long long)G) * (unsigned long long)G;  // arrivals before this launch
+      misc[5] = (int)(unsigned int)(base >> 32);
+      misc[6] = (int)(unsigned int)(base & 0xffffffffull);
       mbar_arrive_cta(rdy);
       trigger_dependents();
+      phase_mark(cta, 9);
       // Slots are freed only by the compute warps, which first wait for the
       // previous grid on the stream; wait for it here too, so that the bounded
       // waits below measure this kernel's own progress, however long that grid runs.
       grid_dependency_wait();
+      phase_mark(cta, 10);
       const int nall = nD + total;
       for (int j = issued; j < nall; ++j) {
         const int s = j % R;
@@ -564,6 +582,7 @@ __global__ void __launch_bounds__(kFThreads, 2) k_decode_fused(const __grid_cons
         issue(j);
         issued = j + 1;
       }
+      phase_mark(cta, 11);
       if (*s_abort)  // let the copies in flight land before the CTA exits
         for (int j = max(0, issued - R); j < issued; ++j) mbar_wait_bounded(full + j % R, (uint32_t)((j / R) & 1), limit);
     }
@@ -571,7 +590,8 @@ __global__ void __launch_bounds__(kFThreads, 2) k_decode_fused(const __grid_cons
     // ------------------------------------------------------------- compute warps
     const int tid = threadIdx.x;
     const int g = lane >> 2, tq = lane & 3;
-    grid_dependency_wait();  // X, Zx, the flags and Y belong to earlier work on the stream
+    grid_dependency_wait();  // X, Zx and Y belong to earlier work on the stream
+    if (tid == 0) phase_mark(cta, 1);
     for (int i = tid; i < prm.n_tp * kFWarps * 16 * MP; i += kFWarps * 32) sts_f32(sbase + prm.red_off + 4 * i, 0.f);
     for (int p = 0; p < n; ++p) {  // stage X rows (element order permuted within 512-byte blocks)
       const FusedProj& pp = prm.p[p];
@@ -585,6 +605,7 @@ __global__ void __launch_bounds__(kFThreads, 2) k_decode_fused(const __grid_cons
       }
     }
     named_bar_sync(1, kFWarps * 32);
+    if (tid == 0) phase_mark(cta, 2);
 
     // ---- stage 1: partial Z of this CTA's D pieces
     float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
@@ -612,7 +633,7 @@ __global__ void __launch_bounds__(kFThreads, 2) k_decode_fused(const __grid_cons
       if (!ok) continue;
       const int np = min(kPiecesPerSlot, N1 - j * kPiecesPerSlot);
       const uint32_t slot = sbase + (uint32_t)s * kFusedSlotBytes;
-      for (int t = (warp + 4 * j) & 7; t < 4 * np; t += kFWarps) {  // quarters dealt round-robin, rotated per slot
+      for (int t = (warp + 4 * j) % kFWarps; t < 4 * np; t += kFWarps) {  // quarters dealt round-robin, rotated per slot
         const int L = j * kPiecesPerSlot + (t >> 2);
         int p = 0;
         for (int q = 1; q < n; ++q)
@@ -664,6 +685,7 @@ __global__ void __launch_bounds__(kFThreads, 2) k_decode_fused(const __grid_cons
     }
     if (cur_tp >= 0) flush(cur_tp);
     named_bar_sync(1, kFWarps * 32);
+    if (tid == 0) phase_mark(cta, 3);
 
     // ---- partial Z of each tile piece (sum over warps, times s_D) to the exchange buffer
     const int ntp = misc[4];
@@ -684,32 +706,32 @@ __global__ void __launch_bounds__(kFThreads, 2) k_decode_fused(const __grid_cons
     }
     named_bar_sync(1, kFWarps * 32);
 
-    // ---- grid-wide exchange: publish this CTA's flag, wait for every CTA's
-    if (warp == 0) {
-      bool ok = mbar_wait_or_abort(rdy, 0, s_abort, limit);
-      ok = __all_sync(0xffffffffu, ok) && !*s_abort;
+    // ---- grid-wide exchange: count this CTA in, wait until every CTA of this launch is
+    // (every CTA adds exactly one per launch, aborted or not, so the count stays a
+    // multiple of G between launches; one thread per CTA polls one word, with backoff)
+    if (tid == 0) {
+      phase_mark(cta, 4);
+      __threadfence();
+      atom_add_release_u64(prm.arrive, 1ull);
+      const bool ok = mbar_wait_or_abort(rdy, 0, s_abort, limit) && !*s_abort;
       if (ok) {
-        const unsigned int fv = (unsigned int)misc[1];
-        if (lane == 0) {
-          __threadfence();
-          st_release_u32(prm.flags + cta, fv);
-        }
+        const unsigned long long target = ((unsigned long long)(unsigned int)misc[5] << 32 |
+                                           (unsigned int)misc[6]) + (unsigned long long)G;
         const long long t0 = clock64();
-        while (true) {
-          bool mine = true;
-          for (int f = lane; f < G; f += 32) mine = mine && ld_relaxed_u32(prm.flags + f) == fv;
-          if (__all_sync(0xffffffffu, mine)) break;
-          const bool give = __any_sync(0xffffffffu, *s_abort != 0 || clock64() - t0 > limit);
-          if (give) {
-            if (lane == 0 && !*s_abort) {
+        unsigned int ns = 32;
+        while (ld_acquire_u64(prm.arrive) < target) {
+          if (*s_abort || clock64() - t0 > limit) {
+            if (!*s_abort) {
               atomicOr(&g_dictproj_error, 1u);
               *s_abort = 1;
             }
             break;
           }
+          __nanosleep(ns);
+          if (ns < 256) ns <<= 1;
         }
-        fence_acq_rel_gpu();
       }
+      phase_mark(cta, 5);
     }
     named_bar_sync(1, kFWarps * 32);
 
@@ -720,6 +742,7 @@ __global__ void __launch_bounds__(kFThreads, 2) k_decode_fused(const __grid_cons
         for (int p = 0; p < n; ++p) load_ztable<MP>(prm.p[p], sbase, tid);
       named_bar_sync(1, kFWarps * 32);
     }
+    if (tid == 0) phase_mark(cta, 6);
     int cur_p = -1;
     for (int i = 0; i < N2; ++i) {
       const int j = nD + i, s = j % R;
@@ -741,7 +764,7 @@ __global__ void __launch_bounds__(kFThreads, 2) k_decode_fused(const __grid_cons
       const uint32_t slot = sbase + (uint32_t)s * kFusedSlotBytes;
       const int ncols = (int)(d.y - d.x);
       const uint32_t zs = sbase + pp.zt_off;
-      for (int t = (warp + i) & 7; t < ncols; t += kFWarps) {
+      for (int t = (warp + i) % kFWarps; t < ncols; t += kFWarps) {
         const uint32_t o = d.x + (uint32_t)t;
         const uint32_t cpa = slot + c.cp_dst + 4u * o - c.cp_src;
         const uint32_t e0 = lds_u32(cpa), e1 = lds_u32(cpa + 4);
@@ -767,6 +790,7 @@ __global__ void __launch_bounds__(kFThreads, 2) k_decode_fused(const __grid_cons
     }
   }
   __syncthreads();
+  if (threadIdx.x == 0) phase_mark(cta, 7);
 }
 
 }  // namespace dictproj
@@ -821,7 +845,7 @@ cudaError_t fused_group_setup(dictproj_group* g, bool* ok) {
     return e;
   if ((e = cudaMalloc((void**)&g->zx, (size_t)g->zslots * g->k * kDecodeMaxTokens * sizeof(float))) != cudaSuccess)
     return e;
-  const size_t sync_bytes = 16 + (size_t)g->n_sm * sizeof(unsigned int);
+  const size_t sync_bytes = 2 * sizeof(unsigned long long);  // ticket, arrivals
   if ((e = cudaMalloc((void**)&g->fsync, sync_bytes)) != cudaSuccess) return e;
   if ((e = cudaMemset(g->fsync, 0, sync_bytes)) != cudaSuccess) return e;
   g->fused_ok = true;
@@ -890,6 +914,12 @@ bool fused_layer_plan(const uint32_t* pcol_ptr, int d_out, int nseg, int fmt, in
   return true;
 }
 
+cudaError_t fused_phase_times(unsigned long long* out, int max_ctas, int* n_ctas) {
+  const int n = std::min(max_ctas, kPhaseCtas);
+  *n_ctas = n;
+  return cudaMemcpyFromSymbol(out, g_phase, (size_t)n * kPhaseSlots * sizeof(unsigned long long));
+}
+
 cudaError_t prepare_fused_kernels(int device) {
   int optin = 0;
   cudaError_t e = cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, device);
@@ -937,7 +967,7 @@ bool fused_plan_launch(int n, const dictproj_group* const* g, const dictproj_lay
   }
   xtot = M * pl.xrow * nx;
   pl.stage_x = xtot <= kStageXMax;
-  const int red = pl.n_tp * 8 * 16 * mp * 4;
+  const int red = pl.n_tp * kFWarps * 16 * mp * 4;
   const int stage1 = (pl.stage_x ? xtot : 0) + red;
   int zall = 0, zone = 0;
   for (int i = 0; i < n; ++i) {
@@ -1012,7 +1042,7 @@ cudaError_t launch_fused(int n, const dictproj_group* const* g, const dictproj_l
     p.zt_off = pl.zt_off[i];
   }
   prm.ticket = g[0]->fsync;
-  prm.flags = reinterpret_cast<unsigned int*>(g[0]->fsync + 2);
+  prm.arrive = g[0]->fsync + 1;
   prm.wait_limit = wait_limit;
   prm.n = n;
   prm.M = M;

@@ -65,6 +65,8 @@ cudaError_t launch_fused(int n, const dictproj_group* const* g, const dictproj_l
                          const __half* const* X, __half* const* Y, int M, const FusedLaunchPlan& pl,
                          long long wait_limit, cudaStream_t stream);
 int smem_optin_of(int device);
+// Diagnostic: per-CTA wall-clock phase marks of the last fused launch.
+cudaError_t fused_phase_times(unsigned long long* out, int max_ctas, int* n_ctas);
 
 // 2-D tensor map over a row-major array (rows x inner elements, row stride in bytes).
 cudaError_t encode_tiled_2d(CUtensorMap* map, CUtensorMapDataType type, const void* base, uint64_t inner,

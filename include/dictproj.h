@@ -399,6 +399,16 @@ int dictproj_layer_load(const char* path, dictproj_layer** out);
  * synchronising `stream`. Returns OK or TIMEOUT (or CUDA). */
 int dictproj_check(void* stream);
 
+/* Diagnostic (no counterpart in the paper): wall-clock marks (ns, the GPU's
+ * global timer) at the phase boundaries of the most recent fused decode launch,
+ * per CTA: out[cta * 16 + slot] for cta < min(max_ctas, 1024); *n_ctas = rows
+ * written. Slots 0-7 (compute warps): start, dependency resolved, X staged,
+ * dictionary stage done, partial Z published, exchange passed, Z tables loaded,
+ * end; 8-11 (producer): first slots issued, dependents released, dependency
+ * resolved, last copy issued; 12-15 unused. Synchronise the stream first.
+ * Errors: NULL, RANGE, UNSUPPORTED, CUDA. */
+int dictproj_diag_phase_times(unsigned long long* out, int max_ctas, int* n_ctas);
+
 /* Self-test of the bounded-wait error path (diagnostic; no counterpart in the
  * paper). Launches one warp on `stream` that waits on an mbarrier which can never
  * complete, with a limit of `cycles` SM clocks (1 <= cycles <= 2^31). The wait
