@@ -174,7 +174,8 @@ void dictproj_free_group(dictproj_group* g) {
   cudaFree(g->z16);
   cudaFree(g->cdense);
   cudaFree(g->err);
-  cudaFree(g->scales_pad);
+  cudaFree(g->fcodes);
+  cudaFree(g->fscales);
   cudaFree(g->zx);
   cudaFree(g->fsync);
   delete g;
@@ -238,7 +239,7 @@ int dictproj_group_upload(const uint8_t* codes, const uint8_t* scales, float s_D
     return cuda_fail(e, "group_upload: tensor map of the dictionary codes");
   }
   bool fused = false;
-  if (fault("alloc") || (e = fused_group_setup(g, &fused)) != cudaSuccess) {
+  if (fault("alloc") || (e = fused_group_setup(g, codes, scales, &fused)) != cudaSuccess) {
     dictproj_free_group(g);
     cudaGetLastError();
     return fail(DICTPROJ_ERR_OOM, "group_upload: fused decode buffers (%s)", cudaGetErrorName(e));

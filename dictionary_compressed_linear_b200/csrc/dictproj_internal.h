@@ -65,14 +65,13 @@ struct dictproj_group {
   CUtensorMap codes_map;   // TMA map of codes: [k] rows x [d_in/2] bytes, box 32 x 256
   // fused decode kernel
   bool fused_ok;           // the fused kernel serves this group
-  CUtensorMap fmap_codes;  // codes: box 16 atoms x 128 bytes, 128-byte swizzle
-  CUtensorMap fmap_scales; // scales (row stride padded to 16 bytes): box 16 atoms x 32 bytes
-  uint8_t* scales_pad;     // padded copy of the scales when d_in/16 is not a multiple of 16
-  float* zx;               // partial-Z exchange buffer [zslots][k][mp]
+  uint8_t* fcodes;         // tile-major copy of the codes: [16-atom tile][512-element piece][16 rows][256 B]
+  uint8_t* fscales;        // tile-major copy of the scales: [tile][piece][16 rows][32 B]
+  unsigned long long* zx;  // partial-Z exchange buffer [zslots][k][mp] of (tag << 32 | fp32 bits)
   int zslots;              // CTAs one 16-atom tile is split over, at most
   int ppr;                 // 512-element pieces per atom row
   int tp_bound;            // tiles one CTA's pieces span, at most
-  unsigned long long* fsync;  // [0] ticket, bytes 16.. flags[n_sm]
+  unsigned long long* fsync;  // [0] launch ticket of the exchange buffer (one per CTA per launch)
 };
 
 struct dictproj_layer {

@@ -1,35 +1,38 @@
 // Decode path (M <= 8 tokens), fused: both stages of Eq. (1) of the DictLLM
 // technical review, Z = X D_g and Y = Z C_l, in ONE kernel per call
 // (k_decode_fused), with every packed weight byte staged through shared memory
-// by the Tensor Memory Accelerator.
+// by bulk asynchronous copies.
 //
 // Why one kernel. At decode a projection moves 9-25 MB of packed weights, which
 // HBM delivers in 1.3-3.7 us; two dependent kernels per call with a global Z
 // round trip cost more than that in fixed latency. Here:
 //   * one CTA per SM (grid = SM count); a producer warp streams the CTA's share
 //     of the packed D_g and C_l into a ring of 16 KB shared-memory slots with
-//     bulk / tensor TMA copies. Weights are never written after upload, so the
-//     producer starts streaming at once, before the kernel waits for the
-//     previous work on the stream (programmatic dependent launch): the ring of
-//     the next call fills while this call computes. A CTA uses at most half of
-//     an SM (M <= 4), so two consecutive calls are resident together.
-//   * stage 1: twelve compute warps take 16-atom x 512-element pieces of D_g
-//     from the ring, decode E2M1 x E4M3 to fp16 (exact) and run swap-AB
-//     mma.sync m16n8k16 (atoms = the 16 rows, tokens = the 8 columns) with fp32
-//     accumulation. Pieces are dealt to CTAs evenly: each CTA gets a contiguous
-//     run of a projection's pieces, so a 16-atom tile is split over at most a
-//     few CTAs, whose partial sums (times s_D) go to a per-group exchange buffer
-//     Zx[slot][k][mp] in L2.
-//   * one grid-wide exchange: each CTA adds one to a 64-bit arrival count when
-//     its partial Z is written and waits until the count reaches this launch's
-//     target (from a 64-bit ticket every CTA takes at start; every CTA adds
-//     exactly one per launch, aborted or not, so later launches stay aligned);
-//     then every CTA sums the slots of each tile in a fixed order into its
-//     shared-memory Z table (bit-exact, independent of timing).
-//   * stage 2: the compute warps take the CTA's column chunks of C_l (columns
-//     split over CTAs by bytes, so by nnz) from the ring; one warp per column,
-//     lanes over 8-entry half-blocks, the same per-window segment logic as the
-//     gather kernel, fp32 sums, fp16 Y.
+//     cp.async.bulk. Weights are never written after upload, so the producer
+//     starts streaming at once, before the kernel waits for the previous work on
+//     the stream (programmatic dependent launch): the ring of the next call
+//     fills while this call computes. A CTA uses at most half of an SM (M <= 4),
+//     so two consecutive calls are resident together.
+//   * D_g is also kept in a tile-major copy made at upload: 16 atoms x 512
+//     elements ("pieces") of codes (4 KB, 16-byte chunks of each row swizzled by
+//     the row number, so that the MMA operand reads are conflict-free) and of
+//     scales (512 B) are contiguous, and a CTA's share of a projection (a run of
+//     consecutive pieces) is one contiguous range: one copy per slot.
+//   * stage 1: twelve compute warps take 128-element quarters of the pieces,
+//     decode E2M1 x E4M3 to fp16 (exact) and run swap-AB mma.sync m16n8k16 (atoms
+//     = the 16 rows, tokens = the 8 columns) with fp32 accumulation. Pieces are
+//     dealt to CTAs evenly, so a 16-atom tile is split over at most a few CTAs;
+//     each writes its partial sums (times s_D) to the group's exchange buffer
+//     Zx[slot][k][mp], every value in one 64-bit store together with this
+//     launch's tag for the buffer (from a 64-bit ticket every CTA takes per group
+//     at start).
+//   * the exchange is the read: each CTA loads every slot of every tile for its
+//     Z table and retries a value until it carries this launch's tag; slots are
+//     summed in a fixed order, so Z is bit-exact and independent of timing.
+//   * stage 2: each half of a compute warp takes one column of the CTA's column
+//     chunks of C_l (columns split over CTAs by bytes, so by nnz); its 16 lanes
+//     take 8-entry half-blocks, the segment of each entry comes from per-window
+//     ballots over seg_start, fp32 sums, fp16 Y.
 // Every wait is bounded (a second by default); a wait that gives up sets the
 // device error word and the CTA unwinds (the producer first waits, bounded,
 // for its copies in flight).
@@ -39,6 +42,7 @@
 
 #include <algorithm>
 #include <climits>
+#include <cstring>
 #include <vector>
 
 #include "common.cuh"
@@ -50,26 +54,56 @@ namespace dictproj {
 // ---------------------------------------------------------------------------------
 // geometry
 // ---------------------------------------------------------------------------------
-constexpr int kFWarps = 12;                      // compute warps (one D quarter each per full slot)
+constexpr int kFWarps = 12;                      // compute warps
 constexpr int kFThreads = 32 * (kFWarps + 1);    // + one producer warp
 constexpr int kPieceElems = 512;                 // d_in elements of one D piece (per atom)
-constexpr int kPieceCodeBytes = 16 * 256;        // 16 atoms x 256 code bytes (two 128-B boxes)
+constexpr int kPieceCodeBytes = 16 * 256;        // 16 atoms x 256 code bytes
 constexpr int kPieceScaleBytes = 16 * 32;        // 16 atoms x 32 scale bytes
 constexpr int kPiecesPerSlot = 3;
 constexpr int kSlotScaleOff = kPiecesPerSlot * kPieceCodeBytes;  // 12 KB
-constexpr int kTasksPerSlot = 4 * kPiecesPerSlot;                // 128-element quarters
 constexpr int kMaxCChunks = 64;                  // coefficient chunks one CTA may own in one launch
+constexpr int kMaxDChunks = 64;                  // dictionary slots one CTA may own in one launch
 constexpr int kFusedMaxBatch = 4;
 
 static_assert(kSlotScaleOff + kPiecesPerSlot * kPieceScaleBytes <= kFusedSlotBytes, "D pieces fit a slot");
+
+// Tile-major copy of a packed dictionary (host side, at upload). Piece x =
+// (tile a, piece pc of the atom row) holds rows r = 0..15 (atom 16a + r),
+// elements [512 pc, 512 pc + 512): codes at x*4096 + r*256, the 16-byte chunk c of
+// the row stored at position (c & 8) | ((c & 7) ^ (r & 7)); scales at x*512 + r*32.
+// Elements at or beyond d_in are zero.
+void fused_pack_dictionary(const uint8_t* codes, const uint8_t* scales, int d_in, int k, uint8_t* fcodes,
+                           uint8_t* fscales) {
+  const int ppr = (d_in + kPieceElems - 1) / kPieceElems;
+  const size_t crow = (size_t)d_in / 2, srow = (size_t)d_in / 16;
+  for (int a = 0; a < k / 16; ++a)
+    for (int pc = 0; pc < ppr; ++pc) {
+      const size_t x = (size_t)a * ppr + pc;
+      for (int r = 0; r < 16; ++r) {
+        const size_t atom = (size_t)16 * a + r;
+        for (int c = 0; c < 16; ++c) {
+          const int pos = (c & 8) | ((c & 7) ^ (r & 7));
+          uint8_t* dst = fcodes + x * kPieceCodeBytes + r * 256 + pos * 16;
+          for (int i = 0; i < 16; ++i) {
+            const size_t byte = (size_t)pc * 256 + c * 16 + i;
+            dst[i] = byte < crow ? codes[atom * crow + byte] : 0;
+          }
+        }
+        for (int i = 0; i < 32; ++i) {
+          const size_t byte = (size_t)pc * 32 + i;
+          fscales[x * kPieceScaleBytes + r * 32 + i] = byte < srow ? scales[atom * srow + byte] : 0;
+        }
+      }
+    }
+}
 
 // Byte layout of one coefficient chunk (columns [o_a, o_b), entries [E_a, E_b))
 // in a ring slot: five 16-byte aligned runs copied from the packed arrays, each
 // rounded outward to 16 bytes (the arrays carry 16 bytes of slack at the end).
 struct CChunk {
   uint32_t idx_src, idx_bytes;    // idx[E_a, E_b)
-  uint32_t code_src, code_bytes;  // codes[E_a/2, E_b/2)
-  uint32_t sc_src, sc_bytes;      // scales[E_a/16, E_b/16)
+  uint32_t code_src, code_bytes;  // values: codes[E_a*v/2, E_b*v/2) for v nibbles per value
+  uint32_t sc_src, sc_bytes;      // scales[E_a/16, E_b/16) (NVFP4 only)
   uint32_t ss_src, ss_bytes;      // seg_start rows o_a .. o_b-1 (bytes)
   uint32_t cp_src, cp_bytes;      // col_ptr[o_a .. o_b] (bytes)
   uint32_t code_dst, sc_dst, ss_dst, cp_dst, total;
@@ -114,11 +148,12 @@ __host__ __device__ inline int split_pos(int x, int q, int r) {
 // launch parameters
 // ---------------------------------------------------------------------------------
 struct FusedProj {
-  CUtensorMap dcodes;    // D codes: [k] rows x [d_in/2] bytes, box 16 x 128, 128-B swizzle
-  CUtensorMap dscales;   // D scales: [k] rows x [d_in/16] bytes (row stride padded to 16), box 16 x 32
+  const uint8_t* fcodes;      // tile-major dictionary codes [P][4096]
+  const uint8_t* fscales;     // tile-major dictionary scales [P][512]
   const __half* X;
   __half* Y;
-  float* zx;             // [zslots][k][MP] partial Z of the tiles' pieces
+  unsigned long long* zx;     // [zslots][k][MP]: (tag << 32) | fp32 bits of a tile piece's partial Z
+  unsigned long long* ticket; // this group's launch ticket (one per CTA per launch)
   const uint32_t* col_ptr;
   const uint8_t* ccodes;
   const uint8_t* cscales;
@@ -129,16 +164,15 @@ struct FusedProj {
   float s_D, s_C;
   int d_in, k, d_out, nseg;
   int ppr, P, pq, pr, rot;    // pieces per atom row, pieces, P = pq*G + pr, position rotation
-  int xoff;                   // byte offset of its staged X rows in shared memory, -1: read X from global
   int cfmt;                   // coefficient value format (DICTPROJ_CFMT_*)
+  int xoff;                   // byte offset of its staged X rows in shared memory, -1: read X from global
   int xfirst;                 // 1: this projection stages X at xoff (later ones with the same X reuse it)
   int zt_off;                 // byte offset of its Z table in shared memory
+  int zslots;                 // slots of the exchange buffer
 };
 
 struct FusedParams {
   FusedProj p[kFusedMaxBatch];
-  unsigned long long* ticket;  // launches of this sync object x G CTAs so far (one ticket per CTA)
-  unsigned long long* arrive;  // CTAs that published their partial Z, over all launches (one per CTA)
   long long wait_limit;        // SM clocks a bounded wait may take
   int n, M, G, R;              // projections, tokens, CTAs, ring slots
   int xrow;                    // bytes per staged X row
@@ -148,15 +182,13 @@ struct FusedParams {
   int bar_off;                 // offset of the barriers and chunk descriptors
 };
 
+}  // namespace dictproj
+
+namespace dictproj {
+
 // ---------------------------------------------------------------------------------
 // device helpers
 // ---------------------------------------------------------------------------------
-__device__ __forceinline__ void tma2d(uint32_t dst, const CUtensorMap* map, int x, int y, uint64_t* bar) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];"
-      ::"r"(dst), "l"(map), "r"(x), "r"(y), "r"(smem_u32(bar))
-      : "memory");
-}
 __device__ __forceinline__ void bulk_g2s_u32(uint32_t dst, const void* src, uint32_t bytes, uint64_t* bar) {
   asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
                ::"r"(dst), "l"(src), "r"(bytes), "r"(smem_u32(bar))
@@ -173,39 +205,19 @@ __device__ __forceinline__ uint4 ld_cg_v4(const void* p) {
   asm volatile("ld.global.cg.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w) : "l"(p));
   return r;
 }
-__device__ __forceinline__ float4 ld_cg_f4(const float* p) {
-  float4 r;
-  asm volatile("ld.global.cg.v4.f32 {%0,%1,%2,%3}, [%4];" : "=f"(r.x), "=f"(r.y), "=f"(r.z), "=f"(r.w) : "l"(p));
-  return r;
-}
-__device__ __forceinline__ void fence_acq_rel_gpu() { asm volatile("fence.acq_rel.gpu;" ::: "memory"); }
-__device__ __forceinline__ void atom_add_release_u64(unsigned long long* p, unsigned long long v) {
-  asm volatile("red.release.gpu.global.add.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
-}
-__device__ __forceinline__ unsigned long long ld_acquire_u64(const unsigned long long* p) {
+__device__ __forceinline__ unsigned long long ld_relaxed_u64(const unsigned long long* p) {
   unsigned long long v;
-  asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+  asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
   return v;
 }
-
-// Diagnostic: wall-clock (ns) at the phase boundaries of the last fused launch,
-// per CTA (slots 0-7 compute side, 8-11 producer side); read by
-// dictproj_diag_phase_times. A few stores per CTA and launch.
-constexpr int kPhaseCtas = 1024, kPhaseSlots = 16;
-static __device__ unsigned long long g_phase[kPhaseCtas * kPhaseSlots];
-__device__ __forceinline__ void phase_mark(int cta, int slot) {
-  unsigned long long t;
-  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-  if (cta < kPhaseCtas) g_phase[cta * kPhaseSlots + slot] = t;
+__device__ __forceinline__ void st_relaxed_u64(unsigned long long* p, unsigned long long v) {
+  asm volatile("st.relaxed.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
 }
 __device__ __forceinline__ void sts_u32x4(uint32_t a, uint4 v) {
   asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};" ::"r"(a), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w) : "memory");
 }
 __device__ __forceinline__ void sts_f32(uint32_t a, float v) {
   asm volatile("st.shared.f32 [%0], %1;" ::"r"(a), "f"(v) : "memory");
-}
-__device__ __forceinline__ void sts_f32x4(uint32_t a, float4 v) {
-  asm volatile("st.shared.v4.f32 [%0], {%1,%2,%3,%4};" ::"r"(a), "f"(v.x), "f"(v.y), "f"(v.z), "f"(v.w) : "memory");
 }
 
 // Bounded wait on an mbarrier phase that also gives up when another warp of the
@@ -225,23 +237,30 @@ __device__ __forceinline__ bool mbar_wait_or_abort(uint64_t* bar, uint32_t phase
   return true;
 }
 
-}  // namespace dictproj
-
-namespace dictproj {
+// Diagnostic: wall-clock (ns) at the phase boundaries of the last fused launch,
+// per CTA (slots 0-7 compute side, 8-11 producer side); read by
+// dictproj_diag_phase_times. A few stores per CTA and launch.
+constexpr int kPhaseCtas = 1024, kPhaseSlots = 16;
+static __device__ unsigned long long g_phase[kPhaseCtas * kPhaseSlots];
+__device__ __forceinline__ void phase_mark(int cta, int slot) {
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  if (cta < kPhaseCtas) g_phase[cta * kPhaseSlots + slot] = t;
+}
 
 // ---------------------------------------------------------------------------------
 // stage 1: one 16-atom x 128-element quarter of a D piece
 // ---------------------------------------------------------------------------------
-// Thread (g, tq) of the warp takes the 16-byte chunk c16 = 2*tq + h of the atom
-// rows g and g+8 of the quarter's 128-byte box (rows are 128-byte swizzled: chunk
-// c of row r sits at position c ^ (r & 7)), i.e. 32 elements per atom, and the
-// same 32 elements of X for token g. mma.sync m16n8k16 with the atoms as the 16
-// rows of A and the tokens as the 8 columns of B: within each thread the same
-// element order is used for A and B, so the sum over k is unchanged.
+// Thread (g, tq) of the warp takes the 16-byte chunk c16 = 2*tq + h of box b of
+// the atom rows g and g+8 (rows of 256 bytes; chunk c of row r stored at
+// (c & 8) | ((c & 7) ^ (r & 7))), i.e. 32 elements per atom, and the same 32
+// elements of X for token g. mma.sync m16n8k16 with the atoms as the 16 rows of A
+// and the tokens as the 8 columns of B: within each thread the same element
+// order is used for A and B, so the sum over k is unchanged.
 __device__ __forceinline__ void piece_quarter(float acc[2][4], uint32_t box, uint32_t scl, int g, int c16,
                                               const uint32_t xw[4][4]) {
-  const uint32_t ra = box + g * 128 + ((uint32_t)(c16 ^ g) << 4);
-  const uint4 wa4 = lds_u32x4(ra), wb4 = lds_u32x4(ra + 1024);
+  const uint32_t ra = box + g * 256 + ((uint32_t)(c16 ^ g) << 4);
+  const uint4 wa4 = lds_u32x4(ra), wb4 = lds_u32x4(ra + 2048);
   const uint32_t ha = e4m3x2_to_f16x2(lds_u16(scl + g * 32 + 2 * c16));
   const uint32_t hb = e4m3x2_to_f16x2(lds_u16(scl + (g + 8) * 32 + 2 * c16));
   const uint32_t wa[4] = {wa4.x, wa4.y, wa4.z, wa4.w};
@@ -268,13 +287,8 @@ __device__ __forceinline__ void piece_quarter(float acc[2][4], uint32_t box, uin
 }
 
 // ---------------------------------------------------------------------------------
-// stage 2: one column from a shared-memory chunk
+// stage 2: coefficient values and one column from a shared-memory chunk
 // ---------------------------------------------------------------------------------
-// idx_a / code_a / sc_a / ss_a: shared addresses of the column's first index
-// byte, first code byte, first scale byte and its seg_start row; nhb 8-entry
-// half-blocks. Lane l takes half-blocks 32 i + l; the segment of each entry
-// comes from per-window ballots over seg_start (one boundary per lane), several
-// boundaries inside one half-block fall back to a walk.
 // Eight stored values of half-block hb as four f16x2 (their fp16 forms are
 // exact: E2M1, E4M3 and small integers are fp16 numbers), for each format.
 template <int FMT>
@@ -307,85 +321,108 @@ __device__ __forceinline__ void half_block_values(uint32_t code_a, int hb, uint3
   }
 }
 
+// Sum over the 8 entries q0 .. q0+7 of a half-block: at most one segment
+// boundary inside (t: first entry in segment sgi+1) unless `walk`, in which case
+// the entries advance through seg_start one by one. Unscaled (block scale and
+// s_C are applied by the caller).
 template <int MP, int FMT>
-__device__ __forceinline__ void column_sum(float acc[MP], uint32_t idx_a, uint32_t code_a, uint32_t sc_a,
-                                           uint32_t ss_a, int nhb, int nseg, uint32_t zs_a, int lane) {
+__device__ __forceinline__ void half_block_sum(float out[MP], uint32_t idx_a, uint32_t code_a, uint32_t ss_a,
+                                               int hb, int q0, int sgi, int t1, bool walk, int nseg, uint32_t zs_a) {
   constexpr uint32_t kRow = MP * 4;
+  const uint2 iv = lds_u32x2(idx_a + 8 * hb);
+  const uint32_t iw[2] = {iv.x, iv.y};
+  uint32_t f[4];
+  half_block_values<FMT>(code_a, hb, f);
+  float a0[MP], a1[MP];
+#pragma unroll
+  for (int m = 0; m < MP; ++m) a0[m] = a1[m] = 0.f;
+  if (!walk) {
+    const int t = min(t1 - q0, 8);
+    const uint32_t z0 = zs_a + ((uint32_t)sgi << 8) * kRow;
+    const uint32_t z1 = z0 + 256u * kRow;
+#pragma unroll
+    for (int p = 0; p < 4; ++p) {
+      const float2 v = __half22float2(*reinterpret_cast<const __half2*>(&f[p]));
+      const int e0 = 2 * p, e1 = e0 + 1;
+      const uint32_t b0 = __byte_perm(iw[e0 >> 2], 0u, 0x4440u | (uint32_t)(e0 & 3));
+      const uint32_t b1 = __byte_perm(iw[e1 >> 2], 0u, 0x4440u | (uint32_t)(e1 & 3));
+      fma_z<MP>(a0, (e0 >= t ? z1 : z0) + b0 * kRow, v.x);
+      fma_z<MP>(a1, (e1 >= t ? z1 : z0) + b1 * kRow, v.y);
+    }
+  } else {
+    int sg = 0;
+    for (int j = 1; j < nseg; ++j) sg += ((int)lds_u16(ss_a + 2 * j) <= q0);
+    int nb = (sg + 1 < nseg) ? (int)lds_u16(ss_a + 2 * (sg + 1)) : INT_MAX;
+#pragma unroll
+    for (int p = 0; p < 4; ++p) {
+      const float2 v = __half22float2(*reinterpret_cast<const __half2*>(&f[p]));
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) {
+        const int ent = 2 * p + hh;
+        while (q0 + ent >= nb) {
+          ++sg;
+          nb = (sg + 1 < nseg) ? (int)lds_u16(ss_a + 2 * (sg + 1)) : INT_MAX;
+        }
+        const uint32_t bb = __byte_perm(iw[ent >> 2], 0u, 0x4440u | (uint32_t)(ent & 3));
+        fma_z<MP>(hh ? a1 : a0, zs_a + (((uint32_t)sg << 8) + bb) * kRow, hh ? v.y : v.x);
+      }
+    }
+  }
+#pragma unroll
+  for (int m = 0; m < MP; ++m) out[m] = a0[m] + a1[m];
+}
+
+// One column by G lanes (G = 32: a warp; G = 16: half a warp, `half` 0 / 1) in
+// windows of 8*G entries: lane l of the group takes half-block G*i + l. The
+// segment of each half-block's first entry, and the first entry of the next
+// segment inside it, come from ballots over seg_start (lane l holds
+// seg_start[l], so nseg <= G); two boundaries inside one half-block make the
+// whole window walk. Returns the column sum (unscaled by s_C) in every lane.
+template <int MP, int FMT, int G>
+__device__ __forceinline__ void column_sum(float acc[MP], uint32_t idx_a, uint32_t code_a, uint32_t sc_a,
+                                           uint32_t ss_a, int nhb, int nseg, uint32_t zs_a, int lane, int half) {
+  const unsigned gmask = G == 32 ? 0xffffffffu : (0xffffu << (16 * half));
+  const int gl = G == 32 ? lane : lane & 15;
+  const unsigned gsh = G == 32 ? 0u : 16u * half;
+  const unsigned lowbits = G == 32 ? 0xffffffffu : 0xffffu;
 #pragma unroll
   for (int m = 0; m < MP; ++m) acc[m] = 0.f;
-  const bool is_bnd = lane >= 1 && lane < nseg;
-  const int b = lane < nseg ? (int)lds_u16(ss_a + 2 * lane) : 0;
-  for (int i = 0; 256 * i < 8 * nhb; ++i) {
-    const int w = 256 * i;
-    const int s_lo = __popc(__ballot_sync(0xffffffffu, is_bnd && b <= w));
-    const bool in_win = is_bnd && b > w && b < w + 256;
+  const bool is_bnd = gl >= 1 && gl < nseg;
+  const int b = gl < nseg ? (int)lds_u16(ss_a + 2 * gl) : 0;
+  for (int i = 0; 8 * G * i < 8 * nhb; ++i) {
+    const int w = 8 * G * i;
+    const int s_lo = __popc((__ballot_sync(gmask, is_bnd && b <= w) >> gsh) & lowbits);
+    const bool in_win = is_bnd && b > w && b < w + 8 * G;
     const int rel = b - w;
     const uint32_t at_start = (in_win && (rel & 7) == 0) ? (1u << (rel >> 3)) : 0u;
     const uint32_t inside = (in_win && (rel & 7) != 0) ? (1u << (rel >> 3)) : 0u;
-    const uint32_t A = __reduce_or_sync(0xffffffffu, at_start);
-    const uint32_t B = __reduce_or_sync(0xffffffffu, inside);
-    const int nwin = __popc(__ballot_sync(0xffffffffu, in_win));
+    const uint32_t A = __reduce_or_sync(gmask, at_start);
+    const uint32_t B = __reduce_or_sync(gmask, inside);
+    const int nwin = __popc((__ballot_sync(gmask, in_win) >> gsh) & lowbits);
     const bool collide = nwin != __popc(A) + __popc(B) || (A & B) != 0u;
-    const uint32_t le = lane == 31 ? 0xffffffffu : ((2u << lane) - 1u);
+    const uint32_t le = gl == 31 ? 0xffffffffu : ((2u << gl) - 1u);
     const int sgi = s_lo + __popc(A & le) + __popc(B & (le >> 1));  // segment of the lane's first entry
-    const int q0 = w + 8 * lane;
-    const int bn = __shfl_sync(0xffffffffu, b, min(sgi + 1, 31));
-    const int t1 = ((B >> lane) & 1u) ? bn : INT_MAX;
-    const int hb = 32 * i + lane;
+    const int q0 = w + 8 * gl;
+    const int bn = __shfl_sync(gmask, b, min(sgi + 1, G - 1), G);
+    const int t1 = ((B >> gl) & 1u) ? bn : INT_MAX;
+    const int hb = G * i + gl;
     if (hb < nhb) {
-      const uint2 iv = lds_u32x2(idx_a + 8 * hb);
-      const uint32_t iw[2] = {iv.x, iv.y};
-      uint32_t f[4];
-      half_block_values<FMT>(code_a, hb, f);
-      float a0[MP], a1[MP];
-#pragma unroll
-      for (int m = 0; m < MP; ++m) a0[m] = a1[m] = 0.f;
-      if (!collide) {  // at most one boundary: entries e >= t use segment sgi+1
-        const int t = min(t1 - q0, 8);
-        const uint32_t z0 = zs_a + ((uint32_t)sgi << 8) * kRow;
-        const uint32_t z1 = z0 + 256u * kRow;
-#pragma unroll
-        for (int p = 0; p < 4; ++p) {
-          const float2 v = __half22float2(*reinterpret_cast<const __half2*>(&f[p]));
-          const int e0 = 2 * p, e1 = e0 + 1;
-          const uint32_t b0 = __byte_perm(iw[e0 >> 2], 0u, 0x4440u | (uint32_t)(e0 & 3));
-          const uint32_t b1 = __byte_perm(iw[e1 >> 2], 0u, 0x4440u | (uint32_t)(e1 & 3));
-          fma_z<MP>(a0, (e0 >= t ? z1 : z0) + b0 * kRow, v.x);
-          fma_z<MP>(a1, (e1 >= t ? z1 : z0) + b1 * kRow, v.y);
-        }
-      } else {  // walk the boundaries one entry at a time
-        int sg = 0;
-        for (int j = 1; j < nseg; ++j) sg += ((int)lds_u16(ss_a + 2 * j) <= q0);
-        int nb = (sg + 1 < nseg) ? (int)lds_u16(ss_a + 2 * (sg + 1)) : INT_MAX;
-#pragma unroll
-        for (int p = 0; p < 4; ++p) {
-          const float2 v = __half22float2(*reinterpret_cast<const __half2*>(&f[p]));
-#pragma unroll
-          for (int hh = 0; hh < 2; ++hh) {
-            const int ent = 2 * p + hh;
-            while (q0 + ent >= nb) {
-              ++sg;
-              nb = (sg + 1 < nseg) ? (int)lds_u16(ss_a + 2 * (sg + 1)) : INT_MAX;
-            }
-            const uint32_t bb = __byte_perm(iw[ent >> 2], 0u, 0x4440u | (uint32_t)(ent & 3));
-            fma_z<MP>(hh ? a1 : a0, zs_a + (((uint32_t)sg << 8) + bb) * kRow, hh ? v.y : v.x);
-          }
-        }
-      }
+      float s8[MP];
+      half_block_sum<MP, FMT>(s8, idx_a, code_a, ss_a, hb, q0, sgi, t1, collide, nseg, zs_a);
       if constexpr (FMT == 0) {
         const float sc = e4m3_to_f32(lds_u8(sc_a + (hb >> 1)));
 #pragma unroll
-        for (int m = 0; m < MP; ++m) acc[m] = fmaf(a0[m] + a1[m], sc, acc[m]);
+        for (int m = 0; m < MP; ++m) acc[m] = fmaf(s8[m], sc, acc[m]);
       } else {
 #pragma unroll
-        for (int m = 0; m < MP; ++m) acc[m] += a0[m] + a1[m];
+        for (int m = 0; m < MP; ++m) acc[m] += s8[m];
       }
     }
   }
 #pragma unroll
   for (int m = 0; m < MP; ++m) {
 #pragma unroll
-    for (int off = 16; off > 0; off >>= 1) acc[m] += __shfl_xor_sync(0xffffffffu, acc[m], off);
+    for (int off = G / 2; off > 0; off >>= 1) acc[m] += __shfl_xor_sync(gmask, acc[m], off, G);
   }
 }
 
@@ -395,47 +432,92 @@ namespace dictproj {
 
 // Shared-memory control block (at FusedParams::bar_off, 16-byte aligned):
 //   uint4   desc[kMaxCChunks]      coefficient chunks {o_a, o_b, E_a, E_b} of this CTA
+//   uint32  dtab[kMaxDChunks]      dictionary slots: first piece | pieces << 28 | projection << 30
 //   u64     full[R], empty[R], rdy mbarriers (ring slot filled / drained; control block ready)
-//   int     misc[8]                abort, flag value, coefficient chunks, D pieces, tile pieces
+//   int     misc[16]               abort, coefficient chunks, D pieces, tile pieces, D slots,
+//                                  exchange tags of the projections (8..11)
 //   int     loc[4][8]              per projection: x0, x1, first local piece, first tile piece,
 //                                  first tile, tiles, position
 //   uint8   desc_p[kMaxCChunks]    projection of each coefficient chunk
-constexpr int kCtlMisc = 8, kCtlLoc = 8;
-inline int fused_ctl_bytes(int R) { return 16 * kMaxCChunks + 16 * R + 8 + 4 * kCtlMisc + 4 * kCtlLoc * kFusedMaxBatch + kMaxCChunks; }
+constexpr int kCtlMisc = 16, kCtlLoc = 8;
+inline int fused_ctl_bytes(int R) {
+  return 16 * kMaxCChunks + 4 * kMaxDChunks + 16 * R + 8 + 4 * kCtlMisc + 4 * kCtlLoc * kFusedMaxBatch + kMaxCChunks;
+}
 
-template <int MP>
-__device__ __forceinline__ void load_ztable(const FusedProj& pp, uint32_t sbase, int tid) {
-  const uint32_t zt = sbase + pp.zt_off;
-  const int nv = pp.k * MP / 4;
-  for (int v = tid; v < nv; v += kFWarps * 32) {
-    const int e = 4 * v, a = (e / MP) >> 4;
-    const int pos0 = split_pos(a * pp.ppr, pp.pq, pp.pr);
-    const int pos1 = split_pos(a * pp.ppr + pp.ppr - 1, pp.pq, pp.pr);
-    float4 s = ld_cg_f4(pp.zx + e);
-    for (int sl = 1; sl <= pos1 - pos0; ++sl) {  // fixed order over the tile's pieces
-      const float4 b = ld_cg_f4(pp.zx + (size_t)sl * pp.k * MP + e);
-      s.x += b.x;
-      s.y += b.y;
-      s.z += b.z;
-      s.w += b.w;
-    }
-    sts_f32x4(zt + 4 * e, s);
+// Tagged read of one exchange value: retry until it carries `tag` (bounded).
+__device__ __forceinline__ float ll_value(const unsigned long long* p, unsigned long long x, uint32_t tag,
+                                          volatile int* abort, long long limit) {
+  if ((uint32_t)(x >> 32) != tag) {
+    const long long t0 = clock64();
+    do {
+      if (*abort) return 0.f;
+      if (clock64() - t0 > limit) {
+        atomicOr(&g_dictproj_error, 1u);
+        *abort = 1;
+        return 0.f;
+      }
+      __nanosleep(64);
+      x = ld_relaxed_u64(p);
+    } while ((uint32_t)(x >> 32) != tag);
   }
-  const int tail = (pp.k + 256) * MP / 4;  // zero rows after the last atom (padding entries read them)
-  for (int v = nv + tid; v < tail; v += kFWarps * 32) sts_f32x4(zt + 16 * v, make_float4(0.f, 0.f, 0.f, 0.f));
+  return __uint_as_float((uint32_t)(x & 0xffffffffull));
+}
+
+// Z table of a projection in shared memory: Z[atom][m] = sum, in slot order, of the
+// tile's partial sums in the exchange buffer (each read waits for this launch's
+// tag), then a zero tail of 256 atom rows (padding entries read it).
+template <int MP>
+__device__ __forceinline__ void load_ztable(const FusedProj& pp, uint32_t sbase, int tid, uint32_t tag,
+                                            volatile int* abort, long long limit) {
+  constexpr int NT = kFWarps * 32, B = 4, S = 4;
+  const uint32_t zt = sbase + pp.zt_off;
+  const int ne = pp.k * MP;
+  const size_t stride = (size_t)pp.k * MP;
+  for (int base = tid; base < ne; base += B * NT) {
+    unsigned long long v[B][S];
+    int ns[B];
+#pragma unroll
+    for (int i = 0; i < B; ++i) {  // issue every load of the batch before using any
+      const int e = base + i * NT;
+      ns[i] = 0;
+      if (e < ne) {
+        const int a = (e / MP) >> 4;
+        ns[i] = split_pos(a * pp.ppr + pp.ppr - 1, pp.pq, pp.pr) - split_pos(a * pp.ppr, pp.pq, pp.pr) + 1;
+      }
+#pragma unroll
+      for (int s = 0; s < S; ++s) v[i][s] = s < ns[i] ? ld_relaxed_u64(pp.zx + s * stride + e) : 0ull;
+    }
+#pragma unroll
+    for (int i = 0; i < B; ++i) {
+      const int e = base + i * NT;
+      if (e >= ne) continue;
+      float sum = 0.f;
+#pragma unroll
+      for (int s = 0; s < S; ++s)
+        if (s < ns[i]) sum += ll_value(pp.zx + s * stride + e, v[i][s], tag, abort, limit);
+      for (int s = S; s < ns[i]; ++s) {
+        const unsigned long long* p = pp.zx + s * stride + e;
+        sum += ll_value(p, ld_relaxed_u64(p), tag, abort, limit);
+      }
+      sts_f32(zt + 4 * e, sum);
+    }
+  }
+  const int tail = (pp.k + 256) * MP;
+  for (int v = ne + tid; v < tail; v += NT) sts_f32(zt + 4 * v, 0.f);
 }
 
 template <int MP>
 __global__ void __launch_bounds__(kFThreads, 2) k_decode_fused(const __grid_constant__ FusedParams prm) {
   extern __shared__ uint8_t fsm_raw[];
   const uint32_t raw = smem_u32(fsm_raw);
-  const uint32_t sbase = (raw + 1023u) & ~1023u;  // 128-byte swizzled TMA boxes need 1024-byte alignment
+  const uint32_t sbase = (raw + 1023u) & ~1023u;
   uint8_t* sg = fsm_raw + (sbase - raw);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int G = prm.G, R = prm.R, n = prm.n, M = prm.M, cta = blockIdx.x;
   const long long limit = prm.wait_limit;
   uint4* desc = reinterpret_cast<uint4*>(sg + prm.bar_off);
-  uint64_t* full = reinterpret_cast<uint64_t*>(desc + kMaxCChunks);
+  uint32_t* dtab = reinterpret_cast<uint32_t*>(desc + kMaxCChunks);
+  uint64_t* full = reinterpret_cast<uint64_t*>(dtab + kMaxDChunks);
   uint64_t* empty = full + R;
   uint64_t* rdy = empty + R;
   int* misc = reinterpret_cast<int*>(rdy + 1);
@@ -450,7 +532,8 @@ __global__ void __launch_bounds__(kFThreads, 2) k_decode_fused(const __grid_cons
     }
     mbar_init(rdy, 1);
     fence_mbar_init();
-    int N1 = 0, ntp = 0;
+    int N1 = 0, ntp = 0, nD = 0;
+    misc[0] = 0;
     for (int p = 0; p < n; ++p) {
       const FusedProj& pp = prm.p[p];
       int pos = cta - pp.rot;
@@ -464,45 +547,43 @@ __global__ void __launch_bounds__(kFThreads, 2) k_decode_fused(const __grid_cons
       L[4] = x1 > x0 ? x0 / pp.ppr : 0;
       L[5] = x1 > x0 ? (x1 - 1) / pp.ppr - x0 / pp.ppr + 1 : 0;
       L[6] = pos;
+      for (int x = x0; x < x1; x += kPiecesPerSlot) {  // slots of this projection's pieces
+        if (nD < kMaxDChunks)
+          dtab[nD] = (uint32_t)x | ((uint32_t)min(kPiecesPerSlot, x1 - x) << 28) | ((uint32_t)p << 30);
+        ++nD;
+      }
       N1 += x1 - x0;
       ntp += L[5];
     }
-    misc[0] = 0;
-    misc[2] = 0;
-    misc[3] = N1;
-    misc[4] = ntp;
-    if (ntp > prm.n_tp) {  // the launcher sized the partial-sum area too small: refuse to run
+    misc[1] = 0;
+    misc[2] = N1;
+    misc[3] = ntp;
+    misc[4] = nD;
+    if (ntp > prm.n_tp || nD > kMaxDChunks) {  // the launcher checks both bounds: refuse rather than overrun
       atomicOr(&g_dictproj_error, 2u);
       misc[0] = 1;
+      misc[4] = 0;
     }
   }
   __syncthreads();
   if (threadIdx.x == 0) phase_mark(cta, 0);
-  const int N1 = misc[3];
-  const int nD = (N1 + kPiecesPerSlot - 1) / kPiecesPerSlot;
+  const int nD = misc[4];
 
   if (warp == kFWarps) {
     // ------------------------------------------------------------- producer warp
     unsigned long long tk = 0;
-    if (lane == 0) tk = atomicAdd(prm.ticket, 1ull);  // before any dependent grid may start
+    if (lane < n) tk = atomicAdd(prm.p[lane].ticket, 1ull);  // before any dependent grid may start
     auto issue = [&](int j) {
       const int s = j % R;
       const uint32_t dst = sbase + (uint32_t)s * kFusedSlotBytes;
       if (j < nD) {
-        const int i0 = j * kPiecesPerSlot, np = min(kPiecesPerSlot, N1 - i0);
+        const uint32_t d = dtab[j];
+        const int x = (int)(d & 0x0fffffffu), np = (int)((d >> 28) & 3u);
+        const FusedProj& pp = prm.p[d >> 30];
         mbar_arrive_expect_tx(full + s, (uint32_t)np * (kPieceCodeBytes + kPieceScaleBytes));
-        for (int i = 0; i < np; ++i) {
-          const int L = i0 + i;
-          int p = 0;
-          for (int q = 1; q < n; ++q)
-            if (L >= loc[kCtlLoc * q + 2]) p = q;
-          const FusedProj& pp = prm.p[p];
-          const int x = loc[kCtlLoc * p] + L - loc[kCtlLoc * p + 2];
-          const int a = x / pp.ppr, pc = x - a * pp.ppr;
-          tma2d(dst + i * kPieceCodeBytes, &pp.dcodes, pc * 256, a * 16, full + s);
-          tma2d(dst + i * kPieceCodeBytes + 2048, &pp.dcodes, pc * 256 + 128, a * 16, full + s);
-          tma2d(dst + kSlotScaleOff + i * kPieceScaleBytes, &pp.dscales, pc * 32, a * 16, full + s);
-        }
+        bulk_g2s_u32(dst, pp.fcodes + (size_t)x * kPieceCodeBytes, (uint32_t)np * kPieceCodeBytes, full + s);
+        bulk_g2s_u32(dst + kSlotScaleOff, pp.fscales + (size_t)x * kPieceScaleBytes, (uint32_t)np * kPieceScaleBytes,
+                     full + s);
       } else {
         const int t = j - nD;
         const uint4 d = desc[t];
@@ -556,16 +637,14 @@ __global__ void __launch_bounds__(kFThreads, 2) k_decode_fused(const __grid_cons
       desc[t] = prm.p[p].cplan[b0 + t - e0];
       desc_p[t] = (uint8_t)p;
     }
+    if (lane < n) misc[8 + lane] = (int)((uint32_t)(tk / (unsigned long long)G) + 1u);  // exchange tags
     __syncwarp();
     if (lane == 0) {
       if (total_raw > kMaxCChunks) {  // the launcher checks this bound; refuse rather than drop chunks
         atomicOr(&g_dictproj_error, 2u);
         *s_abort = 1;
       }
-      misc[2] = total;
-      const unsigned long long base = (tk / (unsigned long long)G) * (unsigned long long)G;  // arrivals before this launch
-      misc[5] = (int)(unsigned int)(base >> 32);
-      misc[6] = (int)(unsigned int)(base & 0xffffffffull);
+      misc[1] = total;
       mbar_arrive_cta(rdy);
       trigger_dependents();
       phase_mark(cta, 9);
@@ -590,7 +669,7 @@ __global__ void __launch_bounds__(kFThreads, 2) k_decode_fused(const __grid_cons
     // ------------------------------------------------------------- compute warps
     const int tid = threadIdx.x;
     const int g = lane >> 2, tq = lane & 3;
-    grid_dependency_wait();  // X, Zx and Y belong to earlier work on the stream
+    grid_dependency_wait();  // X, the exchange buffer and Y belong to earlier work on the stream
     if (tid == 0) phase_mark(cta, 1);
     for (int i = tid; i < prm.n_tp * kFWarps * 16 * MP; i += kFWarps * 32) sts_f32(sbase + prm.red_off + 4 * i, 0.f);
     for (int p = 0; p < n; ++p) {  // stage X rows (element order permuted within 512-byte blocks)
@@ -631,15 +710,12 @@ __global__ void __launch_bounds__(kFThreads, 2) k_decode_fused(const __grid_cons
       bool ok = mbar_wait_or_abort(full + s, (uint32_t)((j / R) & 1), s_abort, limit);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) continue;
-      const int np = min(kPiecesPerSlot, N1 - j * kPiecesPerSlot);
+      const uint32_t d = dtab[j];
+      const int x_first = (int)(d & 0x0fffffffu), np = (int)((d >> 28) & 3u), p = (int)(d >> 30);
+      const FusedProj& pp = prm.p[p];
       const uint32_t slot = sbase + (uint32_t)s * kFusedSlotBytes;
-      for (int t = (warp + 4 * j) % kFWarps; t < 4 * np; t += kFWarps) {  // quarters dealt round-robin, rotated per slot
-        const int L = j * kPiecesPerSlot + (t >> 2);
-        int p = 0;
-        for (int q = 1; q < n; ++q)
-          if (L >= loc[kCtlLoc * q + 2]) p = q;
-        const FusedProj& pp = prm.p[p];
-        const int x = loc[kCtlLoc * p] + L - loc[kCtlLoc * p + 2];
+      for (int t = (warp + 4 * j) % kFWarps; t < 4 * np; t += kFWarps) {  // quarters round-robin, rotated per slot
+        const int i = t >> 2, x = x_first + i;
         const int a = x / pp.ppr, pc = x - a * pp.ppr;
         const int tp = loc[kCtlLoc * p + 3] + a - loc[kCtlLoc * p + 4];
         if (tp != cur_tp) {
@@ -676,9 +752,8 @@ __global__ void __launch_bounds__(kFThreads, 2) k_decode_fused(const __grid_cons
             }
           }
         }
-        const uint32_t piece = slot + (uint32_t)(t >> 2) * kPieceCodeBytes;
-        piece_quarter(acc, piece + b * 2048, slot + kSlotScaleOff + (uint32_t)(t >> 2) * kPieceScaleBytes + b * 16, g,
-                      c16, xw);
+        piece_quarter(acc, slot + (uint32_t)i * kPieceCodeBytes + b * 128,
+                      slot + kSlotScaleOff + (uint32_t)i * kPieceScaleBytes + b * 16, g, c16, xw);
       }
       __syncwarp();
       if (lane == 0) mbar_arrive_cta(empty + s);
@@ -687,9 +762,10 @@ __global__ void __launch_bounds__(kFThreads, 2) k_decode_fused(const __grid_cons
     named_bar_sync(1, kFWarps * 32);
     if (tid == 0) phase_mark(cta, 3);
 
-    // ---- partial Z of each tile piece (sum over warps, times s_D) to the exchange buffer
-    const int ntp = misc[4];
-    if (!*s_abort) {
+    // ---- partial Z of each tile piece (sum over warps, times s_D), tagged, to the exchange buffer
+    const bool ready = __all_sync(0xffffffffu, mbar_wait_or_abort(rdy, 0, s_abort, limit));
+    const int ntp = misc[3];
+    if (ready && !*s_abort) {
       for (int v = tid; v < ntp * 16 * MP; v += kFWarps * 32) {
         const int tp = v / (16 * MP), r = v - tp * 16 * MP;
         float sum = 0.f;
@@ -701,55 +777,34 @@ __global__ void __launch_bounds__(kFThreads, 2) k_decode_fused(const __grid_cons
         const FusedProj& pp = prm.p[p];
         const int a = loc[kCtlLoc * p + 4] + tp - loc[kCtlLoc * p + 3];
         const int slot = loc[kCtlLoc * p + 6] - split_pos(a * pp.ppr, pp.pq, pp.pr);
-        pp.zx[((size_t)slot * pp.k + 16 * a) * MP + r] = sum * pp.s_D;
+        const unsigned long long word = ((unsigned long long)(uint32_t)misc[8 + p] << 32) |
+                                        (unsigned long long)__float_as_uint(sum * pp.s_D);
+        st_relaxed_u64(pp.zx + ((size_t)slot * pp.k + 16 * a) * MP + r, word);
       }
     }
-    named_bar_sync(1, kFWarps * 32);
+    if (tid == 0) phase_mark(cta, 4);
 
-    // ---- grid-wide exchange: count this CTA in, wait until every CTA of this launch is
-    // (every CTA adds exactly one per launch, aborted or not, so the count stays a
-    // multiple of G between launches; one thread per CTA polls one word, with backoff)
-    if (tid == 0) {
-      phase_mark(cta, 4);
-      __threadfence();
-      atom_add_release_u64(prm.arrive, 1ull);
-      const bool ok = mbar_wait_or_abort(rdy, 0, s_abort, limit) && !*s_abort;
-      if (ok) {
-        const unsigned long long target = ((unsigned long long)(unsigned int)misc[5] << 32 |
-                                           (unsigned int)misc[6]) + (unsigned long long)G;
-        const long long t0 = clock64();
-        unsigned int ns = 32;
-        while (ld_acquire_u64(prm.arrive) < target) {
-          if (*s_abort || clock64() - t0 > limit) {
-            if (!*s_abort) {
-              atomicOr(&g_dictproj_error, 1u);
-              *s_abort = 1;
-            }
-            break;
-          }
-          __nanosleep(ns);
-          if (ns < 256) ns <<= 1;
-        }
-      }
-      phase_mark(cta, 5);
-    }
-    named_bar_sync(1, kFWarps * 32);
-
-    // ---- stage 2: Y = Z C over this CTA's column chunks
-    const int N2 = misc[2];
+    // ---- Z tables (the exchange: each value read waits for this launch's tag)
+    const int N2 = misc[1];
     if (prm.zt_resident) {
       if (!*s_abort)
-        for (int p = 0; p < n; ++p) load_ztable<MP>(prm.p[p], sbase, tid);
+        for (int p = 0; p < n; ++p) load_ztable<MP>(prm.p[p], sbase, tid, (uint32_t)misc[8 + p], s_abort, limit);
       named_bar_sync(1, kFWarps * 32);
     }
-    if (tid == 0) phase_mark(cta, 6);
+    if (tid == 0) {
+      phase_mark(cta, 5);
+      phase_mark(cta, 6);
+    }
+
+    // ---- stage 2: Y = Z C over this CTA's column chunks, a column per half warp
+    const int half = lane >> 4;
     int cur_p = -1;
     for (int i = 0; i < N2; ++i) {
       const int j = nD + i, s = j % R;
       const int p = desc_p[i];
       if (!prm.zt_resident && p != cur_p) {  // one Z table at a time: reload between projections
         named_bar_sync(1, kFWarps * 32);
-        if (!*s_abort) load_ztable<MP>(prm.p[p], sbase, tid);
+        if (!*s_abort) load_ztable<MP>(prm.p[p], sbase, tid, (uint32_t)misc[8 + p], s_abort, limit);
         named_bar_sync(1, kFWarps * 32);
       }
       cur_p = p;
@@ -764,7 +819,11 @@ __global__ void __launch_bounds__(kFThreads, 2) k_decode_fused(const __grid_cons
       const uint32_t slot = sbase + (uint32_t)s * kFusedSlotBytes;
       const int ncols = (int)(d.y - d.x);
       const uint32_t zs = sbase + pp.zt_off;
-      for (int t = (warp + i) % kFWarps; t < ncols; t += kFWarps) {
+      const bool halves = pp.nseg <= 16;  // a column per half warp needs the segment starts in 16 lanes
+      const int per = halves ? 2 : 1;
+      for (int t0 = ((warp + i) % kFWarps) * per; t0 < ncols; t0 += kFWarps * per) {
+        const int t = t0 + (halves ? half : 0);
+        if (t >= ncols) continue;  // (halves only: this half idles; the other half's ballots use its own mask)
         const uint32_t o = d.x + (uint32_t)t;
         const uint32_t cpa = slot + c.cp_dst + 4u * o - c.cp_src;
         const uint32_t e0 = lds_u32(cpa), e1 = lds_u32(cpa + 4);
@@ -773,13 +832,22 @@ __global__ void __launch_bounds__(kFThreads, 2) k_decode_fused(const __grid_cons
         const uint32_t ssa = slot + c.ss_dst + 2u * o * (uint32_t)pp.nseg - c.ss_src;
         const int nhb = (int)((e1 - e0) >> 3);
         float y[MP];
-        switch (fmt) {  // uniform over the chunk
-          case 0: column_sum<MP, 0>(y, ia, ca, sa, ssa, nhb, pp.nseg, zs, lane); break;
-          case 1: column_sum<MP, 1>(y, ia, ca, sa, ssa, nhb, pp.nseg, zs, lane); break;
-          case 2: column_sum<MP, 2>(y, ia, ca, sa, ssa, nhb, pp.nseg, zs, lane); break;
-          default: column_sum<MP, 3>(y, ia, ca, sa, ssa, nhb, pp.nseg, zs, lane); break;
+        if (halves) {
+          switch (fmt) {  // uniform over the chunk
+            case 0: column_sum<MP, 0, 16>(y, ia, ca, sa, ssa, nhb, pp.nseg, zs, lane, half); break;
+            case 1: column_sum<MP, 1, 16>(y, ia, ca, sa, ssa, nhb, pp.nseg, zs, lane, half); break;
+            case 2: column_sum<MP, 2, 16>(y, ia, ca, sa, ssa, nhb, pp.nseg, zs, lane, half); break;
+            default: column_sum<MP, 3, 16>(y, ia, ca, sa, ssa, nhb, pp.nseg, zs, lane, half); break;
+          }
+        } else {
+          switch (fmt) {
+            case 0: column_sum<MP, 0, 32>(y, ia, ca, sa, ssa, nhb, pp.nseg, zs, lane, 0); break;
+            case 1: column_sum<MP, 1, 32>(y, ia, ca, sa, ssa, nhb, pp.nseg, zs, lane, 0); break;
+            case 2: column_sum<MP, 2, 32>(y, ia, ca, sa, ssa, nhb, pp.nseg, zs, lane, 0); break;
+            default: column_sum<MP, 3, 32>(y, ia, ca, sa, ssa, nhb, pp.nseg, zs, lane, 0); break;
+          }
         }
-        if (lane == 0) {
+        if ((lane & (halves ? 15 : 31)) == 0) {
 #pragma unroll
           for (int m = 0; m < MP; ++m)
             if (m < M) pp.Y[(size_t)m * pp.d_out + o] = __float2half_rn(y[m] * pp.s_C);
@@ -817,37 +885,32 @@ static void fused_split_bounds(int tiles, int ppr, int G, int* tp_bound, int* sl
   *slots = sl;
 }
 
-cudaError_t fused_group_setup(dictproj_group* g, bool* ok) {
+cudaError_t fused_group_setup(dictproj_group* g, const uint8_t* codes, const uint8_t* scales, bool* ok) {
   *ok = false;
   g->fused_ok = false;
-  // the TMA boxes (128 code bytes, 32 scale bytes per atom row) fit inside a row
-  // from d_in = 512 on; k must keep the gather's segments in one warp
-  if (g->d_in < kPieceElems || g->k > 8192) return cudaSuccess;
+  if (g->k > 8192) return cudaSuccess;  // the gather keeps the segment starts in one warp
   const int tiles = g->k / 16;
   g->ppr = fused_pieces_per_row(g->d_in);
   fused_split_bounds(tiles, g->ppr, g->n_sm, &g->tp_bound, &g->zslots);
-  cudaError_t e;
-  const size_t srow = (size_t)g->d_in / 16;
-  const size_t spad = (srow + 15) & ~size_t(15);
-  const uint8_t* sbase = g->scales;
-  if (spad != srow) {  // tensor-map rows must be 16-byte multiples: a padded copy of the scales
-    if ((e = cudaMalloc((void**)&g->scales_pad, spad * g->k)) != cudaSuccess) return e;
-    if ((e = cudaMemset(g->scales_pad, 0, spad * g->k)) != cudaSuccess) return e;
-    if ((e = cudaMemcpy2D(g->scales_pad, spad, g->scales, srow, srow, g->k, cudaMemcpyDeviceToDevice)) != cudaSuccess)
-      return e;
-    sbase = g->scales_pad;
+  const size_t P = (size_t)tiles * g->ppr;
+  std::vector<uint8_t> fc, fs;
+  try {
+    fc.resize(P * kPieceCodeBytes);
+    fs.resize(P * kPieceScaleBytes);
+  } catch (...) {
+    return cudaErrorMemoryAllocation;
   }
-  if ((e = encode_tiled_2d(&g->fmap_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, g->codes, (uint64_t)g->d_in / 2,
-                           (uint64_t)g->k, (uint64_t)g->d_in / 2, 128, 16, CU_TENSOR_MAP_SWIZZLE_128B)) != cudaSuccess)
-    return e;
-  if ((e = encode_tiled_2d(&g->fmap_scales, CU_TENSOR_MAP_DATA_TYPE_UINT8, sbase, (uint64_t)srow, (uint64_t)g->k,
-                           (uint64_t)spad, 32, 16, CU_TENSOR_MAP_SWIZZLE_NONE)) != cudaSuccess)
-    return e;
-  if ((e = cudaMalloc((void**)&g->zx, (size_t)g->zslots * g->k * kDecodeMaxTokens * sizeof(float))) != cudaSuccess)
-    return e;
-  const size_t sync_bytes = 2 * sizeof(unsigned long long);  // ticket, arrivals
-  if ((e = cudaMalloc((void**)&g->fsync, sync_bytes)) != cudaSuccess) return e;
-  if ((e = cudaMemset(g->fsync, 0, sync_bytes)) != cudaSuccess) return e;
+  fused_pack_dictionary(codes, scales, g->d_in, g->k, fc.data(), fs.data());
+  cudaError_t e;
+  if ((e = cudaMalloc((void**)&g->fcodes, fc.size())) != cudaSuccess) return e;
+  if ((e = cudaMalloc((void**)&g->fscales, fs.size())) != cudaSuccess) return e;
+  if ((e = cudaMemcpy(g->fcodes, fc.data(), fc.size(), cudaMemcpyHostToDevice)) != cudaSuccess) return e;
+  if ((e = cudaMemcpy(g->fscales, fs.data(), fs.size(), cudaMemcpyHostToDevice)) != cudaSuccess) return e;
+  const size_t zx_bytes = (size_t)g->zslots * g->k * kDecodeMaxTokens * sizeof(unsigned long long);
+  if ((e = cudaMalloc((void**)&g->zx, zx_bytes)) != cudaSuccess) return e;
+  if ((e = cudaMemset(g->zx, 0, zx_bytes)) != cudaSuccess) return e;  // tag 0: never a launch's tag
+  if ((e = cudaMalloc((void**)&g->fsync, 16)) != cudaSuccess) return e;
+  if ((e = cudaMemset(g->fsync, 0, 16)) != cudaSuccess) return e;
   g->fused_ok = true;
   *ok = true;
   return cudaSuccess;
@@ -942,14 +1005,16 @@ bool fused_plan_launch(int n, const dictproj_group* const* g, const dictproj_lay
   pl = FusedLaunchPlan{};
   if (n < 1 || n > kFusedMaxBatch || M < 1 || M > kDecodeMaxTokens) return false;
   const int mp = decode_mp(M);
-  int chunks = 0, tp = 0, max_ppr = 0;
+  int chunks = 0, tp = 0, max_ppr = 0, dslots = 0;
   for (int i = 0; i < n; ++i) {
     if (!g[i]->fused_ok || !l[i]->fused_ok || g[i]->n_sm != g[0]->n_sm || l[i]->n_sm != g[0]->n_sm) return false;
     chunks += l[i]->cplan_max;
     tp += g[i]->tp_bound;
     max_ppr = std::max(max_ppr, g[i]->ppr);
+    const int P = (g[i]->k / 16) * g[i]->ppr;
+    dslots += (P / g[i]->n_sm + 1 + kPiecesPerSlot - 1) / kPiecesPerSlot;
   }
-  if (chunks > kMaxCChunks) return false;
+  if (chunks > kMaxCChunks || dslots > kMaxDChunks) return false;
   pl.mp = mp;
   pl.n_tp = std::max(tp, 1);
   pl.xrow = max_ppr * 1024 + 16;
@@ -1012,11 +1077,12 @@ cudaError_t launch_fused(int n, const dictproj_group* const* g, const dictproj_l
   int rot = 0;
   for (int i = 0; i < n; ++i) {
     FusedProj& p = prm.p[i];
-    p.dcodes = g[i]->fmap_codes;
-    p.dscales = g[i]->fmap_scales;
+    p.fcodes = g[i]->fcodes;
+    p.fscales = g[i]->fscales;
     p.X = X[i];
     p.Y = Y[i];
     p.zx = g[i]->zx;
+    p.ticket = g[i]->fsync;
     p.col_ptr = l[i]->col_ptr;
     p.ccodes = l[i]->codes;
     p.cscales = l[i]->scales;
@@ -1040,9 +1106,8 @@ cudaError_t launch_fused(int n, const dictproj_group* const* g, const dictproj_l
     p.xoff = pl.xoff[i];
     p.xfirst = pl.xfirst[i];
     p.zt_off = pl.zt_off[i];
+    p.zslots = g[i]->zslots;
   }
-  prm.ticket = g[0]->fsync;
-  prm.arrive = g[0]->fsync + 1;
   prm.wait_limit = wait_limit;
   prm.n = n;
   prm.M = M;

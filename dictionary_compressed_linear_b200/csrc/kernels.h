@@ -51,9 +51,10 @@ struct FusedLaunchPlan {
   int xoff[4], xfirst[4], xslot[4], zt_off[4];
 };
 cudaError_t prepare_fused_kernels(int device);
-// Tensor maps, exchange buffer and sync words of a group (sets g->fused_ok when
-// the shape is served; allocation failures are returned).
-cudaError_t fused_group_setup(dictproj_group* g, bool* ok);
+// Tile-major dictionary copy (from the host's packed arrays), exchange buffer and
+// ticket of a group (sets g->fused_ok when the shape is served; allocation
+// failures are returned).
+cudaError_t fused_group_setup(dictproj_group* g, const uint8_t* codes, const uint8_t* scales, bool* ok);
 // Column chunks of a layer for G positions: off[G+1] into chunks {o_a, o_b, E_a, E_b}.
 // False if a column does not fit a ring slot (the layer then runs the two-kernel path).
 bool fused_layer_plan(const uint32_t* pcol_ptr, int d_out, int nseg, int fmt, int G, std::vector<uint32_t>& off,
