@@ -619,8 +619,8 @@ int dictproj_forward_path(const void* X, int M, const dictproj_layer* layer, con
     }
     if (layer->cfmt != DICTPROJ_CFMT_NVFP4)
       return fail(DICTPROJ_ERR_UNSUPPORTED,
-                  "forward: FP16 / FP8 / INT8 coefficients are decoded by the fused kernel only (d_in >= 512, k <= "
-                  "8192, Z within shared memory); this call falls outside it");
+                  "forward: FP16 / FP8 / INT8 coefficients are decoded by the fused kernel only (k <= 8192, Z "
+                  "within shared memory); this call falls outside it");
     if (!coeff_smem_fits(group->k, mp, dev))
       return fail(DICTPROJ_ERR_UNSUPPORTED,
                   "forward: the decode path stages (k + 256) * %d floats of Z in shared memory; k=%d does not fit "

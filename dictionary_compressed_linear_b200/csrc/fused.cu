@@ -337,17 +337,34 @@ __device__ __forceinline__ void half_block_sum(float out[MP], uint32_t idx_a, ui
 #pragma unroll
   for (int m = 0; m < MP; ++m) a0[m] = a1[m] = 0.f;
   if (!walk) {
+    // Entries e >= t lie in segment sgi + 1: a bump byte of 1 for them, paired with
+    // the index byte by one byte permute, gives two 9-bit atom offsets from z0.
     const int t = min(t1 - q0, 8);
+    const unsigned long long bump = t >= 8 ? 0ull : (~0ull << (8 * t)) & 0x0101010101010101ull;
+    const uint32_t bw[2] = {(uint32_t)bump, (uint32_t)(bump >> 32)};
     const uint32_t z0 = zs_a + ((uint32_t)sgi << 8) * kRow;
-    const uint32_t z1 = z0 + 256u * kRow;
+    unsigned long long acc2 = 0ull;  // (even, odd) entry sums for MP == 1
 #pragma unroll
     for (int p = 0; p < 4; ++p) {
       const float2 v = __half22float2(*reinterpret_cast<const __half2*>(&f[p]));
-      const int e0 = 2 * p, e1 = e0 + 1;
-      const uint32_t b0 = __byte_perm(iw[e0 >> 2], 0u, 0x4440u | (uint32_t)(e0 & 3));
-      const uint32_t b1 = __byte_perm(iw[e1 >> 2], 0u, 0x4440u | (uint32_t)(e1 & 3));
-      fma_z<MP>(a0, (e0 >= t ? z1 : z0) + b0 * kRow, v.x);
-      fma_z<MP>(a1, (e1 >= t ? z1 : z0) + b1 * kRow, v.y);
+      const int j0 = (2 * p) & 3, w = p >> 1;
+      const uint32_t pr = __byte_perm(iw[w], bw[w], (uint32_t)(j0 | ((j0 + 4) << 4) | ((j0 + 1) << 8) | ((j0 + 5) << 12)));
+      const uint32_t ad0 = z0 + (pr & 0xFFFFu) * kRow, ad1 = z0 + (pr >> 16) * kRow;
+      if constexpr (MP == 1) {
+        unsigned long long zz, vv;
+        asm("mov.b64 %0, {%1, %2};" : "=l"(zz) : "f"(lds_f32(ad0)), "f"(lds_f32(ad1)));
+        asm("mov.b64 %0, {%1, %2};" : "=l"(vv) : "f"(v.x), "f"(v.y));
+        asm("fma.rn.f32x2 %0, %1, %2, %0;" : "+l"(acc2) : "l"(zz), "l"(vv));
+      } else {
+        fma_z<MP>(a0, ad0, v.x);
+        fma_z<MP>(a1, ad1, v.y);
+      }
+    }
+    if constexpr (MP == 1) {
+      float lo, hi;
+      asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(acc2));
+      a0[0] = lo;
+      a1[0] = hi;
     }
   } else {
     int sg = 0;

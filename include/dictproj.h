@@ -195,7 +195,7 @@ int dictproj_pack_layer(const int32_t* col_ptr, const int32_t* atom_idx, const f
 /* A C_l with FP16 / FP8 / INT8 values (dictproj_pack_layer_fmt_host's arrays,
  * `values` of dictproj_cfmt_value_bytes(fmt) bytes per stored entry) on the
  * current device. Such a layer is decoded by the fused decode kernel
- * (M <= 8, d_in >= 512, k <= 8192) and by the prefill path; other calls with it
+ * (M <= 8, k <= 8192) and by the prefill path; other calls with it
  * return UNSUPPORTED before any launch. dictproj_layer_save refuses it (the
  * packed file holds NVFP4 layers). Errors as dictproj_layer_upload, plus RANGE
  * (fmt not FP16 / FP8 / INT8). */

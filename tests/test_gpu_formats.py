@@ -78,9 +78,9 @@ def test_prefill_parity(fmt, M):
 
 
 def test_paths_that_do_not_decode_the_format_refuse_before_launch():
-    # d_in = 256 is below the fused kernel's range: the two-kernel decode path
-    # reads NVFP4 only, so the call is refused and Y is untouched
-    g, l, pd, pf = _proj(4, 256, 128, 64, 0.5, "fp8")
+    # k = 8448 (33 segments of 256 atoms) is beyond the fused kernel's range: the
+    # two-kernel decode path reads NVFP4 only, so the call is refused and Y is untouched
+    g, l, pd, pf = _proj(4, 256, 8448, 64, 0.05, "fp8")
     X = torch.zeros((1, 256), dtype=torch.float16, device="cuda")
     Y = torch.full((1, 64), 3.0, dtype=torch.float16, device="cuda")
     st = torch.cuda.current_stream().cuda_stream

@@ -2,7 +2,7 @@
 memory by TMA, one grid-wide exchange of partial Z) against the fp64 oracle.
 
 dictproj_forward and dictproj_forward_batch route every decode call (M <= 8)
-with d_in >= 512 and k <= 8192 to it. These cases cover its edges: a reduction
+with k <= 8192 to it. These cases cover its edges: a reduction
 length that leaves a partial 512-element piece (zero-filled out of bounds), a
 single 16-atom tile, 32 segments of 256 atoms, fewer output columns than SMs
 (CTAs without columns), empty / full / one-atom columns, columns that straddle
