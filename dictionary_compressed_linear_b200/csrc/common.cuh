@@ -108,6 +108,15 @@ __device__ __forceinline__ float e4m3_to_f32(uint32_t byte) {
   return __half2float(__ushort_as_half((unsigned short)(h2 & 0xFFFF)));
 }
 
+// One E4M3 byte -> f32 with integer operations and one multiply (no conversion
+// unit): the 7 magnitude bits placed at bit 20 read as an fp32 whose exponent is
+// the E4M3 exponent field (subnormals read as fp32 subnormals), so scaling by
+// 2^(127-7) gives the E4M3 value exactly; the sign bit moves to bit 31.
+__device__ __forceinline__ float e4m3_to_f32_int(uint32_t byte) {
+  const uint32_t bits = ((byte & 0x7Fu) << 20) | ((byte & 0x80u) << 24);
+  return __uint_as_float(bits) * 0x1p120f;
+}
+
 __device__ __forceinline__ uint32_t hmul2_u32(uint32_t a, uint32_t b) {
   __half2 r = __hmul2(*reinterpret_cast<__half2*>(&a), *reinterpret_cast<__half2*>(&b));
   return *reinterpret_cast<uint32_t*>(&r);
@@ -194,14 +203,15 @@ __device__ __forceinline__ uint4 lds_u32x4(uint32_t a) {
   asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(a));
   return v;
 }
+// 8- and 16-bit loads zero-extended straight into a 32-bit register.
 __device__ __forceinline__ uint32_t lds_u8(uint32_t a) {
-  unsigned short v;
-  asm volatile("ld.shared.u8 %0, [%1];" : "=h"(v) : "r"(a));
+  uint32_t v;
+  asm volatile("ld.shared.u8 %0, [%1];" : "=r"(v) : "r"(a));
   return v;
 }
 __device__ __forceinline__ uint32_t lds_u16(uint32_t a) {
-  unsigned short v;
-  asm volatile("ld.shared.u16 %0, [%1];" : "=h"(v) : "r"(a));
+  uint32_t v;
+  asm volatile("ld.shared.u16 %0, [%1];" : "=r"(v) : "r"(a));
   return v;
 }
 

@@ -54,7 +54,10 @@ namespace dictproj {
 // ---------------------------------------------------------------------------------
 // geometry
 // ---------------------------------------------------------------------------------
-constexpr int kFWarps = 12;                      // compute warps
+#ifndef DICTPROJ_FUSED_COMPUTE_WARPS
+#define DICTPROJ_FUSED_COMPUTE_WARPS 12
+#endif
+constexpr int kFWarps = DICTPROJ_FUSED_COMPUTE_WARPS;  // compute warps
 constexpr int kFThreads = 32 * (kFWarps + 1);    // + one producer warp
 constexpr int kPieceElems = 512;                 // d_in elements of one D piece (per atom)
 constexpr int kPieceCodeBytes = 16 * 256;        // 16 atoms x 256 code bytes
@@ -64,6 +67,7 @@ constexpr int kSlotScaleOff = kPiecesPerSlot * kPieceCodeBytes;  // 12 KB
 constexpr int kMaxCChunks = 64;                  // coefficient chunks one CTA may own in one launch
 constexpr int kMaxDChunks = 64;                  // dictionary slots one CTA may own in one launch
 constexpr int kFusedMaxBatch = 4;
+constexpr int kMaxStage2Batch = 4;                         // coefficient chunks per stage-2 batch
 
 static_assert(kSlotScaleOff + kPiecesPerSlot * kPieceScaleBytes <= kFusedSlotBytes, "D pieces fit a slot");
 
@@ -180,6 +184,8 @@ struct FusedParams {
   int n_tp;                    // tile pieces the red area holds per CTA
   int zt_resident;             // 1: every projection's Z table is resident; 0: one table reloaded per projection
   int bar_off;                 // offset of the barriers and chunk descriptors
+  int part_off;                // offset of the stage-2 partial sums (two buffers of 2 x threads x MP floats)
+  int W;                       // coefficient chunks per stage-2 batch
 };
 
 }  // namespace dictproj
@@ -238,7 +244,9 @@ __device__ __forceinline__ bool mbar_wait_or_abort(uint64_t* bar, uint32_t phase
 }
 
 // Diagnostic: wall-clock (ns) at the phase boundaries of the last fused launch,
-// per CTA (slots 0-7 compute side, 8-11 producer side); read by
+// per CTA (slots 0-5 and 7 compute side, 8-11 producer side, 13 end of warp 0's
+// stage 2), and as plain values: 6 and 12 ns warp 0 waited for dictionary slots
+// and coefficient chunks, 14 coefficient chunks, 15 dictionary slots; read by
 // dictproj_diag_phase_times. A few stores per CTA and launch.
 constexpr int kPhaseCtas = 1024, kPhaseSlots = 16;
 static __device__ unsigned long long g_phase[kPhaseCtas * kPhaseSlots];
@@ -257,7 +265,7 @@ __device__ __forceinline__ void phase_mark(int cta, int slot) {
 // elements of X for token g. mma.sync m16n8k16 with the atoms as the 16 rows of A
 // and the tokens as the 8 columns of B: within each thread the same element
 // order is used for A and B, so the sum over k is unchanged.
-__device__ __forceinline__ void piece_quarter(float acc[2][4], uint32_t box, uint32_t scl, int g, int c16,
+__device__ __forceinline__ void piece_quarter(float acc[4][4], uint32_t box, uint32_t scl, int g, int c16,
                                               const uint32_t xw[4][4]) {
   const uint32_t ra = box + g * 256 + ((uint32_t)(c16 ^ g) << 4);
   const uint4 wa4 = lds_u32x4(ra), wb4 = lds_u32x4(ra + 2048);
@@ -281,7 +289,7 @@ __device__ __forceinline__ void piece_quarter(float acc[2][4], uint32_t box, uin
     for (int h = 0; h < 2; ++h) {
       const uint32_t a[4] = {fa[2 * h], fb[2 * h], fa[2 * h + 1], fb[2 * h + 1]};
       const uint32_t b[2] = {xw[q][2 * h], xw[q][2 * h + 1]};
-      mma_16816(acc[h], a, b);
+      mma_16816(acc[2 * (q & 1) + h], a, b);  // four accumulators: two MMAs in each chain
     }
   }
 }
@@ -289,27 +297,36 @@ __device__ __forceinline__ void piece_quarter(float acc[2][4], uint32_t box, uin
 // ---------------------------------------------------------------------------------
 // stage 2: coefficient values and one column from a shared-memory chunk
 // ---------------------------------------------------------------------------------
-// Eight stored values of half-block hb as four f16x2 (their fp16 forms are
-// exact: E2M1, E4M3 and small integers are fp16 numbers), for each format.
+// The stored values of half-block hb (8 entries) as raw words, and as four f16x2
+// (their fp16 forms are exact: E2M1, E4M3 and small integers are fp16 numbers),
+// for each format.
 template <int FMT>
-__device__ __forceinline__ void half_block_values(uint32_t code_a, int hb, uint32_t f[4]) {
+__device__ __forceinline__ uint4 hb_load(uint32_t code_a, int hb) {
   if constexpr (FMT == 0) {  // NVFP4: 8 nibbles
-    e2m1x8_to_f16x2x4(lds_u32(code_a + 4 * hb), f);
+    return make_uint4(lds_u32(code_a + 4u * (uint32_t)hb), 0u, 0u, 0u);
   } else if constexpr (FMT == 1) {  // FP16
-    const uint4 v = lds_u32x4(code_a + 16 * hb);
-    f[0] = v.x;
-    f[1] = v.y;
-    f[2] = v.z;
-    f[3] = v.w;
-  } else if constexpr (FMT == 2) {  // FP8 E4M3
-    const uint2 v = lds_u32x2(code_a + 8 * hb);
-    f[0] = e4m3x2_to_f16x2(v.x & 0xFFFF);
-    f[1] = e4m3x2_to_f16x2(v.x >> 16);
-    f[2] = e4m3x2_to_f16x2(v.y & 0xFFFF);
-    f[3] = e4m3x2_to_f16x2(v.y >> 16);
+    return lds_u32x4(code_a + 16u * (uint32_t)hb);
+  } else {  // FP8 / INT8
+    const uint2 v = lds_u32x2(code_a + 8u * (uint32_t)hb);
+    return make_uint4(v.x, v.y, 0u, 0u);
+  }
+}
+template <int FMT>
+__device__ __forceinline__ void hb_decode(uint4 r, uint32_t f[4]) {
+  if constexpr (FMT == 0) {
+    e2m1x8_to_f16x2x4(r.x, f);
+  } else if constexpr (FMT == 1) {
+    f[0] = r.x;
+    f[1] = r.y;
+    f[2] = r.z;
+    f[3] = r.w;
+  } else if constexpr (FMT == 2) {  // E4M3
+    f[0] = e4m3x2_to_f16x2(r.x & 0xFFFF);
+    f[1] = e4m3x2_to_f16x2(r.x >> 16);
+    f[2] = e4m3x2_to_f16x2(r.y & 0xFFFF);
+    f[3] = e4m3x2_to_f16x2(r.y >> 16);
   } else {  // INT8: |code| <= 127 is exact in fp16
-    const uint2 v = lds_u32x2(code_a + 8 * hb);
-    const uint32_t w[2] = {v.x, v.y};
+    const uint32_t w[2] = {r.x, r.y};
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
       const uint32_t word = w[i >> 1];
@@ -321,125 +338,191 @@ __device__ __forceinline__ void half_block_values(uint32_t code_a, int hb, uint3
   }
 }
 
-// Sum over the 8 entries q0 .. q0+7 of a half-block: at most one segment
-// boundary inside (t: first entry in segment sgi+1) unless `walk`, in which case
-// the entries advance through seg_start one by one. Unscaled (block scale and
-// s_C are applied by the caller).
-template <int MP, int FMT>
-__device__ __forceinline__ void half_block_sum(float out[MP], uint32_t idx_a, uint32_t code_a, uint32_t ss_a,
-                                               int hb, int q0, int sgi, int t1, bool walk, int nseg, uint32_t zs_a) {
+// x << n with the PTX rule for n >= 32 (the result is 0).
+__device__ __forceinline__ uint32_t shl_clamped(uint32_t x, uint32_t n) {
+  uint32_t r;
+  asm("shl.b32 %0, %1, %2;" : "=r"(r) : "r"(x), "r"(n));
+  return r;
+}
+
+// Segment state of a thread inside one column of C_l: sg is the segment of the
+// current entry q (the number of segment starts s >= 1 with seg_start[s] <= q),
+// nb and nb2 the next two segment starts (kSegNone past the last one).
+constexpr int kSegNone = 1 << 30;
+struct SegState {
+  int sg, nb, nb2;
+};
+__device__ __forceinline__ int seg_at(uint32_t ssa, int s, int nseg) {
+  return s < nseg ? (int)lds_u16(ssa + 2u * (uint32_t)s) : kSegNone;
+}
+__device__ __forceinline__ SegState seg_find(uint32_t ssa, int q, int nseg) {
+  SegState st;
+  st.sg = 0;
+  for (int s = 1; s < nseg; ++s) st.sg += ((int)lds_u16(ssa + 2u * (uint32_t)s) <= q);
+  st.nb = seg_at(ssa, st.sg + 1, nseg);
+  st.nb2 = seg_at(ssa, st.sg + 2, nseg);
+  return st;
+}
+// Move the state forward to the segment of entry q (segment starts only grow).
+__device__ __forceinline__ void seg_advance(SegState& st, uint32_t ssa, int q, int nseg) {
+  while (st.nb <= q) {
+    ++st.sg;
+    st.nb = st.nb2;
+    st.nb2 = seg_at(ssa, st.sg + 2, nseg);
+  }
+}
+
+// Sum over the 8 entries of a half-block (index bytes iv, values f) whose entries
+// lie in at most two segments: entries e >= t belong to the segment `delta` after
+// the one whose Z rows start at z0 (t >= 8: none). A bump byte of delta for those
+// entries, paired with the index byte by one byte permute, gives two atom offsets
+// from z0. Unscaled (block scale and s_C are applied by the caller).
+// Sum over the 8 entries of a half-block (index bytes iv, values f) whose entries
+// lie in at most two segments: entries e >= t belong to the segment after the one
+// whose Z rows start at z0 (t >= 8: none). A bump byte of 1 for those entries,
+// paired with the index byte by one byte permute, gives two atom offsets from z0.
+// Unscaled (block scale and s_C are applied by the caller).
+template <int MP>
+__device__ __forceinline__ void hb_sum(float out[MP], uint2 iv, const uint32_t f[4], uint32_t z0, int t) {
   constexpr uint32_t kRow = MP * 4;
-  const uint2 iv = lds_u32x2(idx_a + 8 * hb);
   const uint32_t iw[2] = {iv.x, iv.y};
-  uint32_t f[4];
-  half_block_values<FMT>(code_a, hb, f);
+  const uint32_t tt = (uint32_t)min(t, 8);  // entries tt..7 get a bump byte of 1
+  const uint32_t bw[2] = {shl_clamped(0x01010101u, 8u * tt), shl_clamped(0x01010101u, 8u * (tt > 4u ? tt - 4u : 0u))};
   float a0[MP], a1[MP];
 #pragma unroll
   for (int m = 0; m < MP; ++m) a0[m] = a1[m] = 0.f;
-  if (!walk) {
-    // Entries e >= t lie in segment sgi + 1: a bump byte of 1 for them, paired with
-    // the index byte by one byte permute, gives two 9-bit atom offsets from z0.
-    const int t = min(t1 - q0, 8);
-    const unsigned long long bump = t >= 8 ? 0ull : (~0ull << (8 * t)) & 0x0101010101010101ull;
-    const uint32_t bw[2] = {(uint32_t)bump, (uint32_t)(bump >> 32)};
-    const uint32_t z0 = zs_a + ((uint32_t)sgi << 8) * kRow;
-    unsigned long long acc2 = 0ull;  // (even, odd) entry sums for MP == 1
 #pragma unroll
-    for (int p = 0; p < 4; ++p) {
-      const float2 v = __half22float2(*reinterpret_cast<const __half2*>(&f[p]));
-      const int j0 = (2 * p) & 3, w = p >> 1;
-      const uint32_t pr = __byte_perm(iw[w], bw[w], (uint32_t)(j0 | ((j0 + 4) << 4) | ((j0 + 1) << 8) | ((j0 + 5) << 12)));
-      const uint32_t ad0 = z0 + (pr & 0xFFFFu) * kRow, ad1 = z0 + (pr >> 16) * kRow;
-      if constexpr (MP == 1) {
-        unsigned long long zz, vv;
-        asm("mov.b64 %0, {%1, %2};" : "=l"(zz) : "f"(lds_f32(ad0)), "f"(lds_f32(ad1)));
-        asm("mov.b64 %0, {%1, %2};" : "=l"(vv) : "f"(v.x), "f"(v.y));
-        asm("fma.rn.f32x2 %0, %1, %2, %0;" : "+l"(acc2) : "l"(zz), "l"(vv));
-      } else {
-        fma_z<MP>(a0, ad0, v.x);
-        fma_z<MP>(a1, ad1, v.y);
-      }
-    }
-    if constexpr (MP == 1) {
-      float lo, hi;
-      asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(acc2));
-      a0[0] = lo;
-      a1[0] = hi;
-    }
-  } else {
-    int sg = 0;
-    for (int j = 1; j < nseg; ++j) sg += ((int)lds_u16(ss_a + 2 * j) <= q0);
-    int nb = (sg + 1 < nseg) ? (int)lds_u16(ss_a + 2 * (sg + 1)) : INT_MAX;
-#pragma unroll
-    for (int p = 0; p < 4; ++p) {
-      const float2 v = __half22float2(*reinterpret_cast<const __half2*>(&f[p]));
-#pragma unroll
-      for (int hh = 0; hh < 2; ++hh) {
-        const int ent = 2 * p + hh;
-        while (q0 + ent >= nb) {
-          ++sg;
-          nb = (sg + 1 < nseg) ? (int)lds_u16(ss_a + 2 * (sg + 1)) : INT_MAX;
-        }
-        const uint32_t bb = __byte_perm(iw[ent >> 2], 0u, 0x4440u | (uint32_t)(ent & 3));
-        fma_z<MP>(hh ? a1 : a0, zs_a + (((uint32_t)sg << 8) + bb) * kRow, hh ? v.y : v.x);
-      }
-    }
+  for (int p = 0; p < 4; ++p) {
+    const float2 v = __half22float2(*reinterpret_cast<const __half2*>(&f[p]));
+    const int j0 = (2 * p) & 3, w = p >> 1;
+    const uint32_t pr = __byte_perm(iw[w], bw[w], (uint32_t)(j0 | ((j0 + 4) << 4) | ((j0 + 1) << 8) | ((j0 + 5) << 12)));
+    fma_z<MP>(a0, z0 + (pr & 0xFFFFu) * kRow, v.x);
+    fma_z<MP>(a1, z0 + (pr >> 16) * kRow, v.y);
   }
 #pragma unroll
   for (int m = 0; m < MP; ++m) out[m] = a0[m] + a1[m];
 }
 
-// One column by G lanes (G = 32: a warp; G = 16: half a warp, `half` 0 / 1) in
-// windows of 8*G entries: lane l of the group takes half-block G*i + l. The
-// segment of each half-block's first entry, and the first entry of the next
-// segment inside it, come from ballots over seg_start (lane l holds
-// seg_start[l], so nseg <= G); two boundaries inside one half-block make the
-// whole window walk. Returns the column sum (unscaled by s_C) in every lane.
-template <int MP, int FMT, int G>
-__device__ __forceinline__ void column_sum(float acc[MP], uint32_t idx_a, uint32_t code_a, uint32_t sc_a,
-                                           uint32_t ss_a, int nhb, int nseg, uint32_t zs_a, int lane, int half) {
-  const unsigned gmask = G == 32 ? 0xffffffffu : (0xffffu << (16 * half));
-  const int gl = G == 32 ? lane : lane & 15;
-  const unsigned gsh = G == 32 ? 0u : 16u * half;
-  const unsigned lowbits = G == 32 ? 0xffffffffu : 0xffffu;
+// The same sum when two or more segment starts lie inside the half-block: the
+// segment advances entry by entry (q: column position of the first entry). Rare,
+// so written as a plain loop to keep the hot loop's code small.
+template <int MP>
+__device__ __forceinline__ void hb_walk(float out[MP], uint2 iv, const uint32_t f[4], uint32_t zs, SegState& st,
+                                        uint32_t ssa, int q, int nseg) {
+  constexpr uint32_t kRow = MP * 4;
+#pragma unroll
+  for (int m = 0; m < MP; ++m) out[m] = 0.f;
+#pragma unroll 1
+  for (int ent = 0; ent < 8; ++ent) {
+    seg_advance(st, ssa, q + ent, nseg);
+    const uint32_t w = ent < 4 ? iv.x : iv.y;
+    const uint32_t bb = (w >> (8 * (ent & 3))) & 0xFFu;
+    const uint32_t fw = f[0];
+    const uint32_t fp = ent < 2 ? fw : ent < 4 ? f[1] : ent < 6 ? f[2] : f[3];
+    const float v = __half2float(__ushort_as_half((unsigned short)((ent & 1) ? fp >> 16 : fp & 0xFFFFu)));
+    fma_z<MP>(out, zs + (((uint32_t)st.sg << 8) + bb) * kRow, v);
+  }
+}
+
+// Stage 2 over a batch of resident coefficient chunks: the batch's half-blocks
+// (chunk after chunk) are split evenly over the NL compute threads, thread L
+// taking a contiguous run; stage2_run does the part of the run that lies in one
+// chunk (columns [d.x, d.y), stored entries [d.z, d.w), in shared memory at
+// `slot`; local half-blocks [h, h1)). Columns never cross chunks. A column that
+// lies inside one run is finished by its thread (Y written); otherwise the thread
+// leaves its share in the partial area `part`: HEAD (slot 0) for a column that
+// began before its run, TAIL (slot 1) for one that began inside it and goes on
+// after it, and then reports the column and its end (tail_o, tail_he): after the
+// batch it adds the HEAD shares of the following threads to its TAIL, in order
+// (the result does not depend on timing). Empty columns are written separately.
+template <int MP, int FMT>
+__device__ __forceinline__ void stage2_run(const FusedProj& pp, uint4 d, const CChunk& c, uint32_t slot,
+                                           uint32_t zs, int h, int h1, int L, uint32_t part, int M, float yscale,
+                                           int* tail_o, int* tail_he) {
+  constexpr uint32_t kRow = MP * 4;
+  if (h >= h1) return;
+  const int nseg = pp.nseg;
+  const uint32_t cpa = slot + c.cp_dst - c.cp_src;  // col_ptr[o] at cpa + 4 o
+  const uint32_t ssb = slot + c.ss_dst - c.ss_src;  // seg_start row of column o at ssb + 2 o nseg
+  const uint32_t ca = slot + c.code_dst + ((d.z * cfmt_nibbles(FMT)) >> 1) - c.code_src;
+  const uint32_t sa = slot + c.sc_dst + (d.z >> 4) - c.sc_src;
+  const uint32_t E0 = d.z + 8u * (uint32_t)h;
+  int lo = (int)d.x, hi = (int)d.y - 1;  // the column holding entry E0: last o with col_ptr[o] <= E0
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (lds_u32(cpa + 4u * (uint32_t)mid) <= E0) lo = mid;
+    else hi = mid - 1;
+  }
+  int o = lo;
+  uint32_t cb = lds_u32(cpa + 4u * (uint32_t)o), ce = lds_u32(cpa + 4u * (uint32_t)o + 4u);
+  bool started = cb == E0;
+  int he = (int)((ce - d.z) >> 3);  // first half-block after column o
+  int q = (int)(E0 - cb);           // column position of the half-block's first entry
+  uint32_t ssa = ssb + 2u * (uint32_t)o * (uint32_t)nseg;
+  SegState st = seg_find(ssa, q, nseg);
+  float acc[MP];
 #pragma unroll
   for (int m = 0; m < MP; ++m) acc[m] = 0.f;
-  const bool is_bnd = gl >= 1 && gl < nseg;
-  const int b = gl < nseg ? (int)lds_u16(ss_a + 2 * gl) : 0;
-  for (int i = 0; 8 * G * i < 8 * nhb; ++i) {
-    const int w = 8 * G * i;
-    const int s_lo = __popc((__ballot_sync(gmask, is_bnd && b <= w) >> gsh) & lowbits);
-    const bool in_win = is_bnd && b > w && b < w + 8 * G;
-    const int rel = b - w;
-    const uint32_t at_start = (in_win && (rel & 7) == 0) ? (1u << (rel >> 3)) : 0u;
-    const uint32_t inside = (in_win && (rel & 7) != 0) ? (1u << (rel >> 3)) : 0u;
-    const uint32_t A = __reduce_or_sync(gmask, at_start);
-    const uint32_t B = __reduce_or_sync(gmask, inside);
-    const int nwin = __popc((__ballot_sync(gmask, in_win) >> gsh) & lowbits);
-    const bool collide = nwin != __popc(A) + __popc(B) || (A & B) != 0u;
-    const uint32_t le = gl == 31 ? 0xffffffffu : ((2u << gl) - 1u);
-    const int sgi = s_lo + __popc(A & le) + __popc(B & (le >> 1));  // segment of the lane's first entry
-    const int q0 = w + 8 * gl;
-    const int bn = __shfl_sync(gmask, b, min(sgi + 1, G - 1), G);
-    const int t1 = ((B >> gl) & 1u) ? bn : INT_MAX;
-    const int hb = G * i + gl;
-    if (hb < nhb) {
-      float s8[MP];
-      half_block_sum<MP, FMT>(s8, idx_a, code_a, ss_a, hb, q0, sgi, t1, collide, nseg, zs_a);
-      if constexpr (FMT == 0) {
-        const float sc = e4m3_to_f32(lds_u8(sc_a + (hb >> 1)));
+  // A column that ends inside the run is finished by its thread: written to Y if it
+  // also began there, else left as HEAD.
+  auto finish = [&]() {
+    if (started) {
 #pragma unroll
-        for (int m = 0; m < MP; ++m) acc[m] = fmaf(s8[m], sc, acc[m]);
-      } else {
+      for (int m = 0; m < MP; ++m)
+        if (m < M) pp.Y[(size_t)m * pp.d_out + o] = __float2half_rn(acc[m] * yscale);
+    } else {
+      const uint32_t pa = part + (uint32_t)(2 * L * MP) * 4u;
 #pragma unroll
-        for (int m = 0; m < MP; ++m) acc[m] += s8[m];
-      }
+      for (int m = 0; m < MP; ++m) sts_f32(pa + 4u * m, acc[m]);
+    }
+  };
+  // One loop over the run's half-blocks for every thread of the warp; a column
+  // change is a short branch inside it.
+  for (; h < h1; ++h, q += 8) {
+    if (h == he) {
+      finish();
+      do {  // the next column with entries (empty columns are written by stage2_combine)
+        ++o;
+        cb = ce;
+        ce = lds_u32(cpa + 4u * (uint32_t)o + 4u);
+      } while (ce == cb);
+      he = (int)((ce - d.z) >> 3);
+      started = true;
+      q = 0;
+      ssa = ssb + 2u * (uint32_t)o * (uint32_t)nseg;
+      st = seg_find(ssa, 0, nseg);
+#pragma unroll
+      for (int m = 0; m < MP; ++m) acc[m] = 0.f;
+    }
+    const uint2 iv = lds_u32x2(slot + 8u * (uint32_t)h);
+    uint32_t f[4];
+    hb_decode<FMT>(hb_load<FMT>(ca, h), f);
+    float s8[MP];
+    if (st.nb2 < q + 8) {  // three or more segments (rare)
+      hb_walk<MP>(s8, iv, f, zs, st, ssa, q, nseg);
+    } else {
+      hb_sum<MP>(s8, iv, f, zs + ((uint32_t)st.sg << 8) * kRow, st.nb - q);
+    }
+    seg_advance(st, ssa, q + 8, nseg);
+    if constexpr (FMT == 0) {
+      const float sc = e4m3_to_f32_int(lds_u8(sa + ((uint32_t)h >> 1)));
+#pragma unroll
+      for (int m = 0; m < MP; ++m) acc[m] = fmaf(s8[m], sc, acc[m]);
+    } else {
+#pragma unroll
+      for (int m = 0; m < MP; ++m) acc[m] += s8[m];
     }
   }
+  if (he == h1) {
+    finish();
+  } else {  // the run ends inside column o: TAIL if it began in the run, else HEAD
+    const uint32_t pa = part + (uint32_t)((2 * L + (started ? 1 : 0)) * MP) * 4u;
 #pragma unroll
-  for (int m = 0; m < MP; ++m) {
-#pragma unroll
-    for (int off = G / 2; off > 0; off >>= 1) acc[m] += __shfl_xor_sync(gmask, acc[m], off, G);
+    for (int m = 0; m < MP; ++m) sts_f32(pa + 4u * m, acc[m]);
+    if (started) {
+      *tail_o = o;
+      *tail_he = he;
+    }
   }
 }
 
@@ -481,12 +564,14 @@ __device__ __forceinline__ float ll_value(const unsigned long long* p, unsigned 
 }
 
 // Z table of a projection in shared memory: Z[atom][m] = sum, in slot order, of the
-// tile's partial sums in the exchange buffer (each read waits for this launch's
-// tag), then a zero tail of 256 atom rows (padding entries read it).
+// tile's partial sums in the exchange buffer, then a zero tail of 256 atom rows
+// (padding entries read it). Each thread loads a batch of words at once and
+// re-reads all of the batch's words that do not yet carry this launch's tag
+// together, so a batch costs one round trip to L2 once its writers are done.
 template <int MP>
 __device__ __forceinline__ void load_ztable(const FusedProj& pp, uint32_t sbase, int tid, uint32_t tag,
                                             volatile int* abort, long long limit) {
-  constexpr int NT = kFWarps * 32, B = 4, S = 4;
+  constexpr int NT = kFWarps * 32, B = 8, S = 2;
   const uint32_t zt = sbase + pp.zt_off;
   const int ne = pp.k * MP;
   const size_t stride = (size_t)pp.k * MP;
@@ -504,6 +589,27 @@ __device__ __forceinline__ void load_ztable(const FusedProj& pp, uint32_t sbase,
 #pragma unroll
       for (int s = 0; s < S; ++s) v[i][s] = s < ns[i] ? ld_relaxed_u64(pp.zx + s * stride + e) : 0ull;
     }
+    long long t0 = -1;
+    while (true) {
+      bool stale = false;
+#pragma unroll
+      for (int i = 0; i < B; ++i)
+#pragma unroll
+        for (int s = 0; s < S; ++s) stale |= s < ns[i] && (uint32_t)(v[i][s] >> 32) != tag;
+      if (!stale || *abort) break;
+      if (t0 < 0) {
+        t0 = clock64();
+      } else if (clock64() - t0 > limit) {
+        atomicOr(&g_dictproj_error, 1u);
+        *abort = 1;
+        break;
+      }
+#pragma unroll
+      for (int i = 0; i < B; ++i)
+#pragma unroll
+        for (int s = 0; s < S; ++s)
+          if (s < ns[i] && (uint32_t)(v[i][s] >> 32) != tag) v[i][s] = ld_relaxed_u64(pp.zx + s * stride + base + i * NT);
+    }
 #pragma unroll
     for (int i = 0; i < B; ++i) {
       const int e = base + i * NT;
@@ -511,8 +617,8 @@ __device__ __forceinline__ void load_ztable(const FusedProj& pp, uint32_t sbase,
       float sum = 0.f;
 #pragma unroll
       for (int s = 0; s < S; ++s)
-        if (s < ns[i]) sum += ll_value(pp.zx + s * stride + e, v[i][s], tag, abort, limit);
-      for (int s = S; s < ns[i]; ++s) {
+        if (s < ns[i]) sum += __uint_as_float((uint32_t)(v[i][s] & 0xffffffffull));
+      for (int s = S; s < ns[i]; ++s) {  // tiles split over more than S positions (rare: one read at a time)
         const unsigned long long* p = pp.zx + s * stride + e;
         sum += ll_value(p, ld_relaxed_u64(p), tag, abort, limit);
       }
@@ -692,40 +798,62 @@ __global__ void __launch_bounds__(kFThreads, 2) k_decode_fused(const __grid_cons
     for (int p = 0; p < n; ++p) {  // stage X rows (element order permuted within 512-byte blocks)
       const FusedProj& pp = prm.p[p];
       if (pp.xoff < 0 || !pp.xfirst) continue;
-      const int vpr = pp.ppr * 64;
-      for (int v = tid; v < M * vpr; v += kFWarps * 32) {
-        const int m = v / vpr, e = 8 * (v - m * vpr);
-        const uint32_t dst = sbase + pp.xoff + m * prm.xrow + (e >> 8) * 512 + ((e >> 3) & 3) * 128 + ((e >> 5) & 7) * 16;
-        const uint4 val = e < pp.d_in ? ld_cg_v4(pp.X + (size_t)m * pp.d_in + e) : make_uint4(0, 0, 0, 0);
-        sts_u32x4(dst, val);
+      constexpr int NT = kFWarps * 32, U = 4;
+      const int vpr = pp.ppr * 64, nv = M * vpr;
+      for (int v0 = tid; v0 < nv; v0 += U * NT) {  // U loads in flight per thread
+        uint4 val[U];
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+          const int v = v0 + u * NT, m = v / vpr, e = 8 * (v - m * vpr);
+          val[u] = v < nv && e < pp.d_in ? ld_cg_v4(pp.X + (size_t)m * pp.d_in + e) : make_uint4(0, 0, 0, 0);
+        }
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+          const int v = v0 + u * NT, m = v / vpr, e = 8 * (v - m * vpr);
+          if (v < nv)
+            sts_u32x4(sbase + pp.xoff + m * prm.xrow + (e >> 8) * 512 + ((e >> 3) & 3) * 128 + ((e >> 5) & 7) * 16,
+                      val[u]);
+        }
       }
     }
     named_bar_sync(1, kFWarps * 32);
     if (tid == 0) phase_mark(cta, 2);
 
     // ---- stage 1: partial Z of this CTA's D pieces
-    float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+    float acc[4][4];
+#pragma unroll
+    for (int h = 0; h < 4; ++h)
+#pragma unroll
+      for (int i = 0; i < 4; ++i) acc[h][i] = 0.f;
     int cur_tp = -1;
     auto flush = [&](int tp) {
       const uint32_t rb = sbase + prm.red_off + (uint32_t)((tp * kFWarps + warp) * 16 * MP) * 4;
       const int m0 = 2 * tq, m1 = 2 * tq + 1;
       if (m0 < MP) {
-        sts_f32(rb + (g * MP + m0) * 4, acc[0][0] + acc[1][0]);
-        sts_f32(rb + ((g + 8) * MP + m0) * 4, acc[0][2] + acc[1][2]);
+        sts_f32(rb + (g * MP + m0) * 4, (acc[0][0] + acc[1][0]) + (acc[2][0] + acc[3][0]));
+        sts_f32(rb + ((g + 8) * MP + m0) * 4, (acc[0][2] + acc[1][2]) + (acc[2][2] + acc[3][2]));
       }
       if (m1 < MP) {
-        sts_f32(rb + (g * MP + m1) * 4, acc[0][1] + acc[1][1]);
-        sts_f32(rb + ((g + 8) * MP + m1) * 4, acc[0][3] + acc[1][3]);
+        sts_f32(rb + (g * MP + m1) * 4, (acc[0][1] + acc[1][1]) + (acc[2][1] + acc[3][1]));
+        sts_f32(rb + ((g + 8) * MP + m1) * 4, (acc[0][3] + acc[1][3]) + (acc[2][3] + acc[3][3]));
       }
 #pragma unroll
-      for (int h = 0; h < 2; ++h)
+      for (int h = 0; h < 4; ++h)
 #pragma unroll
         for (int i = 0; i < 4; ++i) acc[h][i] = 0.f;
     };
+    unsigned long long s1_wait = 0;  // ns warp 0 waited for dictionary slots (diagnostic)
     for (int j = 0; j < nD; ++j) {
       const int s = j % R;
+      unsigned long long tw0 = 0;
+      if (tid == 0) asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(tw0));
       bool ok = mbar_wait_or_abort(full + s, (uint32_t)((j / R) & 1), s_abort, limit);
       ok = __all_sync(0xffffffffu, ok);
+      if (tid == 0) {
+        unsigned long long tw1;
+        asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(tw1));
+        s1_wait += tw1 - tw0;
+      }
       if (!ok) continue;
       const uint32_t d = dtab[j];
       const int x_first = (int)(d & 0x0fffffffu), np = (int)((d >> 28) & 3u), p = (int)(d >> 30);
@@ -803,75 +931,115 @@ __global__ void __launch_bounds__(kFThreads, 2) k_decode_fused(const __grid_cons
 
     // ---- Z tables (the exchange: each value read waits for this launch's tag)
     const int N2 = misc[1];
-    if (prm.zt_resident) {
-      if (!*s_abort)
-        for (int p = 0; p < n; ++p) load_ztable<MP>(prm.p[p], sbase, tid, (uint32_t)misc[8 + p], s_abort, limit);
+    if (prm.zt_resident) {  // (every compute thread calls it: it holds a barrier; an abort only cuts the waits)
+      for (int p = 0; p < n; ++p)
+        load_ztable<MP>(prm.p[p], sbase, tid, (uint32_t)misc[8 + p], s_abort, limit);
       named_bar_sync(1, kFWarps * 32);
     }
     if (tid == 0) {
       phase_mark(cta, 5);
-      phase_mark(cta, 6);
+      if (cta < kPhaseCtas) g_phase[cta * kPhaseSlots + 6] = s1_wait;
     }
 
-    // ---- stage 2: Y = Z C over this CTA's column chunks, a column per half warp
-    const int half = lane >> 4;
-    int cur_p = -1;
-    for (int i = 0; i < N2; ++i) {
-      const int j = nD + i, s = j % R;
-      const int p = desc_p[i];
+    // ---- stage 2: Y = Z C over this CTA's column chunks, in batches of up to W
+    // resident chunks of one projection: the batch's half-blocks split evenly over
+    // the compute threads, then split columns combined
+    constexpr int NL = kFWarps * 32;
+    const int W = prm.W;
+    int cur_p = -1, nb_done = 0;
+    unsigned long long s2_wait = 0;  // ns thread 0 waited for coefficient chunks (diagnostic)
+    for (int i0 = 0; i0 < N2; ++nb_done) {
+      const int p = desc_p[i0];
+      int i1 = i0 + 1;
+      while (i1 < N2 && i1 - i0 < W && desc_p[i1] == p) ++i1;
       if (!prm.zt_resident && p != cur_p) {  // one Z table at a time: reload between projections
-        named_bar_sync(1, kFWarps * 32);
-        if (!*s_abort) load_ztable<MP>(prm.p[p], sbase, tid, (uint32_t)misc[8 + p], s_abort, limit);
-        named_bar_sync(1, kFWarps * 32);
+        named_bar_sync(1, NL);
+        load_ztable<MP>(prm.p[p], sbase, tid, (uint32_t)misc[8 + p], s_abort, limit);
+        named_bar_sync(1, NL);
       }
       cur_p = p;
-      bool ok = mbar_wait_or_abort(full + s, (uint32_t)((j / R) & 1), s_abort, limit);
-      ok = __all_sync(0xffffffffu, ok);
-      if (!ok) continue;
       const FusedProj& pp = prm.p[p];
-      const uint4 d = desc[i];
-      const int fmt = pp.cfmt;
-      const CChunk c = c_chunk_layout(d.x, d.y, d.z, d.w, (uint32_t)pp.nseg, fmt);
-      const uint32_t vn = cfmt_nibbles(fmt);
-      const uint32_t slot = sbase + (uint32_t)s * kFusedSlotBytes;
-      const int ncols = (int)(d.y - d.x);
+      const int fmt = pp.cfmt, nseg = pp.nseg;
       const uint32_t zs = sbase + pp.zt_off;
-      const bool halves = pp.nseg <= 16;  // a column per half warp needs the segment starts in 16 lanes
-      const int per = halves ? 2 : 1;
-      for (int t0 = ((warp + i) % kFWarps) * per; t0 < ncols; t0 += kFWarps * per) {
-        const int t = t0 + (halves ? half : 0);
-        if (t >= ncols) continue;  // (halves only: this half idles; the other half's ballots use its own mask)
-        const uint32_t o = d.x + (uint32_t)t;
-        const uint32_t cpa = slot + c.cp_dst + 4u * o - c.cp_src;
-        const uint32_t e0 = lds_u32(cpa), e1 = lds_u32(cpa + 4);
-        const uint32_t ia = slot + (e0 - d.z), ca = slot + c.code_dst + ((e0 * vn) >> 1) - c.code_src;
-        const uint32_t sa = slot + c.sc_dst + (e0 >> 4) - c.sc_src;
-        const uint32_t ssa = slot + c.ss_dst + 2u * o * (uint32_t)pp.nseg - c.ss_src;
-        const int nhb = (int)((e1 - e0) >> 3);
-        float y[MP];
-        if (halves) {
-          switch (fmt) {  // uniform over the chunk
-            case 0: column_sum<MP, 0, 16>(y, ia, ca, sa, ssa, nhb, pp.nseg, zs, lane, half); break;
-            case 1: column_sum<MP, 1, 16>(y, ia, ca, sa, ssa, nhb, pp.nseg, zs, lane, half); break;
-            case 2: column_sum<MP, 2, 16>(y, ia, ca, sa, ssa, nhb, pp.nseg, zs, lane, half); break;
-            default: column_sum<MP, 3, 16>(y, ia, ca, sa, ssa, nhb, pp.nseg, zs, lane, half); break;
-          }
-        } else {
-          switch (fmt) {
-            case 0: column_sum<MP, 0, 32>(y, ia, ca, sa, ssa, nhb, pp.nseg, zs, lane, 0); break;
-            case 1: column_sum<MP, 1, 32>(y, ia, ca, sa, ssa, nhb, pp.nseg, zs, lane, 0); break;
-            case 2: column_sum<MP, 2, 32>(y, ia, ca, sa, ssa, nhb, pp.nseg, zs, lane, 0); break;
-            default: column_sum<MP, 3, 32>(y, ia, ca, sa, ssa, nhb, pp.nseg, zs, lane, 0); break;
-          }
-        }
-        if ((lane & (halves ? 15 : 31)) == 0) {
-#pragma unroll
-          for (int m = 0; m < MP; ++m)
-            if (m < M) pp.Y[(size_t)m * pp.d_out + o] = __float2half_rn(y[m] * pp.s_C);
-        }
+      const float yscale = pp.s_C;
+      const uint32_t part = sbase + prm.part_off + (uint32_t)(nb_done & 1) * (uint32_t)(2 * NL * MP * 4);
+      unsigned long long tw0 = 0;
+      if (tid == 0) asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(tw0));
+      bool ok = true;
+      int H = 0;
+      for (int i = i0; i < i1; ++i) {
+        const int j = nD + i;
+        ok = ok && mbar_wait_or_abort(full + j % R, (uint32_t)((j / R) & 1), s_abort, limit);
+        H += (int)((desc[i].w - desc[i].z) >> 3);
       }
-      __syncwarp();
-      if (lane == 0) mbar_arrive_cta(empty + s);
+      if (tid == 0) {
+        unsigned long long tw1;
+        asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(tw1));
+        s2_wait += tw1 - tw0;
+      }
+      ok = ok && !*s_abort;
+      const int hq = H / NL, hr = H - hq * NL;
+      const int g1 = split_begin(tid + 1, hq, hr);
+      int h = split_begin(tid, hq, hr), i = i0, P = 0;
+      if (ok && h < g1)
+        while (P + (int)((desc[i].w - desc[i].z) >> 3) <= h) P += (int)((desc[i].w - desc[i].z) >> 3), ++i;
+      int tail_o = -1, tail_he = 0;  // the column this thread's run ends inside (if it began in the run)
+      while (ok && h < g1) {  // the run's part in chunk i (threads step through their parts together)
+        const uint4 d = desc[i];
+        int to = -1, the = 0;
+        const int Hc = (int)((d.w - d.z) >> 3), hi = min(g1 - P, Hc);
+        const int s = (nD + i) % R;
+        const CChunk c = c_chunk_layout(d.x, d.y, d.z, d.w, (uint32_t)nseg, fmt);
+        const uint32_t slot = sbase + (uint32_t)s * kFusedSlotBytes;
+        switch (fmt) {  // uniform over the projection
+          case 0: stage2_run<MP, 0>(pp, d, c, slot, zs, h - P, hi, tid, part, M, yscale, &to, &the); break;
+          case 1: stage2_run<MP, 1>(pp, d, c, slot, zs, h - P, hi, tid, part, M, yscale, &to, &the); break;
+          case 2: stage2_run<MP, 2>(pp, d, c, slot, zs, h - P, hi, tid, part, M, yscale, &to, &the); break;
+          default: stage2_run<MP, 3>(pp, d, c, slot, zs, h - P, hi, tid, part, M, yscale, &to, &the); break;
+        }
+        if (to >= 0) {
+          tail_o = to;
+          tail_he = P + the;
+        }
+        h = P + hi;
+        P += Hc;
+        ++i;
+      }
+      named_bar_sync(1, NL);  // every share of the batch is in `part`
+      if (ok && tail_o >= 0 && !*s_abort) {  // TAIL + HEAD of each following thread that starts inside the column
+        float y[MP];
+        const uint32_t ta = part + (uint32_t)((2 * tid + 1) * MP) * 4u;
+#pragma unroll
+        for (int m = 0; m < MP; ++m) y[m] = lds_f32(ta + 4u * m);
+        for (int Lx = tid + 1; Lx < NL && split_begin(Lx, hq, hr) < tail_he; ++Lx) {
+          const uint32_t ha = part + (uint32_t)(2 * Lx * MP) * 4u;
+#pragma unroll
+          for (int m = 0; m < MP; ++m) y[m] += lds_f32(ha + 4u * m);
+        }
+#pragma unroll
+        for (int m = 0; m < MP; ++m)
+          if (m < M) pp.Y[(size_t)m * pp.d_out + tail_o] = __float2half_rn(y[m] * yscale);
+      }
+      for (i = i0; i < i1; ++i) {  // empty columns are zero; then release each chunk's slot
+        const uint4 d = desc[i];
+        const int s = (nD + i) % R;
+        if (ok && !*s_abort) {
+          const CChunk c = c_chunk_layout(d.x, d.y, d.z, d.w, (uint32_t)nseg, fmt);
+          const uint32_t cpa = sbase + (uint32_t)s * kFusedSlotBytes + c.cp_dst - c.cp_src;
+          for (int o = (int)d.x + tid; o < (int)d.y; o += NL)
+            if (lds_u32(cpa + 4u * (uint32_t)o) == lds_u32(cpa + 4u * (uint32_t)o + 4u))
+              for (int m = 0; m < M; ++m) pp.Y[(size_t)m * pp.d_out + o] = __float2half_rn(0.f);
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive_cta(empty + s);
+      }
+      i0 = i1;
+    }
+    if (tid == 0 && cta < kPhaseCtas) {
+      phase_mark(cta, 13);
+      g_phase[cta * kPhaseSlots + 12] = s2_wait;
+      g_phase[cta * kPhaseSlots + 14] = (unsigned long long)N2;
+      g_phase[cta * kPhaseSlots + 15] = (unsigned long long)nD;
     }
   }
   __syncthreads();
@@ -1057,7 +1225,9 @@ bool fused_plan_launch(int n, const dictproj_group* const* g, const dictproj_lay
     zall += zb;
     zone = std::max(zone, zb);
   }
-  auto total = [&](int R, int U) { return 1024 + R * kFusedSlotBytes + U + fused_ctl_bytes(R); };
+  const int part = 2 * 2 * kFWarps * 32 * mp * 4;  // stage-2 partial sums, two buffers
+  auto batch_of = [](int R) { return std::max(1, std::min(kMaxStage2Batch, R - 2)); };
+  auto total = [&](int R, int U) { return 1024 + R * kFusedSlotBytes + U + part + fused_ctl_bytes(R); };
   for (int pass = 0; pass < 2 && !pl.R; ++pass) {  // first: two CTAs per SM; then: one
     const int cap = pass == 0 ? kCoResidentSmem : smem_optin;
     const int rmin = pass == 0 ? 3 : 2;
@@ -1075,7 +1245,9 @@ bool fused_plan_launch(int n, const dictproj_group* const* g, const dictproj_lay
   }
   if (!pl.R) return false;
   pl.red_off = pl.R * kFusedSlotBytes + (pl.stage_x ? xtot : 0);
-  pl.bar_off = pl.R * kFusedSlotBytes + pl.U;
+  pl.part_off = pl.R * kFusedSlotBytes + pl.U;
+  pl.W = batch_of(pl.R);
+  pl.bar_off = pl.part_off + part;
   int zo = pl.R * kFusedSlotBytes;
   for (int i = 0; i < n; ++i) {
     pl.xoff[i] = pl.stage_x ? pl.R * kFusedSlotBytes + pl.xslot[i] * M * pl.xrow : -1;
@@ -1135,6 +1307,8 @@ cudaError_t launch_fused(int n, const dictproj_group* const* g, const dictproj_l
   prm.n_tp = pl.n_tp;
   prm.zt_resident = pl.zt_resident;
   prm.bar_off = pl.bar_off;
+  prm.part_off = pl.part_off;
+  prm.W = pl.W;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(G);
   cfg.blockDim = dim3(kFThreads);

@@ -47,7 +47,7 @@ cudaError_t take_decode_error(unsigned int* out);
 // through shared memory by TMA (fused.cu)
 constexpr int kFusedSlotBytes = 16384;  // one ring slot
 struct FusedLaunchPlan {
-  int mp, R, U, smem, zt_resident, stage_x, xrow, red_off, bar_off, n_tp;
+  int mp, R, U, smem, zt_resident, stage_x, xrow, red_off, bar_off, part_off, W, n_tp;
   int xoff[4], xfirst[4], xslot[4], zt_off[4];
 };
 cudaError_t prepare_fused_kernels(int device);
