@@ -433,6 +433,43 @@ def capture(torch, stream, fn):
     return g
 
 
+def stage_rooflines(torch, dp, stack, stream, M, peak, reps=20):
+    """Average launch time and HBM roofline of each stage kernel of the two-kernel
+    decode path: a graph of the dictionary stage for every projection of the
+    step (Z to a per-projection buffer), then one of the coefficient stage."""
+    mp = 1 if M <= 1 else 2 if M <= 2 else 4 if M <= 4 else 8
+    sh = stream.cuda_stream
+    projs = stack.w.projections
+    zs = [torch.zeros(p.k * mp, dtype=torch.float32, device="cuda") for p in projs]
+    xs, ys = [], []
+    for i, p in enumerate(projs):
+        xs.append(stack.x.data_ptr() + 2 * stack.x_off[(p.layer, p.site)][0])
+        ys.append(stack.y.data_ptr() + 2 * stack.y_off[i])
+    groups = [stack.groups[(p.group, p.ptype)] for p in projs]
+
+    def dict_all():
+        for i in range(len(projs)):
+            dp.dictproj_dictionary_stage(xs[i], M, groups[i], zs[i].data_ptr(), sh)
+
+    def coeff_all():
+        for i in range(len(projs)):
+            dp.dictproj_coefficient_stage(zs[i].data_ptr(), M, stack.layers[i], ys[i], sh)
+
+    out = {}
+    for name, fn, byte_idx in (("k_dict_decode", dict_all, 0), ("k_coeff_gather", coeff_all, 1)):
+        g = capture(torch, stream, fn)
+        time_replays(torch, stream, g, 3)
+        ms = time_replays(torch, stream, g, reps) / reps
+        del g
+        nbytes = sum(stage_bytes(p, M)[byte_idx] for p in projs)
+        per_launch_ms = ms / len(projs)
+        gbs = nbytes / len(projs) / (per_launch_ms / 1e3) / 1e9
+        out[name] = {"ms_per_step": round(ms, 4), "launches": len(projs), "avg_launch_us": round(per_launch_ms * 1e3, 3),
+                     "algorithmic_bytes_per_launch": int(nbytes / len(projs)), "GB/s": round(gbs, 1),
+                     "frac": round(gbs / peak, 4)}
+    return out
+
+
 def time_replays(torch, stream, graph, n, pre=None, post=None):
     a = torch.cuda.Event(enable_timing=True)
     b = torch.cuda.Event(enable_timing=True)
@@ -576,6 +613,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-prefill", action="store_true", help="skip the prefill (M = 128, 512, 2048) leg")
     ap.add_argument("--no-shapes", action="store_true", help="skip the per-projection-shape rows (M = 1, 8)")
+    ap.add_argument("--decode-kernels", choices=("auto", "fused", "split"), default="auto",
+                    help="decode kernels for M <= 8 calls (dictproj_set_decode_kernels); default: the library's choice")
     ap.add_argument("--no-batch", action="store_true",
                     help="one dictproj_forward per projection instead of batching q/k/v and gate/up")
     args = ap.parse_args()
@@ -608,6 +647,8 @@ def main():
     if dist:
         dist.barrier()
 
+    dp.dictproj_set_decode_kernels({"auto": dp.DECODE_AUTO, "fused": dp.DECODE_FUSED,
+                                    "split": dp.DECODE_SPLIT}[args.decode_kernels])
     wl = synth.full_step(n_layers=args.layers)
     M = 1
     stack = Stack(wl, M, torch, dp, log)
@@ -643,24 +684,34 @@ def main():
         ms_unbatched = time_replays(torch, stream, g_u, max(10, args.steps // 4)) / max(10, args.steps // 4)
         del g_u
 
-    # ---------------- roofline of the step's kernel, from the timed step itself
+    # ---------------- roofline of the dominant kernel
     launches_per_step = stack.launches_per_step(dp, batched=not args.no_batch)
     step_bytes = sum(d_bytes(p) + c_bytes(p) + 2 * M * (p.d_in + p.d_out) for p in wl.projections)
     peak, peak_kind = measured_peaks()
-    avg_launch_ms = ms_per_step / launches_per_step
-    bytes_per_launch = step_bytes / launches_per_step
+    peak_source = "measured (MEASURED_PEAKS.json hbm_gbs)" if peak_kind == "measured" else "fallback 6650 GB/s"
+    if launches_per_step == calls_per_step:  # every call is one fused launch: the step itself times it
+        avg_launch_ms = ms_per_step / launches_per_step
+        bytes_per_launch = step_bytes / launches_per_step
+        kernel, stages = "k_decode_fused", None
+        timing = ("the timed step itself: CUDA events on the launching stream around the replays of the step's "
+                  "graph; every launch is k_decode_fused, one per call")
+    else:  # two-kernel path: each stage's kernel timed in a graph of that stage's 224 launches alone
+        stages = stage_rooflines(torch, dp, stack, stream, M, peak)
+        dom = max(stages, key=lambda n: stages[n]["ms_per_step"])
+        avg_launch_ms = stages[dom]["avg_launch_us"] / 1e3
+        bytes_per_launch = stages[dom]["algorithmic_bytes_per_launch"]
+        kernel = dom
+        timing = ("CUDA events on the launching stream around replays of a graph holding only this kernel's "
+                  "launches for the step's 224 projections (one per projection, through the public stage entry "
+                  "points); the dominant kernel is the one with the larger share of the step")
     achieved = bytes_per_launch / (avg_launch_ms / 1e3) / 1e9
     roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
-                "frac": round(achieved / peak, 4), "traffic": profiled_traffic("k_decode_fused", bytes_per_launch),
-                "kernel": "k_decode_fused",
-                "peak_source": "measured (MEASURED_PEAKS.json hbm_gbs)" if peak_kind == "measured" else "fallback 6650 GB/s",
+                "frac": round(achieved / peak, 4), "traffic": profiled_traffic(kernel, bytes_per_launch),
+                "kernel": kernel, "peak_source": peak_source,
                 "avg_launch_us": round(avg_launch_ms * 1e3, 3), "algorithmic_bytes_per_launch": int(bytes_per_launch),
-                "launches_per_step": launches_per_step,
-                "timing": "the timed step itself: CUDA events on the launching stream around the replays of the "
-                          "step's graph; the average launch duration is the step time over its launches"
-                          + (" (every launch is k_decode_fused, one per call)" if launches_per_step == calls_per_step
-                             else f" ({launches_per_step} launches for {calls_per_step} calls: some calls ran the "
-                                  "two-kernel path)")}
+                "launches_per_step": launches_per_step, "timing": timing}
+    if stages:
+        roofline["stages"] = stages
 
     # ---------------- step-level accounting
     d_once = sum(d_bytes(p) for p in {(q.group, q.ptype): q for q in wl.projections}.values())
@@ -705,6 +756,8 @@ def main():
         "calls_per_step": calls_per_step,
         "batching": "q/k/v and gate/up share a call (dictproj_forward_batch)" if not args.no_batch
                     else "one dictproj_forward per projection",
+        "decode_kernels": {"auto": "library default (two-kernel path for NVFP4 layers)",
+                           "fused": "fused single kernel", "split": "two-kernel path"}[args.decode_kernels],
         "roofline": roofline,
         "cpu_baseline": cpu,
         "e2e": {"value": round(e2e_value, 2), "unit": "tokens/s", "h2d_bytes_per_step": h2d,

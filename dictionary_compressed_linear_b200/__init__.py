@@ -8,7 +8,10 @@ binding of that ABI; it loads the in-tree library and fails loudly if it is
 missing.
 """
 from .binding import (  # noqa: F401
-    PATH_AUTO, PATH_DECODE, PATH_PREFILL, DeviceGroup, DeviceLayer, DictprojError, Group, Layer, LIB_PATH,
+    PATH_AUTO, PATH_DECODE, PATH_PREFILL, DECODE_AUTO, DECODE_FUSED, DECODE_SPLIT, dictproj_set_decode_kernels,
+    dictproj_get_decode_kernels, IFMT, dictproj_layer_upload_bitmap, dictproj_pack_layer_bitmap,
+    dictproj_layer_upload_blocks, dictproj_pack_layer_blocks, dictproj_layer_index_format, dictproj_layer_export_bitmap,
+    dictproj_layer_export_blocks, DeviceGroup, DeviceLayer, DictprojError, Group, Layer, LIB_PATH,
     SIGNATURES, dictproj_forward_noalloc, dictproj_forward_noalloc_status, lib,
     dictproj_check, dictproj_check_status, dictproj_diag_phase_times, dictproj_launch_count, dictproj_selftest_wait_timeout, dictproj_coefficient_stage, dictproj_dictionary_stage, dictproj_dictionary_stage_prefill,
     dictproj_group_reserve_prefill, dictproj_forward, dictproj_rank_for_budget, dictproj_budget,

@@ -23,6 +23,8 @@ STATUS = {
     -10: "DICTPROJ_ERR_VALUE", -11: "DICTPROJ_ERR_IO",
 }
 PATH_AUTO, PATH_DECODE, PATH_PREFILL = 0, 1, 2
+DECODE_AUTO, DECODE_FUSED, DECODE_SPLIT = 0, 1, 2
+IFMT = {"u8": 0, "bitmap": 1, "blocks": 2}
 CFMT = {"nvfp4": 0, "fp16": 1, "fp8": 2, "int8": 3}  # DICTPROJ_CFMT_*
 
 
@@ -89,6 +91,25 @@ SIGNATURES = [
     ("dictproj_free_group", None, [C.c_void_p]),
     ("dictproj_free_layer", None, [C.c_void_p]),
     ("dictproj_forward", C.c_int, [C.c_void_p, C.c_int, C.c_void_p, C.c_void_p, C.c_void_p, C.c_void_p]),
+    ("dictproj_layer_upload_bitmap", C.c_int,
+     [C.POINTER(C.c_uint32), C.POINTER(C.c_uint8), C.POINTER(C.c_uint8), C.POINTER(C.c_uint32), C.c_float, C.c_int,
+      C.c_int, C.POINTER(C.c_void_p)]),
+    ("dictproj_pack_layer_bitmap", C.c_int,
+     [C.POINTER(C.c_int32), C.POINTER(C.c_int32), C.POINTER(C.c_float), C.c_int, C.c_int, C.POINTER(C.c_void_p)]),
+    ("dictproj_layer_upload_blocks", C.c_int,
+     [C.POINTER(C.c_uint32), C.POINTER(C.c_uint16), C.POINTER(C.c_uint8), C.POINTER(C.c_uint8), C.c_float, C.c_int,
+      C.c_int, C.POINTER(C.c_void_p)]),
+    ("dictproj_pack_layer_blocks", C.c_int,
+     [C.POINTER(C.c_int32), C.POINTER(C.c_int32), C.POINTER(C.c_float), C.c_int, C.c_int, C.POINTER(C.c_void_p)]),
+    ("dictproj_layer_index_format", C.c_int, [C.c_void_p, _intp]),
+    ("dictproj_layer_export_bitmap", C.c_int,
+     [C.c_void_p, C.POINTER(C.c_uint32), C.POINTER(C.c_uint8), C.POINTER(C.c_uint8), C.POINTER(C.c_uint32),
+      C.POINTER(C.c_float)]),
+    ("dictproj_layer_export_blocks", C.c_int,
+     [C.c_void_p, C.POINTER(C.c_uint32), C.POINTER(C.c_uint16), C.POINTER(C.c_uint8), C.POINTER(C.c_uint8),
+      C.POINTER(C.c_float)]),
+    ("dictproj_set_decode_kernels", C.c_int, [C.c_int]),
+    ("dictproj_get_decode_kernels", C.c_int, []),
     ("dictproj_forward_path", C.c_int,
      [C.c_void_p, C.c_int, C.c_void_p, C.c_void_p, C.c_void_p, C.c_void_p, C.c_int]),
     ("dictproj_forward_batch", C.c_int,
@@ -452,6 +473,88 @@ def dictproj_layer_export_fmt(layer: Layer) -> dict:
     return out
 
 
+def dictproj_layer_upload_bitmap(packed: dict) -> Layer:
+    """Upload a layer packed by dictproj_pack_layer_bitmap_host."""
+    h = C.c_void_p()
+    a = {n: np.ascontiguousarray(packed[n]) for n in ("col_ptr", "codes", "scales", "bitmap")}
+    _check(lib().dictproj_layer_upload_bitmap(_ptr(a["col_ptr"], C.c_uint32), _ptr(a["codes"], C.c_uint8),
+                                              _ptr(a["scales"], C.c_uint8), _ptr(a["bitmap"], C.c_uint32),
+                                              float(packed["s"]), packed["k"], packed["d_out"], C.byref(h)))
+    return Layer(h.value, packed["k"], packed["d_out"])
+
+
+def dictproj_pack_layer_bitmap(col_ptr, atom_idx, vals, k: int, d_out: int) -> Layer:
+    col_ptr = np.ascontiguousarray(col_ptr, dtype=np.int32)
+    atom_idx = np.ascontiguousarray(atom_idx, dtype=np.int32)
+    vals = np.ascontiguousarray(vals, dtype=np.float32)
+    h = C.c_void_p()
+    _check(lib().dictproj_pack_layer_bitmap(_ptr(col_ptr, C.c_int32), _ptr(atom_idx, C.c_int32),
+                                            _ptr(vals, C.c_float), k, d_out, C.byref(h)))
+    return Layer(h.value, k, d_out)
+
+
+def dictproj_layer_upload_blocks(packed: dict) -> Layer:
+    """Upload a layer packed by dictproj_pack_layer_blocks_host."""
+    h = C.c_void_p()
+    a = {n: np.ascontiguousarray(packed[n]) for n in ("blk_ptr", "blk_idx", "codes", "scales")}
+    blk_idx = a["blk_idx"] if a["blk_idx"].size else np.zeros(1, np.uint16)
+    codes = a["codes"] if a["codes"].size else np.zeros(8, np.uint8)
+    scales = a["scales"] if a["scales"].size else np.zeros(1, np.uint8)
+    _check(lib().dictproj_layer_upload_blocks(_ptr(a["blk_ptr"], C.c_uint32), _ptr(blk_idx, C.c_uint16),
+                                              _ptr(codes, C.c_uint8), _ptr(scales, C.c_uint8), float(packed["s"]),
+                                              packed["k"], packed["d_out"], C.byref(h)))
+    return Layer(h.value, packed["k"], packed["d_out"])
+
+
+def dictproj_pack_layer_blocks(col_ptr, atom_idx, vals, k: int, d_out: int) -> Layer:
+    col_ptr = np.ascontiguousarray(col_ptr, dtype=np.int32)
+    atom_idx = np.ascontiguousarray(atom_idx, dtype=np.int32)
+    vals = np.ascontiguousarray(vals, dtype=np.float32)
+    h = C.c_void_p()
+    _check(lib().dictproj_pack_layer_blocks(_ptr(col_ptr, C.c_int32), _ptr(atom_idx, C.c_int32),
+                                            _ptr(vals, C.c_float), k, d_out, C.byref(h)))
+    return Layer(h.value, k, d_out)
+
+
+def dictproj_layer_index_format(layer: Layer) -> str:
+    f = C.c_int()
+    _check(lib().dictproj_layer_index_format(layer.handle, C.byref(f)))
+    return {v: k for k, v in IFMT.items()}[f.value]
+
+
+def dictproj_layer_export_bitmap(layer: Layer) -> dict:
+    k, d_out = layer.k, layer.d_out
+    t = C.c_size_t()
+    _check(lib().dictproj_layer_info(layer.handle, None, None, C.byref(t), None))
+    words = -(-k // 32)
+    out = {"col_ptr": np.zeros(d_out + 1, np.uint32), "codes": np.zeros(t.value // 2, np.uint8),
+           "scales": np.zeros(t.value // 16, np.uint8), "bitmap": np.zeros(d_out * words, np.uint32)}
+    s = C.c_float()
+    _check(lib().dictproj_layer_export_bitmap(layer.handle, _ptr(out["col_ptr"], C.c_uint32),
+                                              _ptr(out["codes"], C.c_uint8), _ptr(out["scales"], C.c_uint8),
+                                              _ptr(out["bitmap"], C.c_uint32), C.byref(s)))
+    out.update(k=k, d_out=d_out, words=words, s=np.float32(s.value))
+    return out
+
+
+def dictproj_layer_export_blocks(layer: Layer) -> dict:
+    k, d_out = layer.k, layer.d_out
+    t = C.c_size_t()
+    _check(lib().dictproj_layer_info(layer.handle, None, None, C.byref(t), None))
+    nblk = t.value // 16
+    out = {"blk_ptr": np.zeros(d_out + 1, np.uint32), "blk_idx": np.zeros(max(nblk, 1), np.uint16),
+           "codes": np.zeros(max(nblk, 1) * 8, np.uint8), "scales": np.zeros(max(nblk, 1), np.uint8)}
+    s = C.c_float()
+    _check(lib().dictproj_layer_export_blocks(layer.handle, _ptr(out["blk_ptr"], C.c_uint32),
+                                              _ptr(out["blk_idx"], C.c_uint16), _ptr(out["codes"], C.c_uint8),
+                                              _ptr(out["scales"], C.c_uint8), C.byref(s)))
+    out["blk_idx"] = out["blk_idx"][:nblk]
+    out["codes"] = out["codes"][:nblk * 8]
+    out["scales"] = out["scales"][:nblk]
+    out.update(k=k, d_out=d_out, s=np.float32(s.value))
+    return out
+
+
 def dictproj_pack(D, max_tokens: int, layers) -> tuple:
     """layers: list of (col_ptr, atom_idx, vals, d_out). Returns (Group, [Layer])."""
     D = np.ascontiguousarray(D, dtype=np.float32)
@@ -509,6 +612,15 @@ def dictproj_layer_export(l: Layer) -> dict:
 def dictproj_forward(X_ptr: int, M: int, layer: Layer, group: Group, Y_ptr: int, stream: int = 0):
     _check(lib().dictproj_forward(C.c_void_p(X_ptr), M, layer.handle, group.handle, C.c_void_p(Y_ptr),
                                   C.c_void_p(stream)))
+
+
+def dictproj_set_decode_kernels(which: int) -> None:
+    """Process-wide choice of decode kernels: DECODE_AUTO, DECODE_FUSED or DECODE_SPLIT."""
+    _check(lib().dictproj_set_decode_kernels(which))
+
+
+def dictproj_get_decode_kernels() -> int:
+    return int(lib().dictproj_get_decode_kernels())
 
 
 def dictproj_forward_path(X_ptr: int, M: int, layer: Layer, group: Group, Y_ptr: int, stream: int = 0,

@@ -17,7 +17,7 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libdictproj.so")
 
-SOURCES = ["api.cu", "decode.cu", "fused.cu", "noalloc.cu", "prefill.cu", "pack.cpp", "packfile.cpp"]
+SOURCES = ["api.cu", "decode.cu", "fused.cu", "indexfmt.cu", "noalloc.cu", "prefill.cu", "pack.cpp", "packfile.cpp"]
 HEADERS = ["common.cuh", "dictproj_internal.h", "kernels.h"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 

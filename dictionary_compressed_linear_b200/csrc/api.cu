@@ -7,6 +7,7 @@
 #include <cstdio>
 #include <cstdlib>
 #include <cstring>
+#include <atomic>
 #include <mutex>
 #include <new>
 #include <vector>
@@ -51,6 +52,26 @@ static cudaError_t h2d(void* d, const void* h, size_t n) {
 }
 
 // One-time per-device set-up (kernel attributes) and capability check.
+static std::atomic<int> g_decode_kernels{DICTPROJ_DECODE_AUTO};
+
+// Whether a decode call goes to the fused kernel: FUSED always tries it; SPLIT
+// and AUTO never while the two-kernel path is the faster one on every LLaMA-7B
+// shape measured on B200 (chained calls, M = 1: 7.9 vs 13.8 us for 4096x2048x4096,
+// 13.3 vs 25.6 us for 4096x3072x11008, 12.5 vs 23.2 us for 11008x3072x4096); AUTO
+// still takes the fused kernel for calls the two-kernel path cannot serve
+// (non-NVFP4 coefficient values, or a Z table beyond its shared memory).
+static bool use_fused(int n, const dictproj_group* const* g, const dictproj_layer* const* l, const __half* const* x,
+                      int M, int dev, FusedLaunchPlan* fp) {
+  const int which = g_decode_kernels.load(std::memory_order_relaxed);
+  if (which == DICTPROJ_DECODE_SPLIT) return false;
+  if (which == DICTPROJ_DECODE_AUTO) {
+    bool split_ok = coeff_smem_fits(g[0]->k, decode_mp(M), dev);
+    for (int i = 0; i < n; ++i) split_ok = split_ok && l[i]->cfmt == DICTPROJ_CFMT_NVFP4 && coeff_smem_fits(g[i]->k, decode_mp(M), dev);
+    if (split_ok) return false;
+  }
+  return fused_plan_launch(n, g, l, x, M, smem_optin_of(dev), fp);
+}
+
 static std::mutex g_dev_mu;
 static std::vector<int> g_dev_ready;
 
@@ -69,6 +90,7 @@ int ensure_device(int* dev_out) {
     if ((e = prepare_decode_kernels(dev)) != cudaSuccess) return cuda_fail(e, "kernel set-up");
     if ((e = prepare_prefill_kernels(dev)) != cudaSuccess) return cuda_fail(e, "prefill kernel set-up");
     if ((e = prepare_fused_kernels(dev)) != cudaSuccess) return cuda_fail(e, "fused kernel set-up");
+    if ((e = prepare_index_kernels(dev)) != cudaSuccess) return cuda_fail(e, "index-format kernel set-up");
     g_dev_ready[dev] = 1;
   }
   *dev_out = dev;
@@ -190,6 +212,9 @@ void dictproj_free_layer(dictproj_layer* l) {
   cudaFree(l->seg_start);
   cudaFree(l->cplan_off);
   cudaFree(l->cplan);
+  cudaFree(l->bitmap);
+  cudaFree(l->blk_ptr);
+  cudaFree(l->blk_idx);
   delete l;
 }
 
@@ -555,6 +580,9 @@ int dictproj_layer_export(const dictproj_layer* l, uint32_t* pcol_ptr, uint8_t* 
     return fail(DICTPROJ_ERR_NULL, "layer_export: NULL pointer");
   if (l->cfmt != DICTPROJ_CFMT_NVFP4)
     return fail(DICTPROJ_ERR_UNSUPPORTED, "layer_export: the layer's values are not NVFP4; use dictproj_layer_export_fmt");
+  if (l->ifmt != DICTPROJ_IFMT_U8)
+    return fail(DICTPROJ_ERR_UNSUPPORTED, "layer_export: the layer has a bitmap or block index; use "
+                                          "dictproj_layer_export_bitmap / dictproj_layer_export_blocks");
   const size_t T = l->total;
   cudaError_t e;
   if ((e = cudaMemcpy(pcol_ptr, l->col_ptr, (l->d_out + 1) * sizeof(uint32_t), cudaMemcpyDeviceToHost)) ||
@@ -563,6 +591,222 @@ int dictproj_layer_export(const dictproj_layer* l, uint32_t* pcol_ptr, uint8_t* 
       (e = cudaMemcpy(idx, l->idx, T, cudaMemcpyDeviceToHost)) ||
       (e = cudaMemcpy(seg_start, l->seg_start, (size_t)l->d_out * l->nseg * sizeof(uint16_t), cudaMemcpyDeviceToHost)))
     return cuda_fail(e, "layer_export");
+  *s_C = l->s;
+  return DICTPROJ_OK;
+}
+
+// ---- bitmap and block-structured C_l ---------------------------------------------------
+// A layer struct with the common fields set and the index-format arrays empty.
+static int new_index_layer(int k, int d_out, float s_C, int ifmt, dictproj_layer** out) {
+  int dev, st;
+  if ((st = ensure_device(&dev))) return st;
+  dictproj_layer* l = new (std::nothrow) dictproj_layer();
+  if (!l) return fail(DICTPROJ_ERR_OOM, "layer upload: host allocation failed");
+  l->device = dev;
+  l->k = k;
+  l->d_out = d_out;
+  l->nseg = (k + 255) / 256;
+  l->s = s_C;
+  l->cfmt = DICTPROJ_CFMT_NVFP4;
+  l->ifmt = ifmt;
+  l->gather_ok = false;  // the gather and fused kernels read the u8 index only
+  l->fused_ok = false;
+  cudaError_t e;
+  int n_sm = 0;
+  if ((e = cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) {
+    delete l;
+    return cuda_fail(e, "layer upload: device attributes");
+  }
+  l->n_sm = n_sm;
+  *out = l;
+  return DICTPROJ_OK;
+}
+
+int dictproj_layer_upload_bitmap(const uint32_t* pcol_ptr, const uint8_t* codes, const uint8_t* scales,
+                                 const uint32_t* bitmap, float s_C, int k, int d_out, dictproj_layer** out) {
+  clear_error();
+  if (!pcol_ptr || !codes || !scales || !bitmap || !out) return fail(DICTPROJ_ERR_NULL, "layer_upload_bitmap: NULL pointer");
+  *out = nullptr;
+  if (k <= 0 || k % 16 || k > 65535 || d_out <= 0)
+    return fail(DICTPROJ_ERR_SHAPE, "layer_upload_bitmap: need 0 < k <= 65535, k %% 16 == 0, d_out > 0 (got k=%d d_out=%d)", k, d_out);
+  if (!(s_C > 0.0f) || !std::isfinite(s_C)) return fail(DICTPROJ_ERR_VALUE, "layer_upload_bitmap: s_C must be finite and > 0");
+  if (pcol_ptr[0] != 0) return fail(DICTPROJ_ERR_RANGE, "layer_upload_bitmap: col_ptr[0] must be 0");
+  const int words = (k + 31) / 32;
+  size_t nnz = 0;
+  for (int o = 0; o < d_out; ++o) {
+    const uint32_t n = pcol_ptr[o + 1] - pcol_ptr[o];
+    if (pcol_ptr[o + 1] < pcol_ptr[o] || n % 16 || n > (uint32_t)((k + 15) / 16 * 16))
+      return fail(DICTPROJ_ERR_RANGE, "layer_upload_bitmap: column %d has a bad padded length %u", o, n);
+    uint32_t bits = 0;
+    for (int w = 0; w < words; ++w) {
+      const uint32_t b = bitmap[(size_t)o * words + w];
+      if (32 * w + 32 > k && (b >> (k - 32 * w)) != 0u && k - 32 * w < 32)
+        return fail(DICTPROJ_ERR_RANGE, "layer_upload_bitmap: column %d marks atoms >= k", o);
+      bits += (uint32_t)__builtin_popcount(b);
+    }
+    // the set bits are the stored entries; the padded length leaves less than one block of padding
+    if (bits > n || n - bits >= 16)
+      return fail(DICTPROJ_ERR_RANGE, "layer_upload_bitmap: column %d has %u retained atoms for %u stored entries", o,
+                  bits, n);
+    nnz += bits;
+  }
+  int st;
+  dictproj_layer* l = nullptr;
+  if ((st = new_index_layer(k, d_out, s_C, DICTPROJ_IFMT_BITMAP, &l))) return st;
+  l->total = pcol_ptr[d_out];
+  l->nnz_total = nnz;
+  l->words = words;
+  const size_t T = l->total;
+  cudaError_t e;
+  if ((e = dmalloc((void**)&l->col_ptr, (d_out + 1) * sizeof(uint32_t) + 16)) ||
+      (e = dmalloc((void**)&l->codes, T / 2 + 16)) || (e = dmalloc((void**)&l->scales, T / 16 + 16)) ||
+      (e = dmalloc((void**)&l->bitmap, (size_t)d_out * words * sizeof(uint32_t) + 16))) {
+    dictproj_free_layer(l);
+    cudaGetLastError();
+    return fail(DICTPROJ_ERR_OOM, "layer_upload_bitmap: device allocation failed (%s)", cudaGetErrorName(e));
+  }
+  if ((e = h2d(l->col_ptr, pcol_ptr, (d_out + 1) * sizeof(uint32_t))) || (e = h2d(l->codes, codes, T / 2)) ||
+      (e = h2d(l->scales, scales, T / 16)) ||
+      (e = h2d(l->bitmap, bitmap, (size_t)d_out * words * sizeof(uint32_t)))) {
+    dictproj_free_layer(l);
+    cudaGetLastError();
+    return cuda_fail(e, "layer_upload_bitmap: copy to device");
+  }
+  *out = l;
+  return DICTPROJ_OK;
+}
+
+int dictproj_pack_layer_bitmap(const int32_t* col_ptr, const int32_t* atom_idx, const float* vals, int k, int d_out,
+                               dictproj_layer** out) {
+  clear_error();
+  if (!col_ptr || !out) return fail(DICTPROJ_ERR_NULL, "pack_layer_bitmap: NULL pointer");
+  *out = nullptr;
+  size_t total = 0;
+  int st = layer_packed_entries(col_ptr, k, d_out, &total);
+  if (st) return st;
+  const int words = (k + 31) / 32;
+  std::vector<uint32_t> pptr, nnz, bitmap;
+  std::vector<uint8_t> codes, scales;
+  try {
+    pptr.resize(d_out + 1);
+    nnz.resize(d_out);
+    bitmap.resize((size_t)d_out * words);
+    codes.resize(total / 2 + 1);
+    scales.resize(total / 16 + 1);
+  } catch (...) {
+    return fail(DICTPROJ_ERR_OOM, "pack_layer_bitmap: host allocation failed");
+  }
+  float s = 0.f;
+  if ((st = pack_layer_bitmap_host(col_ptr, atom_idx, vals, k, d_out, pptr.data(), nnz.data(), codes.data(),
+                                   scales.data(), bitmap.data(), &s)))
+    return st;
+  return dictproj_layer_upload_bitmap(pptr.data(), codes.data(), scales.data(), bitmap.data(), s, k, d_out, out);
+}
+
+int dictproj_layer_upload_blocks(const uint32_t* blk_ptr, const uint16_t* blk_idx, const uint8_t* codes,
+                                 const uint8_t* scales, float s_C, int k, int d_out, dictproj_layer** out) {
+  clear_error();
+  if (!blk_ptr || !blk_idx || !codes || !scales || !out) return fail(DICTPROJ_ERR_NULL, "layer_upload_blocks: NULL pointer");
+  *out = nullptr;
+  if (k <= 0 || k % 16 || k > 65535 || d_out <= 0)
+    return fail(DICTPROJ_ERR_SHAPE, "layer_upload_blocks: need 0 < k <= 65535, k %% 16 == 0, d_out > 0 (got k=%d d_out=%d)", k, d_out);
+  if (!(s_C > 0.0f) || !std::isfinite(s_C)) return fail(DICTPROJ_ERR_VALUE, "layer_upload_blocks: s_C must be finite and > 0");
+  if (blk_ptr[0] != 0) return fail(DICTPROJ_ERR_RANGE, "layer_upload_blocks: blk_ptr[0] must be 0");
+  const int nb_max = k / 16;
+  for (int o = 0; o < d_out; ++o) {
+    if (blk_ptr[o + 1] < blk_ptr[o] || blk_ptr[o + 1] - blk_ptr[o] > (uint32_t)nb_max)
+      return fail(DICTPROJ_ERR_RANGE, "layer_upload_blocks: column %d has a bad block count", o);
+    for (uint32_t b = blk_ptr[o]; b < blk_ptr[o + 1]; ++b)
+      if (blk_idx[b] >= nb_max || (b > blk_ptr[o] && blk_idx[b] <= blk_idx[b - 1]))
+        return fail(DICTPROJ_ERR_RANGE, "layer_upload_blocks: column %d block numbers not ascending below k/16", o);
+  }
+  int st;
+  dictproj_layer* l = nullptr;
+  if ((st = new_index_layer(k, d_out, s_C, DICTPROJ_IFMT_BLOCKS, &l))) return st;
+  const size_t nb = blk_ptr[d_out];
+  l->nblk = nb;
+  l->total = nb * 16;
+  l->nnz_total = nb * 16;
+  cudaError_t e;
+  if ((e = dmalloc((void**)&l->blk_ptr, (d_out + 1) * sizeof(uint32_t) + 16)) ||
+      (e = dmalloc((void**)&l->blk_idx, nb * sizeof(uint16_t) + 16)) || (e = dmalloc((void**)&l->codes, nb * 8 + 16)) ||
+      (e = dmalloc((void**)&l->scales, nb + 16))) {
+    dictproj_free_layer(l);
+    cudaGetLastError();
+    return fail(DICTPROJ_ERR_OOM, "layer_upload_blocks: device allocation failed (%s)", cudaGetErrorName(e));
+  }
+  if ((e = h2d(l->blk_ptr, blk_ptr, (d_out + 1) * sizeof(uint32_t))) ||
+      (e = h2d(l->blk_idx, blk_idx, nb * sizeof(uint16_t))) || (e = h2d(l->codes, codes, nb * 8)) ||
+      (e = h2d(l->scales, scales, nb))) {
+    dictproj_free_layer(l);
+    cudaGetLastError();
+    return cuda_fail(e, "layer_upload_blocks: copy to device");
+  }
+  *out = l;
+  return DICTPROJ_OK;
+}
+
+int dictproj_pack_layer_blocks(const int32_t* col_ptr, const int32_t* atom_idx, const float* vals, int k, int d_out,
+                               dictproj_layer** out) {
+  clear_error();
+  if (!col_ptr || !out) return fail(DICTPROJ_ERR_NULL, "pack_layer_blocks: NULL pointer");
+  *out = nullptr;
+  if (k <= 0 || k % 16 || d_out <= 0) return fail(DICTPROJ_ERR_SHAPE, "pack_layer_blocks: k must be a positive multiple of 16");
+  const size_t nz = (size_t)col_ptr[d_out];
+  std::vector<uint32_t> bptr;
+  std::vector<uint16_t> bidx;
+  std::vector<uint8_t> codes, scales;
+  try {
+    bptr.resize(d_out + 1);
+    bidx.resize(nz / 16 + 1);
+    codes.resize(nz / 2 + 1);
+    scales.resize(nz / 16 + 1);
+  } catch (...) {
+    return fail(DICTPROJ_ERR_OOM, "pack_layer_blocks: host allocation failed");
+  }
+  float s = 0.f;
+  int st;
+  if ((st = pack_layer_blocks_host(col_ptr, atom_idx, vals, k, d_out, bptr.data(), bidx.data(), codes.data(),
+                                   scales.data(), &s)))
+    return st;
+  return dictproj_layer_upload_blocks(bptr.data(), bidx.data(), codes.data(), scales.data(), s, k, d_out, out);
+}
+
+int dictproj_layer_index_format(const dictproj_layer* l, int* ifmt) {
+  clear_error();
+  if (!l || !ifmt) return fail(DICTPROJ_ERR_NULL, "layer_index_format: NULL pointer");
+  *ifmt = l->ifmt;
+  return DICTPROJ_OK;
+}
+
+int dictproj_layer_export_bitmap(const dictproj_layer* l, uint32_t* pcol_ptr, uint8_t* codes, uint8_t* scales,
+                                 uint32_t* bitmap, float* s_C) {
+  clear_error();
+  if (!l || !pcol_ptr || !codes || !scales || !bitmap || !s_C) return fail(DICTPROJ_ERR_NULL, "layer_export_bitmap: NULL pointer");
+  if (l->ifmt != DICTPROJ_IFMT_BITMAP) return fail(DICTPROJ_ERR_UNSUPPORTED, "layer_export_bitmap: not a bitmap layer");
+  const size_t T = l->total;
+  cudaError_t e;
+  if ((e = cudaMemcpy(pcol_ptr, l->col_ptr, (l->d_out + 1) * sizeof(uint32_t), cudaMemcpyDeviceToHost)) ||
+      (e = cudaMemcpy(codes, l->codes, T / 2, cudaMemcpyDeviceToHost)) ||
+      (e = cudaMemcpy(scales, l->scales, T / 16, cudaMemcpyDeviceToHost)) ||
+      (e = cudaMemcpy(bitmap, l->bitmap, (size_t)l->d_out * l->words * sizeof(uint32_t), cudaMemcpyDeviceToHost)))
+    return cuda_fail(e, "layer_export_bitmap");
+  *s_C = l->s;
+  return DICTPROJ_OK;
+}
+
+int dictproj_layer_export_blocks(const dictproj_layer* l, uint32_t* blk_ptr, uint16_t* blk_idx, uint8_t* codes,
+                                 uint8_t* scales, float* s_C) {
+  clear_error();
+  if (!l || !blk_ptr || !blk_idx || !codes || !scales || !s_C) return fail(DICTPROJ_ERR_NULL, "layer_export_blocks: NULL pointer");
+  if (l->ifmt != DICTPROJ_IFMT_BLOCKS) return fail(DICTPROJ_ERR_UNSUPPORTED, "layer_export_blocks: not a block layer");
+  const size_t nb = l->nblk;
+  cudaError_t e;
+  if ((e = cudaMemcpy(blk_ptr, l->blk_ptr, (l->d_out + 1) * sizeof(uint32_t), cudaMemcpyDeviceToHost)) ||
+      (nb && (e = cudaMemcpy(blk_idx, l->blk_idx, nb * sizeof(uint16_t), cudaMemcpyDeviceToHost))) ||
+      (nb && (e = cudaMemcpy(codes, l->codes, nb * 8, cudaMemcpyDeviceToHost))) ||
+      (nb && (e = cudaMemcpy(scales, l->scales, nb, cudaMemcpyDeviceToHost))))
+    return cuda_fail(e, "layer_export_blocks");
   *s_C = l->s;
   return DICTPROJ_OK;
 }
@@ -612,16 +856,23 @@ int dictproj_forward_path(const void* X, int M, const dictproj_layer* layer, con
   if (decode) {
     const int mp = decode_mp(M);
     FusedLaunchPlan fp;
-    if (fused_plan_launch(1, &group, &layer, &x, M, smem_optin_of(dev), &fp)) {
+    if (use_fused(1, &group, &layer, &x, M, dev, &fp)) {
       if ((e = launch_fused(1, &group, &layer, &x, &y, M, fp, kWaitLimitCycles, s)) != cudaSuccess)
         return cuda_fail(e, "forward: fused decode launch");
       return DICTPROJ_OK;
     }
+    if (g_decode_kernels.load(std::memory_order_relaxed) == DICTPROJ_DECODE_FUSED)
+      return fail(DICTPROJ_ERR_UNSUPPORTED, "forward: the fused decode kernel does not serve this call "
+                                            "(k > 8192 or its shared-memory plan does not fit)");
     if (layer->cfmt != DICTPROJ_CFMT_NVFP4)
       return fail(DICTPROJ_ERR_UNSUPPORTED,
                   "forward: FP16 / FP8 / INT8 coefficients are decoded by the fused kernel only (k <= 8192, Z "
                   "within shared memory); this call falls outside it");
-    if (!coeff_smem_fits(group->k, mp, dev))
+    if (layer->ifmt != DICTPROJ_IFMT_U8 && !index_smem_fits(group->k, mp, dev))
+      return fail(DICTPROJ_ERR_UNSUPPORTED,
+                  "forward: the bitmap / block decode stages k * %d floats of Z in shared memory; k=%d does not fit "
+                  "at M=%d", mp, group->k, M);
+    if (layer->ifmt == DICTPROJ_IFMT_U8 && !coeff_smem_fits(group->k, mp, dev))
       return fail(DICTPROJ_ERR_UNSUPPORTED,
                   "forward: the decode path stages (k + 256) * %d floats of Z in shared memory; k=%d does not fit "
                   "at M=%d", mp, group->k, M);
@@ -690,21 +941,25 @@ int dictproj_forward_batch(int n, const void* const* X, int M, const dictproj_la
       ys[i] = static_cast<__half*>(Y[i]);
     }
     FusedLaunchPlan fp;
-    if (fused_plan_launch(n, groups, layers, xs, M, smem_optin_of(dev), &fp)) {
+    if (use_fused(n, groups, layers, xs, M, dev, &fp)) {
       if ((e = launch_fused(n, groups, layers, xs, ys, M, fp, kWaitLimitCycles, s)) != cudaSuccess)
         return cuda_fail(e, "forward_batch: fused decode launch");
       return DICTPROJ_OK;
     }
+    if (g_decode_kernels.load(std::memory_order_relaxed) == DICTPROJ_DECODE_FUSED)
+      return fail(DICTPROJ_ERR_UNSUPPORTED, "forward_batch: the fused decode kernel does not serve this call "
+                                            "(k > 8192 or its shared-memory plan does not fit)");
   }
   for (int i = 0; i < n; ++i)
     if (layers[i]->cfmt != DICTPROJ_CFMT_NVFP4)
       return fail(DICTPROJ_ERR_UNSUPPORTED, "forward_batch: entry %d has FP16 / FP8 / INT8 coefficients, which only "
                   "the fused kernel decodes, and the batch falls outside it", i);
   for (int i = 0; i < n; ++i)
-    if (!coeff_smem_fits(groups[i]->k, mp, dev))
+    if (layers[i]->ifmt == DICTPROJ_IFMT_U8 ? !coeff_smem_fits(groups[i]->k, mp, dev)
+                                            : !index_smem_fits(groups[i]->k, mp, dev))
       return fail(DICTPROJ_ERR_UNSUPPORTED,
-                  "forward_batch: the decode path stages (k + 256) * %d floats of Z in shared memory; k=%d "
-                  "(entry %d) does not fit at M=%d", mp, groups[i]->k, i, M);
+                  "forward_batch: the decode path stages Z (k=%d atoms x %d floats) in shared memory; entry %d "
+                  "does not fit at M=%d", groups[i]->k, mp, i, M);
   DictPlan plans[kDecodeMaxBatch];
   const __half* xs[kDecodeMaxBatch];
   float* zs[kDecodeMaxBatch];
@@ -739,7 +994,7 @@ int dictproj_launch_count(int n, const void* const* X, int M, const dictproj_lay
   const __half* xs[kDecodeMaxBatch];
   for (int i = 0; i < n; ++i) xs[i] = static_cast<const __half*>(X[i]);
   FusedLaunchPlan fp;
-  if (fused_plan_launch(n, groups, layers, xs, M, smem_optin_of(groups[0]->device), &fp)) {
+  if (use_fused(n, groups, layers, xs, M, groups[0]->device, &fp)) {
     *count = 1;
     return DICTPROJ_OK;
   }
@@ -748,6 +1003,16 @@ int dictproj_launch_count(int n, const void* const* X, int M, const dictproj_lay
   *count = 1 + (all_gather ? 1 : n);
   return DICTPROJ_OK;
 }
+
+int dictproj_set_decode_kernels(int which) {
+  clear_error();
+  if (which < DICTPROJ_DECODE_AUTO || which > DICTPROJ_DECODE_SPLIT)
+    return fail(DICTPROJ_ERR_RANGE, "set_decode_kernels: unknown value %d", which);
+  g_decode_kernels.store(which, std::memory_order_relaxed);
+  return DICTPROJ_OK;
+}
+
+int dictproj_get_decode_kernels(void) { return g_decode_kernels.load(std::memory_order_relaxed); }
 
 int dictproj_forward(const void* X, int M, const dictproj_layer* layer, const dictproj_group* group, void* Y,
                      void* stream) {

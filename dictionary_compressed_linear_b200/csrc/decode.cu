@@ -745,7 +745,7 @@ static cudaError_t launch_gather_batch(int n, const dictproj_layer* const* l, co
 
 cudaError_t launch_coeff_decode_batch(int n, const dictproj_layer* const* l, const float* const* Zpart,
                                       const int* nslices, int M, int mp, __half* const* Y, cudaStream_t stream) {
-  bool all_gather = true;
+  bool all_gather = true;  // (bitmap and block layers have gather_ok false: one launch each)
   for (int i = 0; i < n; ++i) all_gather = all_gather && l[i]->gather_ok;
   if (all_gather) return launch_gather_batch(n, l, Zpart, nslices, M, mp, Y, stream);
   for (int i = 0; i < n; ++i) {
@@ -757,6 +757,7 @@ cudaError_t launch_coeff_decode_batch(int n, const dictproj_layer* const* l, con
 
 cudaError_t launch_coeff_decode(const dictproj_layer* l, const float* Zpart, int nslices, int M, int mp,
                                 __half* Y, cudaStream_t stream) {
+  if (l->ifmt != DICTPROJ_IFMT_U8) return launch_coeff_index(l, Zpart, nslices, M, mp, Y, stream);
   const uint8_t* codes = l->codes;
   const uint8_t* scales = l->scales;
   const uint8_t* idx = l->idx;

@@ -88,6 +88,12 @@ struct dictproj_layer {
   int n_sm;                // SMs of the device
   bool gather_ok;          // the gather kernel serves this layer (else the direct kernel)
   int cfmt;                // coefficient value format: NVFP4 (codes + scales) or FP16 / FP8 / INT8 (codes = values)
+  int ifmt;                // support index format (DICTPROJ_IFMT_*): u8 idx + seg_start, bitmap, or 16-atom blocks
+  uint32_t* bitmap;        // bitmap layers: [d_out][words] retained-atom masks
+  int words;               // 32-bit words per bitmap row, ceil(k/32)
+  uint32_t* blk_ptr;       // block layers: [d_out+1] kept blocks before each column
+  uint16_t* blk_idx;       // block layers: [nblk] block number (atom / 16), ascending per column
+  size_t nblk;             // block layers: kept blocks
   // fused decode kernel: column chunks of each of the n_sm positions
   bool fused_ok;
   uint32_t* cplan_off;     // [n_sm + 1]

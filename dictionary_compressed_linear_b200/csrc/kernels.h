@@ -51,6 +51,12 @@ struct FusedLaunchPlan {
   int xoff[4], xfirst[4], xslot[4], zt_off[4];
 };
 cudaError_t prepare_fused_kernels(int device);
+// Bitmap and block-structured C_l (indexfmt.cu)
+cudaError_t prepare_index_kernels(int device);
+bool index_smem_fits(int k, int mp, int device);
+cudaError_t launch_coeff_index(const dictproj_layer* l, const float* Zpart, int nslices, int M, int mp, __half* Y,
+                               cudaStream_t stream);
+cudaError_t launch_densify_index(const dictproj_layer* l, __half* Cd, cudaStream_t stream);
 // Tile-major dictionary copy (from the host's packed arrays), exchange buffer and
 // ticket of a group (sets g->fused_ok when the shape is served; allocation
 // failures are returned).

@@ -632,6 +632,7 @@ cudaError_t launch_dict_prefill(const dictproj_group* g, const __half* X, int M,
 }
 
 cudaError_t launch_densify_coeff(const dictproj_layer* l, __half* Cd, cudaStream_t stream) {
+  if (l->ifmt != DICTPROJ_IFMT_U8) return launch_densify_index(l, Cd, stream);
   const size_t per_warp = (size_t)l->k * 2 + (size_t)l->nseg * 2;
   const int warps = std::max(1, std::min(8, (int)((200 * 1024) / per_warp)));
   cudaLaunchConfig_t cfg = {};

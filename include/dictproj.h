@@ -137,6 +137,51 @@ int dictproj_pack_layer_blocks_host(const int32_t* col_ptr, const int32_t* atom_
                                     int k, int d_out, uint32_t* blk_ptr, uint16_t* blk_idx, uint8_t* codes,
                                     uint8_t* scales, float* s_C);
 
+/* Support index formats of a device layer (DICTPROJ_IFMT_*): the u8
+ * segment-relative index with seg_start (the default layout above), the bitmap
+ * of dictproj_pack_layer_bitmap_host, or the 16-atom blocks of
+ * dictproj_pack_layer_blocks_host. Bitmap and block layers hold NVFP4 values and
+ * are served by the two-kernel decode path (their own coefficient kernels; Z of
+ * k * mp floats in shared memory, mp = the power of two >= M) and by the
+ * prefill path (their own densify kernels, the same GEMM); the fused decode
+ * kernel, dictproj_layer_export and dictproj_layer_save take u8 layers only
+ * (UNSUPPORTED otherwise). */
+enum { DICTPROJ_IFMT_U8 = 0, DICTPROJ_IFMT_BITMAP = 1, DICTPROJ_IFMT_BLOCKS = 2 };
+
+/* Upload a bitmap C_l (the arrays of dictproj_pack_layer_bitmap_host) to the
+ * current device. Validation: k % 16 == 0, 0 < k <= 65535, d_out > 0; col_ptr[0]
+ * == 0, columns padded to multiples of 16 with less than 16 padding entries
+ * beyond their set bits; no bit at atoms >= k; s_C finite and > 0 (else SHAPE /
+ * RANGE / VALUE). Errors also NULL, OOM, CUDA. */
+int dictproj_layer_upload_bitmap(const uint32_t* pcol_ptr, const uint8_t* codes, const uint8_t* scales,
+                                 const uint32_t* bitmap, float s_C, int k, int d_out, dictproj_layer** out);
+/* dictproj_pack_layer_bitmap_host + dictproj_layer_upload_bitmap. */
+int dictproj_pack_layer_bitmap(const int32_t* col_ptr, const int32_t* atom_idx, const float* vals, int k,
+                               int d_out, dictproj_layer** out);
+
+/* Upload a block-structured C_l (the arrays of dictproj_pack_layer_blocks_host,
+ * nblk = blk_ptr[d_out]; codes nblk*8 bytes, scales nblk bytes). Validation:
+ * blk_ptr[0] == 0 and non-decreasing with at most k/16 blocks per column; block
+ * numbers ascending per column and below k/16 (RANGE); shape and s_C as
+ * dictproj_layer_upload_bitmap. */
+int dictproj_layer_upload_blocks(const uint32_t* blk_ptr, const uint16_t* blk_idx, const uint8_t* codes,
+                                 const uint8_t* scales, float s_C, int k, int d_out, dictproj_layer** out);
+/* dictproj_pack_layer_blocks_host + dictproj_layer_upload_blocks (VALUE / RANGE
+ * when a column's support is not a union of aligned 16-atom blocks). */
+int dictproj_pack_layer_blocks(const int32_t* col_ptr, const int32_t* atom_idx, const float* vals, int k,
+                               int d_out, dictproj_layer** out);
+
+/* The support index format of a layer (DICTPROJ_IFMT_*). Errors: NULL. */
+int dictproj_layer_index_format(const dictproj_layer* l, int* ifmt);
+
+/* Copy a bitmap / block layer's arrays back to host buffers of their packed
+ * sizes (bitmap: d_out * ceil(k/32) words). Errors: NULL, UNSUPPORTED (the other
+ * index format), CUDA. */
+int dictproj_layer_export_bitmap(const dictproj_layer* l, uint32_t* pcol_ptr, uint8_t* codes, uint8_t* scales,
+                                 uint32_t* bitmap, float* s_C);
+int dictproj_layer_export_blocks(const dictproj_layer* l, uint32_t* blk_ptr, uint16_t* blk_idx, uint8_t* codes,
+                                 uint8_t* scales, float* s_C);
+
 /* Coefficient value formats: NVFP4 (the default layout above) and the three
  * other coefficient formats of the paper's Table 4 (with an NVFP4 dictionary). */
 enum { DICTPROJ_CFMT_NVFP4 = 0, DICTPROJ_CFMT_FP16 = 1, DICTPROJ_CFMT_FP8 = 2, DICTPROJ_CFMT_INT8 = 3 };
@@ -281,6 +326,22 @@ int dictproj_forward_batch(int n, const void* const* X, int M, const dictproj_la
  * Host only; nothing is launched. Errors: NULL, RANGE. */
 int dictproj_launch_count(int n, const void* const* X, int M, const dictproj_layer* const* layers,
                           const dictproj_group* const* groups, int* count);
+
+/* Which kernels serve decode calls (M <= 8), process-wide (default AUTO):
+ *   DICTPROJ_DECODE_AUTO   the two-kernel path, which is the faster one on B200 for every
+ *                          LLaMA-7B shape measured, and the fused kernel for calls the
+ *                          two-kernel path cannot serve (FP16 / FP8 / INT8 coefficient
+ *                          values, or a Z table beyond its shared memory);
+ *   DICTPROJ_DECODE_FUSED  the single fused kernel only; a call it cannot serve (k > 8192,
+ *                          or its shared memory plan does not fit) fails with UNSUPPORTED;
+ *   DICTPROJ_DECODE_SPLIT  the two-kernel path only (dictionary stage, then coefficient
+ *                          stage); NVFP4 coefficients only, else UNSUPPORTED.
+ * Both compute the same function within the same tolerance (their fp32 summation
+ * orders differ). Set it between calls, not while another thread enqueues work.
+ * Errors: RANGE (unknown value). */
+enum { DICTPROJ_DECODE_AUTO = 0, DICTPROJ_DECODE_FUSED = 1, DICTPROJ_DECODE_SPLIT = 2 };
+int dictproj_set_decode_kernels(int which);
+int dictproj_get_decode_kernels(void);
 
 /* Forward with an explicit path: DICTPROJ_PATH_AUTO, DICTPROJ_PATH_DECODE (M <= 8)
  * or DICTPROJ_PATH_PREFILL (any M). Errors as dictproj_forward, plus

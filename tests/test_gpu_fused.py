@@ -1,8 +1,9 @@
 """The fused decode kernel (one kernel per call, weights staged through shared
 memory by TMA, one grid-wide exchange of partial Z) against the fp64 oracle.
 
-dictproj_forward and dictproj_forward_batch route every decode call (M <= 8)
-with k <= 8192 to it. These cases cover its edges: a reduction
+This module selects it for every decode call (dictproj_set_decode_kernels with
+DECODE_FUSED; the library's default sends NVFP4 projections to the faster
+two-kernel path). These cases cover its edges: a reduction
 length that leaves a partial 512-element piece (zero-filled out of bounds), a
 single 16-atom tile, 32 segments of 256 atoms, fewer output columns than SMs
 (CTAs without columns), empty / full / one-atom columns, columns that straddle
@@ -24,6 +25,13 @@ if not torch.cuda.is_available():  # pragma: no cover - CPU container
 import dictionary_compressed_linear_b200 as dp  # noqa: E402
 from gpu_helpers import (assert_parity, device_projection, oracle_forward,  # noqa: E402
                          oracle_projection, run_forward)
+
+
+@pytest.fixture(autouse=True, scope="module")
+def _fused_kernel():
+    dp.dictproj_set_decode_kernels(dp.DECODE_FUSED)
+    yield
+    dp.dictproj_set_decode_kernels(dp.DECODE_AUTO)
 
 
 def _case(seed, d_in, k, d_out, rho):
@@ -165,3 +173,17 @@ def test_fused_long_chain_in_a_graph_is_exact_and_repeatable():
         x = (fresh[i // 2] if i % 2 == 0 else ref[i - 1]).cpu().numpy()
         assert_parity(ref[i].float().cpu().numpy().astype(np.float64), oracle_forward(x, pd, pcs[i % 2]), f"call {i}")
     assert dp.dictproj_check_status(s.cuda_stream) == 0
+
+
+def test_decode_kernel_choice_sets_the_launch_count():
+    D, C = _case(9, 1024, 512, 300, 0.3)
+    g, l = device_projection(D, C, max_tokens=8)
+    X = torch.zeros((1, 1024), dtype=torch.float16, device="cuda")
+    assert dp.dictproj_launch_count([X.data_ptr()], 1, [l], [g]) == 1  # this module: fused
+    dp.dictproj_set_decode_kernels(dp.DECODE_SPLIT)
+    try:
+        assert dp.dictproj_launch_count([X.data_ptr()], 1, [l], [g]) == 2
+        dp.dictproj_set_decode_kernels(dp.DECODE_AUTO)
+        assert dp.dictproj_launch_count([X.data_ptr()], 1, [l], [g]) == 2  # NVFP4: the two-kernel path
+    finally:
+        dp.dictproj_set_decode_kernels(dp.DECODE_FUSED)

@@ -251,3 +251,44 @@ def test_block_layer_packer_rejects_unaligned_supports(dp):
     with pytest.raises(DictprojError) as e:
         dp.dictproj_pack_layer_blocks_host(np.array([0, 8]), np.arange(8), np.ones(8), 32, 1)
     assert e.value.status == -5
+
+
+def test_decode_kernel_choice_is_validated_and_kept(dp):
+    assert dp.dictproj_get_decode_kernels() == dp.DECODE_AUTO
+    for which in (dp.DECODE_FUSED, dp.DECODE_SPLIT, dp.DECODE_AUTO):
+        dp.dictproj_set_decode_kernels(which)
+        assert dp.dictproj_get_decode_kernels() == which
+    for bad in (-1, 3):
+        with pytest.raises(dp.DictprojError) as err:
+            dp.dictproj_set_decode_kernels(bad)
+        assert err.value.status == -5
+    assert dp.dictproj_get_decode_kernels() == dp.DECODE_AUTO
+
+
+def test_index_format_uploads_validate_before_touching_a_device(dp):
+    """Bitmap and block uploads check their arrays first (no device is needed to
+    be refused)."""
+    import numpy as np
+    k, d_out = 48, 2
+    good = {"col_ptr": np.array([0, 16, 32], np.uint32), "codes": np.zeros(16, np.uint8),
+            "scales": np.zeros(2, np.uint8), "bitmap": np.array([0xF, 0, 0x1, 0], np.uint32),
+            "s": np.float32(1.0), "k": k, "d_out": d_out}
+    bad_bit = dict(good, bitmap=np.array([0xF, 1 << 20, 0x1, 0], np.uint32))  # atom 52 >= k
+    too_many = dict(good, bitmap=np.array([0xFFFFFFFF, 0, 0x1, 0], np.uint32))  # 32 bits for 16 entries
+    for packed, status in ((bad_bit, -5), (too_many, -5), (dict(good, s=np.float32(0.0)), -10)):
+        with pytest.raises(dp.DictprojError) as err:
+            dp.dictproj_layer_upload_bitmap(packed)
+        assert err.value.status == status
+    blocks = {"blk_ptr": np.array([0, 2, 3], np.uint32), "blk_idx": np.array([2, 1, 0], np.uint16),
+              "codes": np.zeros(24, np.uint8), "scales": np.zeros(3, np.uint8), "s": np.float32(1.0), "k": k,
+              "d_out": d_out}
+    with pytest.raises(dp.DictprojError) as err:  # column 0's blocks not ascending
+        dp.dictproj_layer_upload_blocks(blocks)
+    assert err.value.status == -5
+    with pytest.raises(dp.DictprojError) as err:  # block 3 of a k = 48 layer
+        dp.dictproj_layer_upload_blocks(dict(blocks, blk_idx=np.array([0, 1, 3], np.uint16)))
+    assert err.value.status == -5
+    with pytest.raises(dp.DictprojError) as err:  # not a union of aligned 16-atom blocks
+        dp.dictproj_pack_layer_blocks(np.array([0, 3], np.int32), np.array([0, 1, 2], np.int32),
+                                      np.ones(3, np.float32), 48, 1)
+    assert err.value.status < 0
