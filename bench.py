@@ -433,39 +433,34 @@ def capture(torch, stream, fn):
     return g
 
 
-def stage_rooflines(torch, dp, stack, stream, M, peak, reps=20):
+def stage_rooflines(torch, dp, stack, stream, M, peak, batched=True, reps=20):
     """Average launch time and HBM roofline of each stage kernel of the two-kernel
-    decode path: a graph of the dictionary stage for every projection of the
-    step (Z to a per-projection buffer), then one of the coefficient stage."""
-    mp = 1 if M <= 1 else 2 if M <= 2 else 4 if M <= 4 else 8
+    decode path in the step's own launch configuration: the step's calls (the same
+    batches, grids and Z scratch, through dictproj_forward_batch_stages) captured
+    twice, once launching only the dictionary kernels and once only the coefficient
+    kernels (which then read the Z the last full step left: the same work)."""
     sh = stream.cuda_stream
     projs = stack.w.projections
-    zs = [torch.zeros(p.k * mp, dtype=torch.float32, device="cuda") for p in projs]
-    xs, ys = [], []
-    for i, p in enumerate(projs):
-        xs.append(stack.x.data_ptr() + 2 * stack.x_off[(p.layer, p.site)][0])
-        ys.append(stack.y.data_ptr() + 2 * stack.y_off[i])
-    groups = [stack.groups[(p.group, p.ptype)] for p in projs]
+    calls = stack.calls(batched)
 
-    def dict_all():
-        for i in range(len(projs)):
-            dp.dictproj_dictionary_stage(xs[i], M, groups[i], zs[i].data_ptr(), sh)
-
-    def coeff_all():
-        for i in range(len(projs)):
-            dp.dictproj_coefficient_stage(zs[i].data_ptr(), M, stack.layers[i], ys[i], sh)
+    def stage_only(mask):
+        def fn():
+            for xs, ls, gs, ys in calls:
+                dp.dictproj_forward_batch_stages(xs, M, ls, gs, ys, sh, mask)
+        return fn
 
     out = {}
-    for name, fn, byte_idx in (("k_dict_decode", dict_all, 0), ("k_coeff_gather", coeff_all, 1)):
-        g = capture(torch, stream, fn)
+    for name, mask, byte_idx in (("k_dict_decode", 1, 0), ("k_coeff_gather", 2, 1)):
+        g = capture(torch, stream, stage_only(mask))
         time_replays(torch, stream, g, 3)
         ms = time_replays(torch, stream, g, reps) / reps
         del g
         nbytes = sum(stage_bytes(p, M)[byte_idx] for p in projs)
-        per_launch_ms = ms / len(projs)
-        gbs = nbytes / len(projs) / (per_launch_ms / 1e3) / 1e9
-        out[name] = {"ms_per_step": round(ms, 4), "launches": len(projs), "avg_launch_us": round(per_launch_ms * 1e3, 3),
-                     "algorithmic_bytes_per_launch": int(nbytes / len(projs)), "GB/s": round(gbs, 1),
+        per_launch_ms = ms / len(calls)
+        gbs = nbytes / (ms / 1e3) / 1e9
+        out[name] = {"ms_per_step": round(ms, 4), "launches": len(calls), "projections": len(projs),
+                     "avg_launch_us": round(per_launch_ms * 1e3, 3),
+                     "algorithmic_bytes_per_launch": int(nbytes / len(calls)), "GB/s": round(gbs, 1),
                      "frac": round(gbs / peak, 4)}
     return out
 
@@ -695,15 +690,15 @@ def main():
         kernel, stages = "k_decode_fused", None
         timing = ("the timed step itself: CUDA events on the launching stream around the replays of the step's "
                   "graph; every launch is k_decode_fused, one per call")
-    else:  # two-kernel path: each stage's kernel timed in a graph of that stage's 224 launches alone
-        stages = stage_rooflines(torch, dp, stack, stream, M, peak)
+    else:  # two-kernel path: each stage's kernel timed in a graph of that stage's launches of the step alone
+        stages = stage_rooflines(torch, dp, stack, stream, M, peak, batched=not args.no_batch)
         dom = max(stages, key=lambda n: stages[n]["ms_per_step"])
         avg_launch_ms = stages[dom]["avg_launch_us"] / 1e3
         bytes_per_launch = stages[dom]["algorithmic_bytes_per_launch"]
         kernel = dom
-        timing = ("CUDA events on the launching stream around replays of a graph holding only this kernel's "
-                  "launches for the step's 224 projections (one per projection, through the public stage entry "
-                  "points); the dominant kernel is the one with the larger share of the step")
+        timing = ("CUDA events on the launching stream around replays of a graph of the step's own calls "
+                  "(same batches, grids and Z scratch) that launches only this kernel "
+                  "(dictproj_forward_batch_stages); the dominant kernel is the one with the larger share of the step")
     achieved = bytes_per_launch / (avg_launch_ms / 1e3) / 1e9
     roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                 "frac": round(achieved / peak, 4), "traffic": profiled_traffic(kernel, bytes_per_launch),

@@ -16,7 +16,7 @@ from .binding import (  # noqa: F401
     dictproj_check, dictproj_check_status, dictproj_diag_phase_times, dictproj_launch_count, dictproj_selftest_wait_timeout, dictproj_coefficient_stage, dictproj_dictionary_stage, dictproj_dictionary_stage_prefill,
     dictproj_group_reserve_prefill, dictproj_forward, dictproj_rank_for_budget, dictproj_budget,
     dictproj_group_file_write, dictproj_group_file_read, dictproj_layer_file_write, dictproj_layer_file_read,
-    dictproj_group_save, dictproj_group_load, dictproj_layer_save, dictproj_layer_load, dictproj_forward_batch, dictproj_forward_path, dictproj_forward_status,
+    dictproj_group_save, dictproj_group_load, dictproj_layer_save, dictproj_layer_load, dictproj_forward_batch, dictproj_forward_batch_stages, dictproj_decode_batch_plan, dictproj_forward_path, dictproj_forward_status,
     dictproj_group_export, dictproj_group_info, dictproj_group_packed_sizes, dictproj_group_upload,
     dictproj_last_error, dictproj_layer_export, dictproj_layer_info, dictproj_layer_packed_entries,
     dictproj_layer_upload, dictproj_pack, dictproj_pack_group, dictproj_pack_group_host,

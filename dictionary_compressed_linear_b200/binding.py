@@ -115,6 +115,11 @@ SIGNATURES = [
     ("dictproj_forward_batch", C.c_int,
      [C.c_int, C.POINTER(C.c_void_p), C.c_int, C.POINTER(C.c_void_p), C.POINTER(C.c_void_p),
       C.POINTER(C.c_void_p), C.c_void_p]),
+    ("dictproj_forward_batch_stages", C.c_int,
+     [C.c_int, C.POINTER(C.c_void_p), C.c_int, C.POINTER(C.c_void_p), C.POINTER(C.c_void_p),
+      C.POINTER(C.c_void_p), C.c_void_p, C.c_int]),
+    ("dictproj_decode_batch_plan", C.c_int,
+     [C.c_int, _intp, _intp, _intp, C.POINTER(C.c_longlong), C.c_int, C.c_int, _intp, _intp, _intp]),
     ("dictproj_launch_count", C.c_int,
      [C.c_int, C.POINTER(C.c_void_p), C.c_int, C.POINTER(C.c_void_p), C.POINTER(C.c_void_p), _intp]),
     ("dictproj_dictionary_stage", C.c_int, [C.c_void_p, C.c_int, C.c_void_p, C.c_void_p, C.c_void_p]),
@@ -641,6 +646,28 @@ def dictproj_forward_batch(X_ptrs, M: int, layers, groups, Y_ptrs, stream: int =
     arr = lambda vals: (C.c_void_p * n)(*[C.c_void_p(v) for v in vals])
     _check(lib().dictproj_forward_batch(n, arr(X_ptrs), M, arr([l.handle for l in layers]),
                                         arr([g.handle for g in groups]), arr(Y_ptrs), C.c_void_p(stream)))
+
+
+def dictproj_forward_batch_stages(X_ptrs, M: int, layers, groups, Y_ptrs, stream: int = 0, stages: int = 3):
+    """dictproj_forward_batch launching only the stage kernels in the mask
+    (1 dictionary, 2 coefficient, 3 both) of the two-kernel decode path."""
+    n = len(layers)
+    arr = lambda vals: (C.c_void_p * n)(*[C.c_void_p(v) for v in vals])
+    _check(lib().dictproj_forward_batch_stages(n, arr(X_ptrs), M, arr([l.handle for l in layers]),
+                                               arr([g.handle for g in groups]), arr(Y_ptrs), C.c_void_p(stream),
+                                               stages))
+
+
+def dictproj_decode_batch_plan(shapes, M: int, n_sm: int):
+    """Grid of a batched two-kernel decode call, host only. shapes: list of
+    (d_in, k, d_out, stored entries). Returns a list of dicts with dict_ctas,
+    dict_slices and coeff_ctas per projection."""
+    n = len(shapes)
+    ints = lambda j: (C.c_int * n)(*[int(sh[j]) for sh in shapes])
+    ent = (C.c_longlong * n)(*[int(sh[3]) for sh in shapes])
+    dc, ds, cc = (C.c_int * n)(), (C.c_int * n)(), (C.c_int * n)()
+    _check(lib().dictproj_decode_batch_plan(n, ints(0), ints(1), ints(2), ent, M, n_sm, dc, ds, cc))
+    return [{"dict_ctas": dc[i], "dict_slices": ds[i], "coeff_ctas": cc[i]} for i in range(n)]
 
 
 def dictproj_group_save(group: "Group", path: str):

@@ -195,7 +195,6 @@ void dictproj_free_group(dictproj_group* g) {
   cudaFree(g->z32);
   cudaFree(g->z16);
   cudaFree(g->cdense);
-  cudaFree(g->err);
   cudaFree(g->fcodes);
   cudaFree(g->fscales);
   cudaFree(g->zx);
@@ -247,14 +246,13 @@ int dictproj_group_upload(const uint8_t* codes, const uint8_t* scales, float s_D
   const size_t zbytes = (size_t)g->zslices * k * kDecodeMaxTokens * sizeof(float);
   const size_t z16bytes = (size_t)max_tokens * k * sizeof(uint16_t);
   if ((e = dmalloc((void**)&g->codes, g->codes_bytes)) || (e = dmalloc((void**)&g->scales, g->scales_bytes)) ||
-      (e = dmalloc((void**)&g->z32, zbytes)) || (e = dmalloc((void**)&g->z16, z16bytes)) ||
-      (e = dmalloc((void**)&g->err, 16))) {
+      (e = dmalloc((void**)&g->z32, zbytes)) || (e = dmalloc((void**)&g->z16, z16bytes))) {
     dictproj_free_group(g);
     cudaGetLastError();
     return fail(DICTPROJ_ERR_OOM, "group_upload: device allocation failed (%s)", cudaGetErrorName(e));
   }
   if ((e = h2d(g->codes, codes, g->codes_bytes)) || (e = h2d(g->scales, scales, g->scales_bytes)) ||
-      (e = cudaMemset(g->err, 0, 16)) || (e = cudaMemset(g->z32, 0, zbytes))) {
+      (e = cudaMemset(g->z32, 0, zbytes))) {
     dictproj_free_group(g);
     cudaGetLastError();
     return cuda_fail(e, "group_upload: copy to device");
@@ -830,6 +828,26 @@ int dictproj_layer_info(const dictproj_layer* l, int* k, int* d_out, size_t* tot
   return DICTPROJ_OK;
 }
 
+// The two-kernel decode path of one call (stages: bit 0 the dictionary kernel,
+// bit 1 the coefficient kernel).
+static int launch_split_decode(int n, const dictproj_group* const* groups, const dictproj_layer* const* layers,
+                               const __half* const* xs, float* const* zs, const DictPlan* plans, int M, int mp,
+                               __half* const* ys, cudaStream_t s, int stages, const char* who) {
+  int ns[kDecodeMaxBatch];
+  for (int i = 0; i < n; ++i) ns[i] = plans[i].slices;
+  cudaError_t e;
+  char what[96];
+  if ((stages & 1) && (e = launch_dict_decode_batch(n, groups, xs, M, mp, zs, plans, s)) != cudaSuccess) {
+    std::snprintf(what, sizeof what, "%s: dictionary stage launch", who);
+    return cuda_fail(e, what);
+  }
+  if ((stages & 2) && (e = launch_coeff_decode_batch(n, layers, zs, ns, M, mp, ys, s)) != cudaSuccess) {
+    std::snprintf(what, sizeof what, "%s: coefficient stage launch", who);
+    return cuda_fail(e, what);
+  }
+  return DICTPROJ_OK;
+}
+
 int dictproj_forward_path(const void* X, int M, const dictproj_layer* layer, const dictproj_group* group,
                           void* Y, void* stream, int path) {
   clear_error();
@@ -876,11 +894,8 @@ int dictproj_forward_path(const void* X, int M, const dictproj_layer* layer, con
       return fail(DICTPROJ_ERR_UNSUPPORTED,
                   "forward: the decode path stages (k + 256) * %d floats of Z in shared memory; k=%d does not fit "
                   "at M=%d", mp, group->k, M);
-    if ((e = launch_dict_decode(group, x, M, mp, group->z32, plan, s)) != cudaSuccess)
-      return cuda_fail(e, "forward: dictionary stage launch");
-    if ((e = launch_coeff_decode(layer, group->z32, plan.slices, M, mp, y, s)) != cudaSuccess)
-      return cuda_fail(e, "forward: coefficient stage launch");
-    return DICTPROJ_OK;
+    float* z = group->z32;
+    return launch_split_decode(1, &group, &layer, &x, &z, &plan, M, mp, &y, s, 3, "forward");
   }
   // Prefill: Z = s_D X D^ (fp16) and Y = s_C Z C^ as tensor-core GEMMs, C^ densified first.
   if (layer->d_out > group->cdense_cols)
@@ -899,9 +914,13 @@ int dictproj_forward_path(const void* X, int M, const dictproj_layer* layer, con
   return DICTPROJ_OK;
 }
 
-int dictproj_forward_batch(int n, const void* const* X, int M, const dictproj_layer* const* layers,
-                           const dictproj_group* const* groups, void* const* Y, void* stream) {
+// stages: bit 0 the dictionary kernel, bit 1 the coefficient kernel of the
+// two-kernel decode path (3 = the whole forward, which is the only mask the
+// fused kernel and the prefill path take).
+static int forward_batch_impl(int n, const void* const* X, int M, const dictproj_layer* const* layers,
+                              const dictproj_group* const* groups, void* const* Y, void* stream, int stages) {
   clear_error();
+  if (stages < 1 || stages > 3) return fail(DICTPROJ_ERR_RANGE, "forward_batch_stages: stage mask %d not 1, 2 or 3", stages);
   if (!X || !layers || !groups || !Y) return fail(DICTPROJ_ERR_NULL, "forward_batch: NULL array");
   if (n < 1 || n > DICTPROJ_MAX_BATCH)
     return fail(DICTPROJ_ERR_RANGE, "forward_batch: n=%d outside [1, %d]", n, DICTPROJ_MAX_BATCH);
@@ -925,6 +944,7 @@ int dictproj_forward_batch(int n, const void* const* X, int M, const dictproj_la
   if (dev != groups[0]->device)
     return fail(DICTPROJ_ERR_MISMATCH, "forward_batch: current device %d, handles on device %d", dev, groups[0]->device);
   if (M > kDecodeMaxTokens) {  // prefill: one projection after another
+    if (stages != 3) return fail(DICTPROJ_ERR_UNSUPPORTED, "forward_batch_stages: a stage mask needs M <= %d", kDecodeMaxTokens);
     for (int i = 0; i < n; ++i) {
       const int st = dictproj_forward_path(X[i], M, layers[i], groups[i], Y[i], stream, DICTPROJ_PATH_AUTO);
       if (st) return st;
@@ -942,6 +962,8 @@ int dictproj_forward_batch(int n, const void* const* X, int M, const dictproj_la
     }
     FusedLaunchPlan fp;
     if (use_fused(n, groups, layers, xs, M, dev, &fp)) {
+      if (stages != 3)
+        return fail(DICTPROJ_ERR_UNSUPPORTED, "forward_batch_stages: the fused decode kernel serves this call; it has one stage");
       if ((e = launch_fused(n, groups, layers, xs, ys, M, fp, kWaitLimitCycles, s)) != cudaSuccess)
         return cuda_fail(e, "forward_batch: fused decode launch");
       return DICTPROJ_OK;
@@ -963,19 +985,57 @@ int dictproj_forward_batch(int n, const void* const* X, int M, const dictproj_la
   DictPlan plans[kDecodeMaxBatch];
   const __half* xs[kDecodeMaxBatch];
   float* zs[kDecodeMaxBatch];
-  int ns[kDecodeMaxBatch];
   __half* ys[kDecodeMaxBatch];
+  int din[kDecodeMaxBatch], kk[kDecodeMaxBatch];
+  for (int i = 0; i < n; ++i) din[i] = groups[i]->d_in, kk[i] = groups[i]->k;
+  dict_plan_batch(n, din, kk, groups[0]->n_sm, M, plans);
   for (int i = 0; i < n; ++i) {
-    plans[i] = dict_plan(groups[i]->d_in, groups[i]->k, groups[i]->n_sm, M, false);
+    if (plans[i].slices > groups[i]->zslices)  // cannot happen: a common J is never below the lone plan's
+      return fail(DICTPROJ_ERR_UNSUPPORTED, "forward_batch: plan needs %d Z slices, entry %d holds %d",
+                  plans[i].slices, i, groups[i]->zslices);
     xs[i] = static_cast<const __half*>(X[i]);
     zs[i] = groups[i]->z32;
-    ns[i] = plans[i].slices;
     ys[i] = static_cast<__half*>(Y[i]);
   }
-  if ((e = launch_dict_decode_batch(n, groups, xs, M, mp, zs, plans, s)) != cudaSuccess)
-    return cuda_fail(e, "forward_batch: dictionary stage launch");
-  if ((e = launch_coeff_decode_batch(n, layers, zs, ns, M, mp, ys, s)) != cudaSuccess)
-    return cuda_fail(e, "forward_batch: coefficient stage launch");
+  return launch_split_decode(n, groups, layers, xs, zs, plans, M, mp, ys, s, stages, "forward_batch");
+}
+
+int dictproj_forward_batch(int n, const void* const* X, int M, const dictproj_layer* const* layers,
+                           const dictproj_group* const* groups, void* const* Y, void* stream) {
+  return forward_batch_impl(n, X, M, layers, groups, Y, stream, 3);
+}
+
+int dictproj_forward_batch_stages(int n, const void* const* X, int M, const dictproj_layer* const* layers,
+                                  const dictproj_group* const* groups, void* const* Y, void* stream, int stages) {
+  return forward_batch_impl(n, X, M, layers, groups, Y, stream, stages);
+}
+
+int dictproj_decode_batch_plan(int n, const int* d_in, const int* k, const int* d_out, const long long* entries,
+                               int M, int n_sm, int* dict_ctas, int* dict_slices, int* coeff_ctas) {
+  clear_error();
+  if (!d_in || !k || !d_out || !entries || !dict_ctas || !dict_slices || !coeff_ctas)
+    return fail(DICTPROJ_ERR_NULL, "decode_batch_plan: NULL pointer");
+  if (n < 1 || n > DICTPROJ_MAX_BATCH)
+    return fail(DICTPROJ_ERR_RANGE, "decode_batch_plan: n=%d outside [1, %d]", n, DICTPROJ_MAX_BATCH);
+  if (M < 1 || M > kDecodeMaxTokens) return fail(DICTPROJ_ERR_RANGE, "decode_batch_plan: M=%d outside [1, %d]", M, kDecodeMaxTokens);
+  if (n_sm < 1) return fail(DICTPROJ_ERR_RANGE, "decode_batch_plan: n_sm=%d < 1", n_sm);
+  size_t ent[kDecodeMaxBatch];
+  for (int i = 0; i < n; ++i) {
+    if (d_in[i] < 16 || d_in[i] % 16 || k[i] < 16 || k[i] % 16 || d_out[i] < 1)
+      return fail(DICTPROJ_ERR_SHAPE, "decode_batch_plan: entry %d has d_in=%d k=%d d_out=%d", i, d_in[i], k[i], d_out[i]);
+    if (entries[i] < 0) return fail(DICTPROJ_ERR_RANGE, "decode_batch_plan: entry %d has %lld entries", i, entries[i]);
+    ent[i] = (size_t)entries[i];
+  }
+  DictPlan plans[kDecodeMaxBatch];
+  dict_plan_batch(n, d_in, k, n_sm, M, plans);
+  int share[kDecodeMaxBatch];
+  gather_batch_shares(n, ent, n_sm, share);
+  for (int i = 0; i < n; ++i) {
+    dict_ctas[i] = (k[i] / 16) * plans[i].slices;
+    dict_slices[i] = plans[i].slices;
+    const int cols = (d_out[i] + share[i] - 1) / share[i];
+    coeff_ctas[i] = (d_out[i] + cols - 1) / cols;
+  }
   return DICTPROJ_OK;
 }
 
@@ -1089,6 +1149,8 @@ int dictproj_check(void* stream) {
   if ((e = take_decode_error(&word)) != cudaSuccess) return cuda_fail(e, "check: read error word");
   unsigned int word2 = 0;
   if ((e = take_prefill_error(&word2)) != cudaSuccess) return cuda_fail(e, "check: read error word");
+  word |= word2;
+  if ((e = take_fused_error(&word2)) != cudaSuccess) return cuda_fail(e, "check: read error word");
   word |= word2;
   if (word) return fail(DICTPROJ_ERR_TIMEOUT, "check: a bounded device wait gave up (error word 0x%x)", word);
   return DICTPROJ_OK;

@@ -45,6 +45,15 @@ __device__ __forceinline__ uint32_t ld_stream_u8(const void* p) {
   asm volatile("ld.global.nc.L1::no_allocate.u8 %0, [%1];" : "=h"(r) : "l"(p));
   return r;
 }
+// Load of data another grid wrote (served by L2, never a stale L1 line).
+__device__ __forceinline__ float4 ld_cg_v4f(const float* p) {
+  float4 r;
+  asm volatile("ld.global.cg.v4.f32 {%0,%1,%2,%3}, [%4];"
+               : "=f"(r.x), "=f"(r.y), "=f"(r.z), "=f"(r.w)
+               : "l"(p)
+               : "memory");
+  return r;
+}
 // Read-only load that may stay in L1 (small operands reused across a CTA).
 __device__ __forceinline__ uint4 ld_nc_v4(const void* p) {
   uint4 r;
@@ -213,6 +222,70 @@ __device__ __forceinline__ uint32_t lds_u16(uint32_t a) {
   uint32_t v;
   asm volatile("ld.shared.u16 %0, [%1];" : "=r"(v) : "r"(a));
   return v;
+}
+
+// x << n with the PTX rule for n >= 32 (the result is 0).
+__device__ __forceinline__ uint32_t shl_clamped(uint32_t x, uint32_t n) {
+  uint32_t r;
+  asm("shl.b32 %0, %1, %2;" : "=r"(r) : "r"(x), "r"(n));
+  return r;
+}
+// prmt.b32 in its default mode: result byte i is byte (sel nibble i & 7) of
+// {b:a}, replaced by copies of that byte's top bit when nibble bit 3 is set.
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
+  uint32_t r;
+  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "r"(b), "r"(sel));
+  return r;
+}
+
+// ---- fp16 Z rows: one mixed-precision FMA per token ---------------------------
+// acc += z * v with z and v fp16 and acc fp32 (fma.rn.f32.f16: the product of two
+// fp16 values is exact in fp32, so only the accumulation rounds). v is half H of
+// an f16x2 register.
+__device__ __forceinline__ unsigned short lds_h16(uint32_t a) {
+  unsigned short v;
+  asm volatile("ld.shared.u16 %0, [%1];" : "=h"(v) : "r"(a));
+  return v;
+}
+template <int H>
+__device__ __forceinline__ void ffma_h(float& acc, unsigned short z, uint32_t v2) {
+  if constexpr (H == 0)
+    asm("{\n\t.reg .f16 vl, vh;\n\tmov.b32 {vl, vh}, %2;\n\tfma.rn.f32.f16 %0, %1, vl, %0;\n\t}"
+        : "+f"(acc) : "h"(z), "r"(v2));
+  else
+    asm("{\n\t.reg .f16 vl, vh;\n\tmov.b32 {vl, vh}, %2;\n\tfma.rn.f32.f16 %0, %1, vh, %0;\n\t}"
+        : "+f"(acc) : "h"(z), "r"(v2));
+}
+// Both halves of an f16x2 word z2 (two tokens) times half H of v2.
+template <int H>
+__device__ __forceinline__ void ffma_h2(float& a0, float& a1, uint32_t z2, uint32_t v2) {
+  if constexpr (H == 0)
+    asm("{\n\t.reg .f16 z0, z1, vl, vh;\n\tmov.b32 {z0, z1}, %2;\n\tmov.b32 {vl, vh}, %3;\n\t"
+        "fma.rn.f32.f16 %0, z0, vl, %0;\n\tfma.rn.f32.f16 %1, z1, vl, %1;\n\t}"
+        : "+f"(a0), "+f"(a1) : "r"(z2), "r"(v2));
+  else
+    asm("{\n\t.reg .f16 z0, z1, vl, vh;\n\tmov.b32 {z0, z1}, %2;\n\tmov.b32 {vl, vh}, %3;\n\t"
+        "fma.rn.f32.f16 %0, z0, vh, %0;\n\tfma.rn.f32.f16 %1, z1, vh, %1;\n\t}"
+        : "+f"(a0), "+f"(a1) : "r"(z2), "r"(v2));
+}
+// Z rows of MP fp16 tokens at byte address a; acc[m] += Z[m] * (half H of v2).
+template <int MP, int H>
+__device__ __forceinline__ void fma_zh(float acc[MP], uint32_t a, uint32_t v2) {
+  if constexpr (MP == 1) {
+    ffma_h<H>(acc[0], lds_h16(a), v2);
+  } else if constexpr (MP == 2) {
+    ffma_h2<H>(acc[0], acc[1], lds_u32(a), v2);
+  } else if constexpr (MP == 4) {
+    const uint2 z = lds_u32x2(a);
+    ffma_h2<H>(acc[0], acc[1], z.x, v2);
+    ffma_h2<H>(acc[2], acc[3], z.y, v2);
+  } else {
+    const uint4 z = lds_u32x4(a);
+    ffma_h2<H>(acc[0], acc[1], z.x, v2);
+    ffma_h2<H>(acc[2], acc[3], z.y, v2);
+    ffma_h2<H>(acc[4], acc[5], z.z, v2);
+    ffma_h2<H>(acc[6], acc[7], z.w, v2);
+  }
 }
 
 // Z rows live in shared memory at byte address zaddr + atom * MP * 4.

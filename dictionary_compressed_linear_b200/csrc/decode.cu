@@ -305,19 +305,55 @@ __device__ __forceinline__ void entries_sum(float blk[MP], uint32_t zaddr, const
 }
 
 // Stage Z (sum of the dictionary stage's slices, fixed order) into shared memory.
+// The slices' loads are issued four at a time before any of them is summed, so
+// the staging costs one L2 round trip per four slices, not one per slice; the
+// sum keeps the slice order (bit-identical to a plain loop).
 template <int MP>
 __device__ __forceinline__ void stage_z(float* zs, const float* __restrict__ Zpart, int nslices, int k, int nthr) {
   const int n = k * MP;
   for (int i = threadIdx.x * 4; i < n; i += nthr * 4) {
-    float4 a = *reinterpret_cast<const float4*>(Zpart + i);
-    for (int sl = 1; sl < nslices; ++sl) {
-      const float4 b = *reinterpret_cast<const float4*>(Zpart + (size_t)sl * n + i);
-      a.x += b.x;
-      a.y += b.y;
-      a.z += b.z;
-      a.w += b.w;
+    float4 a = ld_cg_v4f(Zpart + i);
+    for (int s0 = 1; s0 < nslices; s0 += 4) {
+      float4 b[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j)
+        if (s0 + j < nslices) b[j] = ld_cg_v4f(Zpart + (size_t)(s0 + j) * n + i);
+#pragma unroll
+      for (int j = 0; j < 4; ++j)
+        if (s0 + j < nslices) {
+          a.x += b[j].x;
+          a.y += b[j].y;
+          a.z += b[j].z;
+          a.w += b[j].w;
+        }
     }
     *reinterpret_cast<float4*>(zs + i) = a;
+  }
+}
+
+// stage_z, rounded to an fp16 table (the gather kernel's Z).
+template <int MP>
+__device__ __forceinline__ void stage_zh(__half* zs, const float* __restrict__ Zpart, int nslices, int k, int nthr) {
+  const int n = k * MP;
+  for (int i = threadIdx.x * 4; i < n; i += nthr * 4) {
+    float4 a = ld_cg_v4f(Zpart + i);
+    for (int s0 = 1; s0 < nslices; s0 += 4) {
+      float4 b[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j)
+        if (s0 + j < nslices) b[j] = ld_cg_v4f(Zpart + (size_t)(s0 + j) * n + i);
+#pragma unroll
+      for (int j = 0; j < 4; ++j)
+        if (s0 + j < nslices) {
+          a.x += b[j].x;
+          a.y += b[j].y;
+          a.z += b[j].z;
+          a.w += b[j].w;
+        }
+    }
+    __half2* d = reinterpret_cast<__half2*>(zs + i);
+    d[0] = __floats2half2_rn(a.x, a.y);
+    d[1] = __floats2half2_rn(a.z, a.w);
   }
 }
 
@@ -372,8 +408,8 @@ template <int MP>
 __device__ __forceinline__ void gather_column(const ColData& d, int o, int nhb, uint32_t zs_a, int nseg,
                                               const uint16_t* __restrict__ seg_start, int lane, int M, int d_out,
                                               float s_C, __half* __restrict__ Y) {
-  constexpr uint32_t kRow = MP * 4;
-    float acc[MP];
+  constexpr uint32_t kRowH = MP * 2;  // bytes per atom row of the fp16 Z table
+  float acc[MP];
 #pragma unroll
   for (int m = 0; m < MP; ++m) acc[m] = 0.f;
   // Lane j holds seg_start[j] (the first entry of segment j). For the window of
@@ -405,7 +441,6 @@ __device__ __forceinline__ void gather_column(const ColData& d, int o, int nhb, 
     const int t2 = collide ? q0 : INT_MAX;  // forces the walk for the whole window
     if (32 * i + lane < nhb) {
       const uint32_t iw[2] = {d.iv[i].x, d.iv[i].y};
-      float blk[MP];
       float a0[MP], a1[MP];
 #pragma unroll
       for (int m = 0; m < MP; ++m) a0[m] = a1[m] = 0.f;
@@ -413,16 +448,19 @@ __device__ __forceinline__ void gather_column(const ColData& d, int o, int nhb, 
       e2m1x8_to_f16x2x4(d.cv[i], f);
       if (q0 + 7 < t2) {  // at most one boundary: entries e >= t use segment sgi+1
         const int t = min(t1 - q0, 8);
-        const uint32_t z0 = zs_a + ((uint32_t)sgi << 8) * kRow;
-        const uint32_t z1 = z0 + 256u * kRow;
+        // flag byte of each entry: 1 past the boundary; prmt then forms the
+        // entry's 9-bit row (index byte + 256 x flag) with zero upper bytes
+        const uint32_t fl[2] = {shl_clamped(0x01010101u, 8u * (uint32_t)t),
+                                shl_clamped(0x01010101u, 8u * (uint32_t)max(t - 4, 0))};
+        const uint32_t z0 = zs_a + ((uint32_t)sgi << 8) * kRowH;
 #pragma unroll
-        for (int p = 0; p < 4; ++p) {
-          const float2 v = __half22float2(*reinterpret_cast<const __half2*>(&f[p]));
-          const int e0 = 2 * p, e1 = e0 + 1;
-          const uint32_t b0 = __byte_perm(iw[e0 >> 2], 0u, 0x4440u | (uint32_t)(e0 & 3));
-          const uint32_t b1 = __byte_perm(iw[e1 >> 2], 0u, 0x4440u | (uint32_t)(e1 & 3));
-          fma_z<MP>(a0, (e0 >= t ? z1 : z0) + b0 * kRow, v.x);
-          fma_z<MP>(a1, (e1 >= t ? z1 : z0) + b1 * kRow, v.y);
+        for (int e = 0; e < 8; ++e) {
+          const uint32_t j = (uint32_t)(e & 3);
+          const uint32_t row = prmt(iw[e >> 2], fl[e >> 2], j | ((4u + j) << 4) | ((12u + j) << 8) | ((12u + j) << 12));
+          if (e & 1)
+            fma_zh<MP, 1>(a1, z0 + row * kRowH, f[e >> 1]);
+          else
+            fma_zh<MP, 0>(a0, z0 + row * kRowH, f[e >> 1]);
         }
       } else {  // several boundaries inside these 8 entries: walk them (row read from memory)
         const uint16_t* ssrow = seg_start + (size_t)o * nseg;
@@ -430,24 +468,22 @@ __device__ __forceinline__ void gather_column(const ColData& d, int o, int nhb, 
         for (int j = 1; j < nseg; ++j) sg += ((int)ssrow[j] <= q0);
         int nb = (sg + 1 < nseg) ? (int)ssrow[sg + 1] : INT_MAX;
 #pragma unroll
-        for (int p = 0; p < 4; ++p) {
-          const float2 v = __half22float2(*reinterpret_cast<const __half2*>(&f[p]));
-#pragma unroll
-          for (int hh = 0; hh < 2; ++hh) {
-            const int ent = 2 * p + hh;
-            while (q0 + ent >= nb) {
-              ++sg;
-              nb = (sg + 1 < nseg) ? (int)ssrow[sg + 1] : INT_MAX;
-            }
-            const uint32_t b = __byte_perm(iw[ent >> 2], 0u, 0x4440u | (uint32_t)(ent & 3));
-            fma_z<MP>(hh ? a1 : a0, zs_a + (((uint32_t)sg << 8) + b) * kRow, hh ? v.y : v.x);
+        for (int e = 0; e < 8; ++e) {
+          while (q0 + e >= nb) {
+            ++sg;
+            nb = (sg + 1 < nseg) ? (int)ssrow[sg + 1] : INT_MAX;
           }
+          const uint32_t b = __byte_perm(iw[e >> 2], 0u, 0x4440u | (uint32_t)(e & 3));
+          const uint32_t ad = zs_a + (((uint32_t)sg << 8) + b) * kRowH;
+          if (e & 1)
+            fma_zh<MP, 1>(a1, ad, f[e >> 1]);
+          else
+            fma_zh<MP, 0>(a0, ad, f[e >> 1]);
         }
       }
-      const float sc = e4m3_to_f32((uint32_t)(d.sc >> (8 * i)) & 0xFFu);
+      const float sc = e4m3_to_f32_int((uint32_t)(d.sc >> (8 * i)) & 0xFFu);
 #pragma unroll
       for (int m = 0; m < MP; ++m) acc[m] = fmaf(a0[m] + a1[m], sc, acc[m]);
-      (void)blk;
     }
   }
 #pragma unroll
@@ -465,7 +501,7 @@ __device__ __forceinline__ void gather_column(const ColData& d, int o, int nhb, 
 template <int MP>
 __global__ void __launch_bounds__(kGatherWarps * 32, 1)  // 1024 threads, at most 64 registers
 k_coeff_gather(const __grid_constant__ CoeffBatch batch) {
-  extern __shared__ __align__(16) float zsg[];  // [k + 256][MP]; the tail is zero
+  extern __shared__ __align__(16) __half zsg[];  // fp16 [k + 256][MP]; the tail is zero
   int pi = 0;
   while (pi + 1 < batch.n && (int)blockIdx.x >= batch.p[pi + 1].block_begin) ++pi;
   const CoeffProj& pr = batch.p[pi];
@@ -499,8 +535,8 @@ k_coeff_gather(const __grid_constant__ CoeffBatch batch) {
   trigger_dependents();
   grid_dependency_wait();  // Z comes from the dictionary stage
 
-  stage_z<MP>(zsg, Zpart, nslices, k, blockDim.x);
-  for (int i = k * MP + threadIdx.x; i < (k + 256) * MP; i += blockDim.x) zsg[i] = 0.f;
+  stage_zh<MP>(zsg, Zpart, nslices, k, blockDim.x);
+  for (int i = k * MP + threadIdx.x; i < (k + 256) * MP; i += blockDim.x) zsg[i] = __float2half_rn(0.f);
   __syncthreads();
   const uint32_t zs_a = smem_u32(zsg);
 
@@ -607,26 +643,43 @@ constexpr size_t kDictXsMax = 96 * 1024;
 
 static size_t dict_xs_bytes(int xlen, int M) { return (size_t)M * (xlen + 8) * sizeof(__half); }
 
-DictPlan dict_plan(int d_in, int k, int n_sm, int M, bool one_slice) {
-  const int units = (d_in + 127) / 128;
-  const int tiles = k / kDictTile;
-  DictPlan p;
-  p.J = 1;
-  if (one_slice) {
-    p.J = (units + kDictWarps - 1) / kDictWarps;
-  } else {
-    // J grows until the grid fits four CTAs per SM (4 x 256 threads x 64
-    // registers fill the register file: the kernel is latency-bound, so resident
-    // warps matter most); it shrinks back while the slice's X rows would not fit
-    // the shared-memory cap
-    while (p.J < units) {
-      const size_t ctas = (size_t)tiles * ((units + kDictWarps * p.J - 1) / (kDictWarps * p.J));
-      if (ctas <= (size_t)4 * n_sm) break;
-      ++p.J;
-    }
-    while (p.J > 1 && dict_xs_bytes(std::min(d_in, kDictWarps * p.J * 128), M) > kDictXsMax) --p.J;
+// J of one projection alone: J grows until its grid fits four CTAs per SM
+// (4 x 256 threads x 64 registers fill the register file: the kernel is
+// latency-bound, so resident warps matter most).
+static int dict_lone_J(int d_in, int k, int n_sm) {
+  const int units = (d_in + 127) / 128, tiles = k / kDictTile;
+  int J = 1;
+  while (J < units && (size_t)tiles * ((units + kDictWarps * J - 1) / (kDictWarps * J)) > (size_t)4 * n_sm) ++J;
+  return J;
+}
+
+void dict_plan_batch(int n, const int* d_in, const int* k, int n_sm, int M, DictPlan* plans) {
+  // One J for the whole batch, the largest any of its projections takes alone:
+  // every CTA then streams the same 8 x J units of 16 atom rows (or all of a
+  // shorter d_in), so each projection's CTAs follow its dictionary bytes
+  // (d_in x k) and the hardware scheduler balances the grid; a batch of equal
+  // shapes gets exactly the lone plan. Per projection, J shrinks back while the
+  // slice's X rows would not fit the shared-memory cap.
+  int J = 1;
+  for (int i = 0; i < n; ++i) J = std::max(J, dict_lone_J(d_in[i], k[i], n_sm));
+  for (int i = 0; i < n; ++i) {
+    const int units = (d_in[i] + 127) / 128;
+    DictPlan& p = plans[i];
+    p.J = std::min(J, units);
+    while (p.J > 1 && dict_xs_bytes(std::min(d_in[i], kDictWarps * p.J * 128), M) > kDictXsMax) --p.J;
+    p.slices = (units + kDictWarps * p.J - 1) / (kDictWarps * p.J);
   }
-  p.slices = (units + kDictWarps * p.J - 1) / (kDictWarps * p.J);
+}
+
+DictPlan dict_plan(int d_in, int k, int n_sm, int M, bool one_slice) {
+  DictPlan p;
+  if (!one_slice) {
+    dict_plan_batch(1, &d_in, &k, n_sm, M, &p);
+    return p;
+  }
+  const int units = (d_in + 127) / 128;
+  p.J = (units + kDictWarps - 1) / kDictWarps;
+  p.slices = 1;
   return p;
 }
 
@@ -705,12 +758,35 @@ cudaError_t launch_dict_decode(const dictproj_group* g, const __half* X, int M, 
   return launch_dict_decode_batch(1, &g, &X, M, mp, &Zpart, &plan, stream);
 }
 
+bool decode_batch_gathers(int n, const dictproj_layer* const* l) {
+  bool all = true;  // (bitmap and block layers have gather_ok false: one launch each)
+  for (int i = 0; i < n; ++i) all = all && l[i]->gather_ok;
+  return all;
+}
+
+void gather_batch_shares(int n, const size_t* entries, int n_sm, int* share) {
+  // CTAs of a batched gather launch shared out in proportion to each projection's
+  // stored entries (its coefficient bytes), at least one each, n_sm in all
+  double wsum = 0.0;
+  for (int i = 0; i < n; ++i) wsum += (double)entries[i] + 1.0;
+  int given = 0;
+  for (int i = 0; i < n; ++i) {
+    share[i] = std::max(1, (int)((double)n_sm * ((double)entries[i] + 1.0) / wsum));
+    given += share[i];
+  }
+  for (int i = 0; given < n_sm; i = (i + 1) % n, ++given) ++share[i];  // the rounding remainder
+}
+
 static cudaError_t launch_gather_batch(int n, const dictproj_layer* const* l, const float* const* Zpart,
                                        const int* nslices, int M, int mp, __half* const* Y, cudaStream_t stream) {
   CoeffBatch b{};
   b.n = n;
   b.M = M;
   int blocks = 0, kmax = 0;
+  size_t entries[kMaxBatch];
+  int share[kMaxBatch];
+  for (int i = 0; i < n; ++i) entries[i] = l[i]->total;
+  gather_batch_shares(n, entries, l[0]->n_sm, share);
   for (int i = 0; i < n; ++i) {
     CoeffProj& p = b.p[i];
     p.col_ptr = l[i]->col_ptr;
@@ -725,8 +801,7 @@ static cudaError_t launch_gather_batch(int n, const dictproj_layer* const* l, co
     p.Zpart = Zpart[i];
     p.nslices = nslices[i];
     p.Y = Y[i];
-    // columns per CTA: one CTA per SM for a single projection, shared out over the batch
-    const int ctas = std::max(1, l[i]->n_sm / n);
+    const int ctas = share[i];
     p.cols_per_cta = (p.d_out + ctas - 1) / ctas;
     p.block_begin = blocks;
     blocks += (p.d_out + p.cols_per_cta - 1) / p.cols_per_cta;
@@ -734,7 +809,7 @@ static cudaError_t launch_gather_batch(int n, const dictproj_layer* const* l, co
   }
   void* args[] = {(void*)&b};
   const dim3 grid(blocks), block(kGatherWarps * 32);
-  const size_t smem = (size_t)(kmax + 256) * mp * sizeof(float);
+  const size_t smem = (size_t)(kmax + 256) * mp * sizeof(__half);
   switch (mp) {
     case 1: return launch_pdl((const void*)k_coeff_gather<1>, grid, block, smem, stream, args);
     case 2: return launch_pdl((const void*)k_coeff_gather<2>, grid, block, smem, stream, args);
@@ -745,9 +820,7 @@ static cudaError_t launch_gather_batch(int n, const dictproj_layer* const* l, co
 
 cudaError_t launch_coeff_decode_batch(int n, const dictproj_layer* const* l, const float* const* Zpart,
                                       const int* nslices, int M, int mp, __half* const* Y, cudaStream_t stream) {
-  bool all_gather = true;  // (bitmap and block layers have gather_ok false: one launch each)
-  for (int i = 0; i < n; ++i) all_gather = all_gather && l[i]->gather_ok;
-  if (all_gather) return launch_gather_batch(n, l, Zpart, nslices, M, mp, Y, stream);
+  if (decode_batch_gathers(n, l)) return launch_gather_batch(n, l, Zpart, nslices, M, mp, Y, stream);
   for (int i = 0; i < n; ++i) {
     cudaError_t e = launch_coeff_decode(l[i], Zpart[i], nslices[i], M, mp, Y[i], stream);
     if (e != cudaSuccess) return e;

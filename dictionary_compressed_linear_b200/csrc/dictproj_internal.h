@@ -61,7 +61,6 @@ struct dictproj_group {
   uint16_t* z16;           // prefill Z, fp16 [max_tokens][k]
   uint16_t* cdense;        // prefill coefficient operand, fp16 [d_out][k] for d_out <= cdense_cols
   int cdense_cols;         // reserved output columns (dictproj_group_reserve_prefill)
-  unsigned int* err;       // device error word for bounded waits
   CUtensorMap codes_map;   // TMA map of codes: [k] rows x [d_in/2] bytes, box 32 x 256
   // fused decode kernel
   bool fused_ok;           // the fused kernel serves this group

@@ -338,12 +338,6 @@ __device__ __forceinline__ void hb_decode(uint4 r, uint32_t f[4]) {
   }
 }
 
-// x << n with the PTX rule for n >= 32 (the result is 0).
-__device__ __forceinline__ uint32_t shl_clamped(uint32_t x, uint32_t n) {
-  uint32_t r;
-  asm("shl.b32 %0, %1, %2;" : "=r"(r) : "r"(x), "r"(n));
-  return r;
-}
 
 // Segment state of a thread inside one column of C_l: sg is the segment of the
 // current entry q (the number of segment starts s >= 1 with seg_start[s] <= q),
@@ -1325,6 +1319,13 @@ cudaError_t launch_fused(int n, const dictproj_group* const* g, const dictproj_l
     case 4: return cudaLaunchKernelEx(&cfg, k_decode_fused<4>, prm);
     default: return cudaLaunchKernelEx(&cfg, k_decode_fused<8>, prm);
   }
+}
+
+cudaError_t take_fused_error(unsigned int* out) {
+  unsigned int zero = 0;
+  cudaError_t e = cudaMemcpyFromSymbol(out, g_dictproj_error, sizeof(unsigned int));
+  if (e != cudaSuccess) return e;
+  return cudaMemcpyToSymbol(g_dictproj_error, &zero, sizeof(unsigned int));
 }
 
 }  // namespace dictproj

@@ -20,6 +20,12 @@ struct DictPlan {
   int slices;  // d_in slices = grid.y
 };
 DictPlan dict_plan(int d_in, int k, int n_sm, int M, bool one_slice);
+// One plan for a batched launch: a common J, so CTAs per projection follow its
+// dictionary bytes; never more slices than dict_plan gives each alone.
+void dict_plan_batch(int n, const int* d_in, const int* k, int n_sm, int M, DictPlan* plans);
+// CTAs of a batched gather launch per projection, in proportion to its stored
+// entries, at least one each.
+void gather_batch_shares(int n, const size_t* entries, int n_sm, int* share);
 int dict_max_slices(int d_in, int k, int n_sm);  // over all decode M
 cudaError_t launch_dict_decode(const dictproj_group* g, const __half* X, int M, int mp, float* Zpart,
                                const DictPlan& plan, cudaStream_t stream);
@@ -31,6 +37,8 @@ cudaError_t launch_dict_decode_batch(int n, const dictproj_group* const* g, cons
                                      int mp, float* const* Zpart, const DictPlan* plans, cudaStream_t stream);
 cudaError_t launch_coeff_decode_batch(int n, const dictproj_layer* const* l, const float* const* Zpart,
                                       const int* nslices, int M, int mp, __half* const* Y, cudaStream_t stream);
+// Whether one gather launch serves the batch's coefficient stage.
+bool decode_batch_gathers(int n, const dictproj_layer* const* l);
 
 // Whether the gather kernel serves a layer (every column <= 1280 padded
 // entries, at most 32 segments); other layers use the direct kernel.
@@ -42,6 +50,7 @@ bool coeff_smem_fits(int k, int mp, int device);
 cudaError_t launch_wait_probe(long long cycles, cudaStream_t stream);
 // Read and clear the device error word of the decode kernels.
 cudaError_t take_decode_error(unsigned int* out);
+cudaError_t take_fused_error(unsigned int* out);
 
 // fused decode path (M <= 8): one kernel per call, both stages, weights staged
 // through shared memory by TMA (fused.cu)

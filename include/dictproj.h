@@ -299,7 +299,8 @@ void dictproj_free_layer(dictproj_layer* l); /* NULL is a no-op */
  * Asynchronous on `stream`: no allocation, no host synchronisation. Kernels are
  * launched with programmatic dependent launch; each kernel waits for the
  * preceding work on the stream before it reads X or writes Z / Y (packed
- * weights, which nothing writes after upload, may be prefetched earlier).
+ * weights, which nothing writes after upload, may be prefetched earlier). A group
+ * serves one stream at a time: its Z scratch is shared by its calls.
  * Errors (checked before any launch): NULL, RANGE (M), MISMATCH (k or device),
  * ALIGN, UNSUPPORTED (k too large for the decode path's shared memory); CUDA if
  * a launch fails. */
@@ -307,8 +308,11 @@ int dictproj_forward(const void* X, int M, const dictproj_layer* layer,
                      const dictproj_group* group, void* Y, void* stream);
 
 /* Up to DICTPROJ_MAX_BATCH independent projections in one call: projection i
- * computes Y[i] = X[i] D_g[i] C_l[i] exactly as dictproj_forward would (the same
- * kernels and arithmetic, so bit-identical results). The projections must be
+ * computes Y[i] = X[i] D_g[i] C_l[i] with the kernels and arithmetic of
+ * dictproj_forward. The dictionary stage's d_in slicing is planned over the whole
+ * batch (dictproj_decode_batch_plan), so Y[i] equals dictproj_forward's bit for
+ * bit where that plan gives projection i the slices it gets alone, and otherwise
+ * agrees within the decode tolerance (its fp32 partial sums split differently). The projections must be
  * independent: no Y[i] may be read as an X[j] of the same call; X entries may
  * alias (e.g. the q, k and v projections of one layer read the same activation);
  * the groups must be distinct (each call uses its group's Z scratch). For
@@ -319,6 +323,29 @@ int dictproj_forward(const void* X, int M, const dictproj_layer* layer,
 #define DICTPROJ_MAX_BATCH 4
 int dictproj_forward_batch(int n, const void* const* X, int M, const dictproj_layer* const* layers,
                            const dictproj_group* const* groups, void* const* Y, void* stream);
+
+/* dictproj_forward_batch with a stage mask, to time each kernel of the two-kernel
+ * decode path in the launch configuration a full call uses (the same batch plan,
+ * grids and Z scratch): bit 0 launches the dictionary kernel (Z = X D_g into each
+ * group's Z scratch), bit 1 the coefficient kernel (Y = Z C_l from that scratch,
+ * as the last dictionary launch on these groups left it); 3 is the full call.
+ * A mask of 1 or 2 needs M <= 8 and a call the two-kernel path serves.
+ * Errors as dictproj_forward_batch, plus RANGE (mask not 1, 2 or 3) and
+ * UNSUPPORTED (a mask of 1 or 2 with M > 8 or on the fused kernel). */
+int dictproj_forward_batch_stages(int n, const void* const* X, int M, const dictproj_layer* const* layers,
+                                  const dictproj_group* const* groups, void* const* Y, void* stream, int stages);
+
+/* The grid a batched two-kernel decode call (1 <= M <= 8) of n <= DICTPROJ_MAX_BATCH
+ * projections would launch, host only: projection i has d_in[i] rows, k[i] atoms,
+ * d_out[i] columns and entries[i] stored (padded) coefficient entries; n_sm is
+ * the device's SM count. Out (caller-owned arrays of n ints): dict_ctas[i] and
+ * dict_slices[i], the dictionary kernel's CTAs and d_in slices for projection i
+ * (every CTA streams the same number of dictionary rows, so CTAs follow
+ * d_in x k), and coeff_ctas[i], the coefficient kernel's CTAs for projection i
+ * (in proportion to entries[i], at least one, n_sm in all before rounding
+ * columns up). Errors: NULL, RANGE (n, M, n_sm, entries < 0), SHAPE. */
+int dictproj_decode_batch_plan(int n, const int* d_in, const int* k, const int* d_out, const long long* entries,
+                               int M, int n_sm, int* dict_ctas, int* dict_slices, int* coeff_ctas);
 
 /* Number of kernels that dictproj_forward_batch with these arguments (n = 1:
  * dictproj_forward) launches: 1 for a decode call served by the fused kernel,

@@ -206,6 +206,45 @@ def test_chain_of_calls_sharing_a_group():
     assert_parity(y2, oracle_forward(Y1.cpu().numpy(), pd, pc2, dense=True), "chain 2")
 
 
+def test_full_and_stage_mask_calls_interleaved_on_one_group():
+    # full calls, single calls and stage-mask calls share the group's Z scratch;
+    # interleaved on one stream they stay ordered, in eager launches and in graph
+    # replays, with no bounded wait giving up
+    D = synth.gen_dictionary(20, 0, 0, 2048, 1024)
+    C = synth.gen_coeff(20, 0, 0, 0, 1024, 1500, 0.3)
+    g, l = device_projection(D, C, max_tokens=8)
+    pd, pc = oracle_projection(D, C)
+    Xn = [synth.gen_activations(20, i, 0, 2, 2048) for i in range(3)]
+    Xs = [torch.from_numpy(x).cuda() for x in Xn]
+    Y = torch.empty((2, 1500), dtype=torch.float16, device="cuda")
+    outs = [torch.empty_like(Y) for _ in range(3)]
+    s = torch.cuda.Stream()
+
+    def seq():
+        for i, x in enumerate(Xs):
+            dp.dictproj_forward(x.data_ptr(), 2, l, g, outs[i].data_ptr(), s.cuda_stream)
+            dp.dictproj_forward_batch_stages([x.data_ptr()], 2, [l], [g], [Y.data_ptr()], s.cuda_stream, 1)
+            dp.dictproj_forward_batch_stages([x.data_ptr()], 2, [l], [g], [Y.data_ptr()], s.cuda_stream, 2)
+            dp.dictproj_forward_batch([x.data_ptr()], 2, [l], [g], [Y.data_ptr()], s.cuda_stream)
+    with torch.cuda.stream(s):
+        seq()
+    dp.dictproj_check(s.cuda_stream)
+    first = [o.clone() for o in outs]
+    for x, o in zip(Xn, outs):
+        assert_parity(o.float().cpu().numpy().astype(np.float64), oracle_forward(x, pd, pc), "interleaved calls")
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=s):
+        seq()
+    for o in outs:
+        o.fill_(float("nan"))
+    with torch.cuda.stream(s):
+        for _ in range(20):
+            graph.replay()
+    dp.dictproj_check(s.cuda_stream)
+    for a, b in zip(first, outs):
+        assert torch.equal(a, b)
+
+
 # ------------------------------------------------------------------ batched forward
 @pytest.mark.parametrize("M", [1, 3, 8, 12])
 def test_batch_matches_single_calls_bitwise(M):
@@ -228,6 +267,46 @@ def test_batch_matches_single_calls_bitwise(M):
     torch.cuda.synchronize()
     for a, b in zip(Ys, Yr):
         assert torch.equal(a, b)
+
+
+@pytest.mark.parametrize("M", [1, 8])
+def test_mixed_shape_batch_with_byte_proportional_grid(M):
+    # LLaMA-7B shapes of different sizes in one call: the dictionary grid shares a
+    # J that differs from some lone plans and the gather CTAs follow stored
+    # entries; each output still meets the oracle bar, and the stage-mask calls
+    # (dictionary kernel, then coefficient kernel) reproduce the full call bit for bit
+    shapes = [(4096, 2048, 4096, 0.3), (11008, 3072, 4096, 0.25), (4096, 3072, 11008, 0.25)]
+    projs, refs = [], []
+    for i, (d_in, k, d_out, rho) in enumerate(shapes):
+        D, C = _case(19, i, i, 0, d_in, k, d_out, rho)
+        g, l = device_projection(D, C, max_tokens=8)
+        projs.append((g, l, d_in, d_out))
+        refs.append(oracle_projection(D, C))
+    Xn = [synth.gen_activations(19, i, 0, M, d) for i, (_, _, d, _) in enumerate(projs)]
+    Xs = [torch.from_numpy(x).cuda() for x in Xn]
+    Ys = [torch.full((M, do), float("nan"), dtype=torch.float16, device="cuda") for (_, _, _, do) in projs]
+    args = ([x.data_ptr() for x in Xs], M, [p[1] for p in projs], [p[0] for p in projs])
+    st = torch.cuda.current_stream().cuda_stream
+    dp.dictproj_forward_batch(*args, [y.data_ptr() for y in Ys], st)
+    torch.cuda.synchronize()
+    for y, x, (pd, pc), i in zip(Ys, Xn, refs, range(3)):
+        assert_parity(y.float().cpu().numpy().astype(np.float64), oracle_forward(x, pd, pc), f"mixed batch {i} M={M}")
+    Y2 = [torch.full_like(y, float("nan")) for y in Ys]
+    dp.dictproj_forward_batch_stages(*args, [y.data_ptr() for y in Y2], st, 1)
+    torch.cuda.synchronize()
+    assert all(torch.isnan(y.float()).all() for y in Y2)  # the dictionary kernel alone writes no output
+    dp.dictproj_forward_batch_stages(*args, [y.data_ptr() for y in Y2], st, 2)
+    torch.cuda.synchronize()
+    for a, b in zip(Ys, Y2):
+        assert torch.equal(a, b)
+    for bad in (0, 4):
+        with pytest.raises(dp.DictprojError) as e:
+            dp.dictproj_forward_batch_stages(*args, [y.data_ptr() for y in Y2], st, bad)
+        assert e.value.status == -5
+    plan = dp.dictproj_decode_batch_plan(
+        [(d_in, k, d_out, int(np.asarray(pc["col_ptr"])[-1])) for (d_in, k, d_out, _), (_, pc) in zip(shapes, refs)],
+        M, torch.cuda.get_device_properties(0).multi_processor_count)
+    assert all(p["dict_ctas"] >= 1 and p["coeff_ctas"] >= 1 for p in plan)
 
 
 def test_batch_rejects_repeated_group():

@@ -292,3 +292,34 @@ def test_index_format_uploads_validate_before_touching_a_device(dp):
         dp.dictproj_pack_layer_blocks(np.array([0, 3], np.int32), np.array([0, 1, 2], np.int32),
                                       np.ones(3, np.float32), 48, 1)
     assert err.value.status < 0
+
+
+def test_batched_decode_grid_follows_each_projections_bytes(dp):
+    # a batch of equal shapes (q/k/v) launches exactly the lone plans; a mixed batch
+    # streams the same dictionary rows per CTA wherever d_in allows and shares the
+    # coefficient kernel's CTAs in proportion to stored entries
+    n_sm = 148
+    qkv = (4096, 2048, 4096, 4096 * 624)
+    lone = dp.dictproj_decode_batch_plan([qkv], 1, n_sm)[0]
+    batch = dp.dictproj_decode_batch_plan([qkv] * 3, 1, n_sm)
+    assert all(b["dict_ctas"] == lone["dict_ctas"] and b["dict_slices"] == lone["dict_slices"] for b in batch)
+    assert sorted(b["coeff_ctas"] for b in batch) == [49, 49, 50]
+    assert n_sm - 2 <= lone["coeff_ctas"] <= n_sm  # columns per CTA rounded up
+    mixed = [(4096, 2048, 4096, 4096 * 624), (11008, 3072, 4096, 4096 * 784), (4096, 3072, 11008, 11008 * 784)]
+    plan = dp.dictproj_decode_batch_plan(mixed, 1, n_sm)
+    rows = [d / p["dict_slices"] for (d, _, _, _), p in zip(mixed, plan)]
+    assert max(rows) / min(rows) < 1.15  # per-CTA dictionary bytes within rounding of one slice
+    for (d_in, k, _, _), p in zip(mixed, plan):
+        assert p["dict_ctas"] == (k // 16) * p["dict_slices"]
+        alone = dp.dictproj_decode_batch_plan([(d_in, k, 16, 0)], 1, n_sm)[0]
+        assert p["dict_slices"] <= alone["dict_slices"]  # never more Z partial sums than the group holds
+    ent = [e for _, _, _, e in mixed]
+    per_cta = [e / p["coeff_ctas"] for e, p in zip(ent, plan)]
+    assert max(per_cta) / min(per_cta) < 1.1
+    assert sum(p["coeff_ctas"] for p in plan) <= n_sm
+    tiny = dp.dictproj_decode_batch_plan([(64, 32, 8, 16), (4096, 2048, 4096, 10 ** 7)], 1, n_sm)
+    assert tiny[0]["coeff_ctas"] >= 1 and tiny[0]["dict_slices"] == 1
+    with pytest.raises(dp.DictprojError):
+        dp.dictproj_decode_batch_plan([qkv], 9, n_sm)
+    with pytest.raises(dp.DictprojError):
+        dp.dictproj_decode_batch_plan([(4096, 2047, 16, 0)], 1, n_sm)
