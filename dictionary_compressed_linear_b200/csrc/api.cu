@@ -990,7 +990,7 @@ static int forward_batch_impl(int n, const void* const* X, int M, const dictproj
   for (int i = 0; i < n; ++i) din[i] = groups[i]->d_in, kk[i] = groups[i]->k;
   dict_plan_batch(n, din, kk, groups[0]->n_sm, M, plans);
   for (int i = 0; i < n; ++i) {
-    if (plans[i].slices > groups[i]->zslices)  // cannot happen: a common J is never below the lone plan's
+    if (plans[i].slices > groups[i]->zslices)  // cannot happen: the scratch holds the slices of J = 1
       return fail(DICTPROJ_ERR_UNSUPPORTED, "forward_batch: plan needs %d Z slices, entry %d holds %d",
                   plans[i].slices, i, groups[i]->zslices);
     xs[i] = static_cast<const __half*>(X[i]);

@@ -370,34 +370,36 @@ struct ColData {
   uint2 iv[kRmax];      // 8 index bytes per step
   uint32_t cv[kRmax];   // 8 codes (4 bytes) per step
   uint64_t sc;          // E4M3 scale byte of each step, packed 8 bits apiece (kRmax <= 8)
-  int ssv;              // seg_start[lane] of the column (lane < nseg)
+  int ssv;              // seg_start[lane] of the column (lane < nseg), else INT_MAX
 };
 
+// The column's loads: lane L takes half-blocks L, L + 32, ... through per-lane
+// base pointers, so every step is one load per stream at a constant offset.
 __device__ __forceinline__ void load_col(ColData& d, int o, int d_out, const uint32_t* __restrict__ col_ptr,
                                          const uint8_t* __restrict__ idx, const uint8_t* __restrict__ codes,
                                          const uint8_t* __restrict__ scales, const uint16_t* __restrict__ seg_start,
-                                         int nseg, int lane, uint32_t& cb, int& nhb) {
-  cb = 0;
+                                         int nseg, int lane, int& nhb) {
   nhb = 0;
   d.sc = 0;
-  d.ssv = 0;
+  d.ssv = INT_MAX;
 #pragma unroll
   for (int i = 0; i < kRmax; ++i) {
     d.iv[i] = make_uint2(0, 0);
     d.cv[i] = 0;
   }
   if (o >= d_out) return;
-  cb = col_ptr[o];
+  const uint32_t cb = col_ptr[o];
   nhb = (int)((col_ptr[o + 1] - cb) >> 3);
   if (lane < nseg) d.ssv = (int)seg_start[(size_t)o * nseg + lane];
+  const uint8_t* pi = idx + cb + 8 * lane;
+  const uint8_t* pc = codes + (cb >> 1) + 4 * lane;
+  const uint8_t* ps = scales + (cb >> 4) + (lane >> 1);
 #pragma unroll
   for (int i = 0; i < kRmax; ++i) {
-    const int h = 32 * i + lane;
-    if (h < nhb) {
-      const uint32_t e = cb + 8u * (uint32_t)h;
-      d.iv[i] = ld_stream_v2(idx + e);
-      d.cv[i] = *reinterpret_cast<const uint32_t*>(codes + (e >> 1));
-      d.sc |= (uint64_t)ld_stream_u8(scales + (e >> 4)) << (8 * i);
+    if (32 * i + lane < nhb) {
+      d.iv[i] = ld_stream_v2(pi + 256 * i);
+      d.cv[i] = *reinterpret_cast<const uint32_t*>(pc + 128 * i);
+      d.sc |= (uint64_t)ld_stream_u8(ps + 16 * i) << (8 * i);
     }
   }
 }
@@ -412,33 +414,32 @@ __device__ __forceinline__ void gather_column(const ColData& d, int o, int nhb, 
   float acc[MP];
 #pragma unroll
   for (int m = 0; m < MP; ++m) acc[m] = 0.f;
-  // Lane j holds seg_start[j] (the first entry of segment j). For the window of
-  // 256 entries starting at w, a boundary b in (w, w+256) lies at the start of
-  // lane p = (b-w)/8's half-block when (b-w) % 8 == 0, else inside it; two
-  // OR-reduced lane masks give every lane its segment with two popcounts.
+  // Lane j (1 <= j < nseg) holds the start of segment j and c_j, that start
+  // rounded up to a multiple of 8. The segment of the half-block starting at q0
+  // is the number of c_j <= q0. In the window of 256 entries starting at w, c_j
+  // with 0 < c_j - w < 256 counts from lane (c_j - w) / 8 on, so one OR-reduced
+  // lane mask and one ballot give every lane its segment. Two starts with the
+  // same c_j (two boundaries inside one half-block, or an empty segment) would
+  // share a mask bit: such a column takes the walk below for every half-block.
   const bool is_bnd = lane >= 1 && lane < nseg;
+  const int c = is_bnd ? ((d.ssv + 7) & ~7) : INT_MAX;
+  const int c_up = __shfl_down_sync(0xffffffffu, c, 1);  // every lane takes part
+  const bool dup = is_bnd && lane + 1 < nseg && c_up == c;
+  const bool col_walk = __any_sync(0xffffffffu, dup);
+  const uint32_t le = lane == 31 ? 0xffffffffu : ((2u << lane) - 1u);
 #pragma unroll
   for (int i = 0; i < kRmax; ++i) {
     const int w = 256 * i;
     if (w >= 8 * nhb) break;
-    const int b = d.ssv;  // boundary held by this lane (meaningful iff is_bnd)
-    const int s_lo = __popc(__ballot_sync(0xffffffffu, is_bnd && b <= w));  // segment of entry w
-    const bool in_win = is_bnd && b > w && b < w + 256;
-    const int rel = b - w;
-    const uint32_t at_start = (in_win && (rel & 7) == 0) ? (1u << (rel >> 3)) : 0u;
-    const uint32_t inside = (in_win && (rel & 7) != 0) ? (1u << (rel >> 3)) : 0u;
-    const uint32_t A = __reduce_or_sync(0xffffffffu, at_start);
-    const uint32_t B = __reduce_or_sync(0xffffffffu, inside);
-    const int nwin = __popc(__ballot_sync(0xffffffffu, in_win));
-    const bool collide = nwin != __popc(A) + __popc(B) || (A & B) != 0u;  // two boundaries in one half-block
-    const uint32_t le = lane == 31 ? 0xffffffffu : ((2u << lane) - 1u);
-    const int before = __popc(A & le) + __popc(B & (le >> 1));  // boundaries <= q0 in the window
-    const int sgi = s_lo + before;                               // segment of q0
+    const int t = c - w;  // a multiple of 8 (INT_MAX - w off the boundary lanes)
+    const int s_lo = __popc(__ballot_sync(0xffffffffu, t <= 0));
+    const uint32_t A = __reduce_or_sync(0xffffffffu, (uint32_t)(t - 1) < 255u ? (1u << ((t >> 3) & 31)) : 0u);
+    const int sgi = s_lo + __popc(A & le);  // segment of q0
     const int q0 = w + 8 * lane;
-    // the boundary inside this half-block, if any, is segment sgi+1's start
-    const int bn = __shfl_sync(0xffffffffu, b, min(sgi + 1, 31));
-    const int t1 = ((B >> lane) & 1u) ? bn : INT_MAX;
-    const int t2 = collide ? q0 : INT_MAX;  // forces the walk for the whole window
+    // the start of segment sgi+1 is the first boundary after q0
+    const int nxt = __shfl_sync(0xffffffffu, d.ssv, min(sgi + 1, 31));
+    const int t1 = sgi + 1 < nseg ? nxt : INT_MAX;
+    const int t2 = col_walk ? q0 : INT_MAX;  // forces the walk
     if (32 * i + lane < nhb) {
       const uint32_t iw[2] = {d.iv[i].x, d.iv[i].y};
       float a0[MP], a1[MP];
@@ -528,10 +529,9 @@ k_coeff_gather(const __grid_constant__ CoeffBatch batch) {
   // Two column buffers in ping-pong: the next column's loads are in flight while
   // this one is summed, and no buffer is ever copied (a copy would wait for them).
   ColData ca, cbuf;
-  uint32_t pa, pb;
   int na, nb;
   int o = o_begin + warp;
-  load_col(ca, o, o_end, col_ptr, idx, codes, scales, seg_start, nseg, lane, pa, na);
+  load_col(ca, o, o_end, col_ptr, idx, codes, scales, seg_start, nseg, lane, na);
   trigger_dependents();
   grid_dependency_wait();  // Z comes from the dictionary stage
 
@@ -541,10 +541,10 @@ k_coeff_gather(const __grid_constant__ CoeffBatch batch) {
   const uint32_t zs_a = smem_u32(zsg);
 
   for (; o < o_end; o += 2 * kGatherWarps) {
-    load_col(cbuf, o + kGatherWarps, o_end, col_ptr, idx, codes, scales, seg_start, nseg, lane, pb, nb);
+    load_col(cbuf, o + kGatherWarps, o_end, col_ptr, idx, codes, scales, seg_start, nseg, lane, nb);
     gather_column<MP>(ca, o, na, zs_a, nseg, seg_start, lane, M, d_out, s_C, Y);
     if (o + kGatherWarps >= o_end) break;
-    load_col(ca, o + 2 * kGatherWarps, o_end, col_ptr, idx, codes, scales, seg_start, nseg, lane, pa, na);
+    load_col(ca, o + 2 * kGatherWarps, o_end, col_ptr, idx, codes, scales, seg_start, nseg, lane, na);
     gather_column<MP>(cbuf, o + kGatherWarps, nb, zs_a, nseg, seg_start, lane, M, d_out, s_C, Y);
   }
 }
@@ -643,29 +643,39 @@ constexpr size_t kDictXsMax = 96 * 1024;
 
 static size_t dict_xs_bytes(int xlen, int M) { return (size_t)M * (xlen + 8) * sizeof(__half); }
 
-// J of one projection alone: J grows until its grid fits four CTAs per SM
-// (4 x 256 threads x 64 registers fill the register file: the kernel is
-// latency-bound, so resident warps matter most).
-static int dict_lone_J(int d_in, int k, int n_sm) {
-  const int units = (d_in + 127) / 128, tiles = k / kDictTile;
-  int J = 1;
-  while (J < units && (size_t)tiles * ((units + kDictWarps * J - 1) / (kDictWarps * J)) > (size_t)4 * n_sm) ++J;
-  return J;
-}
+// Cost of a dictionary grid in rows of D streamed by one CTA: the launch takes
+// ceil(CTAs / (4 x n_sm)) waves (four 256-thread CTAs fill an SM's registers),
+// each as long as its longest CTA, and a CTA costs a fixed part (launch, X
+// staging, the cross-warp reduction) worth kDictFixedRows rows plus its rows.
+// Fitted on B200 to the LLaMA-7B shapes at M = 1 (q/k/v and gate/up batches, o
+// and down alone, J = 1..8): it picks the fastest J measured for each.
+constexpr long kDictFixedRows = 1700;
 
 void dict_plan_batch(int n, const int* d_in, const int* k, int n_sm, int M, DictPlan* plans) {
-  // One J for the whole batch, the largest any of its projections takes alone:
-  // every CTA then streams the same 8 x J units of 16 atom rows (or all of a
-  // shorter d_in), so each projection's CTAs follow its dictionary bytes
-  // (d_in x k) and the hardware scheduler balances the grid; a batch of equal
-  // shapes gets exactly the lone plan. Per projection, J shrinks back while the
-  // slice's X rows would not fit the shared-memory cap.
-  int J = 1;
-  for (int i = 0; i < n; ++i) J = std::max(J, dict_lone_J(d_in[i], k[i], n_sm));
+  // One J for the whole batch (every CTA then streams the same 8 x J units of 16
+  // atom rows, or all of a shorter d_in, so each projection's CTAs follow its
+  // dictionary bytes), chosen by the cost above. Per projection, J is capped at
+  // the units one slice needs and shrinks back while the slice's X rows would not
+  // fit the shared-memory cap.
+  int jmax = 1;
+  for (int i = 0; i < n; ++i) jmax = std::max(jmax, ((d_in[i] + 127) / 128 + kDictWarps - 1) / kDictWarps);
+  int best = 1;
+  long best_cost = LONG_MAX;
+  for (int J = 1; J <= jmax; ++J) {
+    long ctas = 0, rows = 0;
+    for (int i = 0; i < n; ++i) {
+      const int units = (d_in[i] + 127) / 128;
+      const int slices = (units + kDictWarps * J - 1) / (kDictWarps * J);
+      ctas += (long)(k[i] / kDictTile) * slices;
+      rows = std::max(rows, (long)std::min(d_in[i], kDictWarps * J * 128));
+    }
+    const long cost = (ctas + 4L * n_sm - 1) / (4L * n_sm) * (kDictFixedRows + rows);
+    if (cost < best_cost) best_cost = cost, best = J;
+  }
   for (int i = 0; i < n; ++i) {
     const int units = (d_in[i] + 127) / 128;
     DictPlan& p = plans[i];
-    p.J = std::min(J, units);
+    p.J = std::min(best, (units + kDictWarps - 1) / kDictWarps);
     while (p.J > 1 && dict_xs_bytes(std::min(d_in[i], kDictWarps * p.J * 128), M) > kDictXsMax) --p.J;
     p.slices = (units + kDictWarps * p.J - 1) / (kDictWarps * p.J);
   }
@@ -684,9 +694,9 @@ DictPlan dict_plan(int d_in, int k, int n_sm, int M, bool one_slice) {
 }
 
 int dict_max_slices(int d_in, int k, int n_sm) {
-  int m = 1;
-  for (int M = 1; M <= kDecodeMaxTokens; ++M) m = std::max(m, dict_plan(d_in, k, n_sm, M, false).slices);
-  return m;
+  (void)k;
+  (void)n_sm;
+  return ((d_in + 127) / 128 + kDictWarps - 1) / kDictWarps;  // J = 1, the most any plan takes
 }
 
 cudaError_t prepare_decode_kernels(int device) {
@@ -704,7 +714,6 @@ cudaError_t prepare_decode_kernels(int device) {
       return e;                                                                                       \
   }
   SET_SMEM((k_dict_decode<1, true>));
-  SET_SMEM((k_dict_decode<2, true>));
   SET_SMEM(k_coeff_gather<1>);
   SET_SMEM(k_coeff_gather<2>);
   SET_SMEM(k_coeff_gather<4>);
@@ -723,7 +732,7 @@ cudaError_t launch_dict_decode_batch(int n, const dictproj_group* const* g, cons
   b.n = n;
   b.M = M;
   b.mp = mp;
-  int blocks = 0, maxJ = 1;
+  int blocks = 0;
   size_t xs = 0;
   for (int i = 0; i < n; ++i) {
     DictProj& p = b.p[i];
@@ -738,19 +747,16 @@ cudaError_t launch_dict_decode_batch(int n, const dictproj_group* const* g, cons
     p.tiles = g[i]->k / kDictTile;
     p.block_begin = blocks;
     blocks += p.tiles * plans[i].slices;
-    maxJ = std::max(maxJ, p.J);
     xs = std::max(xs, dict_xs_bytes(std::min(p.d_in, kDictWarps * p.J * 128), M));
   }
   void* args[] = {(void*)&b};
   const dim3 grid(blocks), block(kDictWarps * 32);
   const bool use_xs = xs <= 200 * 1024;
   const size_t smem = use_xs ? xs : 0;
-#define DICT_LAUNCH(R)                                                                                \
-  return use_xs ? launch_pdl((const void*)k_dict_decode<R, true>, grid, block, smem, stream, args)     \
-                : launch_pdl((const void*)k_dict_decode<R, false>, grid, block, 0, stream, args);
-  if (maxJ == 1) DICT_LAUNCH(1)
-  DICT_LAUNCH(2)
-#undef DICT_LAUNCH
+  // One unit in flight per warp (RING = 1): on B200 it measured as fast as two or
+  // four for J = 2..8, with the CTA's slice already on its way to L2.
+  return use_xs ? launch_pdl((const void*)k_dict_decode<1, true>, grid, block, smem, stream, args)
+                : launch_pdl((const void*)k_dict_decode<1, false>, grid, block, 0, stream, args);
 }
 
 cudaError_t launch_dict_decode(const dictproj_group* g, const __half* X, int M, int mp, float* Zpart,
