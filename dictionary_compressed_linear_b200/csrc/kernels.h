@@ -20,8 +20,9 @@ struct DictPlan {
   int slices;  // d_in slices = grid.y
 };
 DictPlan dict_plan(int d_in, int k, int n_sm, int M, bool one_slice);
-// One plan for a batched launch: a common J, so CTAs per projection follow its
-// dictionary bytes; never more slices than dict_plan gives each alone.
+// One plan for a batched launch: a common J, chosen by a fitted cost (waves x
+// (fixed + rows per CTA)), so CTAs per projection follow its dictionary bytes;
+// never more slices than J = 1 gives (dict_max_slices, the group's Z scratch).
 void dict_plan_batch(int n, const int* d_in, const int* k, int n_sm, int M, DictPlan* plans);
 // CTAs of a batched gather launch per projection, in proportion to its stored
 // entries, at least one each.
@@ -96,6 +97,12 @@ cudaError_t encode_dict_codes_map(const dictproj_group* g, CUtensorMap* map);
 // `other` tiles along the other side, n_sm SMs (prefill GEMM grids).
 int prefill_tile_width(long extent, long other, int n_sm);
 // Z = s_D X D^ (fp16 out, s_D applied in fp32 before rounding)
+// Grid of the prefill dictionary stage: token-tile width nt and the number of
+// CTAs (one cluster) the d_in stages of a tile are split over (1: no split).
+struct PrefillDictPlan {
+  int nt, splits;
+};
+PrefillDictPlan prefill_dict_plan(int M, int d_in, int k, int n_sm);
 cudaError_t launch_dict_prefill(const dictproj_group* g, const __half* X, int M, __half* Z, cudaStream_t stream);
 // Cd[o][a] = C^ densified to fp16 (zeros off the support), [d_out][k]
 cudaError_t launch_densify_coeff(const dictproj_layer* l, __half* Cd, cudaStream_t stream);

@@ -26,6 +26,7 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <atomic>
 #include <mutex>
 
 #include "common.cuh"
@@ -55,6 +56,22 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map
       "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];"
       ::"r"(dst), "l"(map), "r"(x), "r"(y), "r"(smem_u32(bar))
       : "memory");
+}
+// Thread-block cluster: barrier over all threads of all CTAs, and loads from
+// another CTA's shared memory (distributed shared memory).
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+__device__ __forceinline__ uint32_t map_dsmem(uint32_t local, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(local), "r"(rank));
+  return r;
+}
+__device__ __forceinline__ float4 ld_dsmem_v4f(uint32_t addr) {
+  float4 v;
+  asm volatile("ld.shared::cluster.v4.f32 {%0,%1,%2,%3}, [%4];" : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "r"(addr)
+               : "memory");
+  return v;
 }
 __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
@@ -271,6 +288,11 @@ struct DictTile {
   static constexpr size_t smem = (size_t)kStages * (kXBytes + kRawBytes) + 1024 + 256;
 };
 
+// Split-K (small M): with gridDim.z = S > 1 the S CTAs of a cluster (1, 1, S)
+// take consecutive ranges of the d_in stages of one (atom tile, token tile);
+// each leaves its fp32 partial tile in its own shared memory, and CTA r of the
+// cluster sums the S partials of its share of the token columns in rank order
+// over distributed shared memory (deterministic), applies s_D and writes Z.
 __global__ void __launch_bounds__(DictTile::kThreads, 1)
     k_dict_prefill(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_codes,
                    const uint8_t* __restrict__ scales, int M, int k, int d_in, int nt, float s_D,
@@ -290,7 +312,10 @@ __global__ void __launch_bounds__(DictTile::kThreads, 1)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int a0 = blockIdx.x * kTA, m0 = blockIdx.y * nt;
-  const int nk = (d_in + BK - 1) / BK;
+  const int nsplit = (int)gridDim.z, split = (int)blockIdx.z;
+  const int nk_all = (d_in + BK - 1) / BK;
+  const int s_lo = (int)((long)nk_all * split / nsplit);  // this CTA's stages [s_lo, s_lo + nk)
+  const int nk = (int)((long)nk_all * (split + 1) / nsplit) - s_lo;
   // kind::f16, A and B fp16, D fp32, K-major, M = 128 atoms, N = nt tokens
   const uint32_t idesc = (1u << 4) | ((uint32_t)(nt >> 3) << 17) | ((uint32_t)(kTA >> 4) << 24);
 
@@ -316,8 +341,8 @@ __global__ void __launch_bounds__(DictTile::kThreads, 1)
         const int slot = s % S, round = s / S;
         if (s >= S && !mbar_wait_bounded(&empty[slot], (round - 1) & 1)) break;
         mbar_arrive_expect_tx(&full[slot], nt * BK * 2 + T::kRawBytes);
-        tma_load_2d(smem_u32(sx + slot * T::kXBytes), &tm_x, s * BK, m0, &full[slot]);
-        tma_load_2d(smem_u32(sr + slot * T::kRawBytes), &tm_codes, s * (BK / 2), a0, &full[slot]);
+        tma_load_2d(smem_u32(sx + slot * T::kXBytes), &tm_x, (s_lo + s) * BK, m0, &full[slot]);
+        tma_load_2d(smem_u32(sr + slot * T::kRawBytes), &tm_codes, (s_lo + s) * (BK / 2), a0, &full[slot]);
       }
     }
   } else if (warp == 1) {
@@ -350,8 +375,8 @@ __global__ void __launch_bounds__(DictTile::kThreads, 1)
     // indexed statically (the loop over it is unrolled): moving a register whose
     // load is still in flight would wait for that load.
     constexpr int G = T::kGroups, R = kScaleAhead;
-    auto scale_at = [&](int st) -> uint32_t {
-      return (row_ok && 4 * st + 2 * h < nblk) ? ld_stream_u16(srow + 4 * st) : 0u;
+    auto scale_at = [&](int st) -> uint32_t {  // st: this CTA's stage number
+      return (row_ok && st < nk && 4 * (s_lo + st) + 2 * h < nblk) ? ld_stream_u16(srow + 4 * (s_lo + st)) : 0u;
     };
     uint32_t scr[R];
 #pragma unroll
@@ -392,11 +417,19 @@ __global__ void __launch_bounds__(DictTile::kThreads, 1)
     const bool ok = mbar_wait_bounded(accf, 0);
     tc_fence_after();
     const int lim = min(nt, M - m0);  // valid token columns of this tile
+    // split-K: the partial tile goes to this CTA's shared memory, token-major
+    // (the stage buffers are idle once the accumulator is complete)
+    float* part = reinterpret_cast<float*>(smem);
 #pragma unroll 1
     for (int c = e >> 2; 32 * c < nt; c += 2 * G) {
       const int col = 32 * c;
       uint32_t v[32];
       tmem_ld32(tmem + lane_base + col, v);
+      if (nsplit > 1) {
+#pragma unroll
+        for (int j = 0; j < 32; ++j) part[(col + j) * kTA + r] = ok ? __uint_as_float(v[j]) : 0.f;
+        continue;
+      }
       if (!ok || !row_ok) continue;
       __half* zc = Z + (size_t)(m0 + col) * k + a0 + r;
 #pragma unroll
@@ -411,6 +444,32 @@ __global__ void __launch_bounds__(DictTile::kThreads, 1)
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem, T::kCols);
+  }
+  if (nsplit > 1) {
+    // every partial is in place: CTA `split` sums its token columns over the
+    // cluster's CTAs in rank order, four atoms per thread
+    cluster_sync_all();
+    const int lim = min(nt, M - m0);
+    const int c_lo = (int)((long)nt * split / nsplit), c_hi = (int)((long)nt * (split + 1) / nsplit);
+    const uint32_t pbase = smem_u32(smem);
+    for (int i = threadIdx.x; i < (c_hi - c_lo) * (kTA / 4); i += blockDim.x) {
+      const int col = c_lo + i / (kTA / 4), a4 = 4 * (i % (kTA / 4));
+      const uint32_t off = (uint32_t)(col * kTA + a4) * 4u;
+      float4 acc = ld_dsmem_v4f(map_dsmem(pbase + off, 0));
+      for (int rk = 1; rk < nsplit; ++rk) {
+        const float4 q = ld_dsmem_v4f(map_dsmem(pbase + off, (uint32_t)rk));
+        acc.x += q.x;
+        acc.y += q.y;
+        acc.z += q.z;
+        acc.w += q.w;
+      }
+      if (col < lim && a0 + a4 < k) {  // k % 16 == 0: the four atoms are all in range
+        __half2* zc = reinterpret_cast<__half2*>(Z + (size_t)(m0 + col) * k + a0 + a4);
+        zc[0] = __floats2half2_rn(acc.x * s_D, acc.y * s_D);
+        zc[1] = __floats2half2_rn(acc.z * s_D, acc.w * s_D);
+      }
+    }
+    cluster_sync_all();  // no CTA leaves while another still reads its partial tile
   }
 }
 
@@ -610,20 +669,92 @@ int prefill_tile_width(long extent, long other, int n_sm) {
   return best;
 }
 
+// Clusters of S CTAs of the prefill dictionary kernel (one CTA per SM at its
+// shared memory) that the device holds at once, from the occupancy query;
+// cached per device and S.
+static int dict_clusters_that_fit(int S) {
+  static std::atomic<int> cache[16][9];
+  static std::once_flag once;
+  std::call_once(once, [] {
+    for (auto& d : cache)
+      for (auto& c : d) c.store(-1);
+  });
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 16 || S < 1 || S > 8) return 0;
+  int v = cache[dev][S].load();
+  if (v >= 0) return v;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(1, 1, S);
+  cfg.blockDim = dim3(DictTile::kThreads);
+  cfg.dynamicSmemBytes = DictTile::smem;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 1;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = (unsigned)S;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, (const void*)k_dict_prefill, &cfg) != cudaSuccess) {
+    cudaGetLastError();
+    n = 0;
+  }
+  cache[dev][S].store(n);
+  return n;
+}
+
+PrefillDictPlan prefill_dict_plan(int M, int d_in, int k, int n_sm) {
+  PrefillDictPlan p;
+  const int tiles_a = (k + kTA - 1) / kTA, nk = (d_in + BK - 1) / BK;
+  p.nt = prefill_tile_width(M, tiles_a, n_sm);
+  p.splits = 1;
+  if (M <= 2 * DictTile::kMaxN) {
+    // Few tokens: the d_in stages split over a cluster of up to 8 CTAs (each at
+    // least 4 stages), so that the grid fills the GPU without every token tile
+    // decoding the same dictionary tile again. Of the splits whose clusters are
+    // all resident at once, the one with the most CTAs; ties go to fewer token
+    // tiles (less decoding).
+    int best = 0;
+    for (int tm = (M + DictTile::kMaxN - 1) / DictTile::kMaxN; tm <= 4; tm *= 2) {
+      const int nt = ((M + tm - 1) / tm + 15) / 16 * 16;
+      if (nt < 16 || (M + nt - 1) / nt != tm) break;
+      const int tiles = tiles_a * tm;
+      for (int S = std::min({8, n_sm / tiles, nk / 4}); S >= 2; --S)
+        if (dict_clusters_that_fit(S) >= tiles) {
+          if (tiles * S > best) {
+            best = tiles * S;
+            p.nt = nt;
+            p.splits = S;
+          }
+          break;
+        }
+    }
+  }
+  return p;
+}
+
 cudaError_t launch_dict_prefill(const dictproj_group* g, const __half* X, int M, __half* Z, cudaStream_t stream) {
-  int nt = prefill_tile_width(M, (g->k + kTA - 1) / kTA, g->n_sm);
+  const PrefillDictPlan plan = prefill_dict_plan(M, g->d_in, g->k, g->n_sm);
+  int nt = plan.nt;
   CUtensorMap tx;
   cudaError_t e = encode_2d(&tx, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, X, (uint64_t)g->d_in, (uint64_t)M,
                             (uint64_t)g->d_in * 2, BK, nt, CU_TENSOR_MAP_SWIZZLE_128B);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((g->k + kTA - 1) / kTA, (M + nt - 1) / nt);
+  cfg.gridDim = dim3((g->k + kTA - 1) / kTA, (M + nt - 1) / nt, plan.splits);
   cfg.blockDim = dim3(DictTile::kThreads);
   cfg.dynamicSmemBytes = DictTile::smem;
   cfg.stream = stream;
-  cudaLaunchAttribute attr[1] = {pdl_attr()};
+  cudaLaunchAttribute attr[2] = {pdl_attr(), {}};
   cfg.attrs = attr;
   cfg.numAttrs = 1;
+  if (plan.splits > 1) {  // the split CTAs of a tile form one cluster
+    attr[1].id = cudaLaunchAttributeClusterDimension;
+    attr[1].val.clusterDim.x = 1;
+    attr[1].val.clusterDim.y = 1;
+    attr[1].val.clusterDim.z = (unsigned)plan.splits;
+    cfg.numAttrs = 2;
+  }
   const uint8_t* sc = g->scales;
   int k = g->k, d_in = g->d_in;
   float s = g->s;
