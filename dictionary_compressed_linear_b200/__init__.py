@@ -13,7 +13,7 @@ from .binding import (  # noqa: F401
     dictproj_layer_upload_blocks, dictproj_pack_layer_blocks, dictproj_layer_index_format, dictproj_layer_export_bitmap,
     dictproj_layer_export_blocks, DeviceGroup, DeviceLayer, DictprojError, Group, Layer, LIB_PATH,
     SIGNATURES, dictproj_forward_noalloc, dictproj_forward_noalloc_status, lib,
-    dictproj_check, dictproj_check_status, dictproj_diag_phase_times, dictproj_launch_count, dictproj_selftest_wait_timeout, dictproj_coefficient_stage, dictproj_dictionary_stage, dictproj_dictionary_stage_prefill,
+    dictproj_check, dictproj_check_status, dictproj_diag_phase_times, dictproj_diag_gather_times, dictproj_launch_count, dictproj_selftest_wait_timeout, dictproj_coefficient_stage, dictproj_dictionary_stage, dictproj_dictionary_stage_prefill,
     dictproj_group_reserve_prefill, dictproj_forward, dictproj_rank_for_budget, dictproj_budget,
     dictproj_group_file_write, dictproj_group_file_read, dictproj_layer_file_write, dictproj_layer_file_read,
     dictproj_group_save, dictproj_group_load, dictproj_layer_save, dictproj_layer_load, dictproj_forward_batch, dictproj_forward_batch_stages, dictproj_decode_batch_plan, dictproj_forward_path, dictproj_forward_status,

@@ -144,6 +144,7 @@ SIGNATURES = [
     ("dictproj_check", C.c_int, [C.c_void_p]),
     ("dictproj_selftest_wait_timeout", C.c_int, [C.c_longlong, C.c_void_p]),
     ("dictproj_diag_phase_times", C.c_int, [C.POINTER(C.c_ulonglong), C.c_int, _intp]),
+    ("dictproj_diag_gather_times", C.c_int, [C.c_void_p, C.c_int]),
     ("dictproj_last_error", C.c_char_p, []),
     ("dictproj_status_string", C.c_char_p, [C.c_int]),
     ("dictproj_version", C.c_int, []),
@@ -750,6 +751,12 @@ def dictproj_launch_count(X_ptrs, M: int, layers, groups) -> int:
                                        arr(*[l.handle for l in layers]), arr(*[g.handle for g in groups]),
                                        C.byref(cnt)))
     return cnt.value
+
+
+def dictproj_diag_gather_times(buf_ptr: int, max_ctas: int):
+    """Arm (device buffer of 2 * max_ctas u64) or disarm (buf_ptr 0) the gather
+    kernel's per-CTA start / end timestamps."""
+    _check(lib().dictproj_diag_gather_times(C.c_void_p(buf_ptr or None), max_ctas))
 
 
 def dictproj_diag_phase_times(max_ctas: int = 1024) -> np.ndarray:

@@ -1020,16 +1020,18 @@ int dictproj_decode_batch_plan(int n, const int* d_in, const int* k, const int* 
   if (M < 1 || M > kDecodeMaxTokens) return fail(DICTPROJ_ERR_RANGE, "decode_batch_plan: M=%d outside [1, %d]", M, kDecodeMaxTokens);
   if (n_sm < 1) return fail(DICTPROJ_ERR_RANGE, "decode_batch_plan: n_sm=%d < 1", n_sm);
   size_t ent[kDecodeMaxBatch];
+  int cols[kDecodeMaxBatch];
   for (int i = 0; i < n; ++i) {
     if (d_in[i] < 16 || d_in[i] % 16 || k[i] < 16 || k[i] % 16 || d_out[i] < 1)
       return fail(DICTPROJ_ERR_SHAPE, "decode_batch_plan: entry %d has d_in=%d k=%d d_out=%d", i, d_in[i], k[i], d_out[i]);
     if (entries[i] < 0) return fail(DICTPROJ_ERR_RANGE, "decode_batch_plan: entry %d has %lld entries", i, entries[i]);
     ent[i] = (size_t)entries[i];
+    cols[i] = d_out[i];
   }
   DictPlan plans[kDecodeMaxBatch];
   dict_plan_batch(n, d_in, k, n_sm, M, plans);
   int share[kDecodeMaxBatch];
-  gather_batch_shares(n, ent, n_sm, share);
+  gather_batch_shares(n, ent, cols, n_sm, share);
   for (int i = 0; i < n; ++i) {
     dict_ctas[i] = (k[i] / 16) * plans[i].slices;
     dict_slices[i] = plans[i].slices;
@@ -1139,6 +1141,16 @@ int dictproj_diag_phase_times(unsigned long long* out, int max_ctas, int* n_ctas
   if ((st = ensure_device(&dev))) return st;
   cudaError_t e = fused_phase_times(out, max_ctas, n_ctas);
   return e == cudaSuccess ? DICTPROJ_OK : cuda_fail(e, "diag_phase_times");
+}
+
+int dictproj_diag_gather_times(unsigned long long* buf, int max_ctas) {
+  clear_error();
+  if (buf && max_ctas < 1) return fail(DICTPROJ_ERR_RANGE, "diag_gather_times: max_ctas=%d < 1", max_ctas);
+  if (((uintptr_t)buf & 7) != 0) return fail(DICTPROJ_ERR_ALIGN, "diag_gather_times: buf must be 8-byte aligned");
+  int dev, st;
+  if ((st = ensure_device(&dev))) return st;
+  cudaError_t e = set_gather_times(buf, max_ctas);
+  return e == cudaSuccess ? DICTPROJ_OK : cuda_fail(e, "diag_gather_times");
 }
 
 int dictproj_check(void* stream) {

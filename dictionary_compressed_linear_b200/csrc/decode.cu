@@ -499,10 +499,22 @@ __device__ __forceinline__ void gather_column(const ColData& d, int o, int nhb, 
   }
 }
 
+// Diagnostic: when set, each gather CTA writes the start of its column work (Z
+// staged) and its end (the GPU's global timer, ns) to g_gather_times[2 * CTA]
+// and [2 * CTA + 1], CTA < g_gather_ctas.
+static __constant__ unsigned long long* g_gather_times;
+static __constant__ int g_gather_ctas;
+__device__ __forceinline__ unsigned long long global_ns() {
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
 template <int MP>
 __global__ void __launch_bounds__(kGatherWarps * 32, 1)  // 1024 threads, at most 64 registers
 k_coeff_gather(const __grid_constant__ CoeffBatch batch) {
   extern __shared__ __align__(16) __half zsg[];  // fp16 [k + 256][MP]; the tail is zero
+  unsigned long long* const tdiag = (int)blockIdx.x < g_gather_ctas ? g_gather_times : nullptr;
   int pi = 0;
   while (pi + 1 < batch.n && (int)blockIdx.x >= batch.p[pi + 1].block_begin) ++pi;
   const CoeffProj& pr = batch.p[pi];
@@ -539,6 +551,7 @@ k_coeff_gather(const __grid_constant__ CoeffBatch batch) {
   for (int i = k * MP + threadIdx.x; i < (k + 256) * MP; i += blockDim.x) zsg[i] = __float2half_rn(0.f);
   __syncthreads();
   const uint32_t zs_a = smem_u32(zsg);
+  if (tdiag && threadIdx.x == 0) tdiag[2 * blockIdx.x] = global_ns();
 
   for (; o < o_end; o += 2 * kGatherWarps) {
     load_col(cbuf, o + kGatherWarps, o_end, col_ptr, idx, codes, scales, seg_start, nseg, lane, nb);
@@ -546,6 +559,10 @@ k_coeff_gather(const __grid_constant__ CoeffBatch batch) {
     if (o + kGatherWarps >= o_end) break;
     load_col(ca, o + 2 * kGatherWarps, o_end, col_ptr, idx, codes, scales, seg_start, nseg, lane, na);
     gather_column<MP>(cbuf, o + kGatherWarps, nb, zs_a, nseg, seg_start, lane, M, d_out, s_C, Y);
+  }
+  if (tdiag) {  // the same for every thread of the CTA
+    __syncthreads();
+    if (threadIdx.x == 0) tdiag[2 * blockIdx.x + 1] = global_ns();
   }
 }
 
@@ -770,17 +787,34 @@ bool decode_batch_gathers(int n, const dictproj_layer* const* l) {
   return all;
 }
 
-void gather_batch_shares(int n, const size_t* entries, int n_sm, int* share) {
-  // CTAs of a batched gather launch shared out in proportion to each projection's
-  // stored entries (its coefficient bytes), at least one each, n_sm in all
-  double wsum = 0.0;
-  for (int i = 0; i < n; ++i) wsum += (double)entries[i] + 1.0;
-  int given = 0;
-  for (int i = 0; i < n; ++i) {
-    share[i] = std::max(1, (int)((double)n_sm * ((double)entries[i] + 1.0) / wsum));
-    given += share[i];
+// Time of a projection's CTAs in the gather kernel, in units of one 256-entry
+// window of one warp: a warp takes whole columns, ceil(ceil(columns / CTAs) / 32)
+// of them, and a column costs a fixed part worth two windows (its loads and
+// addresses, the reduction and store; 1.06 us against 0.52 us per window,
+// measured on B200) plus its windows, ceil(entries per column / 256).
+static double gather_cta_time(size_t entries, int columns, int ctas, bool quantised) {
+  const size_t epc = (entries + (size_t)std::max(1, columns) - 1) / (size_t)std::max(1, columns);
+  const double cost = 2.0 + (double)((epc + 255) / 256);
+  if (!quantised) return (double)columns / ctas / kGatherWarps * cost;
+  const int cols = (columns + ctas - 1) / ctas;
+  return (double)((cols + kGatherWarps - 1) / kGatherWarps) * cost;
+}
+
+void gather_batch_shares(int n, const size_t* entries, const int* columns, int n_sm, int* share) {
+  // CTAs of a batched gather launch: one each, then one at a time to the
+  // projection that would finish last (largest quantised time, then largest
+  // smooth time), so that the launch ends as early as the cost allows; n_sm in all
+  for (int i = 0; i < n; ++i) share[i] = 1;
+  for (int given = n; given < n_sm; ++given) {
+    int worst = 0;
+    double wq = -1.0, ws = -1.0;
+    for (int i = 0; i < n; ++i) {
+      const double q = gather_cta_time(entries[i], columns[i], share[i], true);
+      const double sm = gather_cta_time(entries[i], columns[i], share[i], false);
+      if (q > wq || (q == wq && sm > ws)) worst = i, wq = q, ws = sm;
+    }
+    ++share[worst];
   }
-  for (int i = 0; given < n_sm; i = (i + 1) % n, ++given) ++share[i];  // the rounding remainder
 }
 
 static cudaError_t launch_gather_batch(int n, const dictproj_layer* const* l, const float* const* Zpart,
@@ -790,9 +824,9 @@ static cudaError_t launch_gather_batch(int n, const dictproj_layer* const* l, co
   b.M = M;
   int blocks = 0, kmax = 0;
   size_t entries[kMaxBatch];
-  int share[kMaxBatch];
-  for (int i = 0; i < n; ++i) entries[i] = l[i]->total;
-  gather_batch_shares(n, entries, l[0]->n_sm, share);
+  int columns[kMaxBatch], share[kMaxBatch];
+  for (int i = 0; i < n; ++i) entries[i] = l[i]->total, columns[i] = l[i]->d_out;
+  gather_batch_shares(n, entries, columns, l[0]->n_sm, share);
   for (int i = 0; i < n; ++i) {
     CoeffProj& p = b.p[i];
     p.col_ptr = l[i]->col_ptr;
@@ -888,6 +922,13 @@ __global__ void k_wait_probe(long long cycles) {
 cudaError_t launch_wait_probe(long long cycles, cudaStream_t stream) {
   k_wait_probe<<<1, 32, 0, stream>>>(cycles);
   return cudaGetLastError();
+}
+
+cudaError_t set_gather_times(unsigned long long* buf, int max_ctas) {
+  cudaError_t e = cudaMemcpyToSymbol(g_gather_times, &buf, sizeof(buf));
+  if (e != cudaSuccess) return e;
+  const int n = buf ? max_ctas : 0;
+  return cudaMemcpyToSymbol(g_gather_ctas, &n, sizeof(n));
 }
 
 cudaError_t take_decode_error(unsigned int* out) {

@@ -24,9 +24,11 @@ DictPlan dict_plan(int d_in, int k, int n_sm, int M, bool one_slice);
 // (fixed + rows per CTA)), so CTAs per projection follow its dictionary bytes;
 // never more slices than J = 1 gives (dict_max_slices, the group's Z scratch).
 void dict_plan_batch(int n, const int* d_in, const int* k, int n_sm, int M, DictPlan* plans);
-// CTAs of a batched gather launch per projection, in proportion to its stored
-// entries, at least one each.
-void gather_batch_shares(int n, const size_t* entries, int n_sm, int* share);
+// CTAs of a batched gather launch per projection (n_sm in all, at least one
+// each), given each projection's stored entries and columns: handed out so that
+// the projection that would finish last gets the next one (a fitted cost per
+// column and per 256-entry window, whole columns per warp).
+void gather_batch_shares(int n, const size_t* entries, const int* columns, int n_sm, int* share);
 int dict_max_slices(int d_in, int k, int n_sm);  // over all decode M
 cudaError_t launch_dict_decode(const dictproj_group* g, const __half* X, int M, int mp, float* Zpart,
                                const DictPlan& plan, cudaStream_t stream);
@@ -51,6 +53,8 @@ bool coeff_smem_fits(int k, int mp, int device);
 cudaError_t launch_wait_probe(long long cycles, cudaStream_t stream);
 // Read and clear the device error word of the decode kernels.
 cudaError_t take_decode_error(unsigned int* out);
+// Diagnostic timestamps of the gather kernel (buf null: off).
+cudaError_t set_gather_times(unsigned long long* buf, int max_ctas);
 cudaError_t take_fused_error(unsigned int* out);
 
 // fused decode path (M <= 8): one kernel per call, both stages, weights staged

@@ -342,8 +342,11 @@ int dictproj_forward_batch_stages(int n, const void* const* X, int M, const dict
  * dict_slices[i], the dictionary kernel's CTAs and d_in slices for projection i
  * (every CTA streams the same number of dictionary rows, so CTAs follow
  * d_in x k), and coeff_ctas[i], the coefficient kernel's CTAs for projection i
- * (in proportion to entries[i], at least one, n_sm in all before rounding
- * columns up). Errors: NULL, RANGE (n, M, n_sm, entries < 0), SHAPE. */
+ * (n_sm in all before rounding columns up, at least one each, handed out one at a
+ * time to the projection whose CTAs would finish last by a cost of whole columns
+ * per warp, each column a fixed part worth two 256-entry windows plus its
+ * windows; equal projections get equal shares).
+ * Errors: NULL, RANGE (n, M, n_sm, entries < 0), SHAPE. */
 int dictproj_decode_batch_plan(int n, const int* d_in, const int* k, const int* d_out, const long long* entries,
                                int M, int n_sm, int* dict_ctas, int* dict_slices, int* coeff_ctas);
 
@@ -496,6 +499,17 @@ int dictproj_check(void* stream);
  * resolved, last copy issued; 12-15 unused. Synchronise the stream first.
  * Errors: NULL, RANGE, UNSUPPORTED, CUDA. */
 int dictproj_diag_phase_times(unsigned long long* out, int max_ctas, int* n_ctas);
+
+/* Diagnostic (no counterpart in the paper): while armed, every launch of the
+ * decode gather kernel (the coefficient stage of the two-kernel path) writes, for
+ * each of its CTAs c < max_ctas, the GPU's global timer (ns) when the CTA's
+ * column work starts (its Z table staged) to buf[2c] and at its end to
+ * buf[2c + 1]. buf is caller-owned device memory of 2 * max_ctas u64, 8-byte
+ * aligned; buf = NULL disarms. The CTAs of a batched launch are the projections'
+ * CTAs in order (dictproj_decode_batch_plan gives how many each has). Set it
+ * between calls, not while kernels run.
+ * Errors: RANGE (max_ctas < 1 with a buffer), ALIGN, UNSUPPORTED, CUDA. */
+int dictproj_diag_gather_times(unsigned long long* buf, int max_ctas);
 
 /* Self-test of the bounded-wait error path (diagnostic; no counterpart in the
  * paper). Launches one warp on `stream` that waits on an mbarrier which can never

@@ -309,6 +309,54 @@ def test_mixed_shape_batch_with_byte_proportional_grid(M):
     assert all(p["dict_ctas"] >= 1 and p["coeff_ctas"] >= 1 for p in plan)
 
 
+def test_batched_projections_finish_together():
+    # a q/k/v-like batch (4096 -> 32768 columns, so that the work spans tens of
+    # microseconds against the global timer's ticks) with C densities 0.2 / 0.3 /
+    # 0.4: the gather kernel hands its CTAs out so that the projection that would
+    # finish last gets the next one (a warp takes whole columns; a column costs two
+    # 256-entry windows plus its windows). Measured from the start of their column
+    # work (device timestamps of the gather kernel's CTAs, median of 5 launches),
+    # the three projections finish within 10% of each other, and within 10% of
+    # the spread that cost predicts
+    rhos = (0.2, 0.3, 0.4)
+    projs = []
+    for i, rho in enumerate(rhos):
+        D, C = _case(24, i, i, 0, 4096, 2048, 32768, rho)
+        projs.append(device_projection(D, C, max_tokens=8))
+    X = torch.from_numpy(synth.gen_activations(24, 0, 0, 1, 4096)).cuda()
+    Ys = [torch.empty((1, 32768), dtype=torch.float16, device="cuda") for _ in rhos]
+    st = torch.cuda.current_stream().cuda_stream
+    call = lambda: dp.dictproj_forward_batch([X.data_ptr()] * 3, 1, [p[1] for p in projs], [p[0] for p in projs],
+                                             [y.data_ptr() for y in Ys], st)
+    n_sm = torch.cuda.get_device_properties(0).multi_processor_count
+    totals = [dp.dictproj_layer_info(l)["total"] for _, l in projs]
+    plan = dp.dictproj_decode_batch_plan([(4096, 2048, 32768, t) for t in totals], 1, n_sm)
+    ctas = [p["coeff_ctas"] for p in plan]
+    model = [-(-(-(-32768 // n)) // 32) * (2 + (t / 32768 + 128) / 256) for n, t in zip(ctas, totals)]
+    buf = torch.zeros(2 * sum(ctas), dtype=torch.int64, device="cuda")
+    call()
+    torch.cuda.synchronize()
+    ratios, last = [], []
+    dp.dictproj_diag_gather_times(buf.data_ptr(), sum(ctas))
+    try:
+        for _ in range(5):
+            buf.zero_()
+            call()
+            torch.cuda.synchronize()
+            t = buf.view(-1, 2).cpu().numpy().astype(np.float64)
+            assert np.all(t[:, 1] >= t[:, 0]) and np.all(t[:, 0] > 0)
+            start, b, ends = t[:, 0].min(), 0, []
+            for n in ctas:
+                ends.append(t[b:b + n, 1].max() - start)
+                b += n
+            ratios.append(max(ends) / min(ends))
+            last.append(ends)
+    finally:
+        dp.dictproj_diag_gather_times(0, 0)
+    r = float(np.median(ratios))
+    assert r <= 1.10 and r <= max(model) / min(model) * 1.10, (ratios, model, ctas, last)
+
+
 def test_batch_rejects_repeated_group():
     D = synth.gen_dictionary(17, 0, 0, 64, 32)
     C = synth.gen_coeff(17, 0, 0, 0, 32, 16, 0.5)

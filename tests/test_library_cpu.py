@@ -299,7 +299,7 @@ def test_batched_decode_grid_follows_each_projections_bytes(dp):
     # rows per CTA)); on the LLaMA-7B shapes that is the fastest J measured: one
     # slice for the q/k/v and gate/up batches, J = 1 for o alone, three slices for
     # down. A mixed batch streams about the same rows per CTA in every projection,
-    # and the coefficient kernel's CTAs follow stored entries.
+    # and the coefficient kernel's CTAs go where the batch would otherwise finish last.
     n_sm = 148
     qkv = (4096, 2048, 4096, 4096 * 624)
     gate = (4096, 3072, 11008, 11008 * 784)
@@ -319,10 +319,15 @@ def test_batched_decode_grid_follows_each_projections_bytes(dp):
     for (d_in, k, _, _), p in zip(mixed, plan):
         assert p["dict_ctas"] == (k // 16) * p["dict_slices"]
         assert p["dict_slices"] <= -(-d_in // 1024)  # at most the J = 1 slices the group's Z scratch holds
-    ent = [e for _, _, _, e in mixed]
-    per_cta = [e / p["coeff_ctas"] for e, p in zip(ent, plan)]
-    assert max(per_cta) / min(per_cta) < 1.1
-    assert sum(p["coeff_ctas"] for p in plan) <= n_sm
+    assert sum(p["coeff_ctas"] for p in plan) <= n_sm and all(p["coeff_ctas"] >= 1 for p in plan)
+    # the gather's CTAs go one at a time to the projection that would finish last
+    # (whole columns per warp; a column costs two 256-entry windows plus its
+    # windows): at densities 0.2 / 0.3 / 0.4 over 32768 columns the sparser
+    # projections get more CTAs per stored entry than a split by entries would give
+    wide = [(4096, 2048, 32768, 32768 * e) for e in (416, 624, 832)]
+    shares = [p["coeff_ctas"] for p in dp.dictproj_decode_batch_plan(wide, 1, n_sm)]
+    assert shares == [40, 49, 59], shares
+    assert sum(shares) == n_sm
     tiny = dp.dictproj_decode_batch_plan([(64, 32, 8, 16), (4096, 2048, 4096, 10 ** 7)], 1, n_sm)
     assert tiny[0]["coeff_ctas"] >= 1 and tiny[0]["dict_slices"] == 1
     with pytest.raises(dp.DictprojError):
