@@ -334,3 +334,20 @@ def test_batched_decode_grid_follows_each_projections_bytes(dp):
         dp.dictproj_decode_batch_plan([qkv], 9, n_sm)
     with pytest.raises(dp.DictprojError):
         dp.dictproj_decode_batch_plan([(4096, 2047, 16, 0)], 1, n_sm)
+
+
+def test_stage_mask_and_diagnostic_calls_validate_on_the_host(dp):
+    # the stage mask and the timestamp buffer are checked before any device call,
+    # so these run without a GPU
+    import ctypes as C
+    lib = C.CDLL(dp.LIB_PATH)
+    lib.dictproj_forward_batch_stages.restype = C.c_int
+    lib.dictproj_forward_batch_stages.argtypes = [C.c_int, C.c_void_p, C.c_int, C.c_void_p, C.c_void_p, C.c_void_p,
+                                                  C.c_void_p, C.c_int]
+    for bad in (0, 4, -1):
+        assert lib.dictproj_forward_batch_stages(1, None, 1, None, None, None, None, bad) == -5
+    assert lib.dictproj_forward_batch_stages(1, None, 1, None, None, None, None, 3) == -1  # NULL arrays
+    lib.dictproj_diag_gather_times.restype = C.c_int
+    lib.dictproj_diag_gather_times.argtypes = [C.c_void_p, C.c_int]
+    assert lib.dictproj_diag_gather_times(C.c_void_p(1 << 40), 0) == -5   # a buffer with no CTAs
+    assert lib.dictproj_diag_gather_times(C.c_void_p((1 << 40) + 4), 8) == -3  # not 8-byte aligned
