@@ -6,9 +6,11 @@
 //
 // Stage 1, dictionary (HBM-bound GEMV over packed NVFP4 D_g), k_dict_decode.
 //   The grid is (k/16 atom tiles) x (d_in slices); each warp owns whole units of
-//   16 atoms x 128 d_in elements. A thread streams the 16-byte code words of two
-//   atoms through a register ring (raw weights are loaded before the dependency
-//   wait; a bulk L2 prefetch covers the rest of the CTA's slice), converts E2M1
+//   16 atoms x 128 d_in elements, J of them, with one J for a whole batched call
+//   chosen by a fitted wave cost (dict_plan_batch). A thread streams the 16-byte
+//   code words of two atoms through a register ring (raw weights are loaded
+//   before the dependency wait; a bulk L2 prefetch covers the rest of the CTA's
+//   slice), converts E2M1
 //   pairs to f16x2 with the hardware cvt, multiplies by the E4M3 block scale in
 //   fp16 (an E2M1 x E4M3 product is exact in fp16), and issues mma.sync m16n8k16
 //   with the atoms as the 16 rows of A and the tokens as the 8 columns of B, fp32
@@ -18,18 +20,21 @@
 // Stage 2, coefficients (sparse gather over column-compressed NVFP4 C_l),
 // k_coeff_gather.
 //   One CTA per SM (1024 threads) owns a contiguous run of columns, one warp per
-//   column. Z = the sum of the dictionary stage's slices (fixed order) is staged
-//   in shared memory with a zero tail. A column's entries (index bytes, codes,
-//   scales, seg_start) are loaded straight from global memory into registers,
-//   the first column before the dependency wait and each next one while the
-//   current one is summed: lane l takes the 8-entry half-blocks 32i + l of the
-//   column (atom = 256*segment + idx; the segment of each 256-entry window comes
-//   from warp-wide ballots over seg_start, several boundaries inside one
-//   half-block fall back to a walk), scales each by its E4M3 block scale, and the
-//   warp reduces with shuffles in a fixed order, so results are bit-reproducible.
-//   Y = s_C * sum in fp16. Columns longer than 1280 stored entries, or k above
-//   8192 atoms, go to k_coeff_decode_direct (one warp per column, lanes over
-//   16-entry blocks, any length).
+//   column; a batched call hands its CTAs to the projection that would finish
+//   last (gather_batch_shares). Z = the sum of the dictionary stage's slices
+//   (fixed order) is staged in shared memory as an fp16 table with a zero tail.
+//   A column's entries (index bytes, codes, scales, seg_start) are loaded
+//   straight from global memory into registers, the first column before the
+//   dependency wait and each next one while the current one is summed: lane l
+//   takes the 8-entry half-blocks 32i + l of the column (atom = 256*segment +
+//   idx; the segment of each half-block comes from one ballot and one OR-reduced
+//   mask of the 8-rounded segment starts per 256-entry window, and a column with
+//   two starts inside one half-block walks its entries instead), multiplies fp16
+//   Z by the fp16 E2M1 value with fma.rn.f32.f16, scales each half-block by its
+//   E4M3 block scale, and the warp reduces with shuffles in a fixed order, so
+//   results are bit-reproducible. Y = s_C * sum in fp16. Columns longer than 1280
+//   stored entries, or k above 8192 atoms, go to k_coeff_decode_direct (one warp
+//   per column, lanes over 16-entry blocks, any length; fp32 Z).
 
 #include <algorithm>
 #include <climits>
