@@ -6,18 +6,19 @@
 // review, Eq. (1) and "Efficiency" section; the compressed factors replace one
 // d_in x d_out product by a d_in x k product and a sparse k x d_out one).
 //
-//   k_prefill_gemm<true>   Z[M][k]   = s_D · X[M][d_in] · D^[d_in][k]
-//       A = X tile (128 tokens x 64 d_in, fp16) by TMA with 128-byte swizzle;
-//       B = 256 atoms x 64 d_in: the packed E2M1 codes arrive by TMA, eight
-//       producer warps decode them (E2M1 x E4M3 block scale, exact in fp16)
-//       straight into the swizzled K-major fp16 operand tile; one thread issues
-//       tcgen05.mma (M=128, N=256, K=16, fp32 accumulate in tensor memory).
-//       The epilogue applies s_D in fp32 before rounding Z to fp16 (the
-//       unscaled sum can exceed the fp16 range).
-//   k_densify_coeff         Cd[d_out][k] = C^ (fp16, zeros off the support)
-//   k_prefill_gemm<false>  Y[M][d_out] = s_C · Z[M][k] · Cd^T, both operands by
-//       TMA. At prefill the tensor cores run the zeros of C faster than CUDA
-//       cores run only its nonzeros (dense fp16 rate / fp32 FMA rate >> 1/rho).
+//   k_dict_prefill   Z[M][k] = s_D · X[M][d_in] · D^[d_in][k], as Z^T tiles of
+//       128 atoms x nt tokens: the packed E2M1 codes and the X tile arrive by
+//       TMA; sixteen producer warps decode the codes (E2M1 x E4M3 block scale,
+//       exact in fp16) straight into tensor memory as operand A; one thread
+//       issues tcgen05.mma with B = X in shared memory and the fp32 accumulator
+//       in tensor memory. The epilogue applies s_D in fp32 before rounding Z to
+//       fp16 (the unscaled sum can exceed the fp16 range). For few tokens the
+//       d_in stages of a tile are split over a thread-block cluster and summed
+//       over distributed shared memory.
+//   k_densify_coeff  Cd[d_out][k] = C^ (fp16, zeros off the support)
+//   k_gemm_tma       Y[M][d_out] = s_C · Z[M][k] · Cd^T, both operands by TMA.
+//       At prefill the tensor cores run the zeros of C faster than CUDA cores run
+//       only its nonzeros (dense fp16 rate / fp32 FMA rate >> 1/rho).
 //
 // Every spin-wait is bounded; a wait that gives up sets bit 0 of the device
 // error word and the kernel unwinds (frees its tensor memory) without hanging.
