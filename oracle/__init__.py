@@ -28,7 +28,9 @@ Modules
 
 Parity status: every function here is pinned by ``tests/test_oracle_*.py``
 against values the pages print, closed forms, library routines or brute
-force, except the end-to-end quantised forward, for which the pages print no
-input/output pair ("parity unpinned" against the pages; it is pinned instead
-to the exact algebra it restates).
+force. The pages print no input/output pair for the end-to-end quantised
+forward; it is pinned by the special case where quantisation is exact (factors
+whose NVFP4 blocks each hold an entry of magnitude 6 x 448 and otherwise values
+of the scaled E2M1 grid), where pack, decode and forward must reproduce the
+integer product of the original factors exactly, for every index layout.
 """
