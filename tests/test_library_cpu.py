@@ -351,3 +351,17 @@ def test_stage_mask_and_diagnostic_calls_validate_on_the_host(dp):
     lib.dictproj_diag_gather_times.argtypes = [C.c_void_p, C.c_int]
     assert lib.dictproj_diag_gather_times(C.c_void_p(1 << 40), 0) == -5   # a buffer with no CTAs
     assert lib.dictproj_diag_gather_times(C.c_void_p((1 << 40) + 4), 8) == -3  # not 8-byte aligned
+
+
+def test_host_packers_on_exactly_representable_factors(dp):
+    # the factors of the oracle's exact-product pin (every NVFP4 block holds an
+    # entry of magnitude 6 x 448): the library's host packers give the oracle's
+    # bytes, tensor scale 1 and block scale 448 throughout, so the device path is
+    # tied to the exact integer product through the same bytes
+    from exact_factors import exact_case
+    X, D, col_ptr, atoms, vals, k, d_out, exact = exact_case()
+    a = dp.dictproj_pack_group_host(D)
+    b = pack_dictionary(D)
+    assert np.array_equal(a["codes"], b["codes"]) and np.array_equal(a["scales"], b["scales"])
+    assert a["s"] == b["s"] == 1.0 and np.all(a["scales"] == 0x7E)
+    _same_layer(dp.dictproj_pack_layer_host(col_ptr, atoms, vals, k, d_out), pack_coeff(col_ptr, atoms, vals, k, d_out))
