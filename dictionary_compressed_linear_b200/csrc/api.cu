@@ -1130,6 +1130,8 @@ int dictproj_selftest_wait_timeout(long long cycles, void* stream) {
   int dev, st;
   if ((st = ensure_device(&dev))) return st;
   cudaError_t e = launch_wait_probe(cycles, (cudaStream_t)stream);
+  if (e == cudaSuccess) e = launch_wait_probe_prefill(cycles, (cudaStream_t)stream);
+  if (e == cudaSuccess) e = launch_wait_probe_fused(cycles, (cudaStream_t)stream);
   return e == cudaSuccess ? DICTPROJ_OK : cuda_fail(e, "selftest_wait_timeout: launch");
 }
 

@@ -1321,6 +1321,31 @@ cudaError_t launch_fused(int n, const dictproj_group* const* g, const dictproj_l
   }
 }
 
+// Self-test of this file's bounded-wait error path (its own device error word):
+// one warp waits on an mbarrier that expects two arrivals and receives one, so
+// the wait can only end by its limit of `cycles` SM clocks. Nothing else is in
+// flight when it gives up.
+__global__ void k_wait_probe_fused(long long cycles) {
+  __shared__ __align__(8) uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 2);
+    fence_mbar_init();
+  }
+  __syncwarp();
+  if (threadIdx.x == 0) {
+    uint64_t state;
+    asm volatile("mbarrier.arrive.shared::cta.b64 %0, [%1];" : "=l"(state) : "r"(smem_u32(&bar)) : "memory");
+    (void)state;
+    mbar_wait_bounded(&bar, 0, cycles);
+  }
+  __syncwarp();
+}
+
+cudaError_t launch_wait_probe_fused(long long cycles, cudaStream_t stream) {
+  k_wait_probe_fused<<<1, 32, 0, stream>>>(cycles);
+  return cudaGetLastError();
+}
+
 cudaError_t take_fused_error(unsigned int* out) {
   unsigned int zero = 0;
   cudaError_t e = cudaMemcpyFromSymbol(out, g_dictproj_error, sizeof(unsigned int));

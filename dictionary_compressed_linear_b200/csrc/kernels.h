@@ -51,6 +51,10 @@ bool gather_supported(const uint32_t* pcol_ptr, int d_out, int nseg);
 bool coeff_smem_fits(int k, int mp, int device);
 // One warp whose bounded wait can only end by its limit (error-path self-test).
 cudaError_t launch_wait_probe(long long cycles, cudaStream_t stream);
+// The same probe in the prefill and fused kernel files (each file has its own
+// device error word).
+cudaError_t launch_wait_probe_prefill(long long cycles, cudaStream_t stream);
+cudaError_t launch_wait_probe_fused(long long cycles, cudaStream_t stream);
 // Read and clear the device error word of the decode kernels.
 cudaError_t take_decode_error(unsigned int* out);
 // Diagnostic timestamps of the gather kernel (buf null: off).

@@ -512,10 +512,11 @@ int dictproj_diag_phase_times(unsigned long long* out, int max_ctas, int* n_ctas
 int dictproj_diag_gather_times(unsigned long long* buf, int max_ctas);
 
 /* Self-test of the bounded-wait error path (diagnostic; no counterpart in the
- * paper). Launches one warp on `stream` that waits on an mbarrier which can never
- * complete, with a limit of `cycles` SM clocks (1 <= cycles <= 2^31). The wait
- * gives up at the limit, sets the device error word and the kernel returns; no
- * copy or tensor-core operation is in flight. A following dictproj_check(stream)
+ * paper). Launches, on `stream`, one warp per kernel file (decode, prefill, fused
+ * decode: each has its own device error word) that waits on an mbarrier which
+ * can never complete, with a limit of `cycles` SM clocks (1 <= cycles <= 2^31).
+ * Each wait gives up at the limit, sets its file's error word and the kernel
+ * returns; no copy or tensor-core operation is in flight. A following dictproj_check(stream)
  * then returns DICTPROJ_ERR_TIMEOUT and clears the word; the device stays usable.
  * Errors: RANGE (cycles), UNSUPPORTED (not sm_100), CUDA. */
 int dictproj_selftest_wait_timeout(long long cycles, void* stream);
